@@ -1,0 +1,85 @@
+"""The vectorised oracle against the loop-level brute force on tiny sizes:
+codes identical (except decisions the oracle flags as ties), floats to 1e-12.
+"""
+import math
+
+import numpy as np
+import pytest
+
+from oracle import brute as B
+from oracle import tq_oracle as O
+
+
+@pytest.mark.parametrize("d,m,b_r,b_t", [(4, 4, 2, 3), (8, 8, 3, 3), (8, 8, 4, 4), (8, 5, 1, 2)])
+def test_encode_matches_brute(d, m, b_r, b_t):
+    rng = np.random.default_rng(d * 100 + m)
+    n = 16
+    x = rng.standard_normal((n, d)).astype(np.float16).astype(np.float64)
+    signs = O.rotation_signs(d + m, d)
+    S = O.qjl_matrix(d + m, m, d)
+    c = O.encode(x, signs, S, b_r, b_t, keep_intermediates=True)
+    for i in range(n):
+        ref = B.encode_one(list(x[i]), list(signs), S.astype(np.float64).tolist(), b_r, b_t)
+        assert ref["s16"] == c.s16[i]
+        if c.vec_tie[i]:
+            continue
+        assert ref["cr"] == list(c.cr[i])
+        assert ref["ct"] == list(c.ct[i])
+        np.testing.assert_allclose(ref["residual"], c.residual[i], rtol=0, atol=1e-12)
+        if not c.tie_rn16[i]:
+            assert ref["rn16"] == c.rn16[i]
+        for j in range(m):
+            if not c.tie_bits[i, j]:
+                assert ref["bits"][j] == c.bits[i, j]
+
+
+def test_rotation_matches_brute():
+    rng = np.random.default_rng(0)
+    for d in (2, 4, 8, 16):
+        signs = O.rotation_signs(d, d)
+        x = rng.standard_normal(d)
+        np.testing.assert_allclose(O.rotate(x[None], signs)[0], B.rotate(list(x), list(signs)), atol=1e-12)
+        np.testing.assert_allclose(O.rotate_inverse(x[None], signs)[0],
+                                   B.rotate_inverse(list(x), list(signs)), atol=1e-12)
+
+
+@pytest.mark.parametrize("d,m,b", [(4, 4, 3), (8, 8, 4), (8, 8, 2)])
+def test_decode_attention_matches_brute(d, m, b):
+    rng = np.random.default_rng(d + 10 * b)
+    hq, hkv, nh, nc = 4, 2, 3, 9
+    q = rng.standard_normal((hq, d))
+    hk = rng.standard_normal((hkv, nh, d))
+    hv = rng.standard_normal((hkv, nh, d))
+    ck_raw = rng.standard_normal((hkv, nc, d))
+    cv_raw = rng.standard_normal((hkv, nc, d))
+    signs = O.rotation_signs(1, d)
+    S = O.qjl_matrix(1, m, d)
+    ck = [O.encode(ck_raw[h], signs, S, b, b) for h in range(hkv)]
+    cv = [O.encode(cv_raw[h], signs, None, b, b) for h in range(hkv)]
+    sigma = 1 / math.sqrt(d)
+    out = O.decode_attention(q, hk, hv, ck, cv, signs, S, hkv)
+    Sl = S.astype(np.float64).tolist()
+    for h in range(hq):
+        g = h // (hq // hkv)
+        recs_k = [dict(s16=ck[g].s16[t], cr=list(ck[g].cr[t]), ct=list(ck[g].ct[t]),
+                       rn16=ck[g].rn16[t], bits=list(ck[g].bits[t])) for t in range(nc)]
+        recs_v = [dict(s16=cv[g].s16[t], cr=list(cv[g].cr[t]), ct=list(cv[g].ct[t])) for t in range(nc)]
+        ref = B.decode_one_head(list(q[h]), hk[g].tolist(), hv[g].tolist(), recs_k, recs_v,
+                                list(signs), Sl, b, b, sigma)
+        np.testing.assert_allclose(out[h], ref, rtol=1e-12, atol=1e-12)
+
+
+def test_inner_products_match_brute():
+    rng = np.random.default_rng(4)
+    d, m, b_r, b_t = 8, 8, 4, 4
+    signs = O.rotation_signs(2, d)
+    S = O.qjl_matrix(2, m, d)
+    x = rng.standard_normal((10, d))
+    q = rng.standard_normal((3, d))
+    c = O.encode(x, signs, S, b_r, b_t)
+    sc = O.ip_scores(q, signs, S, c)
+    for i in range(3):
+        for t in range(10):
+            rec = dict(s16=c.s16[t], cr=list(c.cr[t]), ct=list(c.ct[t]), rn16=c.rn16[t], bits=list(c.bits[t]))
+            assert abs(sc[i, t] - B.key_ip(list(q[i]), list(signs), S.astype(np.float64).tolist(),
+                                            rec, b_r, b_t)) < 1e-12
