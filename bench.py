@@ -1,0 +1,419 @@
+#!/usr/bin/env python
+"""Decode-step benchmark of the compressed KV-cache path.
+
+One step = one decode token through every layer of the Llama-3.1-8B-shaped
+workload (32 layers, batch 8, 32 q / 8 kv heads, head_dim 128, 512 hot fp16
+tokens + 32256 compressed cold tokens, b_r = b_theta = 3, m = 128): per
+layer tq_evict_window (the new token enters the hot ring, the oldest hot
+token is compressed into the cold store) then tq_decode_attention (q-prep,
+hot + cold attention, combine).  Inputs are seeded synthetic tensors with
+the workload's value recipe, generated on the device; the 32 layers' caches
+(8.4 GB) are far larger than L2, and every layer has its own buffers.
+
+Prints ONE JSON line (rank 0).  ``--impl reference`` times the fp64 CPU
+oracle on the same metric instead (a bounded sample per step).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "cold-KV decode attention keys/s and achieved HBM GB/s (% of B200 peak)"
+UNIT = "keys/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="tq", choices=["tq", "reference"])
+    ap.add_argument("--workload", default="llama8b")
+    ap.add_argument("--layers", type=int, default=0, help="0: the workload's layer count")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--seed", type=int, default=0)
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+# --------------------------------------------------------------------------
+# clocks during the timed region
+# --------------------------------------------------------------------------
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"tq_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(f[1]), smax=float(f[2]), hw=f[5], hwt=f[6], swt=f[7],
+                                 pcap=f[8]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        reasons = set()
+        for r in rows:
+            if r["hw"] == "Active": reasons.add("hw_slowdown")
+            if r["hwt"] == "Active": reasons.add("hw_thermal_slowdown")
+            if r["swt"] == "Active": reasons.add("sw_thermal_slowdown")
+            if r["pcap"] == "Active": reasons.add("sw_power_cap")
+        return {"sm_mhz": statistics.median(r["sm"] for r in rows),
+                "sm_max_mhz": max(r["smax"] for r in rows), "samples": len(rows),
+                "reasons": sorted(reasons)}
+
+
+# --------------------------------------------------------------------------
+# oracle timing (cpu_baseline and the reference arm)
+# --------------------------------------------------------------------------
+def oracle_sample(wl, seed: int, kv_heads: int):
+    """One batch row, `kv_heads` kv heads of layer 0: oracle-encoded records
+    (built once, untimed) and the query."""
+    import numpy as np
+    from compressed_decode_attention_encode_b200.inputs import kv_stream, queries
+    from oracle import tq_oracle as O
+    d = wl.head_dim
+    signs = O.rotation_signs(seed, d)
+    S = O.qjl_matrix(seed, wl.qjl_bits, d)
+    ck, cv, hk, hv = [], [], [], []
+    for h in range(kv_heads):
+        k = kv_stream(wl, 0, seed, 0, 0, h, 0, wl.cold + wl.hot).astype(np.float64)
+        v = kv_stream(wl, 0, seed, 1, 0, h, 0, wl.cold + wl.hot).astype(np.float64)
+        ck.append(O.encode(k[: wl.cold], signs, S, wl.b_r, wl.b_theta))
+        cv.append(O.encode(v[: wl.cold], signs, None, wl.b_r, wl.b_theta))
+        hk.append(k[wl.cold:])
+        hv.append(v[wl.cold:])
+    q = queries(wl, 0, seed)[0, : kv_heads * wl.group].astype(np.float64)
+    return dict(q=q, hk=np.stack(hk), hv=np.stack(hv), ck=ck, cv=cv, signs=signs, S=S,
+                kv_heads=kv_heads)
+
+
+def time_oracle(sample):
+    """Seconds and keys of one oracle decode over the sample."""
+    from oracle import tq_oracle as O
+    t0 = time.perf_counter()
+    O.decode_attention(sample["q"], sample["hk"], sample["hv"], sample["ck"], sample["cv"],
+                       sample["signs"], sample["S"], sample["kv_heads"])
+    dt = time.perf_counter() - t0
+    keys = sample["kv_heads"] * (sample["hk"].shape[1] + sample["ck"][0].s16.shape[0])
+    return dt, keys
+
+
+def oracle_threads() -> int:
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        n = max((i.get("num_threads", 1) for i in info), default=1)
+        return int(n)
+    except Exception:
+        return 1
+
+
+def run_reference(args, wl):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    sample = oracle_sample(wl, args.seed, kv_heads=2)
+    for _ in range(args.warmup):
+        time_oracle(sample)
+    tot_t, tot_k = 0.0, 0
+    for _ in range(args.steps):
+        dt, k = time_oracle(sample)
+        tot_t += dt
+        tot_k += k
+    v = tot_k / tot_t
+    desc = (f"per step: oracle decode attention of 1 batch row x 2 kv heads (8 q heads) of "
+            f"layer 0, {wl.cold} cold + {wl.hot} hot tokens")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "layers": wl.layers, "batch": wl.batch,
+                   "num_q_heads": wl.num_q_heads, "num_kv_heads": wl.num_kv_heads,
+                   "head_dim": wl.head_dim, "hot": wl.hot, "cold": wl.cold,
+                   "b_r": wl.b_r, "b_theta": wl.b_theta, "qjl_bits": wl.qjl_bits},
+        "cpu_baseline": {"value": v, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+# --------------------------------------------------------------------------
+# GPU arm
+# --------------------------------------------------------------------------
+def gen_kv(wl, layer, seed, which, b_rows, start, count, device, gen):
+    """fp16 [B, Hkv, count, d] with the workload's channel scales (device RNG)."""
+    import torch
+    from compressed_decode_attention_encode_b200.inputs import channel_scales
+    sc = torch.from_numpy(channel_scales(wl, layer, seed, which)).to(device=device, dtype=torch.float32)
+    z = torch.randn((b_rows, wl.num_kv_heads, count, wl.head_dim), generator=gen, device=device,
+                    dtype=torch.float32)
+    return (z * sc[None, :, None, :]).to(torch.float16)
+
+
+def run_gpu(args, wl):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from compressed_decode_attention_encode_b200 import build as B
+    from compressed_decode_attention_encode_b200 import tq
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if rank == 0:
+        B.build()
+    if world > 1:
+        dist.barrier()
+    tq.lib()
+
+    L = args.layers or wl.layers
+    total_steps = args.warmup + 2 * args.steps + 2
+    cap = wl.cold + total_steps + 64
+    cfg = tq.make_config(wl.batch, wl.num_q_heads, wl.num_kv_heads, wl.head_dim, wl.hot, cap,
+                         wl.b_r, wl.b_theta, wl.qjl_bits, seed=args.seed)
+    stream = torch.cuda.current_stream()
+    gen = torch.Generator(device=dev)
+    caches = []
+    chunk = 4096
+    for layer in range(L):
+        gen.manual_seed(1_000_003 * (args.seed + 1) + 7919 * layer + rank)
+        c = tq.TQCache(cfg, device=dev)
+        pos = 0
+        while pos < wl.cold:
+            n = min(chunk, wl.cold - pos)
+            k = gen_kv(wl, layer, args.seed, 0, wl.batch, pos, n, dev, gen)
+            v = gen_kv(wl, layer, args.seed, 1, wl.batch, pos, n, dev, gen)
+            c.encode_append(k, v)
+            pos += n
+        k = gen_kv(wl, layer, args.seed, 0, wl.batch, 0, wl.hot, dev, gen)
+        v = gen_kv(wl, layer, args.seed, 1, wl.batch, 0, wl.hot, dev, gen)
+        c.evict_window(k, v)
+        if c.get_status() != 0:
+            raise RuntimeError("device status after prefill")
+        caches.append(c)
+    # per-step inputs (new token K/V per layer, queries per layer)
+    knew = [gen_kv(wl, l, args.seed, 0, wl.batch, 0, total_steps, dev, gen) for l in range(L)]
+    vnew = [gen_kv(wl, l, args.seed, 1, wl.batch, 0, total_steps, dev, gen) for l in range(L)]
+    knew = [[x[:, :, s:s + 1].contiguous() for s in range(total_steps)] for x in knew]
+    vnew = [[x[:, :, s:s + 1].contiguous() for s in range(total_steps)] for x in vnew]
+    qs = [torch.randn((wl.batch, wl.num_q_heads, wl.head_dim), generator=gen, device=dev).half()
+          for _ in range(L)]
+    outs = [torch.empty((wl.batch, wl.num_q_heads, wl.head_dim), dtype=torch.float32, device=dev)
+            for _ in range(L)]
+    torch.cuda.synchronize()
+
+    units = wl.batch * wl.num_kv_heads
+    kc = wl.head_dim // 2 * (wl.b_r + wl.b_theta) // 8
+    cold_tok_bytes = 2 * kc + wl.qjl_bits // 8 + 6     # K and V record bytes
+    hot_tok_bytes = 4 * wl.head_dim                     # K and V fp16
+
+    step_idx = [0]
+
+    def one_step(ev_pairs=None):
+        s = step_idx[0]
+        step_idx[0] += 1
+        keys = 0
+        abytes = 0
+        for l in range(L):
+            caches[l].evict_window(knew[l][s], vnew[l][s])
+            nc, nh, _ = caches[l].counts()
+            keys += units * (nc + nh)
+            abytes += units * (nc * cold_tok_bytes + nh * hot_tok_bytes)
+            if ev_pairs is not None:
+                caches[l].set_attend_events(*ev_pairs[l])
+            caches[l].decode_attention(qs[l], out=outs[l])
+            if ev_pairs is not None:
+                caches[l].set_attend_events(None, None)
+        return keys, abytes
+
+    for _ in range(args.warmup):
+        one_step()
+    for c in caches:
+        if c.get_status() != 0:
+            raise RuntimeError("device status after warm-up")
+
+    # ---- timed region: device-resident inputs --------------------------
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(L)] for _ in range(args.steps)]
+    for row in ev:                       # torch creates CUDA events lazily
+        for a_, b_ in row:
+            a_.record(stream)
+            b_.record(stream)
+    clock = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clock.start()
+    time.sleep(0.3)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    keys_total = 0
+    bytes_total = 0
+    for s in range(args.steps):
+        k_, b_ = one_step(ev[s])
+        keys_total += k_
+        bytes_total += b_
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clocks = clock.stop()
+    ms = t0.elapsed_time(t1)
+    attend_ms = sum(a.elapsed_time(b) for row in ev for (a, b) in row)
+    for c in caches:
+        if c.get_status() != 0:
+            raise RuntimeError("device status in timed region")
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    launches_per_step = L * (2 + 3)   # evict: encode + ring write; decode: qprep, attend, combine
+
+    # ---- e2e: host buffers through the public API ------------------------
+    hk = [[x.cpu().pin_memory() for x in knew[l]] for l in range(L)]
+    hv = [[x.cpu().pin_memory() for x in vnew[l]] for l in range(L)]
+    hq = [x.cpu().pin_memory() for x in qs]
+    hout = [torch.empty(o.shape, dtype=torch.float32).pin_memory() for o in outs]
+    dk = [torch.empty_like(knew[0][0]) for _ in range(L)]
+    dv = [torch.empty_like(vnew[0][0]) for _ in range(L)]
+    dq = [torch.empty_like(qs[0]) for _ in range(L)]
+    e2e_steps = args.steps
+    h2d = d2h = 0
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    e2e_keys = 0
+    for _ in range(e2e_steps):
+        s = step_idx[0]
+        step_idx[0] += 1
+        h2d = d2h = 0
+        for l in range(L):
+            dk[l].copy_(hk[l][s], non_blocking=True)
+            dv[l].copy_(hv[l][s], non_blocking=True)
+            dq[l].copy_(hq[l], non_blocking=True)
+            h2d += 2 * dk[l].numel() * 2 + dq[l].numel() * 2
+            caches[l].evict_window(dk[l], dv[l])
+            nc, nh, _ = caches[l].counts()
+            e2e_keys += units * (nc + nh)
+            caches[l].decode_attention(dq[l], out=outs[l])
+            hout[l].copy_(outs[l], non_blocking=True)
+            d2h += outs[l].numel() * 4
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    value = world * keys_total / (ms / 1e3)
+    e2e_value = world * e2e_keys / (e2e_ms / 1e3)
+    hbm_peak, peak_kind = peaks()
+    attend_launches = L * args.steps
+    achieved = bytes_total / (attend_ms / 1e3) / 1e9
+    result = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f16-in/f32-acc", "data": "synthetic",
+        "config": {"workload": wl.name, "layers": L, "batch": wl.batch,
+                   "num_q_heads": wl.num_q_heads, "num_kv_heads": wl.num_kv_heads,
+                   "head_dim": wl.head_dim, "hot": wl.hot, "cold": wl.cold,
+                   "b_r": wl.b_r, "b_theta": wl.b_theta, "qjl_bits": wl.qjl_bits,
+                   "l2": "inputs larger than L2 (each of the layers has its own "
+                         f"{caches[0].bytes['cold'] / 1e6:.0f} MB cold store)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "hbm": {"step_gbs": bytes_total / (ms / 1e3) / 1e9, "attend_gbs": achieved,
+                "frac_of_measured": achieved / hbm_peak, "frac_of_8tbs_spec": achieved / 8000.0},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved / hbm_peak, "traffic": None, "kernel": "attend_kernel",
+                     "peak_kind": peak_kind,
+                     "avg_launch_us": 1e3 * attend_ms / attend_launches,
+                     "bytes_per_launch": bytes_total / attend_launches},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / e2e_steps},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        sample = oracle_sample(wl, args.seed, kv_heads=1)
+        time_oracle(sample)
+        tt, kk = 0.0, 0
+        while tt < 10.0:
+            dt, k_ = time_oracle(sample)
+            tt += dt
+            kk += k_
+        result["cpu_baseline"] = {
+            "value": kk / tt, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
+            "sample": f"fp64 oracle decode attention, 1 batch row x 1 kv head (4 q heads) of "
+                      f"layer 0 ({wl.cold} cold + {wl.hot} hot tokens), repeated for ~10 s"}
+    for c in caches:
+        c.close()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    from compressed_decode_attention_encode_b200.inputs import WORKLOADS
+    wl = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, wl)
+    else:
+        run_gpu(args, wl)
+
+
+if __name__ == "__main__":
+    main()

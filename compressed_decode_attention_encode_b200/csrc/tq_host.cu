@@ -1,0 +1,469 @@
+// C-ABI entry points of the compressed KV-cache library: argument checks,
+// buffer layout, the seeded method randomness (rotation signs D, QJL matrix
+// S) and the launch sequence of each call.  See include/tq.h for the
+// contract of every function.
+#include <algorithm>
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "tq_internal.cuh"
+
+namespace tq {
+
+namespace {
+
+constexpr int kMaxSplits = 64;     // split partials kept per (row, kv head)
+constexpr size_t kAlign = 256;
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// ---- seeded generator (SplitMix64 finalizer over a Weyl sequence) --------
+// Steele, Lea & Flood, "Fast splittable pseudorandom number generators"
+// (OOPSLA 2014): mix64 is the SplitMix64 output function.
+uint64_t mix64(uint64_t z) {
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+uint64_t rand64(uint64_t seed, uint64_t stream, uint64_t i) {
+  const uint64_t base = mix64(seed + stream);
+  return mix64(base + (i + 1) * 0x9E3779B97F4A7C15ull);
+}
+
+void gen_signs(uint64_t seed, int d, double* out) {
+  for (int i = 0; i < d; ++i) out[i] = (rand64(seed, 0, (uint64_t)i) >> 63) ? -1.0 : 1.0;
+}
+
+void gen_qjl(uint64_t seed, int m, int d, float* out) {
+  const double two_pi = 2.0 * M_PI;
+  const double scale = 1.0 / 9007199254740992.0;  // 2^-53
+  const uint64_t total = (uint64_t)m * (uint64_t)d;
+  for (uint64_t k = 0; k < total; ++k) {
+    const uint64_t a = rand64(seed, 1, 2 * k);
+    const uint64_t b = rand64(seed, 1, 2 * k + 1);
+    const double u1 = (double)((a >> 11) + 1) * scale;
+    const double u2 = (double)(b >> 11) * scale;
+    const double z = std::sqrt(-2.0 * std::log(u1)) * std::cos(two_pi * u2);
+    out[k] = (float)z;
+  }
+}
+
+bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+
+}  // namespace
+
+Layout make_layout(int d, int b_r, int b_theta, int m, int64_t capacity) {
+  Layout L{};
+  L.d = d;
+  L.pairs = d / 2;
+  L.b_r = b_r;
+  L.b_theta = b_theta;
+  L.bw = b_r + b_theta;
+  L.m = m;
+  L.kc_bytes = L.pairs * L.bw / 8;
+  L.sg_bytes = m / 8;
+  const int TB = kTokensPerBlock;
+  L.off_kc = 0;
+  L.off_ks = L.off_kc + TB * L.kc_bytes;
+  L.off_ksc = L.off_ks + TB * L.sg_bytes;
+  L.off_krn = L.off_ksc + TB * 2;
+  L.off_vc = L.off_krn + TB * 2;
+  L.off_vsc = L.off_vc + TB * L.kc_bytes;
+  L.block_bytes = L.off_vsc + TB * 2;
+  L.blocks_per_unit = (capacity + TB - 1) / TB;
+  return L;
+}
+
+struct WsLayout {
+  size_t status, signs, S, St, qrot, qsk, qscale, part, total;
+};
+
+static WsLayout ws_layout(const tq_config& c) {
+  WsLayout w{};
+  const size_t heads = (size_t)c.batch * c.num_q_heads;
+  const size_t units = (size_t)c.batch * c.num_kv_heads;
+  const size_t G = (size_t)(c.num_q_heads / c.num_kv_heads);
+  size_t off = 0;
+  w.status = off; off += kAlign;
+  w.signs = off;  off += round_up(sizeof(double) * c.head_dim, kAlign);
+  w.S = off;      off += round_up(sizeof(float) * c.head_dim * c.qjl_bits, kAlign);
+  w.St = off;     off += round_up(sizeof(float) * c.head_dim * c.qjl_bits, kAlign);
+  w.qrot = off;   off += round_up(2 * heads * c.head_dim, kAlign);
+  w.qsk = off;    off += round_up(2 * heads * c.qjl_bits, kAlign);
+  w.qscale = off; off += round_up(sizeof(float) * 2 * heads, kAlign);
+  w.part = off;   off += round_up(sizeof(float) * units * kMaxSplits * G * (c.head_dim + 2), kAlign);
+  w.total = off;
+  return w;
+}
+
+static tq_status check_config(const tq_config* c) {
+  if (!c) return TQ_ERR_INVALID_ARG;
+  if (c->batch < 1 || c->num_q_heads < 1 || c->num_kv_heads < 1 || c->hot_window < 1 ||
+      c->cold_capacity < 0 || c->b_r < 1 || c->b_theta < 1 || c->qjl_bits < 8 ||
+      c->head_dim < 2 || (c->qjl_bits % 8) != 0 || !is_pow2(c->head_dim))
+    return TQ_ERR_INVALID_ARG;
+  if (c->num_q_heads % c->num_kv_heads != 0) return TQ_ERR_INVALID_ARG;
+  if (c->b_r + c->b_theta > 8) return TQ_ERR_INVALID_ARG;
+  if (c->head_dim != 64 && c->head_dim != 128) return TQ_ERR_UNSUPPORTED;
+  if (c->qjl_bits != 64 && c->qjl_bits != 128) return TQ_ERR_UNSUPPORTED;
+  if (c->num_q_heads / c->num_kv_heads > 8) return TQ_ERR_UNSUPPORTED;
+  return TQ_OK;
+}
+
+}  // namespace tq
+
+using namespace tq;
+
+struct tq_cache {
+  tq_config cfg;
+  Layout L;
+  WsLayout W;
+  uint8_t* hot;
+  uint8_t* cold;
+  uint8_t* ws;
+  int64_t n_cold;
+  int32_t n_hot;
+  int32_t ring_pos;
+  int num_sms;
+  int ctas_per_sm;
+  int device;
+  cudaEvent_t ev_start;
+  cudaEvent_t ev_stop;
+  __half* hot_k() const { return (__half*)hot; }
+  __half* hot_v() const {
+    return (__half*)(hot + (size_t)cfg.batch * cfg.num_kv_heads * cfg.hot_window * cfg.head_dim * 2);
+  }
+  int* status() const { return (int*)(ws + W.status); }
+  double* signs() const { return (double*)(ws + W.signs); }
+  float* S() const { return (float*)(ws + W.S); }
+  float* St() const { return (float*)(ws + W.St); }
+};
+
+extern "C" {
+
+const char* tq_status_string(tq_status s) {
+  switch (s) {
+    case TQ_OK: return "TQ_OK";
+    case TQ_ERR_INVALID_ARG: return "TQ_ERR_INVALID_ARG";
+    case TQ_ERR_UNSUPPORTED: return "TQ_ERR_UNSUPPORTED";
+    case TQ_ERR_CAPACITY: return "TQ_ERR_CAPACITY";
+    case TQ_ERR_RANGE: return "TQ_ERR_RANGE";
+    case TQ_ERR_TIMEOUT: return "TQ_ERR_TIMEOUT";
+    case TQ_ERR_CUDA: return "TQ_ERR_CUDA";
+  }
+  return "TQ_UNKNOWN";
+}
+
+int32_t tq_abi_version(void) { return TQ_ABI_VERSION; }
+
+tq_status tq_cache_bytes(const tq_config* cfg, size_t* hot_bytes, size_t* cold_bytes,
+                         size_t* workspace_bytes) {
+  tq_status st = check_config(cfg);
+  if (st != TQ_OK) return st;
+  const Layout L = make_layout(cfg->head_dim, cfg->b_r, cfg->b_theta, cfg->qjl_bits,
+                               cfg->cold_capacity);
+  const size_t units = (size_t)cfg->batch * cfg->num_kv_heads;
+  if (hot_bytes) *hot_bytes = 2 * units * cfg->hot_window * cfg->head_dim * 2;
+  if (cold_bytes) *cold_bytes = units * (size_t)L.blocks_per_unit * L.block_bytes;
+  if (workspace_bytes) *workspace_bytes = ws_layout(*cfg).total;
+  return TQ_OK;
+}
+
+tq_status tq_cache_create(const tq_config* cfg, void* hot_mem, void* cold_mem,
+                          void* workspace_mem, cudaStream_t stream, tq_cache** out) {
+  tq_status st = check_config(cfg);
+  if (st != TQ_OK) return st;
+  if (!out || !hot_mem || !workspace_mem || (!cold_mem && cfg->cold_capacity > 0))
+    return TQ_ERR_INVALID_ARG;
+  if (((uintptr_t)hot_mem | (uintptr_t)cold_mem | (uintptr_t)workspace_mem) % kAlign)
+    return TQ_ERR_INVALID_ARG;
+  tq_cache* c = new (std::nothrow) tq_cache();
+  if (!c) return TQ_ERR_INVALID_ARG;
+  c->cfg = *cfg;
+  c->L = make_layout(cfg->head_dim, cfg->b_r, cfg->b_theta, cfg->qjl_bits, cfg->cold_capacity);
+  c->W = ws_layout(*cfg);
+  c->hot = (uint8_t*)hot_mem;
+  c->cold = (uint8_t*)cold_mem;
+  c->ws = (uint8_t*)workspace_mem;
+  c->n_cold = 0;
+  c->n_hot = 0;
+  c->ring_pos = 0;
+  if (cudaGetDevice(&c->device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, c->device) != cudaSuccess) {
+    delete c;
+    return TQ_ERR_CUDA;
+  }
+  c->ctas_per_sm = attend_ctas_per_sm(c->L);
+  if (c->ctas_per_sm <= 0) {
+    delete c;
+    return TQ_ERR_CUDA;
+  }
+  const int d = cfg->head_dim, m = cfg->qjl_bits;
+  std::vector<double> signs(d);
+  std::vector<float> S((size_t)m * d), St((size_t)m * d);
+  gen_signs(cfg->seed, d, signs.data());
+  gen_qjl(cfg->seed, m, d, S.data());
+  for (int i = 0; i < m; ++i)
+    for (int j = 0; j < d; ++j) St[(size_t)j * m + i] = S[(size_t)i * d + j];
+  // Pageable sources: cudaMemcpyAsync returns once the data is staged, so
+  // the vectors may be released when the calls return.
+  cudaError_t e = cudaMemsetAsync(c->status(), 0, kAlign, stream);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(c->signs(), signs.data(), sizeof(double) * d, cudaMemcpyHostToDevice, stream);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(c->S(), S.data(), sizeof(float) * S.size(), cudaMemcpyHostToDevice, stream);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(c->St(), St.data(), sizeof(float) * St.size(), cudaMemcpyHostToDevice, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) {
+    delete c;
+    return TQ_ERR_CUDA;
+  }
+  *out = c;
+  return TQ_OK;
+}
+
+tq_status tq_cache_destroy(tq_cache* cache) {
+  delete cache;
+  return TQ_OK;
+}
+
+tq_status tq_cache_counts(const tq_cache* c, int64_t* n_cold, int32_t* n_hot, int32_t* ring_pos) {
+  if (!c) return TQ_ERR_INVALID_ARG;
+  if (n_cold) *n_cold = c->n_cold;
+  if (n_hot) *n_hot = c->n_hot;
+  if (ring_pos) *ring_pos = c->ring_pos;
+  return TQ_OK;
+}
+
+static EncodeArgs base_encode_args(tq_cache* c) {
+  EncodeArgs a{};
+  a.W = c->cfg.hot_window;
+  a.cold = c->cold;
+  a.cold_start = c->n_cold;
+  a.units = c->cfg.batch * c->cfg.num_kv_heads;
+  a.L = c->L;
+  a.signs = c->signs();
+  a.St = c->St();
+  a.status = c->status();
+  a.inv_sqrt_d = 1.0 / std::sqrt((double)c->cfg.head_dim);
+  return a;
+}
+
+tq_status tq_encode_append(tq_cache* c, const void* k, const void* v, int64_t n, cudaStream_t stream) {
+  if (!c || n < 0) return TQ_ERR_INVALID_ARG;
+  if (n == 0) return TQ_OK;
+  if (!k || !v) return TQ_ERR_INVALID_ARG;
+  if (c->n_cold + n > c->cfg.cold_capacity) return TQ_ERR_CAPACITY;
+  EncodeArgs a = base_encode_args(c);
+  a.src_k = (const __half*)k;
+  a.src_v = (const __half*)v;
+  a.src_tokens = n;
+  a.nB = n;
+  a.nA = 0;
+  if (launch_encode(a, stream) != cudaSuccess) return TQ_ERR_CUDA;
+  c->n_cold += n;
+  return TQ_OK;
+}
+
+tq_status tq_evict_window(tq_cache* c, const void* k_new, const void* v_new, int32_t n,
+                          cudaStream_t stream) {
+  if (!c || !k_new || !v_new || n < 1) return TQ_ERR_INVALID_ARG;
+  const int W = c->cfg.hot_window;
+  const int64_t E = std::max<int64_t>(0, (int64_t)c->n_hot + n - W);
+  if (c->n_cold + E > c->cfg.cold_capacity) return TQ_ERR_CAPACITY;
+  if (E > 0) {
+    EncodeArgs a = base_encode_args(c);
+    a.nA = (int)std::min<int64_t>(E, c->n_hot);
+    a.nB = E - a.nA;
+    a.ring_k = c->hot_k();
+    a.ring_v = c->hot_v();
+    a.ring_start = ((c->ring_pos - c->n_hot) % W + W) % W;
+    a.src_k = (const __half*)k_new;
+    a.src_v = (const __half*)v_new;
+    a.src_tokens = n;
+    if (launch_encode(a, stream) != cudaSuccess) return TQ_ERR_CUDA;
+  }
+  const int first = std::max(0, n - W);
+  if (launch_ring_write(c->hot_k(), c->hot_v(), (const __half*)k_new, (const __half*)v_new,
+                        c->cfg.batch * c->cfg.num_kv_heads, W, c->cfg.head_dim, n, first,
+                        c->ring_pos, stream) != cudaSuccess)
+    return TQ_ERR_CUDA;
+  c->n_cold += E;
+  c->n_hot = (int32_t)std::min<int64_t>(W, (int64_t)c->n_hot + n);
+  c->ring_pos = (int32_t)(((int64_t)c->ring_pos + n) % W);
+  return TQ_OK;
+}
+
+tq_status tq_decode_attention(tq_cache* c, const void* q, float* out, float softmax_scale,
+                              cudaStream_t stream) {
+  if (!c || !q || !out || !(softmax_scale >= 0.0f) || std::isinf(softmax_scale))
+    return TQ_ERR_INVALID_ARG;
+  const tq_config& cf = c->cfg;
+  const int d = cf.head_dim, m = cf.qjl_bits;
+  const int heads = cf.batch * cf.num_q_heads;
+  const int units = cf.batch * cf.num_kv_heads;
+  const int G = cf.num_q_heads / cf.num_kv_heads;
+  const float sigma = softmax_scale == 0.0f ? (float)(1.0 / std::sqrt((double)d)) : softmax_scale;
+  const int TB = kTokensPerBlock;
+
+  // Split plan: fill the device with about one wave of CTAs; hot tiles and
+  // cold blocks get CTAs in proportion to their bytes.
+  const int64_t cold_blocks = (c->n_cold + TB - 1) / TB;
+  const int hot_tiles = (c->n_hot + TB - 1) / TB;
+  const int slots = c->num_sms * c->ctas_per_sm;
+  const int target = std::max(1, std::min(kMaxSplits, slots / std::max(1, units)));
+  const double cold_b = (double)cold_blocks * c->L.block_bytes;
+  const double hot_b = (double)hot_tiles * TB * d * 4.0;
+  // Every non-empty region gets at least one split; together at most
+  // kMaxSplits (the partial slots reserved per unit).
+  int ns_hot = 0, ns_cold = 0;
+  if (hot_tiles > 0) {
+    ns_hot = std::max(1, (int)std::lround(target * hot_b / (hot_b + cold_b)));
+    ns_hot = std::min(ns_hot, hot_tiles);
+    if (cold_blocks > 0) ns_hot = std::min(ns_hot, kMaxSplits - 1);
+  }
+  if (cold_blocks > 0) {
+    ns_cold = std::max(1, target - ns_hot);
+    ns_cold = (int)std::min<int64_t>(ns_cold, cold_blocks);
+    ns_cold = std::min(ns_cold, kMaxSplits - ns_hot);
+  }
+  int blocks_per_split = 1, tiles_per_split = 1;
+  if (ns_cold > 0) {
+    blocks_per_split = (int)((cold_blocks + ns_cold - 1) / ns_cold);
+    ns_cold = (int)((cold_blocks + blocks_per_split - 1) / blocks_per_split);
+  }
+  if (ns_hot > 0) {
+    tiles_per_split = (hot_tiles + ns_hot - 1) / ns_hot;
+    ns_hot = (hot_tiles + tiles_per_split - 1) / tiles_per_split;
+  }
+
+  __half* qrot = (__half*)(c->ws + c->W.qrot);
+  __half* qsk = (__half*)(c->ws + c->W.qsk);
+  float* qscale = (float*)(c->ws + c->W.qscale);
+  float* part = (float*)(c->ws + c->W.part);
+
+  if (ns_cold > 0) {
+    QPrepArgs qa{};
+    qa.q = (const __half*)q;
+    qa.signs = c->signs();
+    qa.St = c->St();
+    qa.qrot = qrot;
+    qa.qsk = qsk;
+    qa.qscale = qscale;
+    qa.heads = heads;
+    qa.d = d;
+    qa.m = m;
+    if (launch_qprep(qa, stream) != cudaSuccess) return TQ_ERR_CUDA;
+  }
+  if (ns_cold + ns_hot > 0) {
+    AttendArgs a{};
+    a.q = (const __half*)q;
+    a.qrot = qrot;
+    a.qsk = qsk;
+    a.qscale = qscale;
+    a.hot_k = c->hot_k();
+    a.hot_v = c->hot_v();
+    a.cold = c->cold;
+    a.part = part;
+    a.status = c->status();
+    a.L = c->L;
+    a.units = units;
+    a.G = G;
+    a.Hq = cf.num_q_heads;
+    a.Hkv = cf.num_kv_heads;
+    a.W = cf.hot_window;
+    a.n_hot = c->n_hot;
+    a.n_cold = c->n_cold;
+    a.ns_cold = ns_cold;
+    a.ns_hot = ns_hot;
+    a.blocks_per_split = blocks_per_split;
+    a.tiles_per_split = tiles_per_split;
+    a.max_splits = kMaxSplits;
+    a.log2e_sigma = (float)(1.4426950408889634 * (double)sigma);
+    if (c->ev_start && cudaEventRecord(c->ev_start, stream) != cudaSuccess) return TQ_ERR_CUDA;
+    if (launch_attend(a, stream) != cudaSuccess) return TQ_ERR_CUDA;
+    if (c->ev_stop && cudaEventRecord(c->ev_stop, stream) != cudaSuccess) return TQ_ERR_CUDA;
+  }
+  CombineArgs ca{};
+  ca.part = part;
+  ca.signs = c->signs();
+  ca.out = out;
+  ca.units = units;
+  ca.G = G;
+  ca.Hkv = cf.num_kv_heads;
+  ca.Hq = cf.num_q_heads;
+  ca.d = d;
+  ca.ns_cold = ns_cold;
+  ca.ns_hot = ns_hot;
+  ca.max_splits = kMaxSplits;
+  ca.batch = cf.batch;
+  if (launch_combine(ca, stream) != cudaSuccess) return TQ_ERR_CUDA;
+  return TQ_OK;
+}
+
+tq_status tq_set_attend_events(tq_cache* c, cudaEvent_t start, cudaEvent_t stop) {
+  if (!c || (start == nullptr) != (stop == nullptr)) return TQ_ERR_INVALID_ARG;
+  c->ev_start = start;
+  c->ev_stop = stop;
+  return TQ_OK;
+}
+
+tq_status tq_get_status(tq_cache* c, cudaStream_t stream) {
+  if (!c) return TQ_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return TQ_ERR_CUDA;
+  int word = 0;
+  if (cudaMemcpy(&word, c->status(), sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return TQ_ERR_CUDA;
+  if (word != 0 && cudaMemset(c->status(), 0, sizeof(int)) != cudaSuccess) return TQ_ERR_CUDA;
+  if (word & kStatusTimeout) return TQ_ERR_TIMEOUT;
+  if (word & kStatusRange) return TQ_ERR_RANGE;
+  return TQ_OK;
+}
+
+tq_status tq_export_cold(tq_cache* c, int32_t row, int32_t kv_head, int64_t start, int64_t count,
+                         uint8_t* k_codes, uint8_t* k_bits, uint16_t* k_s16, uint16_t* k_rn16,
+                         uint8_t* v_codes, uint16_t* v_s16, cudaStream_t stream) {
+  if (!c || row < 0 || row >= c->cfg.batch || kv_head < 0 || kv_head >= c->cfg.num_kv_heads ||
+      start < 0 || count < 0 || start + count > c->n_cold)
+    return TQ_ERR_INVALID_ARG;
+  if (count == 0) return TQ_OK;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return TQ_ERR_CUDA;
+  const Layout& L = c->L;
+  const int TB = kTokensPerBlock;
+  const int64_t unit = (int64_t)row * c->cfg.num_kv_heads + kv_head;
+  const int64_t b0 = start / TB, b1 = (start + count - 1) / TB;
+  std::vector<uint8_t> buf((size_t)(b1 - b0 + 1) * L.block_bytes);
+  const uint8_t* src = c->cold + ((size_t)unit * L.blocks_per_unit + b0) * L.block_bytes;
+  if (cudaMemcpy(buf.data(), src, buf.size(), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return TQ_ERR_CUDA;
+  for (int64_t i = 0; i < count; ++i) {
+    const int64_t t = start + i;
+    const uint8_t* blk = buf.data() + (size_t)(t / TB - b0) * L.block_bytes;
+    const int r = (int)(t % TB);
+    if (k_codes) std::memcpy(k_codes + i * L.kc_bytes, blk + L.off_kc + r * L.kc_bytes, L.kc_bytes);
+    if (k_bits) std::memcpy(k_bits + i * L.sg_bytes, blk + L.off_ks + r * L.sg_bytes, L.sg_bytes);
+    if (k_s16) std::memcpy(k_s16 + i, blk + L.off_ksc + 2 * r, 2);
+    if (k_rn16) std::memcpy(k_rn16 + i, blk + L.off_krn + 2 * r, 2);
+    if (v_codes) std::memcpy(v_codes + i * L.kc_bytes, blk + L.off_vc + r * L.kc_bytes, L.kc_bytes);
+    if (v_s16) std::memcpy(v_s16 + i, blk + L.off_vsc + 2 * r, 2);
+  }
+  return TQ_OK;
+}
+
+tq_status tq_rotation_signs(uint64_t seed, int32_t d, int8_t* signs) {
+  if (!signs || d < 1) return TQ_ERR_INVALID_ARG;
+  std::vector<double> s(d);
+  gen_signs(seed, d, s.data());
+  for (int i = 0; i < d; ++i) signs[i] = (int8_t)s[i];
+  return TQ_OK;
+}
+
+tq_status tq_qjl_matrix(uint64_t seed, int32_t m, int32_t d, float* S) {
+  if (!S || m < 1 || d < 1) return TQ_ERR_INVALID_ARG;
+  gen_qjl(seed, m, d, S);
+  return TQ_OK;
+}
+
+}  // extern "C"

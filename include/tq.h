@@ -1,0 +1,226 @@
+/*
+ * tq.h -- C ABI of the compressed KV-cache library (B200, sm_100a).
+ *
+ * One hot path: TurboQuant-style compression of the KV cache (a seeded
+ * randomized Hadamard rotation, 2-D polar quantization with an fp16 scale,
+ * a 1-bit QJL sketch of the key residual) and single-token decode attention
+ * computed straight from the packed cold cache next to a full-precision hot
+ * ring of the most recent tokens (Monarch's hot/cold split).
+ *
+ * Sources (page title, section):
+ *  [TQ-PL]   "TurboQuant: kompresja KV-cache w LLM 6 razy bez utraty
+ *            dokładności" -- "Zasada działania PolarQuant" (rotate, then
+ *            radius/angle, then quantize), "Kompensacja błędów przez QJL"
+ *            (1-bit code of the residual that preserves inner products).
+ *  [TQ-ES]   "TurboQuant: optimización de memoria para KV caches en
+ *            inferencia de LLMs" -- "Flujo de Cuantificación de KV Cache con
+ *            TurboQuant", steps 1-7 (step 6: attention logits computed from
+ *            the compressed cache).
+ *  [TQ-3B]   "Compresión del caché KV de los LLM a 3 bits: TurboQuant de
+ *            Google Research" -- "Aplicaciones más allá de los LLMs"
+ *            (vector search over the same codes).
+ *  [MONARCH] "Monarch v3: Paginación KV Inspirada en NES para una Inferencia
+ *            de LLM 78% Más Rápida" -- "Cómo funciona" (hot region at full
+ *            precision, cold region compressed, sliding-window eviction),
+ *            "Bucle de Decodificación Simplificado" (evict_oldest_to_cold;
+ *            aggregate, softmax, apply).
+ *  [TC]      "Tensor Cache: Eviction-conditioned Associative Memory for
+ *            Transformers" -- "Metodología" (the first-level cache is a ring
+ *            whose overwrite becomes a write into the second tier).
+ *
+ * Conventions for every call
+ *  - Memory: the caller allocates every device buffer (sizes from
+ *    tq_cache_bytes); the library never calls cudaMalloc.  The library owns
+ *    only the host-side handle (freed by tq_cache_destroy).  Input buffers
+ *    are borrowed until the stream-ordered work that reads them completes.
+ *  - Streams: every device call is asynchronous on the given stream and
+ *    never synchronizes, except tq_get_status and the tq_export_* helpers.
+ *  - Errors: argument, shape and capacity errors are returned synchronously
+ *    before any launch, and leave the handle unchanged.  Launch failures
+ *    return TQ_ERR_CUDA.  Conditions detected on the device (an fp16 scale
+ *    that overflows, a bounded wait that gave up) are latched into a device
+ *    status word and returned (and cleared) by tq_get_status.  Nothing in
+ *    the library traps or asserts on the device.
+ *  - Layouts: fp16 buffers are IEEE binary16, passed as void*.  Shapes are
+ *    row-major and contiguous.  B = batch, Hq / Hkv = query / KV heads,
+ *    G = Hq / Hkv, d = head_dim, W = hot window, m = QJL bits.
+ *  - Thread safety: a handle may be used from one host thread at a time.
+ */
+#ifndef TQ_H_
+#define TQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define TQ_ABI_VERSION 1
+
+typedef enum tq_status {
+  TQ_OK = 0,
+  TQ_ERR_INVALID_ARG = 1,   /* null pointer, bad shape or value            */
+  TQ_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. head_dim 96) */
+  TQ_ERR_CAPACITY = 3,      /* the cold store would exceed its capacity    */
+  TQ_ERR_RANGE = 4,         /* (device) an fp16 scale or norm overflowed   */
+  TQ_ERR_TIMEOUT = 5,       /* (device) a bounded wait gave up             */
+  TQ_ERR_CUDA = 6           /* a CUDA runtime call or launch failed        */
+} tq_status;
+
+/* One handle per attention layer. */
+typedef struct tq_config {
+  int32_t batch;            /* B >= 1                                        */
+  int32_t num_q_heads;      /* Hq, a multiple of Hkv with G = Hq/Hkv <= 8    */
+  int32_t num_kv_heads;     /* Hkv >= 1                                      */
+  int32_t head_dim;         /* d: 64 or 128                                  */
+  int32_t hot_window;       /* W >= 1: tokens kept at fp16 in the hot ring   */
+  int64_t cold_capacity;    /* max compressed tokens per (row, kv head)      */
+  int32_t b_r;              /* radius bits   >= 1                            */
+  int32_t b_theta;          /* angle bits    >= 1, b_r + b_theta <= 8        */
+  int32_t qjl_bits;         /* m: 64 or 128 sign bits per key                */
+  uint64_t seed;            /* drives the rotation signs D and QJL matrix S  */
+} tq_config;
+
+typedef struct tq_cache tq_cache;
+
+/* Human-readable name of a status code (static string). */
+const char* tq_status_string(tq_status s);
+
+/* TQ_ABI_VERSION of the loaded library. */
+int32_t tq_abi_version(void);
+
+/*
+ * Device memory the caller must provide for a configuration.
+ *   hot_bytes   fp16 hot ring, K then V, each [B, Hkv, W, d].
+ *   cold_bytes  packed cold store: per (row, kv head) a run of 64-token
+ *               blocks; inside a block, field planes (K codes, K sign bits,
+ *               K scales, K residual norms, V codes, V scales), token-major
+ *               and 16-byte aligned.  Bytes per cold token per kv head:
+ *               K: d/2*(b_r+b_theta)/8 + m/8 + 4, V: d/2*(b_r+b_theta)/8 + 2.
+ *   workspace_bytes  rotation signs, QJL matrix, per-call query transforms,
+ *               split partials and the device status word.
+ * Each buffer must be 256-byte aligned.  Any output pointer may be NULL.
+ */
+tq_status tq_cache_bytes(const tq_config* cfg, size_t* hot_bytes,
+                         size_t* cold_bytes, size_t* workspace_bytes);
+
+/*
+ * Bind a handle to caller-owned device buffers and upload the seeded method
+ * randomness (D and S, generated on the host by the library) into the
+ * workspace with stream-ordered copies.  The cache starts empty.  *out is
+ * valid until tq_cache_destroy.  The buffers' previous contents are ignored.
+ */
+tq_status tq_cache_create(const tq_config* cfg, void* hot_mem, void* cold_mem,
+                          void* workspace_mem, cudaStream_t stream,
+                          tq_cache** out);
+
+/* Free the host handle (device buffers stay the caller's). NULL is a no-op. */
+tq_status tq_cache_destroy(tq_cache* cache);
+
+/* Host-side counters: compressed tokens, valid hot tokens, next ring slot. */
+tq_status tq_cache_counts(const tq_cache* cache, int64_t* n_cold,
+                          int32_t* n_hot, int32_t* ring_pos);
+
+/*
+ * Compress n new tokens straight into the cold store (prefill path).
+ * [TQ-PL] "Zasada działania PolarQuant" + "Kompensacja błędów przez QJL";
+ * [TQ-ES] steps 1-5.  For every (row, kv head) and token, K and V are
+ * rotated (y = H_d D x / sqrt(d)), split into d/2 pairs mapped to
+ * (rho, theta), coded on an endpoint radius grid (b_r bits, scale
+ * s16 = fp16(max rho)) and a periodic angle grid (b_theta bits); keys also
+ * store fp16(||r||) and m bits [(S r)_i >= 0] of the residual r = y - y_hat.
+ * The code decisions are computed in float64 on the device.
+ *   k, v  device fp16 [B, Hkv, n, d] (contiguous)
+ *   n     >= 0 (0 is a no-op)
+ * Tokens land at cold indices n_cold .. n_cold+n-1 of every (row, kv head).
+ * Returns TQ_ERR_CAPACITY (nothing launched) if n_cold + n > cold_capacity.
+ */
+tq_status tq_encode_append(tq_cache* cache, const void* k, const void* v,
+                           int64_t n, cudaStream_t stream);
+
+/*
+ * Insert n new tokens into the hot ring (decode path).
+ * [MONARCH] "Cómo funciona" (sliding-window eviction) and "Bucle de
+ * Decodificación Simplificado" (evict_oldest_to_cold); [TC] "Metodología"
+ * (ring overwrite feeds the second tier).  Equivalent to n single inserts in
+ * order: when the ring already holds W tokens, the oldest one is encoded
+ * exactly as tq_encode_append does and appended to the cold store, then the
+ * new token takes its slot (pos mod W).
+ *   k_new, v_new  device fp16 [B, Hkv, n, d];  n >= 1
+ * Returns TQ_ERR_CAPACITY (nothing launched) if the evictions would overflow
+ * the cold store.
+ */
+tq_status tq_evict_window(tq_cache* cache, const void* k_new,
+                          const void* v_new, int32_t n, cudaStream_t stream);
+
+/*
+ * Single-token decode attention over hot U cold tokens.
+ * [TQ-ES] step 6 (logits from the compressed cache); [MONARCH] "Bucle de
+ * Decodificación Simplificado" (aggregate, softmax, apply).  For query head
+ * h (kv head h / G), with q' = R q and q'' = S q':
+ *   hot token:  l = sigma <q, k>
+ *   cold token: l = sigma ( s16/(2^b_r-1) <q', y_hat_unit>
+ *                           + rn16 sqrt(pi/2)/m <q'', 2 bits - 1> )
+ *   p = softmax(l) over every valid hot and cold token
+ *   out = sum_hot p v + R^T sum_cold p s16_v/(2^b_r-1) v_hat_unit
+ * Accumulation is fp32; the products run on tensor cores with fp16
+ * operands.  Every valid token is attended (no mask; K is cached after any
+ * positional encoding).
+ *   q      device fp16 [B, Hq, d]
+ *   out    device fp32 [B, Hq, d]
+ *   softmax_scale  sigma; 0 selects 1/sqrt(d)
+ * With no valid token at all, out is zero.
+ */
+tq_status tq_decode_attention(tq_cache* cache, const void* q, float* out,
+                              float softmax_scale, cudaStream_t stream);
+
+/*
+ * Synchronize `stream`, then return and clear the latched device status
+ * (TQ_OK, TQ_ERR_RANGE or TQ_ERR_TIMEOUT), or TQ_ERR_CUDA if the stream
+ * itself reports an error.
+ */
+tq_status tq_get_status(tq_cache* cache, cudaStream_t stream);
+
+/*
+ * Copy cold records of one (row, kv head) to HOST buffers in canonical
+ * form (synchronizes `stream`): pair j's word (c_r << b_theta) | c_theta
+ * LSB-first at bit j*(b_r+b_theta); sign bit i at bit i; fp16 raw bits.
+ *   k_codes [count, d/2*(b_r+b_theta)/8]  k_bits [count, m/8]
+ *   k_s16 [count]  k_rn16 [count]  v_codes [count, ...]  v_s16 [count]
+ * Requires start + count <= n_cold.  Any output pointer may be NULL.
+ */
+tq_status tq_export_cold(tq_cache* cache, int32_t row, int32_t kv_head,
+                         int64_t start, int64_t count, uint8_t* k_codes,
+                         uint8_t* k_bits, uint16_t* k_s16, uint16_t* k_rn16,
+                         uint8_t* v_codes, uint16_t* v_s16,
+                         cudaStream_t stream);
+
+/*
+ * Measurement hook: when `start` and `stop` are non-NULL, every following
+ * tq_decode_attention call on this handle records `start` on its stream
+ * right before the attention kernel and `stop` right after it, so that a
+ * caller can time that kernel alone with cudaEventElapsedTime.  Pass NULLs
+ * to stop recording.  The events are borrowed, not owned.
+ */
+tq_status tq_set_attend_events(tq_cache* cache, cudaEvent_t start, cudaEvent_t stop);
+
+/*
+ * The library's own seeded method randomness (host only, no GPU needed),
+ * exactly as uploaded by tq_cache_create:
+ *   signs[i] = +1 / -1  (i < d)         QJL matrix S [m, d] float32.
+ * Generator: rand64(seed, stream, i) = mix64(mix64(seed + stream)
+ * + (i + 1) * 0x9E3779B97F4A7C15) with the SplitMix64 finalizer mix64;
+ * stream 0: sign = top bit clear ? +1 : -1; stream 1: Box-Muller (first
+ * output) from draws 2k, 2k+1 for entry k = row * d + col, in float64 with
+ * the C library's log/cos/sqrt, rounded to float32.
+ */
+tq_status tq_rotation_signs(uint64_t seed, int32_t d, int8_t* signs);
+tq_status tq_qjl_matrix(uint64_t seed, int32_t m, int32_t d, float* S);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TQ_H_ */
