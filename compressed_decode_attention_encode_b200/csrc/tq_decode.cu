@@ -5,22 +5,25 @@
 // and cold scores, softmax, apply).
 //
 // Three launches per call:
-//   qprep    q' = R q (fp32 Hadamard butterflies), q'' = S q', both stored
-//            as fp16 with a power-of-two scale per head.
-//   attend   one CTA per (row, kv head, split).  A split streams either
-//            64-token cold blocks or 64-token hot tiles through shared
-//            memory.  Per warp and 16-token tile the three products run on
-//            tensor cores (mma.sync m16n8k16, fp16 in, fp32 accumulate):
-//              cold logits  [16 tok x d] . q'   -- A operand = LUT-dequantized
-//                           polar pairs, one 32-bit LUT load per pair
-//              QJL term     [16 tok x m] . q''  -- A operand = +-1 built from
-//                           the sign bits with one shift and one LOP3
-//              P V          [d x 16 tok] . P    -- P transposed in registers
-//                           with movmatrix
-//            with an online softmax across tiles (exp2 domain).  The GQA
-//            group (G <= 8 query heads) is the n = 8 side of every MMA.
-//   combine  merges the split partials, applies R^T once to the cold sum
-//            (Hadamard butterflies), normalizes.
+//   qprep    q' = R q (fp32 Hadamard butterflies) split into fp16 hi + lo
+//            parts, q'' = S q' in fp16; power-of-two scale per head.
+//   attend   one wave of CTAs.  Cold CTAs take equal contiguous runs of the
+//            flattened (unit, 64-token block) list and stream them through a
+//            multi-stage shared-memory ring filled by cp.async.bulk copies
+//            (mbarrier completion, bounded waits).  Per warp and 16-token
+//            tile the products run on tensor cores (mma.sync m16n8k16, fp16
+//            in, fp32 accumulate):
+//              cold logits [16 tok x d] . (q'hi + q'lo) -- A = LUT-dequantized
+//                          polar pairs, one 32-bit LUT load per pair
+//              QJL term    [16 tok x m] . q''        -- A = +-1 from the sign
+//                          bits (one shift + one LOP3 per pair)
+//              P V         [d x 16 tok] . P          -- P transposed in
+//                          registers with movmatrix
+//            with an online softmax (exp2 domain).  The GQA group (G <= 8
+//            query heads) is the n = 8 side of every MMA.  Hot CTAs stream
+//            fp16 tiles through padded shared memory (ldmatrix).
+//   combine  merges the partials of each (row, head), applies R^T once to
+//            the cold sum (Hadamard butterflies) and normalizes.
 #include <cfloat>
 
 #include "tq_internal.cuh"
@@ -32,7 +35,9 @@ constexpr unsigned kFull = 0xffffffffu;
 constexpr int kThreads = 128;          // 4 warps; each takes 16 tokens of a 64-token block
 constexpr float kNegInf = -INFINITY;
 constexpr float kSqrtHalfPi = 1.2533141373155001f;   // sqrt(pi / 2)
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // bounded mbarrier waits
 
+// ---- PTX helpers -----------------------------------------------------------
 __device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                          uint32_t a3, uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -62,6 +67,71 @@ __device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], uint32_t addr) {
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ float fast_log2(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Waits for phase `parity` of an mbarrier, giving up after kWaitLimitNs.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_ns() - t0 > kWaitLimitNs) return false;
+  }
+  return true;
+}
+
+// Global -> shared bulk copy completing on an mbarrier (no multicast).
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes,
+                                         uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
 }
 
 __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
@@ -100,9 +170,25 @@ __device__ __forceinline__ uint32_t field(const uint32_t (&w)[NW], int pos) {
   return v & ((1u << BW) - 1u);
 }
 
+// The BW-bit field at bit `pos` (compile-time after unrolling), returned
+// already shifted left by SH and masked, so that `| lane * (1 << SH) / 32`
+// gives the byte offset of this lane's copy of the LUT entry: one funnel
+// shift plus one LOP3.
+template <int BW, int SH, int NW>
+__device__ __forceinline__ uint32_t field_shifted(const uint32_t (&w)[NW], int pos) {
+  const int wi = pos >> 5, bi = pos & 31;
+  uint32_t v;
+  if (bi + BW <= 32 || wi + 1 >= NW)
+    v = bi >= SH ? (w[wi] >> (bi - SH)) : (w[wi] << (SH - bi));
+  else
+    v = __funnelshift_r(w[wi], w[wi + 1], bi - SH);   // straddling: bi > 32 - BW >= SH
+  return v & (((1u << BW) - 1u) << SH);
+}
+
 // Online-softmax step over one 16-token tile for the thread's two heads
-// (2*tig, 2*tig+1).  l2[0..1]: token gid, l2[2..3]: token gid+8.  Returns the
-// factor by which previously accumulated sums must be rescaled.
+// (2*tig, 2*tig+1).  l2[0..1]: token gid, l2[2..3]: token gid+8 (log2
+// domain).  Writes p = exp2(l2 - m_new) and the factor corr by which sums
+// accumulated so far must be rescaled.
 __device__ __forceinline__ void softmax_tile(const float (&l2)[4], float (&m_run)[2],
                                              float (&p)[4], float (&corr)[2]) {
   float t0 = fmaxf(l2[0], l2[2]), t1 = fmaxf(l2[1], l2[3]);
@@ -113,74 +199,105 @@ __device__ __forceinline__ void softmax_tile(const float (&l2)[4], float (&m_run
   }
   const float n0 = fmaxf(m_run[0], t0), n1 = fmaxf(m_run[1], t1);
   const float r0 = n0 == kNegInf ? 0.f : n0, r1 = n1 == kNegInf ? 0.f : n1;
-  corr[0] = exp2f(m_run[0] - r0);
-  corr[1] = exp2f(m_run[1] - r1);
-  p[0] = exp2f(l2[0] - r0);
-  p[1] = exp2f(l2[1] - r1);
-  p[2] = exp2f(l2[2] - r0);
-  p[3] = exp2f(l2[3] - r1);
+  corr[0] = fast_exp2(m_run[0] - r0);
+  corr[1] = fast_exp2(m_run[1] - r1);
+  p[0] = fast_exp2(l2[0] - r0);
+  p[1] = fast_exp2(l2[1] - r1);
+  p[2] = fast_exp2(l2[2] - r0);
+  p[3] = fast_exp2(l2[3] - r1);
   m_run[0] = n0;
   m_run[1] = n1;
 }
 
 // ---------------------------------------------------------------------------
-// q-prep
+// q-prep: 8 heads per block, one warp per head for the rotation; S q' is
+// register-blocked so that every S element is read once per block.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(128) qprep_kernel(const QPrepArgs a) {
-  __shared__ float sv[256];
-  __shared__ float sq[256];
-  __shared__ float red[32];
-  const int h = blockIdx.x, t = threadIdx.x, D = a.d, M = a.m;
-  for (int i = t; i < D; i += blockDim.x)
-    sv[i] = __half2float(a.q[(size_t)h * D + i]) * (float)a.signs[i];
-  __syncthreads();
+template <int D, int M>
+__global__ void __launch_bounds__(256) qprep_kernel(const QPrepArgs a) {
+  constexpr int E = D / 32;
+  constexpr int HPT = 8 * M / 256;       // heads per thread in S q'
+  __shared__ float sq[8][D];
+  __shared__ float sqq[8][M];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int h = blockIdx.x * 8 + warp;
+  const bool live = h < a.heads;
+  float x[E];
+#pragma unroll
+  for (int i = 0; i < E; ++i)
+    x[i] = live ? __half2float(a.q[(size_t)h * D + lane * E + i]) * (float)a.signs[lane * E + i] : 0.f;
+#pragma unroll
   for (int hh = 1; hh < D; hh <<= 1) {
-    for (int i = t; i < D; i += blockDim.x) {
-      if (!(i & hh)) {
-        const float x = sv[i], y = sv[i + hh];
-        sv[i] = x + y;
-        sv[i + hh] = x - y;
+    if (hh < E) {
+#pragma unroll
+      for (int i = 0; i < E; ++i)
+        if (!(i & hh)) {
+          const float p = x[i], q = x[i + hh];
+          x[i] = p + q;
+          x[i + hh] = p - q;
+        }
+    } else {
+      const int lm = hh / E;
+#pragma unroll
+      for (int i = 0; i < E; ++i) {
+        const float o = __shfl_xor_sync(kFull, x[i], lm);
+        x[i] = (lane & lm) ? (o - x[i]) : (x[i] + o);
       }
     }
-    __syncthreads();
   }
   const float inv = rsqrtf((float)D);
   float amax = 0.f;
-  for (int i = t; i < D; i += blockDim.x) {
-    sv[i] *= inv;
-    amax = fmaxf(amax, fabsf(sv[i]));
+#pragma unroll
+  for (int i = 0; i < E; ++i) {
+    x[i] *= inv;
+    sq[warp][lane * E + i] = x[i];
+    amax = fmaxf(amax, fabsf(x[i]));
   }
+#pragma unroll
   for (int o = 16; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, o));
-  if ((t & 31) == 0) red[t >> 5] = amax;
-  __syncthreads();
-  amax = 0.f;
-  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) amax = fmaxf(amax, red[w]);
   const float al1 = amax > 0.f ? exp2f(-floorf(log2f(amax))) : 1.f;
-  for (int i = t; i < D; i += blockDim.x) a.qrot[(size_t)h * D + i] = __float2half_rn(sv[i] * al1);
+  if (live) {
+#pragma unroll
+    for (int i = 0; i < E; ++i) {
+      const float v = x[i] * al1;
+      const __half hi = __float2half_rn(v);
+      a.qrot[(size_t)h * 2 * D + lane * E + i] = hi;
+      a.qrot[(size_t)h * 2 * D + D + lane * E + i] = __float2half_rn(v - __half2float(hi));
+    }
+  }
+  __syncthreads();
+  {
+    const int i = threadIdx.x % M;
+    const int hb = (threadIdx.x / M) * HPT;
+    float acc[HPT];
+#pragma unroll
+    for (int k = 0; k < HPT; ++k) acc[k] = 0.f;
+#pragma unroll 4
+    for (int j = 0; j < D; ++j) {
+      const float sv = __ldg(a.St + (size_t)j * M + i);
+#pragma unroll
+      for (int k = 0; k < HPT; ++k) acc[k] = fmaf(sv, sq[hb + k][j], acc[k]);
+    }
+#pragma unroll
+    for (int k = 0; k < HPT; ++k) sqq[hb + k][i] = acc[k];
+  }
   __syncthreads();
   float bmax = 0.f;
-  for (int i = t; i < M; i += blockDim.x) {
-    float acc = 0.f;
-    for (int j = 0; j < D; ++j) acc = fmaf(__ldg(a.St + (size_t)j * M + i), sv[j], acc);
-    sq[i] = acc;
-    bmax = fmaxf(bmax, fabsf(acc));
-  }
+  for (int i = lane; i < M; i += 32) bmax = fmaxf(bmax, fabsf(sqq[warp][i]));
+#pragma unroll
   for (int o = 16; o; o >>= 1) bmax = fmaxf(bmax, __shfl_xor_sync(kFull, bmax, o));
-  if ((t & 31) == 0) red[8 + (t >> 5)] = bmax;
-  __syncthreads();
-  bmax = 0.f;
-  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) bmax = fmaxf(bmax, red[8 + w]);
   const float al2 = bmax > 0.f ? exp2f(-floorf(log2f(bmax))) : 1.f;
+  if (!live) return;
   // sign-fragment order: for chunk tig (m/4 signs) and slot u < m/8 the pair
   // (q''[c + m/8 - 1 - u], q''[c + m/4 - 1 - u]), c = tig * m/4.
-  const int Q4 = M / 4, H = M / 8;
-  for (int i = t; i < M; i += blockDim.x) {
+  constexpr int Q4 = M / 4, H = M / 8;
+  for (int i = lane; i < M; i += 32) {
     const int tg = i / Q4, j = i % Q4;
     const int u = j < H ? (H - 1 - j) : (2 * H - 1 - j);
     const int pos = (tg * H + u) * 2 + (j < H ? 0 : 1);
-    a.qsk[(size_t)h * M + pos] = __float2half_rn(sq[i] * al2);
+    a.qsk[(size_t)h * M + pos] = __float2half_rn(sqq[warp][i] * al2);
   }
-  if (t == 0) {
+  if (lane == 0) {
     a.qscale[2 * h] = 1.f / al1;
     a.qscale[2 * h + 1] = 1.f / al2;
   }
@@ -194,308 +311,508 @@ struct AttendShape {
   static constexpr int P = D / 2;
   static constexpr int NT = D / 16;                 // k-steps of the K logits == PV m-tiles
   static constexpr int QS = M / 16;                 // k-steps of the QJL product
-  static constexpr int KC = P * BW / 8;             // code bytes per vector
-  static constexpr int SG = M / 8;                  // sign bytes per key
-  static constexpr int TB = kTokensPerBlock;
+  static constexpr int PT = P / 4;                  // K pairs per lane (per token)
+  static constexpr int PV = P / 8;                  // V pairs per lane (per token)
+  static constexpr int KWT = (2 * PT * BW + 31) / 32;
+  static constexpr int SW = (2 * (M / 4) + 31) / 32;
+  static constexpr int VWT = (4 * PV * BW + 31) / 32;
   static constexpr int OFF_KC = 0;
-  static constexpr int OFF_KS = OFF_KC + TB * KC;
-  static constexpr int OFF_KSC = OFF_KS + TB * SG;
-  static constexpr int OFF_KRN = OFF_KSC + TB * 2;
-  static constexpr int OFF_VC = OFF_KRN + TB * 2;
-  static constexpr int OFF_VSC = OFF_VC + TB * KC;
-  static constexpr int BLOCK = OFF_VSC + TB * 2;
-  static constexpr int KBITS = (P / 4) * BW;        // bits of a thread's K chunk
-  static constexpr int KW = (KBITS + 31) / 32;
-  static constexpr int VBITS = (P / 8) * BW;        // bits of a thread's V chunk
-  static constexpr int VW = (VBITS + 31) / 32;
+  static constexpr int OFF_KS = OFF_KC + 128 * KWT;
+  static constexpr int OFF_KSC = OFF_KS + 128 * SW;
+  static constexpr int OFF_VC = OFF_KSC + 64;
+  static constexpr int OFF_VSC = OFF_VC + 128 * VWT;
+  static constexpr int TT = OFF_VSC + 32;           // tile bytes
+  static constexpr int TB = kTokensPerBlock;
+  static constexpr int BLOCK = kTilesPerBlock * TT;
   static constexpr int NLUT = 1 << BW;
-  static constexpr int LUT_BYTES = NLUT * 32 * 4;   // one copy per lane: no bank conflicts
+  static constexpr int KLUT_BYTES = NLUT * 32 * 8;  // (hi, lo) half2 per lane copy
+  static constexpr int VLUT_BYTES = NLUT * 32 * 4;  // hi half2 per lane copy
+  // LUTs up to 48 KB live in static shared memory, whose address the
+  // compiler folds into the load's immediate; larger ones are dynamic.
+  static constexpr bool STATIC_LUT = KLUT_BYTES + VLUT_BYTES <= 49152;
+  static constexpr int DYN_LUT = STATIC_LUT ? 0 : KLUT_BYTES + VLUT_BYTES;
   static constexpr int RS = 2 * D + 16;             // padded hot row stride (bytes)
   static constexpr int HOT_BYTES = 2 * TB * RS;
-  static constexpr int MERGE_BYTES = (64 + 4 * 8 * D) * 4;
-  static constexpr int STAGE = (BLOCK > HOT_BYTES ? (BLOCK > MERGE_BYTES ? BLOCK : MERGE_BYTES)
-                                                   : (HOT_BYTES > MERGE_BYTES ? HOT_BYTES : MERGE_BYTES));
-  static constexpr int SMEM = LUT_BYTES + STAGE;
+  static constexpr int RING_BUDGET = KLUT_BYTES >= 65536 ? 20480 : 30720;
+  static constexpr int NS_RAW = RING_BUDGET / BLOCK;
+  static constexpr int NS = NS_RAW < 2 ? 2 : (NS_RAW > 8 ? 8 : NS_RAW);   // ring stages
+  static constexpr int RING = NS * BLOCK > HOT_BYTES ? NS * BLOCK : HOT_BYTES;
+  static constexpr int MERGE_BYTES = (64 + 8 * D) * 4;
+  static constexpr int OFF_VLUT = KLUT_BYTES;        // (dynamic LUT case)
+  static constexpr int OFF_RING = DYN_LUT;
+  static constexpr int OFF_MERGE = OFF_RING + RING;
+  static constexpr int OFF_BAR = OFF_MERGE + MERGE_BYTES;
+  static constexpr int SMEM = OFF_BAR + 8 * NS + 8 * NS + 16;   // + per-stage counters, flags
 };
 
-template <int D, int M, int BW>
-__global__ void __launch_bounds__(kThreads) attend_kernel(const AttendArgs a) {
-  using S = AttendShape<D, M, BW>;
-  extern __shared__ __align__(16) uint8_t smem[];
-  uint32_t* lut = reinterpret_cast<uint32_t*>(smem);
-  uint8_t* stage = smem + S::LUT_BYTES;
+// 2-word-major per-lane words of a tile plane (see Layout).
+template <int NW>
+__device__ __forceinline__ void load_lane_words(const uint8_t* plane, int lane, uint32_t (&w)[NW]) {
+#pragma unroll
+  for (int g = 0; 2 * g < NW; ++g) {
+    if (2 * g + 1 < NW) {
+      const uint2 v = *reinterpret_cast<const uint2*>(plane + g * 256 + lane * 8);
+      w[2 * g] = v.x;
+      w[2 * g + 1] = v.y;
+    } else {
+      w[2 * g] = *reinterpret_cast<const uint32_t*>(plane + g * 256 + lane * 4);
+    }
+  }
+}
 
+// Spreads two 16-bit sign chunks so that slot u's bits land at 15 and 31
+// after a left shift by u (m = 64 layout).
+__device__ __forceinline__ uint32_t spread16(uint32_t c) {
+  return ((c & 0xffu) << 8) | ((c >> 8 & 0xffu) << 24);
+}
+
+constexpr float kLazyHeadroom = 8.f;   // log2 units the reference max may lag
+
+// Per-warp softmax / accumulator state for one unit.
+template <int NT>
+struct WarpState {
+  float m_run[2], l_run[2], mp_run[2];
+  float O[NT][4];
+  __device__ __forceinline__ void reset() {
+    m_run[0] = m_run[1] = kNegInf;
+    mp_run[0] = mp_run[1] = kNegInf;
+    l_run[0] = l_run[1] = 0.f;
+#pragma unroll
+    for (int i = 0; i < NT; ++i) O[i][0] = O[i][1] = O[i][2] = O[i][3] = 0.f;
+  }
+};
+
+// Merges the 4 warps' states into one partial {m, l, o[D]} per head and
+// writes it to `dst` ([G][D + 2]).  Called by all threads of the CTA; uses
+// 4 KB of shared memory (per-warp m / l, then the o sums by shared atomics).
+template <int D, int NT>
+__device__ __forceinline__ void flush_partial(WarpState<NT>& st, bool hot, int Lr, int G,
+                                              float* merge, float* dst) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int gid = lane >> 2, tig = lane & 3;
-  const int per_unit = a.ns_cold + a.ns_hot;
-  const int unit = blockIdx.x / per_unit;
-  const int split = blockIdx.x % per_unit;
-  const bool hot = split >= a.ns_cold;
-  const int b = unit / a.Hkv, kvh = unit % a.Hkv;
-  const int G = a.G;
-  const int head0 = b * a.Hq + kvh * G;
-  const int Lr = (1 << a.L.b_r) - 1;
-  const int tb = warp * 16;            // this warp's tokens inside a block / tile
-
-  float m_run[2] = {kNegInf, kNegInf};
-  float l_run[2] = {0.f, 0.f};
-  float mp_run[2] = {kNegInf, kNegInf};
-  float O[S::NT][4];
-#pragma unroll
-  for (int i = 0; i < S::NT; ++i) O[i][0] = O[i][1] = O[i][2] = O[i][3] = 0.f;
-
-  if (!hot) {
-    // LUT of 'unit' pair reconstructions c_r * (cos, sin)(2 pi c_th / 2^b_th)
-    const int bt = a.L.b_theta;
-    for (int i = tid; i < S::NLUT * 32; i += kThreads) {
-      const int w = i >> 5;
-      const int cr = w >> bt, ct = w & ((1 << bt) - 1);
-      float sn, cs;
-      sincospif(2.0f * (float)ct / (float)(1 << bt), &sn, &cs);
-      lut[i] = pack_h2((float)cr * cs, (float)cr * sn);
-    }
-    // B fragments: q' pairs (P/4)*tig + {2s, 2s+1}; q'' sign slots 2s, 2s+1
-    uint32_t qf[S::NT][2], qs[S::QS][2];
-    float kpol[2], kqjl[2];
-    if (gid < G) {
-      const uint32_t* qp = reinterpret_cast<const uint32_t*>(a.qrot + (size_t)(head0 + gid) * D) + (S::P / 4) * tig;
-      const uint32_t* qk = reinterpret_cast<const uint32_t*>(a.qsk + (size_t)(head0 + gid) * M) + tig * (M / 8);
-#pragma unroll
-      for (int s = 0; s < S::NT; ++s) { qf[s][0] = qp[2 * s]; qf[s][1] = qp[2 * s + 1]; }
-#pragma unroll
-      for (int s = 0; s < S::QS; ++s) { qs[s][0] = qk[2 * s]; qs[s][1] = qk[2 * s + 1]; }
-    } else {
-#pragma unroll
-      for (int s = 0; s < S::NT; ++s) qf[s][0] = qf[s][1] = 0u;
-#pragma unroll
-      for (int s = 0; s < S::QS; ++s) qs[s][0] = qs[s][1] = 0u;
-    }
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      const int g = 2 * tig + hh;
-      kpol[hh] = g < G ? a.log2e_sigma * a.qscale[2 * (head0 + g)] / (float)Lr : 0.f;
-      kqjl[hh] = g < G ? a.log2e_sigma * kSqrtHalfPi / (float)M * a.qscale[2 * (head0 + g) + 1] : 0.f;
-    }
-
-    const int64_t nblk = (a.n_cold + S::TB - 1) / S::TB;
-    const int64_t blk0 = (int64_t)split * a.blocks_per_split;
-    const int64_t blk1 = blk0 + a.blocks_per_split < nblk ? blk0 + a.blocks_per_split : nblk;
-    const uint8_t* ubase = a.cold + (size_t)unit * a.L.blocks_per_unit * S::BLOCK;
-    for (int64_t blk = blk0; blk < blk1; ++blk) {
-      __syncthreads();
-      const uint4* src = reinterpret_cast<const uint4*>(ubase + (size_t)blk * S::BLOCK);
-      uint4* dst = reinterpret_cast<uint4*>(stage);
-      for (int i = tid; i < S::BLOCK / 16; i += kThreads) dst[i] = __ldg(src + i);
-      __syncthreads();
-      const int nvalid = (int)((a.n_cold - blk * S::TB) < S::TB ? (a.n_cold - blk * S::TB) : S::TB);
-      if (tb >= nvalid) continue;
-
-      const int t0 = tb + gid, t1 = tb + gid + 8;
-      // ---- cold logits: polar part -------------------------------------
-      uint32_t k0[S::KW], k1[S::KW];
-      load_chunk<S::KW>(stage + S::OFF_KC + t0 * S::KC, tig * S::KBITS, k0);
-      load_chunk<S::KW>(stage + S::OFF_KC + t1 * S::KC, tig * S::KBITS, k1);
-      float cp[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int s = 0; s < S::NT; ++s) {
-        const uint32_t a0 = lut[(field<BW>(k0, (2 * s) * BW) << 5) + lane];
-        const uint32_t a1 = lut[(field<BW>(k1, (2 * s) * BW) << 5) + lane];
-        const uint32_t a2 = lut[(field<BW>(k0, (2 * s + 1) * BW) << 5) + lane];
-        const uint32_t a3 = lut[(field<BW>(k1, (2 * s + 1) * BW) << 5) + lane];
-        mma16816(cp, a0, a1, a2, a3, qf[s][0], qf[s][1]);
-      }
-      // ---- cold logits: QJL part ---------------------------------------
-      uint32_t x0, x1;
-      if constexpr (M == 128) {
-        x0 = *reinterpret_cast<const uint32_t*>(stage + S::OFF_KS + t0 * S::SG + 4 * tig);
-        x1 = *reinterpret_cast<const uint32_t*>(stage + S::OFF_KS + t1 * S::SG + 4 * tig);
-      } else {
-        const uint32_t c0 = *reinterpret_cast<const uint16_t*>(stage + S::OFF_KS + t0 * S::SG + 2 * tig);
-        const uint32_t c1 = *reinterpret_cast<const uint16_t*>(stage + S::OFF_KS + t1 * S::SG + 2 * tig);
-        x0 = ((c0 & 0xffu) << 8) | ((c0 >> 8) << 24);
-        x1 = ((c1 & 0xffu) << 8) | ((c1 >> 8) << 24);
-      }
-      float cq[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int s = 0; s < S::QS; ++s)
-        mma16816(cq, sign_pair(x0, 2 * s), sign_pair(x1, 2 * s), sign_pair(x0, 2 * s + 1),
-                 sign_pair(x1, 2 * s + 1), qs[s][0], qs[s][1]);
-
-      const __half* ksc = reinterpret_cast<const __half*>(stage + S::OFF_KSC);
-      const __half* krn = reinterpret_cast<const __half*>(stage + S::OFF_KRN);
-      const __half* vsc = reinterpret_cast<const __half*>(stage + S::OFF_VSC);
-      const bool v0 = t0 < nvalid, v1 = t1 < nvalid;
-      const float sk0 = __half2float(ksc[t0]), sk1 = __half2float(ksc[t1]);
-      const float rn0 = __half2float(krn[t0]), rn1 = __half2float(krn[t1]);
-      float l2[4];
-      l2[0] = v0 ? fmaf(rn0 * kqjl[0], cq[0], sk0 * kpol[0] * cp[0]) : kNegInf;
-      l2[1] = v0 ? fmaf(rn0 * kqjl[1], cq[1], sk0 * kpol[1] * cp[1]) : kNegInf;
-      l2[2] = v1 ? fmaf(rn1 * kqjl[0], cq[2], sk1 * kpol[0] * cp[2]) : kNegInf;
-      l2[3] = v1 ? fmaf(rn1 * kqjl[1], cq[3], sk1 * kpol[1] * cp[3]) : kNegInf;
-      float p[4], corr[2];
-      softmax_tile(l2, m_run, p, corr);
-      l_run[0] = l_run[0] * corr[0] + p[0] + p[2];
-      l_run[1] = l_run[1] * corr[1] + p[1] + p[3];
-
-      // ---- V weights p * s16_v, kept on their own running max -----------
-      const float lv0 = v0 ? log2f(__half2float(vsc[t0])) : kNegInf;
-      const float lv1 = v1 ? log2f(__half2float(vsc[t1])) : kNegInf;
-      float xv[4] = {l2[0] + lv0, l2[1] + lv0, l2[2] + lv1, l2[3] + lv1};
-      float pv[4], co[2];
-      softmax_tile(xv, mp_run, pv, co);
-#pragma unroll
-      for (int i = 0; i < S::NT; ++i) {
-        O[i][0] *= co[0]; O[i][1] *= co[1]; O[i][2] *= co[0]; O[i][3] *= co[1];
-      }
-      const uint32_t pb0 = movmatrix_trans(pack_h2(pv[0], pv[1]));
-      const uint32_t pb1 = movmatrix_trans(pack_h2(pv[2], pv[3]));
-
-      // ---- P V: V codes of pairs (P/8)*gid + i for tokens 2tig(+1)(+8) ---
-      uint32_t w0[S::VW], w1[S::VW], w2[S::VW], w3[S::VW];
-      const uint8_t* vc = stage + S::OFF_VC;
-      load_chunk<S::VW>(vc + (tb + 2 * tig) * S::KC, gid * S::VBITS, w0);
-      load_chunk<S::VW>(vc + (tb + 2 * tig + 1) * S::KC, gid * S::VBITS, w1);
-      load_chunk<S::VW>(vc + (tb + 2 * tig + 8) * S::KC, gid * S::VBITS, w2);
-      load_chunk<S::VW>(vc + (tb + 2 * tig + 9) * S::KC, gid * S::VBITS, w3);
-#pragma unroll
-      for (int i = 0; i < S::NT; ++i) {
-        const uint32_t L0 = lut[(field<BW>(w0, i * BW) << 5) + lane];
-        const uint32_t L1 = lut[(field<BW>(w1, i * BW) << 5) + lane];
-        const uint32_t L2 = lut[(field<BW>(w2, i * BW) << 5) + lane];
-        const uint32_t L3 = lut[(field<BW>(w3, i * BW) << 5) + lane];
-        mma16816(O[i], __byte_perm(L0, L1, 0x5410), __byte_perm(L0, L1, 0x7632),
-                 __byte_perm(L2, L3, 0x5410), __byte_perm(L2, L3, 0x7632), pb0, pb1);
-      }
-    }
-  } else {
-    // ---- hot tiles: fp16 K / V through padded shared memory --------------
-    uint32_t qh[S::NT][2];
-    if (gid < G) {
-      const __half* qp = a.q + (size_t)(head0 + gid) * D;
-#pragma unroll
-      for (int s = 0; s < S::NT; ++s) {
-        qh[s][0] = *reinterpret_cast<const uint32_t*>(qp + 16 * s + 2 * tig);
-        qh[s][1] = *reinterpret_cast<const uint32_t*>(qp + 16 * s + 8 + 2 * tig);
-      }
-    } else {
-#pragma unroll
-      for (int s = 0; s < S::NT; ++s) qh[s][0] = qh[s][1] = 0u;
-    }
-    const int ntiles = (a.n_hot + S::TB - 1) / S::TB;
-    const int hs = split - a.ns_cold;
-    const int tile0 = hs * a.tiles_per_split;
-    const int tile1 = tile0 + a.tiles_per_split < ntiles ? tile0 + a.tiles_per_split : ntiles;
-    constexpr int CH = D / 8;        // 16-byte chunks per token row
-    for (int tile = tile0; tile < tile1; ++tile) {
-      __syncthreads();
-      for (int i = tid; i < 2 * S::TB * CH; i += kThreads) {
-        const int kv = i / (S::TB * CH);
-        const int rem = i % (S::TB * CH);
-        const int r = rem / CH, c = rem % CH;
-        const int slot = tile * S::TB + r;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (slot < a.n_hot)
-          v = __ldg(reinterpret_cast<const uint4*>((kv ? a.hot_v : a.hot_k) + ((size_t)unit * a.W + slot) * D) + c);
-        *reinterpret_cast<uint4*>(stage + kv * S::TB * S::RS + r * S::RS + c * 16) = v;
-      }
-      __syncthreads();
-      const int nvalid = a.n_hot - tile * S::TB < S::TB ? a.n_hot - tile * S::TB : S::TB;
-      if (tb >= nvalid) continue;
-      const uint32_t kbase = smem_addr(stage);
-      const uint32_t vbase = kbase + S::TB * S::RS;
-      const int mi = lane >> 3, rr = lane & 7;
-      float c[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int s = 0; s < S::NT; ++s) {
-        uint32_t af[4];
-        ldsm_x4(af, kbase + (tb + rr + (mi & 1) * 8) * S::RS + (16 * s + (mi >> 1) * 8) * 2);
-        mma16816(c, af[0], af[1], af[2], af[3], qh[s][0], qh[s][1]);
-      }
-      const bool v0 = tb + gid < nvalid, v1 = tb + gid + 8 < nvalid;
-      float l2[4];
-      l2[0] = v0 ? a.log2e_sigma * c[0] : kNegInf;
-      l2[1] = v0 ? a.log2e_sigma * c[1] : kNegInf;
-      l2[2] = v1 ? a.log2e_sigma * c[2] : kNegInf;
-      l2[3] = v1 ? a.log2e_sigma * c[3] : kNegInf;
-      float p[4], corr[2];
-      softmax_tile(l2, m_run, p, corr);
-      l_run[0] = l_run[0] * corr[0] + p[0] + p[2];
-      l_run[1] = l_run[1] * corr[1] + p[1] + p[3];
-#pragma unroll
-      for (int i = 0; i < S::NT; ++i) {
-        O[i][0] *= corr[0]; O[i][1] *= corr[1]; O[i][2] *= corr[0]; O[i][3] *= corr[1];
-      }
-      const uint32_t pb0 = movmatrix_trans(pack_h2(p[0], p[1]));
-      const uint32_t pb1 = movmatrix_trans(pack_h2(p[2], p[3]));
-#pragma unroll
-      for (int i = 0; i < S::NT; ++i) {
-        uint32_t af[4];
-        ldsm_x4_trans(af, vbase + (tb + rr + (mi >> 1) * 8) * S::RS + (16 * i + (mi & 1) * 8) * 2);
-        mma16816(O[i], af[0], af[1], af[2], af[3], pb0, pb1);
-      }
-    }
-    mp_run[0] = m_run[0];
-    mp_run[1] = m_run[1];
-  }
-
-  // ---- finalize: per-warp state -> shared -> one partial per head -------
 #pragma unroll
   for (int o = 4; o < 32; o <<= 1) {
-    l_run[0] += __shfl_xor_sync(kFull, l_run[0], o);
-    l_run[1] += __shfl_xor_sync(kFull, l_run[1], o);
+    st.l_run[0] += __shfl_xor_sync(kFull, st.l_run[0], o);
+    st.l_run[1] += __shfl_xor_sync(kFull, st.l_run[1], o);
   }
-  float f[2];
-#pragma unroll
-  for (int hh = 0; hh < 2; ++hh) {
-    if (m_run[hh] == kNegInf) f[hh] = 0.f;
-    else if (hot) f[hh] = 1.f;
-    else f[hh] = exp2f(mp_run[hh] - m_run[hh]) / (float)Lr;
-  }
-  __syncthreads();
-  float* mw = reinterpret_cast<float*>(stage);     // [4 warps][8 heads]
-  float* lw = mw + 32;
-  float* ow = mw + 64;                              // [4][8][D]
+  float* mw = merge;          // [4 warps][8 heads]
+  float* lw = merge + 32;
+  float* ow = merge + 64;     // [8 heads][D]
   if (gid == 0) {
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
-      mw[warp * 8 + 2 * tig + hh] = m_run[hh];
-      lw[warp * 8 + 2 * tig + hh] = l_run[hh];
+      mw[warp * 8 + 2 * tig + hh] = st.m_run[hh];
+      lw[warp * 8 + 2 * tig + hh] = st.l_run[hh];
     }
   }
+  for (int i = tid; i < 8 * D; i += kThreads) ow[i] = 0.f;
+  __syncthreads();
+  float f[2];
 #pragma unroll
-  for (int i = 0; i < S::NT; ++i) {
+  for (int hh = 0; hh < 2; ++hh) {
+    const int g = 2 * tig + hh;
+    float mx = kNegInf;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) mx = fmaxf(mx, mw[w * 8 + g]);
+    if (st.m_run[hh] == kNegInf) f[hh] = 0.f;
+    else f[hh] = fast_exp2(st.m_run[hh] - mx) *
+                 (hot ? 1.f : fast_exp2(st.mp_run[hh] - st.m_run[hh]) / (float)Lr);
+  }
+  constexpr int P8 = D / 16;   // (D/2) / 8 pairs per gid for the cold mapping
+#pragma unroll
+  for (int i = 0; i < NT; ++i) {
 #pragma unroll
     for (int r2 = 0; r2 < 2; ++r2) {
-      const int dim = hot ? (16 * i + gid + 8 * r2) : (2 * ((S::P / 8) * gid + i) + r2);
+      const int dim = hot ? (16 * i + gid + 8 * r2) : (2 * (P8 * gid + i) + r2);
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         const int g = 2 * tig + hh;
-        ow[(warp * 8 + g) * D + dim] = O[i][2 * r2 + hh] * f[hh];
+        if (g < G && f[hh] != 0.f) atomicAdd(&ow[g * D + dim], st.O[i][2 * r2 + hh] * f[hh]);
       }
     }
   }
   __syncthreads();
   for (int idx = tid; idx < G * D; idx += kThreads) {
     const int g = idx / D, dim = idx % D;
-    float mx = kNegInf;
-#pragma unroll
-    for (int w = 0; w < 4; ++w) mx = fmaxf(mx, mw[w * 8 + g]);
-    float o = 0.f, l = 0.f;
-    if (mx != kNegInf) {
-#pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        const float mv = mw[w * 8 + g];
-        if (mv == kNegInf) continue;
-        const float sc = exp2f(mv - mx);
-        o += sc * ow[(w * 8 + g) * D + dim];
-        l += sc * lw[w * 8 + g];
-      }
-    }
-    float* pp = a.part + (((size_t)unit * a.max_splits + split) * G + g) * (D + 2);
-    pp[2 + dim] = o;
+    float* pp = dst + g * (D + 2);
+    pp[2 + dim] = ow[g * D + dim];
     if (dim == 0) {
+      float mx = kNegInf;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) mx = fmaxf(mx, mw[w * 8 + g]);
+      float l = 0.f;
+      if (mx != kNegInf) {
+#pragma unroll
+        for (int w = 0; w < 4; ++w)
+          if (mw[w * 8 + g] != kNegInf) l += fast_exp2(mw[w * 8 + g] - mx) * lw[w * 8 + g];
+      }
       pp[0] = mx;
       pp[1] = l;
+    }
+  }
+  __syncthreads();
+}
+
+// Lazy online softmax for one tile: the reference max moves (with a warp
+// reduction and a rescale of the sums) only when some logit exceeds it by
+// more than kLazyHeadroom, so p = exp2(l - ref) stays <= 2^8.  Returns the
+// rescale factor of the running sums (1 when nothing moved).
+__device__ __forceinline__ void lazy_softmax(const float (&l2)[4], float (&ref)[2], float (&p)[4],
+                                             float (&corr)[2]) {
+  const bool need = l2[0] > ref[0] + kLazyHeadroom || l2[1] > ref[1] + kLazyHeadroom ||
+                    l2[2] > ref[0] + kLazyHeadroom || l2[3] > ref[1] + kLazyHeadroom;
+  if (__any_sync(kFull, need)) {
+    softmax_tile(l2, ref, p, corr);
+  } else {
+    const float r0 = ref[0] == kNegInf ? 0.f : ref[0], r1 = ref[1] == kNegInf ? 0.f : ref[1];
+    p[0] = fast_exp2(l2[0] - r0);
+    p[1] = fast_exp2(l2[1] - r1);
+    p[2] = fast_exp2(l2[2] - r0);
+    p[3] = fast_exp2(l2[3] - r1);
+    corr[0] = corr[1] = 1.f;
+  }
+}
+
+template <int D, int M, int BW>
+__global__ void __launch_bounds__(kThreads, 3) attend_kernel(const AttendArgs a) {
+  using S = AttendShape<D, M, BW>;
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ __align__(16) uint2 klut_static[S::STATIC_LUT ? S::NLUT * 32 : 2];
+  __shared__ __align__(16) uint32_t vlut_static[S::STATIC_LUT ? S::NLUT * 32 : 4];
+  uint2* klut_w = S::STATIC_LUT ? klut_static : reinterpret_cast<uint2*>(smem);
+  uint32_t* vlut_w = S::STATIC_LUT ? vlut_static : reinterpret_cast<uint32_t*>(smem + S::OFF_VLUT);
+  const char* klut = reinterpret_cast<const char*>(klut_w);
+  const char* vlut = reinterpret_cast<const char*>(vlut_w);
+  uint8_t* ring = smem + S::OFF_RING;
+  float* merge = reinterpret_cast<float*>(smem + S::OFF_MERGE);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::OFF_BAR);
+  int* arrivals = reinterpret_cast<int*>(smem + S::OFF_BAR + 8 * S::NS);    // [NS] warps done
+  int* copies = arrivals + S::NS;                                           // [NS] copies issued
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(copies + S::NS);
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int gid = lane >> 2, tig = lane & 3;
+  const int G = a.G;
+  const int Lr = (1 << a.L.b_r) - 1;
+  const int tb = warp * 16;            // this warp's tokens inside a block / tile
+  const uint32_t lane8 = (uint32_t)lane * 8u, lane4 = (uint32_t)lane * 4u;
+  const SplitPlan& pl = a.plan;
+  const int slots = pl.slots_cold + pl.slots_hot;
+  WarpState<S::NT> st;
+  st.reset();
+
+  if ((int)blockIdx.x < pl.cold_ctas) {
+    // ======================= cold CTA =======================
+    const int c = blockIdx.x;
+    const int64_t nb = pl.cold_blocks;
+    const int64_t total = (int64_t)a.units * nb;
+    const int64_t f_lo = (int64_t)c * pl.cold_bpc;
+    const int64_t f_hi = f_lo + pl.cold_bpc < total ? f_lo + pl.cold_bpc : total;
+    const int nblk = (int)(f_hi - f_lo);
+    const uint32_t bar0 = smem_addr(bars);
+    const uint32_t ring0 = smem_addr(ring);
+    auto src_of = [&](int64_t f) {
+      const int64_t u = f / nb, blk = f % nb;
+      return a.cold + ((size_t)u * a.L.blocks_per_unit + (size_t)blk) * S::BLOCK;
+    };
+    if (tid < S::NS) {
+      arrivals[tid] = 0;
+      copies[tid] = tid < nblk ? 1 : 0;
+    }
+    if (tid == 0) {
+      *abort_flag = 0;
+      for (int s = 0; s < S::NS; ++s) mbar_init(bar0 + 8 * s, 1);
+      fence_barrier_init();
+      for (int s = 0; s < S::NS && s < nblk; ++s) {
+        mbar_expect_tx(bar0 + 8 * s, S::BLOCK);
+        bulk_g2s(ring0 + s * S::BLOCK, src_of(f_lo + s), S::BLOCK, bar0 + 8 * s);
+      }
+    }
+    // LUTs of 'unit' pair reconstructions c_r * (cos, sin)(2 pi c_th / 2^b_th):
+    // keys as fp16 hi + lo (the lo part removes the fp16 rounding of the
+    // table from the logits), values as fp16.
+    {
+      // 2^bw distinct entries (float64 sincospi once each), then one copy
+      // per lane; the merge area is free at this point.
+      const int bt = a.L.b_theta;
+      uint2* base = reinterpret_cast<uint2*>(merge);
+      for (int e = tid; e < S::NLUT; e += kThreads) {
+        const int cr = e >> bt, ct = e & ((1 << bt) - 1);
+        double sn, cs;
+        sincospi(2.0 * (double)ct / (double)(1 << bt), &sn, &cs);
+        const float x = (float)((double)cr * cs), y = (float)((double)cr * sn);
+        const __half hx = __float2half_rn(x), hy = __float2half_rn(y);
+        base[e] = make_uint2(pack_h2(__half2float(hx), __half2float(hy)),
+                               pack_h2(x - __half2float(hx), y - __half2float(hy)));
+      }
+      __syncthreads();
+      for (int i = tid; i < S::NLUT * 32; i += kThreads) {
+        const uint2 e = base[i >> 5];
+        klut_w[i] = e;
+        vlut_w[i] = e.x;
+      }
+    }
+    __syncthreads();
+
+    uint32_t qfh[S::NT][2], qfl[S::NT][2], qs[S::QS][2];
+    float kpol[2], kqjl[2];
+    int unit_cur = -1;
+    int slot_cur = 0;
+    bool aborted = false;
+    for (int i = 0; i < nblk; ++i) {
+      const int64_t f = f_lo + i;
+      const int unit = (int)(f / nb);
+      const int64_t blk = f % nb;
+      if (unit != unit_cur) {
+        if (unit_cur >= 0) {
+          flush_partial<D, S::NT>(st, false, Lr, G, merge,
+                                  a.part + (((size_t)unit_cur * slots + slot_cur) * G) * (D + 2));
+          st.reset();
+        }
+        unit_cur = unit;
+        slot_cur = c - (int)(((int64_t)unit * nb) / pl.cold_bpc);
+        const int b = unit / a.Hkv, kvh = unit % a.Hkv;
+        const int head0 = b * a.Hq + kvh * G;
+        if (gid < G) {
+          const uint32_t* qp = reinterpret_cast<const uint32_t*>(a.qrot + (size_t)(head0 + gid) * 2 * D) + S::PT * tig;
+          const uint32_t* qk = reinterpret_cast<const uint32_t*>(a.qsk + (size_t)(head0 + gid) * M) + tig * (M / 8);
+#pragma unroll
+          for (int s = 0; s < S::NT; ++s) {
+            qfh[s][0] = qp[2 * s];
+            qfh[s][1] = qp[2 * s + 1];
+            qfl[s][0] = qp[S::P + 2 * s];
+            qfl[s][1] = qp[S::P + 2 * s + 1];
+          }
+#pragma unroll
+          for (int s = 0; s < S::QS; ++s) { qs[s][0] = qk[2 * s]; qs[s][1] = qk[2 * s + 1]; }
+        } else {
+#pragma unroll
+          for (int s = 0; s < S::NT; ++s) qfh[s][0] = qfh[s][1] = qfl[s][0] = qfl[s][1] = 0u;
+#pragma unroll
+          for (int s = 0; s < S::QS; ++s) qs[s][0] = qs[s][1] = 0u;
+        }
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const int g = 2 * tig + hh;
+          kpol[hh] = g < G ? a.log2e_sigma * a.qscale[2 * (head0 + g)] / (float)Lr : 0.f;
+          kqjl[hh] = g < G ? a.log2e_sigma * kSqrtHalfPi / (float)M * a.qscale[2 * (head0 + g) + 1] : 0.f;
+        }
+      }
+      // ---- wait for this block's stage (every warp on its own) ----------
+      const int stage = i % S::NS;
+      if (!aborted && *abort_flag) aborted = true;
+      if (!aborted) {
+        const bool got = mbar_wait_bounded(bar0 + 8 * stage, (uint32_t)((i / S::NS) & 1));
+        if (!__all_sync(kFull, got)) {
+          aborted = true;
+          if (lane == 0) *abort_flag = 1;
+        }
+      }
+      const int64_t left = a.n_cold - blk * S::TB - tb;
+      if (!aborted && left > 0) {
+      const int nvalid = left < 16 ? (int)left : 16;     // valid tokens of this warp's tile
+      const uint8_t* tile = ring + stage * S::BLOCK + warp * S::TT;
+
+      uint32_t kw[S::KWT], sw[S::SW], vw[S::VWT];
+      load_lane_words<S::KWT>(tile + S::OFF_KC, lane, kw);
+      load_lane_words<S::SW>(tile + S::OFF_KS, lane, sw);
+      load_lane_words<S::VWT>(tile + S::OFF_VC, lane, vw);
+      const uint2 ksc = *reinterpret_cast<const uint2*>(tile + S::OFF_KSC + gid * 8);
+      const uint32_t vsc = *reinterpret_cast<const uint32_t*>(tile + S::OFF_VSC + gid * 4);
+
+      // ---- cold logits: polar part, (A_hi + A_lo) . (q'_hi + q'_lo) ------
+      // even / odd k-steps accumulate separately to halve the MMA chains
+      float cph[2][4] = {}, cpl[2][4] = {};
+#pragma unroll
+      for (int s = 0; s < S::NT; ++s) {
+        const uint2 a0 = *reinterpret_cast<const uint2*>(klut + (field_shifted<BW, 8>(kw, (2 * s) * BW) | lane8));
+        const uint2 a1 = *reinterpret_cast<const uint2*>(klut + (field_shifted<BW, 8>(kw, (S::PT + 2 * s) * BW) | lane8));
+        const uint2 a2 = *reinterpret_cast<const uint2*>(klut + (field_shifted<BW, 8>(kw, (2 * s + 1) * BW) | lane8));
+        const uint2 a3 = *reinterpret_cast<const uint2*>(klut + (field_shifted<BW, 8>(kw, (S::PT + 2 * s + 1) * BW) | lane8));
+        mma16816(cph[s & 1], a0.x, a1.x, a2.x, a3.x, qfh[s][0], qfh[s][1]);
+        mma16816(cpl[s & 1], a0.x, a1.x, a2.x, a3.x, qfl[s][0], qfl[s][1]);
+        mma16816(cpl[s & 1], a0.y, a1.y, a2.y, a3.y, qfh[s][0], qfh[s][1]);
+      }
+      // ---- cold logits: QJL part ---------------------------------------
+      uint32_t x0, x1;
+      if constexpr (M == 128) {
+        x0 = sw[0];
+        x1 = sw[S::SW - 1];
+      } else {
+        x0 = spread16(sw[0] & 0xffffu);
+        x1 = spread16(sw[0] >> 16);
+      }
+      float cq0[4] = {0.f, 0.f, 0.f, 0.f}, cq1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int s = 0; s < S::QS; s += 2) {
+        mma16816(cq0, sign_pair(x0, 2 * s), sign_pair(x1, 2 * s), sign_pair(x0, 2 * s + 1),
+                 sign_pair(x1, 2 * s + 1), qs[s][0], qs[s][1]);
+        mma16816(cq1, sign_pair(x0, 2 * s + 2), sign_pair(x1, 2 * s + 2), sign_pair(x0, 2 * s + 3),
+                 sign_pair(x1, 2 * s + 3), qs[s + 1][0], qs[s + 1][1]);
+      }
+
+      const bool v0 = gid < nvalid, v1 = gid + 8 < nvalid;
+      const float sk0 = __half2float(__ushort_as_half((unsigned short)(ksc.x & 0xffffu)));
+      const float sk1 = __half2float(__ushort_as_half((unsigned short)(ksc.x >> 16)));
+      const float rn0 = __half2float(__ushort_as_half((unsigned short)(ksc.y & 0xffffu)));
+      const float rn1 = __half2float(__ushort_as_half((unsigned short)(ksc.y >> 16)));
+      float l2[4];
+      float cp[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) cp[j] = (cph[0][j] + cph[1][j]) + (cpl[0][j] + cpl[1][j]);
+      l2[0] = v0 ? fmaf(rn0 * kqjl[0], cq0[0] + cq1[0], sk0 * kpol[0] * cp[0]) : kNegInf;
+      l2[1] = v0 ? fmaf(rn0 * kqjl[1], cq0[1] + cq1[1], sk0 * kpol[1] * cp[1]) : kNegInf;
+      l2[2] = v1 ? fmaf(rn1 * kqjl[0], cq0[2] + cq1[2], sk1 * kpol[0] * cp[2]) : kNegInf;
+      l2[3] = v1 ? fmaf(rn1 * kqjl[1], cq0[3] + cq1[3], sk1 * kpol[1] * cp[3]) : kNegInf;
+      float p[4], corr[2];
+      lazy_softmax(l2, st.m_run, p, corr);
+      st.l_run[0] = st.l_run[0] * corr[0] + p[0] + p[2];
+      st.l_run[1] = st.l_run[1] * corr[1] + p[1] + p[3];
+
+      // ---- V weights p * s16_v, on their own lazy reference ---------------
+      const float lv0 = v0 ? fast_log2(__half2float(__ushort_as_half((unsigned short)(vsc & 0xffffu)))) : kNegInf;
+      const float lv1 = v1 ? fast_log2(__half2float(__ushort_as_half((unsigned short)(vsc >> 16)))) : kNegInf;
+      const float xv[4] = {l2[0] + lv0, l2[1] + lv0, l2[2] + lv1, l2[3] + lv1};
+      float pv[4], co[2];
+      lazy_softmax(xv, st.mp_run, pv, co);
+      if (co[0] != 1.f || co[1] != 1.f) {
+#pragma unroll
+        for (int j = 0; j < S::NT; ++j) {
+          st.O[j][0] *= co[0]; st.O[j][1] *= co[1]; st.O[j][2] *= co[0]; st.O[j][3] *= co[1];
+        }
+      }
+      const uint32_t pb0 = movmatrix_trans(pack_h2(pv[0], pv[1]));
+      const uint32_t pb1 = movmatrix_trans(pack_h2(pv[2], pv[3]));
+
+      // ---- P V: V codes of pairs PV*gid + j for tokens 2tig, 2tig+1, +8, +9
+#pragma unroll
+      for (int j = 0; j < S::NT; ++j) {
+        const uint32_t L0 = *reinterpret_cast<const uint32_t*>(vlut + (field_shifted<BW, 7>(vw, (0 * S::PV + j) * BW) | lane4));
+        const uint32_t L1 = *reinterpret_cast<const uint32_t*>(vlut + (field_shifted<BW, 7>(vw, (1 * S::PV + j) * BW) | lane4));
+        const uint32_t L2 = *reinterpret_cast<const uint32_t*>(vlut + (field_shifted<BW, 7>(vw, (2 * S::PV + j) * BW) | lane4));
+        const uint32_t L3 = *reinterpret_cast<const uint32_t*>(vlut + (field_shifted<BW, 7>(vw, (3 * S::PV + j) * BW) | lane4));
+        mma16816(st.O[j], __byte_perm(L0, L1, 0x5410), __byte_perm(L0, L1, 0x7632),
+                 __byte_perm(L2, L3, 0x5410), __byte_perm(L2, L3, 0x7632), pb0, pb1);
+      }
+      }   // tile compute
+      // ---- release the stage; the last of the 4 warps refills it ----------
+      __syncwarp();
+      if (lane == 0) {
+        __threadfence_block();
+        const int old = atomicAdd(&arrivals[stage], 1);
+        if ((old & 3) == 3 && i + S::NS < nblk && !*abort_flag) {
+          __threadfence_block();
+          fence_proxy_async();
+          mbar_expect_tx(bar0 + 8 * stage, S::BLOCK);
+          bulk_g2s(ring0 + stage * S::BLOCK, src_of(f_lo + i + S::NS), S::BLOCK, bar0 + 8 * stage);
+          copies[stage] += 1;
+        }
+      }
+    }
+    __syncthreads();
+    if (*abort_flag) {
+      // A bulk copy did not complete in time: latch the error, give the
+      // copies still in flight a bounded chance to land, and leave.
+      if (tid == 0) {
+        atomicOr(a.status, kStatusTimeout);
+        for (int s = 0; s < S::NS; ++s)
+          if (copies[s] > 0) mbar_wait_bounded(bar0 + 8 * s, (uint32_t)((copies[s] - 1) & 1));
+      }
+      return;
+    }
+    if (unit_cur >= 0)
+      flush_partial<D, S::NT>(st, false, Lr, G, merge,
+                              a.part + (((size_t)unit_cur * slots + slot_cur) * G) * (D + 2));
+  } else {
+    // ======================= hot CTA =======================
+    const int c = blockIdx.x - pl.cold_ctas;
+    const int ht = pl.hot_tiles;
+    const int64_t total = (int64_t)a.units * ht;
+    const int64_t f_lo = (int64_t)c * pl.hot_tpc;
+    const int64_t f_hi = f_lo + pl.hot_tpc < total ? f_lo + pl.hot_tpc : total;
+    constexpr int CH = D / 8;        // 16-byte chunks per token row
+    uint32_t qh[S::NT][2];
+    int unit_cur = -1, slot_cur = 0;
+    for (int64_t f = f_lo; f < f_hi; ++f) {
+      const int unit = (int)(f / ht);
+      const int tile = (int)(f % ht);
+      if (unit != unit_cur) {
+        if (unit_cur >= 0) {
+          flush_partial<D, S::NT>(st, true, Lr, G, merge,
+                                  a.part + (((size_t)unit_cur * slots + slot_cur) * G) * (D + 2));
+          st.reset();
+        }
+        unit_cur = unit;
+        slot_cur = pl.slots_cold + (c - (int)(((int64_t)unit * ht) / pl.hot_tpc));
+        const int b = unit / a.Hkv, kvh = unit % a.Hkv;
+        const int head0 = b * a.Hq + kvh * G;
+        if (gid < G) {
+          const __half* qp = a.q + (size_t)(head0 + gid) * D;
+#pragma unroll
+          for (int s = 0; s < S::NT; ++s) {
+            qh[s][0] = *reinterpret_cast<const uint32_t*>(qp + 16 * s + 2 * tig);
+            qh[s][1] = *reinterpret_cast<const uint32_t*>(qp + 16 * s + 8 + 2 * tig);
+          }
+        } else {
+#pragma unroll
+          for (int s = 0; s < S::NT; ++s) qh[s][0] = qh[s][1] = 0u;
+        }
+      }
+      __syncthreads();
+      for (int i = tid; i < 2 * S::TB * CH; i += kThreads) {
+        const int kv = i / (S::TB * CH);
+        const int rem = i % (S::TB * CH);
+        const int r = rem / CH, cc = rem % CH;
+        const int slot = tile * S::TB + r;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (slot < a.n_hot)
+          v = __ldg(reinterpret_cast<const uint4*>((kv ? a.hot_v : a.hot_k) + ((size_t)unit * a.W + slot) * D) + cc);
+        *reinterpret_cast<uint4*>(ring + kv * S::TB * S::RS + r * S::RS + cc * 16) = v;
+      }
+      __syncthreads();
+      const int nvalid = a.n_hot - tile * S::TB < S::TB ? a.n_hot - tile * S::TB : S::TB;
+      if (tb >= nvalid) continue;
+      const uint32_t kbase = smem_addr(ring);
+      const uint32_t vbase = kbase + S::TB * S::RS;
+      const int mi = lane >> 3, rr = lane & 7;
+      float cc4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int s = 0; s < S::NT; ++s) {
+        uint32_t af[4];
+        ldsm_x4(af, kbase + (tb + rr + (mi & 1) * 8) * S::RS + (16 * s + (mi >> 1) * 8) * 2);
+        mma16816(cc4, af[0], af[1], af[2], af[3], qh[s][0], qh[s][1]);
+      }
+      const bool v0 = tb + gid < nvalid, v1 = tb + gid + 8 < nvalid;
+      float l2[4];
+      l2[0] = v0 ? a.log2e_sigma * cc4[0] : kNegInf;
+      l2[1] = v0 ? a.log2e_sigma * cc4[1] : kNegInf;
+      l2[2] = v1 ? a.log2e_sigma * cc4[2] : kNegInf;
+      l2[3] = v1 ? a.log2e_sigma * cc4[3] : kNegInf;
+      float p[4], corr[2];
+      softmax_tile(l2, st.m_run, p, corr);
+      st.l_run[0] = st.l_run[0] * corr[0] + p[0] + p[2];
+      st.l_run[1] = st.l_run[1] * corr[1] + p[1] + p[3];
+      if (__any_sync(kFull, corr[0] != 1.f || corr[1] != 1.f)) {
+#pragma unroll
+        for (int j = 0; j < S::NT; ++j) {
+          st.O[j][0] *= corr[0]; st.O[j][1] *= corr[1]; st.O[j][2] *= corr[0]; st.O[j][3] *= corr[1];
+        }
+      }
+      const uint32_t pb0 = movmatrix_trans(pack_h2(p[0], p[1]));
+      const uint32_t pb1 = movmatrix_trans(pack_h2(p[2], p[3]));
+#pragma unroll
+      for (int j = 0; j < S::NT; ++j) {
+        uint32_t af[4];
+        ldsm_x4_trans(af, vbase + (tb + rr + (mi >> 1) * 8) * S::RS + (16 * j + (mi & 1) * 8) * 2);
+        mma16816(st.O[j], af[0], af[1], af[2], af[3], pb0, pb1);
+      }
+    }
+    st.mp_run[0] = st.m_run[0];
+    st.mp_run[1] = st.m_run[1];
+    if (unit_cur >= 0) {
+      __syncthreads();
+      flush_partial<D, S::NT>(st, true, Lr, G, merge,
+                              a.part + (((size_t)unit_cur * slots + slot_cur) * G) * (D + 2));
     }
   }
 }
@@ -510,19 +827,31 @@ __global__ void combine_kernel(const CombineArgs a) {
   const int kvh = hq / a.G, g = hq % a.G;
   const int unit = b * a.Hkv + kvh;
   const int D = a.d, t = threadIdx.x;
-  const int ns = a.ns_cold + a.ns_hot;
-  const float* base = a.part + (size_t)unit * a.max_splits * a.G * (D + 2);
+  const SplitPlan& pl = a.plan;
+  const int slots = pl.slots_cold + pl.slots_hot;
+  const float* base = a.part + (size_t)unit * slots * a.G * (D + 2);
+  int nc = 0, nh = 0;
+  if (pl.cold_ctas > 0 && pl.cold_blocks > 0) {
+    const int64_t nb = pl.cold_blocks;
+    nc = (int)(((unit + 1) * nb - 1) / pl.cold_bpc - (unit * nb) / pl.cold_bpc + 1);
+  }
+  if (pl.hot_ctas > 0 && pl.hot_tiles > 0) {
+    const int64_t ht = pl.hot_tiles;
+    nh = (int)(((unit + 1) * ht - 1) / pl.hot_tpc - (unit * ht) / pl.hot_tpc + 1);
+  }
+  auto rec = [&](int s) { return base + ((size_t)s * a.G + g) * (D + 2); };
   float mx = kNegInf;
-  for (int s = 0; s < ns; ++s) mx = fmaxf(mx, base[((size_t)s * a.G + g) * (D + 2)]);
+  for (int s = 0; s < nc; ++s) mx = fmaxf(mx, rec(s)[0]);
+  for (int s = 0; s < nh; ++s) mx = fmaxf(mx, rec(pl.slots_cold + s)[0]);
   float lsum = 0.f, oc = 0.f, oh = 0.f;
   if (mx != kNegInf) {
-    for (int s = 0; s < ns; ++s) {
-      const float* pp = base + ((size_t)s * a.G + g) * (D + 2);
+    for (int s = 0; s < nc + nh; ++s) {
+      const float* pp = rec(s < nc ? s : pl.slots_cold + (s - nc));
       if (pp[0] == kNegInf) continue;
       const float w = exp2f(pp[0] - mx);
       lsum += w * pp[1];
       const float v = w * pp[2 + t];
-      if (s < a.ns_cold) oc += v; else oh += v;
+      if (s < nc) oc += v; else oh += v;
     }
   }
   buf[t] = oc;
@@ -585,7 +914,12 @@ int attend_ctas_per_sm(const Layout& L) {
 }
 
 cudaError_t launch_qprep(const QPrepArgs& a, cudaStream_t s) {
-  qprep_kernel<<<a.heads, 128, 0, s>>>(a);
+  const int grid = (a.heads + 7) / 8;
+  if (a.d == 64 && a.m == 64) qprep_kernel<64, 64><<<grid, 256, 0, s>>>(a);
+  else if (a.d == 64 && a.m == 128) qprep_kernel<64, 128><<<grid, 256, 0, s>>>(a);
+  else if (a.d == 128 && a.m == 64) qprep_kernel<128, 64><<<grid, 256, 0, s>>>(a);
+  else if (a.d == 128 && a.m == 128) qprep_kernel<128, 128><<<grid, 256, 0, s>>>(a);
+  else return cudaErrorInvalidValue;
   return cudaGetLastError();
 }
 
@@ -593,7 +927,8 @@ cudaError_t launch_attend(const AttendArgs& a, cudaStream_t s) {
   int smem = 0;
   AttendFn fn = pick_attend(a.L, &smem);
   if (!fn) return cudaErrorInvalidValue;
-  const int grid = a.units * (a.ns_cold + a.ns_hot);
+  const int grid = a.plan.cold_ctas + a.plan.hot_ctas;
+  if (grid == 0) return cudaSuccess;
   fn<<<grid, kThreads, smem, s>>>(a);
   return cudaGetLastError();
 }

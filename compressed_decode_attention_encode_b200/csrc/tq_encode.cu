@@ -51,159 +51,276 @@ __device__ __forceinline__ void load_vec(const __half* p, int lane, double (&x)[
   }
 }
 
-// One vector per warp.  D = padded length (power of two, >= 64).
+// Encodes one vector (K or V) held at `src` in float64; writes its code
+// words into `codes[0..D/2)` (shared memory, one byte per pair) and, for
+// keys, its sign words into `bits` (canonical order, bit i of word i/32)
+// and the raw fp16 scalars.  Whole warp; returns nothing else.
 template <int D>
-__global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
+__device__ __forceinline__ void encode_vector(const EncodeArgs& a, const __half* src, bool is_key,
+                                              double* rbuf, uint8_t* codes, uint32_t* bits,
+                                              uint16_t* s16_out, uint16_t* rn16_out) {
   constexpr int E = D / 32;      // elements per lane
   constexpr int PL = E / 2;      // pairs per lane
+  const int lane = threadIdx.x & 31;
+  const Layout& L = a.L;
+  const int Lr = (1 << L.b_r) - 1;
+  const int nt = 1 << L.b_theta;
+
+  // ---- rotation: y = H (D x) / sqrt(d) ----------------------------------
+  double x[E];
+  load_vec<E>(src, lane, x);
+#pragma unroll
+  for (int i = 0; i < E; ++i) x[i] = __dmul_rn(x[i], a.signs[lane * E + i]);
+#pragma unroll
+  for (int h = 1; h < D; h <<= 1) {
+    if (h < E) {
+#pragma unroll
+      for (int i = 0; i < E; ++i) {
+        if (!(i & h)) {
+          const double p = x[i], q = x[i + h];
+          x[i] = __dadd_rn(p, q);
+          x[i + h] = __dsub_rn(p, q);
+        }
+      }
+    } else {
+      const int lm = h / E;
+#pragma unroll
+      for (int i = 0; i < E; ++i) {
+        const double o = __shfl_xor_sync(kFull, x[i], lm);
+        x[i] = (lane & lm) ? __dsub_rn(o, x[i]) : __dadd_rn(x[i], o);
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < E; ++i) x[i] = __dmul_rn(x[i], a.inv_sqrt_d);
+
+  // ---- polar: rho, theta per pair; scale s16 = fp16(max rho) ------------
+  double rho[PL], th[PL];
+  double smax = 0.0;
+#pragma unroll
+  for (int k = 0; k < PL; ++k) {
+    const double y0 = x[2 * k], y1 = x[2 * k + 1];
+    rho[k] = __dsqrt_rn(__dadd_rn(__dmul_rn(y0, y0), __dmul_rn(y1, y1)));
+    th[k] = atan2(y1, y0);
+    smax = fmax(smax, rho[k]);
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) smax = fmax(smax, __shfl_xor_sync(kFull, smax, o));
+  uint16_t s16b = f64_to_f16_bits(smax);
+  if ((s16b & 0x7c00u) == 0x7c00u) {       // overflow: latch, store a zero record
+    if (lane == 0) atomicOr(a.status, kStatusRange);
+    s16b = 0;
+  }
+  const double s16 = f16_bits_to_f64(s16b);
+  const bool zero = (s16 == 0.0);
+
+  // ---- codes ---------------------------------------------------------------
+  int cr[PL], ct[PL];
+#pragma unroll
+  for (int k = 0; k < PL; ++k) {
+    const double tr = __dmul_rn(__ddiv_rn(rho[k], zero ? 1.0 : s16), (double)Lr);
+    const int c = (int)rint(tr);
+    cr[k] = c < 0 ? 0 : (c > Lr ? Lr : c);
+    const double tt = __ddiv_rn(__dmul_rn(th[k], (double)nt), kTwoPi);
+    ct[k] = ((int)rint(tt)) & (nt - 1);
+    if (zero) { cr[k] = 0; ct[k] = 0; }
+    codes[lane * PL + k] = (uint8_t)((cr[k] << L.b_theta) | ct[k]);
+  }
+  if (lane == 0) *s16_out = s16b;
+
+  // ---- residual and QJL sketch (keys) -------------------------------------
+  if (is_key) {
+    double r[E];
+    double ss = 0.0;
+#pragma unroll
+    for (int k = 0; k < PL; ++k) {
+      const double rh = __ddiv_rn(__dmul_rn((double)cr[k], s16), (double)Lr);
+      const double ang = __ddiv_rn(__dmul_rn((double)ct[k], kTwoPi), (double)nt);
+      double sn, cs;
+      sincos(ang, &sn, &cs);
+      r[2 * k] = __dsub_rn(x[2 * k], __dmul_rn(rh, cs));
+      r[2 * k + 1] = __dsub_rn(x[2 * k + 1], __dmul_rn(rh, sn));
+      ss = __dadd_rn(ss, __dadd_rn(__dmul_rn(r[2 * k], r[2 * k]), __dmul_rn(r[2 * k + 1], r[2 * k + 1])));
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) ss = __dadd_rn(ss, __shfl_xor_sync(kFull, ss, o));
+    const uint16_t rnb = f64_to_f16_bits(__dsqrt_rn(ss));
+    if ((rnb & 0x7c00u) == 0x7c00u && lane == 0) atomicOr(a.status, kStatusRange);
+    if (lane == 0) *rn16_out = rnb;
+#pragma unroll
+    for (int i = 0; i < E; ++i) rbuf[lane * E + i] = r[i];
+    __syncwarp();
+    const int m = L.m;
+    for (int k = 0; k < (m + 31) / 32; ++k) {
+      const int i = lane + 32 * k;
+      double acc = 0.0;
+      if (i < m) {
+        const float* col = a.St + i;
+#pragma unroll 8
+        for (int jj = 0; jj < D; ++jj) acc = fma((double)__ldg(col + (size_t)jj * m), rbuf[jj], acc);
+      }
+      const unsigned word = __ballot_sync(kFull, i < m && acc >= 0.0);
+      if (lane == 0) bits[k] = word;
+    }
+  }
+  __syncwarp();
+}
+
+// Merges `val` into the 32-bit word at `addr` under `mask` (bits of tokens
+// written by this launch); bits of other tokens are kept.
+__device__ __forceinline__ void merge_word(uint32_t* addr, uint32_t val, uint32_t mask) {
+  if (mask == 0u) return;
+  if (mask != 0xffffffffu) val = (*addr & ~mask) | (val & mask);
+  *addr = val;
+}
+
+// Bits of word w of a lane chunk whose codes are laid out at code index q
+// (bit q*bw); `code_of(q, &c)` returns false for codes of tokens that this
+// launch does not write.
+template <typename F>
+__device__ __forceinline__ void chunk_word(int w, int ncodes, int bw, F code_of, uint32_t& val,
+                                           uint32_t& mask) {
+  val = 0u;
+  mask = 0u;
+  const uint32_t cm = (1u << bw) - 1u;
+  int q0 = (32 * w) / bw - 1;
+  if (q0 < 0) q0 = 0;
+  for (int q = q0; q < ncodes && q * bw < 32 * (w + 1); ++q) {
+    const int bit = q * bw - 32 * w;
+    if (bit + bw <= 0) continue;
+    uint32_t c;
+    if (!code_of(q, &c)) continue;
+    if (bit >= 0) {
+      val |= c << bit;
+      mask |= cm << bit;
+    } else {
+      val |= c >> (-bit);
+      mask |= cm >> (-bit);
+    }
+  }
+}
+
+// One warp per group of 4 tokens {2c, 2c+1, 2c+8, 2c+9} of a 16-token tile:
+// exactly the tokens whose fragment-major words can share a 32-bit word, so
+// no two warps ever write the same word.  D = padded length (power of two).
+template <int D>
+__global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
+  constexpr int P = D / 2;
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int warps = blockDim.x >> 5;
   extern __shared__ double smem[];
-  double* rbuf = smem + warp * D;                                        // residual
-  uint8_t* cbuf = reinterpret_cast<uint8_t*>(smem + warps * D) + warp * (D / 2);  // code words
+  double* rbuf = smem + warp * D;
+  uint8_t* wbase = reinterpret_cast<uint8_t*>(smem + warps * D) + warp * (8 * P + 4 * 32 + 32);
+  uint8_t* kc = wbase;                       // [4][P] key code words
+  uint8_t* vc = wbase + 4 * P;               // [4][P] value code words
+  uint32_t* kb = reinterpret_cast<uint32_t*>(wbase + 8 * P);   // [4][8] sign words
+  uint16_t* sc = reinterpret_cast<uint16_t*>(wbase + 8 * P + 128);  // [4][4] s16_k, rn16, s16_v
 
   const Layout& L = a.L;
-  const int Lr = (1 << L.b_r) - 1;
-  const int nt = 1 << L.b_theta;
   const int bw = L.bw;
-  const int m = L.m;
-  const int64_t per_unit = (int64_t)a.nA + a.nB;
-  const int64_t per_kind = (int64_t)a.units * per_unit;
-  const int64_t jobs = 2 * per_kind;
+  const int64_t n = (int64_t)a.nA + a.nB;
+  if (n == 0) return;
+  const int64_t t_first = a.cold_start / kTokensPerTile;
+  const int64_t t_last = (a.cold_start + n - 1) / kTokensPerTile;
+  const int64_t groups = (t_last - t_first + 1) * 4;
+  const int64_t jobs = (int64_t)a.units * groups;
 
   for (int64_t job = (int64_t)blockIdx.x * warps + warp; job < jobs;
        job += (int64_t)gridDim.x * warps) {
-    const bool is_key = job < per_kind;
-    const int64_t j = is_key ? job : job - per_kind;
-    const int unit = (int)(j / per_unit);
-    const int64_t e = j % per_unit;
-    const __half* src;
-    if (e < a.nA) {
-      const int slot = (int)((a.ring_start + e) % a.W);
-      src = (is_key ? a.ring_k : a.ring_v) + ((int64_t)unit * a.W + slot) * D;
-    } else {
-      src = (is_key ? a.src_k : a.src_v) + ((int64_t)unit * a.src_tokens + (e - a.nA)) * D;
+    const int unit = (int)(job / groups);
+    const int64_t g = job % groups;
+    const int64_t tile = t_first + g / 4;
+    const int c = (int)(g % 4);
+    bool inr[4];
+    int64_t seq[4];
+    bool any = false;
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      const int r = 2 * c + (s & 1) + 8 * (s >> 1);
+      const int64_t t = tile * kTokensPerTile + r;
+      seq[s] = t - a.cold_start;
+      inr[s] = seq[s] >= 0 && seq[s] < n;
+      any |= inr[s];
     }
-
-    // ---- rotation: y = H (D x) / sqrt(d) --------------------------------
-    double x[E];
-    load_vec<E>(src, lane, x);
-#pragma unroll
-    for (int i = 0; i < E; ++i) x[i] = __dmul_rn(x[i], a.signs[lane * E + i]);
-#pragma unroll
-    for (int h = 1; h < D; h <<= 1) {
-      if (h < E) {
-#pragma unroll
-        for (int i = 0; i < E; ++i) {
-          if (!(i & h)) {
-            const double p = x[i], q = x[i + h];
-            x[i] = __dadd_rn(p, q);
-            x[i + h] = __dsub_rn(p, q);
-          }
-        }
+    if (!any) continue;
+    for (int s = 0; s < 4; ++s) {
+      if (!inr[s]) continue;
+      const int64_t e = seq[s];
+      const __half* ksrc;
+      const __half* vsrc;
+      if (e < a.nA) {
+        const int slot = (int)((a.ring_start + e) % a.W);
+        ksrc = a.ring_k + ((int64_t)unit * a.W + slot) * D;
+        vsrc = a.ring_v + ((int64_t)unit * a.W + slot) * D;
       } else {
-        const int lm = h / E;
-#pragma unroll
-        for (int i = 0; i < E; ++i) {
-          const double o = __shfl_xor_sync(kFull, x[i], lm);
-          x[i] = (lane & lm) ? __dsub_rn(o, x[i]) : __dadd_rn(x[i], o);
-        }
+        ksrc = a.src_k + ((int64_t)unit * a.src_tokens + (e - a.nA)) * D;
+        vsrc = a.src_v + ((int64_t)unit * a.src_tokens + (e - a.nA)) * D;
       }
+      encode_vector<D>(a, ksrc, true, rbuf, kc + s * P, kb + s * 8, sc + s * 4, sc + s * 4 + 1);
+      encode_vector<D>(a, vsrc, false, rbuf, vc + s * P, nullptr, sc + s * 4 + 2, nullptr);
     }
-#pragma unroll
-    for (int i = 0; i < E; ++i) x[i] = __dmul_rn(x[i], a.inv_sqrt_d);
-
-    // ---- polar: rho, theta per pair; scale s16 = fp16(max rho) ----------
-    double rho[PL], th[PL];
-    double smax = 0.0;
-#pragma unroll
-    for (int k = 0; k < PL; ++k) {
-      const double y0 = x[2 * k], y1 = x[2 * k + 1];
-      rho[k] = __dsqrt_rn(__dadd_rn(__dmul_rn(y0, y0), __dmul_rn(y1, y1)));
-      th[k] = atan2(y1, y0);
-      smax = fmax(smax, rho[k]);
-    }
-#pragma unroll
-    for (int o = 16; o; o >>= 1) smax = fmax(smax, __shfl_xor_sync(kFull, smax, o));
-    uint16_t s16b = f64_to_f16_bits(smax);
-    if ((s16b & 0x7c00u) == 0x7c00u) {       // overflow: latch, store a zero record
-      if (lane == 0) atomicOr(a.status, kStatusRange);
-      s16b = 0;
-    }
-    const double s16 = f16_bits_to_f64(s16b);
-    const bool zero = (s16 == 0.0);
-
-    // ---- codes ---------------------------------------------------------
-    int cr[PL], ct[PL];
-#pragma unroll
-    for (int k = 0; k < PL; ++k) {
-      const double tr = __dmul_rn(__ddiv_rn(rho[k], zero ? 1.0 : s16), (double)Lr);
-      int c = (int)rint(tr);
-      cr[k] = c < 0 ? 0 : (c > Lr ? Lr : c);
-      const double tt = __ddiv_rn(__dmul_rn(th[k], (double)nt), kTwoPi);
-      ct[k] = ((int)rint(tt)) & (nt - 1);
-      if (zero) { cr[k] = 0; ct[k] = 0; }
-      cbuf[lane * PL + k] = (uint8_t)((cr[k] << L.b_theta) | ct[k]);
-    }
-
-    const int64_t t = a.cold_start + e;
-    uint8_t* blk = a.cold + ((int64_t)unit * L.blocks_per_unit + t / kTokensPerBlock) * L.block_bytes;
-    const int row = (int)(t % kTokensPerBlock);
-    uint8_t* rec_codes = blk + (is_key ? L.off_kc : L.off_vc) + row * L.kc_bytes;
-    uint16_t* rec_scale = reinterpret_cast<uint16_t*>(blk + (is_key ? L.off_ksc : L.off_vsc)) + row;
-
-    // ---- residual and QJL sketch (keys) ---------------------------------
-    if (is_key) {
-      double r[E];
-      double ss = 0.0;
-#pragma unroll
-      for (int k = 0; k < PL; ++k) {
-        const double rh = __ddiv_rn(__dmul_rn((double)cr[k], s16), (double)Lr);
-        const double ang = __ddiv_rn(__dmul_rn((double)ct[k], kTwoPi), (double)nt);
-        double sn, cs;
-        sincos(ang, &sn, &cs);
-        r[2 * k] = __dsub_rn(x[2 * k], __dmul_rn(rh, cs));
-        r[2 * k + 1] = __dsub_rn(x[2 * k + 1], __dmul_rn(rh, sn));
-        ss = __dadd_rn(ss, __dadd_rn(__dmul_rn(r[2 * k], r[2 * k]), __dmul_rn(r[2 * k + 1], r[2 * k + 1])));
-      }
-#pragma unroll
-      for (int o = 16; o; o >>= 1) ss = __dadd_rn(ss, __shfl_xor_sync(kFull, ss, o));
-      uint16_t rnb = f64_to_f16_bits(__dsqrt_rn(ss));
-      if ((rnb & 0x7c00u) == 0x7c00u && lane == 0) atomicOr(a.status, kStatusRange);
-#pragma unroll
-      for (int i = 0; i < E; ++i) rbuf[lane * E + i] = r[i];
-      __syncwarp();
-      uint8_t* rec_bits = blk + L.off_ks + row * L.sg_bytes;
-      for (int k = 0; k < (m + 31) / 32; ++k) {
-        const int i = lane + 32 * k;
-        double acc = 0.0;
-        if (i < m) {
-          const float* col = a.St + i;
-#pragma unroll 8
-          for (int jj = 0; jj < D; ++jj) acc = fma((double)__ldg(col + (size_t)jj * m), rbuf[jj], acc);
-        }
-        const unsigned word = __ballot_sync(kFull, i < m && acc >= 0.0);
-        if (lane < 4 && 4 * k + lane < L.sg_bytes) rec_bits[4 * k + lane] = (uint8_t)(word >> (8 * lane));
-      }
-      if (lane == 0) reinterpret_cast<uint16_t*>(blk + L.off_krn)[row] = rnb;
-    }
-
-    // ---- pack code words LSB-first into the record ---------------------
     __syncwarp();
-    const int nwords = L.kc_bytes / 4;
-    for (int w = lane; w < nwords; w += 32) {
-      const int bit0 = 32 * w;
-      uint32_t word = 0;
-      const int j0 = bit0 / bw, j1 = (bit0 + 31) / bw;
-      for (int jj = j0; jj <= j1 && jj < D / 2; ++jj) {
-        const int pos = jj * bw - bit0;
-        const uint32_t c = cbuf[jj];
-        word |= pos >= 0 ? (c << pos) : (c >> (-pos));
-      }
-      reinterpret_cast<uint32_t*>(rec_codes)[w] = word;
+
+    uint8_t* tb = a.cold + ((int64_t)unit * L.blocks_per_unit + tile / kTilesPerBlock) * L.block_bytes +
+                  (tile % kTilesPerBlock) * L.tile_bytes;
+    // K code words: lanes (gid = 2c + e, tig), codes q: half h = q / pt, pair tig*pt + q % pt
+    for (int q = lane; q < 8 * L.kwt; q += 32) {
+      const int ch = q / L.kwt, w = q % L.kwt;
+      const int e = ch / 4, tig = ch % 4;
+      const int l = 4 * (2 * c + e) + tig;
+      uint32_t val, mask;
+      chunk_word(w, 2 * L.pt, bw, [&](int qi, uint32_t* out) {
+        const int h = qi / L.pt, k = qi % L.pt, s = e + 2 * h;
+        if (!inr[s]) return false;
+        *out = kc[s * P + tig * L.pt + k];
+        return true;
+      }, val, mask);
+      merge_word(reinterpret_cast<uint32_t*>(tb + L.off_kc + lane_word_offset(w, l, L.kwt)), val, mask);
     }
-    if (lane == 0) *rec_scale = s16b;
+    // V code words: lanes (gid_v, tig = c), codes q: slot q / pv, pair gid_v*pv + q % pv
+    for (int q = lane; q < 8 * L.vwt; q += 32) {
+      const int gv = q / L.vwt, w = q % L.vwt;
+      const int l = 4 * gv + c;
+      uint32_t val, mask;
+      chunk_word(w, 4 * L.pv, bw, [&](int qi, uint32_t* out) {
+        const int s = qi / L.pv, k = qi % L.pv;
+        if (!inr[s]) return false;
+        *out = vc[s * P + gv * L.pv + k];
+        return true;
+      }, val, mask);
+      merge_word(reinterpret_cast<uint32_t*>(tb + L.off_vc + lane_word_offset(w, l, L.vwt)), val, mask);
+    }
+    // sign words: lanes (gid = 2c + e, tig); m/4 bits per (token, tig)
+    const int qb = L.m / 4;
+    for (int q = lane; q < 8 * L.sw; q += 32) {
+      const int ch = q / L.sw, w = q % L.sw;
+      const int e = ch / 4, tig = ch % 4;
+      const int l = 4 * (2 * c + e) + tig;
+      uint32_t val = 0u, mask = 0u;
+      for (int h = 0; h < 2; ++h) {
+        const int s = e + 2 * h;
+        const int bit0 = h * qb - 32 * w;        // chunk bit of this token's first sign
+        if (!inr[s] || bit0 >= 32 || bit0 + qb <= 0) continue;
+        // qb is 16 or 32: the token's bits lie in one word
+        const int i0 = tig * qb;                 // first canonical sign index
+        const uint32_t src = kb[s * 8 + (i0 >> 5)] >> (i0 & 31);
+        const uint32_t m32 = qb == 32 ? 0xffffffffu : ((1u << qb) - 1u);
+        val |= (src & m32) << bit0;
+        mask |= m32 << bit0;
+      }
+      merge_word(reinterpret_cast<uint32_t*>(tb + L.off_ks + lane_word_offset(w, l, L.sw)), val, mask);
+    }
+    // scalars
+    if (lane < 4 && inr[lane]) {
+      const int s = lane;
+      const int e = s & 1, h = s >> 1, gid = 2 * c + e;
+      uint16_t* ks = reinterpret_cast<uint16_t*>(tb + L.off_ksc);
+      uint16_t* vs = reinterpret_cast<uint16_t*>(tb + L.off_vsc);
+      ks[gid * 4 + h] = sc[s * 4];
+      ks[gid * 4 + 2 + h] = sc[s * 4 + 1];
+      vs[gid * 2 + h] = sc[s * 4 + 2];
+    }
     __syncwarp();
   }
 }
@@ -232,14 +349,16 @@ __global__ void ring_write_kernel(__half* ring_k, __half* ring_v, const __half* 
 template <int D>
 cudaError_t launch_encode_d(const EncodeArgs& a, cudaStream_t s) {
   const int warps = 8;
-  const int64_t jobs = 2 * (int64_t)a.units * ((int64_t)a.nA + a.nB);
-  if (jobs == 0) return cudaSuccess;
+  const int64_t n = (int64_t)a.nA + a.nB;
+  if (n == 0) return cudaSuccess;
+  const int64_t tiles = (a.cold_start + n - 1) / kTokensPerTile - a.cold_start / kTokensPerTile + 1;
+  const int64_t jobs = (int64_t)a.units * tiles * 4;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t want = (jobs + warps - 1) / warps;
   const int grid = (int)(want < (int64_t)sms * 16 ? want : (int64_t)sms * 16);
-  const size_t smem = (size_t)warps * D * sizeof(double) + (size_t)warps * (D / 2);
+  const size_t smem = (size_t)warps * D * sizeof(double) + (size_t)warps * (8 * (D / 2) + 4 * 32 + 32);
   encode_kernel<D><<<grid, warps * 32, smem, s>>>(a);
   return cudaGetLastError();
 }

@@ -15,7 +15,8 @@ namespace tq {
 
 namespace {
 
-constexpr int kMaxSplits = 64;     // split partials kept per (row, kv head)
+constexpr int kSlotsCold = 96;     // partial slots per (row, kv head) for cold CTAs
+constexpr int kSlotsHot = 32;      // ... and for hot CTAs
 constexpr size_t kAlign = 256;
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -56,28 +57,6 @@ bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 
 }  // namespace
 
-Layout make_layout(int d, int b_r, int b_theta, int m, int64_t capacity) {
-  Layout L{};
-  L.d = d;
-  L.pairs = d / 2;
-  L.b_r = b_r;
-  L.b_theta = b_theta;
-  L.bw = b_r + b_theta;
-  L.m = m;
-  L.kc_bytes = L.pairs * L.bw / 8;
-  L.sg_bytes = m / 8;
-  const int TB = kTokensPerBlock;
-  L.off_kc = 0;
-  L.off_ks = L.off_kc + TB * L.kc_bytes;
-  L.off_ksc = L.off_ks + TB * L.sg_bytes;
-  L.off_krn = L.off_ksc + TB * 2;
-  L.off_vc = L.off_krn + TB * 2;
-  L.off_vsc = L.off_vc + TB * L.kc_bytes;
-  L.block_bytes = L.off_vsc + TB * 2;
-  L.blocks_per_unit = (capacity + TB - 1) / TB;
-  return L;
-}
-
 struct WsLayout {
   size_t status, signs, S, St, qrot, qsk, qscale, part, total;
 };
@@ -92,10 +71,10 @@ static WsLayout ws_layout(const tq_config& c) {
   w.signs = off;  off += round_up(sizeof(double) * c.head_dim, kAlign);
   w.S = off;      off += round_up(sizeof(float) * c.head_dim * c.qjl_bits, kAlign);
   w.St = off;     off += round_up(sizeof(float) * c.head_dim * c.qjl_bits, kAlign);
-  w.qrot = off;   off += round_up(2 * heads * c.head_dim, kAlign);
+  w.qrot = off;   off += round_up(2 * 2 * heads * c.head_dim, kAlign);
   w.qsk = off;    off += round_up(2 * heads * c.qjl_bits, kAlign);
   w.qscale = off; off += round_up(sizeof(float) * 2 * heads, kAlign);
-  w.part = off;   off += round_up(sizeof(float) * units * kMaxSplits * G * (c.head_dim + 2), kAlign);
+  w.part = off;   off += round_up(sizeof(float) * units * (kSlotsCold + kSlotsHot) * G * (c.head_dim + 2), kAlign);
   w.total = off;
   return w;
 }
@@ -164,7 +143,7 @@ tq_status tq_cache_bytes(const tq_config* cfg, size_t* hot_bytes, size_t* cold_b
                          size_t* workspace_bytes) {
   tq_status st = check_config(cfg);
   if (st != TQ_OK) return st;
-  const Layout L = make_layout(cfg->head_dim, cfg->b_r, cfg->b_theta, cfg->qjl_bits,
+  const Layout L = layout_of(cfg->head_dim, cfg->b_r, cfg->b_theta, cfg->qjl_bits,
                                cfg->cold_capacity);
   const size_t units = (size_t)cfg->batch * cfg->num_kv_heads;
   if (hot_bytes) *hot_bytes = 2 * units * cfg->hot_window * cfg->head_dim * 2;
@@ -184,7 +163,7 @@ tq_status tq_cache_create(const tq_config* cfg, void* hot_mem, void* cold_mem,
   tq_cache* c = new (std::nothrow) tq_cache();
   if (!c) return TQ_ERR_INVALID_ARG;
   c->cfg = *cfg;
-  c->L = make_layout(cfg->head_dim, cfg->b_r, cfg->b_theta, cfg->qjl_bits, cfg->cold_capacity);
+  c->L = layout_of(cfg->head_dim, cfg->b_r, cfg->b_theta, cfg->qjl_bits, cfg->cold_capacity);
   c->W = ws_layout(*cfg);
   c->hot = (uint8_t*)hot_mem;
   c->cold = (uint8_t*)cold_mem;
@@ -308,35 +287,36 @@ tq_status tq_decode_attention(tq_cache* c, const void* q, float* out, float soft
   const float sigma = softmax_scale == 0.0f ? (float)(1.0 / std::sqrt((double)d)) : softmax_scale;
   const int TB = kTokensPerBlock;
 
-  // Split plan: fill the device with about one wave of CTAs; hot tiles and
-  // cold blocks get CTAs in proportion to their bytes.
+  // Split plan: one wave of CTAs.  Hot tiles and cold blocks get CTAs in
+  // proportion to their bytes; each CTA takes an equal run of the flattened
+  // (unit, block) list, so every SM streams about the same number of bytes.
   const int64_t cold_blocks = (c->n_cold + TB - 1) / TB;
   const int hot_tiles = (c->n_hot + TB - 1) / TB;
+  const int64_t N = (int64_t)units * cold_blocks;
+  const int64_t Nh = (int64_t)units * hot_tiles;
   const int slots = c->num_sms * c->ctas_per_sm;
-  const int target = std::max(1, std::min(kMaxSplits, slots / std::max(1, units)));
-  const double cold_b = (double)cold_blocks * c->L.block_bytes;
-  const double hot_b = (double)hot_tiles * TB * d * 4.0;
-  // Every non-empty region gets at least one split; together at most
-  // kMaxSplits (the partial slots reserved per unit).
-  int ns_hot = 0, ns_cold = 0;
-  if (hot_tiles > 0) {
-    ns_hot = std::max(1, (int)std::lround(target * hot_b / (hot_b + cold_b)));
-    ns_hot = std::min(ns_hot, hot_tiles);
-    if (cold_blocks > 0) ns_hot = std::min(ns_hot, kMaxSplits - 1);
+  const double cold_b = (double)N * c->L.block_bytes;
+  const double hot_b = (double)Nh * TB * d * 4.0;
+  SplitPlan pl{};
+  pl.cold_blocks = cold_blocks;
+  pl.hot_tiles = hot_tiles;
+  pl.slots_cold = kSlotsCold;
+  pl.slots_hot = kSlotsHot;
+  if (Nh > 0) {
+    int ch = (int)std::lround(slots * hot_b / (hot_b + cold_b));
+    ch = (int)std::max<int64_t>(1, std::min<int64_t>(ch, Nh));
+    int64_t tpc = (Nh + ch - 1) / ch;
+    // a unit's tiles may span at most kSlotsHot CTAs
+    tpc = std::max<int64_t>(tpc, hot_tiles > 1 ? (hot_tiles - 1 + kSlotsHot - 3) / (kSlotsHot - 2) : 1);
+    pl.hot_tpc = (int)tpc;
+    pl.hot_ctas = (int)((Nh + tpc - 1) / tpc);
   }
-  if (cold_blocks > 0) {
-    ns_cold = std::max(1, target - ns_hot);
-    ns_cold = (int)std::min<int64_t>(ns_cold, cold_blocks);
-    ns_cold = std::min(ns_cold, kMaxSplits - ns_hot);
-  }
-  int blocks_per_split = 1, tiles_per_split = 1;
-  if (ns_cold > 0) {
-    blocks_per_split = (int)((cold_blocks + ns_cold - 1) / ns_cold);
-    ns_cold = (int)((cold_blocks + blocks_per_split - 1) / blocks_per_split);
-  }
-  if (ns_hot > 0) {
-    tiles_per_split = (hot_tiles + ns_hot - 1) / ns_hot;
-    ns_hot = (hot_tiles + tiles_per_split - 1) / tiles_per_split;
+  if (N > 0) {
+    const int cc = std::max(1, slots - pl.hot_ctas);
+    int64_t bpc = (N + cc - 1) / cc;
+    bpc = std::max<int64_t>(bpc, cold_blocks > 1 ? (cold_blocks - 1 + kSlotsCold - 3) / (kSlotsCold - 2) : 1);
+    pl.cold_bpc = bpc;
+    pl.cold_ctas = (int)((N + bpc - 1) / bpc);
   }
 
   __half* qrot = (__half*)(c->ws + c->W.qrot);
@@ -344,7 +324,7 @@ tq_status tq_decode_attention(tq_cache* c, const void* q, float* out, float soft
   float* qscale = (float*)(c->ws + c->W.qscale);
   float* part = (float*)(c->ws + c->W.part);
 
-  if (ns_cold > 0) {
+  if (pl.cold_ctas > 0) {
     QPrepArgs qa{};
     qa.q = (const __half*)q;
     qa.signs = c->signs();
@@ -357,7 +337,7 @@ tq_status tq_decode_attention(tq_cache* c, const void* q, float* out, float soft
     qa.m = m;
     if (launch_qprep(qa, stream) != cudaSuccess) return TQ_ERR_CUDA;
   }
-  if (ns_cold + ns_hot > 0) {
+  if (pl.cold_ctas + pl.hot_ctas > 0) {
     AttendArgs a{};
     a.q = (const __half*)q;
     a.qrot = qrot;
@@ -376,11 +356,7 @@ tq_status tq_decode_attention(tq_cache* c, const void* q, float* out, float soft
     a.W = cf.hot_window;
     a.n_hot = c->n_hot;
     a.n_cold = c->n_cold;
-    a.ns_cold = ns_cold;
-    a.ns_hot = ns_hot;
-    a.blocks_per_split = blocks_per_split;
-    a.tiles_per_split = tiles_per_split;
-    a.max_splits = kMaxSplits;
+    a.plan = pl;
     a.log2e_sigma = (float)(1.4426950408889634 * (double)sigma);
     if (c->ev_start && cudaEventRecord(c->ev_start, stream) != cudaSuccess) return TQ_ERR_CUDA;
     if (launch_attend(a, stream) != cudaSuccess) return TQ_ERR_CUDA;
@@ -395,9 +371,7 @@ tq_status tq_decode_attention(tq_cache* c, const void* q, float* out, float soft
   ca.Hkv = cf.num_kv_heads;
   ca.Hq = cf.num_q_heads;
   ca.d = d;
-  ca.ns_cold = ns_cold;
-  ca.ns_hot = ns_hot;
-  ca.max_splits = kMaxSplits;
+  ca.plan = pl;
   ca.batch = cf.batch;
   if (launch_combine(ca, stream) != cudaSuccess) return TQ_ERR_CUDA;
   return TQ_OK;
@@ -438,16 +412,61 @@ tq_status tq_export_cold(tq_cache* c, int32_t row, int32_t kv_head, int64_t star
   const uint8_t* src = c->cold + ((size_t)unit * L.blocks_per_unit + b0) * L.block_bytes;
   if (cudaMemcpy(buf.data(), src, buf.size(), cudaMemcpyDeviceToHost) != cudaSuccess)
     return TQ_ERR_CUDA;
+  const int bw = L.bw;
+  auto word_at = [&](const uint8_t* plane, int w, int lane, int nw) {
+    uint32_t v;
+    std::memcpy(&v, plane + lane_word_offset(w, lane, nw), 4);
+    return v;
+  };
+  // bit `bit` of a lane chunk stream of nw words
+  auto chunk_bits = [&](const uint8_t* plane, int lane, int nw, int bit, int width) {
+    const int w = bit >> 5, sh = bit & 31;
+    uint64_t v = word_at(plane, w, lane, nw);
+    if (sh + width > 32 && w + 1 < nw) v |= (uint64_t)word_at(plane, w + 1, lane, nw) << 32;
+    return (uint32_t)((v >> sh) & ((1ull << width) - 1));
+  };
+  auto put_bits = [](uint8_t* out, int bit, uint32_t val, int width) {
+    for (int b = 0; b < width; ++b)
+      if ((val >> b) & 1u) out[(bit + b) >> 3] |= (uint8_t)(1u << ((bit + b) & 7));
+  };
   for (int64_t i = 0; i < count; ++i) {
     const int64_t t = start + i;
     const uint8_t* blk = buf.data() + (size_t)(t / TB - b0) * L.block_bytes;
-    const int r = (int)(t % TB);
-    if (k_codes) std::memcpy(k_codes + i * L.kc_bytes, blk + L.off_kc + r * L.kc_bytes, L.kc_bytes);
-    if (k_bits) std::memcpy(k_bits + i * L.sg_bytes, blk + L.off_ks + r * L.sg_bytes, L.sg_bytes);
-    if (k_s16) std::memcpy(k_s16 + i, blk + L.off_ksc + 2 * r, 2);
-    if (k_rn16) std::memcpy(k_rn16 + i, blk + L.off_krn + 2 * r, 2);
-    if (v_codes) std::memcpy(v_codes + i * L.kc_bytes, blk + L.off_vc + r * L.kc_bytes, L.kc_bytes);
-    if (v_s16) std::memcpy(v_s16 + i, blk + L.off_vsc + 2 * r, 2);
+    const int tok = (int)(t % TB);
+    const uint8_t* tile = blk + (tok / kTokensPerTile) * L.tile_bytes;
+    const int r = tok % kTokensPerTile;
+    const int gid = r % 8, h = r / 8;
+    if (k_codes) {
+      uint8_t* out = k_codes + i * L.kc_bytes;
+      std::memset(out, 0, L.kc_bytes);
+      for (int p = 0; p < L.pairs; ++p) {
+        const int tig = p / L.pt, k = p % L.pt;
+        put_bits(out, p * bw, chunk_bits(tile + L.off_kc, 4 * gid + tig, L.kwt, (h * L.pt + k) * bw, bw), bw);
+      }
+    }
+    if (v_codes) {
+      uint8_t* out = v_codes + i * L.kc_bytes;
+      std::memset(out, 0, L.kc_bytes);
+      const int tig = (r % 8) / 2, slot = (r % 2) + 2 * h;
+      for (int p = 0; p < L.pairs; ++p) {
+        const int gv = p / L.pv, k = p % L.pv;
+        put_bits(out, p * bw, chunk_bits(tile + L.off_vc, 4 * gv + tig, L.vwt, (slot * L.pv + k) * bw, bw), bw);
+      }
+    }
+    if (k_bits) {
+      uint8_t* out = k_bits + i * L.sg_bytes;
+      std::memset(out, 0, L.sg_bytes);
+      const int qb = L.m / 4;
+      for (int tig = 0; tig < 4; ++tig) {
+        const uint32_t v = chunk_bits(tile + L.off_ks, 4 * gid + tig, L.sw, h * qb, qb == 32 ? 32 : qb);
+        put_bits(out, tig * qb, qb == 32 ? v : (v & ((1u << qb) - 1)), qb);
+      }
+    }
+    const uint16_t* ks = reinterpret_cast<const uint16_t*>(tile + L.off_ksc);
+    const uint16_t* vs = reinterpret_cast<const uint16_t*>(tile + L.off_vsc);
+    if (k_s16) k_s16[i] = ks[gid * 4 + h];
+    if (k_rn16) k_rn16[i] = ks[gid * 4 + 2 + h];
+    if (v_s16) v_s16[i] = vs[gid * 2 + h];
   }
   return TQ_OK;
 }

@@ -11,30 +11,81 @@
 
 namespace tq {
 
-// Tokens per cold block.  A block holds field planes, each token-major:
-//   K codes [TB][kc_bytes] | K signs [TB][sg_bytes] | K s16 [TB] | K rn16 [TB]
-//   | V codes [TB][kc_bytes] | V s16 [TB]
-// With TB = 64 every plane starts on a 16-byte boundary.
+// Tokens per cold block (one bulk copy) and per tile (one warp's MMA rows).
 constexpr int kTokensPerBlock = 64;
+constexpr int kTokensPerTile = 16;
+constexpr int kTilesPerBlock = kTokensPerBlock / kTokensPerTile;
 
 // Device status word bits (latched, cleared by tq_get_status).
 constexpr int kStatusRange = 1;
 constexpr int kStatusTimeout = 2;
 
+// Cold-store layout.  Per (row, kv head): 64-token blocks of 4 tiles.  A
+// tile (16 tokens) is laid out fragment-major for the decode warp that
+// reads it: lane l = 4*gid + tig owns
+//   K codes : tokens gid and gid+8, pairs [tig*PT, tig*PT + PT), PT = d/8
+//             (code k of token half h at bit (h*PT + k)*bw of the lane chunk)
+//   K signs : tokens gid and gid+8, sign bits [tig*m/4, (tig+1)*m/4)
+//             (m = 128: word h = token half h; m = 64: bits 16h.. of word 0)
+//   V codes : tokens 2tig, 2tig+1, 2tig+8, 2tig+9 (slot 0..3), pairs
+//             [gid*PV, gid*PV + PV), PV = d/16 (code k of slot s at bit
+//             (s*PV + k)*bw)
+// Per-lane word streams are stored "2-word-major": words 2g, 2g+1 of every
+// lane sit together (8 bytes per lane) so a warp reads them with one
+// conflict-free 64-bit load.  Per-token scalars are grouped by gid:
+//   K scalars [gid][s16(gid), s16(gid+8), rn16(gid), rn16(gid+8)]
+//   V scalars [gid][s16(gid), s16(gid+8)]
+// Planes inside a tile: K codes | K signs | K scalars (64 B) | V codes |
+// V scalars (32 B); every plane size is a multiple of 16 bytes.
 struct Layout {
   int d;            // head_dim (power of two)
   int pairs;        // d / 2
   int b_r, b_theta, bw;
   int m;            // QJL bits
-  int kc_bytes;     // packed code bytes per vector: pairs * bw / 8
+  int kc_bytes;     // canonical packed code bytes per vector: pairs * bw / 8
   int sg_bytes;     // m / 8
-  // plane offsets inside a block
-  int off_kc, off_ks, off_ksc, off_krn, off_vc, off_vsc;
+  int pt, pv;       // pairs per lane in the K / V fragments
+  int kwt, sw, vwt; // 32-bit words per lane: K codes, K signs, V codes
+  int off_kc, off_ks, off_ksc, off_vc, off_vsc;   // plane offsets inside a tile
+  int tile_bytes;
   int block_bytes;
-  int64_t blocks_per_unit;  // ceil(cold_capacity / TB)
+  int64_t blocks_per_unit;  // ceil(cold_capacity / 64)
 };
 
-Layout make_layout(int d, int b_r, int b_theta, int m, int64_t capacity);
+__host__ __device__ inline int words_for_bits(int bits) { return (bits + 31) / 32; }
+
+// Byte offset of word w (of nw) of lane l in a 2-word-major plane.
+__host__ __device__ inline int lane_word_offset(int w, int l, int nw) {
+  const int width = ((w | 1) < nw) ? 8 : 4;
+  return (w >> 1) * 256 + l * width + (w & 1) * 4;
+}
+
+__host__ __device__ inline Layout layout_of(int d, int b_r, int b_theta, int m, int64_t capacity) {
+  Layout L{};
+  L.d = d;
+  L.pairs = d / 2;
+  L.b_r = b_r;
+  L.b_theta = b_theta;
+  L.bw = b_r + b_theta;
+  L.m = m;
+  L.kc_bytes = L.pairs * L.bw / 8;
+  L.sg_bytes = m / 8;
+  L.pt = L.pairs / 4;
+  L.pv = L.pairs / 8;
+  L.kwt = words_for_bits(2 * L.pt * L.bw);
+  L.sw = words_for_bits(2 * (m / 4));
+  L.vwt = words_for_bits(4 * L.pv * L.bw);
+  L.off_kc = 0;
+  L.off_ks = L.off_kc + 128 * L.kwt;
+  L.off_ksc = L.off_ks + 128 * L.sw;
+  L.off_vc = L.off_ksc + 64;
+  L.off_vsc = L.off_vc + 128 * L.vwt;
+  L.tile_bytes = L.off_vsc + 32;
+  L.block_bytes = kTilesPerBlock * L.tile_bytes;
+  L.blocks_per_unit = (capacity + kTokensPerBlock - 1) / kTokensPerBlock;
+  return L;
+}
+
 
 // ---- encode -------------------------------------------------------------
 // Encodes a sequence of E vectors per unit (unit = row * Hkv + kv head), K
@@ -73,35 +124,47 @@ struct QPrepArgs {
   const __half* q;          // [B*Hq, d]
   const double* signs;      // [d]
   const float* St;          // [d, m]
-  __half* qrot;             // [B*Hq, d]   q' * alpha'
-  __half* qsk;              // [B*Hq, m]   q'' * alpha'' in sign-fragment order
-  float* qscale;            // [B*Hq, 2]   1/alpha', 1/alpha''
+  __half* qrot;             // [B*Hq, 2, d]  q' * alpha' as fp16 hi and lo parts
+  __half* qsk;              // [B*Hq, m]     q'' * alpha'' in sign-fragment order
+  float* qscale;            // [B*Hq, 2]     1/alpha', 1/alpha''
   int heads;                // B*Hq
   int d, m;
 };
 
 cudaError_t launch_qprep(const QPrepArgs& a, cudaStream_t s);
 
-struct Partial;  // per (unit, split, head): m (log2 units), l, o[d]
+// Work partition of one decode call.  The cold blocks of all units form one
+// flattened list (unit-major); cold CTA c takes blocks [c*cold_bpc,
+// (c+1)*cold_bpc) of it and writes one partial per unit it touches, into
+// slot c - first_cta(unit).  Hot tiles are split the same way by hot CTAs,
+// whose partials follow the cold slots.
+struct SplitPlan {
+  int64_t cold_blocks;      // 64-token blocks holding valid cold tokens, per unit
+  int cold_ctas;
+  int64_t cold_bpc;         // blocks per cold CTA
+  int hot_tiles;            // 64-token hot tiles per unit
+  int hot_ctas;
+  int hot_tpc;              // tiles per hot CTA
+  int slots_cold;           // partial slots per unit reserved for cold CTAs
+  int slots_hot;
+};
 
+// Partial record per (unit, slot, head): {m (log2 units), l, o[d]}.
 struct AttendArgs {
   const __half* q;          // [B*Hq, d]  (hot logits use q itself)
-  const __half* qrot;       // q' fragments source
-  const __half* qsk;        // q'' fragments source
-  const float* qscale;
+  const __half* qrot;       // [B*Hq, 2, d]
+  const __half* qsk;        // [B*Hq, m]
+  const float* qscale;      // [B*Hq, 2]
   const __half* hot_k;      // [units, W, d]
   const __half* hot_v;
   const uint8_t* cold;
-  float* part;              // [units, max_splits, G, d + 2]
+  float* part;              // [units, slots_cold + slots_hot, G, d + 2]
   int* status;
   Layout L;
+  SplitPlan plan;
   int units, G, Hq, Hkv;
   int W, n_hot;
   int64_t n_cold;
-  int ns_cold, ns_hot;      // splits per unit
-  int blocks_per_split;     // cold blocks per cold split
-  int tiles_per_split;      // 64-token hot tiles per hot split
-  int max_splits;
   float log2e_sigma;        // log2(e) * softmax scale
 };
 
@@ -112,8 +175,8 @@ struct CombineArgs {
   const float* part;
   const double* signs;
   float* out;               // [B*Hq, d]
+  SplitPlan plan;
   int units, G, Hkv, Hq, d, batch;
-  int ns_cold, ns_hot, max_splits;
 };
 
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s);

@@ -108,3 +108,20 @@ def test_null_arguments_rejected_before_device(lib):
     assert lib.tq_get_status(None, None) == 1
     assert lib.tq_cache_destroy(None) == 0
     assert lib.tq_rotation_signs(0, 0, None) == 1
+
+
+@pytest.mark.parametrize("d,m", [(64, 64), (64, 128), (128, 64), (128, 128)])
+@pytest.mark.parametrize("b_r,b_t", [(1, 1), (2, 2), (3, 3), (2, 3), (4, 4), (1, 7), (5, 3)])
+def test_cold_store_holds_exactly_the_algorithmic_bytes(lib, d, m, b_r, b_t):
+    """The fragment-major tile layout adds no padding: a 64-token block is
+    64 x (2 * d/2*bw/8 + m/8 + 6) bytes, except that d = 64 with an odd bit
+    width rounds each lane's 16*bw-bit chunk up to whole words."""
+    bw = b_r + b_t
+    cfg = _cfg(batch=1, num_q_heads=4, num_kv_heads=1, head_dim=d, qjl_bits=m, b_r=b_r,
+               b_theta=b_t, cold_capacity=64)
+    _, cold, _ = tq.tq_cache_bytes(cfg)
+    per_token = 2 * (d // 2 * bw // 8) + m // 8 + 6
+    if d == 64 and bw % 2:
+        words = -(-16 * bw // 32)
+        per_token = 2 * (words * 4 * 32 // 16) + m // 8 + 6
+    assert cold == 64 * per_token
