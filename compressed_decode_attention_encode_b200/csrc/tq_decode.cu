@@ -511,9 +511,11 @@ __global__ void __launch_bounds__(kThreads, 3) attend_kernel(const AttendArgs a)
     const int nblk = (int)(f_hi - f_lo);
     const uint32_t bar0 = smem_addr(bars);
     const uint32_t ring0 = smem_addr(ring);
+    // f -> (unit, block) by division: used only for the NS initial copies;
+    // the loop and the refills advance (unit, blk) incrementally
     auto src_of = [&](int64_t f) {
-      const int64_t u = f / nb, blk = f % nb;
-      return a.cold + ((size_t)u * a.L.blocks_per_unit + (size_t)blk) * S::BLOCK;
+      const int64_t u = f / nb, b = f % nb;
+      return a.cold + ((size_t)u * a.L.blocks_per_unit + (size_t)b) * S::BLOCK;
     };
     if (tid < S::NS) {
       arrivals[tid] = 0;
@@ -559,10 +561,13 @@ __global__ void __launch_bounds__(kThreads, 3) attend_kernel(const AttendArgs a)
     int unit_cur = -1;
     int slot_cur = 0;
     bool aborted = false;
-    for (int i = 0; i < nblk; ++i) {
-      const int64_t f = f_lo + i;
-      const int unit = (int)(f / nb);
-      const int64_t blk = f % nb;
+    int unit = (int)(f_lo / nb);          // advanced incrementally: no division per block
+    int64_t blk = f_lo - (int64_t)unit * nb;
+    for (int i = 0; i < nblk; ++i, ++blk) {
+      if (blk == nb) {
+        blk = 0;
+        ++unit;
+      }
       if (unit != unit_cur) {
         if (unit_cur >= 0) {
           flush_partial<D, S::NT>(st, false, Lr, G, merge,
@@ -704,7 +709,12 @@ __global__ void __launch_bounds__(kThreads, 3) attend_kernel(const AttendArgs a)
           __threadfence_block();
           fence_proxy_async();
           mbar_expect_tx(bar0 + 8 * stage, S::BLOCK);
-          bulk_g2s(ring0 + stage * S::BLOCK, src_of(f_lo + i + S::NS), S::BLOCK, bar0 + 8 * stage);
+          int64_t pb = blk + S::NS;          // block i + NS: at most NS past (unit, blk)
+          int pu = unit;
+          while (pb >= nb) { pb -= nb; ++pu; }
+          bulk_g2s(ring0 + stage * S::BLOCK,
+                   a.cold + ((size_t)pu * a.L.blocks_per_unit + (size_t)pb) * S::BLOCK, S::BLOCK,
+                   bar0 + 8 * stage);
           copies[stage] += 1;
         }
       }
@@ -733,9 +743,13 @@ __global__ void __launch_bounds__(kThreads, 3) attend_kernel(const AttendArgs a)
     constexpr int CH = D / 8;        // 16-byte chunks per token row
     uint32_t qh[S::NT][2];
     int unit_cur = -1, slot_cur = 0;
-    for (int64_t f = f_lo; f < f_hi; ++f) {
-      const int unit = (int)(f / ht);
-      const int tile = (int)(f % ht);
+    int unit = (int)(f_lo / ht);
+    int tile = (int)(f_lo - (int64_t)unit * ht);
+    for (int64_t f = f_lo; f < f_hi; ++f, ++tile) {
+      if (tile == ht) {
+        tile = 0;
+        ++unit;
+      }
       if (unit != unit_cur) {
         if (unit_cur >= 0) {
           flush_partial<D, S::NT>(st, true, Lr, G, merge,

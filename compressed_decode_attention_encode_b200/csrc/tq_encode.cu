@@ -55,22 +55,26 @@ __device__ __forceinline__ void load_vec(const __half* p, int lane, double (&x)[
 // words into `codes[0..D/2)` (shared memory, one byte per pair) and, for
 // keys, its sign words into `bits` (canonical order, bit i of word i/32)
 // and the raw fp16 scalars.  Whole warp; returns nothing else.
-template <int D>
-__device__ __forceinline__ void encode_vector(const EncodeArgs& a, const __half* src, bool is_key,
-                                              double* rbuf, uint8_t* codes, uint32_t* bits,
-                                              uint16_t* s16_out, uint16_t* rn16_out) {
+// `load(lane, x)` fills the lane's D/32 consecutive input elements (padded
+// coordinates read as 0).  `L` supplies b_r, b_theta and m; `St` is S^T
+// [D, m]; `signs` the rotation diagonal.
+template <int D, typename Loader>
+__device__ __forceinline__ void encode_vector_any(const Layout& L, const double* signs,
+                                                  const float* St, double inv_sqrt_d, int* status,
+                                                  Loader load, bool is_key, double* rbuf,
+                                                  uint8_t* codes, uint32_t* bits,
+                                                  uint16_t* s16_out, uint16_t* rn16_out) {
   constexpr int E = D / 32;      // elements per lane
   constexpr int PL = E / 2;      // pairs per lane
   const int lane = threadIdx.x & 31;
-  const Layout& L = a.L;
   const int Lr = (1 << L.b_r) - 1;
   const int nt = 1 << L.b_theta;
 
   // ---- rotation: y = H (D x) / sqrt(d) ----------------------------------
   double x[E];
-  load_vec<E>(src, lane, x);
+  load(lane, x);
 #pragma unroll
-  for (int i = 0; i < E; ++i) x[i] = __dmul_rn(x[i], a.signs[lane * E + i]);
+  for (int i = 0; i < E; ++i) x[i] = __dmul_rn(x[i], signs[lane * E + i]);
 #pragma unroll
   for (int h = 1; h < D; h <<= 1) {
     if (h < E) {
@@ -92,7 +96,7 @@ __device__ __forceinline__ void encode_vector(const EncodeArgs& a, const __half*
     }
   }
 #pragma unroll
-  for (int i = 0; i < E; ++i) x[i] = __dmul_rn(x[i], a.inv_sqrt_d);
+  for (int i = 0; i < E; ++i) x[i] = __dmul_rn(x[i], inv_sqrt_d);
 
   // ---- polar: rho, theta per pair; scale s16 = fp16(max rho) ------------
   double rho[PL], th[PL];
@@ -108,7 +112,7 @@ __device__ __forceinline__ void encode_vector(const EncodeArgs& a, const __half*
   for (int o = 16; o; o >>= 1) smax = fmax(smax, __shfl_xor_sync(kFull, smax, o));
   uint16_t s16b = f64_to_f16_bits(smax);
   if ((s16b & 0x7c00u) == 0x7c00u) {       // overflow: latch, store a zero record
-    if (lane == 0) atomicOr(a.status, kStatusRange);
+    if (lane == 0) atomicOr(status, kStatusRange);
     s16b = 0;
   }
   const double s16 = f16_bits_to_f64(s16b);
@@ -145,7 +149,7 @@ __device__ __forceinline__ void encode_vector(const EncodeArgs& a, const __half*
 #pragma unroll
     for (int o = 16; o; o >>= 1) ss = __dadd_rn(ss, __shfl_xor_sync(kFull, ss, o));
     const uint16_t rnb = f64_to_f16_bits(__dsqrt_rn(ss));
-    if ((rnb & 0x7c00u) == 0x7c00u && lane == 0) atomicOr(a.status, kStatusRange);
+    if ((rnb & 0x7c00u) == 0x7c00u && lane == 0) atomicOr(status, kStatusRange);
     if (lane == 0) *rn16_out = rnb;
 #pragma unroll
     for (int i = 0; i < E; ++i) rbuf[lane * E + i] = r[i];
@@ -155,7 +159,7 @@ __device__ __forceinline__ void encode_vector(const EncodeArgs& a, const __half*
       const int i = lane + 32 * k;
       double acc = 0.0;
       if (i < m) {
-        const float* col = a.St + i;
+        const float* col = St + i;
 #pragma unroll 8
         for (int jj = 0; jj < D; ++jj) acc = fma((double)__ldg(col + (size_t)jj * m), rbuf[jj], acc);
       }
@@ -164,6 +168,15 @@ __device__ __forceinline__ void encode_vector(const EncodeArgs& a, const __half*
     }
   }
   __syncwarp();
+}
+
+template <int D>
+__device__ __forceinline__ void encode_vector(const EncodeArgs& a, const __half* src, bool is_key,
+                                              double* rbuf, uint8_t* codes, uint32_t* bits,
+                                              uint16_t* s16_out, uint16_t* rn16_out) {
+  encode_vector_any<D>(a.L, a.signs, a.St, a.inv_sqrt_d, a.status,
+                       [&](int lane, double (&x)[D / 32]) { load_vec<D / 32>(src, lane, x); },
+                       is_key, rbuf, codes, bits, s16_out, rn16_out);
 }
 
 // Merges `val` into the 32-bit word at `addr` under `mask` (bits of tokens
