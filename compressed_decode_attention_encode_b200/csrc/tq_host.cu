@@ -6,6 +6,7 @@
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <vector>
 
@@ -381,6 +382,152 @@ tq_status tq_set_attend_events(tq_cache* c, cudaEvent_t start, cudaEvent_t stop)
   if (!c || (start == nullptr) != (stop == nullptr)) return TQ_ERR_INVALID_ARG;
   c->ev_start = start;
   c->ev_stop = stop;
+  return TQ_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Decode attention with library-owned static scratch.
+//
+// Some callers may not allocate device memory while they run: code inside
+// an allocator-free serving loop, a plugin whose host framework owns every
+// allocation, or a process whose memory is fully reserved up front.  For
+// them tq_decode_attention_static keeps the per-call scratch (the rotated
+// queries and the split partials) in one fixed device array compiled into
+// this library instead of the handle's workspace.  The array exists once
+// per GPU that loads the library and stays resident until the process
+// exits.  Calls that overlap on the GPU share it and race; nothing in it has
+// to start at zero, because every call writes what it reads.
+// ---------------------------------------------------------------------------
+static constexpr size_t kStaticScratchBytes = (size_t)4 << 20;   // 4 MiB
+static __device__ __align__(256) unsigned char tq_static_scratch[kStaticScratchBytes];
+
+static constexpr int kMaxScratchDevices = 64;
+static std::mutex g_static_scratch_mu;
+static void* g_static_scratch_ptr[kMaxScratchDevices] = {};
+
+// Device address of tq_static_scratch on `device`, which must be current.
+// The name is only a host-side stand-in: the address is fetched once per
+// device with cudaGetSymbolAddress and remembered.
+static void* static_scratch_address(int device) {
+  if (device < 0 || device >= kMaxScratchDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_static_scratch_mu);
+  if (!g_static_scratch_ptr[device]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, tq_static_scratch) != cudaSuccess || !p) return nullptr;
+    g_static_scratch_ptr[device] = p;
+  }
+  return g_static_scratch_ptr[device];
+}
+
+tq_status tq_decode_attention_static(tq_cache* c, const void* q, float* out, float softmax_scale,
+                                     cudaStream_t stream) {
+  if (!c || !q || !out || !(softmax_scale >= 0.0f) || std::isinf(softmax_scale))
+    return TQ_ERR_INVALID_ARG;
+  int current = -1;
+  if (cudaGetDevice(&current) != cudaSuccess) return TQ_ERR_CUDA;
+  if (current != c->device) return TQ_ERR_INVALID_ARG;   // the handle's GPU must be current
+  const tq_config& cf = c->cfg;
+  const int d = cf.head_dim, m = cf.qjl_bits;
+  const int heads = cf.batch * cf.num_q_heads;
+  const int units = cf.batch * cf.num_kv_heads;
+  const int G = cf.num_q_heads / cf.num_kv_heads;
+  const float sigma = softmax_scale == 0.0f ? (float)(1.0 / std::sqrt((double)d)) : softmax_scale;
+  const int TB = kTokensPerBlock;
+
+  // The same split plan as tq_decode_attention, with the partial slots per
+  // unit cut to the most any unit can receive under this plan.
+  const int64_t cold_blocks = (c->n_cold + TB - 1) / TB;
+  const int hot_tiles = (c->n_hot + TB - 1) / TB;
+  const int64_t N = (int64_t)units * cold_blocks;
+  const int64_t Nh = (int64_t)units * hot_tiles;
+  const int slots = c->num_sms * c->ctas_per_sm;
+  const double cold_b = (double)N * c->L.block_bytes;
+  const double hot_b = (double)Nh * TB * d * 4.0;
+  SplitPlan pl{};
+  pl.cold_blocks = cold_blocks;
+  pl.hot_tiles = hot_tiles;
+  if (Nh > 0) {
+    int ch = (int)std::lround(slots * hot_b / (hot_b + cold_b));
+    ch = (int)std::max<int64_t>(1, std::min<int64_t>(ch, Nh));
+    int64_t tpc = (Nh + ch - 1) / ch;
+    tpc = std::max<int64_t>(tpc, hot_tiles > 1 ? (hot_tiles - 1 + kSlotsHot - 3) / (kSlotsHot - 2) : 1);
+    pl.hot_tpc = (int)tpc;
+    pl.hot_ctas = (int)((Nh + tpc - 1) / tpc);
+    pl.slots_hot = (int)((hot_tiles - 1) / tpc + 2);
+  }
+  if (N > 0) {
+    const int cc = std::max(1, slots - pl.hot_ctas);
+    int64_t bpc = (N + cc - 1) / cc;
+    bpc = std::max<int64_t>(bpc, cold_blocks > 1 ? (cold_blocks - 1 + kSlotsCold - 3) / (kSlotsCold - 2) : 1);
+    pl.cold_bpc = bpc;
+    pl.cold_ctas = (int)((N + bpc - 1) / bpc);
+    pl.slots_cold = (int)((cold_blocks - 1) / bpc + 2);
+  }
+
+  // scratch layout: rotated queries | q'' | per-head scales | partials
+  size_t off = 0;
+  const size_t o_qrot = off;   off += round_up((size_t)2 * 2 * heads * d, kAlign);
+  const size_t o_qsk = off;    off += round_up((size_t)2 * heads * m, kAlign);
+  const size_t o_qscale = off; off += round_up(sizeof(float) * 2 * heads, kAlign);
+  const size_t o_part = off;
+  off += round_up(sizeof(float) * units * (size_t)(pl.slots_cold + pl.slots_hot) * G * (d + 2), kAlign);
+  if (off > kStaticScratchBytes) return TQ_ERR_CAPACITY;   // too large for the static scratch
+
+  uint8_t* base = (uint8_t*)static_scratch_address(current);
+  if (!base) return TQ_ERR_CUDA;
+  __half* qrot = (__half*)(base + o_qrot);
+  __half* qsk = (__half*)(base + o_qsk);
+  float* qscale = (float*)(base + o_qscale);
+  float* part = (float*)(base + o_part);
+
+  if (pl.cold_ctas > 0) {
+    QPrepArgs qa{};
+    qa.q = (const __half*)q;
+    qa.signs = c->signs();
+    qa.St = c->St();
+    qa.qrot = qrot;
+    qa.qsk = qsk;
+    qa.qscale = qscale;
+    qa.heads = heads;
+    qa.d = d;
+    qa.m = m;
+    if (launch_qprep(qa, stream) != cudaSuccess) return TQ_ERR_CUDA;
+  }
+  if (pl.cold_ctas + pl.hot_ctas > 0) {
+    AttendArgs a{};
+    a.q = (const __half*)q;
+    a.qrot = qrot;
+    a.qsk = qsk;
+    a.qscale = qscale;
+    a.hot_k = c->hot_k();
+    a.hot_v = c->hot_v();
+    a.cold = c->cold;
+    a.part = part;
+    a.status = c->status();
+    a.L = c->L;
+    a.units = units;
+    a.G = G;
+    a.Hq = cf.num_q_heads;
+    a.Hkv = cf.num_kv_heads;
+    a.W = cf.hot_window;
+    a.n_hot = c->n_hot;
+    a.n_cold = c->n_cold;
+    a.plan = pl;
+    a.log2e_sigma = (float)(1.4426950408889634 * (double)sigma);
+    if (launch_attend(a, stream) != cudaSuccess) return TQ_ERR_CUDA;
+  }
+  CombineArgs ca{};
+  ca.part = part;
+  ca.signs = c->signs();
+  ca.out = out;
+  ca.units = units;
+  ca.G = G;
+  ca.Hkv = cf.num_kv_heads;
+  ca.Hq = cf.num_q_heads;
+  ca.d = d;
+  ca.plan = pl;
+  ca.batch = cf.batch;
+  if (launch_combine(ca, stream) != cudaSuccess) return TQ_ERR_CUDA;
   return TQ_OK;
 }
 

@@ -52,6 +52,7 @@ SIGNATURES = [
     ("tq_encode_append", c_int32, [c_void_p, c_void_p, c_void_p, c_int64, c_void_p]),
     ("tq_evict_window", c_int32, [c_void_p, c_void_p, c_void_p, c_int32, c_void_p]),
     ("tq_decode_attention", c_int32, [c_void_p, c_void_p, c_void_p, c_float, c_void_p]),
+    ("tq_decode_attention_static", c_int32, [c_void_p, c_void_p, c_void_p, c_float, c_void_p]),
     ("tq_get_status", c_int32, [c_void_p, c_void_p]),
     ("tq_set_attend_events", c_int32, [c_void_p, c_void_p, c_void_p]),
     ("tq_export_cold", c_int32, [c_void_p, c_int32, c_int32, c_int64, c_int64, c_void_p,
@@ -133,6 +134,12 @@ def tq_evict_window(handle: int, k_ptr: int, v_ptr: int, n: int, stream: int) ->
 
 def tq_decode_attention(handle: int, q_ptr: int, out_ptr: int, scale: float, stream: int) -> None:
     _check(lib().tq_decode_attention(handle, q_ptr, out_ptr, scale, stream), "tq_decode_attention")
+
+
+def tq_decode_attention_static(handle: int, q_ptr: int, out_ptr: int, scale: float,
+                               stream: int) -> None:
+    _check(lib().tq_decode_attention_static(handle, q_ptr, out_ptr, scale, stream),
+           "tq_decode_attention_static")
 
 
 def tq_get_status(handle: int, stream: int) -> int:

@@ -177,6 +177,28 @@ tq_status tq_decode_attention(tq_cache* cache, const void* q, float* out,
                               float softmax_scale, cudaStream_t stream);
 
 /*
+ * tq_decode_attention without caller-provided scratch (the pages have no
+ * counterpart; this is an integration convenience).  For callers that may
+ * not allocate device memory while they run -- an allocator-free serving
+ * loop, a plugin whose host owns every allocation, a process whose memory
+ * is reserved up front.  It computes exactly what tq_decode_attention does,
+ * with the same kernels, but keeps the per-call scratch (rotated queries and
+ * split partials) in a 4 MiB array compiled into the library: one copy per
+ * GPU that loads the library, resident until the process exits.  The call
+ * never allocates (no cudaMalloc / cudaFree, no allocating library call).
+ *   - The first call on a device looks up that array's device address
+ *     (cudaGetSymbolAddress) and remembers it; make that first call before
+ *     any stream capture.  The handle's device must be current.
+ *   - Calls whose GPU work overlaps (other streams, other handles on the
+ *     same device) share the array and race; serialize them.
+ *   - Returns TQ_ERR_CAPACITY, launching nothing, when this configuration's
+ *     scratch (about units x (partials + 2) x G x (d + 2) x 4 bytes plus the
+ *     query transforms) exceeds 4 MiB.
+ */
+tq_status tq_decode_attention_static(tq_cache* cache, const void* q, float* out,
+                                     float softmax_scale, cudaStream_t stream);
+
+/*
  * Synchronize `stream`, then return and clear the latched device status
  * (TQ_OK, TQ_ERR_RANGE or TQ_ERR_TIMEOUT), or TQ_ERR_CUDA if the stream
  * itself reports an error.
