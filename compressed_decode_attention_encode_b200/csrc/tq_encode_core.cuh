@@ -1,0 +1,164 @@
+// The float64 per-vector encode shared by the KV-cache encoder and the
+// vector-search encoder: randomized Hadamard rotation, polar codes with an
+// fp16 scale, and (for keys) the QJL sign sketch of the residual.
+#pragma once
+
+#include "tq_internal.cuh"
+
+namespace tq {
+namespace enc {
+
+constexpr unsigned kFull = 0xffffffffu;
+constexpr double kTwoPi = 6.283185307179586476925286766559;  // rounds to 2 * fp64(pi)
+
+__device__ __forceinline__ uint16_t f64_to_f16_bits(double x) {
+  uint16_t h;
+  asm("cvt.rn.f16.f64 %0, %1;" : "=h"(h) : "d"(x));
+  return h;
+}
+
+__device__ __forceinline__ double f16_bits_to_f64(uint16_t h) {
+  return (double)__half2float(__ushort_as_half(h));
+}
+
+template <int E>
+__device__ __forceinline__ void load_vec(const __half* p, int lane, double (&x)[E]) {
+  const __half* q = p + lane * E;
+  if constexpr (E == 2) {
+    const __half2 v = *reinterpret_cast<const __half2*>(q);
+    x[0] = (double)__low2float(v);
+    x[1] = (double)__high2float(v);
+  } else if constexpr (E == 4) {
+    const uint2 v = *reinterpret_cast<const uint2*>(q);
+    const __half2 a = *reinterpret_cast<const __half2*>(&v.x);
+    const __half2 b = *reinterpret_cast<const __half2*>(&v.y);
+    x[0] = (double)__low2float(a); x[1] = (double)__high2float(a);
+    x[2] = (double)__low2float(b); x[3] = (double)__high2float(b);
+  } else {
+#pragma unroll
+    for (int i = 0; i < E; ++i) x[i] = (double)__half2float(q[i]);
+  }
+}
+
+// Encodes one vector (K or V) held at `src` in float64; writes its code
+// words into `codes[0..D/2)` (shared memory, one byte per pair) and, for
+// keys, its sign words into `bits` (canonical order, bit i of word i/32)
+// and the raw fp16 scalars.  Whole warp; returns nothing else.
+// `load(lane, x)` fills the lane's D/32 consecutive input elements (padded
+// coordinates read as 0).  `L` supplies b_r, b_theta and m; `St` is S^T
+// [D, m]; `signs` the rotation diagonal.
+template <int D, typename Loader>
+__device__ __forceinline__ void encode_vector_any(const Layout& L, const double* signs,
+                                                  const float* St, double inv_sqrt_d, int* status,
+                                                  Loader load, bool is_key, double* rbuf,
+                                                  uint8_t* codes, uint32_t* bits,
+                                                  uint16_t* s16_out, uint16_t* rn16_out) {
+  constexpr int E = D / 32;      // elements per lane
+  constexpr int PL = E / 2;      // pairs per lane
+  const int lane = threadIdx.x & 31;
+  const int Lr = (1 << L.b_r) - 1;
+  const int nt = 1 << L.b_theta;
+
+  // ---- rotation: y = H (D x) / sqrt(d) ----------------------------------
+  double x[E];
+  load(lane, x);
+#pragma unroll
+  for (int i = 0; i < E; ++i) x[i] = __dmul_rn(x[i], signs[lane * E + i]);
+#pragma unroll
+  for (int h = 1; h < D; h <<= 1) {
+    if (h < E) {
+#pragma unroll
+      for (int i = 0; i < E; ++i) {
+        if (!(i & h)) {
+          const double p = x[i], q = x[i + h];
+          x[i] = __dadd_rn(p, q);
+          x[i + h] = __dsub_rn(p, q);
+        }
+      }
+    } else {
+      const int lm = h / E;
+#pragma unroll
+      for (int i = 0; i < E; ++i) {
+        const double o = __shfl_xor_sync(kFull, x[i], lm);
+        x[i] = (lane & lm) ? __dsub_rn(o, x[i]) : __dadd_rn(x[i], o);
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < E; ++i) x[i] = __dmul_rn(x[i], inv_sqrt_d);
+
+  // ---- polar: rho, theta per pair; scale s16 = fp16(max rho) ------------
+  double rho[PL], th[PL];
+  double smax = 0.0;
+#pragma unroll
+  for (int k = 0; k < PL; ++k) {
+    const double y0 = x[2 * k], y1 = x[2 * k + 1];
+    rho[k] = __dsqrt_rn(__dadd_rn(__dmul_rn(y0, y0), __dmul_rn(y1, y1)));
+    th[k] = atan2(y1, y0);
+    smax = fmax(smax, rho[k]);
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) smax = fmax(smax, __shfl_xor_sync(kFull, smax, o));
+  uint16_t s16b = f64_to_f16_bits(smax);
+  if ((s16b & 0x7c00u) == 0x7c00u) {       // overflow: latch, store a zero record
+    if (lane == 0) atomicOr(status, kStatusRange);
+    s16b = 0;
+  }
+  const double s16 = f16_bits_to_f64(s16b);
+  const bool zero = (s16 == 0.0);
+
+  // ---- codes ---------------------------------------------------------------
+  int cr[PL], ct[PL];
+#pragma unroll
+  for (int k = 0; k < PL; ++k) {
+    const double tr = __dmul_rn(__ddiv_rn(rho[k], zero ? 1.0 : s16), (double)Lr);
+    const int c = (int)rint(tr);
+    cr[k] = c < 0 ? 0 : (c > Lr ? Lr : c);
+    const double tt = __ddiv_rn(__dmul_rn(th[k], (double)nt), kTwoPi);
+    ct[k] = ((int)rint(tt)) & (nt - 1);
+    if (zero) { cr[k] = 0; ct[k] = 0; }
+    codes[lane * PL + k] = (uint8_t)((cr[k] << L.b_theta) | ct[k]);
+  }
+  if (lane == 0) *s16_out = s16b;
+
+  // ---- residual and QJL sketch (keys) -------------------------------------
+  if (is_key) {
+    double r[E];
+    double ss = 0.0;
+#pragma unroll
+    for (int k = 0; k < PL; ++k) {
+      const double rh = __ddiv_rn(__dmul_rn((double)cr[k], s16), (double)Lr);
+      const double ang = __ddiv_rn(__dmul_rn((double)ct[k], kTwoPi), (double)nt);
+      double sn, cs;
+      sincos(ang, &sn, &cs);
+      r[2 * k] = __dsub_rn(x[2 * k], __dmul_rn(rh, cs));
+      r[2 * k + 1] = __dsub_rn(x[2 * k + 1], __dmul_rn(rh, sn));
+      ss = __dadd_rn(ss, __dadd_rn(__dmul_rn(r[2 * k], r[2 * k]), __dmul_rn(r[2 * k + 1], r[2 * k + 1])));
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) ss = __dadd_rn(ss, __shfl_xor_sync(kFull, ss, o));
+    const uint16_t rnb = f64_to_f16_bits(__dsqrt_rn(ss));
+    if ((rnb & 0x7c00u) == 0x7c00u && lane == 0) atomicOr(status, kStatusRange);
+    if (lane == 0) *rn16_out = rnb;
+#pragma unroll
+    for (int i = 0; i < E; ++i) rbuf[lane * E + i] = r[i];
+    __syncwarp();
+    const int m = L.m;
+    for (int k = 0; k < (m + 31) / 32; ++k) {
+      const int i = lane + 32 * k;
+      double acc = 0.0;
+      if (i < m) {
+        const float* col = St + i;
+#pragma unroll 8
+        for (int jj = 0; jj < D; ++jj) acc = fma((double)__ldg(col + (size_t)jj * m), rbuf[jj], acc);
+      }
+      const unsigned word = __ballot_sync(kFull, i < m && acc >= 0.0);
+      if (lane == 0) bits[k] = word;
+    }
+  }
+  __syncwarp();
+}
+
+
+}  // namespace enc
+}  // namespace tq

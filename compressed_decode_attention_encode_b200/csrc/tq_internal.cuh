@@ -181,4 +181,57 @@ struct CombineArgs {
 
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s);
 
+// ---- vector search ----------------------------------------------------
+struct VecEncodeArgs {
+  const float* x;           // [count, dim]
+  int64_t start, count;
+  int dim;
+  Layout L;                 // d (padded), b_r, b_theta, m
+  const double* signs;
+  const float* St;          // [d, m]
+  double inv_sqrt_d;
+  int* status;
+  uint8_t* codes;           // [n][d/2]
+  uint8_t* signs_out;       // [n][32]
+  uint16_t* s16_out;        // [n]
+  uint16_t* rn16_out;       // [n]
+};
+
+struct VecQPrepArgs {
+  const float* q;           // [nq, dim]
+  int nq, dim, d, m;
+  const double* signs;
+  const float* St;
+  __half* A;                // [nq, d + 256] fp16 MMA operand
+  float* qscale;            // [nq]
+};
+
+struct SearchArgs {
+  const __half* A;
+  const uint8_t* codes;
+  const uint8_t* signs;
+  const uint16_t* s16;
+  const uint16_t* rn16;
+  int64_t n;
+  int nq, d, b_theta, nsplit;
+  float inv_levels;         // 1 / (2^b_r - 1)
+  float qjl_const;          // sqrt(pi/2) / m
+  float* part_s;            // [nq][nsplit][2][16]
+  int* part_i;
+};
+
+struct MergeArgs {
+  const float* part_s;
+  const int* part_i;
+  const float* qscale;
+  int nq, nsplit, k;
+  float* scores;            // [nq, k]
+  int* idx;
+};
+
+cudaError_t launch_vec_encode(const VecEncodeArgs& a, cudaStream_t s);
+cudaError_t launch_vec_qprep(const VecQPrepArgs& a, cudaStream_t s);
+cudaError_t launch_search(const SearchArgs& a, cudaStream_t s);
+cudaError_t launch_topk_merge(const MergeArgs& a, cudaStream_t s);
+
 }  // namespace tq

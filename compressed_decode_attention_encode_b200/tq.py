@@ -37,6 +37,11 @@ class tq_config(Structure):
                 ("seed", c_uint64)]
 
 
+class tq_vec_config(Structure):
+    _fields_ = [("dim", c_int32), ("b_r", c_int32), ("b_theta", c_int32), ("qjl_bits", c_int32),
+                ("seed", c_uint64)]
+
+
 _lib = None
 
 # (name, restype, argtypes) of every exported symbol
@@ -57,6 +62,16 @@ SIGNATURES = [
     ("tq_set_attend_events", c_int32, [c_void_p, c_void_p, c_void_p]),
     ("tq_export_cold", c_int32, [c_void_p, c_int32, c_int32, c_int64, c_int64, c_void_p,
                                  c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
+    ("tq_vec_bytes", c_int32, [POINTER(tq_vec_config), c_int64, c_int32, POINTER(c_size_t),
+                               POINTER(c_size_t)]),
+    ("tq_vec_create", c_int32, [POINTER(tq_vec_config), c_int64, c_int32, c_void_p, c_void_p,
+                                POINTER(c_void_p)]),
+    ("tq_vec_destroy", c_int32, [c_void_p]),
+    ("tq_encode_vectors", c_int32, [c_void_p, c_void_p, c_int64, c_int64, c_void_p, c_void_p]),
+    ("tq_ip_search", c_int32, [c_void_p, c_void_p, c_void_p, c_int32, c_int32, c_void_p, c_void_p,
+                               c_void_p]),
+    ("tq_export_vectors", c_int32, [c_void_p, c_void_p, c_int64, c_int64, c_void_p, c_void_p,
+                                    c_void_p, c_void_p, c_void_p]),
     ("tq_rotation_signs", c_int32, [c_uint64, c_int32, POINTER(c_int8)]),
     ("tq_qjl_matrix", c_int32, [c_uint64, c_int32, c_int32, POINTER(c_float)]),
 ]
@@ -261,4 +276,78 @@ class TQCache:
         _check(lib().tq_export_cold(self.handle, row, kv_head, start, count, p["k_codes"],
                                     p["k_bits"], p["k_s16"], p["k_rn16"], p["v_codes"], p["v_s16"],
                                     _stream_handle(stream)), "tq_export_cold")
+        return out
+
+
+# ---- vector search ----------------------------------------------------------
+
+def tq_vec_bytes(cfg: tq_vec_config, n: int, max_queries: int):
+    c, w = c_size_t(), c_size_t()
+    _check(lib().tq_vec_bytes(ctypes.byref(cfg), n, max_queries, ctypes.byref(c), ctypes.byref(w)),
+           "tq_vec_bytes")
+    return c.value, w.value
+
+
+class TQVecIndex:
+    """Compressed vector database + search handle (device memory from
+    PyTorch; every method is a direct call into libtq.so)."""
+
+    def __init__(self, dim, n, b_r=4, b_theta=4, qjl_bits=200, seed=0, max_queries=1024,
+                 device="cuda", stream=None):
+        import torch
+        self.cfg = tq_vec_config(dim, b_r, b_theta, qjl_bits, seed)
+        self.n = n
+        cb, wb = tq_vec_bytes(self.cfg, n, max_queries)
+        self.codes = torch.empty(max(cb, 256), dtype=torch.uint8, device=device)
+        self.ws = torch.empty(max(wb, 256), dtype=torch.uint8, device=device)
+        out = c_void_p()
+        _check(lib().tq_vec_create(ctypes.byref(self.cfg), n, max_queries, self.ws.data_ptr(),
+                                   _stream_handle(stream), ctypes.byref(out)), "tq_vec_create")
+        self.handle = out.value
+
+    def close(self):
+        if getattr(self, "handle", None):
+            _check(lib().tq_vec_destroy(self.handle), "tq_vec_destroy")
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def encode(self, x, start=0, stream=None):
+        """x: contiguous CUDA float32 [count, dim] -> database rows start.."""
+        import torch
+        if x.dtype != torch.float32 or not x.is_cuda or not x.is_contiguous():
+            raise ValueError("expected a contiguous CUDA float32 tensor")
+        _check(lib().tq_encode_vectors(self.handle, x.data_ptr(), start, x.shape[0],
+                                       self.codes.data_ptr(), _stream_handle(stream)),
+               "tq_encode_vectors")
+
+    def search(self, q, k=10, stream=None):
+        """q: contiguous CUDA float32 [nq, dim] -> (scores [nq, k], idx [nq, k])."""
+        import torch
+        if q.dtype != torch.float32 or not q.is_cuda or not q.is_contiguous():
+            raise ValueError("expected a contiguous CUDA float32 tensor")
+        nq = q.shape[0]
+        scores = torch.empty((nq, k), dtype=torch.float32, device=q.device)
+        idx = torch.empty((nq, k), dtype=torch.int32, device=q.device)
+        _check(lib().tq_ip_search(self.handle, self.codes.data_ptr(), q.data_ptr(), nq, k,
+                                  scores.data_ptr(), idx.data_ptr(), _stream_handle(stream)),
+               "tq_ip_search")
+        return scores, idx
+
+    def export(self, start, count, stream=None):
+        d = 64
+        while d < self.cfg.dim:
+            d *= 2
+        kc = d // 2 * (self.cfg.b_r + self.cfg.b_theta) // 8
+        mb = self.cfg.qjl_bits // 8
+        out = dict(codes=np.zeros((count, kc), np.uint8), bits=np.zeros((count, mb), np.uint8),
+                   s16=np.zeros(count, np.uint16), rn16=np.zeros(count, np.uint16))
+        p = {k: v.ctypes.data for k, v in out.items()}
+        _check(lib().tq_export_vectors(self.handle, self.codes.data_ptr(), start, count, p["codes"],
+                                       p["bits"], p["s16"], p["rn16"], _stream_handle(stream)),
+               "tq_export_vectors")
         return out

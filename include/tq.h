@@ -219,6 +219,70 @@ tq_status tq_export_cold(tq_cache* cache, int32_t row, int32_t kv_head,
                          uint8_t* v_codes, uint16_t* v_s16,
                          cudaStream_t stream);
 
+/* ------------------------------------------------------------------------
+ * Vector inner-product search over the same codes.
+ * [TQ-3B] "Aplicaciones más allá de los LLMs": the compressed vectors serve
+ * vector search / RAG ranking.  Database vectors (float32, dimension d_in,
+ * zero-padded to d = the next power of two >= 64) are encoded exactly like
+ * keys: rotation, polar codes, fp16 scale, m QJL sign bits of the residual
+ * and its fp16 norm.  A query q is scored against vector i by the same
+ * estimator as a cold attention logit, without the softmax scale:
+ *   score = s16_i/(2^b_r-1) <q', x_hat_unit_i> + rn16_i sqrt(pi/2)/m <q'', 2 bits_i - 1>
+ * and the k best scores per query are returned (descending; equal scores
+ * in index order).
+ * ---------------------------------------------------------------------- */
+typedef struct tq_vec_config {
+  int32_t dim;              /* d_in, 1..256                                  */
+  int32_t b_r;              /* radius bits; b_r + b_theta must equal 8       */
+  int32_t b_theta;          /* angle bits                                    */
+  int32_t qjl_bits;         /* m: 8..256, a multiple of 8                    */
+  uint64_t seed;            /* rotation signs D and QJL matrix S             */
+} tq_vec_config;
+
+typedef struct tq_vec_index tq_vec_index;
+
+/*
+ * Sizes for an index over n vectors:
+ *   codes_bytes      the packed database: codes [n][d/2] (one byte per pair),
+ *                    sign bits [n][32] (m bits, zero-padded to 256), s16 [n],
+ *                    rn16 [n]; each section 256-byte aligned.
+ *   workspace_bytes  D, S, query transforms for up to `max_queries` queries
+ *                    and the per-split top-k partials of a search.
+ */
+tq_status tq_vec_bytes(const tq_vec_config* cfg, int64_t n, int32_t max_queries,
+                       size_t* codes_bytes, size_t* workspace_bytes);
+
+/* Bind a search handle to a caller-owned workspace (uploads D and S). */
+tq_status tq_vec_create(const tq_vec_config* cfg, int64_t n, int32_t max_queries,
+                        void* workspace_mem, cudaStream_t stream, tq_vec_index** out);
+tq_status tq_vec_destroy(tq_vec_index* index);
+
+/*
+ * Encode database vectors [start, start + count) of x (device float32
+ * [count, d_in], row-major) into `codes` (device, tq_vec_bytes layout).
+ * Decisions in float64 as for tq_encode_append.
+ */
+tq_status tq_encode_vectors(tq_vec_index* index, const float* x, int64_t start,
+                            int64_t count, void* codes, cudaStream_t stream);
+
+/*
+ * Top-k estimated inner products of nq queries (device float32 [nq, d_in])
+ * against all n encoded vectors.  scores: device float32 [nq, k]; idx:
+ * device int32 [nq, k].  1 <= k <= 16, nq <= max_queries.  The products
+ * run on tensor cores (fp16 operands, fp32 accumulation).
+ */
+tq_status tq_ip_search(tq_vec_index* index, const void* codes, const float* q, int32_t nq,
+                       int32_t k, float* scores, int32_t* idx, cudaStream_t stream);
+
+/*
+ * Canonical records of database vectors [start, start + count) to HOST
+ * buffers (synchronizes): codes [count][d/2*(b_r+b_theta)/8] in the
+ * LSB-first stream form of tq_export_cold, bits [count][m/8], s16, rn16.
+ */
+tq_status tq_export_vectors(tq_vec_index* index, const void* codes, int64_t start,
+                            int64_t count, uint8_t* codes_out, uint8_t* bits_out,
+                            uint16_t* s16_out, uint16_t* rn16_out, cudaStream_t stream);
+
 /*
  * Measurement hook: when `start` and `stop` are non-NULL, every following
  * tq_decode_attention call on this handle records `start` on its stream

@@ -125,3 +125,31 @@ def test_cold_store_holds_exactly_the_algorithmic_bytes(lib, d, m, b_r, b_t):
         words = -(-16 * bw // 32)
         per_token = 2 * (words * 4 * 32 // 16) + m // 8 + 6
     assert cold == 64 * per_token
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(b_r=3, b_theta=3), 2),      # the search kernel reads one byte per pair
+    (dict(dim=300), 2),
+    (dict(qjl_bits=20), 1),
+    (dict(qjl_bits=264), 2),
+    (dict(dim=0), 1),
+])
+def test_vector_config_validation(lib, kw, code):
+    base = dict(dim=200, b_r=4, b_theta=4, qjl_bits=200, seed=0)
+    base.update(kw)
+    cfg = tq.tq_vec_config(base["dim"], base["b_r"], base["b_theta"], base["qjl_bits"], base["seed"])
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_vec_bytes(cfg, 1000, 16)
+    assert e.value.code == code
+
+
+def test_vector_codes_bytes():
+    """codes [n][d/2] + signs [n][32] + s16 [n] + rn16 [n], each section
+    rounded up to 256 bytes (d = 200 pads to 256)."""
+    tq.lib()
+    cfg = tq.tq_vec_config(200, 4, 4, 200, 0)
+    n = 1_000_000
+    cb, wb = tq.tq_vec_bytes(cfg, n, 1024)
+    r = lambda x: -(-x // 256) * 256
+    assert cb == r(n * 128) + r(n * 32) + 2 * r(n * 2)
+    assert wb > 0
