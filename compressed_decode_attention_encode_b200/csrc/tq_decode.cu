@@ -33,6 +33,9 @@ namespace {
 
 constexpr unsigned kFull = 0xffffffffu;
 constexpr int kThreads = 128;          // 4 warps; each takes 16 tokens of a 64-token block
+constexpr int kAttendMinBlocks = 4;    // attention CTAs per SM the shapes are sized for
+constexpr int kSmemPerSm = 233472;     // shared memory per SM (bytes)
+constexpr int kAccSplit = 1;           // independent accumulator chains per tile product
 constexpr float kNegInf = -INFINITY;
 constexpr float kSqrtHalfPi = 1.2533141373155001f;   // sqrt(pi / 2)
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // bounded mbarrier waits
@@ -139,155 +142,112 @@ __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-// +-1 fp16 pair from the two sign bits at positions 15 and 31 of (x << u):
-// bit 1 -> +1.0 (0x3C00), bit 0 -> -1.0 (0xBC00).
+// +-1 fp16 pair from sign bits 15-u and 31-u of x: bit 1 -> +1.0 (0x3C00),
+// bit 0 -> -1.0 (0xBC00).  The mask is a logic op; moving the bits to the
+// fp16 sign positions and mapping them is one integer multiply-add
+// (0xBC00BC00 - b * 2^u), which runs beside the logic ops.
 __device__ __forceinline__ uint32_t sign_pair(uint32_t x, int u) {
-  return ((x << u) & 0x80008000u) ^ 0xBC00BC00u;
+  return 0xBC00BC00u - (x & (0x80008000u >> u)) * (1u << u);
 }
 
-// Loads NW 32-bit words of a bit stream starting at bit `start` of `rec`
-// (4-byte aligned), re-based so that bit `start` becomes bit 0 of out[0].
-template <int NW>
-__device__ __forceinline__ void load_chunk(const uint8_t* rec, int start, uint32_t (&out)[NW]) {
-  const uint32_t* p = reinterpret_cast<const uint32_t*>(rec) + (start >> 5);
-  const int sh = start & 31;
-  uint32_t raw[NW + 1];
-#pragma unroll
-  for (int i = 0; i <= NW; ++i) raw[i] = p[i];
-#pragma unroll
-  for (int i = 0; i < NW; ++i) out[i] = __funnelshift_r(raw[i], raw[i + 1], sh);
-}
-
-// The BW-bit field at bit `pos` (a compile-time constant after unrolling).
-template <int BW, int NW>
-__device__ __forceinline__ uint32_t field(const uint32_t (&w)[NW], int pos) {
-  const int wi = pos >> 5, bi = pos & 31;
-  uint32_t v;
-  if (bi + BW <= 32 || wi + 1 >= NW)
-    v = w[wi] >> bi;
-  else
-    v = __funnelshift_r(w[wi], w[wi + 1], bi);
-  return v & ((1u << BW) - 1u);
-}
-
-// The BW-bit field at bit `pos` (compile-time after unrolling), returned
-// already shifted left by SH and masked, so that `| lane * (1 << SH) / 32`
-// gives the byte offset of this lane's copy of the LUT entry: one funnel
-// shift plus one LOP3.
+// Byte offset in a LUT whose entries are 2^SH bytes apart, of the entry
+// named by the BW-bit field at bit `pos` of the lane's word stream (`pos`
+// is a compile-time constant after unrolling), plus `lane_off` (the lane's
+// copy inside the entry).  A field inside one word costs a mask and an
+// integer multiply-add (a left shift, or a high-half multiply for a right
+// shift); a field straddling two words costs a funnel shift and a mask.
 template <int BW, int SH, int NW>
-__device__ __forceinline__ uint32_t field_shifted(const uint32_t (&w)[NW], int pos) {
+__device__ __forceinline__ uint32_t lut_offset(const uint32_t (&w)[NW], int pos, uint32_t lane_off) {
+  constexpr uint32_t kMask = (1u << BW) - 1u;
   const int wi = pos >> 5, bi = pos & 31;
-  uint32_t v;
-  if (bi + BW <= 32 || wi + 1 >= NW)
-    v = bi >= SH ? (w[wi] >> (bi - SH)) : (w[wi] << (SH - bi));
-  else
-    v = __funnelshift_r(w[wi], w[wi + 1], bi - SH);   // straddling: bi > 32 - BW >= SH
-  return v & (((1u << BW) - 1u) << SH);
-}
-
-// Online-softmax step over one 16-token tile for the thread's two heads
-// (2*tig, 2*tig+1).  l2[0..1]: token gid, l2[2..3]: token gid+8 (log2
-// domain).  Writes p = exp2(l2 - m_new) and the factor corr by which sums
-// accumulated so far must be rescaled.
-__device__ __forceinline__ void softmax_tile(const float (&l2)[4], float (&m_run)[2],
-                                             float (&p)[4], float (&corr)[2]) {
-  float t0 = fmaxf(l2[0], l2[2]), t1 = fmaxf(l2[1], l2[3]);
-#pragma unroll
-  for (int o = 4; o < 32; o <<= 1) {
-    t0 = fmaxf(t0, __shfl_xor_sync(kFull, t0, o));
-    t1 = fmaxf(t1, __shfl_xor_sync(kFull, t1, o));
+  if (bi + BW <= 32 || wi + 1 >= NW) {
+    const uint32_t f = w[wi] & (kMask << bi);
+    if (bi <= SH) return f * (1u << (SH - bi)) + lane_off;
+    return __umulhi(f, 1u << (32 - (bi - SH))) + lane_off;
   }
-  const float n0 = fmaxf(m_run[0], t0), n1 = fmaxf(m_run[1], t1);
-  const float r0 = n0 == kNegInf ? 0.f : n0, r1 = n1 == kNegInf ? 0.f : n1;
-  corr[0] = fast_exp2(m_run[0] - r0);
-  corr[1] = fast_exp2(m_run[1] - r1);
-  p[0] = fast_exp2(l2[0] - r0);
-  p[1] = fast_exp2(l2[1] - r1);
-  p[2] = fast_exp2(l2[2] - r0);
-  p[3] = fast_exp2(l2[3] - r1);
-  m_run[0] = n0;
-  m_run[1] = n1;
+  return (__funnelshift_r(w[wi], w[wi + 1], bi - SH) & (kMask << SH)) | lane_off;
 }
 
 // ---------------------------------------------------------------------------
-// q-prep: 8 heads per block, one warp per head for the rotation; S q' is
-// register-blocked so that every S element is read once per block.
+// q-prep: HB = 256 / M heads per block (2 for m = 128), so that the grid
+// spreads over the SMs.  One warp per head rotates q (butterflies in
+// registers and across lanes); then every thread computes one element of
+// S q' from S^T staged in shared memory (loads issued before the rotation).
 // ---------------------------------------------------------------------------
 template <int D, int M>
 __global__ void __launch_bounds__(256) qprep_kernel(const QPrepArgs a) {
   constexpr int E = D / 32;
-  constexpr int HPT = 8 * M / 256;       // heads per thread in S q'
-  __shared__ float sq[8][D];
-  __shared__ float sqq[8][M];
+  constexpr int HB = 256 / M;            // heads per block
+  __shared__ float sq[HB][D];
+  __shared__ float sqq[HB][M];
+  extern __shared__ float4 sst4[];       // S^T [D][M]
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int h = blockIdx.x * 8 + warp;
-  const bool live = h < a.heads;
-  float x[E];
+  for (int i = threadIdx.x; i < D * M / 4; i += blockDim.x)
+    sst4[i] = __ldg(reinterpret_cast<const float4*>(a.St) + i);
+  const float* sst = reinterpret_cast<const float*>(sst4);
+  const int h = blockIdx.x * HB + warp;          // head of this warp (warps < HB)
+  if (warp < HB) {
+    const bool live = h < a.heads;
+    float x[E];
 #pragma unroll
-  for (int i = 0; i < E; ++i)
-    x[i] = live ? __half2float(a.q[(size_t)h * D + lane * E + i]) * (float)a.signs[lane * E + i] : 0.f;
+    for (int i = 0; i < E; ++i)
+      x[i] = live ? __half2float(a.q[(size_t)h * D + lane * E + i]) * (float)a.signs[lane * E + i] : 0.f;
 #pragma unroll
-  for (int hh = 1; hh < D; hh <<= 1) {
-    if (hh < E) {
+    for (int hh = 1; hh < D; hh <<= 1) {
+      if (hh < E) {
 #pragma unroll
-      for (int i = 0; i < E; ++i)
-        if (!(i & hh)) {
-          const float p = x[i], q = x[i + hh];
-          x[i] = p + q;
-          x[i + hh] = p - q;
+        for (int i = 0; i < E; ++i)
+          if (!(i & hh)) {
+            const float p = x[i], q = x[i + hh];
+            x[i] = p + q;
+            x[i + hh] = p - q;
+          }
+      } else {
+        const int lm = hh / E;
+#pragma unroll
+        for (int i = 0; i < E; ++i) {
+          const float o = __shfl_xor_sync(kFull, x[i], lm);
+          x[i] = (lane & lm) ? (o - x[i]) : (x[i] + o);
         }
-    } else {
-      const int lm = hh / E;
-#pragma unroll
-      for (int i = 0; i < E; ++i) {
-        const float o = __shfl_xor_sync(kFull, x[i], lm);
-        x[i] = (lane & lm) ? (o - x[i]) : (x[i] + o);
       }
     }
-  }
-  const float inv = rsqrtf((float)D);
-  float amax = 0.f;
-#pragma unroll
-  for (int i = 0; i < E; ++i) {
-    x[i] *= inv;
-    sq[warp][lane * E + i] = x[i];
-    amax = fmaxf(amax, fabsf(x[i]));
-  }
-#pragma unroll
-  for (int o = 16; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, o));
-  const float al1 = amax > 0.f ? exp2f(-floorf(log2f(amax))) : 1.f;
-  if (live) {
+    const float inv = rsqrtf((float)D);
+    float amax = 0.f;
 #pragma unroll
     for (int i = 0; i < E; ++i) {
-      const float v = x[i] * al1;
-      const __half hi = __float2half_rn(v);
-      a.qrot[(size_t)h * 2 * D + lane * E + i] = hi;
-      a.qrot[(size_t)h * 2 * D + D + lane * E + i] = __float2half_rn(v - __half2float(hi));
+      x[i] *= inv;
+      sq[warp][lane * E + i] = x[i];
+      amax = fmaxf(amax, fabsf(x[i]));
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, o));
+    const float al1 = amax > 0.f ? exp2f(-floorf(log2f(amax))) : 1.f;
+    if (live) {
+#pragma unroll
+      for (int i = 0; i < E; ++i) {
+        const float v = x[i] * al1;
+        const __half hi = __float2half_rn(v);
+        a.qrot[(size_t)h * 2 * D + lane * E + i] = hi;
+        a.qrot[(size_t)h * 2 * D + D + lane * E + i] = __float2half_rn(v - __half2float(hi));
+      }
+      if (lane == 0) a.qscale[2 * h] = 1.f / al1;
     }
   }
   __syncthreads();
   {
-    const int i = threadIdx.x % M;
-    const int hb = (threadIdx.x / M) * HPT;
-    float acc[HPT];
-#pragma unroll
-    for (int k = 0; k < HPT; ++k) acc[k] = 0.f;
-#pragma unroll 4
-    for (int j = 0; j < D; ++j) {
-      const float sv = __ldg(a.St + (size_t)j * M + i);
-#pragma unroll
-      for (int k = 0; k < HPT; ++k) acc[k] = fmaf(sv, sq[hb + k][j], acc[k]);
-    }
-#pragma unroll
-    for (int k = 0; k < HPT; ++k) sqq[hb + k][i] = acc[k];
+    const int hb = threadIdx.x / M, i = threadIdx.x % M;
+    float acc = 0.f;
+#pragma unroll 8
+    for (int j = 0; j < D; ++j) acc = fmaf(sst[j * M + i], sq[hb][j], acc);
+    sqq[hb][i] = acc;
   }
   __syncthreads();
+  if (warp >= HB || h >= a.heads) return;
   float bmax = 0.f;
   for (int i = lane; i < M; i += 32) bmax = fmaxf(bmax, fabsf(sqq[warp][i]));
 #pragma unroll
   for (int o = 16; o; o >>= 1) bmax = fmaxf(bmax, __shfl_xor_sync(kFull, bmax, o));
   const float al2 = bmax > 0.f ? exp2f(-floorf(log2f(bmax))) : 1.f;
-  if (!live) return;
   // sign-fragment order: for chunk tig (m/4 signs) and slot u < m/8 the pair
   // (q''[c + m/8 - 1 - u], q''[c + m/4 - 1 - u]), c = tig * m/4.
   constexpr int Q4 = M / 4, H = M / 8;
@@ -297,10 +257,7 @@ __global__ void __launch_bounds__(256) qprep_kernel(const QPrepArgs a) {
     const int pos = (tg * H + u) * 2 + (j < H ? 0 : 1);
     a.qsk[(size_t)h * M + pos] = __float2half_rn(sqq[warp][i] * al2);
   }
-  if (lane == 0) {
-    a.qscale[2 * h] = 1.f / al1;
-    a.qscale[2 * h + 1] = 1.f / al2;
-  }
+  if (lane == 0) a.qscale[2 * h + 1] = 1.f / al2;
 }
 
 // ---------------------------------------------------------------------------
@@ -325,20 +282,24 @@ struct AttendShape {
   static constexpr int TB = kTokensPerBlock;
   static constexpr int BLOCK = kTilesPerBlock * TT;
   static constexpr int NLUT = 1 << BW;
-  static constexpr int KLUT_BYTES = NLUT * 32 * 8;  // (hi, lo) half2 per lane copy
-  static constexpr int VLUT_BYTES = NLUT * 32 * 4;  // hi half2 per lane copy
+  // two LUTs of fp16 pairs, one 4-byte copy per lane per entry: hi (keys
+  // and values) and lo (the keys' rounding remainder)
+  static constexpr int LUT_BYTES = NLUT * 32 * 4;
   // LUTs up to 48 KB live in static shared memory, whose address the
   // compiler folds into the load's immediate; larger ones are dynamic.
-  static constexpr bool STATIC_LUT = KLUT_BYTES + VLUT_BYTES <= 49152;
-  static constexpr int DYN_LUT = STATIC_LUT ? 0 : KLUT_BYTES + VLUT_BYTES;
+  static constexpr bool STATIC_LUT = 2 * LUT_BYTES <= 49152;
+  static constexpr int DYN_LUT = STATIC_LUT ? 0 : 2 * LUT_BYTES;
   static constexpr int RS = 2 * D + 16;             // padded hot row stride (bytes)
-  static constexpr int HOT_BYTES = 2 * TB * RS;
-  static constexpr int RING_BUDGET = KLUT_BYTES >= 65536 ? 20480 : 30720;
+  static constexpr int HOT_BYTES = TB * RS;          // one hot tile, K then V
+  static constexpr int MERGE_BYTES = (64 + 8 * D) * 4;
+  // ring stages: as many as fit beside the LUTs and the merge area when
+  // kAttendMinBlocks CTAs share an SM (at least 2, at most 8)
+  static constexpr int SMEM_PER_CTA = kSmemPerSm / kAttendMinBlocks - 1024;
+  static constexpr int RING_BUDGET = SMEM_PER_CTA - 2 * LUT_BYTES - MERGE_BYTES - 256;
   static constexpr int NS_RAW = RING_BUDGET / BLOCK;
   static constexpr int NS = NS_RAW < 2 ? 2 : (NS_RAW > 8 ? 8 : NS_RAW);   // ring stages
   static constexpr int RING = NS * BLOCK > HOT_BYTES ? NS * BLOCK : HOT_BYTES;
-  static constexpr int MERGE_BYTES = (64 + 8 * D) * 4;
-  static constexpr int OFF_VLUT = KLUT_BYTES;        // (dynamic LUT case)
+  static constexpr int OFF_LO = LUT_BYTES;           // (dynamic LUT case)
   static constexpr int OFF_RING = DYN_LUT;
   static constexpr int OFF_MERGE = OFF_RING + RING;
   static constexpr int OFF_BAR = OFF_MERGE + MERGE_BYTES;
@@ -366,27 +327,85 @@ __device__ __forceinline__ uint32_t spread16(uint32_t c) {
   return ((c & 0xffu) << 8) | ((c >> 8 & 0xffu) << 24);
 }
 
-constexpr float kLazyHeadroom = 8.f;   // log2 units the reference max may lag
+constexpr float kPvMax = 256.f;        // V weights p * s16_v stay <= 2^8 (fp16 operands)
+constexpr float kPMax = 0x1p100f;      // softmax numerators p stay <= 2^100 (fp32 sums)
+constexpr float kPRange = 100.f;
 
-// Per-warp softmax / accumulator state for one unit.
+// Per-warp softmax / accumulator state for one unit: the reference `ref`
+// (log2 domain) of the numerators p = 2^(l - ref) summed in `l_run`, and
+// the accumulators O of the V weights p * s16_v.
 template <int NT>
 struct WarpState {
-  float m_run[2], l_run[2], mp_run[2];
+  float ref[2], l_run[2];
   float O[NT][4];
   __device__ __forceinline__ void reset() {
-    m_run[0] = m_run[1] = kNegInf;
-    mp_run[0] = mp_run[1] = kNegInf;
+    ref[0] = ref[1] = kNegInf;
     l_run[0] = l_run[1] = 0.f;
 #pragma unroll
     for (int i = 0; i < NT; ++i) O[i][0] = O[i][1] = O[i][2] = O[i][3] = 0.f;
   }
 };
 
+// Online softmax over one 16-token tile with a lazily moved reference.
+// l2: log2-domain logits of tokens gid (l2[0..1]) and gid + 8 (l2[2..3]) for
+// the thread's two heads; sv0 / sv1: the two tokens' V weights (the V
+// record's s16, or 1 for hot tokens).  Produces p = 2^(l2 - ref) (added to
+// l_run) and pv = p * sv (the V weights).  The reference moves -- one warp
+// reduction, and a rescale of the sums -- only when some pv would exceed
+// 2^8 or some p 2^100, so every pv fits fp16.
+template <int NT>
+__device__ __forceinline__ void softmax_step(WarpState<NT>& st, const float (&l2)[4], float sv0,
+                                             float sv1, float (&pv)[4]) {
+  const float sv[4] = {sv0, sv0, sv1, sv1};
+  float p[4];
+  bool ok = true;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    p[j] = fast_exp2(l2[j] - st.ref[j & 1]);
+    pv[j] = p[j] * sv[j];
+    ok &= (pv[j] <= kPvMax) & (p[j] <= kPMax);   // false for NaN (no reference yet)
+  }
+  if (!__all_sync(kFull, ok)) {
+    // new reference: max over the tile of max(l2 + log2 sv, l2 - 100)
+    float t[2] = {kNegInf, kNegInf};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float tau = fmaxf(l2[j] + fast_log2(sv[j]), l2[j] - kPRange);
+      t[j & 1] = fmaxf(t[j & 1], tau);
+    }
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      t[0] = fmaxf(t[0], __shfl_xor_sync(kFull, t[0], o));
+      t[1] = fmaxf(t[1], __shfl_xor_sync(kFull, t[1], o));
+    }
+    float corr[2];
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const float nr = fmaxf(st.ref[hh], t[hh]);
+      corr[hh] = st.ref[hh] == kNegInf ? 0.f : fast_exp2(st.ref[hh] - nr);
+      st.ref[hh] = nr;
+      st.l_run[hh] *= corr[hh];
+    }
+#pragma unroll
+    for (int i = 0; i < NT; ++i) {
+      st.O[i][0] *= corr[0]; st.O[i][1] *= corr[1]; st.O[i][2] *= corr[0]; st.O[i][3] *= corr[1];
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      p[j] = fast_exp2(l2[j] - st.ref[j & 1]);
+      pv[j] = p[j] * sv[j];
+    }
+  }
+  st.l_run[0] += p[0] + p[2];
+  st.l_run[1] += p[1] + p[3];
+}
+
 // Merges the 4 warps' states into one partial {m, l, o[D]} per head and
-// writes it to `dst` ([G][D + 2]).  Called by all threads of the CTA; uses
-// 4 KB of shared memory (per-warp m / l, then the o sums by shared atomics).
+// writes it to `dst` ([G][D + 2]).  Lane (gid, tig) holds heads 2*tig + hh
+// (heads >= G are dropped).  Called by all threads of the CTA; uses the
+// merge area: per-warp m / l, then per-warp o rows summed by the threads.
 template <int D, int NT>
-__device__ __forceinline__ void flush_partial(WarpState<NT>& st, bool hot, int Lr, int G,
+__device__ __forceinline__ void flush_partial(WarpState<NT>& st, bool hot, float inv_levels, int G,
                                               float* merge, float* dst) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int gid = lane >> 2, tig = lane & 3;
@@ -401,7 +420,7 @@ __device__ __forceinline__ void flush_partial(WarpState<NT>& st, bool hot, int L
   if (gid == 0) {
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
-      mw[warp * 8 + 2 * tig + hh] = st.m_run[hh];
+      mw[warp * 8 + 2 * tig + hh] = st.ref[hh];
       lw[warp * 8 + 2 * tig + hh] = st.l_run[hh];
     }
   }
@@ -414,24 +433,27 @@ __device__ __forceinline__ void flush_partial(WarpState<NT>& st, bool hot, int L
     float mx = kNegInf;
 #pragma unroll
     for (int w = 0; w < 4; ++w) mx = fmaxf(mx, mw[w * 8 + g]);
-    if (st.m_run[hh] == kNegInf) f[hh] = 0.f;
-    else f[hh] = fast_exp2(st.m_run[hh] - mx) *
-                 (hot ? 1.f : fast_exp2(st.mp_run[hh] - st.m_run[hh]) / (float)Lr);
+    f[hh] = st.ref[hh] == kNegInf ? 0.f : fast_exp2(st.ref[hh] - mx) * (hot ? 1.f : inv_levels);
   }
   constexpr int P8 = D / 16;   // (D/2) / 8 pairs per gid for the cold mapping
+  // the 4 warps add their rows in turn: no two threads touch one word at once
+  for (int w = 0; w < 4; ++w) {
+    if (warp == w) {
 #pragma unroll
-  for (int i = 0; i < NT; ++i) {
+      for (int i = 0; i < NT; ++i) {
 #pragma unroll
-    for (int r2 = 0; r2 < 2; ++r2) {
-      const int dim = hot ? (16 * i + gid + 8 * r2) : (2 * (P8 * gid + i) + r2);
+        for (int r2 = 0; r2 < 2; ++r2) {
+          const int dim = hot ? (16 * i + gid + 8 * r2) : (2 * (P8 * gid + i) + r2);
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const int g = 2 * tig + hh;
-        if (g < G && f[hh] != 0.f) atomicAdd(&ow[g * D + dim], st.O[i][2 * r2 + hh] * f[hh]);
+          for (int hh = 0; hh < 2; ++hh) {
+            const int g = 2 * tig + hh;
+            if (g < G && f[hh] != 0.f) ow[g * D + dim] += st.O[i][2 * r2 + hh] * f[hh];
+          }
+        }
       }
     }
+    __syncthreads();
   }
-  __syncthreads();
   for (int idx = tid; idx < G * D; idx += kThreads) {
     const int g = idx / D, dim = idx % D;
     float* pp = dst + g * (D + 2);
@@ -453,36 +475,23 @@ __device__ __forceinline__ void flush_partial(WarpState<NT>& st, bool hot, int L
   __syncthreads();
 }
 
-// Lazy online softmax for one tile: the reference max moves (with a warp
-// reduction and a rescale of the sums) only when some logit exceeds it by
-// more than kLazyHeadroom, so p = exp2(l - ref) stays <= 2^8.  Returns the
-// rescale factor of the running sums (1 when nothing moved).
-__device__ __forceinline__ void lazy_softmax(const float (&l2)[4], float (&ref)[2], float (&p)[4],
-                                             float (&corr)[2]) {
-  const bool need = l2[0] > ref[0] + kLazyHeadroom || l2[1] > ref[1] + kLazyHeadroom ||
-                    l2[2] > ref[0] + kLazyHeadroom || l2[3] > ref[1] + kLazyHeadroom;
-  if (__any_sync(kFull, need)) {
-    softmax_tile(l2, ref, p, corr);
-  } else {
-    const float r0 = ref[0] == kNegInf ? 0.f : ref[0], r1 = ref[1] == kNegInf ? 0.f : ref[1];
-    p[0] = fast_exp2(l2[0] - r0);
-    p[1] = fast_exp2(l2[1] - r1);
-    p[2] = fast_exp2(l2[2] - r0);
-    p[3] = fast_exp2(l2[3] - r1);
-    corr[0] = corr[1] = 1.f;
-  }
-}
-
-template <int D, int M, int BW>
-__global__ void __launch_bounds__(kThreads, 3) attend_kernel(const AttendArgs a) {
+// PACK (groups of at most 4 query heads): the MMA's 8 columns carry
+// [q'_hi | q'_lo] of the 4 heads, so the K-logit products take 2 MMAs per
+// k-step instead of 3; lanes tig and tig ^ 2 then hold the same two heads
+// 2 * (tig & 1) + hh.  Without PACK (8 heads) lane (gid, tig) holds heads
+// 2 * tig + hh.
+template <int D, int M, int BW, bool PACK>
+__global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(const AttendArgs a) {
   using S = AttendShape<D, M, BW>;
   extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ __align__(16) uint2 klut_static[S::STATIC_LUT ? S::NLUT * 32 : 2];
-  __shared__ __align__(16) uint32_t vlut_static[S::STATIC_LUT ? S::NLUT * 32 : 4];
-  uint2* klut_w = S::STATIC_LUT ? klut_static : reinterpret_cast<uint2*>(smem);
-  uint32_t* vlut_w = S::STATIC_LUT ? vlut_static : reinterpret_cast<uint32_t*>(smem + S::OFF_VLUT);
-  const char* klut = reinterpret_cast<const char*>(klut_w);
-  const char* vlut = reinterpret_cast<const char*>(vlut_w);
+  // Separate 4-byte hi and lo tables (rather than one 8-byte entry) let
+  // each looked-up register land directly in the MMA's operand registers.
+  __shared__ __align__(16) uint32_t lhi_static[S::STATIC_LUT ? S::NLUT * 32 : 4];
+  __shared__ __align__(16) uint32_t llo_static[S::STATIC_LUT ? S::NLUT * 32 : 4];
+  uint32_t* lhi_w = S::STATIC_LUT ? lhi_static : reinterpret_cast<uint32_t*>(smem);
+  uint32_t* llo_w = S::STATIC_LUT ? llo_static : reinterpret_cast<uint32_t*>(smem + S::OFF_LO);
+  const char* lhi = reinterpret_cast<const char*>(lhi_w);
+  const char* llo = reinterpret_cast<const char*>(llo_w);
   uint8_t* ring = smem + S::OFF_RING;
   float* merge = reinterpret_cast<float*>(smem + S::OFF_MERGE);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::OFF_BAR);
@@ -494,8 +503,9 @@ __global__ void __launch_bounds__(kThreads, 3) attend_kernel(const AttendArgs a)
   const int gid = lane >> 2, tig = lane & 3;
   const int G = a.G;
   const int Lr = (1 << a.L.b_r) - 1;
+  const float inv_levels = 1.f / (float)Lr;
   const int tb = warp * 16;            // this warp's tokens inside a block / tile
-  const uint32_t lane8 = (uint32_t)lane * 8u, lane4 = (uint32_t)lane * 4u;
+  const uint32_t lane4 = (uint32_t)lane * 4u;
   const SplitPlan& pl = a.plan;
   const int slots = pl.slots_cold + pl.slots_hot;
   WarpState<S::NT> st;
@@ -550,13 +560,16 @@ __global__ void __launch_bounds__(kThreads, 3) attend_kernel(const AttendArgs a)
       __syncthreads();
       for (int i = tid; i < S::NLUT * 32; i += kThreads) {
         const uint2 e = base[i >> 5];
-        klut_w[i] = e;
-        vlut_w[i] = e.x;
+        lhi_w[i] = e.x;
+        llo_w[i] = e.y;
       }
     }
     __syncthreads();
 
-    uint32_t qfh[S::NT][2], qfl[S::NT][2], qs[S::QS][2];
+    // B operands of the K-logit MMAs (per k-step) and of the QJL MMAs.
+    //   PACK:  bq = [q'_hi | q'_lo] by column, bq2 = [q'_hi | q'_hi]
+    //   else:  bq = q'_hi, bq2 = q'_lo
+    uint32_t bq[S::NT][2], bq2[S::NT][2], qs[S::QS][2];
     float kpol[2], kqjl[2];
     int unit_cur = -1;
     int slot_cur = 0;
@@ -570,7 +583,7 @@ __global__ void __launch_bounds__(kThreads, 3) attend_kernel(const AttendArgs a)
       }
       if (unit != unit_cur) {
         if (unit_cur >= 0) {
-          flush_partial<D, S::NT>(st, false, Lr, G, merge,
+          flush_partial<D, S::NT>(st, false, inv_levels, G, merge,
                                   a.part + (((size_t)unit_cur * slots + slot_cur) * G) * (D + 2));
           st.reset();
         }
@@ -578,28 +591,31 @@ __global__ void __launch_bounds__(kThreads, 3) attend_kernel(const AttendArgs a)
         slot_cur = c - (int)(((int64_t)unit * nb) / pl.cold_bpc);
         const int b = unit / a.Hkv, kvh = unit % a.Hkv;
         const int head0 = b * a.Hq + kvh * G;
-        if (gid < G) {
-          const uint32_t* qp = reinterpret_cast<const uint32_t*>(a.qrot + (size_t)(head0 + gid) * 2 * D) + S::PT * tig;
-          const uint32_t* qk = reinterpret_cast<const uint32_t*>(a.qsk + (size_t)(head0 + gid) * M) + tig * (M / 8);
+        const int hcol = PACK ? (gid & 3) : gid;       // head of this lane's B column
+        if (hcol < G) {
+          const uint32_t* qp = reinterpret_cast<const uint32_t*>(a.qrot + (size_t)(head0 + hcol) * 2 * D) + S::PT * tig;
+          const uint32_t* qk = reinterpret_cast<const uint32_t*>(a.qsk + (size_t)(head0 + hcol) * M) + tig * (M / 8);
+          const int o1 = (PACK && gid >= 4) ? S::P : 0;
+          const int o2 = PACK ? 0 : S::P;
 #pragma unroll
           for (int s = 0; s < S::NT; ++s) {
-            qfh[s][0] = qp[2 * s];
-            qfh[s][1] = qp[2 * s + 1];
-            qfl[s][0] = qp[S::P + 2 * s];
-            qfl[s][1] = qp[S::P + 2 * s + 1];
+            bq[s][0] = qp[o1 + 2 * s];
+            bq[s][1] = qp[o1 + 2 * s + 1];
+            bq2[s][0] = qp[o2 + 2 * s];
+            bq2[s][1] = qp[o2 + 2 * s + 1];
           }
 #pragma unroll
           for (int s = 0; s < S::QS; ++s) { qs[s][0] = qk[2 * s]; qs[s][1] = qk[2 * s + 1]; }
         } else {
 #pragma unroll
-          for (int s = 0; s < S::NT; ++s) qfh[s][0] = qfh[s][1] = qfl[s][0] = qfl[s][1] = 0u;
+          for (int s = 0; s < S::NT; ++s) bq[s][0] = bq[s][1] = bq2[s][0] = bq2[s][1] = 0u;
 #pragma unroll
           for (int s = 0; s < S::QS; ++s) qs[s][0] = qs[s][1] = 0u;
         }
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
-          const int g = 2 * tig + hh;
-          kpol[hh] = g < G ? a.log2e_sigma * a.qscale[2 * (head0 + g)] / (float)Lr : 0.f;
+          const int g = (PACK ? 2 * (tig & 1) : 2 * tig) + hh;
+          kpol[hh] = g < G ? a.log2e_sigma * a.qscale[2 * (head0 + g)] * inv_levels : 0.f;
           kqjl[hh] = g < G ? a.log2e_sigma * kSqrtHalfPi / (float)M * a.qscale[2 * (head0 + g) + 1] : 0.f;
         }
       }
@@ -626,17 +642,25 @@ __global__ void __launch_bounds__(kThreads, 3) attend_kernel(const AttendArgs a)
       const uint32_t vsc = *reinterpret_cast<const uint32_t*>(tile + S::OFF_VSC + gid * 4);
 
       // ---- cold logits: polar part, (A_hi + A_lo) . (q'_hi + q'_lo) ------
-      // even / odd k-steps accumulate separately to halve the MMA chains
-      float cph[2][4] = {}, cpl[2][4] = {};
+      // k-steps accumulate round-robin into kAccSplit chains
+      float c1[kAccSplit][4] = {}, c2[kAccSplit][4] = {};
 #pragma unroll
       for (int s = 0; s < S::NT; ++s) {
-        const uint2 a0 = *reinterpret_cast<const uint2*>(klut + (field_shifted<BW, 8>(kw, (2 * s) * BW) | lane8));
-        const uint2 a1 = *reinterpret_cast<const uint2*>(klut + (field_shifted<BW, 8>(kw, (S::PT + 2 * s) * BW) | lane8));
-        const uint2 a2 = *reinterpret_cast<const uint2*>(klut + (field_shifted<BW, 8>(kw, (2 * s + 1) * BW) | lane8));
-        const uint2 a3 = *reinterpret_cast<const uint2*>(klut + (field_shifted<BW, 8>(kw, (S::PT + 2 * s + 1) * BW) | lane8));
-        mma16816(cph[s & 1], a0.x, a1.x, a2.x, a3.x, qfh[s][0], qfh[s][1]);
-        mma16816(cpl[s & 1], a0.x, a1.x, a2.x, a3.x, qfl[s][0], qfl[s][1]);
-        mma16816(cpl[s & 1], a0.y, a1.y, a2.y, a3.y, qfh[s][0], qfh[s][1]);
+        const uint32_t o0 = lut_offset<BW, 7>(kw, (2 * s) * BW, lane4);
+        const uint32_t o1 = lut_offset<BW, 7>(kw, (S::PT + 2 * s) * BW, lane4);
+        const uint32_t o2 = lut_offset<BW, 7>(kw, (2 * s + 1) * BW, lane4);
+        const uint32_t o3 = lut_offset<BW, 7>(kw, (S::PT + 2 * s + 1) * BW, lane4);
+        const uint2 a0 = make_uint2(*reinterpret_cast<const uint32_t*>(lhi + o0), *reinterpret_cast<const uint32_t*>(llo + o0));
+        const uint2 a1 = make_uint2(*reinterpret_cast<const uint32_t*>(lhi + o1), *reinterpret_cast<const uint32_t*>(llo + o1));
+        const uint2 a2 = make_uint2(*reinterpret_cast<const uint32_t*>(lhi + o2), *reinterpret_cast<const uint32_t*>(llo + o2));
+        const uint2 a3 = make_uint2(*reinterpret_cast<const uint32_t*>(lhi + o3), *reinterpret_cast<const uint32_t*>(llo + o3));
+        mma16816(c1[s % kAccSplit], a0.x, a1.x, a2.x, a3.x, bq[s][0], bq[s][1]);
+        if constexpr (PACK) {
+          mma16816(c2[s % kAccSplit], a0.y, a1.y, a2.y, a3.y, bq2[s][0], bq2[s][1]);
+        } else {
+          mma16816(c2[s % kAccSplit], a0.x, a1.x, a2.x, a3.x, bq2[s][0], bq2[s][1]);
+          mma16816(c2[s % kAccSplit], a0.y, a1.y, a2.y, a3.y, bq[s][0], bq[s][1]);
+        }
       }
       // ---- cold logits: QJL part ---------------------------------------
       uint32_t x0, x1;
@@ -661,41 +685,37 @@ __global__ void __launch_bounds__(kThreads, 3) attend_kernel(const AttendArgs a)
       const float sk1 = __half2float(__ushort_as_half((unsigned short)(ksc.x >> 16)));
       const float rn0 = __half2float(__ushort_as_half((unsigned short)(ksc.y & 0xffffu)));
       const float rn1 = __half2float(__ushort_as_half((unsigned short)(ksc.y >> 16)));
-      float l2[4];
       float cp[4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) cp[j] = (cph[0][j] + cph[1][j]) + (cpl[0][j] + cpl[1][j]);
+      for (int j = 0; j < 4; ++j) {
+        float h1 = c1[0][j], h2 = c2[0][j];
+#pragma unroll
+        for (int k = 1; k < kAccSplit; ++k) {
+          h1 += c1[k][j];
+          h2 += c2[k][j];
+        }
+        cp[j] = (PACK ? h1 + __shfl_xor_sync(kFull, h1, 2) : h1) + h2;
+      }
+      float l2[4];
       l2[0] = v0 ? fmaf(rn0 * kqjl[0], cq0[0] + cq1[0], sk0 * kpol[0] * cp[0]) : kNegInf;
       l2[1] = v0 ? fmaf(rn0 * kqjl[1], cq0[1] + cq1[1], sk0 * kpol[1] * cp[1]) : kNegInf;
       l2[2] = v1 ? fmaf(rn1 * kqjl[0], cq0[2] + cq1[2], sk1 * kpol[0] * cp[2]) : kNegInf;
       l2[3] = v1 ? fmaf(rn1 * kqjl[1], cq0[3] + cq1[3], sk1 * kpol[1] * cp[3]) : kNegInf;
-      float p[4], corr[2];
-      lazy_softmax(l2, st.m_run, p, corr);
-      st.l_run[0] = st.l_run[0] * corr[0] + p[0] + p[2];
-      st.l_run[1] = st.l_run[1] * corr[1] + p[1] + p[3];
-
-      // ---- V weights p * s16_v, on their own lazy reference ---------------
-      const float lv0 = v0 ? fast_log2(__half2float(__ushort_as_half((unsigned short)(vsc & 0xffffu)))) : kNegInf;
-      const float lv1 = v1 ? fast_log2(__half2float(__ushort_as_half((unsigned short)(vsc >> 16)))) : kNegInf;
-      const float xv[4] = {l2[0] + lv0, l2[1] + lv0, l2[2] + lv1, l2[3] + lv1};
-      float pv[4], co[2];
-      lazy_softmax(xv, st.mp_run, pv, co);
-      if (co[0] != 1.f || co[1] != 1.f) {
-#pragma unroll
-        for (int j = 0; j < S::NT; ++j) {
-          st.O[j][0] *= co[0]; st.O[j][1] *= co[1]; st.O[j][2] *= co[0]; st.O[j][3] *= co[1];
-        }
-      }
+      // V weights of tokens past the end are 0 (their records are not written)
+      const float sv0 = v0 ? __half2float(__ushort_as_half((unsigned short)(vsc & 0xffffu))) : 0.f;
+      const float sv1 = v1 ? __half2float(__ushort_as_half((unsigned short)(vsc >> 16))) : 0.f;
+      float pv[4];
+      softmax_step(st, l2, sv0, sv1, pv);
       const uint32_t pb0 = movmatrix_trans(pack_h2(pv[0], pv[1]));
       const uint32_t pb1 = movmatrix_trans(pack_h2(pv[2], pv[3]));
 
       // ---- P V: V codes of pairs PV*gid + j for tokens 2tig, 2tig+1, +8, +9
 #pragma unroll
       for (int j = 0; j < S::NT; ++j) {
-        const uint32_t L0 = *reinterpret_cast<const uint32_t*>(vlut + (field_shifted<BW, 7>(vw, (0 * S::PV + j) * BW) | lane4));
-        const uint32_t L1 = *reinterpret_cast<const uint32_t*>(vlut + (field_shifted<BW, 7>(vw, (1 * S::PV + j) * BW) | lane4));
-        const uint32_t L2 = *reinterpret_cast<const uint32_t*>(vlut + (field_shifted<BW, 7>(vw, (2 * S::PV + j) * BW) | lane4));
-        const uint32_t L3 = *reinterpret_cast<const uint32_t*>(vlut + (field_shifted<BW, 7>(vw, (3 * S::PV + j) * BW) | lane4));
+        const uint32_t L0 = *reinterpret_cast<const uint32_t*>(lhi + lut_offset<BW, 7>(vw, (0 * S::PV + j) * BW, lane4));
+        const uint32_t L1 = *reinterpret_cast<const uint32_t*>(lhi + lut_offset<BW, 7>(vw, (1 * S::PV + j) * BW, lane4));
+        const uint32_t L2 = *reinterpret_cast<const uint32_t*>(lhi + lut_offset<BW, 7>(vw, (2 * S::PV + j) * BW, lane4));
+        const uint32_t L3 = *reinterpret_cast<const uint32_t*>(lhi + lut_offset<BW, 7>(vw, (3 * S::PV + j) * BW, lane4));
         mma16816(st.O[j], __byte_perm(L0, L1, 0x5410), __byte_perm(L0, L1, 0x7632),
                  __byte_perm(L2, L3, 0x5410), __byte_perm(L2, L3, 0x7632), pb0, pb1);
       }
@@ -730,9 +750,12 @@ __global__ void __launch_bounds__(kThreads, 3) attend_kernel(const AttendArgs a)
       }
       return;
     }
-    if (unit_cur >= 0)
-      flush_partial<D, S::NT>(st, false, Lr, G, merge,
+    // with PACK, lanes tig >= 2 duplicate the heads of lanes tig - 2;
+    // flush_partial keeps head 2 * tig + hh < G <= 4 only, i.e. tig < 2
+    if (unit_cur >= 0) {
+      flush_partial<D, S::NT>(st, false, inv_levels, G, merge,
                               a.part + (((size_t)unit_cur * slots + slot_cur) * G) * (D + 2));
+    }
   } else {
     // ======================= hot CTA =======================
     const int c = blockIdx.x - pl.cold_ctas;
@@ -752,7 +775,7 @@ __global__ void __launch_bounds__(kThreads, 3) attend_kernel(const AttendArgs a)
       }
       if (unit != unit_cur) {
         if (unit_cur >= 0) {
-          flush_partial<D, S::NT>(st, true, Lr, G, merge,
+          flush_partial<D, S::NT>(st, true, inv_levels, G, merge,
                                   a.part + (((size_t)unit_cur * slots + slot_cur) * G) * (D + 2));
           st.reset();
         }
@@ -772,60 +795,57 @@ __global__ void __launch_bounds__(kThreads, 3) attend_kernel(const AttendArgs a)
           for (int s = 0; s < S::NT; ++s) qh[s][0] = qh[s][1] = 0u;
         }
       }
-      __syncthreads();
-      for (int i = tid; i < 2 * S::TB * CH; i += kThreads) {
-        const int kv = i / (S::TB * CH);
-        const int rem = i % (S::TB * CH);
-        const int r = rem / CH, cc = rem % CH;
-        const int slot = tile * S::TB + r;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (slot < a.n_hot)
-          v = __ldg(reinterpret_cast<const uint4*>((kv ? a.hot_v : a.hot_k) + ((size_t)unit * a.W + slot) * D) + cc);
-        *reinterpret_cast<uint4*>(ring + kv * S::TB * S::RS + r * S::RS + cc * 16) = v;
-      }
-      __syncthreads();
+      // the tile's K rows, then (in the same buffer) its V rows
+      auto stage_rows = [&](const __half* src) {
+        __syncthreads();
+        for (int i = tid; i < S::TB * CH; i += kThreads) {
+          const int r = i / CH, cc = i % CH;
+          const int slot = tile * S::TB + r;
+          uint4 v = make_uint4(0u, 0u, 0u, 0u);
+          if (slot < a.n_hot)
+            v = __ldg(reinterpret_cast<const uint4*>(src + ((size_t)unit * a.W + slot) * D) + cc);
+          *reinterpret_cast<uint4*>(ring + r * S::RS + cc * 16) = v;
+        }
+        __syncthreads();
+      };
       const int nvalid = a.n_hot - tile * S::TB < S::TB ? a.n_hot - tile * S::TB : S::TB;
-      if (tb >= nvalid) continue;
-      const uint32_t kbase = smem_addr(ring);
-      const uint32_t vbase = kbase + S::TB * S::RS;
+      const bool live = tb < nvalid;
+      const uint32_t base = smem_addr(ring);
       const int mi = lane >> 3, rr = lane & 7;
-      float cc4[4] = {0.f, 0.f, 0.f, 0.f};
+      stage_rows(a.hot_k);
+      uint32_t pb0 = 0u, pb1 = 0u;
+      if (live) {
+        float cc4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int s = 0; s < S::NT; ++s) {
-        uint32_t af[4];
-        ldsm_x4(af, kbase + (tb + rr + (mi & 1) * 8) * S::RS + (16 * s + (mi >> 1) * 8) * 2);
-        mma16816(cc4, af[0], af[1], af[2], af[3], qh[s][0], qh[s][1]);
+        for (int s = 0; s < S::NT; ++s) {
+          uint32_t af[4];
+          ldsm_x4(af, base + (tb + rr + (mi & 1) * 8) * S::RS + (16 * s + (mi >> 1) * 8) * 2);
+          mma16816(cc4, af[0], af[1], af[2], af[3], qh[s][0], qh[s][1]);
+        }
+        const bool v0 = tb + gid < nvalid, v1 = tb + gid + 8 < nvalid;
+        float l2[4];
+        l2[0] = v0 ? a.log2e_sigma * cc4[0] : kNegInf;
+        l2[1] = v0 ? a.log2e_sigma * cc4[1] : kNegInf;
+        l2[2] = v1 ? a.log2e_sigma * cc4[2] : kNegInf;
+        l2[3] = v1 ? a.log2e_sigma * cc4[3] : kNegInf;
+        float pv[4];
+        softmax_step(st, l2, 1.f, 1.f, pv);
+        pb0 = movmatrix_trans(pack_h2(pv[0], pv[1]));
+        pb1 = movmatrix_trans(pack_h2(pv[2], pv[3]));
       }
-      const bool v0 = tb + gid < nvalid, v1 = tb + gid + 8 < nvalid;
-      float l2[4];
-      l2[0] = v0 ? a.log2e_sigma * cc4[0] : kNegInf;
-      l2[1] = v0 ? a.log2e_sigma * cc4[1] : kNegInf;
-      l2[2] = v1 ? a.log2e_sigma * cc4[2] : kNegInf;
-      l2[3] = v1 ? a.log2e_sigma * cc4[3] : kNegInf;
-      float p[4], corr[2];
-      softmax_tile(l2, st.m_run, p, corr);
-      st.l_run[0] = st.l_run[0] * corr[0] + p[0] + p[2];
-      st.l_run[1] = st.l_run[1] * corr[1] + p[1] + p[3];
-      if (__any_sync(kFull, corr[0] != 1.f || corr[1] != 1.f)) {
+      stage_rows(a.hot_v);
+      if (live) {
 #pragma unroll
         for (int j = 0; j < S::NT; ++j) {
-          st.O[j][0] *= corr[0]; st.O[j][1] *= corr[1]; st.O[j][2] *= corr[0]; st.O[j][3] *= corr[1];
+          uint32_t af[4];
+          ldsm_x4_trans(af, base + (tb + rr + (mi >> 1) * 8) * S::RS + (16 * j + (mi & 1) * 8) * 2);
+          mma16816(st.O[j], af[0], af[1], af[2], af[3], pb0, pb1);
         }
       }
-      const uint32_t pb0 = movmatrix_trans(pack_h2(p[0], p[1]));
-      const uint32_t pb1 = movmatrix_trans(pack_h2(p[2], p[3]));
-#pragma unroll
-      for (int j = 0; j < S::NT; ++j) {
-        uint32_t af[4];
-        ldsm_x4_trans(af, vbase + (tb + rr + (mi >> 1) * 8) * S::RS + (16 * j + (mi & 1) * 8) * 2);
-        mma16816(st.O[j], af[0], af[1], af[2], af[3], pb0, pb1);
-      }
     }
-    st.mp_run[0] = st.m_run[0];
-    st.mp_run[1] = st.m_run[1];
     if (unit_cur >= 0) {
       __syncthreads();
-      flush_partial<D, S::NT>(st, true, Lr, G, merge,
+      flush_partial<D, S::NT>(st, true, inv_levels, G, merge,
                               a.part + (((size_t)unit_cur * slots + slot_cur) * G) * (D + 2));
     }
   }
@@ -834,13 +854,22 @@ __global__ void __launch_bounds__(kThreads, 3) attend_kernel(const AttendArgs a)
 // ---------------------------------------------------------------------------
 // combine
 // ---------------------------------------------------------------------------
+// One block per query head, one thread per output dimension.  The split
+// records' (m, l) pairs are read once by as many threads, so every global
+// load of the block is independent of the others; R^T is applied to the
+// cold sum with butterflies in registers (shuffles) and, for strides of a
+// warp or more, through shared memory.
+constexpr int kCombineMaxSlots = 128;
+
 __global__ void combine_kernel(const CombineArgs a) {
-  __shared__ float buf[256];
+  __shared__ float sw[kCombineMaxSlots];     // per-slot weight 2^(m_s - m)
+  __shared__ float red[2][8];
+  __shared__ float xbuf[256];
   const int hg = blockIdx.x;
   const int b = hg / a.Hq, hq = hg % a.Hq;
   const int kvh = hq / a.G, g = hq % a.G;
   const int unit = b * a.Hkv + kvh;
-  const int D = a.d, t = threadIdx.x;
+  const int D = a.d, t = threadIdx.x, lane = t & 31, warp = t >> 5, nw = blockDim.x >> 5;
   const SplitPlan& pl = a.plan;
   const int slots = pl.slots_cold + pl.slots_hot;
   const float* base = a.part + (size_t)unit * slots * a.G * (D + 2);
@@ -853,31 +882,71 @@ __global__ void combine_kernel(const CombineArgs a) {
     const int64_t ht = pl.hot_tiles;
     nh = (int)(((unit + 1) * ht - 1) / pl.hot_tpc - (unit * ht) / pl.hot_tpc + 1);
   }
-  auto rec = [&](int s) { return base + ((size_t)s * a.G + g) * (D + 2); };
+  const int ns = nc + nh;
+  auto rec = [&](int s) {
+    return base + ((size_t)(s < nc ? s : pl.slots_cold + (s - nc)) * a.G + g) * (D + 2);
+  };
+  // ---- m = max over slots, then w_s and l = sum w_s l_s ----------------------
+  float ms[kCombineMaxSlots / 64], ls[kCombineMaxSlots / 64];
   float mx = kNegInf;
-  for (int s = 0; s < nc; ++s) mx = fmaxf(mx, rec(s)[0]);
-  for (int s = 0; s < nh; ++s) mx = fmaxf(mx, rec(pl.slots_cold + s)[0]);
-  float lsum = 0.f, oc = 0.f, oh = 0.f;
-  if (mx != kNegInf) {
-    for (int s = 0; s < nc + nh; ++s) {
-      const float* pp = rec(s < nc ? s : pl.slots_cold + (s - nc));
-      if (pp[0] == kNegInf) continue;
-      const float w = exp2f(pp[0] - mx);
-      lsum += w * pp[1];
-      const float v = w * pp[2 + t];
-      if (s < nc) oc += v; else oh += v;
+#pragma unroll
+  for (int k = 0; k < kCombineMaxSlots / 64; ++k) {
+    const int s = t + k * blockDim.x;
+    ms[k] = kNegInf;
+    ls[k] = 0.f;
+    if (s < ns) {
+      const float* pp = rec(s);
+      ms[k] = pp[0];
+      ls[k] = pp[1];
+    }
+    mx = fmaxf(mx, ms[k]);
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, o));
+  if (lane == 0) red[0][warp] = mx;
+  __syncthreads();
+  mx = red[0][0];
+  for (int w = 1; w < nw; ++w) mx = fmaxf(mx, red[0][w]);
+  float lsum = 0.f;
+#pragma unroll
+  for (int k = 0; k < kCombineMaxSlots / 64; ++k) {
+    const int s = t + k * blockDim.x;
+    if (s < ns) {
+      const float w = ms[k] == kNegInf ? 0.f : exp2f(ms[k] - mx);
+      sw[s] = w;
+      lsum += w * ls[k];
     }
   }
-  buf[t] = oc;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) lsum += __shfl_xor_sync(kFull, lsum, o);
+  if (lane == 0) red[1][warp] = lsum;
   __syncthreads();
-  for (int h = 1; h < D; h <<= 1) {
-    const float x = buf[t], y = buf[t ^ h];
+  lsum = 0.f;
+  for (int w = 0; w < nw; ++w) lsum += red[1][w];
+  // ---- weighted sums of the o vectors (independent loads) --------------------
+  float oc = 0.f, oh = 0.f;
+  if (mx != kNegInf) {
+#pragma unroll 8
+    for (int s = 0; s < nc; ++s) oc += sw[s] * rec(s)[2 + t];
+#pragma unroll 4
+    for (int s = nc; s < ns; ++s) oh += sw[s] * rec(s)[2 + t];
+  }
+  // ---- R^T on the cold sum: unnormalised Hadamard, then signs / sqrt(d) ------
+  float x = oc;
+#pragma unroll
+  for (int h = 1; h < 32; h <<= 1) {
+    const float o = __shfl_xor_sync(kFull, x, h);
+    x = (t & h) ? (o - x) : (x + o);
+  }
+  for (int h = 32; h < D; h <<= 1) {
+    xbuf[t] = x;
     __syncthreads();
-    buf[t] = (t & h) ? (y - x) : (x + y);
+    const float o = xbuf[t ^ h];
     __syncthreads();
+    x = (t & h) ? (o - x) : (x + o);
   }
   const float res = mx == kNegInf ? 0.f
-                                  : (oh + (float)a.signs[t] * buf[t] * rsqrtf((float)D)) / lsum;
+                                  : (oh + (float)a.signs[t] * x * rsqrtf((float)D)) / lsum;
   a.out[(size_t)hg * D + t] = res;
 }
 
@@ -887,38 +956,40 @@ __global__ void combine_kernel(const CombineArgs a) {
 typedef void (*AttendFn)(const AttendArgs);
 
 template <int D, int M, int BW>
-AttendFn attend_fn(int* smem) {
+AttendFn attend_fn(bool pack, int* smem) {
   *smem = AttendShape<D, M, BW>::SMEM;
-  return attend_kernel<D, M, BW>;
+  return pack ? attend_kernel<D, M, BW, true> : attend_kernel<D, M, BW, false>;
 }
 
 template <int D, int M>
-AttendFn pick_bw(int bw, int* smem) {
+AttendFn pick_bw(int bw, bool pack, int* smem) {
   switch (bw) {
-    case 2: return attend_fn<D, M, 2>(smem);
-    case 3: return attend_fn<D, M, 3>(smem);
-    case 4: return attend_fn<D, M, 4>(smem);
-    case 5: return attend_fn<D, M, 5>(smem);
-    case 6: return attend_fn<D, M, 6>(smem);
-    case 7: return attend_fn<D, M, 7>(smem);
-    case 8: return attend_fn<D, M, 8>(smem);
+    case 2: return attend_fn<D, M, 2>(pack, smem);
+    case 3: return attend_fn<D, M, 3>(pack, smem);
+    case 4: return attend_fn<D, M, 4>(pack, smem);
+    case 5: return attend_fn<D, M, 5>(pack, smem);
+    case 6: return attend_fn<D, M, 6>(pack, smem);
+    case 7: return attend_fn<D, M, 7>(pack, smem);
+    case 8: return attend_fn<D, M, 8>(pack, smem);
   }
   return nullptr;
 }
 
-AttendFn pick_attend(const Layout& L, int* smem) {
-  if (L.d == 64 && L.m == 64) return pick_bw<64, 64>(L.bw, smem);
-  if (L.d == 64 && L.m == 128) return pick_bw<64, 128>(L.bw, smem);
-  if (L.d == 128 && L.m == 64) return pick_bw<128, 64>(L.bw, smem);
-  if (L.d == 128 && L.m == 128) return pick_bw<128, 128>(L.bw, smem);
+// groups of up to 4 query heads use the packed [q'_hi | q'_lo] columns
+AttendFn pick_attend(const Layout& L, int G, int* smem) {
+  const bool pack = G <= 4;
+  if (L.d == 64 && L.m == 64) return pick_bw<64, 64>(L.bw, pack, smem);
+  if (L.d == 64 && L.m == 128) return pick_bw<64, 128>(L.bw, pack, smem);
+  if (L.d == 128 && L.m == 64) return pick_bw<128, 64>(L.bw, pack, smem);
+  if (L.d == 128 && L.m == 128) return pick_bw<128, 128>(L.bw, pack, smem);
   return nullptr;
 }
 
 }  // namespace
 
-int attend_ctas_per_sm(const Layout& L) {
+int attend_ctas_per_sm(const Layout& L, int G) {
   int smem = 0;
-  AttendFn fn = pick_attend(L, &smem);
+  AttendFn fn = pick_attend(L, G, &smem);
   if (!fn) return 0;
   if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return 0;
@@ -927,19 +998,30 @@ int attend_ctas_per_sm(const Layout& L) {
   return n;
 }
 
-cudaError_t launch_qprep(const QPrepArgs& a, cudaStream_t s) {
-  const int grid = (a.heads + 7) / 8;
-  if (a.d == 64 && a.m == 64) qprep_kernel<64, 64><<<grid, 256, 0, s>>>(a);
-  else if (a.d == 64 && a.m == 128) qprep_kernel<64, 128><<<grid, 256, 0, s>>>(a);
-  else if (a.d == 128 && a.m == 64) qprep_kernel<128, 64><<<grid, 256, 0, s>>>(a);
-  else if (a.d == 128 && a.m == 128) qprep_kernel<128, 128><<<grid, 256, 0, s>>>(a);
-  else return cudaErrorInvalidValue;
+template <int D, int M>
+cudaError_t launch_qprep_dm(const QPrepArgs& a, cudaStream_t s) {
+  const int grid = (a.heads + 256 / M - 1) / (256 / M);
+  constexpr int smem = D * M * 4;
+  if (smem > 48 * 1024) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(qprep_kernel<D, M>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+  }
+  qprep_kernel<D, M><<<grid, 256, smem, s>>>(a);
   return cudaGetLastError();
+}
+
+cudaError_t launch_qprep(const QPrepArgs& a, cudaStream_t s) {
+  if (a.d == 64 && a.m == 64) return launch_qprep_dm<64, 64>(a, s);
+  if (a.d == 64 && a.m == 128) return launch_qprep_dm<64, 128>(a, s);
+  if (a.d == 128 && a.m == 64) return launch_qprep_dm<128, 64>(a, s);
+  if (a.d == 128 && a.m == 128) return launch_qprep_dm<128, 128>(a, s);
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_attend(const AttendArgs& a, cudaStream_t s) {
   int smem = 0;
-  AttendFn fn = pick_attend(a.L, &smem);
+  AttendFn fn = pick_attend(a.L, a.G, &smem);
   if (!fn) return cudaErrorInvalidValue;
   const int grid = a.plan.cold_ctas + a.plan.hot_ctas;
   if (grid == 0) return cudaSuccess;

@@ -21,11 +21,29 @@ namespace {
 
 using namespace enc;
 
+constexpr int kStStageBytes = 64 * 1024;   // largest S^T staged in shared memory
+
+__host__ __device__ constexpr bool st_staged(int d, int m) { return d * m * 4 <= kStStageBytes; }
+
+// Per-block shared memory: [warps][D] doubles (residuals), per-warp code /
+// sign / scalar staging, then S^T when staged (16-byte aligned).
+__host__ __device__ constexpr size_t st_offset(int d, int warps) {
+  return ((size_t)warps * d * sizeof(double) + (size_t)warps * (8 * (d / 2) + 4 * 32 + 32) + 15) /
+         16 * 16;
+}
+
+// encode_small_kernel's shared memory: [2][D] doubles, [2][D/32] doubles,
+// [2][D/2] code bytes, 4 sign words, 3 scalars; then S^T (16-byte aligned).
+__host__ __device__ constexpr size_t small_st_offset(int d) {
+  return ((size_t)2 * d * 8 + (size_t)2 * (d / 32) * 8 + (size_t)d + 16 + 8 + 15) / 16 * 16;
+}
+
 template <int D>
-__device__ __forceinline__ void encode_vector(const EncodeArgs& a, const __half* src, bool is_key,
+__device__ __forceinline__ void encode_vector(const EncodeArgs& a, const float* St,
+                                              const __half* src, bool is_key,
                                               double* rbuf, uint8_t* codes, uint32_t* bits,
                                               uint16_t* s16_out, uint16_t* rn16_out) {
-  encode_vector_any<D>(a.L, a.signs, a.St, a.inv_sqrt_d, a.status,
+  encode_vector_any<D>(a.L, a.signs, St, a.inv_sqrt_d, a.status,
                        [&](int lane, double (&x)[D / 32]) { load_vec<D / 32>(src, lane, x); },
                        is_key, rbuf, codes, bits, s16_out, rn16_out);
 }
@@ -85,6 +103,18 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
   const int bw = L.bw;
   const int64_t n = (int64_t)a.nA + a.nB;
   if (n == 0) return;
+  // S^T in shared memory when it fits: the sign loop then waits on shared
+  // memory instead of a chain of L2 round trips (the decode-step eviction
+  // encodes one token per unit, so latency is all there is).
+  const float* St = a.St;
+  if (st_staged(D, L.m)) {
+    float* sst = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(smem) + st_offset(D, warps));
+    const int n16 = D * L.m / 4;
+    for (int i = threadIdx.x; i < n16; i += blockDim.x)
+      reinterpret_cast<float4*>(sst)[i] = __ldg(reinterpret_cast<const float4*>(a.St) + i);
+    __syncthreads();
+    St = sst;
+  }
   const int64_t t_first = a.cold_start / kTokensPerTile;
   const int64_t t_last = (a.cold_start + n - 1) / kTokensPerTile;
   const int64_t groups = (t_last - t_first + 1) * 4;
@@ -121,8 +151,8 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
         ksrc = a.src_k + ((int64_t)unit * a.src_tokens + (e - a.nA)) * D;
         vsrc = a.src_v + ((int64_t)unit * a.src_tokens + (e - a.nA)) * D;
       }
-      encode_vector<D>(a, ksrc, true, rbuf, kc + s * P, kb + s * 8, sc + s * 4, sc + s * 4 + 1);
-      encode_vector<D>(a, vsrc, false, rbuf, vc + s * P, nullptr, sc + s * 4 + 2, nullptr);
+      encode_vector<D>(a, St, ksrc, true, rbuf, kc + s * P, kb + s * 8, sc + s * 4, sc + s * 4 + 1);
+      encode_vector<D>(a, St, vsrc, false, rbuf, vc + s * P, nullptr, sc + s * 4 + 2, nullptr);
     }
     __syncwarp();
 
@@ -189,6 +219,192 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
   }
 }
 
+// Latency path for a few tokens per unit (the decode-step eviction): one
+// CTA per (unit, token); threads [0, D) encode the key with one element per
+// thread, threads [D, 2D) the value.  The float64 operations are those of
+// encode_vector_any (the polar and residual steps run on one thread per
+// pair, in parallel instead of PL pairs in turn per lane), so the codes
+// match the float64 definition the same way.  The token's fields are merged
+// into the fragment-major words with atomicAnd / atomicOr: CTAs writing
+// other tokens of the same words never lose each other's bits.
+template <int D>
+__global__ void __launch_bounds__(2 * D) encode_small_kernel(EncodeArgs a) {
+  constexpr int P = D / 2;
+  constexpr int NW = D / 32;                 // warps per team
+  const Layout& L = a.L;
+  const int64_t n = (int64_t)a.nA + a.nB;
+  const int unit = (int)(blockIdx.x / n);
+  const int64_t e = blockIdx.x % n;
+  const int tid = threadIdx.x, team = tid / D, el = tid % D;
+  const int lane = tid & 31, wt = el >> 5;
+  extern __shared__ double sm[];
+  double* xb = sm + team * D;                                  // [2][D] exchange / residual
+  double* red = sm + 2 * D;                                    // [2][NW] reductions
+  uint8_t* codes = reinterpret_cast<uint8_t*>(red + 2 * NW);   // [2][P] key / value codes
+  uint32_t* bits = reinterpret_cast<uint32_t*>(codes + 2 * P); // [4] key sign words
+  uint16_t* sc = reinterpret_cast<uint16_t*>(bits + 4);        // s16_k, rn16, s16_v
+  float* sst = reinterpret_cast<float*>(sm) + small_st_offset(D) / 4;   // S^T [D][m]
+  for (int i = tid; i < D * L.m / 4; i += blockDim.x)
+    reinterpret_cast<float4*>(sst)[i] = __ldg(reinterpret_cast<const float4*>(a.St) + i);
+
+  const __half* src;
+  if (e < a.nA) {
+    const int slot = (int)((a.ring_start + e) % a.W);
+    src = (team ? a.ring_v : a.ring_k) + ((int64_t)unit * a.W + slot) * D;
+  } else {
+    src = (team ? a.src_v : a.src_k) + ((int64_t)unit * a.src_tokens + (e - a.nA)) * D;
+  }
+  // ---- rotation: y = H (D x) / sqrt(d) ----------------------------------
+  double x = __dmul_rn((double)__half2float(src[el]), a.signs[el]);
+#pragma unroll
+  for (int h = 1; h < D; h <<= 1) {
+    double o;
+    if (h < 32) {
+      o = __shfl_xor_sync(kFull, x, h);
+    } else {
+      xb[el] = x;
+      __syncthreads();
+      o = xb[el ^ h];
+      __syncthreads();
+    }
+    x = (el & h) ? __dsub_rn(o, x) : __dadd_rn(x, o);
+  }
+  x = __dmul_rn(x, a.inv_sqrt_d);
+
+  // ---- polar (even threads own pair el / 2) -------------------------------
+  const double y1 = __shfl_xor_sync(kFull, x, 1);
+  const bool ev = !(el & 1);
+  double rho = 0.0, th = 0.0;
+  if (ev) {
+    rho = __dsqrt_rn(__dadd_rn(__dmul_rn(x, x), __dmul_rn(y1, y1)));
+    th = atan2(y1, x);
+  }
+  double mr = rho;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) mr = fmax(mr, __shfl_xor_sync(kFull, mr, o));
+  if (lane == 0) red[team * NW + wt] = mr;
+  __syncthreads();
+  double smax = red[team * NW];
+#pragma unroll
+  for (int w = 1; w < NW; ++w) smax = fmax(smax, red[team * NW + w]);
+  uint16_t s16b = f64_to_f16_bits(smax);
+  if ((s16b & 0x7c00u) == 0x7c00u) {
+    if (el == 0) atomicOr(a.status, kStatusRange);
+    s16b = 0;
+  }
+  const double s16 = f16_bits_to_f64(s16b);
+  const bool zero = (s16 == 0.0);
+  const int Lr = (1 << L.b_r) - 1, nt = 1 << L.b_theta;
+  int cr = 0, ct = 0;
+  if (ev) {
+    const double tr = __dmul_rn(__ddiv_rn(rho, zero ? 1.0 : s16), (double)Lr);
+    const int c = (int)rint(tr);
+    cr = c < 0 ? 0 : (c > Lr ? Lr : c);
+    const double tt = __ddiv_rn(__dmul_rn(th, (double)nt), kTwoPi);
+    ct = ((int)rint(tt)) & (nt - 1);
+    if (zero) { cr = 0; ct = 0; }
+    codes[team * P + el / 2] = (uint8_t)((cr << L.b_theta) | ct);
+  }
+  if (el == 0) sc[team ? 2 : 0] = s16b;
+
+  // ---- keys: residual, its norm and the QJL signs --------------------------
+  double ss = 0.0;
+  if (team == 0 && ev) {
+    const double rh = __ddiv_rn(__dmul_rn((double)cr, s16), (double)Lr);
+    const double ang = __ddiv_rn(__dmul_rn((double)ct, kTwoPi), (double)nt);
+    double sn, cs;
+    sincos(ang, &sn, &cs);
+    const double r0 = __dsub_rn(x, __dmul_rn(rh, cs));
+    const double r1 = __dsub_rn(y1, __dmul_rn(rh, sn));
+    xb[el] = r0;
+    xb[el + 1] = r1;
+    ss = __dadd_rn(__dmul_rn(r0, r0), __dmul_rn(r1, r1));
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) ss = __dadd_rn(ss, __shfl_xor_sync(kFull, ss, o));
+  __syncthreads();            // residual complete, S^T staged, reduction slots free
+  if (team == 0) {
+    if (lane == 0) red[wt] = ss;
+  }
+  __syncthreads();
+  if (team == 0) {
+    if (el == 0) {
+      double tot = red[0];
+      for (int w = 1; w < NW; ++w) tot = __dadd_rn(tot, red[w]);
+      const uint16_t rnb = f64_to_f16_bits(__dsqrt_rn(tot));
+      if ((rnb & 0x7c00u) == 0x7c00u) atomicOr(a.status, kStatusRange);
+      sc[1] = rnb;
+    }
+    for (int i0 = 0; i0 < L.m; i0 += D) {
+      const int i = i0 + el;
+      double acc = 0.0;
+      if (i < L.m) {
+#pragma unroll 8
+        for (int j = 0; j < D; ++j) acc = fma((double)sst[j * L.m + i], xb[j], acc);
+      }
+      const unsigned word = __ballot_sync(kFull, i < L.m && acc >= 0.0);
+      if (lane == 0 && i < L.m) bits[i >> 5] = word;
+    }
+  }
+  __syncthreads();
+
+  // ---- merge the token's fields into its tile ------------------------------
+  const int64_t tok = a.cold_start + e;
+  const int64_t tile = tok / kTokensPerTile;
+  const int r = (int)(tok % kTokensPerTile), gid = r % 8, h = r / 8;
+  uint8_t* tb = a.cold + ((int64_t)unit * L.blocks_per_unit + tile / kTilesPerBlock) * L.block_bytes +
+                (tile % kTilesPerBlock) * L.tile_bytes;
+  auto merge_atomic = [](uint8_t* addr, uint32_t val, uint32_t mask) {
+    if (mask == 0u) return;
+    uint32_t* w = reinterpret_cast<uint32_t*>(addr);
+    atomicAnd(w, ~mask);
+    atomicOr(w, val & mask);
+  };
+  const int bw = L.bw;
+  // K code words: lanes (gid, tig), codes q of half h: pair tig * pt + q % pt
+  for (int q = tid; q < 4 * L.kwt; q += blockDim.x) {
+    const int tg = q / L.kwt, w = q % L.kwt;
+    uint32_t val, mask;
+    chunk_word(w, 2 * L.pt, bw, [&](int qi, uint32_t* out) {
+      if (qi / L.pt != h) return false;
+      *out = codes[tg * L.pt + qi % L.pt];
+      return true;
+    }, val, mask);
+    merge_atomic(tb + L.off_kc + lane_word_offset(w, 4 * gid + tg, L.kwt), val, mask);
+  }
+  // V code words: lanes (gv, c = gid / 2), codes q of slot s: pair gv * pv + q % pv
+  const int cgrp = gid >> 1, slot_v = (gid & 1) + 2 * h;
+  for (int q = tid; q < 8 * L.vwt; q += blockDim.x) {
+    const int gv = q / L.vwt, w = q % L.vwt;
+    uint32_t val, mask;
+    chunk_word(w, 4 * L.pv, bw, [&](int qi, uint32_t* out) {
+      if (qi / L.pv != slot_v) return false;
+      *out = codes[P + gv * L.pv + qi % L.pv];
+      return true;
+    }, val, mask);
+    merge_atomic(tb + L.off_vc + lane_word_offset(w, 4 * gv + cgrp, L.vwt), val, mask);
+  }
+  // sign words: lanes (gid, tig); m/4 bits per (token, tig), in one word
+  const int qb = L.m / 4;
+  for (int q = tid; q < 4 * L.sw; q += blockDim.x) {
+    const int tg = q / L.sw, w = q % L.sw;
+    const int bit0 = h * qb - 32 * w;
+    if (bit0 >= 32 || bit0 + qb <= 0) continue;
+    const int i0 = tg * qb;
+    const uint32_t srcw = bits[i0 >> 5] >> (i0 & 31);
+    const uint32_t m32 = qb == 32 ? 0xffffffffu : ((1u << qb) - 1u);
+    merge_atomic(tb + L.off_ks + lane_word_offset(w, 4 * gid + tg, L.sw), (srcw & m32) << bit0,
+                 m32 << bit0);
+  }
+  if (tid == 0) {
+    uint16_t* ks = reinterpret_cast<uint16_t*>(tb + L.off_ksc);
+    uint16_t* vs = reinterpret_cast<uint16_t*>(tb + L.off_vsc);
+    ks[gid * 4 + h] = sc[0];
+    ks[gid * 4 + 2 + h] = sc[1];
+    vs[gid * 2 + h] = sc[2];
+  }
+}
+
 __global__ void ring_write_kernel(__half* ring_k, __half* ring_v, const __half* k_new,
                                   const __half* v_new, int units, int W, int d, int n,
                                   int first, int ring_pos) {
@@ -210,11 +426,23 @@ __global__ void ring_write_kernel(__half* ring_k, __half* ring_v, const __half* 
   }
 }
 
+constexpr int64_t kSmallEncodeTokens = 8;   // tokens per unit up to which the latency path runs
+
 template <int D>
 cudaError_t launch_encode_d(const EncodeArgs& a, cudaStream_t s) {
   const int warps = 8;
   const int64_t n = (int64_t)a.nA + a.nB;
   if (n == 0) return cudaSuccess;
+  if (D <= 128 && n <= kSmallEncodeTokens) {
+    const size_t smem = small_st_offset(D) + (size_t)D * a.L.m * sizeof(float);
+    if (smem > 48 * 1024) {
+      const cudaError_t e = cudaFuncSetAttribute(encode_small_kernel<D>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+    }
+    encode_small_kernel<D><<<(unsigned)(a.units * n), 2 * D, smem, s>>>(a);
+    return cudaGetLastError();
+  }
   const int64_t tiles = (a.cold_start + n - 1) / kTokensPerTile - a.cold_start / kTokensPerTile + 1;
   const int64_t jobs = (int64_t)a.units * tiles * 4;
   int dev = 0, sms = 148;
@@ -222,7 +450,13 @@ cudaError_t launch_encode_d(const EncodeArgs& a, cudaStream_t s) {
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t want = (jobs + warps - 1) / warps;
   const int grid = (int)(want < (int64_t)sms * 16 ? want : (int64_t)sms * 16);
-  const size_t smem = (size_t)warps * D * sizeof(double) + (size_t)warps * (8 * (D / 2) + 4 * 32 + 32);
+  size_t smem = st_offset(D, warps);
+  if (st_staged(D, a.L.m)) smem += (size_t)D * a.L.m * sizeof(float);
+  if (smem > 48 * 1024) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(encode_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
   encode_kernel<D><<<grid, warps * 32, smem, s>>>(a);
   return cudaGetLastError();
 }

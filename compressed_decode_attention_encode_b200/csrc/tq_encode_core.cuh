@@ -10,6 +10,7 @@ namespace enc {
 
 constexpr unsigned kFull = 0xffffffffu;
 constexpr double kTwoPi = 6.283185307179586476925286766559;  // rounds to 2 * fp64(pi)
+constexpr int kMaxSignWords = 8;   // m <= 256 sign bits per vector
 
 __device__ __forceinline__ uint16_t f64_to_f16_bits(double x) {
   uint16_t h;
@@ -46,7 +47,7 @@ __device__ __forceinline__ void load_vec(const __half* p, int lane, double (&x)[
 // and the raw fp16 scalars.  Whole warp; returns nothing else.
 // `load(lane, x)` fills the lane's D/32 consecutive input elements (padded
 // coordinates read as 0).  `L` supplies b_r, b_theta and m; `St` is S^T
-// [D, m]; `signs` the rotation diagonal.
+// [D, m] (global or shared memory); `signs` the rotation diagonal.
 template <int D, typename Loader>
 __device__ __forceinline__ void encode_vector_any(const Layout& L, const double* signs,
                                                   const float* St, double inv_sqrt_d, int* status,
@@ -143,17 +144,39 @@ __device__ __forceinline__ void encode_vector_any(const Layout& L, const double*
 #pragma unroll
     for (int i = 0; i < E; ++i) rbuf[lane * E + i] = r[i];
     __syncwarp();
+    // (S r)_i for the lane's outputs i = lane + 32 k, all k at once so that
+    // the loads of a batch of rows of S^T are in flight together; each
+    // output still sums over j in ascending order.
     const int m = L.m;
-    for (int k = 0; k < (m + 31) / 32; ++k) {
-      const int i = lane + 32 * k;
-      double acc = 0.0;
-      if (i < m) {
-        const float* col = St + i;
-#pragma unroll 8
-        for (int jj = 0; jj < D; ++jj) acc = fma((double)__ldg(col + (size_t)jj * m), rbuf[jj], acc);
+    const int nk = (m + 31) >> 5;
+    double acc[kMaxSignWords];
+#pragma unroll
+    for (int k = 0; k < kMaxSignWords; ++k) acc[k] = 0.0;
+    constexpr int JB = 4;
+    for (int j0 = 0; j0 < D; j0 += JB) {
+      float sv[JB][kMaxSignWords];
+#pragma unroll
+      for (int jj = 0; jj < JB; ++jj) {
+#pragma unroll
+        for (int k = 0; k < kMaxSignWords; ++k) {
+          const int i = lane + 32 * k;
+          sv[jj][k] = (k < nk && i < m) ? St[(size_t)(j0 + jj) * m + i] : 0.f;
+        }
       }
-      const unsigned word = __ballot_sync(kFull, i < m && acc >= 0.0);
-      if (lane == 0) bits[k] = word;
+#pragma unroll
+      for (int jj = 0; jj < JB; ++jj) {
+        const double rj = rbuf[j0 + jj];
+#pragma unroll
+        for (int k = 0; k < kMaxSignWords; ++k)
+          if (k < nk) acc[k] = fma((double)sv[jj][k], rj, acc[k]);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < kMaxSignWords; ++k) {
+      if (k < nk) {
+        const unsigned word = __ballot_sync(kFull, lane + 32 * k < m && acc[k] >= 0.0);
+        if (lane == 0) bits[k] = word;
+      }
     }
   }
   __syncwarp();

@@ -177,7 +177,7 @@ tq_status tq_cache_create(const tq_config* cfg, void* hot_mem, void* cold_mem,
     delete c;
     return TQ_ERR_CUDA;
   }
-  c->ctas_per_sm = attend_ctas_per_sm(c->L);
+  c->ctas_per_sm = attend_ctas_per_sm(c->L, cfg->num_q_heads / cfg->num_kv_heads);
   if (c->ctas_per_sm <= 0) {
     delete c;
     return TQ_ERR_CUDA;

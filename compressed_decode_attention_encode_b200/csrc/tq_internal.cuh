@@ -169,7 +169,7 @@ struct AttendArgs {
 };
 
 cudaError_t launch_attend(const AttendArgs& a, cudaStream_t s);
-int attend_ctas_per_sm(const Layout& L);
+int attend_ctas_per_sm(const Layout& L, int G);
 
 struct CombineArgs {
   const float* part;

@@ -58,6 +58,29 @@ def test_encode_chunked_appends_equal_one_append():
     _encode_and_compare(wl, 1, 200, seed=3, chunks=(1, 63, 70, 66))
 
 
+@pytest.mark.parametrize("name,batch,chunks", [
+    ("llama8b", 2, (3, 8, 1, 5, 64, 2, 7, 30, 1, 1)),    # appends of <= 8 tokens take the
+    ("tinyllama", 1, (1, 2, 3, 4, 5, 6, 7, 8, 60, 8)),   # per-token path, others the group path
+])
+def test_encode_small_appends_interleaved(name, batch, chunks):
+    # neighbouring tokens of one 32-bit word arrive in different appends
+    _encode_and_compare(WORKLOADS[name], batch, sum(chunks), seed=4, chunks=chunks)
+
+
+def test_encode_small_append_zero_and_overflow():
+    cfg = tq.make_config(1, 4, 1, 128, 64, 16, 3, 3, 128, seed=6)
+    cache = tq.TQCache(cfg)
+    z = torch.zeros((1, 1, 1, 128), dtype=torch.float16, device="cuda")
+    cache.encode_append(z, z)                                  # zero vector, alone
+    big = torch.full((1, 1, 1, 128), 60000.0, dtype=torch.float16, device="cuda")
+    cache.encode_append(big, z)                                # overflowing key, alone
+    assert cache.get_status() == 4
+    exp = cache.export_cold(0, 0, 0, 2)
+    assert exp["k_s16"][0] == 0 and exp["v_s16"][0] == 0 and exp["k_s16"][1] == 0
+    assert (exp["k_bits"][0] == 0xFF).all()
+    cache.close()
+
+
 @pytest.mark.parametrize("b_r,b_t,m,d", [(1, 1, 64, 64), (1, 7, 128, 128), (7, 1, 64, 128),
                                          (5, 3, 128, 64), (2, 2, 64, 64)])
 def test_encode_bit_widths(b_r, b_t, m, d):
