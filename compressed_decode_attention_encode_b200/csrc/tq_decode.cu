@@ -35,6 +35,11 @@ constexpr unsigned kFull = 0xffffffffu;
 constexpr int kThreads = 128;          // 4 warps; each takes 16 tokens of a 64-token block
 constexpr int kAttendMinBlocks = 4;    // attention CTAs per SM the shapes are sized for
 constexpr int kSmemPerSm = 233472;     // shared memory per SM (bytes)
+// Shared-window address of a kernel's dynamic shared memory when it has no
+// static shared variables: the first kilobyte of a CTA's window is reserved
+// for the system.  The attention kernel checks it and reports a layout
+// error rather than reading a misaligned table.
+constexpr int kDynSmemBase = 1024;
 constexpr int kAccSplit = 1;           // independent accumulator chains per tile product
 constexpr float kNegInf = -INFINITY;
 constexpr float kSqrtHalfPi = 1.2533141373155001f;   // sqrt(pi / 2)
@@ -70,6 +75,21 @@ __device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], uint32_t addr) {
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+// Shared-memory loads of ring stages by shared-window address, volatile so
+// that they stay after the stage's wait.
+
+__device__ __forceinline__ uint2 lds_ring64(uint32_t addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ uint32_t lds_ring32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
 }
 
 __device__ __forceinline__ float fast_exp2(float x) {
@@ -143,29 +163,36 @@ __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
 }
 
 // +-1 fp16 pair from sign bits 15-u and 31-u of x: bit 1 -> +1.0 (0x3C00),
-// bit 0 -> -1.0 (0xBC00).  The mask is a logic op; moving the bits to the
-// fp16 sign positions and mapping them is one integer multiply-add
-// (0xBC00BC00 - b * 2^u), which runs beside the logic ops.
+// bit 0 -> -1.0 (0xBC00).  Written as one shift and one three-input logic
+// op ((x << u) & 0x80008000) ^ 0xBC00BC00 in PTX, which the compiler keeps
+// as two instructions (its own lowering of the C++ form took three).
 __device__ __forceinline__ uint32_t sign_pair(uint32_t x, int u) {
-  return 0xBC00BC00u - (x & (0x80008000u >> u)) * (1u << u);
+  uint32_t r;
+  asm("{\n .reg .b32 s;\n shl.b32 s, %1, %2;\n lop3.b32 %0, s, 0x80008000, 0xBC00BC00, 0x6A;\n}"
+      : "=r"(r)
+      : "r"(x), "r"(u));
+  return r;
 }
 
 // Byte offset in a LUT whose entries are 2^SH bytes apart, of the entry
 // named by the BW-bit field at bit `pos` of the lane's word stream (`pos`
 // is a compile-time constant after unrolling), plus `lane_off` (the lane's
-// copy inside the entry).  A field inside one word costs a mask and an
-// integer multiply-add (a left shift, or a high-half multiply for a right
-// shift); a field straddling two words costs a funnel shift and a mask.
+// copy inside the entry): one shift (a funnel shift for a field straddling
+// two words) and one three-input logic op, written in PTX so that the
+// compiler keeps it at two instructions.
 template <int BW, int SH, int NW>
 __device__ __forceinline__ uint32_t lut_offset(const uint32_t (&w)[NW], int pos, uint32_t lane_off) {
-  constexpr uint32_t kMask = (1u << BW) - 1u;
+  constexpr uint32_t kMask = ((1u << BW) - 1u) << SH;
   const int wi = pos >> 5, bi = pos & 31;
+  uint32_t t, r;
   if (bi + BW <= 32 || wi + 1 >= NW) {
-    const uint32_t f = w[wi] & (kMask << bi);
-    if (bi <= SH) return f * (1u << (SH - bi)) + lane_off;
-    return __umulhi(f, 1u << (32 - (bi - SH))) + lane_off;
+    if (bi >= SH) asm("shr.b32 %0, %1, %2;" : "=r"(t) : "r"(w[wi]), "r"(bi - SH));
+    else asm("shl.b32 %0, %1, %2;" : "=r"(t) : "r"(w[wi]), "r"(SH - bi));
+  } else {
+    asm("shf.r.wrap.b32 %0, %1, %2, %3;" : "=r"(t) : "r"(w[wi]), "r"(w[wi + 1]), "r"(bi - SH));
   }
-  return (__funnelshift_r(w[wi], w[wi + 1], bi - SH) & (kMask << SH)) | lane_off;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(t), "n"(kMask), "r"(lane_off));   // (t & m) | l
+  return r;
 }
 
 // ---------------------------------------------------------------------------
@@ -282,41 +309,51 @@ struct AttendShape {
   static constexpr int TB = kTokensPerBlock;
   static constexpr int BLOCK = kTilesPerBlock * TT;
   static constexpr int NLUT = 1 << BW;
-  // two LUTs of fp16 pairs, one 4-byte copy per lane per entry: hi (keys
-  // and values) and lo (the keys' rounding remainder)
+  // Two LUTs of fp16 pairs, one 4-byte copy per lane per entry (entries
+  // 128 bytes apart): hi (keys and values), then lo (the keys' rounding
+  // remainder).  The hi table starts on a LUT_ALIGN boundary of the shared
+  // window, so a lookup's address is (table | entry << 7 | lane << 2) -- one
+  // logic op -- and the lo entry is the same address + LUT_BYTES.
   static constexpr int LUT_BYTES = NLUT * 32 * 4;
-  // LUTs up to 48 KB live in static shared memory, whose address the
-  // compiler folds into the load's immediate; larger ones are dynamic.
-  static constexpr bool STATIC_LUT = 2 * LUT_BYTES <= 49152;
-  static constexpr int DYN_LUT = STATIC_LUT ? 0 : 2 * LUT_BYTES;
+  static constexpr int LUT_ALIGN = 128 << BW;
   static constexpr int RS = 2 * D + 16;             // padded hot row stride (bytes)
   static constexpr int HOT_BYTES = TB * RS;          // one hot tile, K then V
   static constexpr int MERGE_BYTES = (64 + 8 * D) * 4;
-  // ring stages: as many as fit beside the LUTs and the merge area when
-  // kAttendMinBlocks CTAs share an SM (at least 2, at most 8)
+  static constexpr int BAR_BYTES = 8 * 8 + 8 * 8 + 16;   // up to 8 stages: barriers, counters, flags
+  // Dynamic shared memory: [ring | pad | LUT hi | LUT lo | merge | barriers],
+  // laid out for a dynamic base at shared address kDynSmemBase.
+  static constexpr int ring_bytes(int ns) { return ns * BLOCK > HOT_BYTES ? ns * BLOCK : HOT_BYTES; }
+  static constexpr int lut_off(int ns) {
+    return (kDynSmemBase + ring_bytes(ns) + LUT_ALIGN - 1) / LUT_ALIGN * LUT_ALIGN - kDynSmemBase;
+  }
+  static constexpr int smem_bytes(int ns) { return lut_off(ns) + 2 * LUT_BYTES + MERGE_BYTES + BAR_BYTES; }
+  // ring stages: as many as fit when kAttendMinBlocks CTAs share an SM (2 to 8)
   static constexpr int SMEM_PER_CTA = kSmemPerSm / kAttendMinBlocks - 1024;
-  static constexpr int RING_BUDGET = SMEM_PER_CTA - 2 * LUT_BYTES - MERGE_BYTES - 256;
-  static constexpr int NS_RAW = RING_BUDGET / BLOCK;
-  static constexpr int NS = NS_RAW < 2 ? 2 : (NS_RAW > 8 ? 8 : NS_RAW);   // ring stages
-  static constexpr int RING = NS * BLOCK > HOT_BYTES ? NS * BLOCK : HOT_BYTES;
-  static constexpr int OFF_LO = LUT_BYTES;           // (dynamic LUT case)
-  static constexpr int OFF_RING = DYN_LUT;
-  static constexpr int OFF_MERGE = OFF_RING + RING;
+  static constexpr int pick_ns() {
+    int ns = 2;
+    for (int k = 3; k <= 8; ++k)
+      if (smem_bytes(k) <= SMEM_PER_CTA) ns = k;
+    return ns;
+  }
+  static constexpr int NS = pick_ns();
+  static constexpr int RING = ring_bytes(NS);
+  static constexpr int OFF_LUT = lut_off(NS);
+  static constexpr int OFF_MERGE = OFF_LUT + 2 * LUT_BYTES;
   static constexpr int OFF_BAR = OFF_MERGE + MERGE_BYTES;
-  static constexpr int SMEM = OFF_BAR + 8 * NS + 8 * NS + 16;   // + per-stage counters, flags
+  static constexpr int SMEM = smem_bytes(NS);
 };
 
 // 2-word-major per-lane words of a tile plane (see Layout).
 template <int NW>
-__device__ __forceinline__ void load_lane_words(const uint8_t* plane, int lane, uint32_t (&w)[NW]) {
+__device__ __forceinline__ void load_lane_words(uint32_t plane, int lane, uint32_t (&w)[NW]) {
 #pragma unroll
   for (int g = 0; 2 * g < NW; ++g) {
     if (2 * g + 1 < NW) {
-      const uint2 v = *reinterpret_cast<const uint2*>(plane + g * 256 + lane * 8);
+      const uint2 v = lds_ring64(plane + g * 256 + lane * 8);
       w[2 * g] = v.x;
       w[2 * g + 1] = v.y;
     } else {
-      w[2 * g] = *reinterpret_cast<const uint32_t*>(plane + g * 256 + lane * 4);
+      w[2 * g] = lds_ring32(plane + g * 256 + lane * 4);
     }
   }
 }
@@ -484,15 +521,11 @@ template <int D, int M, int BW, bool PACK>
 __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(const AttendArgs a) {
   using S = AttendShape<D, M, BW>;
   extern __shared__ __align__(128) uint8_t smem[];
-  // Separate 4-byte hi and lo tables (rather than one 8-byte entry) let
+  // Separate 4-byte hi and lo entries (rather than one 8-byte entry) let
   // each looked-up register land directly in the MMA's operand registers.
-  __shared__ __align__(16) uint32_t lhi_static[S::STATIC_LUT ? S::NLUT * 32 : 4];
-  __shared__ __align__(16) uint32_t llo_static[S::STATIC_LUT ? S::NLUT * 32 : 4];
-  uint32_t* lhi_w = S::STATIC_LUT ? lhi_static : reinterpret_cast<uint32_t*>(smem);
-  uint32_t* llo_w = S::STATIC_LUT ? llo_static : reinterpret_cast<uint32_t*>(smem + S::OFF_LO);
-  const char* lhi = reinterpret_cast<const char*>(lhi_w);
-  const char* llo = reinterpret_cast<const char*>(llo_w);
-  uint8_t* ring = smem + S::OFF_RING;
+  uint32_t* lhi_w = reinterpret_cast<uint32_t*>(smem + S::OFF_LUT);
+  uint32_t* llo_w = lhi_w + S::NLUT * 32;
+  uint8_t* ring = smem;
   float* merge = reinterpret_cast<float*>(smem + S::OFF_MERGE);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::OFF_BAR);
   int* arrivals = reinterpret_cast<int*>(smem + S::OFF_BAR + 8 * S::NS);    // [NS] warps done
@@ -505,7 +538,22 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
   const int Lr = (1 << a.L.b_r) - 1;
   const float inv_levels = 1.f / (float)Lr;
   const int tb = warp * 16;            // this warp's tokens inside a block / tile
-  const uint32_t lane4 = (uint32_t)lane * 4u;
+  const uint32_t lut_sa = smem_addr(lhi_w);
+  if (lut_sa & (S::LUT_ALIGN - 1)) {   // dynamic base not where the layout assumes
+    if (tid == 0) atomicOr(a.status, kStatusLayout);
+    return;
+  }
+  const uint32_t lane_lut = lut_sa | ((uint32_t)lane * 4u);   // this lane's copy, hi table
+  auto lut_hi = [&](uint32_t addr) {
+    uint32_t v;
+    asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
+  };
+  auto lut_lo = [&](uint32_t addr) {
+    uint32_t v;
+    asm("ld.shared.u32 %0, [%1+%2];" : "=r"(v) : "r"(addr), "n"(S::LUT_BYTES));
+    return v;
+  };
   const SplitPlan& pl = a.plan;
   const int slots = pl.slots_cold + pl.slots_hot;
   WarpState<S::NT> st;
@@ -632,28 +680,28 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
       const int64_t left = a.n_cold - blk * S::TB - tb;
       if (!aborted && left > 0) {
       const int nvalid = left < 16 ? (int)left : 16;     // valid tokens of this warp's tile
-      const uint8_t* tile = ring + stage * S::BLOCK + warp * S::TT;
+      const uint32_t tile = ring0 + stage * S::BLOCK + warp * S::TT;
 
       uint32_t kw[S::KWT], sw[S::SW], vw[S::VWT];
       load_lane_words<S::KWT>(tile + S::OFF_KC, lane, kw);
       load_lane_words<S::SW>(tile + S::OFF_KS, lane, sw);
       load_lane_words<S::VWT>(tile + S::OFF_VC, lane, vw);
-      const uint2 ksc = *reinterpret_cast<const uint2*>(tile + S::OFF_KSC + gid * 8);
-      const uint32_t vsc = *reinterpret_cast<const uint32_t*>(tile + S::OFF_VSC + gid * 4);
+      const uint2 ksc = lds_ring64(tile + S::OFF_KSC + gid * 8);
+      const uint32_t vsc = lds_ring32(tile + S::OFF_VSC + gid * 4);
 
       // ---- cold logits: polar part, (A_hi + A_lo) . (q'_hi + q'_lo) ------
       // k-steps accumulate round-robin into kAccSplit chains
       float c1[kAccSplit][4] = {}, c2[kAccSplit][4] = {};
 #pragma unroll
       for (int s = 0; s < S::NT; ++s) {
-        const uint32_t o0 = lut_offset<BW, 7>(kw, (2 * s) * BW, lane4);
-        const uint32_t o1 = lut_offset<BW, 7>(kw, (S::PT + 2 * s) * BW, lane4);
-        const uint32_t o2 = lut_offset<BW, 7>(kw, (2 * s + 1) * BW, lane4);
-        const uint32_t o3 = lut_offset<BW, 7>(kw, (S::PT + 2 * s + 1) * BW, lane4);
-        const uint2 a0 = make_uint2(*reinterpret_cast<const uint32_t*>(lhi + o0), *reinterpret_cast<const uint32_t*>(llo + o0));
-        const uint2 a1 = make_uint2(*reinterpret_cast<const uint32_t*>(lhi + o1), *reinterpret_cast<const uint32_t*>(llo + o1));
-        const uint2 a2 = make_uint2(*reinterpret_cast<const uint32_t*>(lhi + o2), *reinterpret_cast<const uint32_t*>(llo + o2));
-        const uint2 a3 = make_uint2(*reinterpret_cast<const uint32_t*>(lhi + o3), *reinterpret_cast<const uint32_t*>(llo + o3));
+        const uint32_t o0 = lut_offset<BW, 7>(kw, (2 * s) * BW, lane_lut);
+        const uint32_t o1 = lut_offset<BW, 7>(kw, (S::PT + 2 * s) * BW, lane_lut);
+        const uint32_t o2 = lut_offset<BW, 7>(kw, (2 * s + 1) * BW, lane_lut);
+        const uint32_t o3 = lut_offset<BW, 7>(kw, (S::PT + 2 * s + 1) * BW, lane_lut);
+        const uint2 a0 = make_uint2(lut_hi(o0), lut_lo(o0));
+        const uint2 a1 = make_uint2(lut_hi(o1), lut_lo(o1));
+        const uint2 a2 = make_uint2(lut_hi(o2), lut_lo(o2));
+        const uint2 a3 = make_uint2(lut_hi(o3), lut_lo(o3));
         mma16816(c1[s % kAccSplit], a0.x, a1.x, a2.x, a3.x, bq[s][0], bq[s][1]);
         if constexpr (PACK) {
           mma16816(c2[s % kAccSplit], a0.y, a1.y, a2.y, a3.y, bq2[s][0], bq2[s][1]);
@@ -712,10 +760,10 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
       // ---- P V: V codes of pairs PV*gid + j for tokens 2tig, 2tig+1, +8, +9
 #pragma unroll
       for (int j = 0; j < S::NT; ++j) {
-        const uint32_t L0 = *reinterpret_cast<const uint32_t*>(lhi + lut_offset<BW, 7>(vw, (0 * S::PV + j) * BW, lane4));
-        const uint32_t L1 = *reinterpret_cast<const uint32_t*>(lhi + lut_offset<BW, 7>(vw, (1 * S::PV + j) * BW, lane4));
-        const uint32_t L2 = *reinterpret_cast<const uint32_t*>(lhi + lut_offset<BW, 7>(vw, (2 * S::PV + j) * BW, lane4));
-        const uint32_t L3 = *reinterpret_cast<const uint32_t*>(lhi + lut_offset<BW, 7>(vw, (3 * S::PV + j) * BW, lane4));
+        const uint32_t L0 = lut_hi(lut_offset<BW, 7>(vw, (0 * S::PV + j) * BW, lane_lut));
+        const uint32_t L1 = lut_hi(lut_offset<BW, 7>(vw, (1 * S::PV + j) * BW, lane_lut));
+        const uint32_t L2 = lut_hi(lut_offset<BW, 7>(vw, (2 * S::PV + j) * BW, lane_lut));
+        const uint32_t L3 = lut_hi(lut_offset<BW, 7>(vw, (3 * S::PV + j) * BW, lane_lut));
         mma16816(st.O[j], __byte_perm(L0, L1, 0x5410), __byte_perm(L0, L1, 0x7632),
                  __byte_perm(L2, L3, 0x5410), __byte_perm(L2, L3, 0x7632), pb0, pb1);
       }

@@ -538,6 +538,7 @@ tq_status tq_get_status(tq_cache* c, cudaStream_t stream) {
   if (cudaMemcpy(&word, c->status(), sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
     return TQ_ERR_CUDA;
   if (word != 0 && cudaMemset(c->status(), 0, sizeof(int)) != cudaSuccess) return TQ_ERR_CUDA;
+  if (word & kStatusLayout) return TQ_ERR_UNSUPPORTED;
   if (word & kStatusTimeout) return TQ_ERR_TIMEOUT;
   if (word & kStatusRange) return TQ_ERR_RANGE;
   return TQ_OK;

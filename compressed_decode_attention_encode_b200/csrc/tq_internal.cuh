@@ -19,6 +19,7 @@ constexpr int kTilesPerBlock = kTokensPerBlock / kTokensPerTile;
 // Device status word bits (latched, cleared by tq_get_status).
 constexpr int kStatusRange = 1;
 constexpr int kStatusTimeout = 2;
+constexpr int kStatusLayout = 4;    // a kernel found shared memory where its layout does not fit
 
 // Cold-store layout.  Per (row, kv head): 64-token blocks of 4 tiles.  A
 // tile (16 tokens) is laid out fragment-major for the decode warp that

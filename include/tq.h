@@ -200,8 +200,10 @@ tq_status tq_decode_attention_static(tq_cache* cache, const void* q, float* out,
 
 /*
  * Synchronize `stream`, then return and clear the latched device status
- * (TQ_OK, TQ_ERR_RANGE or TQ_ERR_TIMEOUT), or TQ_ERR_CUDA if the stream
- * itself reports an error.
+ * (TQ_OK, TQ_ERR_RANGE or TQ_ERR_TIMEOUT; TQ_ERR_UNSUPPORTED when the
+ * attention kernel found its dynamic shared memory at a window address its
+ * table layout does not fit, in which case it wrote no output), or
+ * TQ_ERR_CUDA if the stream itself reports an error.
  */
 tq_status tq_get_status(tq_cache* cache, cudaStream_t stream);
 
