@@ -559,9 +559,9 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
   WarpState<S::NT> st;
   st.reset();
 
-  if ((int)blockIdx.x < pl.cold_ctas) {
-    // ======================= cold CTA =======================
-    const int c = blockIdx.x;
+  const int c = blockIdx.x;
+  if (c < pl.cold_ctas) {
+    // ============ cold run: blocks [c * bpc, (c + 1) * bpc) ============
     const int64_t nb = pl.cold_blocks;
     const int64_t total = (int64_t)a.units * nb;
     const int64_t f_lo = (int64_t)c * pl.cold_bpc;
@@ -803,10 +803,11 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
     if (unit_cur >= 0) {
       flush_partial<D, S::NT>(st, false, inv_levels, G, merge,
                               a.part + (((size_t)unit_cur * slots + slot_cur) * G) * (D + 2));
+      st.reset();
     }
-  } else {
-    // ======================= hot CTA =======================
-    const int c = blockIdx.x - pl.cold_ctas;
+  }
+  if (c < pl.hot_ctas) {
+    // ====== then hot tiles [c * tpc, (c + 1) * tpc): the ring is idle ======
     const int ht = pl.hot_tiles;
     const int64_t total = (int64_t)a.units * ht;
     const int64_t f_lo = (int64_t)c * pl.hot_tpc;
@@ -1071,7 +1072,7 @@ cudaError_t launch_attend(const AttendArgs& a, cudaStream_t s) {
   int smem = 0;
   AttendFn fn = pick_attend(a.L, a.G, &smem);
   if (!fn) return cudaErrorInvalidValue;
-  const int grid = a.plan.cold_ctas + a.plan.hot_ctas;
+  const int grid = a.plan.cold_ctas > a.plan.hot_ctas ? a.plan.cold_ctas : a.plan.hot_ctas;
   if (grid == 0) return cudaSuccess;
   fn<<<grid, kThreads, smem, s>>>(a);
   return cudaGetLastError();

@@ -276,6 +276,43 @@ tq_status tq_evict_window(tq_cache* c, const void* k_new, const void* v_new, int
   return TQ_OK;
 }
 
+// Split plan: one wave of `ctas` CTAs.  Every CTA streams an equal run of
+// the flattened (unit, cold block) list; CTAs [0, hot_ctas) then also take
+// hot_tpc hot tiles each (one for the usual window sizes), so the latency
+// of the fp16 hot tiles is paid once per CTA at the end of its cold run
+// rather than by a few CTAs in turn.  `tight` sizes the partial slots per
+// unit to the most any unit can receive under the plan (the static-scratch
+// entry point); otherwise they are the workspace's fixed kSlotsCold /
+// kSlotsHot.
+static SplitPlan make_plan(int64_t n_cold, int n_hot, int units, int ctas, bool tight) {
+  const int TB = kTokensPerBlock;
+  const int64_t cold_blocks = (n_cold + TB - 1) / TB;
+  const int hot_tiles = (n_hot + TB - 1) / TB;
+  const int64_t N = (int64_t)units * cold_blocks;
+  const int64_t Nh = (int64_t)units * hot_tiles;
+  SplitPlan pl{};
+  pl.cold_blocks = cold_blocks;
+  pl.hot_tiles = hot_tiles;
+  pl.slots_cold = kSlotsCold;
+  pl.slots_hot = kSlotsHot;
+  if (Nh > 0) {
+    int64_t tpc = (Nh + ctas - 1) / ctas;
+    // a unit's tiles may span at most kSlotsHot - 2 CTAs
+    tpc = std::max<int64_t>(tpc, hot_tiles > 1 ? (hot_tiles - 1 + kSlotsHot - 3) / (kSlotsHot - 2) : 1);
+    pl.hot_tpc = (int)tpc;
+    pl.hot_ctas = (int)((Nh + tpc - 1) / tpc);
+    if (tight) pl.slots_hot = (int)((hot_tiles - 1) / tpc + 2);
+  }
+  if (N > 0) {
+    int64_t bpc = (N + ctas - 1) / ctas;
+    bpc = std::max<int64_t>(bpc, cold_blocks > 1 ? (cold_blocks - 1 + kSlotsCold - 3) / (kSlotsCold - 2) : 1);
+    pl.cold_bpc = bpc;
+    pl.cold_ctas = (int)((N + bpc - 1) / bpc);
+    if (tight) pl.slots_cold = (int)((cold_blocks - 1) / bpc + 2);
+  }
+  return pl;
+}
+
 tq_status tq_decode_attention(tq_cache* c, const void* q, float* out, float softmax_scale,
                               cudaStream_t stream) {
   if (!c || !q || !out || !(softmax_scale >= 0.0f) || std::isinf(softmax_scale))
@@ -286,39 +323,8 @@ tq_status tq_decode_attention(tq_cache* c, const void* q, float* out, float soft
   const int units = cf.batch * cf.num_kv_heads;
   const int G = cf.num_q_heads / cf.num_kv_heads;
   const float sigma = softmax_scale == 0.0f ? (float)(1.0 / std::sqrt((double)d)) : softmax_scale;
-  const int TB = kTokensPerBlock;
 
-  // Split plan: one wave of CTAs.  Hot tiles and cold blocks get CTAs in
-  // proportion to their bytes; each CTA takes an equal run of the flattened
-  // (unit, block) list, so every SM streams about the same number of bytes.
-  const int64_t cold_blocks = (c->n_cold + TB - 1) / TB;
-  const int hot_tiles = (c->n_hot + TB - 1) / TB;
-  const int64_t N = (int64_t)units * cold_blocks;
-  const int64_t Nh = (int64_t)units * hot_tiles;
-  const int slots = c->num_sms * c->ctas_per_sm;
-  const double cold_b = (double)N * c->L.block_bytes;
-  const double hot_b = (double)Nh * TB * d * 4.0;
-  SplitPlan pl{};
-  pl.cold_blocks = cold_blocks;
-  pl.hot_tiles = hot_tiles;
-  pl.slots_cold = kSlotsCold;
-  pl.slots_hot = kSlotsHot;
-  if (Nh > 0) {
-    int ch = (int)std::lround(slots * hot_b / (hot_b + cold_b));
-    ch = (int)std::max<int64_t>(1, std::min<int64_t>(ch, Nh));
-    int64_t tpc = (Nh + ch - 1) / ch;
-    // a unit's tiles may span at most kSlotsHot CTAs
-    tpc = std::max<int64_t>(tpc, hot_tiles > 1 ? (hot_tiles - 1 + kSlotsHot - 3) / (kSlotsHot - 2) : 1);
-    pl.hot_tpc = (int)tpc;
-    pl.hot_ctas = (int)((Nh + tpc - 1) / tpc);
-  }
-  if (N > 0) {
-    const int cc = std::max(1, slots - pl.hot_ctas);
-    int64_t bpc = (N + cc - 1) / cc;
-    bpc = std::max<int64_t>(bpc, cold_blocks > 1 ? (cold_blocks - 1 + kSlotsCold - 3) / (kSlotsCold - 2) : 1);
-    pl.cold_bpc = bpc;
-    pl.cold_ctas = (int)((N + bpc - 1) / bpc);
-  }
+  const SplitPlan pl = make_plan(c->n_cold, c->n_hot, units, c->num_sms * c->ctas_per_sm, false);
 
   __half* qrot = (__half*)(c->ws + c->W.qrot);
   __half* qsk = (__half*)(c->ws + c->W.qsk);
@@ -432,37 +438,10 @@ tq_status tq_decode_attention_static(tq_cache* c, const void* q, float* out, flo
   const int units = cf.batch * cf.num_kv_heads;
   const int G = cf.num_q_heads / cf.num_kv_heads;
   const float sigma = softmax_scale == 0.0f ? (float)(1.0 / std::sqrt((double)d)) : softmax_scale;
-  const int TB = kTokensPerBlock;
 
   // The same split plan as tq_decode_attention, with the partial slots per
   // unit cut to the most any unit can receive under this plan.
-  const int64_t cold_blocks = (c->n_cold + TB - 1) / TB;
-  const int hot_tiles = (c->n_hot + TB - 1) / TB;
-  const int64_t N = (int64_t)units * cold_blocks;
-  const int64_t Nh = (int64_t)units * hot_tiles;
-  const int slots = c->num_sms * c->ctas_per_sm;
-  const double cold_b = (double)N * c->L.block_bytes;
-  const double hot_b = (double)Nh * TB * d * 4.0;
-  SplitPlan pl{};
-  pl.cold_blocks = cold_blocks;
-  pl.hot_tiles = hot_tiles;
-  if (Nh > 0) {
-    int ch = (int)std::lround(slots * hot_b / (hot_b + cold_b));
-    ch = (int)std::max<int64_t>(1, std::min<int64_t>(ch, Nh));
-    int64_t tpc = (Nh + ch - 1) / ch;
-    tpc = std::max<int64_t>(tpc, hot_tiles > 1 ? (hot_tiles - 1 + kSlotsHot - 3) / (kSlotsHot - 2) : 1);
-    pl.hot_tpc = (int)tpc;
-    pl.hot_ctas = (int)((Nh + tpc - 1) / tpc);
-    pl.slots_hot = (int)((hot_tiles - 1) / tpc + 2);
-  }
-  if (N > 0) {
-    const int cc = std::max(1, slots - pl.hot_ctas);
-    int64_t bpc = (N + cc - 1) / cc;
-    bpc = std::max<int64_t>(bpc, cold_blocks > 1 ? (cold_blocks - 1 + kSlotsCold - 3) / (kSlotsCold - 2) : 1);
-    pl.cold_bpc = bpc;
-    pl.cold_ctas = (int)((N + bpc - 1) / bpc);
-    pl.slots_cold = (int)((cold_blocks - 1) / bpc + 2);
-  }
+  const SplitPlan pl = make_plan(c->n_cold, c->n_hot, units, c->num_sms * c->ctas_per_sm, true);
 
   // scratch layout: rotated queries | q'' | per-head scales | partials
   size_t off = 0;
