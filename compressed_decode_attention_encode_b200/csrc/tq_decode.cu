@@ -199,7 +199,8 @@ __device__ __forceinline__ uint32_t lut_offset(const uint32_t (&w)[NW], int pos,
 // q-prep: HB = 256 / M heads per block (2 for m = 128), so that the grid
 // spreads over the SMs.  One warp per head rotates q (butterflies in
 // registers and across lanes); then every thread computes one element of
-// S q' from S^T staged in shared memory (loads issued before the rotation).
+// S q' from S^T staged in shared memory (asynchronous copies issued before
+// the rotation).
 // ---------------------------------------------------------------------------
 template <int D, int M>
 __global__ void __launch_bounds__(256) qprep_kernel(const QPrepArgs a) {
@@ -209,8 +210,7 @@ __global__ void __launch_bounds__(256) qprep_kernel(const QPrepArgs a) {
   __shared__ float sqq[HB][M];
   extern __shared__ float4 sst4[];       // S^T [D][M]
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int i = threadIdx.x; i < D * M / 4; i += blockDim.x)
-    sst4[i] = __ldg(reinterpret_cast<const float4*>(a.St) + i);
+  async_copy_g2s(sst4, a.St, D * M * 4);       // lands while the rotation runs
   const float* sst = reinterpret_cast<const float*>(sst4);
   const int h = blockIdx.x * HB + warp;          // head of this warp (warps < HB)
   if (warp < HB) {
@@ -260,6 +260,7 @@ __global__ void __launch_bounds__(256) qprep_kernel(const QPrepArgs a) {
       if (lane == 0) a.qscale[2 * h] = 1.f / al1;
     }
   }
+  async_copy_wait();
   __syncthreads();
   {
     const int hb = threadIdx.x / M, i = threadIdx.x % M;
@@ -336,7 +337,6 @@ struct AttendShape {
     return ns;
   }
   static constexpr int NS = pick_ns();
-  static constexpr int RING = ring_bytes(NS);
   static constexpr int OFF_LUT = lut_off(NS);
   static constexpr int OFF_MERGE = OFF_LUT + 2 * LUT_BYTES;
   static constexpr int OFF_BAR = OFF_MERGE + MERGE_BYTES;
@@ -623,9 +623,11 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
     int slot_cur = 0;
     bool aborted = false;
     int unit = (int)(f_lo / nb);          // advanced incrementally: no division per block
-    int64_t blk = f_lo - (int64_t)unit * nb;
+    int blk = (int)(f_lo - (int64_t)unit * nb);   // block inside the unit (< 2^31)
+    const int nbi = (int)nb;
+    const int tail = (int)(a.n_cold - (int64_t)(nbi - 1) * S::TB);   // valid tokens of a unit's last block
     for (int i = 0; i < nblk; ++i, ++blk) {
-      if (blk == nb) {
+      if (blk == nbi) {
         blk = 0;
         ++unit;
       }
@@ -669,7 +671,6 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
       }
       // ---- wait for this block's stage (every warp on its own) ----------
       const int stage = i % S::NS;
-      if (!aborted && *abort_flag) aborted = true;
       if (!aborted) {
         const bool got = mbar_wait_bounded(bar0 + 8 * stage, (uint32_t)((i / S::NS) & 1));
         if (!__all_sync(kFull, got)) {
@@ -677,7 +678,7 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
           if (lane == 0) *abort_flag = 1;
         }
       }
-      const int64_t left = a.n_cold - blk * S::TB - tb;
+      const int left = (blk == nbi - 1 ? tail : S::TB) - tb;
       if (!aborted && left > 0) {
       const int nvalid = left < 16 ? (int)left : 16;     // valid tokens of this warp's tile
       const uint32_t tile = ring0 + stage * S::BLOCK + warp * S::TT;
@@ -777,9 +778,9 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
           __threadfence_block();
           fence_proxy_async();
           mbar_expect_tx(bar0 + 8 * stage, S::BLOCK);
-          int64_t pb = blk + S::NS;          // block i + NS: at most NS past (unit, blk)
+          int pb = blk + S::NS;              // block i + NS: at most NS past (unit, blk)
           int pu = unit;
-          while (pb >= nb) { pb -= nb; ++pu; }
+          while (pb >= nbi) { pb -= nbi; ++pu; }
           bulk_g2s(ring0 + stage * S::BLOCK,
                    a.cold + ((size_t)pu * a.L.blocks_per_unit + (size_t)pb) * S::BLOCK, S::BLOCK,
                    bar0 + 8 * stage);

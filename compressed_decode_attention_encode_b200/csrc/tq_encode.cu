@@ -109,9 +109,8 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
   const float* St = a.St;
   if (st_staged(D, L.m)) {
     float* sst = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(smem) + st_offset(D, warps));
-    const int n16 = D * L.m / 4;
-    for (int i = threadIdx.x; i < n16; i += blockDim.x)
-      reinterpret_cast<float4*>(sst)[i] = __ldg(reinterpret_cast<const float4*>(a.St) + i);
+    async_copy_g2s(sst, a.St, D * L.m * 4);
+    async_copy_wait();
     __syncthreads();
     St = sst;
   }
@@ -244,8 +243,7 @@ __global__ void __launch_bounds__(2 * D) encode_small_kernel(EncodeArgs a) {
   uint32_t* bits = reinterpret_cast<uint32_t*>(codes + 2 * P); // [4] key sign words
   uint16_t* sc = reinterpret_cast<uint16_t*>(bits + 4);        // s16_k, rn16, s16_v
   float* sst = reinterpret_cast<float*>(sm) + small_st_offset(D) / 4;   // S^T [D][m]
-  for (int i = tid; i < D * L.m / 4; i += blockDim.x)
-    reinterpret_cast<float4*>(sst)[i] = __ldg(reinterpret_cast<const float4*>(a.St) + i);
+  async_copy_g2s(sst, a.St, D * L.m * 4);      // lands while the rotation and polar steps run
 
   const __half* src;
   if (e < a.nA) {
@@ -255,7 +253,12 @@ __global__ void __launch_bounds__(2 * D) encode_small_kernel(EncodeArgs a) {
     src = (team ? a.src_v : a.src_k) + ((int64_t)unit * a.src_tokens + (e - a.nA)) * D;
   }
   // ---- rotation: y = H (D x) / sqrt(d) ----------------------------------
-  double x = __dmul_rn((double)__half2float(src[el]), a.signs[el]);
+  const __half xin = src[el];
+  if (a.write_new) {         // the slot just read now takes the new token (same thread, same element)
+    const __half* nsrc = (team ? a.src_v : a.src_k) + ((int64_t)unit * a.src_tokens + e) * D;
+    const_cast<__half*>(src)[el] = nsrc[el];
+  }
+  double x = __dmul_rn((double)__half2float(xin), a.signs[el]);
 #pragma unroll
   for (int h = 1; h < D; h <<= 1) {
     double o;
@@ -322,6 +325,7 @@ __global__ void __launch_bounds__(2 * D) encode_small_kernel(EncodeArgs a) {
   }
 #pragma unroll
   for (int o = 16; o; o >>= 1) ss = __dadd_rn(ss, __shfl_xor_sync(kFull, ss, o));
+  async_copy_wait();
   __syncthreads();            // residual complete, S^T staged, reduction slots free
   if (team == 0) {
     if (lane == 0) red[wt] = ss;
@@ -425,8 +429,6 @@ __global__ void ring_write_kernel(__half* ring_k, __half* ring_v, const __half* 
     *dst = *s;
   }
 }
-
-constexpr int64_t kSmallEncodeTokens = 8;   // tokens per unit up to which the latency path runs
 
 template <int D>
 cudaError_t launch_encode_d(const EncodeArgs& a, cudaStream_t s) {

@@ -253,6 +253,9 @@ tq_status tq_evict_window(tq_cache* c, const void* k_new, const void* v_new, int
   const int W = c->cfg.hot_window;
   const int64_t E = std::max<int64_t>(0, (int64_t)c->n_hot + n - W);
   if (c->n_cold + E > c->cfg.cold_capacity) return TQ_ERR_CAPACITY;
+  // Steady state (a full window, a few new tokens): each new token evicts
+  // the token in the slot it takes, and one launch does both.
+  const bool fused = E == n && c->n_hot == W && n <= W && n <= kSmallEncodeTokens;
   if (E > 0) {
     EncodeArgs a = base_encode_args(c);
     a.nA = (int)std::min<int64_t>(E, c->n_hot);
@@ -263,13 +266,16 @@ tq_status tq_evict_window(tq_cache* c, const void* k_new, const void* v_new, int
     a.src_k = (const __half*)k_new;
     a.src_v = (const __half*)v_new;
     a.src_tokens = n;
+    a.write_new = fused ? 1 : 0;
     if (launch_encode(a, stream) != cudaSuccess) return TQ_ERR_CUDA;
   }
-  const int first = std::max(0, n - W);
-  if (launch_ring_write(c->hot_k(), c->hot_v(), (const __half*)k_new, (const __half*)v_new,
-                        c->cfg.batch * c->cfg.num_kv_heads, W, c->cfg.head_dim, n, first,
-                        c->ring_pos, stream) != cudaSuccess)
-    return TQ_ERR_CUDA;
+  if (!fused) {
+    const int first = std::max(0, n - W);
+    if (launch_ring_write(c->hot_k(), c->hot_v(), (const __half*)k_new, (const __half*)v_new,
+                          c->cfg.batch * c->cfg.num_kv_heads, W, c->cfg.head_dim, n, first,
+                          c->ring_pos, stream) != cudaSuccess)
+      return TQ_ERR_CUDA;
+  }
   c->n_cold += E;
   c->n_hot = (int32_t)std::min<int64_t>(W, (int64_t)c->n_hot + n);
   c->ring_pos = (int32_t)(((int64_t)c->ring_pos + n) % W);

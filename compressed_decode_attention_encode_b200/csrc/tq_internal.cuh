@@ -111,7 +111,32 @@ struct EncodeArgs {
   const float* St;          // S transposed, [d, m]
   int* status;
   double inv_sqrt_d;        // 1 / sqrt(d), correctly rounded on the host
+  // Steady-state eviction (per-token path only): after reading ring slot
+  // (ring_start + e) mod W, token e's CTA writes src_k/src_v token e into
+  // that same slot, so the ring write needs no launch of its own.
+  int write_new;
 };
+
+// Global -> shared copy of `bytes` (a multiple of 16, both addresses 16-byte
+// aligned) as asynchronous 16-byte copies spread over the block's threads:
+// no thread waits for them here.  Before reading, every thread calls
+// async_copy_wait() (its own copies) and the block meets at a barrier.
+__device__ __forceinline__ void async_copy_g2s(void* dst, const void* src, int bytes) {
+  const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst);
+  for (int i = (int)threadIdx.x * 16; i < bytes; i += (int)blockDim.x * 16)
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(d + i),
+                 "l"(reinterpret_cast<const char*>(src) + i)
+                 : "memory");
+  asm volatile("cp.async.commit_group;\n" ::: "memory");
+}
+
+__device__ __forceinline__ void async_copy_wait() {
+  asm volatile("cp.async.wait_group 0;\n" ::: "memory");
+}
+
+// Appends of up to this many tokens per unit take the per-token (latency)
+// encode path; longer ones the warp-per-vector (throughput) path.
+constexpr int64_t kSmallEncodeTokens = 8;
 
 cudaError_t launch_encode(const EncodeArgs& a, cudaStream_t s);
 
