@@ -331,7 +331,7 @@ def run_gpu(args, wl):
         t = torch.tensor([ms], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms = float(t.item())
-    launches_per_step = L * (2 + 3)   # evict: encode + ring write; decode: qprep, attend, combine
+    launches_per_step = L * (1 + 3)   # evict: per-token encode (ring write fused); decode: qprep, attend, combine
 
     # ---- e2e: host buffers through the public API ------------------------
     hk = [[x.cpu().pin_memory() for x in knew[l]] for l in range(L)]

@@ -319,68 +319,61 @@ static SplitPlan make_plan(int64_t n_cold, int n_hot, int units, int ctas, bool 
   return pl;
 }
 
-tq_status tq_decode_attention(tq_cache* c, const void* q, float* out, float softmax_scale,
-                              cudaStream_t stream) {
-  if (!c || !q || !out || !(softmax_scale >= 0.0f) || std::isinf(softmax_scale))
-    return TQ_ERR_INVALID_ARG;
+// The launches of one decode call: q-prep, the attention kernel (split
+// partials), and the merge of the partials into the output rows.  Scratch
+// buffers are the caller's (workspace or static scratch).
+static tq_status launch_decode(tq_cache* c, const void* q, float* out, float softmax_scale,
+                               const SplitPlan& pl, __half* qrot, __half* qsk, float* qscale,
+                               float* part, cudaStream_t stream) {
   const tq_config& cf = c->cfg;
-  const int d = cf.head_dim, m = cf.qjl_bits;
-  const int heads = cf.batch * cf.num_q_heads;
+  const int d = cf.head_dim;
   const int units = cf.batch * cf.num_kv_heads;
-  const int G = cf.num_q_heads / cf.num_kv_heads;
   const float sigma = softmax_scale == 0.0f ? (float)(1.0 / std::sqrt((double)d)) : softmax_scale;
-
-  const SplitPlan pl = make_plan(c->n_cold, c->n_hot, units, c->num_sms * c->ctas_per_sm, false);
-
-  __half* qrot = (__half*)(c->ws + c->W.qrot);
-  __half* qsk = (__half*)(c->ws + c->W.qsk);
-  float* qscale = (float*)(c->ws + c->W.qscale);
-  float* part = (float*)(c->ws + c->W.part);
-
-  if (pl.cold_ctas > 0) {
-    QPrepArgs qa{};
-    qa.q = (const __half*)q;
-    qa.signs = c->signs();
-    qa.St = c->St();
-    qa.qrot = qrot;
-    qa.qsk = qsk;
-    qa.qscale = qscale;
-    qa.heads = heads;
-    qa.d = d;
-    qa.m = m;
-    if (launch_qprep(qa, stream) != cudaSuccess) return TQ_ERR_CUDA;
+  if (pl.cold_ctas == 0 && pl.hot_ctas == 0) {    // nothing cached: the output is zero
+    if (cudaMemsetAsync(out, 0, sizeof(float) * cf.batch * cf.num_q_heads * d, stream) != cudaSuccess)
+      return TQ_ERR_CUDA;
+    return TQ_OK;
   }
-  if (pl.cold_ctas + pl.hot_ctas > 0) {
-    AttendArgs a{};
-    a.q = (const __half*)q;
-    a.qrot = qrot;
-    a.qsk = qsk;
-    a.qscale = qscale;
-    a.hot_k = c->hot_k();
-    a.hot_v = c->hot_v();
-    a.cold = c->cold;
-    a.part = part;
-    a.status = c->status();
-    a.L = c->L;
-    a.units = units;
-    a.G = G;
-    a.Hq = cf.num_q_heads;
-    a.Hkv = cf.num_kv_heads;
-    a.W = cf.hot_window;
-    a.n_hot = c->n_hot;
-    a.n_cold = c->n_cold;
-    a.plan = pl;
-    a.log2e_sigma = (float)(1.4426950408889634 * (double)sigma);
-    if (c->ev_start && cudaEventRecord(c->ev_start, stream) != cudaSuccess) return TQ_ERR_CUDA;
-    if (launch_attend(a, stream) != cudaSuccess) return TQ_ERR_CUDA;
-    if (c->ev_stop && cudaEventRecord(c->ev_stop, stream) != cudaSuccess) return TQ_ERR_CUDA;
-  }
+  QPrepArgs qa{};
+  qa.q = (const __half*)q;
+  qa.signs = c->signs();
+  qa.St = c->St();
+  qa.qrot = qrot;
+  qa.qsk = qsk;
+  qa.qscale = qscale;
+  qa.heads = cf.batch * cf.num_q_heads;
+  qa.d = d;
+  qa.m = cf.qjl_bits;
+  if (launch_qprep(qa, stream) != cudaSuccess) return TQ_ERR_CUDA;
+  AttendArgs a{};
+  a.q = (const __half*)q;
+  a.qrot = qrot;
+  a.qsk = qsk;
+  a.qscale = qscale;
+  a.hot_k = c->hot_k();
+  a.hot_v = c->hot_v();
+  a.cold = c->cold;
+  a.part = part;
+  a.status = c->status();
+  a.L = c->L;
+  a.units = units;
+  a.G = cf.num_q_heads / cf.num_kv_heads;
+  a.Hq = cf.num_q_heads;
+  a.Hkv = cf.num_kv_heads;
+  a.W = cf.hot_window;
+  a.n_hot = c->n_hot;
+  a.n_cold = c->n_cold;
+  a.plan = pl;
+  a.log2e_sigma = (float)(1.4426950408889634 * (double)sigma);
+  if (c->ev_start && cudaEventRecord(c->ev_start, stream) != cudaSuccess) return TQ_ERR_CUDA;
+  if (launch_attend(a, stream) != cudaSuccess) return TQ_ERR_CUDA;
+  if (c->ev_stop && cudaEventRecord(c->ev_stop, stream) != cudaSuccess) return TQ_ERR_CUDA;
   CombineArgs ca{};
   ca.part = part;
   ca.signs = c->signs();
   ca.out = out;
   ca.units = units;
-  ca.G = G;
+  ca.G = a.G;
   ca.Hkv = cf.num_kv_heads;
   ca.Hq = cf.num_q_heads;
   ca.d = d;
@@ -388,6 +381,17 @@ tq_status tq_decode_attention(tq_cache* c, const void* q, float* out, float soft
   ca.batch = cf.batch;
   if (launch_combine(ca, stream) != cudaSuccess) return TQ_ERR_CUDA;
   return TQ_OK;
+}
+
+tq_status tq_decode_attention(tq_cache* c, const void* q, float* out, float softmax_scale,
+                              cudaStream_t stream) {
+  if (!c || !q || !out || !(softmax_scale >= 0.0f) || std::isinf(softmax_scale))
+    return TQ_ERR_INVALID_ARG;
+  const int units = c->cfg.batch * c->cfg.num_kv_heads;
+  const SplitPlan pl = make_plan(c->n_cold, c->n_hot, units, c->num_sms * c->ctas_per_sm, false);
+  return launch_decode(c, q, out, softmax_scale, pl, (__half*)(c->ws + c->W.qrot),
+                       (__half*)(c->ws + c->W.qsk), (float*)(c->ws + c->W.qscale),
+                       (float*)(c->ws + c->W.part), stream);
 }
 
 tq_status tq_set_attend_events(tq_cache* c, cudaEvent_t start, cudaEvent_t stop) {
@@ -443,7 +447,6 @@ tq_status tq_decode_attention_static(tq_cache* c, const void* q, float* out, flo
   const int heads = cf.batch * cf.num_q_heads;
   const int units = cf.batch * cf.num_kv_heads;
   const int G = cf.num_q_heads / cf.num_kv_heads;
-  const float sigma = softmax_scale == 0.0f ? (float)(1.0 / std::sqrt((double)d)) : softmax_scale;
 
   // The same split plan as tq_decode_attention, with the partial slots per
   // unit cut to the most any unit can receive under this plan.
@@ -460,60 +463,8 @@ tq_status tq_decode_attention_static(tq_cache* c, const void* q, float* out, flo
 
   uint8_t* base = (uint8_t*)static_scratch_address(current);
   if (!base) return TQ_ERR_CUDA;
-  __half* qrot = (__half*)(base + o_qrot);
-  __half* qsk = (__half*)(base + o_qsk);
-  float* qscale = (float*)(base + o_qscale);
-  float* part = (float*)(base + o_part);
-
-  if (pl.cold_ctas > 0) {
-    QPrepArgs qa{};
-    qa.q = (const __half*)q;
-    qa.signs = c->signs();
-    qa.St = c->St();
-    qa.qrot = qrot;
-    qa.qsk = qsk;
-    qa.qscale = qscale;
-    qa.heads = heads;
-    qa.d = d;
-    qa.m = m;
-    if (launch_qprep(qa, stream) != cudaSuccess) return TQ_ERR_CUDA;
-  }
-  if (pl.cold_ctas + pl.hot_ctas > 0) {
-    AttendArgs a{};
-    a.q = (const __half*)q;
-    a.qrot = qrot;
-    a.qsk = qsk;
-    a.qscale = qscale;
-    a.hot_k = c->hot_k();
-    a.hot_v = c->hot_v();
-    a.cold = c->cold;
-    a.part = part;
-    a.status = c->status();
-    a.L = c->L;
-    a.units = units;
-    a.G = G;
-    a.Hq = cf.num_q_heads;
-    a.Hkv = cf.num_kv_heads;
-    a.W = cf.hot_window;
-    a.n_hot = c->n_hot;
-    a.n_cold = c->n_cold;
-    a.plan = pl;
-    a.log2e_sigma = (float)(1.4426950408889634 * (double)sigma);
-    if (launch_attend(a, stream) != cudaSuccess) return TQ_ERR_CUDA;
-  }
-  CombineArgs ca{};
-  ca.part = part;
-  ca.signs = c->signs();
-  ca.out = out;
-  ca.units = units;
-  ca.G = G;
-  ca.Hkv = cf.num_kv_heads;
-  ca.Hq = cf.num_q_heads;
-  ca.d = d;
-  ca.plan = pl;
-  ca.batch = cf.batch;
-  if (launch_combine(ca, stream) != cudaSuccess) return TQ_ERR_CUDA;
-  return TQ_OK;
+  return launch_decode(c, q, out, softmax_scale, pl, (__half*)(base + o_qrot), (__half*)(base + o_qsk),
+                       (float*)(base + o_qscale), (float*)(base + o_part), stream);
 }
 
 tq_status tq_get_status(tq_cache* c, cudaStream_t stream) {
