@@ -7,14 +7,16 @@
 //                       float64 decision path of the KV encoder.
 //   vec_qprep_kernel    q' = R q, q'' = S q' written as the fp16 A operand of
 //                       the search MMAs, in the fragments' column order.
-//   search_kernel       per CTA: 64 queries x a contiguous run of database
-//                       vectors.  The database side is dequantized straight
-//                       into mma.sync B fragments (one shared LUT load per
-//                       polar pair, scaled by the vector's s16/(2^b_r-1);
-//                       sign bits become +-rn16*sqrt(pi/2)/m with one LOP3),
-//                       so each looked-up register feeds 4 MMAs.  Scores go
-//                       to shared memory and every thread keeps a running
-//                       top-k for half of one query's columns.
+//   search_kernel       per CTA (8 warps): 64 queries x a contiguous run of
+//                       database vectors.  The database side is dequantized
+//                       straight into mma.sync B fragments (one shared LUT
+//                       load per polar pair, scaled by the vector's
+//                       s16/(2^b_r-1); sign bits become +-rn16*sqrt(pi/2)/m
+//                       with one LOP3), so each looked-up register feeds 4
+//                       MMAs.  Each thread compares its accumulators with
+//                       its queries' current k-th best and appends only
+//                       better candidates to a per-query buffer, which a
+//                       warp re-selects when it could overflow.
 //   topk_merge_kernel   merges the per-split candidate lists.
 #include <cmath>
 #include <cstring>
@@ -29,7 +31,8 @@ namespace {
 using enc::encode_vector_any;
 using enc::kFull;
 constexpr int kQT = 64;                  // queries per CTA
-constexpr int kChunk = 128;              // database vectors per CTA step (32 per warp)
+constexpr int kListK = 16;               // best candidates kept per (query, split); k <= kListK
+constexpr int kMaxSplits = 32;           // database splits per search (grid y)
 constexpr float kNegInf = -INFINITY;
 
 __device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
@@ -178,6 +181,13 @@ __global__ void __launch_bounds__(256) vec_qprep_kernel(const VecQPrepArgs a) {
 // ---------------------------------------------------------------------------
 // search
 // ---------------------------------------------------------------------------
+// Per CTA: kQT = 64 queries (4 MMA m-tiles, A operand in shared memory)
+// against a contiguous run of the database, kStepVec = 128 vectors per step
+// (8 warps x 2 n-tiles of 8).  Scores never go to shared memory: each
+// thread compares its accumulators with the query's current k-th best
+// (`thr`) and appends only better candidates to the query's buffer; a warp
+// re-selects a query's k best whenever its buffer could overflow in the
+// next step.
 template <int D>
 struct SearchShape {
   static constexpr int P = D / 2;
@@ -186,17 +196,71 @@ struct SearchShape {
   static constexpr int KS_QJL = 16;           // QJL k-steps (256 sign slots)
   static constexpr int KA = D + 256;
   static constexpr int AS = KA + 8;           // padded A row (halves)
-  static constexpr int SCS = kChunk + 4;      // padded score row (floats)
-  static constexpr int SMEM = kQT * AS * 2 + kQT * SCS * 4;
+  static constexpr int WARPS = 8;
+  static constexpr int NJ = 2;                // n-tiles per warp per step
+  static constexpr int STEP = WARPS * NJ * 8; // vectors per step
+  static constexpr int CAP = kListK + STEP + 32;   // candidate slots per query
+  static constexpr int OFF_CAND = kQT * AS * 2;
+  static constexpr int OFF_CNT = OFF_CAND + kQT * CAP * 8;
+  static constexpr int OFF_THR = OFF_CNT + kQT * 4;
+  static constexpr int SMEM = OFF_THR + kQT * 4;
 };
 
+// Warp: replaces query q's candidates (n of them, (score, index) pairs) by
+// its best min(n, K), in order, and returns the new count; *thr becomes the
+// K-th best score (-inf while fewer than K are known).
+template <int CAP, int K>
+__device__ int select_top(float2* cand, int n, float* thr) {
+  constexpr int PER = (CAP + 31) / 32;
+  const int lane = threadIdx.x & 31;
+  float sv[PER];
+  int iv[PER];
+#pragma unroll
+  for (int r = 0; r < PER; ++r) {
+    const int e = r * 32 + lane;
+    const float2 c = e < n ? cand[e] : make_float2(kNegInf, 0.f);
+    sv[r] = c.x;
+    iv[r] = e < n ? __float_as_int(c.y) : 0x7fffffff;
+  }
+  __syncwarp();
+  const int keep = n < K ? n : K;
+  for (int k = 0; k < keep; ++k) {
+    // this lane's best, then the warp's (score desc, index asc)
+    float bs = sv[0];
+    int bi = iv[0], br = 0;
+#pragma unroll
+    for (int r = 1; r < PER; ++r)
+      if (better(sv[r], iv[r], bs, bi)) { bs = sv[r]; bi = iv[r]; br = r; }
+    float ws = bs;
+    int wi = bi;
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      const float os = __shfl_xor_sync(kFull, ws, o);
+      const int oi = __shfl_xor_sync(kFull, wi, o);
+      if (better(os, oi, ws, wi)) { ws = os; wi = oi; }
+    }
+    if (bs == ws && bi == wi) {          // the owner drops it from its registers
+#pragma unroll
+      for (int r = 0; r < PER; ++r)
+        if (r == br) { sv[r] = kNegInf; iv[r] = 0x7fffffff; }
+    }
+    if (lane == 0) cand[k] = make_float2(ws, __int_as_float(wi));
+  }
+  __syncwarp();
+  if (lane == 0) *thr = keep == K ? cand[K - 1].x : kNegInf;
+  __syncwarp();
+  return keep;
+}
+
 template <int D, int K>
-__global__ void __launch_bounds__(128, 1) search_kernel(const SearchArgs a) {
+__global__ void __launch_bounds__(256, 1) search_kernel(const SearchArgs a) {
   using S = SearchShape<D>;
   extern __shared__ __align__(16) uint8_t smem[];
   __shared__ __align__(16) uint32_t lut[256 * 32];
   __half* As = reinterpret_cast<__half*>(smem);
-  float* scores = reinterpret_cast<float*>(smem + kQT * S::AS * 2);
+  float2* cand = reinterpret_cast<float2*>(smem + S::OFF_CAND);
+  int* cnt = reinterpret_cast<int*>(smem + S::OFF_CNT);
+  float* thr = reinterpret_cast<float*>(smem + S::OFF_THR);
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int gid = lane >> 2, tig = lane & 3;
@@ -222,30 +286,25 @@ __global__ void __launch_bounds__(128, 1) search_kernel(const SearchArgs a) {
     if (r < nq_tile) v = *reinterpret_cast<const uint4*>(a.A + (size_t)(q0 + r) * S::KA + cc * 8);
     *reinterpret_cast<uint4*>(As + r * S::AS + cc * 8) = v;
   }
+  for (int q = tid; q < kQT; q += blockDim.x) {
+    cnt[q] = 0;
+    thr[q] = kNegInf;
+  }
   __syncthreads();
 
-  // running top-k of this thread: query tid / 2, columns of half tid % 2
-  float ts[K];
-  int ti[K];
-#pragma unroll
-  for (int j = 0; j < K; ++j) {
-    ts[j] = kNegInf;
-    ti[j] = 0x7fffffff;
-  }
-  const int my_q = tid >> 1, my_half = tid & 1;
   const uint32_t a_base = smem_addr(As);
   const int mi = lane >> 3, rr = lane & 7;
   const uint32_t lane4 = (uint32_t)lane * 4u;
   const char* lutb = reinterpret_cast<const char*>(lut);
 
-  for (int64_t c0 = v_lo; c0 < v_hi; c0 += kChunk) {
-    // ---- B operand data for this warp's 4 n-tiles (8 vectors each) ------
-    uint32_t cw[4][S::PT / 4];
-    uint32_t sg[4][2];
-    uint32_t sa[4], sb[4];
+  for (int64_t c0 = v_lo; c0 < v_hi; c0 += S::STEP) {
+    // ---- B operand data for this warp's n-tiles (8 vectors each) --------
+    uint32_t cw[S::NJ][S::PT / 4];
+    uint32_t sg[S::NJ][2];
+    uint32_t sa[S::NJ], sb[S::NJ];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int64_t v = c0 + warp * 32 + j * 8 + gid;
+    for (int j = 0; j < S::NJ; ++j) {
+      const int64_t v = c0 + warp * (8 * S::NJ) + j * 8 + gid;
       if (v < v_hi) {
         const uint32_t* cp = reinterpret_cast<const uint32_t*>(a.codes + v * S::P + S::PT * tig);
 #pragma unroll
@@ -265,14 +324,14 @@ __global__ void __launch_bounds__(128, 1) search_kernel(const SearchArgs a) {
         for (int k = 0; k < S::PT / 4; ++k) cw[j][k] = 0u;
         sg[j][0] = sg[j][1] = 0u;
         sa[j] = 0u;
-        sb[j] = 0u;        // +-0: padded vectors score 0 (masked below)
+        sb[j] = 0u;        // +-0: vectors past the run score 0 (not appended below)
       }
     }
-    float acc[4][4][4];
+    float acc[4][S::NJ][4];
 #pragma unroll
     for (int m = 0; m < 4; ++m)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) acc[m][j][0] = acc[m][j][1] = acc[m][j][2] = acc[m][j][3] = 0.f;
+      for (int j = 0; j < S::NJ; ++j) acc[m][j][0] = acc[m][j][1] = acc[m][j][2] = acc[m][j][3] = 0.f;
 
     // ---- polar part ----------------------------------------------------
 #pragma unroll
@@ -282,7 +341,7 @@ __global__ void __launch_bounds__(128, 1) search_kernel(const SearchArgs a) {
       for (int m = 0; m < 4; ++m)
         ldsm_x4(af[m], a_base + ((16 * m + rr + (mi & 1) * 8) * S::AS + 16 * s + (mi >> 1) * 8) * 2);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
+      for (int j = 0; j < S::NJ; ++j) {
         const uint32_t w = cw[j][(2 * s) / 4];
         const uint32_t c0b = (w >> (8 * ((2 * s) % 4))) & 0xffu;
         const uint32_t c1b = (w >> (8 * ((2 * s + 1) % 4))) & 0xffu;
@@ -301,7 +360,7 @@ __global__ void __launch_bounds__(128, 1) search_kernel(const SearchArgs a) {
         ldsm_x4(af[m], a_base + ((16 * m + rr + (mi & 1) * 8) * S::AS + D + 16 * s + (mi >> 1) * 8) * 2);
       const int u = 2 * (s % 8);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
+      for (int j = 0; j < S::NJ; ++j) {
         const uint32_t x = sg[j][s / 8];
         const uint32_t b0 = ((x << u) & 0x80008000u) ^ sb[j];
         const uint32_t b1 = ((x << (u + 1)) & 0x80008000u) ^ sb[j];
@@ -309,55 +368,49 @@ __global__ void __launch_bounds__(128, 1) search_kernel(const SearchArgs a) {
         for (int m = 0; m < 4; ++m) mma16816(acc[m][j], af[m][0], af[m][1], af[m][2], af[m][3], b0, b1);
       }
     }
-    // ---- scores -> shared; per-thread running top-k ----------------------
+    // ---- candidates: scores at least the query's current k-th best -------
 #pragma unroll
-    for (int m = 0; m < 4; ++m)
+    for (int m = 0; m < 4; ++m) {
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int col = warp * 32 + j * 8 + 2 * tig;
-        float* r0 = scores + (16 * m + gid) * S::SCS + col;
-        float* r1 = scores + (16 * m + gid + 8) * S::SCS + col;
-        r0[0] = acc[m][j][0];
-        r0[1] = acc[m][j][1];
-        r1[0] = acc[m][j][2];
-        r1[1] = acc[m][j][3];
-      }
-    __syncthreads();
-    if (my_q < nq_tile) {
-      const float* row = scores + my_q * S::SCS + my_half * (kChunk / 2);
-      for (int cc = 0; cc < kChunk / 2; ++cc) {
-        const int64_t v = c0 + my_half * (kChunk / 2) + cc;
-        if (v >= v_hi) break;
-        float sv = row[cc];
-        if (!better(sv, (int)v, ts[K - 1], ti[K - 1])) continue;
-        int iv = (int)v;
+      for (int r2 = 0; r2 < 2; ++r2) {
+        const int q = 16 * m + gid + 8 * r2;
+        if (q >= nq_tile) continue;
+        const float t = thr[q];
 #pragma unroll
-        for (int j = 0; j < K; ++j) {      // bubble the candidate into place
-          if (better(sv, iv, ts[j], ti[j])) {
-            const float t = ts[j];
-            const int ii = ti[j];
-            ts[j] = sv;
-            ti[j] = iv;
-            sv = t;
-            iv = ii;
+        for (int j = 0; j < S::NJ; ++j) {
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            const int64_t v = c0 + warp * (8 * S::NJ) + j * 8 + 2 * tig + c;
+            const float sc = acc[m][j][2 * r2 + c];
+            if (v < v_hi && sc >= t) {
+              const int pos = atomicAdd(&cnt[q], 1);
+              cand[q * S::CAP + pos] = make_float2(sc, __int_as_float((int)v));
+            }
           }
         }
       }
     }
     __syncthreads();
+    // ---- re-select where the next step could overflow a buffer ----------
+    for (int q = warp; q < nq_tile; q += S::WARPS) {
+      const int n = cnt[q];
+      if (n > S::CAP - S::STEP) cnt[q] = select_top<S::CAP, K>(cand + q * S::CAP, n, thr + q);
+    }
+    __syncthreads();
   }
-  // ---- write this thread's list -------------------------------------------
-  if (my_q < nq_tile) {
-    const size_t base = (((size_t)(q0 + my_q) * gridDim.y + blockIdx.y) * 2 + my_half) * K;
-#pragma unroll
-    for (int j = 0; j < K; ++j) {
-      a.part_s[base + j] = ts[j];
-      a.part_i[base + j] = ti[j];
+  // ---- this CTA's list per query --------------------------------------------
+  for (int q = warp; q < nq_tile; q += S::WARPS) {
+    const int n = select_top<S::CAP, K>(cand + q * S::CAP, cnt[q], thr + q);
+    const size_t base = ((size_t)(q0 + q) * gridDim.y + blockIdx.y) * K;
+    for (int j = lane; j < K; j += 32) {
+      const float2 c = j < n ? cand[q * S::CAP + j] : make_float2(kNegInf, __int_as_float(0x7fffffff));
+      a.part_s[base + j] = c.x;
+      a.part_i[base + j] = __float_as_int(c.y);
     }
   }
 }
 
-// One thread per query: the k best of its nsplit * 2 candidate lists.
+// One thread per query: the k best of its nsplit candidate lists.
 template <int K>
 __global__ void topk_merge_kernel(const MergeArgs a) {
   const int q = blockIdx.x * blockDim.x + threadIdx.x;
@@ -369,7 +422,7 @@ __global__ void topk_merge_kernel(const MergeArgs a) {
     ts[j] = kNegInf;
     ti[j] = 0x7fffffff;
   }
-  const int lists = a.nsplit * 2;
+  const int lists = a.nsplit;
   const size_t base = (size_t)q * lists * K;
   for (int e = 0; e < lists * K; ++e) {
     float sv = a.part_s[base + e];
@@ -411,11 +464,11 @@ cudaError_t launch_vec_encode_d(const VecEncodeArgs& a, cudaStream_t s) {
 template <int D>
 cudaError_t launch_search_d(const SearchArgs& a, cudaStream_t s) {
   using S = SearchShape<D>;
-  if (cudaFuncSetAttribute(search_kernel<D, 16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(search_kernel<D, kListK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            S::SMEM) != cudaSuccess)
     return cudaErrorInvalidValue;
   dim3 grid((a.nq + kQT - 1) / kQT, a.nsplit);
-  search_kernel<D, 16><<<grid, 128, S::SMEM, s>>>(a);
+  search_kernel<D, kListK><<<grid, 32 * S::WARPS, S::SMEM, s>>>(a);
   return cudaGetLastError();
 }
 
@@ -464,9 +517,6 @@ namespace tq {
 namespace {
 
 constexpr size_t kVAlign = 256;
-constexpr int kMaxSplits = 32;
-constexpr int kListK = 16;
-
 size_t vround(size_t x) { return (x + kVAlign - 1) / kVAlign * kVAlign; }
 
 int pad_dim(int d_in) {
@@ -502,8 +552,8 @@ VecWsLayout vec_ws_layout(int d, int m, int max_q) {
   w.St = off;     off += vround(sizeof(float) * (size_t)d * m);
   w.A = off;      off += vround((size_t)2 * max_q * (d + 256));
   w.qscale = off; off += vround(sizeof(float) * max_q);
-  w.part_s = off; off += vround(sizeof(float) * (size_t)max_q * kMaxSplits * 2 * kListK);
-  w.part_i = off; off += vround(sizeof(int) * (size_t)max_q * kMaxSplits * 2 * kListK);
+  w.part_s = off; off += vround(sizeof(float) * (size_t)max_q * kMaxSplits * kListK);
+  w.part_i = off; off += vround(sizeof(int) * (size_t)max_q * kMaxSplits * kListK);
   w.total = off;
   return w;
 }
