@@ -370,103 +370,123 @@ constexpr float kPRange = 100.f;
 
 // Per-warp softmax / accumulator state for one unit: the reference `ref`
 // (log2 domain) of the numerators p = 2^(l - ref) summed in `l_run`, and
-// the accumulators O of the V weights p * s16_v.
-template <int NT>
+// the accumulators O of the V weights p * s16_v.  A lane holds HPL query
+// heads: 2 (heads 2 tig, 2 tig + 1: an MMA column per head) or 1 (head
+// tig: the packed layout, where columns 2 tig and 2 tig + 1 carry the same
+// head and the O columns are duplicates).
+template <int NT, int HPL>
 struct WarpState {
-  float ref[2], l_run[2];
+  float ref[HPL], l_run[HPL];
   float O[NT][4];
   __device__ __forceinline__ void reset() {
-    ref[0] = ref[1] = kNegInf;
-    l_run[0] = l_run[1] = 0.f;
+#pragma unroll
+    for (int h = 0; h < HPL; ++h) {
+      ref[h] = kNegInf;
+      l_run[h] = 0.f;
+    }
 #pragma unroll
     for (int i = 0; i < NT; ++i) O[i][0] = O[i][1] = O[i][2] = O[i][3] = 0.f;
   }
 };
 
 // Online softmax over one 16-token tile with a lazily moved reference.
-// l2: log2-domain logits of tokens gid (l2[0..1]) and gid + 8 (l2[2..3]) for
-// the thread's two heads; sv0 / sv1: the two tokens' V weights (the V
+// l2: log2-domain logits, entry j for token gid + 8 (j / HPL) and the
+// lane's head j % HPL; sv0 / sv1: the two tokens' V weights (the V
 // record's s16, or 1 for hot tokens).  Produces p = 2^(l2 - ref) (added to
 // l_run) and pv = p * sv (the V weights).  The reference moves -- one warp
 // reduction, and a rescale of the sums -- only when some pv would exceed
 // 2^8 or some p 2^100, so every pv fits fp16.
-template <int NT>
-__device__ __forceinline__ void softmax_step(WarpState<NT>& st, const float (&l2)[4], float sv0,
-                                             float sv1, float (&pv)[4]) {
-  const float sv[4] = {sv0, sv0, sv1, sv1};
-  float p[4];
+template <int NT, int HPL>
+__device__ __forceinline__ void softmax_step(WarpState<NT, HPL>& st, const float (&l2)[2 * HPL],
+                                             float sv0, float sv1, float (&pv)[2 * HPL]) {
+  constexpr int J = 2 * HPL;
+  float p[J];
   bool ok = true;
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    p[j] = fast_exp2(l2[j] - st.ref[j & 1]);
-    pv[j] = p[j] * sv[j];
+  for (int j = 0; j < J; ++j) {
+    p[j] = fast_exp2(l2[j] - st.ref[j % HPL]);
+    pv[j] = p[j] * (j < HPL ? sv0 : sv1);
     ok &= (pv[j] <= kPvMax) & (p[j] <= kPMax);   // false for NaN (no reference yet)
   }
   if (!__all_sync(kFull, ok)) {
     // new reference: max over the tile of max(l2 + log2 sv, l2 - 100)
-    float t[2] = {kNegInf, kNegInf};
+    float t[HPL];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float tau = fmaxf(l2[j] + fast_log2(sv[j]), l2[j] - kPRange);
-      t[j & 1] = fmaxf(t[j & 1], tau);
+    for (int h = 0; h < HPL; ++h) t[h] = kNegInf;
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+      const float tau = fmaxf(l2[j] + fast_log2(j < HPL ? sv0 : sv1), l2[j] - kPRange);
+      t[j % HPL] = fmaxf(t[j % HPL], tau);
     }
 #pragma unroll
-    for (int o = 4; o < 32; o <<= 1) {
-      t[0] = fmaxf(t[0], __shfl_xor_sync(kFull, t[0], o));
-      t[1] = fmaxf(t[1], __shfl_xor_sync(kFull, t[1], o));
-    }
-    float corr[2];
+    for (int o = 4; o < 32; o <<= 1)
 #pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      const float nr = fmaxf(st.ref[hh], t[hh]);
-      corr[hh] = st.ref[hh] == kNegInf ? 0.f : fast_exp2(st.ref[hh] - nr);
-      st.ref[hh] = nr;
-      st.l_run[hh] *= corr[hh];
+      for (int h = 0; h < HPL; ++h) t[h] = fmaxf(t[h], __shfl_xor_sync(kFull, t[h], o));
+    float corr[HPL];
+#pragma unroll
+    for (int h = 0; h < HPL; ++h) {
+      const float nr = fmaxf(st.ref[h], t[h]);
+      corr[h] = st.ref[h] == kNegInf ? 0.f : fast_exp2(st.ref[h] - nr);
+      st.ref[h] = nr;
+      st.l_run[h] *= corr[h];
     }
 #pragma unroll
     for (int i = 0; i < NT; ++i) {
-      st.O[i][0] *= corr[0]; st.O[i][1] *= corr[1]; st.O[i][2] *= corr[0]; st.O[i][3] *= corr[1];
+      st.O[i][0] *= corr[0]; st.O[i][1] *= corr[HPL - 1];
+      st.O[i][2] *= corr[0]; st.O[i][3] *= corr[HPL - 1];
     }
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      p[j] = fast_exp2(l2[j] - st.ref[j & 1]);
-      pv[j] = p[j] * sv[j];
+    for (int j = 0; j < J; ++j) {
+      p[j] = fast_exp2(l2[j] - st.ref[j % HPL]);
+      pv[j] = p[j] * (j < HPL ? sv0 : sv1);
     }
   }
-  st.l_run[0] += p[0] + p[2];
-  st.l_run[1] += p[1] + p[3];
+#pragma unroll
+  for (int h = 0; h < HPL; ++h) st.l_run[h] += p[h] + p[HPL + h];
+}
+
+// The PV MMA's B fragments (P^T: tokens x head columns) from the V weights.
+template <int HPL>
+__device__ __forceinline__ void pv_fragments(const float (&pv)[2 * HPL], uint32_t& pb0, uint32_t& pb1) {
+  if constexpr (HPL == 2) {
+    pb0 = movmatrix_trans(pack_h2(pv[0], pv[1]));
+    pb1 = movmatrix_trans(pack_h2(pv[2], pv[3]));
+  } else {                     // the head's weight in both of its columns
+    pb0 = movmatrix_trans(pack_h2(pv[0], pv[0]));
+    pb1 = movmatrix_trans(pack_h2(pv[1], pv[1]));
+  }
 }
 
 // Merges the 4 warps' states into one partial {m, l, o[D]} per head and
-// writes it to `dst` ([G][D + 2]).  Lane (gid, tig) holds heads 2*tig + hh
-// (heads >= G are dropped).  Called by all threads of the CTA; uses the
-// merge area: per-warp m / l, then per-warp o rows summed by the threads.
-template <int D, int NT>
-__device__ __forceinline__ void flush_partial(WarpState<NT>& st, bool hot, float inv_levels, int G,
+// writes it to `dst` ([G][D + 2]).  Lane (gid, tig) holds heads
+// HPL * tig + hh (heads >= G are dropped).  Called by all threads of the
+// CTA; uses the merge area: per-warp m / l, then per-warp o rows summed by
+// the threads.
+template <int D, int NT, int HPL>
+__device__ __forceinline__ void flush_partial(WarpState<NT, HPL>& st, bool hot, float inv_levels, int G,
                                               float* merge, float* dst) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int gid = lane >> 2, tig = lane & 3;
 #pragma unroll
-  for (int o = 4; o < 32; o <<= 1) {
-    st.l_run[0] += __shfl_xor_sync(kFull, st.l_run[0], o);
-    st.l_run[1] += __shfl_xor_sync(kFull, st.l_run[1], o);
-  }
+  for (int o = 4; o < 32; o <<= 1)
+#pragma unroll
+    for (int h = 0; h < HPL; ++h) st.l_run[h] += __shfl_xor_sync(kFull, st.l_run[h], o);
   float* mw = merge;          // [4 warps][8 heads]
   float* lw = merge + 32;
   float* ow = merge + 64;     // [8 heads][D]
   if (gid == 0) {
 #pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      mw[warp * 8 + 2 * tig + hh] = st.ref[hh];
-      lw[warp * 8 + 2 * tig + hh] = st.l_run[hh];
+    for (int hh = 0; hh < HPL; ++hh) {
+      mw[warp * 8 + HPL * tig + hh] = st.ref[hh];
+      lw[warp * 8 + HPL * tig + hh] = st.l_run[hh];
     }
   }
   for (int i = tid; i < 8 * D; i += kThreads) ow[i] = 0.f;
   __syncthreads();
-  float f[2];
+  float f[HPL];
 #pragma unroll
-  for (int hh = 0; hh < 2; ++hh) {
-    const int g = 2 * tig + hh;
+  for (int hh = 0; hh < HPL; ++hh) {
+    const int g = HPL * tig + hh;
     float mx = kNegInf;
 #pragma unroll
     for (int w = 0; w < 4; ++w) mx = fmaxf(mx, mw[w * 8 + g]);
@@ -482,8 +502,8 @@ __device__ __forceinline__ void flush_partial(WarpState<NT>& st, bool hot, float
         for (int r2 = 0; r2 < 2; ++r2) {
           const int dim = hot ? (16 * i + gid + 8 * r2) : (2 * (P8 * gid + i) + r2);
 #pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            const int g = 2 * tig + hh;
+          for (int hh = 0; hh < HPL; ++hh) {
+            const int g = HPL * tig + hh;
             if (g < G && f[hh] != 0.f) ow[g * D + dim] += st.O[i][2 * r2 + hh] * f[hh];
           }
         }
@@ -556,7 +576,8 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
   };
   const SplitPlan& pl = a.plan;
   const int slots = pl.slots_cold + pl.slots_hot;
-  WarpState<S::NT> st;
+  constexpr int HPL = PACK ? 1 : 2;      // query heads per lane on the cold path
+  WarpState<S::NT, HPL> st;
   st.reset();
 
   const int c = blockIdx.x;
@@ -618,7 +639,7 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
     //   PACK:  bq = [q'_hi | q'_lo] by column, bq2 = [q'_hi | q'_hi]
     //   else:  bq = q'_hi, bq2 = q'_lo
     uint32_t bq[S::NT][2], bq2[S::NT][2], qs[S::QS][2];
-    float kpol[2], kqjl[2];
+    float kpol[HPL], kqjl[HPL];
     int unit_cur = -1;
     int slot_cur = 0;
     bool aborted = false;
@@ -633,7 +654,7 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
       }
       if (unit != unit_cur) {
         if (unit_cur >= 0) {
-          flush_partial<D, S::NT>(st, false, inv_levels, G, merge,
+          flush_partial<D, S::NT, HPL>(st, false, inv_levels, G, merge,
                                   a.part + (((size_t)unit_cur * slots + slot_cur) * G) * (D + 2));
           st.reset();
         }
@@ -641,21 +662,27 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
         slot_cur = c - (int)(((int64_t)unit * nb) / pl.cold_bpc);
         const int b = unit / a.Hkv, kvh = unit % a.Hkv;
         const int head0 = b * a.Hq + kvh * G;
-        const int hcol = PACK ? (gid & 3) : gid;       // head of this lane's B column
+        // B column gid: head gid (8 heads) or, packed, head gid / 2 with
+        // column parity 0 = q'_hi, 1 = q'_lo (QJL and the A_lo product use
+        // the even columns only)
+        const int hcol = PACK ? (gid >> 1) : gid;
+        const bool odd = PACK && (gid & 1);
         if (hcol < G) {
           const uint32_t* qp = reinterpret_cast<const uint32_t*>(a.qrot + (size_t)(head0 + hcol) * 2 * D) + S::PT * tig;
           const uint32_t* qk = reinterpret_cast<const uint32_t*>(a.qsk + (size_t)(head0 + hcol) * M) + tig * (M / 8);
-          const int o1 = (PACK && gid >= 4) ? S::P : 0;
-          const int o2 = PACK ? 0 : S::P;
+          const int o1 = odd ? S::P : 0;
 #pragma unroll
           for (int s = 0; s < S::NT; ++s) {
             bq[s][0] = qp[o1 + 2 * s];
             bq[s][1] = qp[o1 + 2 * s + 1];
-            bq2[s][0] = qp[o2 + 2 * s];
-            bq2[s][1] = qp[o2 + 2 * s + 1];
+            bq2[s][0] = odd ? 0u : qp[(PACK ? 0 : S::P) + 2 * s];
+            bq2[s][1] = odd ? 0u : qp[(PACK ? 0 : S::P) + 2 * s + 1];
           }
 #pragma unroll
-          for (int s = 0; s < S::QS; ++s) { qs[s][0] = qk[2 * s]; qs[s][1] = qk[2 * s + 1]; }
+          for (int s = 0; s < S::QS; ++s) {
+            qs[s][0] = odd ? 0u : qk[2 * s];
+            qs[s][1] = odd ? 0u : qk[2 * s + 1];
+          }
         } else {
 #pragma unroll
           for (int s = 0; s < S::NT; ++s) bq[s][0] = bq[s][1] = bq2[s][0] = bq2[s][1] = 0u;
@@ -663,8 +690,8 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
           for (int s = 0; s < S::QS; ++s) qs[s][0] = qs[s][1] = 0u;
         }
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const int g = (PACK ? 2 * (tig & 1) : 2 * tig) + hh;
+        for (int hh = 0; hh < HPL; ++hh) {
+          const int g = HPL * tig + hh;
           kpol[hh] = g < G ? a.log2e_sigma * a.qscale[2 * (head0 + g)] * inv_levels : 0.f;
           kqjl[hh] = g < G ? a.log2e_sigma * kSqrtHalfPi / (float)M * a.qscale[2 * (head0 + g) + 1] : 0.f;
         }
@@ -705,7 +732,7 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
         const uint2 a3 = make_uint2(lut_hi(o3), lut_lo(o3));
         mma16816(c1[s % kAccSplit], a0.x, a1.x, a2.x, a3.x, bq[s][0], bq[s][1]);
         if constexpr (PACK) {
-          mma16816(c2[s % kAccSplit], a0.y, a1.y, a2.y, a3.y, bq2[s][0], bq2[s][1]);
+          mma16816(c1[s % kAccSplit], a0.y, a1.y, a2.y, a3.y, bq2[s][0], bq2[s][1]);
         } else {
           mma16816(c2[s % kAccSplit], a0.x, a1.x, a2.x, a3.x, bq2[s][0], bq2[s][1]);
           mma16816(c2[s % kAccSplit], a0.y, a1.y, a2.y, a3.y, bq[s][0], bq[s][1]);
@@ -737,26 +764,28 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
       float cp[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        float h1 = c1[0][j], h2 = c2[0][j];
+        cp[j] = c1[0][j] + c2[0][j];
 #pragma unroll
-        for (int k = 1; k < kAccSplit; ++k) {
-          h1 += c1[k][j];
-          h2 += c2[k][j];
-        }
-        cp[j] = (PACK ? h1 + __shfl_xor_sync(kFull, h1, 2) : h1) + h2;
+        for (int k = 1; k < kAccSplit; ++k) cp[j] += c1[k][j] + c2[k][j];
       }
-      float l2[4];
-      l2[0] = v0 ? fmaf(rn0 * kqjl[0], cq0[0] + cq1[0], sk0 * kpol[0] * cp[0]) : kNegInf;
-      l2[1] = v0 ? fmaf(rn0 * kqjl[1], cq0[1] + cq1[1], sk0 * kpol[1] * cp[1]) : kNegInf;
-      l2[2] = v1 ? fmaf(rn1 * kqjl[0], cq0[2] + cq1[2], sk1 * kpol[0] * cp[2]) : kNegInf;
-      l2[3] = v1 ? fmaf(rn1 * kqjl[1], cq0[3] + cq1[3], sk1 * kpol[1] * cp[3]) : kNegInf;
+      // entry j: token gid + 8 (j / HPL), head j % HPL
+      float l2[2 * HPL];
+      if constexpr (PACK) {       // columns 2 tig (hi) and 2 tig + 1 (lo) of head tig
+        l2[0] = v0 ? fmaf(rn0 * kqjl[0], cq0[0] + cq1[0], sk0 * kpol[0] * (cp[0] + cp[1])) : kNegInf;
+        l2[1] = v1 ? fmaf(rn1 * kqjl[0], cq0[2] + cq1[2], sk1 * kpol[0] * (cp[2] + cp[3])) : kNegInf;
+      } else {
+        l2[0] = v0 ? fmaf(rn0 * kqjl[0], cq0[0] + cq1[0], sk0 * kpol[0] * cp[0]) : kNegInf;
+        l2[1] = v0 ? fmaf(rn0 * kqjl[1], cq0[1] + cq1[1], sk0 * kpol[1] * cp[1]) : kNegInf;
+        l2[2] = v1 ? fmaf(rn1 * kqjl[0], cq0[2] + cq1[2], sk1 * kpol[0] * cp[2]) : kNegInf;
+        l2[3] = v1 ? fmaf(rn1 * kqjl[1], cq0[3] + cq1[3], sk1 * kpol[1] * cp[3]) : kNegInf;
+      }
       // V weights of tokens past the end are 0 (their records are not written)
       const float sv0 = v0 ? __half2float(__ushort_as_half((unsigned short)(vsc & 0xffffu))) : 0.f;
       const float sv1 = v1 ? __half2float(__ushort_as_half((unsigned short)(vsc >> 16))) : 0.f;
-      float pv[4];
+      float pv[2 * HPL];
       softmax_step(st, l2, sv0, sv1, pv);
-      const uint32_t pb0 = movmatrix_trans(pack_h2(pv[0], pv[1]));
-      const uint32_t pb1 = movmatrix_trans(pack_h2(pv[2], pv[3]));
+      uint32_t pb0, pb1;
+      pv_fragments<HPL>(pv, pb0, pb1);
 
       // ---- P V: V codes of pairs PV*gid + j for tokens 2tig, 2tig+1, +8, +9
 #pragma unroll
@@ -802,7 +831,7 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
     // with PACK, lanes tig >= 2 duplicate the heads of lanes tig - 2;
     // flush_partial keeps head 2 * tig + hh < G <= 4 only, i.e. tig < 2
     if (unit_cur >= 0) {
-      flush_partial<D, S::NT>(st, false, inv_levels, G, merge,
+      flush_partial<D, S::NT, HPL>(st, false, inv_levels, G, merge,
                               a.part + (((size_t)unit_cur * slots + slot_cur) * G) * (D + 2));
       st.reset();
     }
@@ -814,6 +843,8 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
     const int64_t f_lo = (int64_t)c * pl.hot_tpc;
     const int64_t f_hi = f_lo + pl.hot_tpc < total ? f_lo + pl.hot_tpc : total;
     constexpr int CH = D / 8;        // 16-byte chunks per token row
+    WarpState<S::NT, 2> sh;          // hot logits use one MMA column per head
+    sh.reset();
     uint32_t qh[S::NT][2];
     int unit_cur = -1, slot_cur = 0;
     int unit = (int)(f_lo / ht);
@@ -825,9 +856,9 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
       }
       if (unit != unit_cur) {
         if (unit_cur >= 0) {
-          flush_partial<D, S::NT>(st, true, inv_levels, G, merge,
+          flush_partial<D, S::NT, 2>(sh, true, inv_levels, G, merge,
                                   a.part + (((size_t)unit_cur * slots + slot_cur) * G) * (D + 2));
-          st.reset();
+          sh.reset();
         }
         unit_cur = unit;
         slot_cur = pl.slots_cold + (c - (int)(((int64_t)unit * ht) / pl.hot_tpc));
@@ -879,9 +910,8 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
         l2[2] = v1 ? a.log2e_sigma * cc4[2] : kNegInf;
         l2[3] = v1 ? a.log2e_sigma * cc4[3] : kNegInf;
         float pv[4];
-        softmax_step(st, l2, 1.f, 1.f, pv);
-        pb0 = movmatrix_trans(pack_h2(pv[0], pv[1]));
-        pb1 = movmatrix_trans(pack_h2(pv[2], pv[3]));
+        softmax_step(sh, l2, 1.f, 1.f, pv);
+        pv_fragments<2>(pv, pb0, pb1);
       }
       stage_rows(a.hot_v);
       if (live) {
@@ -889,13 +919,13 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
         for (int j = 0; j < S::NT; ++j) {
           uint32_t af[4];
           ldsm_x4_trans(af, base + (tb + rr + (mi >> 1) * 8) * S::RS + (16 * j + (mi & 1) * 8) * 2);
-          mma16816(st.O[j], af[0], af[1], af[2], af[3], pb0, pb1);
+          mma16816(sh.O[j], af[0], af[1], af[2], af[3], pb0, pb1);
         }
       }
     }
     if (unit_cur >= 0) {
       __syncthreads();
-      flush_partial<D, S::NT>(st, true, inv_levels, G, merge,
+      flush_partial<D, S::NT, 2>(sh, true, inv_levels, G, merge,
                               a.part + (((size_t)unit_cur * slots + slot_cur) * G) * (D + 2));
     }
   }
