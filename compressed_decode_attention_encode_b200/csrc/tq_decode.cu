@@ -203,7 +203,18 @@ __device__ __forceinline__ uint32_t lut_offset(const uint32_t (&w)[NW], int pos,
 // the rotation).
 // ---------------------------------------------------------------------------
 template <int D, int M>
+__device__ __forceinline__ void qprep_body(const QPrepArgs& a);
+
+template <int D, int M>
 __global__ void __launch_bounds__(256) qprep_kernel(const QPrepArgs a) {
+  qprep_body<D, M>(a);
+  // launched as a programmatic dependent of the previous kernel: finish
+  // only after that kernel has (its writes visible to what follows q-prep)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+template <int D, int M>
+__device__ __forceinline__ void qprep_body(const QPrepArgs& a) {
   constexpr int E = D / 32;
   constexpr int HB = 256 / M;            // heads per block
   __shared__ float sq[HB][D];
@@ -1087,8 +1098,21 @@ cudaError_t launch_qprep_dm(const QPrepArgs& a, cudaStream_t s) {
         cudaFuncSetAttribute(qprep_kernel<D, M>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
   }
-  qprep_kernel<D, M><<<grid, 256, smem, s>>>(a);
-  return cudaGetLastError();
+  // Programmatic dependent launch: q-prep reads only the query and S^T,
+  // so it may overlap the kernel before it (the eviction encode); it waits
+  // for that kernel before it exits, so work after q-prep still finds the
+  // encode complete.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, qprep_kernel<D, M>, a);
 }
 
 cudaError_t launch_qprep(const QPrepArgs& a, cudaStream_t s) {

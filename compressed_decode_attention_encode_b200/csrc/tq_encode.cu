@@ -236,6 +236,9 @@ __global__ void __launch_bounds__(2 * D) encode_small_kernel(EncodeArgs a) {
   const int64_t e = blockIdx.x % n;
   const int tid = threadIdx.x, team = tid / D, el = tid % D;
   const int lane = tid & 31, wt = el >> 5;
+  // A following launch that opted in (the decode step's q-prep, which does
+  // not read what this kernel writes) may start now.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   extern __shared__ double sm[];
   double* xb = sm + team * D;                                  // [2][D] exchange / residual
   double* red = sm + 2 * D;                                    // [2][NW] reductions
