@@ -334,13 +334,28 @@ def run_gpu(args, wl):
     launches_per_step = L * (1 + 3)   # evict: per-token encode (ring write fused); decode: qprep, attend, combine
 
     # ---- e2e: host buffers through the public API ------------------------
-    hk = [[x.cpu().pin_memory() for x in knew[l]] for l in range(L)]
-    hv = [[x.cpu().pin_memory() for x in vnew[l]] for l in range(L)]
-    hq = [x.cpu().pin_memory() for x in qs]
-    hout = [torch.empty(o.shape, dtype=torch.float32).pin_memory() for o in outs]
-    dk = [torch.empty_like(knew[0][0]) for _ in range(L)]
-    dv = [torch.empty_like(vnew[0][0]) for _ in range(L)]
-    dq = [torch.empty_like(qs[0]) for _ in range(L)]
+    # Each step's inputs (every layer's new K, V token and queries) travel in
+    # one host->device copy from pinned memory, and the step's outputs come
+    # back in one device->host copy.
+    kn, vn, qn = knew[0][0].numel(), vnew[0][0].numel(), qs[0].numel()
+    per_layer = kn + vn + qn
+    nsteps_in = len(knew[0])
+    hin = torch.empty((nsteps_in, L * per_layer), dtype=torch.float16).pin_memory()
+    for st_i in range(nsteps_in):
+        for l in range(L):
+            o = l * per_layer
+            hin[st_i, o:o + kn] = knew[l][st_i].reshape(-1).cpu()
+            hin[st_i, o + kn:o + kn + vn] = vnew[l][st_i].reshape(-1).cpu()
+            hin[st_i, o + kn + vn:o + per_layer] = qs[l].reshape(-1).cpu()
+    din = torch.empty((L * per_layer,), dtype=torch.float16, device=dev)
+    on = outs[0].numel()
+    dout = torch.empty((L, on), dtype=torch.float32, device=dev)
+    hout = torch.empty((L, on), dtype=torch.float32).pin_memory()
+    views = []
+    for l in range(L):
+        o = l * per_layer
+        views.append((din[o:o + kn].view(knew[0][0].shape), din[o + kn:o + kn + vn].view(vnew[0][0].shape),
+                      din[o + kn + vn:o + per_layer].view(qs[0].shape), dout[l].view(outs[0].shape)))
     e2e_steps = args.steps
     h2d = d2h = 0
     torch.cuda.synchronize()
@@ -349,20 +364,18 @@ def run_gpu(args, wl):
     e0.record(stream)
     e2e_keys = 0
     for _ in range(e2e_steps):
-        s = step_idx[0]
+        s = step_idx[0] % nsteps_in
         step_idx[0] += 1
-        h2d = d2h = 0
+        din.copy_(hin[s], non_blocking=True)
+        h2d = din.numel() * 2
         for l in range(L):
-            dk[l].copy_(hk[l][s], non_blocking=True)
-            dv[l].copy_(hv[l][s], non_blocking=True)
-            dq[l].copy_(hq[l], non_blocking=True)
-            h2d += 2 * dk[l].numel() * 2 + dq[l].numel() * 2
-            caches[l].evict_window(dk[l], dv[l])
+            dk, dv, dq, do = views[l]
+            caches[l].evict_window(dk, dv)
             nc, nh, _ = caches[l].counts()
             e2e_keys += units * (nc + nh)
-            caches[l].decode_attention(dq[l], out=outs[l])
-            hout[l].copy_(outs[l], non_blocking=True)
-            d2h += outs[l].numel() * 4
+            caches[l].decode_attention(dq, out=do)
+        hout.copy_(dout, non_blocking=True)
+        d2h = dout.numel() * 4
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
