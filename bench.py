@@ -59,6 +59,34 @@ def attend_traffic(same_workload: bool):
     return ATTEND_TRAFFIC.get(h) if same_workload else None
 
 
+# --------------------------------------------------------------------------
+# ranks: one process per GPU (torchrun); every rank runs the full per-GPU
+# workload (weak scaling, no data-path collective)
+# --------------------------------------------------------------------------
+def rank_env():
+    """(world size, rank, local rank) from the launcher's environment."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def max_over_ranks(x: float, device) -> float:
+    """The largest per-rank value over the process group (x with one rank):
+    a job's time is its slowest rank's."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(world: int, units_per_rank: float, ms_max: float) -> float:
+    """Whole-job rate of a weak-scaling run: every rank processes
+    `units_per_rank` in the slowest rank's `ms_max` milliseconds."""
+    return world * units_per_rank / (ms_max / 1e3)
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -167,8 +195,8 @@ def oracle_threads() -> int:
 
 
 def run_reference(args, wl):
-    rank = int(os.environ.get("RANK", "0"))
-    if rank != 0:
+    _, rank, _ = rank_env()
+    if rank != 0:              # the reference arm runs on rank 0 only
         return
     sample = oracle_sample(wl, args.seed, kv_heads=2)
     for _ in range(args.warmup):
@@ -217,9 +245,7 @@ def run_gpu(args, wl):
     from compressed_decode_attention_encode_b200 import build as B
     from compressed_decode_attention_encode_b200 import tq
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = rank_env()
     if world > 1:
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
@@ -327,10 +353,7 @@ def run_gpu(args, wl):
     for c in caches:
         if c.get_status() != 0:
             raise RuntimeError("device status in timed region")
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, dev)
     launches_per_step = L * (1 + 3)   # evict: per-token encode (ring write fused); decode: qprep, attend, combine
 
     # ---- e2e: host buffers through the public API ------------------------
@@ -379,13 +402,10 @@ def run_gpu(args, wl):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, dev)
 
-    value = world * keys_total / (ms / 1e3)
-    e2e_value = world * e2e_keys / (e2e_ms / 1e3)
+    value = job_rate(world, keys_total, ms)
+    e2e_value = job_rate(world, e2e_keys, e2e_ms)
     hbm_peak, peak_kind = peaks()
     attend_launches = L * args.steps
     achieved = bytes_total / (attend_ms / 1e3) / 1e9
@@ -454,9 +474,7 @@ def run_search(args, sw):
     from compressed_decode_attention_encode_b200 import tq
     from compressed_decode_attention_encode_b200.inputs import mixture_centres
 
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
+    world, rank, local = rank_env()
     if world > 1:
         import datetime
         import torch.distributed as dist
@@ -496,13 +514,9 @@ def run_search(args, sw):
     torch.cuda.synchronize()
     clocks = clock.stop()
     ms = t0.elapsed_time(t1) / args.steps
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, dev)
     ips = sw.n_queries * sw.n
-    value = world * ips / (ms / 1e3)
+    value = job_rate(world, ips, ms)
     # e2e: queries from pinned host memory, results back to the host
     hq = q.cpu().pin_memory()
     hs = torch.empty((sw.n_queries, sw.k), dtype=torch.float32).pin_memory()
@@ -518,7 +532,7 @@ def run_search(args, sw):
         hi.copy_(ix, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / args.steps
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dev)
     flops = 2.0 * ips * (256 + sw.qjl_bits)        # algorithmic: polar d=256 + m sign terms
     peak, peak_kind = _search_peak()
     achieved = flops / (ms / 1e3) / 1e12
@@ -532,7 +546,7 @@ def run_search(args, sw):
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": None, "kernel": "tq_ip_search (q-prep, search, merge)",
                      "peak_kind": peak_kind, "flop_per_step": flops},
-        "e2e": {"value": world * ips / (e2e_ms / 1e3), "unit": "inner products/s",
+        "e2e": {"value": job_rate(world, ips, e2e_ms), "unit": "inner products/s",
                 "h2d_bytes_per_step": q.numel() * 4, "d2h_bytes_per_step": sw.n_queries * sw.k * 8,
                 "ms_per_step": e2e_ms},
         "gpu_launches": 3 * args.steps,
