@@ -331,7 +331,8 @@ struct AttendShape {
   static constexpr int RS = 2 * D + 16;             // padded hot row stride (bytes)
   static constexpr int HOT_BYTES = TB * RS;          // one hot tile, K then V
   static constexpr int MERGE_BYTES = (64 + 8 * D) * 4;
-  static constexpr int BAR_BYTES = 8 * 8 + 8 * 8 + 16;   // up to 8 stages: barriers, counters, flags
+  // up to 8 stages per warp: 4 x 8 barriers, 4 x 8 copy counters, flags
+  static constexpr int BAR_BYTES = 4 * 8 * 8 + 4 * 8 * 4 + 16;
   // Dynamic shared memory: [ring | pad | LUT hi | LUT lo | merge | barriers],
   // laid out for a dynamic base at shared address kDynSmemBase.
   static constexpr int ring_bytes(int ns) { return ns * BLOCK > HOT_BYTES ? ns * BLOCK : HOT_BYTES; }
@@ -558,10 +559,12 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
   uint32_t* llo_w = lhi_w + S::NLUT * 32;
   uint8_t* ring = smem;
   float* merge = reinterpret_cast<float*>(smem + S::OFF_MERGE);
+  // Each warp streams its own tiles (tile `warp` of every block of the
+  // CTA's run) through its own NS-stage ring: barriers [4][NS], copies
+  // issued per stage [4][NS], and a CTA-wide abort flag.
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::OFF_BAR);
-  int* arrivals = reinterpret_cast<int*>(smem + S::OFF_BAR + 8 * S::NS);    // [NS] warps done
-  int* copies = arrivals + S::NS;                                           // [NS] copies issued
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(copies + S::NS);
+  int* copies_all = reinterpret_cast<int*>(smem + S::OFF_BAR + 8 * 4 * S::NS);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(copies_all + 4 * S::NS);
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int gid = lane >> 2, tig = lane & 3;
@@ -599,25 +602,30 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
     const int64_t f_lo = (int64_t)c * pl.cold_bpc;
     const int64_t f_hi = f_lo + pl.cold_bpc < total ? f_lo + pl.cold_bpc : total;
     const int nblk = (int)(f_hi - f_lo);
-    const uint32_t bar0 = smem_addr(bars);
-    const uint32_t ring0 = smem_addr(ring);
-    // f -> (unit, block) by division: used only for the NS initial copies;
-    // the loop and the refills advance (unit, blk) incrementally
-    auto src_of = [&](int64_t f) {
-      const int64_t u = f / nb, b = f % nb;
-      return a.cold + ((size_t)u * a.L.blocks_per_unit + (size_t)b) * S::BLOCK;
+    const int nbi = (int)nb;
+    const uint32_t bar_w = smem_addr(bars) + 8 * S::NS * warp;           // this warp's barriers
+    const uint32_t ring_w = smem_addr(ring) + S::NS * S::TT * warp;      // this warp's stages
+    int* copies = copies_all + S::NS * warp;                               // copies issued per stage
+    // this warp's tile of block b of unit u
+    auto tile_src = [&](int u, int b) {
+      return a.cold + ((size_t)u * a.L.blocks_per_unit + (size_t)b) * S::BLOCK + warp * S::TT;
     };
-    if (tid < S::NS) {
-      arrivals[tid] = 0;
-      copies[tid] = tid < nblk ? 1 : 0;
-    }
-    if (tid == 0) {
-      *abort_flag = 0;
-      for (int s = 0; s < S::NS; ++s) mbar_init(bar0 + 8 * s, 1);
+    if (tid == 0) *abort_flag = 0;
+    if (lane == 0) {
+      for (int s = 0; s < S::NS; ++s) mbar_init(bar_w + 8 * s, 1);
       fence_barrier_init();
-      for (int s = 0; s < S::NS && s < nblk; ++s) {
-        mbar_expect_tx(bar0 + 8 * s, S::BLOCK);
-        bulk_g2s(ring0 + s * S::BLOCK, src_of(f_lo + s), S::BLOCK, bar0 + 8 * s);
+      int u = (int)(f_lo / nb), b = (int)(f_lo - (int64_t)u * nb);
+      for (int s = 0; s < S::NS; ++s) {
+        copies[s] = 0;
+        if (s < nblk) {
+          mbar_expect_tx(bar_w + 8 * s, S::TT);
+          bulk_g2s(ring_w + s * S::TT, tile_src(u, b), S::TT, bar_w + 8 * s);
+          copies[s] = 1;
+        }
+        if (++b == nbi) {
+          b = 0;
+          ++u;
+        }
       }
     }
     // LUTs of 'unit' pair reconstructions c_r * (cos, sin)(2 pi c_th / 2^b_th):
@@ -656,7 +664,6 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
     bool aborted = false;
     int unit = (int)(f_lo / nb);          // advanced incrementally: no division per block
     int blk = (int)(f_lo - (int64_t)unit * nb);   // block inside the unit (< 2^31)
-    const int nbi = (int)nb;
     const int tail = (int)(a.n_cold - (int64_t)(nbi - 1) * S::TB);   // valid tokens of a unit's last block
     for (int i = 0; i < nblk; ++i, ++blk) {
       if (blk == nbi) {
@@ -707,10 +714,10 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
           kqjl[hh] = g < G ? a.log2e_sigma * kSqrtHalfPi / (float)M * a.qscale[2 * (head0 + g) + 1] : 0.f;
         }
       }
-      // ---- wait for this block's stage (every warp on its own) ----------
+      // ---- wait for this tile's stage of the warp's ring --------------------
       const int stage = i % S::NS;
       if (!aborted) {
-        const bool got = mbar_wait_bounded(bar0 + 8 * stage, (uint32_t)((i / S::NS) & 1));
+        const bool got = mbar_wait_bounded(bar_w + 8 * stage, (uint32_t)((i / S::NS) & 1));
         if (!__all_sync(kFull, got)) {
           aborted = true;
           if (lane == 0) *abort_flag = 1;
@@ -719,7 +726,7 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
       const int left = (blk == nbi - 1 ? tail : S::TB) - tb;
       if (!aborted && left > 0) {
       const int nvalid = left < 16 ? (int)left : 16;     // valid tokens of this warp's tile
-      const uint32_t tile = ring0 + stage * S::BLOCK + warp * S::TT;
+      const uint32_t tile = ring_w + stage * S::TT;
 
       uint32_t kw[S::KWT], sw[S::SW], vw[S::VWT];
       load_lane_words<S::KWT>(tile + S::OFF_KC, lane, kw);
@@ -809,34 +816,26 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
                  __byte_perm(L2, L3, 0x5410), __byte_perm(L2, L3, 0x7632), pb0, pb1);
       }
       }   // tile compute
-      // ---- release the stage; the last of the 4 warps refills it ----------
+      // ---- refill the stage with this warp's tile of block i + NS --------
       __syncwarp();
-      if (lane == 0) {
-        __threadfence_block();
-        const int old = atomicAdd(&arrivals[stage], 1);
-        if ((old & 3) == 3 && i + S::NS < nblk && !*abort_flag) {
-          __threadfence_block();
-          fence_proxy_async();
-          mbar_expect_tx(bar0 + 8 * stage, S::BLOCK);
-          int pb = blk + S::NS;              // block i + NS: at most NS past (unit, blk)
-          int pu = unit;
-          while (pb >= nbi) { pb -= nbi; ++pu; }
-          bulk_g2s(ring0 + stage * S::BLOCK,
-                   a.cold + ((size_t)pu * a.L.blocks_per_unit + (size_t)pb) * S::BLOCK, S::BLOCK,
-                   bar0 + 8 * stage);
-          copies[stage] += 1;
-        }
+      if (lane == 0 && !aborted && i + S::NS < nblk) {
+        fence_proxy_async();
+        int pb = blk + S::NS;              // block i + NS: at most NS past (unit, blk)
+        int pu = unit;
+        while (pb >= nbi) { pb -= nbi; ++pu; }
+        mbar_expect_tx(bar_w + 8 * stage, S::TT);
+        bulk_g2s(ring_w + stage * S::TT, tile_src(pu, pb), S::TT, bar_w + 8 * stage);
+        copies[stage] += 1;
       }
     }
     __syncthreads();
     if (*abort_flag) {
       // A bulk copy did not complete in time: latch the error, give the
       // copies still in flight a bounded chance to land, and leave.
-      if (tid == 0) {
-        atomicOr(a.status, kStatusTimeout);
+      if (tid == 0) atomicOr(a.status, kStatusTimeout);
+      if (lane == 0)
         for (int s = 0; s < S::NS; ++s)
-          if (copies[s] > 0) mbar_wait_bounded(bar0 + 8 * s, (uint32_t)((copies[s] - 1) & 1));
-      }
+          if (copies[s] > 0) mbar_wait_bounded(bar_w + 8 * s, (uint32_t)((copies[s] - 1) & 1));
       return;
     }
     // with PACK, lanes tig >= 2 duplicate the heads of lanes tig - 2;
