@@ -40,7 +40,6 @@ constexpr int kSmemPerSm = 233472;     // shared memory per SM (bytes)
 // for the system.  The attention kernel checks it and reports a layout
 // error rather than reading a misaligned table.
 constexpr int kDynSmemBase = 1024;
-constexpr int kAccSplit = 1;           // independent accumulator chains per tile product
 constexpr float kNegInf = -INFINITY;
 constexpr float kSqrtHalfPi = 1.2533141373155001f;   // sqrt(pi / 2)
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // bounded mbarrier waits
@@ -655,9 +654,12 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
     __syncthreads();
 
     // B operands of the K-logit MMAs (per k-step) and of the QJL MMAs.
-    //   PACK:  bq = [q'_hi | q'_lo] by column, bq2 = [q'_hi | q'_hi]
+    //   PACK:  bq = q'_hi / q'_lo in the even / odd column of each head; both
+    //          A_hi and A_lo multiply it (the odd column's A_lo q'_lo term is
+    //          2^-22 of the logit, and makes the product exact)
     //   else:  bq = q'_hi, bq2 = q'_lo
-    uint32_t bq[S::NT][2], bq2[S::NT][2], qs[S::QS][2];
+    constexpr int kAccSplit = PACK ? 2 : 1;    // independent accumulator chains
+    uint32_t bq[S::NT][2], bq2[PACK ? 1 : S::NT][2], qs[S::QS][2];
     float kpol[HPL], kqjl[HPL];
     int unit_cur = -1;
     int slot_cur = 0;
@@ -693,8 +695,10 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
           for (int s = 0; s < S::NT; ++s) {
             bq[s][0] = qp[o1 + 2 * s];
             bq[s][1] = qp[o1 + 2 * s + 1];
-            bq2[s][0] = odd ? 0u : qp[(PACK ? 0 : S::P) + 2 * s];
-            bq2[s][1] = odd ? 0u : qp[(PACK ? 0 : S::P) + 2 * s + 1];
+            if constexpr (!PACK) {
+              bq2[s][0] = qp[S::P + 2 * s];
+              bq2[s][1] = qp[S::P + 2 * s + 1];
+            }
           }
 #pragma unroll
           for (int s = 0; s < S::QS; ++s) {
@@ -703,7 +707,11 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
           }
         } else {
 #pragma unroll
-          for (int s = 0; s < S::NT; ++s) bq[s][0] = bq[s][1] = bq2[s][0] = bq2[s][1] = 0u;
+          for (int s = 0; s < S::NT; ++s) bq[s][0] = bq[s][1] = 0u;
+          if constexpr (!PACK) {
+#pragma unroll
+            for (int s = 0; s < S::NT; ++s) bq2[s][0] = bq2[s][1] = 0u;
+          }
 #pragma unroll
           for (int s = 0; s < S::QS; ++s) qs[s][0] = qs[s][1] = 0u;
         }
@@ -750,7 +758,7 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
         const uint2 a3 = make_uint2(lut_hi(o3), lut_lo(o3));
         mma16816(c1[s % kAccSplit], a0.x, a1.x, a2.x, a3.x, bq[s][0], bq[s][1]);
         if constexpr (PACK) {
-          mma16816(c1[s % kAccSplit], a0.y, a1.y, a2.y, a3.y, bq2[s][0], bq2[s][1]);
+          mma16816(c1[s % kAccSplit], a0.y, a1.y, a2.y, a3.y, bq[s][0], bq[s][1]);
         } else {
           mma16816(c2[s % kAccSplit], a0.x, a1.x, a2.x, a3.x, bq2[s][0], bq2[s][1]);
           mma16816(c2[s % kAccSplit], a0.y, a1.y, a2.y, a3.y, bq[s][0], bq[s][1]);
