@@ -963,6 +963,9 @@ __global__ void combine_kernel(const CombineArgs a) {
   __shared__ float sw[kCombineMaxSlots];     // per-slot weight 2^(m_s - m)
   __shared__ float red[2][8];
   __shared__ float xbuf[256];
+  // The next step's eviction encode may start its prologue now (it waits
+  // for this kernel before reading its inputs).
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int hg = blockIdx.x;
   const int b = hg / a.Hq, hq = hg % a.Hq;
   const int kvh = hq / a.G, g = hq % a.G;

@@ -247,6 +247,10 @@ __global__ void __launch_bounds__(2 * D) encode_small_kernel(EncodeArgs a) {
   uint16_t* sc = reinterpret_cast<uint16_t*>(bits + 4);        // s16_k, rn16, s16_v
   float* sst = reinterpret_cast<float*>(sm) + small_st_offset(D) / 4;   // S^T [D][m]
   async_copy_g2s(sst, a.St, D * L.m * 4);      // lands while the rotation and polar steps run
+  // Launched as a programmatic dependent of the kernel before it: S^T (set
+  // at cache creation) may be fetched early, the inputs only once that
+  // kernel has finished.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   const __half* src;
   if (e < a.nA) {
@@ -445,8 +449,17 @@ cudaError_t launch_encode_d(const EncodeArgs& a, cudaStream_t s) {
                                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       if (e != cudaSuccess) return e;
     }
-    encode_small_kernel<D><<<(unsigned)(a.units * n), 2 * D, smem, s>>>(a);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(a.units * n));
+    cfg.blockDim = dim3(2 * D);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, encode_small_kernel<D>, a);
   }
   const int64_t tiles = (a.cold_start + n - 1) / kTokensPerTile - a.cold_start / kTokensPerTile + 1;
   const int64_t jobs = (int64_t)a.units * tiles * 4;
