@@ -330,8 +330,8 @@ struct AttendShape {
   static constexpr int RS = 2 * D + 16;             // padded hot row stride (bytes)
   static constexpr int HOT_BYTES = TB * RS;          // one hot tile, K then V
   static constexpr int MERGE_BYTES = (64 + 8 * D) * 4;
-  // up to 8 stages per warp: 4 x 8 barriers, 4 x 8 copy counters, flags
-  static constexpr int BAR_BYTES = 4 * 8 * 8 + 4 * 8 * 4 + 16;
+  // up to 8 stages per warp: 4 x 8 barriers, the abort flag
+  static constexpr int BAR_BYTES = 4 * 8 * 8 + 16;
   // Dynamic shared memory: [ring | pad | LUT hi | LUT lo | merge | barriers],
   // laid out for a dynamic base at shared address kDynSmemBase.
   static constexpr int ring_bytes(int ns) { return ns * BLOCK > HOT_BYTES ? ns * BLOCK : HOT_BYTES; }
@@ -559,11 +559,10 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
   uint8_t* ring = smem;
   float* merge = reinterpret_cast<float*>(smem + S::OFF_MERGE);
   // Each warp streams its own tiles (tile `warp` of every block of the
-  // CTA's run) through its own NS-stage ring: barriers [4][NS], copies
-  // issued per stage [4][NS], and a CTA-wide abort flag.
+  // CTA's run) through its own NS-stage ring: barriers [4][NS], and a
+  // CTA-wide abort flag.
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::OFF_BAR);
-  int* copies_all = reinterpret_cast<int*>(smem + S::OFF_BAR + 8 * 4 * S::NS);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(copies_all + 4 * S::NS);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + S::OFF_BAR + 8 * 4 * S::NS);
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int gid = lane >> 2, tig = lane & 3;
@@ -604,28 +603,32 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
     const int nbi = (int)nb;
     const uint32_t bar_w = smem_addr(bars) + 8 * S::NS * warp;           // this warp's barriers
     const uint32_t ring_w = smem_addr(ring) + S::NS * S::TT * warp;      // this warp's stages
-    int* copies = copies_all + S::NS * warp;                               // copies issued per stage
-    // this warp's tile of block b of unit u
-    auto tile_src = [&](int u, int b) {
-      return a.cold + ((size_t)u * a.L.blocks_per_unit + (size_t)b) * S::BLOCK + warp * S::TT;
+    // The warp's tile stream: `nsrc` is the next tile to fetch (block
+    // `nblk_b` of its unit); it advances a block at a time and skips a
+    // unit's unused blocks at the unit's end.  `issued` counts the copies.
+    const uint8_t* nsrc;
+    int nblk_b = 0, issued = 0;
+    const size_t unit_gap = (size_t)(a.L.blocks_per_unit - nb) * S::BLOCK;
+    {
+      const int64_t u = f_lo / nb;
+      nblk_b = (int)(f_lo - u * nb);
+      nsrc = a.cold + ((size_t)u * a.L.blocks_per_unit + (size_t)nblk_b) * S::BLOCK + warp * S::TT;
+    }
+    auto fetch_next = [&](int s) {       // lane 0: the next tile into stage s
+      mbar_expect_tx(bar_w + 8 * s, S::TT);
+      bulk_g2s(ring_w + s * S::TT, nsrc, S::TT, bar_w + 8 * s);
+      ++issued;
+      nsrc += S::BLOCK;
+      if (++nblk_b == nbi) {
+        nblk_b = 0;
+        nsrc += unit_gap;
+      }
     };
     if (tid == 0) *abort_flag = 0;
     if (lane == 0) {
       for (int s = 0; s < S::NS; ++s) mbar_init(bar_w + 8 * s, 1);
       fence_barrier_init();
-      int u = (int)(f_lo / nb), b = (int)(f_lo - (int64_t)u * nb);
-      for (int s = 0; s < S::NS; ++s) {
-        copies[s] = 0;
-        if (s < nblk) {
-          mbar_expect_tx(bar_w + 8 * s, S::TT);
-          bulk_g2s(ring_w + s * S::TT, tile_src(u, b), S::TT, bar_w + 8 * s);
-          copies[s] = 1;
-        }
-        if (++b == nbi) {
-          b = 0;
-          ++u;
-        }
-      }
+      for (int s = 0; s < S::NS && s < nblk; ++s) fetch_next(s);
     }
     // LUTs of 'unit' pair reconstructions c_r * (cos, sin)(2 pi c_th / 2^b_th):
     // keys as fp16 hi + lo (the lo part removes the fp16 rounding of the
@@ -828,12 +831,7 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
       __syncwarp();
       if (lane == 0 && !aborted && i + S::NS < nblk) {
         fence_proxy_async();
-        int pb = blk + S::NS;              // block i + NS: at most NS past (unit, blk)
-        int pu = unit;
-        while (pb >= nbi) { pb -= nbi; ++pu; }
-        mbar_expect_tx(bar_w + 8 * stage, S::TT);
-        bulk_g2s(ring_w + stage * S::TT, tile_src(pu, pb), S::TT, bar_w + 8 * stage);
-        copies[stage] += 1;
+        fetch_next(stage);
       }
     }
     __syncthreads();
@@ -841,9 +839,11 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
       // A bulk copy did not complete in time: latch the error, give the
       // copies still in flight a bounded chance to land, and leave.
       if (tid == 0) atomicOr(a.status, kStatusTimeout);
-      if (lane == 0)
-        for (int s = 0; s < S::NS; ++s)
-          if (copies[s] > 0) mbar_wait_bounded(bar_w + 8 * s, (uint32_t)((copies[s] - 1) & 1));
+      if (lane == 0)             // stage s received copies s, s + NS, ...: wait for its last one
+        for (int s = 0; s < S::NS && s < issued; ++s) {
+          const int n_s = (issued - s + S::NS - 1) / S::NS;
+          mbar_wait_bounded(bar_w + 8 * s, (uint32_t)((n_s - 1) & 1));
+        }
       return;
     }
     // with PACK, lanes tig >= 2 duplicate the heads of lanes tig - 2;
