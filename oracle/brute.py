@@ -132,3 +132,22 @@ def decode_one_head(q, hot_k, hot_v, cold_k, cold_v, signs, S, b_r, b_theta, sig
             acc[2 * j + 1] += w * rec["cr"][j] * math.sin(a)
     back = rotate_inverse(acc, signs)
     return [o[i] + back[i] for i in range(d)]
+
+
+def decode_one_head_gated(q, hot_k, hot_v, cold_k, cold_v, signs, S, b_r, b_theta, sigma,
+                          threshold):
+    """The cold tier is read only when the hot window is empty or its largest
+    plain score q.k is below ``threshold``; otherwise one softmax over the
+    hot tokens alone.  Returns (output, skipped)."""
+    d = len(q)
+    best = None
+    for k in hot_k:
+        sc = 0.0
+        for i in range(d):
+            sc += q[i] * k[i]
+        if best is None or sc > best:
+            best = sc
+    skipped = best is not None and best >= threshold
+    if skipped:
+        return decode_one_head(q, hot_k, hot_v, [], [], signs, S, b_r, b_theta, sigma), True
+    return decode_one_head(q, hot_k, hot_v, cold_k, cold_v, signs, S, b_r, b_theta, sigma), False

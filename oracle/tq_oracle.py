@@ -472,6 +472,43 @@ def decode_attention(q: np.ndarray, hot_k: np.ndarray, hot_v: np.ndarray,
     return out
 
 
+def hot_gate(q: np.ndarray, hot_k: np.ndarray, num_kv_heads: int, threshold: float) -> np.ndarray:
+    """Which query heads skip the cold tier (Monarch v3 page, section "Bucle
+    de Decodificación Simplificado": the cold pages are read only while the
+    largest hot score q.k stays below a threshold).
+
+    READINGS: the score is the plain product q.k over the hot window (the
+    loop computes it before any softmax scale); a head with an empty hot
+    window always reads the cold tier.  Returns a bool per query head, True
+    where max_t q.k_t >= threshold over a non-empty hot window.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    hq = q.shape[0]
+    g = hq // num_kv_heads
+    skip = np.zeros(hq, dtype=bool)
+    if hot_k is None or hot_k.shape[1] == 0:
+        return skip
+    for h in range(hq):
+        scores = np.asarray(hot_k[h // g], dtype=np.float64) @ q[h]
+        skip[h] = scores.max() >= threshold
+    return skip
+
+
+def decode_attention_gated(q: np.ndarray, hot_k: np.ndarray, hot_v: np.ndarray,
+                           cold_k: Optional[Codes], cold_v: Optional[Codes],
+                           signs: np.ndarray, S: Optional[np.ndarray], num_kv_heads: int,
+                           threshold: float, softmax_scale: Optional[float] = None):
+    """Decode attention with the threshold-gated cold tier (Monarch v3 page,
+    "Bucle de Decodificación Simplificado").  A head that ``hot_gate`` marks
+    attends to its hot window alone (one softmax over the hot tokens); every
+    other head is ``decode_attention`` over hot and cold.  Returns
+    (out [Hq, d], skip [Hq])."""
+    skip = hot_gate(q, hot_k, num_kv_heads, threshold)
+    full = decode_attention(q, hot_k, hot_v, cold_k, cold_v, signs, S, num_kv_heads, softmax_scale)
+    hot_only = decode_attention(q, hot_k, hot_v, None, None, signs, S, num_kv_heads, softmax_scale)
+    return np.where(skip[:, None], hot_only, full), skip
+
+
 def attention_reference(q: np.ndarray, k: np.ndarray, v: np.ndarray,
                         num_kv_heads: int, softmax_scale: Optional[float] = None) -> np.ndarray:
     """Textbook softmax(q K^T * sigma) V per query head, fp64 (GQA mapping)."""

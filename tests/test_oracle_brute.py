@@ -83,3 +83,36 @@ def test_inner_products_match_brute():
             rec = dict(s16=c.s16[t], cr=list(c.cr[t]), ct=list(c.ct[t]), rn16=c.rn16[t], bits=list(c.bits[t]))
             assert abs(sc[i, t] - B.key_ip(list(q[i]), list(signs), S.astype(np.float64).tolist(),
                                             rec, b_r, b_t)) < 1e-12
+
+
+@pytest.mark.parametrize("d,m,b", [(4, 4, 3), (8, 8, 4)])
+def test_gated_decode_matches_brute(d, m, b):
+    """Threshold-gated cold tier: per-head skip decisions and outputs of the
+    oracle against the loop-level restatement, at thresholds that split the
+    heads both ways."""
+    rng = np.random.default_rng(7 * d + b)
+    hq, hkv, nh, nc = 6, 2, 5, 7
+    q = rng.standard_normal((hq, d))
+    hk = rng.standard_normal((hkv, nh, d))
+    hv = rng.standard_normal((hkv, nh, d))
+    signs = O.rotation_signs(3, d)
+    S = O.qjl_matrix(3, m, d)
+    ck = [O.encode(rng.standard_normal((nc, d)), signs, S, b, b) for _ in range(hkv)]
+    cv = [O.encode(rng.standard_normal((nc, d)), signs, None, b, b) for _ in range(hkv)]
+    gmax = np.array([(hk[h // (hq // hkv)] @ q[h]).max() for h in range(hq)])
+    order = np.sort(gmax)
+    sigma = 0.7 / math.sqrt(d)
+    Sl = S.astype(np.float64).tolist()
+    for thr in (order[0] - 1.0, 0.5 * (order[2] + order[3]), order[-1] + 1.0, order[1]):
+        out, skip = O.decode_attention_gated(q, hk, hv, ck, cv, signs, S, hkv, thr, sigma)
+        for h in range(hq):
+            g = h // (hq // hkv)
+            recs_k = [dict(s16=ck[g].s16[t], cr=list(ck[g].cr[t]), ct=list(ck[g].ct[t]),
+                           rn16=ck[g].rn16[t], bits=list(ck[g].bits[t])) for t in range(nc)]
+            recs_v = [dict(s16=cv[g].s16[t], cr=list(cv[g].cr[t]), ct=list(cv[g].ct[t]))
+                      for t in range(nc)]
+            ref, ref_skip = B.decode_one_head_gated(list(q[h]), hk[g].tolist(), hv[g].tolist(),
+                                                    recs_k, recs_v, list(signs), Sl, b, b, sigma, thr)
+            assert ref_skip == skip[h]
+            np.testing.assert_allclose(out[h], ref, rtol=1e-12, atol=1e-12)
+        assert skip.sum() == (gmax >= thr).sum()

@@ -419,3 +419,56 @@ def test_top_k_matches_full_sort_with_index_tiebreak():
         order = sorted(range(500), key=lambda j: (-sc[i, j], j))[:10]
         assert list(idx[i]) == order
         np.testing.assert_array_equal(val[i], sc[i, order])
+
+
+# ---- threshold-gated cold tier (Monarch v3, simplified decode loop) ------
+
+def _gated_case(seed=11, d=16, m=16, b=3, hq=4, hkv=2, nh=6, nc=20):
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((hq, d))
+    hk = rng.standard_normal((hkv, nh, d))
+    hv = rng.standard_normal((hkv, nh, d))
+    signs = O.rotation_signs(5, d)
+    S = O.qjl_matrix(5, m, d)
+    ck = [O.encode(rng.standard_normal((nc, d)), signs, S, b, b) for _ in range(hkv)]
+    cv = [O.encode(rng.standard_normal((nc, d)), signs, None, b, b) for _ in range(hkv)]
+    return q, hk, hv, ck, cv, signs, S, hkv
+
+
+def test_gate_closed_is_plain_decode():
+    """A threshold above every hot score reads the cold tier for every head:
+    the gated output is the ungated one."""
+    q, hk, hv, ck, cv, signs, S, hkv = _gated_case()
+    out, skip = O.decode_attention_gated(q, hk, hv, ck, cv, signs, S, hkv, math.inf)
+    assert not skip.any()
+    np.testing.assert_array_equal(out, O.decode_attention(q, hk, hv, ck, cv, signs, S, hkv))
+
+
+def test_gate_open_is_textbook_hot_attention():
+    """A threshold of -inf skips the cold tier of every head with a hot
+    window: the output is textbook softmax attention over the hot tokens,
+    here written out with scipy's softmax."""
+    from scipy.special import softmax
+    q, hk, hv, ck, cv, signs, S, hkv = _gated_case()
+    out, skip = O.decode_attention_gated(q, hk, hv, ck, cv, signs, S, hkv, -math.inf)
+    assert skip.all()
+    d = q.shape[1]
+    for h in range(q.shape[0]):
+        g = h // (q.shape[0] // hkv)
+        p = softmax(hk[g] @ q[h] / math.sqrt(d))
+        np.testing.assert_allclose(out[h], p @ hv[g], rtol=1e-12, atol=1e-14)
+
+
+def test_gate_boundary_and_empty_hot_window():
+    """Equality with the threshold skips (the cold tier is read only below
+    it); an empty hot window always reads the cold tier."""
+    q, hk, hv, ck, cv, signs, S, hkv = _gated_case()
+    g = q.shape[0] // hkv
+    best = [float((hk[h // g] @ q[h]).max()) for h in range(q.shape[0])]
+    skip = O.hot_gate(q, hk, hkv, best[0])
+    assert skip[0]
+    assert list(skip) == [b >= best[0] for b in best]
+    empty = hk[:, :0]
+    out, skip = O.decode_attention_gated(q, empty, hv[:, :0], ck, cv, signs, S, hkv, -math.inf)
+    assert not skip.any()
+    np.testing.assert_array_equal(out, O.decode_attention(q, empty, hv[:, :0], ck, cv, signs, S, hkv))
