@@ -41,6 +41,8 @@ def parse():
     ap.add_argument("--layers", type=int, default=0, help="0: the workload's layer count")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--encode", action="store_true",
+                    help="time the prefill encode (tq_encode_append of 4096-token chunks) instead")
     return ap.parse_args()
 
 
@@ -455,6 +457,110 @@ def run_gpu(args, wl):
 
 
 # --------------------------------------------------------------------------
+# prefill encode: tq_encode_append of 4096-token chunks into one layer handle
+# --------------------------------------------------------------------------
+ENCODE_METRIC = "prefill encode token-heads/s (K and V of one token of one kv head)"
+FP64_PEAK_TFLOPS = 148 * 64 * 2 * 1965e6 / 1e12   # SMs x FP64 FMA/clk x 2 x max SM clock
+
+
+def run_encode(args, wl):
+    import torch
+
+    from compressed_decode_attention_encode_b200 import build as B
+    from compressed_decode_attention_encode_b200 import tq
+    from compressed_decode_attention_encode_b200.inputs import WORKLOADS  # noqa: F401
+
+    world, rank, local = rank_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if rank == 0:
+        B.build()
+    tq.lib()
+    chunk = 4096
+    nsteps = args.warmup + 2 * args.steps
+    cfg = tq.make_config(wl.batch, wl.num_q_heads, wl.num_kv_heads, wl.head_dim, wl.hot,
+                         nsteps * chunk, wl.b_r, wl.b_theta, wl.qjl_bits, seed=args.seed)
+    cache = tq.TQCache(cfg, device=dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1000 + rank)
+    k = gen_kv(wl, 0, args.seed, 0, wl.batch, 0, chunk, dev, gen)
+    v = gen_kv(wl, 0, args.seed, 1, wl.batch, 0, chunk, dev, gen)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        cache.encode_append(k, v)
+    torch.cuda.synchronize()
+    if cache.get_status() != 0:
+        raise RuntimeError("device status after warm-up")
+    clock = ClockSampler(local)
+    clock.start()
+    time.sleep(0.3)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        cache.encode_append(k, v)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clocks = clock.stop()
+    ms = max_over_ranks(t0.elapsed_time(t1) / args.steps, dev)
+    units = wl.batch * wl.num_kv_heads
+    per_step = units * chunk                        # token-heads (K and V) per append
+    value = job_rate(world, per_step, ms)
+    # e2e: the chunk from pinned host memory, then the device status back
+    hk = k.cpu().pin_memory()
+    hv = v.cpu().pin_memory()
+    dk, dv = torch.empty_like(k), torch.empty_like(v)
+    hstat = torch.empty(1, dtype=torch.int32).pin_memory()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        cache.encode_append(dk, dv)
+        hstat.copy_(cache.ws[:4].view(torch.int32), non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dev)
+    if cache.get_status() != 0:
+        raise RuntimeError("device status after timing")
+    kc = wl.head_dim // 2 * (wl.b_r + wl.b_theta) // 8
+    rec_bytes = 2 * kc + wl.qjl_bits // 8 + 6            # K and V records per token-head
+    flops = 2.0 * wl.qjl_bits * wl.head_dim * per_step   # S r in float64, one per key
+    achieved = flops / (ms / 1e3) / 1e12
+    result = {
+        "metric": ENCODE_METRIC, "value": value, "unit": "token-heads/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64 decisions, fp16 in", "data": "synthetic",
+        "config": {"workload": wl.name + "-prefill-encode", "batch": wl.batch,
+                   "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim, "chunk": chunk,
+                   "b_r": wl.b_r, "b_theta": wl.b_theta, "qjl_bits": wl.qjl_bits,
+                   "l2": "inputs 134 MB per chunk (> L2)"},
+        "records_gbs": value * rec_bytes / 1e9,
+        "roofline": {"bound": "alu", "achieved": achieved, "peak": FP64_PEAK_TFLOPS,
+                     "unit": "TFLOP/s (fp64)", "frac": achieved / FP64_PEAK_TFLOPS, "traffic": None,
+                     "kernel": "encode_kernel", "peak_kind": "derived: 148 SMs x 64 FP64 FMA/clk x 1965 MHz",
+                     "flop_per_step": flops},
+        "e2e": {"value": job_rate(world, per_step, e2e_ms), "unit": "token-heads/s",
+                "h2d_bytes_per_step": 2 * k.numel() * 2, "d2h_bytes_per_step": 4,
+                "ms_per_step": e2e_ms},
+        "gpu_launches": args.steps,
+        "clocks": clocks,
+    }
+    cache.close()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+# --------------------------------------------------------------------------
 # vector-search workload (1M x 200 database, 1024 queries, top-10)
 # --------------------------------------------------------------------------
 SEARCH_METRIC = "estimated inner products/s (vector search, top-10)"
@@ -592,6 +698,13 @@ def main():
         run_search(args, SEARCH_WORKLOADS[args.workload])
         return
     wl = WORKLOADS[args.workload]
+    if args.encode:
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable": "the encode reference arm is not "
+                              "timed; run the default workload"}))
+            return
+        run_encode(args, wl)
+        return
     if args.impl == "reference":
         run_reference(args, wl)
     else:
