@@ -41,6 +41,9 @@ def parse():
     ap.add_argument("--layers", type=int, default=0, help="0: the workload's layer count")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--gate-quantile", type=float, default=None,
+                    help="decode with the threshold-gated cold tier; each layer's threshold is this "
+                         "quantile of its heads' hot-window maxima q.k at the start")
     ap.add_argument("--encode", action="store_true",
                     help="time the prefill encode (tq_encode_append of 4096-token chunks) instead")
     return ap.parse_args()
@@ -50,7 +53,7 @@ def parse():
 # from an ncu capture, keyed by the SHA-1 of the kernel source it was taken
 # on; any other source reports null (the counters no longer describe it).
 ATTEND_TRAFFIC = {
-    "dddae1ebd5feb9ebb27854e51ebaae3717b16c00": 261383424 + 5899008,
+    "478e5ac804a02c25b454d732ad2890d24475ea8a": 261373184 + 4224000,
 }
 
 
@@ -300,6 +303,27 @@ def run_gpu(args, wl):
     cold_tok_bytes = 2 * kc + wl.qjl_bits // 8 + 6     # K and V record bytes
     hot_tok_bytes = 4 * wl.head_dim                     # K and V fp16
 
+    gate_tau = None
+    skip_bufs = None
+    if args.gate_quantile is not None:
+        # per-layer thresholds: a quantile of max_t q.k over each head's hot
+        # window (a configuration choice made once, outside the timed path)
+        G = wl.num_q_heads // wl.num_kv_heads
+        gate_tau = []
+        for l in range(L):
+            hk, _ = caches[l].hot_ring()
+            qf = qs[l].float().view(wl.batch, wl.num_kv_heads, G, wl.head_dim)
+            sc = torch.einsum("bhgd,bhtd->bhgt", qf, hk.float())
+            gate_tau.append(float(torch.quantile(sc.amax(dim=-1).flatten(), args.gate_quantile)))
+        skip_bufs = [torch.zeros((wl.batch, wl.num_q_heads), dtype=torch.int32, device=dev)
+                     for _ in range(L)]
+
+    def attend(l, q, out):
+        if gate_tau is None:
+            caches[l].decode_attention(q, out=out)
+        else:
+            caches[l].decode_attention_gated(q, gate_tau[l], out=out, head_skip=skip_bufs[l])
+
     step_idx = [0]
 
     def one_step(ev_pairs=None):
@@ -314,7 +338,7 @@ def run_gpu(args, wl):
             abytes += units * (nc * cold_tok_bytes + nh * hot_tok_bytes)
             if ev_pairs is not None:
                 caches[l].set_attend_events(*ev_pairs[l])
-            caches[l].decode_attention(qs[l], out=outs[l])
+            attend(l, qs[l], outs[l])
             if ev_pairs is not None:
                 caches[l].set_attend_events(None, None)
         return keys, abytes
@@ -356,7 +380,8 @@ def run_gpu(args, wl):
         if c.get_status() != 0:
             raise RuntimeError("device status in timed region")
     ms = max_over_ranks(ms, dev)
-    launches_per_step = L * (1 + 3)   # evict: per-token encode (ring write fused); decode: qprep, attend, combine
+    # evict: per-token encode (ring write fused); decode: qprep, [gate,] attend, combine
+    launches_per_step = L * (1 + 3 + (gate_tau is not None))
 
     # ---- e2e: host buffers through the public API ------------------------
     # Each step's inputs (every layer's new K, V token and queries) travel in
@@ -398,7 +423,7 @@ def run_gpu(args, wl):
             caches[l].evict_window(dk, dv)
             nc, nh, _ = caches[l].counts()
             e2e_keys += units * (nc + nh)
-            caches[l].decode_attention(dq, out=do)
+            attend(l, dq, do)
         hout.copy_(dout, non_blocking=True)
         d2h = dout.numel() * 4
     e1.record(stream)
@@ -435,7 +460,36 @@ def run_gpu(args, wl):
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if gate_tau is not None:
+        # what the gate skipped (last step's decisions) and what it changed:
+        # the gated output against the ungated one on the same cache state
+        G = wl.num_q_heads // wl.num_kv_heads
+        sk = torch.stack(skip_bufs).bool()                       # [L, B, Hq]
+        whole = sk.view(L, wl.batch, wl.num_kv_heads, G).all(dim=-1)
+        errs = []
+        for l in range(L):
+            a_ = caches[l].decode_attention(qs[l])
+            b_ = caches[l].decode_attention_gated(qs[l], gate_tau[l])
+            errs.append(((b_ - a_).norm(dim=-1) / a_.norm(dim=-1).clamp_min(1e-30)).flatten())
+        errs = torch.cat(errs)
+        nc, nh, _ = caches[0].counts()
+        read = (~whole).sum().item() * nc * cold_tok_bytes + L * units * nh * hot_tok_bytes
+        achieved_g = read / L / (attend_ms / attend_launches / 1e3) / 1e9
+        result["metric"] = "gated decode: context keys/s (cold tier read only below the hot-max threshold)"
+        result["config"]["gate_quantile"] = args.gate_quantile
+        result["gate"] = {
+            "thresholds_first_layers": gate_tau[:4],
+            "heads_skipped_frac": sk.float().mean().item(),
+            "units_skipped_frac": whole.float().mean().item(),
+            "out_rel_l2_vs_ungated": {"max": errs.max().item(), "mean": errs.mean().item(),
+                                      "heads_over_2e-3": int((errs > 2e-3).sum().item())},
+        }
+        result["roofline"].update({"achieved": achieved_g, "frac": achieved_g / hbm_peak,
+                                   "traffic": None,
+                                   "bytes_per_launch": read / L,
+                                   "bytes_note": "cold bytes of the units the last step read"})
+        result["hbm"] = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and gate_tau is None:
         sample = oracle_sample(wl, args.seed, kv_heads=1)
         time_oracle(sample)
         tt, kk = 0.0, 0

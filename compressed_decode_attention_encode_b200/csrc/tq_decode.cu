@@ -24,6 +24,10 @@
 //            fp16 tiles through padded shared memory (ldmatrix).
 //   combine  merges the partials of each (row, head), applies R^T once to
 //            the cold sum (Hadamard butterflies) and normalizes.
+// A gated call (tq_decode_attention_gated) runs the gate of tq_gate.cu
+// between qprep and attend; its attention kernel streams the cold blocks of
+// the listed units only, split again over the same CTAs, and combine leaves
+// out the cold partials of the heads that skipped.
 #include <cfloat>
 
 #include "tq_internal.cuh"
@@ -548,7 +552,7 @@ __device__ __forceinline__ void flush_partial(WarpState<NT, HPL>& st, bool hot, 
 // k-step instead of 3; lanes tig and tig ^ 2 then hold the same two heads
 // 2 * (tig & 1) + hh.  Without PACK (8 heads) lane (gid, tig) holds heads
 // 2 * tig + hh.
-template <int D, int M, int BW, bool PACK>
+template <int D, int M, int BW, bool PACK, bool GATE>
 __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(const AttendArgs a) {
   using S = AttendShape<D, M, BW>;
   extern __shared__ __align__(128) uint8_t smem[];
@@ -593,12 +597,28 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
   st.reset();
 
   const int c = blockIdx.x;
-  if (c < pl.cold_ctas) {
+  // Ungated: the cold runs cover every unit.  Gated: they cover the units
+  // of the active list (position p reads unit alist[p]), split again over
+  // at most the plan's cold CTAs.
+  int64_t g_bpc = 0, g_units = 0;
+  int g_ctas = 0;
+  if constexpr (GATE) {
+    g_units = *a.n_active;
+    gated_cold_split(g_units, pl.cold_blocks, pl.cold_ctas, &g_bpc, &g_ctas);
+  }
+  // (ungated, these stay reads of the launch parameters: no registers held)
+  auto cold_bpc = [&]() -> int64_t {
+    if constexpr (GATE) return g_bpc; else return pl.cold_bpc;
+  };
+  auto cold_units = [&]() -> int64_t {
+    if constexpr (GATE) return g_units; else return a.units;
+  };
+  if (c < (GATE ? g_ctas : pl.cold_ctas)) {
     // ============ cold run: blocks [c * bpc, (c + 1) * bpc) ============
     const int64_t nb = pl.cold_blocks;
-    const int64_t total = (int64_t)a.units * nb;
-    const int64_t f_lo = (int64_t)c * pl.cold_bpc;
-    const int64_t f_hi = f_lo + pl.cold_bpc < total ? f_lo + pl.cold_bpc : total;
+    const int64_t total = cold_units() * nb;
+    const int64_t f_lo = (int64_t)c * cold_bpc();
+    const int64_t f_hi = f_lo + cold_bpc() < total ? f_lo + cold_bpc() : total;
     const int nblk = (int)(f_hi - f_lo);
     const int nbi = (int)nb;
     const uint32_t bar_w = smem_addr(bars) + 8 * S::NS * warp;           // this warp's barriers
@@ -608,11 +628,14 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
     // unit's unused blocks at the unit's end.  `issued` counts the copies.
     const uint8_t* nsrc;
     int nblk_b = 0, issued = 0;
+    int fpos = 0;                        // gated: active-list position of nsrc's unit
     const size_t unit_gap = (size_t)(a.L.blocks_per_unit - nb) * S::BLOCK;
     {
       const int64_t u = f_lo / nb;
       nblk_b = (int)(f_lo - u * nb);
-      nsrc = a.cold + ((size_t)u * a.L.blocks_per_unit + (size_t)nblk_b) * S::BLOCK + warp * S::TT;
+      fpos = (int)u;
+      const int64_t uid = GATE ? (int64_t)a.alist[u] : u;
+      nsrc = a.cold + ((size_t)uid * a.L.blocks_per_unit + (size_t)nblk_b) * S::BLOCK + warp * S::TT;
     }
     auto fetch_next = [&](int s) {       // lane 0: the next tile into stage s
       mbar_expect_tx(bar_w + 8 * s, S::TT);
@@ -621,7 +644,10 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
       nsrc += S::BLOCK;
       if (++nblk_b == nbi) {
         nblk_b = 0;
-        nsrc += unit_gap;
+        if constexpr (GATE)   // alist[n_active] exists (and is 0) for the run's last step
+          nsrc = a.cold + (size_t)a.alist[++fpos] * a.L.blocks_per_unit * S::BLOCK + warp * S::TT;
+        else
+          nsrc += unit_gap;
       }
     };
     if (tid == 0) *abort_flag = 0;
@@ -664,7 +690,8 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
     constexpr int kAccSplit = PACK ? 2 : 1;    // independent accumulator chains
     uint32_t bq[S::NT][2], bq2[PACK ? 1 : S::NT][2], qs[S::QS][2];
     float kpol[HPL], kqjl[HPL];
-    int unit_cur = -1;
+    int unit_cur = -1;                    // active-list position when gated
+    int uid_cur = 0;                      // gated: the unit itself (alist[unit_cur])
     int slot_cur = 0;
     bool aborted = false;
     int unit = (int)(f_lo / nb);          // advanced incrementally: no division per block
@@ -678,12 +705,14 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
       if (unit != unit_cur) {
         if (unit_cur >= 0) {
           flush_partial<D, S::NT, HPL>(st, false, inv_levels, G, merge,
-                                  a.part + (((size_t)unit_cur * slots + slot_cur) * G) * (D + 2));
+                                  a.part + (((size_t)(GATE ? uid_cur : unit_cur) * slots + slot_cur) * G) * (D + 2));
           st.reset();
         }
         unit_cur = unit;
-        slot_cur = c - (int)(((int64_t)unit * nb) / pl.cold_bpc);
-        const int b = unit / a.Hkv, kvh = unit % a.Hkv;
+        if constexpr (GATE) uid_cur = a.alist[unit];
+        slot_cur = c - (int)(((int64_t)unit * nb) / cold_bpc());
+        const int uid = GATE ? uid_cur : unit;
+        const int b = uid / a.Hkv, kvh = uid % a.Hkv;
         const int head0 = b * a.Hq + kvh * G;
         // B column gid: head gid (8 heads) or, packed, head gid / 2 with
         // column parity 0 = q'_hi, 1 = q'_lo (QJL and the A_lo product use
@@ -850,7 +879,7 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
     // flush_partial keeps head 2 * tig + hh < G <= 4 only, i.e. tig < 2
     if (unit_cur >= 0) {
       flush_partial<D, S::NT, HPL>(st, false, inv_levels, G, merge,
-                              a.part + (((size_t)unit_cur * slots + slot_cur) * G) * (D + 2));
+                              a.part + (((size_t)(GATE ? uid_cur : unit_cur) * slots + slot_cur) * G) * (D + 2));
       st.reset();
     }
   }
@@ -977,7 +1006,17 @@ __global__ void combine_kernel(const CombineArgs a) {
   int nc = 0, nh = 0;
   if (pl.cold_ctas > 0 && pl.cold_blocks > 0) {
     const int64_t nb = pl.cold_blocks;
-    nc = (int)(((unit + 1) * nb - 1) / pl.cold_bpc - (unit * nb) / pl.cold_bpc + 1);
+    if (a.unit_pos == nullptr) {
+      nc = (int)(((unit + 1) * nb - 1) / pl.cold_bpc - (unit * nb) / pl.cold_bpc + 1);
+    } else if (!a.head_skip[hg]) {       // gated: this head reads its unit's cold runs
+      const int64_t p = a.unit_pos[unit];
+      if (p >= 0) {
+        int64_t bpc;
+        int ctas;
+        gated_cold_split(*a.n_active, nb, pl.cold_ctas, &bpc, &ctas);
+        nc = (int)(((p + 1) * nb - 1) / bpc - (p * nb) / bpc + 1);
+      }
+    }
   }
   if (pl.hot_ctas > 0 && pl.hot_tiles > 0) {
     const int64_t ht = pl.hot_tiles;
@@ -1057,32 +1096,33 @@ __global__ void combine_kernel(const CombineArgs a) {
 typedef void (*AttendFn)(const AttendArgs);
 
 template <int D, int M, int BW>
-AttendFn attend_fn(bool pack, int* smem) {
+AttendFn attend_fn(bool pack, bool gate, int* smem) {
   *smem = AttendShape<D, M, BW>::SMEM;
-  return pack ? attend_kernel<D, M, BW, true> : attend_kernel<D, M, BW, false>;
+  if (gate) return pack ? attend_kernel<D, M, BW, true, true> : attend_kernel<D, M, BW, false, true>;
+  return pack ? attend_kernel<D, M, BW, true, false> : attend_kernel<D, M, BW, false, false>;
 }
 
 template <int D, int M>
-AttendFn pick_bw(int bw, bool pack, int* smem) {
+AttendFn pick_bw(int bw, bool pack, bool gate, int* smem) {
   switch (bw) {
-    case 2: return attend_fn<D, M, 2>(pack, smem);
-    case 3: return attend_fn<D, M, 3>(pack, smem);
-    case 4: return attend_fn<D, M, 4>(pack, smem);
-    case 5: return attend_fn<D, M, 5>(pack, smem);
-    case 6: return attend_fn<D, M, 6>(pack, smem);
-    case 7: return attend_fn<D, M, 7>(pack, smem);
-    case 8: return attend_fn<D, M, 8>(pack, smem);
+    case 2: return attend_fn<D, M, 2>(pack, gate, smem);
+    case 3: return attend_fn<D, M, 3>(pack, gate, smem);
+    case 4: return attend_fn<D, M, 4>(pack, gate, smem);
+    case 5: return attend_fn<D, M, 5>(pack, gate, smem);
+    case 6: return attend_fn<D, M, 6>(pack, gate, smem);
+    case 7: return attend_fn<D, M, 7>(pack, gate, smem);
+    case 8: return attend_fn<D, M, 8>(pack, gate, smem);
   }
   return nullptr;
 }
 
 // groups of up to 4 query heads use the packed [q'_hi | q'_lo] columns
-AttendFn pick_attend(const Layout& L, int G, int* smem) {
+AttendFn pick_attend(const Layout& L, int G, bool gate, int* smem) {
   const bool pack = G <= 4;
-  if (L.d == 64 && L.m == 64) return pick_bw<64, 64>(L.bw, pack, smem);
-  if (L.d == 64 && L.m == 128) return pick_bw<64, 128>(L.bw, pack, smem);
-  if (L.d == 128 && L.m == 64) return pick_bw<128, 64>(L.bw, pack, smem);
-  if (L.d == 128 && L.m == 128) return pick_bw<128, 128>(L.bw, pack, smem);
+  if (L.d == 64 && L.m == 64) return pick_bw<64, 64>(L.bw, pack, gate, smem);
+  if (L.d == 64 && L.m == 128) return pick_bw<64, 128>(L.bw, pack, gate, smem);
+  if (L.d == 128 && L.m == 64) return pick_bw<128, 64>(L.bw, pack, gate, smem);
+  if (L.d == 128 && L.m == 128) return pick_bw<128, 128>(L.bw, pack, gate, smem);
   return nullptr;
 }
 
@@ -1090,9 +1130,11 @@ AttendFn pick_attend(const Layout& L, int G, int* smem) {
 
 int attend_ctas_per_sm(const Layout& L, int G) {
   int smem = 0;
-  AttendFn fn = pick_attend(L, G, &smem);
-  if (!fn) return 0;
-  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+  AttendFn fn = pick_attend(L, G, false, &smem);
+  AttendFn fg = pick_attend(L, G, true, &smem);
+  if (!fn || !fg) return 0;
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
+      cudaFuncSetAttribute(fg, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return 0;
   int n = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, kThreads, smem) != cudaSuccess) return 0;
@@ -1135,7 +1177,7 @@ cudaError_t launch_qprep(const QPrepArgs& a, cudaStream_t s) {
 
 cudaError_t launch_attend(const AttendArgs& a, cudaStream_t s) {
   int smem = 0;
-  AttendFn fn = pick_attend(a.L, a.G, &smem);
+  AttendFn fn = pick_attend(a.L, a.G, a.alist != nullptr, &smem);
   if (!fn) return cudaErrorInvalidValue;
   const int grid = a.plan.cold_ctas > a.plan.hot_ctas ? a.plan.cold_ctas : a.plan.hot_ctas;
   if (grid == 0) return cudaSuccess;

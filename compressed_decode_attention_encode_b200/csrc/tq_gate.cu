@@ -1,0 +1,189 @@
+// Threshold gate of the cold tier for gated decode calls ("Monarch v3 ...",
+// "Bucle de Decodificación Simplificado": the hot scores come first, and the
+// cold pages are read only while the largest hot score is below a
+// threshold).  Writes the per-head decisions and the list of (row, kv head)
+// units whose cold tier the attention kernel still streams.
+#include <cfloat>
+
+#include "tq_internal.cuh"
+
+namespace tq {
+namespace {
+
+constexpr unsigned kFull = 0xffffffffu;
+
+// ---------------------------------------------------------------------------
+// Blocks of 256 threads; block (unit, c) takes rows [c * ROWS, (c + 1) *
+// ROWS) of the unit's hot window.  A hot K row is read as D/8 lanes x 16
+// bytes, so one warp load covers 32/(D/8) rows, and each lane issues all
+// kGateUnroll of its loads before it computes.  Per row and query head a
+// lane multiplies its 8 coordinates and a butterfly over the row's lanes
+// gives q.k.  The block's per-head maxima merge into gmax with integer
+// atomics on the float bits (max for non-negative values, unsigned min for
+// negative ones; the all-ones empty pattern loses to both).  The block that
+// finishes last takes the decisions, lists the units that still read their
+// cold tier, and leaves gmax empty and the counter at 0 for the next call.
+// ---------------------------------------------------------------------------
+constexpr int kGateThreads = 256;
+constexpr int kGateMaxGroup = 8;
+constexpr int kGateUnroll = 8;
+
+template <int D>
+struct GateShape {
+  static constexpr int LPR = D / 8;                 // lanes per row (16 bytes each)
+  static constexpr int RPI = 32 / LPR;              // rows per warp load
+  static constexpr int NW = kGateThreads / 32;
+  static constexpr int ROWS = NW * RPI * kGateUnroll;   // rows per block
+};
+
+__device__ __forceinline__ void gate_atomic_max(unsigned* p, float v) {
+  v += 0.0f;                                        // -0 -> +0
+  if (v >= 0.0f)
+    atomicMax(reinterpret_cast<int*>(p), __float_as_int(v));
+  else
+    atomicMin(p, __float_as_uint(v));
+}
+
+template <int D>
+__global__ void __launch_bounds__(kGateThreads) gate_kernel(const GateArgs a) {
+  using S = GateShape<D>;
+  constexpr int LPR = S::LPR, RPI = S::RPI, NW = S::NW;
+  __shared__ float wmax[NW][kGateMaxGroup];
+  __shared__ int wcnt[NW];
+  __shared__ int is_last;
+  const int chunks = gridDim.x / a.units;
+  const int unit = blockIdx.x / chunks, r0 = (blockIdx.x % chunks) * S::ROWS;
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int head0 = (unit / a.Hkv) * a.Hq + (unit % a.Hkv) * a.G;
+  const int col = (lane % LPR) * 8;                 // this lane's 8 coordinates
+  const int sub = lane / LPR;                       // its row within a warp load
+  // the window's loads first ...
+  const __half* kbase = a.hot_k + (size_t)unit * a.W * D + col;
+  uint4 kw[kGateUnroll];
+  int row[kGateUnroll];
+#pragma unroll
+  for (int u = 0; u < kGateUnroll; ++u) {
+    row[u] = r0 + (u * NW + warp) * RPI + sub;
+    kw[u] = row[u] < a.n_hot ? __ldg(reinterpret_cast<const uint4*>(kbase + (size_t)row[u] * D))
+                             : make_uint4(0u, 0u, 0u, 0u);
+  }
+  // ... then the queries
+  float qr[kGateMaxGroup][8], mx[kGateMaxGroup];
+#pragma unroll
+  for (int g = 0; g < kGateMaxGroup; ++g) {
+    mx[g] = -INFINITY;
+    if (g < a.G) {
+      const uint4 w = *reinterpret_cast<const uint4*>(a.q + (size_t)(head0 + g) * D + col);
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&ws[e]));
+        qr[g][2 * e] = f.x;
+        qr[g][2 * e + 1] = f.y;
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) qr[g][e] = 0.f;
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < kGateUnroll; ++u) {
+    float kf[8];
+    const uint32_t ws[4] = {kw[u].x, kw[u].y, kw[u].z, kw[u].w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&ws[e]));
+      kf[2 * e] = f.x;
+      kf[2 * e + 1] = f.y;
+    }
+#pragma unroll
+    for (int g = 0; g < kGateMaxGroup; ++g) {
+      if (g < a.G) {
+        float sc = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) sc = fmaf(qr[g][e], kf[e], sc);
+#pragma unroll
+        for (int o = LPR / 2; o; o >>= 1) sc += __shfl_xor_sync(kFull, sc, o);
+        if (row[u] < a.n_hot) mx[g] = fmaxf(mx[g], sc);
+      }
+    }
+  }
+#pragma unroll
+  for (int g = 0; g < kGateMaxGroup; ++g)
+#pragma unroll
+    for (int o = LPR; o < 32; o <<= 1) mx[g] = fmaxf(mx[g], __shfl_xor_sync(kFull, mx[g], o));
+  if (lane == 0) {
+#pragma unroll
+    for (int g = 0; g < kGateMaxGroup; ++g) wmax[warp][g] = mx[g];
+  }
+  __syncthreads();
+  if (t < a.G) {
+    float m = wmax[0][t];
+    for (int w = 1; w < NW; ++w) m = fmaxf(m, wmax[w][t]);
+    if (m != -INFINITY) gate_atomic_max(a.gmax + head0 + t, m);
+    __threadfence();              // the merge is visible before this block counts itself done
+  }
+  __syncthreads();
+  if (t == 0) {
+    __threadfence();
+    is_last = atomicAdd(a.counter, 1u) == gridDim.x - 1;
+  }
+  __syncthreads();
+  if (!is_last) return;
+  // ---- last block: decisions, then the active units in unit order -------
+  __threadfence();
+  int base = 0;
+  for (int u0 = 0; u0 < a.units; u0 += kGateThreads) {
+    const int u = u0 + t;
+    int act = 0;
+    if (u < a.units) {
+      const int h0 = (u / a.Hkv) * a.Hq + (u % a.Hkv) * a.G;
+      for (int g = 0; g < a.G; ++g) {
+        volatile unsigned* gp = a.gmax + h0 + g;
+        const unsigned bits = *gp;
+        const int skip = (bits != kGateEmpty && __uint_as_float(bits) >= a.threshold) ? 1 : 0;
+        a.head_skip[h0 + g] = skip;
+        *gp = kGateEmpty;
+        act |= !skip;
+      }
+    }
+    const unsigned bal = __ballot_sync(kFull, act);
+    if (lane == 0) wcnt[warp] = __popc(bal);
+    __syncthreads();
+    int off = base, tot = 0;
+    for (int w = 0; w < NW; ++w) {
+      if (w < warp) off += wcnt[w];
+      tot += wcnt[w];
+    }
+    if (u < a.units) {
+      const int p = off + __popc(bal & ((1u << lane) - 1u));
+      a.unit_pos[u] = act ? p : -1;
+      if (act) a.alist[p] = u;
+    }
+    base += tot;
+    __syncthreads();
+  }
+  for (int p = base + t; p <= a.units; p += kGateThreads) a.alist[p] = 0;
+  if (t == 0) {
+    *a.n_active = base;
+    *a.counter = 0u;
+  }
+}
+
+}  // namespace
+
+template <int D>
+cudaError_t launch_gate_d(const GateArgs& a, cudaStream_t s) {
+  const int chunks = a.n_hot > 0 ? (a.n_hot + GateShape<D>::ROWS - 1) / GateShape<D>::ROWS : 1;
+  gate_kernel<D><<<a.units * chunks, kGateThreads, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gate(const GateArgs& a, cudaStream_t s) {
+  if (a.G > kGateMaxGroup) return cudaErrorInvalidValue;
+  if (a.d == 64) return launch_gate_d<64>(a, s);
+  if (a.d == 128) return launch_gate_d<128>(a, s);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace tq

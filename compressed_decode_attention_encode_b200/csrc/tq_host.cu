@@ -16,8 +16,6 @@ namespace tq {
 
 namespace {
 
-constexpr int kSlotsCold = 96;     // partial slots per (row, kv head) for cold CTAs
-constexpr int kSlotsHot = 32;      // ... and for hot CTAs
 constexpr size_t kAlign = 256;
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -59,7 +57,7 @@ bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 }  // namespace
 
 struct WsLayout {
-  size_t status, signs, S, St, qrot, qsk, qscale, part, total;
+  size_t status, signs, S, St, qrot, qsk, qscale, part, gate, total;
 };
 
 static WsLayout ws_layout(const tq_config& c) {
@@ -76,6 +74,8 @@ static WsLayout ws_layout(const tq_config& c) {
   w.qsk = off;    off += round_up(2 * heads * c.qjl_bits, kAlign);
   w.qscale = off; off += round_up(sizeof(float) * 2 * heads, kAlign);
   w.part = off;   off += round_up(sizeof(float) * units * (kSlotsCold + kSlotsHot) * G * (c.head_dim + 2), kAlign);
+  // gated decode: head_skip, gmax [heads], unit_pos [units], alist [units + 1], n_active
+  w.gate = off;   off += round_up(sizeof(int) * (2 * heads + 2 * units + 2), kAlign);
   w.total = off;
   return w;
 }
@@ -192,6 +192,9 @@ tq_status tq_cache_create(const tq_config* cfg, void* hot_mem, void* cold_mem,
   // Pageable sources: cudaMemcpyAsync returns once the data is staged, so
   // the vectors may be released when the calls return.
   cudaError_t e = cudaMemsetAsync(c->status(), 0, kAlign, stream);
+  const size_t heads = (size_t)cfg->batch * cfg->num_q_heads;
+  if (e == cudaSuccess)      // the gate's per-head maxima start empty (all bits set)
+    e = cudaMemsetAsync(c->ws + c->W.gate + sizeof(int) * heads, 0xff, sizeof(int) * heads, stream);
   if (e == cudaSuccess) e = cudaMemcpyAsync(c->signs(), signs.data(), sizeof(double) * d, cudaMemcpyHostToDevice, stream);
   if (e == cudaSuccess) e = cudaMemcpyAsync(c->S(), S.data(), sizeof(float) * S.size(), cudaMemcpyHostToDevice, stream);
   if (e == cudaSuccess) e = cudaMemcpyAsync(c->St(), St.data(), sizeof(float) * St.size(), cudaMemcpyHostToDevice, stream);
@@ -319,12 +322,24 @@ static SplitPlan make_plan(int64_t n_cold, int n_hot, int units, int ctas, bool 
   return pl;
 }
 
-// The launches of one decode call: q-prep, the attention kernel (split
-// partials), and the merge of the partials into the output rows.  Scratch
-// buffers are the caller's (workspace or static scratch).
+// Gated decode: the workspace's gate area and the caller's threshold.
+struct GateBuffers {
+  int* head_skip;
+  unsigned* gmax;
+  int* unit_pos;
+  int* alist;
+  int* n_active;
+  unsigned* counter;
+  float threshold;
+};
+
+// The launches of one decode call: q-prep, the gate of the cold tier (gated
+// calls only), the attention kernel (split partials), and the merge of the
+// partials into the output rows.  Scratch buffers are the caller's
+// (workspace or static scratch).
 static tq_status launch_decode(tq_cache* c, const void* q, float* out, float softmax_scale,
                                const SplitPlan& pl, __half* qrot, __half* qsk, float* qscale,
-                               float* part, cudaStream_t stream) {
+                               float* part, cudaStream_t stream, const GateBuffers* gate = nullptr) {
   const tq_config& cf = c->cfg;
   const int d = cf.head_dim;
   const int units = cf.batch * cf.num_kv_heads;
@@ -345,6 +360,26 @@ static tq_status launch_decode(tq_cache* c, const void* q, float* out, float sof
   qa.d = d;
   qa.m = cf.qjl_bits;
   if (launch_qprep(qa, stream) != cudaSuccess) return TQ_ERR_CUDA;
+  if (gate) {
+    GateArgs ga{};
+    ga.q = (const __half*)q;
+    ga.hot_k = c->hot_k();
+    ga.head_skip = gate->head_skip;
+    ga.gmax = gate->gmax;
+    ga.unit_pos = gate->unit_pos;
+    ga.alist = gate->alist;
+    ga.n_active = gate->n_active;
+    ga.counter = gate->counter;
+    ga.units = units;
+    ga.G = cf.num_q_heads / cf.num_kv_heads;
+    ga.Hq = cf.num_q_heads;
+    ga.Hkv = cf.num_kv_heads;
+    ga.W = cf.hot_window;
+    ga.n_hot = c->n_hot;
+    ga.d = d;
+    ga.threshold = gate->threshold;
+    if (launch_gate(ga, stream) != cudaSuccess) return TQ_ERR_CUDA;
+  }
   AttendArgs a{};
   a.q = (const __half*)q;
   a.qrot = qrot;
@@ -365,6 +400,10 @@ static tq_status launch_decode(tq_cache* c, const void* q, float* out, float sof
   a.n_cold = c->n_cold;
   a.plan = pl;
   a.log2e_sigma = (float)(1.4426950408889634 * (double)sigma);
+  if (gate) {
+    a.alist = gate->alist;
+    a.n_active = gate->n_active;
+  }
   if (c->ev_start && cudaEventRecord(c->ev_start, stream) != cudaSuccess) return TQ_ERR_CUDA;
   if (launch_attend(a, stream) != cudaSuccess) return TQ_ERR_CUDA;
   if (c->ev_stop && cudaEventRecord(c->ev_stop, stream) != cudaSuccess) return TQ_ERR_CUDA;
@@ -379,19 +418,51 @@ static tq_status launch_decode(tq_cache* c, const void* q, float* out, float sof
   ca.d = d;
   ca.plan = pl;
   ca.batch = cf.batch;
+  if (gate) {
+    ca.head_skip = gate->head_skip;
+    ca.unit_pos = gate->unit_pos;
+    ca.n_active = gate->n_active;
+  }
   if (launch_combine(ca, stream) != cudaSuccess) return TQ_ERR_CUDA;
   return TQ_OK;
 }
 
 tq_status tq_decode_attention(tq_cache* c, const void* q, float* out, float softmax_scale,
                               cudaStream_t stream) {
-  if (!c || !q || !out || !(softmax_scale >= 0.0f) || std::isinf(softmax_scale))
+  if (!c || !q || !out || !(softmax_scale >= 0.0f) || std::isinf(softmax_scale) ||
+      (uintptr_t)q % 16)
     return TQ_ERR_INVALID_ARG;
   const int units = c->cfg.batch * c->cfg.num_kv_heads;
   const SplitPlan pl = make_plan(c->n_cold, c->n_hot, units, c->num_sms * c->ctas_per_sm, false);
   return launch_decode(c, q, out, softmax_scale, pl, (__half*)(c->ws + c->W.qrot),
                        (__half*)(c->ws + c->W.qsk), (float*)(c->ws + c->W.qscale),
                        (float*)(c->ws + c->W.part), stream);
+}
+
+tq_status tq_decode_attention_gated(tq_cache* c, const void* q, float* out, float softmax_scale,
+                                    float threshold, int32_t* head_skip, cudaStream_t stream) {
+  if (!c || !q || !out || !(softmax_scale >= 0.0f) || std::isinf(softmax_scale) ||
+      std::isnan(threshold) || (uintptr_t)q % 16)
+    return TQ_ERR_INVALID_ARG;
+  const tq_config& cf = c->cfg;
+  const int units = cf.batch * cf.num_kv_heads;
+  const int heads = cf.batch * cf.num_q_heads;
+  int* area = (int*)(c->ws + c->W.gate);
+  GateBuffers gb{};
+  gb.head_skip = head_skip ? (int*)head_skip : area;
+  gb.gmax = (unsigned*)(area + heads);
+  gb.unit_pos = area + 2 * heads;
+  gb.alist = gb.unit_pos + units;
+  gb.n_active = gb.alist + units + 1;
+  gb.counter = (unsigned*)(c->ws + c->W.status + 64);   // zeroed at create, reset by each gate
+  gb.threshold = threshold;
+  const SplitPlan pl = make_plan(c->n_cold, c->n_hot, units, c->num_sms * c->ctas_per_sm, false);
+  if (pl.cold_ctas == 0 && pl.hot_ctas == 0 &&        // nothing cached: no head skips
+      cudaMemsetAsync(gb.head_skip, 0, sizeof(int) * heads, stream) != cudaSuccess)
+    return TQ_ERR_CUDA;
+  return launch_decode(c, q, out, softmax_scale, pl, (__half*)(c->ws + c->W.qrot),
+                       (__half*)(c->ws + c->W.qsk), (float*)(c->ws + c->W.qscale),
+                       (float*)(c->ws + c->W.part), stream, &gb);
 }
 
 tq_status tq_set_attend_events(tq_cache* c, cudaEvent_t start, cudaEvent_t stop) {
@@ -437,7 +508,8 @@ static void* static_scratch_address(int device) {
 
 tq_status tq_decode_attention_static(tq_cache* c, const void* q, float* out, float softmax_scale,
                                      cudaStream_t stream) {
-  if (!c || !q || !out || !(softmax_scale >= 0.0f) || std::isinf(softmax_scale))
+  if (!c || !q || !out || !(softmax_scale >= 0.0f) || std::isinf(softmax_scale) ||
+      (uintptr_t)q % 16)
     return TQ_ERR_INVALID_ARG;
   int current = -1;
   if (cudaGetDevice(&current) != cudaSuccess) return TQ_ERR_CUDA;

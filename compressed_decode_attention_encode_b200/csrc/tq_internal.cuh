@@ -164,6 +164,9 @@ cudaError_t launch_qprep(const QPrepArgs& a, cudaStream_t s);
 // (c+1)*cold_bpc) of it and writes one partial per unit it touches, into
 // slot c - first_cta(unit).  Hot tiles are split the same way by hot CTAs,
 // whose partials follow the cold slots.
+constexpr int kSlotsCold = 96;     // partial slots per (row, kv head) for cold CTAs
+constexpr int kSlotsHot = 32;      // ... and for hot CTAs
+
 struct SplitPlan {
   int64_t cold_blocks;      // 64-token blocks holding valid cold tokens, per unit
   int cold_ctas;
@@ -174,6 +177,20 @@ struct SplitPlan {
   int slots_cold;           // partial slots per unit reserved for cold CTAs
   int slots_hot;
 };
+
+// Cold split of a gated decode call, over the n_active units whose cold
+// tier is read: blocks per CTA as in the host plan (at least enough that a
+// unit spans at most kSlotsCold - 1 CTAs), for at most `ctas_max` CTAs (the
+// launch's cold CTAs when every unit is read).
+__host__ __device__ inline void gated_cold_split(int64_t n_active, int64_t nb, int ctas_max,
+                                                 int64_t* bpc, int* ctas) {
+  const int64_t total = n_active * nb;
+  int64_t b = ctas_max > 0 ? (total + ctas_max - 1) / ctas_max : 1;
+  const int64_t lo = nb > 1 ? (nb - 1 + kSlotsCold - 3) / (kSlotsCold - 2) : 1;
+  if (b < lo) b = lo;
+  *bpc = b;
+  *ctas = (int)((total + b - 1) / b);
+}
 
 // Partial record per (unit, slot, head): {m (log2 units), l, o[d]}.
 struct AttendArgs {
@@ -192,6 +209,10 @@ struct AttendArgs {
   int W, n_hot;
   int64_t n_cold;
   float log2e_sigma;        // log2(e) * softmax scale
+  // gated calls only (null otherwise): the units whose cold tier is read,
+  // in unit order, and their count (written by gate_kernel)
+  const int* alist;         // [units + 1]
+  const int* n_active;
 };
 
 cudaError_t launch_attend(const AttendArgs& a, cudaStream_t s);
@@ -203,7 +224,34 @@ struct CombineArgs {
   float* out;               // [B*Hq, d]
   SplitPlan plan;
   int units, G, Hkv, Hq, d, batch;
+  // gated calls only (null otherwise)
+  const int* head_skip;     // [B*Hq]  1: the head's cold partials are left out
+  const int* unit_pos;      // [units] position in the active list, or -1
+  const int* n_active;
 };
+
+// Threshold gate of the cold tier: per query head, the largest plain score
+// q.k over the hot window; the head skips its cold tier when the window is
+// non-empty and that score is at least `threshold`.  Several blocks share a
+// unit's window and merge their maxima in `gmax`; the last block to finish
+// takes the decisions and lists the units with at least one head that reads
+// its cold tier.
+constexpr unsigned kGateEmpty = 0xffffffffu;   // gmax entry no block has written
+
+struct GateArgs {
+  const __half* q;          // [B*Hq, d]
+  const __half* hot_k;      // [units, W, d]
+  int* head_skip;           // [B*Hq]
+  unsigned* gmax;           // [B*Hq] float bits, kGateEmpty between calls
+  int* unit_pos;            // [units]
+  int* alist;               // [units + 1]
+  int* n_active;
+  unsigned* counter;        // 0 between calls
+  int units, G, Hq, Hkv, W, n_hot, d;
+  float threshold;
+};
+
+cudaError_t launch_gate(const GateArgs& a, cudaStream_t s);
 
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s);
 

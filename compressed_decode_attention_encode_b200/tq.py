@@ -58,6 +58,8 @@ SIGNATURES = [
     ("tq_evict_window", c_int32, [c_void_p, c_void_p, c_void_p, c_int32, c_void_p]),
     ("tq_decode_attention", c_int32, [c_void_p, c_void_p, c_void_p, c_float, c_void_p]),
     ("tq_decode_attention_static", c_int32, [c_void_p, c_void_p, c_void_p, c_float, c_void_p]),
+    ("tq_decode_attention_gated", c_int32, [c_void_p, c_void_p, c_void_p, c_float, c_float, c_void_p,
+                                            c_void_p]),
     ("tq_get_status", c_int32, [c_void_p, c_void_p]),
     ("tq_set_attend_events", c_int32, [c_void_p, c_void_p, c_void_p]),
     ("tq_export_cold", c_int32, [c_void_p, c_int32, c_int32, c_int64, c_int64, c_void_p,
@@ -157,6 +159,12 @@ def tq_decode_attention_static(handle: int, q_ptr: int, out_ptr: int, scale: flo
            "tq_decode_attention_static")
 
 
+def tq_decode_attention_gated(handle: int, q_ptr: int, out_ptr: int, scale: float, threshold: float,
+                              head_skip_ptr, stream: int) -> None:
+    _check(lib().tq_decode_attention_gated(handle, q_ptr, out_ptr, scale, threshold, head_skip_ptr,
+                                           stream), "tq_decode_attention_gated")
+
+
 def tq_get_status(handle: int, stream: int) -> int:
     return lib().tq_get_status(handle, stream)
 
@@ -241,6 +249,25 @@ class TQCache:
             raise ValueError("out must be contiguous float32")
         tq_decode_attention(self.handle, self._dev16(q), _ptr(out), softmax_scale,
                             _stream_handle(stream))
+        return out
+
+    def decode_attention_gated(self, q, threshold, out=None, head_skip=None, softmax_scale=0.0,
+                               stream=None):
+        """Decode attention whose cold tier is read only by the query heads
+        whose largest hot score q.k is below ``threshold``; ``head_skip``
+        (int32 [B, Hq] on the device) receives 1 for the heads that skipped."""
+        import torch
+        if out is None:
+            out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+        if out.dtype != torch.float32 or not out.is_contiguous():
+            raise ValueError("out must be contiguous float32")
+        hs = None
+        if head_skip is not None:
+            if head_skip.dtype != torch.int32 or not head_skip.is_cuda or not head_skip.is_contiguous():
+                raise ValueError("head_skip must be a contiguous CUDA int32 tensor")
+            hs = _ptr(head_skip)
+        tq_decode_attention_gated(self.handle, self._dev16(q), _ptr(out), softmax_scale,
+                                  float(threshold), hs, _stream_handle(stream))
         return out
 
     def get_status(self, stream=None) -> int:

@@ -168,7 +168,7 @@ tq_status tq_evict_window(tq_cache* cache, const void* k_new,
  * Accumulation is fp32; the products run on tensor cores with fp16
  * operands.  Every valid token is attended (no mask; K is cached after any
  * positional encoding).
- *   q      device fp16 [B, Hq, d]
+ *   q      device fp16 [B, Hq, d], 16-byte aligned (else TQ_ERR_INVALID_ARG)
  *   out    device fp32 [B, Hq, d]
  *   softmax_scale  sigma; 0 selects 1/sqrt(d)
  * With no valid token at all, out is zero.
@@ -197,6 +197,31 @@ tq_status tq_decode_attention(tq_cache* cache, const void* q, float* out,
  */
 tq_status tq_decode_attention_static(tq_cache* cache, const void* q, float* out,
                                      float softmax_scale, cudaStream_t stream);
+
+/*
+ * Decode attention with a threshold-gated cold tier.  This is the loop on
+ * the Monarch v3 page ("Bucle de Decodificación Simplificado"): the hot
+ * scores are computed first, and the cold pages are read only while the
+ * largest hot score is below a threshold.  Per query head h:
+ *   g_h = max over the hot window of q_h . k_t, the plain product without
+ *         softmax_scale, in fp32 from the fp16 q and K;
+ *   if the hot window is non-empty and g_h >= threshold, h attends to its
+ *   hot window alone (one softmax over the hot tokens);
+ *   otherwise h gets exactly tq_decode_attention's result (hot and cold).
+ * A (row, kv head) whose query heads all skip has none of its cold records
+ * read.  The remaining cold work is split again over all CTAs, so the time
+ * saved scales with the skipped units.
+ *   q, out, softmax_scale  as tq_decode_attention
+ *   threshold  any non-NaN float (+inf: never skip; -inf: skip whenever
+ *              the hot window is non-empty)
+ *   head_skip  NULL, or device int32 [B, Hq]: written with 1 for the heads
+ *              that skipped their cold tier, else 0
+ * Scratch comes from the handle's workspace (as tq_decode_attention).
+ * Returns TQ_ERR_INVALID_ARG for a NaN threshold or a NULL q / out.
+ */
+tq_status tq_decode_attention_gated(tq_cache* cache, const void* q, float* out,
+                                    float softmax_scale, float threshold, int32_t* head_skip,
+                                    cudaStream_t stream);
 
 /*
  * Synchronize `stream`, then return and clear the latched device status
