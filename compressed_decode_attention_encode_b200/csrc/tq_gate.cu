@@ -18,11 +18,10 @@ constexpr unsigned kFull = 0xffffffffu;
 // bytes, so one warp load covers 32/(D/8) rows, and each lane issues all
 // kGateUnroll of its loads before it computes.  Per row and query head a
 // lane multiplies its 8 coordinates and a butterfly over the row's lanes
-// gives q.k.  The block's per-head maxima merge into gmax with integer
-// atomics on the float bits (max for non-negative values, unsigned min for
-// negative ones; the all-ones empty pattern loses to both).  The block that
-// finishes last takes the decisions, lists the units that still read their
-// cold tier, and leaves gmax empty and the counter at 0 for the next call.
+// gives q.k.  The block stores its per-head maxima in its own cmax slot;
+// the block that finishes last reduces each head's slots (all loads issued
+// at once), takes the decisions, lists the units that still read their
+// cold tier and leaves the counter at 0 for the next call.
 // ---------------------------------------------------------------------------
 constexpr int kGateThreads = 256;
 constexpr int kGateMaxGroup = 8;
@@ -36,13 +35,8 @@ struct GateShape {
   static constexpr int ROWS = NW * RPI * kGateUnroll;   // rows per block
 };
 
-__device__ __forceinline__ void gate_atomic_max(unsigned* p, float v) {
-  v += 0.0f;                                        // -0 -> +0
-  if (v >= 0.0f)
-    atomicMax(reinterpret_cast<int*>(p), __float_as_int(v));
-  else
-    atomicMin(p, __float_as_uint(v));
-}
+static_assert(GateShape<128>::ROWS == kGateRowsMin && GateShape<64>::ROWS >= kGateRowsMin,
+              "gate blocks take at least kGateRowsMin rows (sizes the cmax slots)");
 
 template <int D>
 __global__ void __launch_bounds__(kGateThreads) gate_kernel(const GateArgs a) {
@@ -52,7 +46,7 @@ __global__ void __launch_bounds__(kGateThreads) gate_kernel(const GateArgs a) {
   __shared__ int wcnt[NW];
   __shared__ int is_last;
   const int chunks = gridDim.x / a.units;
-  const int unit = blockIdx.x / chunks, r0 = (blockIdx.x % chunks) * S::ROWS;
+  const int unit = blockIdx.x / chunks, chunk = blockIdx.x % chunks, r0 = chunk * S::ROWS;
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int head0 = (unit / a.Hkv) * a.Hq + (unit % a.Hkv) * a.G;
   const int col = (lane % LPR) * 8;                 // this lane's 8 coordinates
@@ -120,8 +114,8 @@ __global__ void __launch_bounds__(kGateThreads) gate_kernel(const GateArgs a) {
   if (t < a.G) {
     float m = wmax[0][t];
     for (int w = 1; w < NW; ++w) m = fmaxf(m, wmax[w][t]);
-    if (m != -INFINITY) gate_atomic_max(a.gmax + head0 + t, m);
-    __threadfence();              // the merge is visible before this block counts itself done
+    a.cmax[(size_t)(head0 + t) * chunks + chunk] = m;
+    __threadfence();              // the slot is visible before this block counts itself done
   }
   __syncthreads();
   if (t == 0) {
@@ -138,13 +132,21 @@ __global__ void __launch_bounds__(kGateThreads) gate_kernel(const GateArgs a) {
     int act = 0;
     if (u < a.units) {
       const int h0 = (u / a.Hkv) * a.Hq + (u % a.Hkv) * a.G;
-      for (int g = 0; g < a.G; ++g) {
-        volatile unsigned* gp = a.gmax + h0 + g;
-        const unsigned bits = *gp;
-        const int skip = (bits != kGateEmpty && __uint_as_float(bits) >= a.threshold) ? 1 : 0;
-        a.head_skip[h0 + g] = skip;
-        *gp = kGateEmpty;
-        act |= !skip;
+      float m[kGateMaxGroup];
+#pragma unroll
+      for (int g = 0; g < kGateMaxGroup; ++g) m[g] = -INFINITY;
+      for (int c = 0; c < chunks; ++c) {
+#pragma unroll
+        for (int g = 0; g < kGateMaxGroup; ++g)      // L2 reads: written by other blocks
+          if (g < a.G) m[g] = fmaxf(m[g], __ldcg(a.cmax + (size_t)(h0 + g) * chunks + c));
+      }
+#pragma unroll
+      for (int g = 0; g < kGateMaxGroup; ++g) {
+        if (g < a.G) {
+          const int skip = (a.n_hot > 0 && m[g] >= a.threshold) ? 1 : 0;
+          a.head_skip[h0 + g] = skip;
+          act |= !skip;
+        }
       }
     }
     const unsigned bal = __ballot_sync(kFull, act);

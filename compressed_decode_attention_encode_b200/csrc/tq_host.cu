@@ -57,7 +57,7 @@ bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 }  // namespace
 
 struct WsLayout {
-  size_t status, signs, S, St, qrot, qsk, qscale, part, gate, total;
+  size_t status, signs, S, St, qrot, qsk, qscale, part, gate, gate_max, total;
 };
 
 static WsLayout ws_layout(const tq_config& c) {
@@ -74,8 +74,11 @@ static WsLayout ws_layout(const tq_config& c) {
   w.qsk = off;    off += round_up(2 * heads * c.qjl_bits, kAlign);
   w.qscale = off; off += round_up(sizeof(float) * 2 * heads, kAlign);
   w.part = off;   off += round_up(sizeof(float) * units * (kSlotsCold + kSlotsHot) * G * (c.head_dim + 2), kAlign);
-  // gated decode: head_skip, gmax [heads], unit_pos [units], alist [units + 1], n_active
-  w.gate = off;   off += round_up(sizeof(int) * (2 * heads + 2 * units + 2), kAlign);
+  // gated decode: head_skip [heads], unit_pos [units], alist [units + 1], n_active, then the
+  // gate blocks' maxima [heads, ceil(W / kGateRowsMin)]
+  const size_t gate_chunks = (c.hot_window + kGateRowsMin - 1) / kGateRowsMin;
+  w.gate = off;   off += round_up(sizeof(int) * (heads + 2 * units + 2), kAlign);
+  w.gate_max = off; off += round_up(sizeof(float) * heads * std::max<size_t>(gate_chunks, 1), kAlign);
   w.total = off;
   return w;
 }
@@ -192,9 +195,6 @@ tq_status tq_cache_create(const tq_config* cfg, void* hot_mem, void* cold_mem,
   // Pageable sources: cudaMemcpyAsync returns once the data is staged, so
   // the vectors may be released when the calls return.
   cudaError_t e = cudaMemsetAsync(c->status(), 0, kAlign, stream);
-  const size_t heads = (size_t)cfg->batch * cfg->num_q_heads;
-  if (e == cudaSuccess)      // the gate's per-head maxima start empty (all bits set)
-    e = cudaMemsetAsync(c->ws + c->W.gate + sizeof(int) * heads, 0xff, sizeof(int) * heads, stream);
   if (e == cudaSuccess) e = cudaMemcpyAsync(c->signs(), signs.data(), sizeof(double) * d, cudaMemcpyHostToDevice, stream);
   if (e == cudaSuccess) e = cudaMemcpyAsync(c->S(), S.data(), sizeof(float) * S.size(), cudaMemcpyHostToDevice, stream);
   if (e == cudaSuccess) e = cudaMemcpyAsync(c->St(), St.data(), sizeof(float) * St.size(), cudaMemcpyHostToDevice, stream);
@@ -325,7 +325,7 @@ static SplitPlan make_plan(int64_t n_cold, int n_hot, int units, int ctas, bool 
 // Gated decode: the workspace's gate area and the caller's threshold.
 struct GateBuffers {
   int* head_skip;
-  unsigned* gmax;
+  float* cmax;
   int* unit_pos;
   int* alist;
   int* n_active;
@@ -365,7 +365,7 @@ static tq_status launch_decode(tq_cache* c, const void* q, float* out, float sof
     ga.q = (const __half*)q;
     ga.hot_k = c->hot_k();
     ga.head_skip = gate->head_skip;
-    ga.gmax = gate->gmax;
+    ga.cmax = gate->cmax;
     ga.unit_pos = gate->unit_pos;
     ga.alist = gate->alist;
     ga.n_active = gate->n_active;
@@ -450,8 +450,8 @@ tq_status tq_decode_attention_gated(tq_cache* c, const void* q, float* out, floa
   int* area = (int*)(c->ws + c->W.gate);
   GateBuffers gb{};
   gb.head_skip = head_skip ? (int*)head_skip : area;
-  gb.gmax = (unsigned*)(area + heads);
-  gb.unit_pos = area + 2 * heads;
+  gb.cmax = (float*)(c->ws + c->W.gate_max);
+  gb.unit_pos = area + heads;
   gb.alist = gb.unit_pos + units;
   gb.n_active = gb.alist + units + 1;
   gb.counter = (unsigned*)(c->ws + c->W.status + 64);   // zeroed at create, reset by each gate

@@ -232,17 +232,17 @@ struct CombineArgs {
 
 // Threshold gate of the cold tier: per query head, the largest plain score
 // q.k over the hot window; the head skips its cold tier when the window is
-// non-empty and that score is at least `threshold`.  Several blocks share a
-// unit's window and merge their maxima in `gmax`; the last block to finish
-// takes the decisions and lists the units with at least one head that reads
-// its cold tier.
-constexpr unsigned kGateEmpty = 0xffffffffu;   // gmax entry no block has written
+// non-empty and that score is at least `threshold`.  Block c of a unit
+// writes its per-head maxima of rows [c * rows, (c + 1) * rows) to cmax;
+// the last block to finish reduces them, takes the decisions and lists the
+// units with at least one head that reads its cold tier.
+constexpr int kGateRowsMin = 128;   // fewest hot rows a gate block takes (d = 128)
 
 struct GateArgs {
   const __half* q;          // [B*Hq, d]
   const __half* hot_k;      // [units, W, d]
   int* head_skip;           // [B*Hq]
-  unsigned* gmax;           // [B*Hq] float bits, kGateEmpty between calls
+  float* cmax;              // [B*Hq, chunks]  per-block maxima
   int* unit_pos;            // [units]
   int* alist;               // [units + 1]
   int* n_active;
