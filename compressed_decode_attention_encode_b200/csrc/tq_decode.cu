@@ -210,6 +210,8 @@ __device__ __forceinline__ void qprep_body(const QPrepArgs& a);
 
 template <int D, int M>
 __global__ void __launch_bounds__(256) qprep_kernel(const QPrepArgs a) {
+  // a gated call's gate kernel (a programmatic dependent) may start now
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   qprep_body<D, M>(a);
   // launched as a programmatic dependent of the previous kernel: finish
   // only after that kernel has (its writes visible to what follows q-prep)

@@ -18,7 +18,14 @@ constexpr unsigned kFull = 0xffffffffu;
 // bytes, so one warp load covers 32/(D/8) rows, and each lane issues all
 // kGateUnroll of its loads before it computes.  Per row and query head a
 // lane multiplies its 8 coordinates and a butterfly over the row's lanes
-// gives q.k.  The block stores its per-head maxima in its own cmax slot;
+// gives q.k.
+// The gate is a programmatic dependent of q-prep, so it starts while the
+// step's eviction and q-prep still run.  Before it waits for them it reads
+// only what they do not write (the queries, and the ring rows other than
+// the last eviction's slots); the evicted-into rows come after the wait.
+// When the last eviction wrote more than kGateEarlyRows slots, the whole
+// window is read after the wait.
+// The block stores its per-head maxima in its own cmax slot;
 // the block that finishes last reduces each head's slots (all loads issued
 // at once), takes the decisions, lists the units that still read their
 // cold tier and leaves the counter at 0 for the next call.
@@ -26,6 +33,7 @@ constexpr unsigned kFull = 0xffffffffu;
 constexpr int kGateThreads = 256;
 constexpr int kGateMaxGroup = 8;
 constexpr int kGateUnroll = 8;
+constexpr int kGateEarlyRows = 8;
 
 template <int D>
 struct GateShape {
@@ -51,21 +59,53 @@ __global__ void __launch_bounds__(kGateThreads) gate_kernel(const GateArgs a) {
   const int head0 = (unit / a.Hkv) * a.Hq + (unit % a.Hkv) * a.G;
   const int col = (lane % LPR) * 8;                 // this lane's 8 coordinates
   const int sub = lane / LPR;                       // its row within a warp load
+  const bool early = a.dirty_n <= kGateEarlyRows;
+  auto dirty = [&](int r) {
+    int o = r - a.dirty_lo;
+    if (o < 0) o += a.W;
+    return o < a.dirty_n;
+  };
+  float qr[kGateMaxGroup][8], mx[kGateMaxGroup];
+#pragma unroll
+  for (int g = 0; g < kGateMaxGroup; ++g) mx[g] = -INFINITY;
+  // q.k of one 16-byte slice per lane, summed over the row's lanes; rows
+  // with ok == false leave the maxima alone
+  auto fold_row = [&](const uint4& w, bool ok) {
+    float kf[8];
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&ws[e]));
+      kf[2 * e] = f.x;
+      kf[2 * e + 1] = f.y;
+    }
+#pragma unroll
+    for (int g = 0; g < kGateMaxGroup; ++g) {
+      if (g < a.G) {
+        float sc = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) sc = fmaf(qr[g][e], kf[e], sc);
+#pragma unroll
+        for (int o = LPR / 2; o; o >>= 1) sc += __shfl_xor_sync(kFull, sc, o);
+        if (ok) mx[g] = fmaxf(mx[g], sc);
+      }
+    }
+  };
+  if (!early) asm volatile("griddepcontrol.wait;" ::: "memory");
   // the window's loads first ...
   const __half* kbase = a.hot_k + (size_t)unit * a.W * D + col;
   uint4 kw[kGateUnroll];
-  int row[kGateUnroll];
+  bool ok[kGateUnroll];
 #pragma unroll
   for (int u = 0; u < kGateUnroll; ++u) {
-    row[u] = r0 + (u * NW + warp) * RPI + sub;
-    kw[u] = row[u] < a.n_hot ? __ldg(reinterpret_cast<const uint4*>(kbase + (size_t)row[u] * D))
-                             : make_uint4(0u, 0u, 0u, 0u);
+    const int row = r0 + (u * NW + warp) * RPI + sub;
+    ok[u] = row < a.n_hot && !(early && dirty(row));
+    kw[u] = ok[u] ? __ldg(reinterpret_cast<const uint4*>(kbase + (size_t)row * D))
+                  : make_uint4(0u, 0u, 0u, 0u);
   }
   // ... then the queries
-  float qr[kGateMaxGroup][8], mx[kGateMaxGroup];
 #pragma unroll
   for (int g = 0; g < kGateMaxGroup; ++g) {
-    mx[g] = -INFINITY;
     if (g < a.G) {
       const uint4 w = *reinterpret_cast<const uint4*>(a.q + (size_t)(head0 + g) * D + col);
       const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
@@ -81,25 +121,18 @@ __global__ void __launch_bounds__(kGateThreads) gate_kernel(const GateArgs a) {
     }
   }
 #pragma unroll
-  for (int u = 0; u < kGateUnroll; ++u) {
-    float kf[8];
-    const uint32_t ws[4] = {kw[u].x, kw[u].y, kw[u].z, kw[u].w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&ws[e]));
-      kf[2 * e] = f.x;
-      kf[2 * e + 1] = f.y;
-    }
-#pragma unroll
-    for (int g = 0; g < kGateMaxGroup; ++g) {
-      if (g < a.G) {
-        float sc = 0.f;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) sc = fmaf(qr[g][e], kf[e], sc);
-#pragma unroll
-        for (int o = LPR / 2; o; o >>= 1) sc += __shfl_xor_sync(kFull, sc, o);
-        if (row[u] < a.n_hot) mx[g] = fmaxf(mx[g], sc);
-      }
+  for (int u = 0; u < kGateUnroll; ++u) fold_row(kw[u], ok[u]);
+  if (early) {
+    // the last eviction's rows, once the eviction and q-prep have finished
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    for (int j = warp; j < a.dirty_n; j += NW) {
+      int slot = a.dirty_lo + j;
+      if (slot >= a.W) slot -= a.W;
+      if (slot < r0 || slot >= r0 + S::ROWS || slot >= a.n_hot) continue;   // warp-uniform
+      const bool mine = sub == 0;          // the first row-group of lanes reads it
+      const uint4 w = mine ? __ldcg(reinterpret_cast<const uint4*>(kbase + (size_t)slot * D))
+                           : make_uint4(0u, 0u, 0u, 0u);
+      fold_row(w, mine);
     }
   }
 #pragma unroll
@@ -135,10 +168,18 @@ __global__ void __launch_bounds__(kGateThreads) gate_kernel(const GateArgs a) {
       float m[kGateMaxGroup];
 #pragma unroll
       for (int g = 0; g < kGateMaxGroup; ++g) m[g] = -INFINITY;
-      for (int c = 0; c < chunks; ++c) {
+      for (int c0 = 0; c0 < chunks; c0 += 4) {
+        float v[4][kGateMaxGroup];                   // every read issued before any is used
 #pragma unroll
-        for (int g = 0; g < kGateMaxGroup; ++g)      // L2 reads: written by other blocks
-          if (g < a.G) m[g] = fmaxf(m[g], __ldcg(a.cmax + (size_t)(h0 + g) * chunks + c));
+        for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+          for (int g = 0; g < kGateMaxGroup; ++g)    // L2 reads: written by other blocks
+            v[cc][g] = (g < a.G && c0 + cc < chunks)
+                           ? __ldcg(a.cmax + (size_t)(h0 + g) * chunks + c0 + cc) : -INFINITY;
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+          for (int g = 0; g < kGateMaxGroup; ++g) m[g] = fmaxf(m[g], v[cc][g]);
       }
 #pragma unroll
       for (int g = 0; g < kGateMaxGroup; ++g) {
@@ -177,8 +218,18 @@ __global__ void __launch_bounds__(kGateThreads) gate_kernel(const GateArgs a) {
 template <int D>
 cudaError_t launch_gate_d(const GateArgs& a, cudaStream_t s) {
   const int chunks = a.n_hot > 0 ? (a.n_hot + GateShape<D>::ROWS - 1) / GateShape<D>::ROWS : 1;
-  gate_kernel<D><<<a.units * chunks, kGateThreads, 0, s>>>(a);
-  return cudaGetLastError();
+  // programmatic dependent of q-prep (which lets dependents start at once)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.units * chunks);
+  cfg.blockDim = dim3(kGateThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gate_kernel<D>, a);
 }
 
 cudaError_t launch_gate(const GateArgs& a, cudaStream_t s) {

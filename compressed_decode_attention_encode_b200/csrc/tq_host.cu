@@ -111,6 +111,7 @@ struct tq_cache {
   int64_t n_cold;
   int32_t n_hot;
   int32_t ring_pos;
+  int32_t dirty_lo, dirty_n;   // ring slots the last tq_evict_window wrote
   int num_sms;
   int ctas_per_sm;
   int device;
@@ -175,6 +176,8 @@ tq_status tq_cache_create(const tq_config* cfg, void* hot_mem, void* cold_mem,
   c->n_cold = 0;
   c->n_hot = 0;
   c->ring_pos = 0;
+  c->dirty_lo = 0;
+  c->dirty_n = 0;
   if (cudaGetDevice(&c->device) != cudaSuccess ||
       cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, c->device) != cudaSuccess) {
     delete c;
@@ -281,6 +284,8 @@ tq_status tq_evict_window(tq_cache* c, const void* k_new, const void* v_new, int
   }
   c->n_cold += E;
   c->n_hot = (int32_t)std::min<int64_t>(W, (int64_t)c->n_hot + n);
+  c->dirty_lo = (int32_t)(((int64_t)c->ring_pos + std::max(0, n - W)) % W);
+  c->dirty_n = std::min(n, W);
   c->ring_pos = (int32_t)(((int64_t)c->ring_pos + n) % W);
   return TQ_OK;
 }
@@ -377,6 +382,8 @@ static tq_status launch_decode(tq_cache* c, const void* q, float* out, float sof
     ga.W = cf.hot_window;
     ga.n_hot = c->n_hot;
     ga.d = d;
+    ga.dirty_lo = c->dirty_lo;
+    ga.dirty_n = c->dirty_n;
     ga.threshold = gate->threshold;
     if (launch_gate(ga, stream) != cudaSuccess) return TQ_ERR_CUDA;
   }

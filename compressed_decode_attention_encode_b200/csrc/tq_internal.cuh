@@ -248,6 +248,7 @@ struct GateArgs {
   int* n_active;
   unsigned* counter;        // 0 between calls
   int units, G, Hq, Hkv, W, n_hot, d;
+  int dirty_lo, dirty_n;    // ring slots [lo, lo + n) mod W written by the last eviction
   float threshold;
 };
 

@@ -20,8 +20,8 @@ from tests.tq_testutil import (ATTN_RTOL, codes_from_export, config_for, oracle_
 pytestmark = pytest.mark.gpu
 
 
-def _cache(wl, batch, n_cold, n_hot, W, seed=0):
-    cfg = config_for(wl, batch=batch, hot_window=W, cold_capacity=max(n_cold, 1), seed=seed)
+def _cache(wl, batch, n_cold, n_hot, W, seed=0, spare=0):
+    cfg = config_for(wl, batch=batch, hot_window=W, cold_capacity=max(n_cold + spare, 1), seed=seed)
     cache = tq.TQCache(cfg)
     total = n_cold + n_hot
     k = kv_block(wl, 0, seed, 0, 0, total)[:batch]
@@ -188,4 +188,50 @@ def test_gated_argument_checks():
         cache.decode_attention(q_off)
     with pytest.raises(tq.TQError):
         cache.decode_attention_gated(q_off, 0.0)
+    cache.close()
+
+
+@pytest.mark.parametrize("name", ["llama8b", "tinyllama"])
+def test_gated_after_single_token_eviction(name):
+    """The decode step: one new token evicts into a full window, then the
+    gated call.  The gate reads the new token's ring slot only after the
+    eviction has finished; the token is built so that it alone lifts some
+    heads' hot maxima past the threshold."""
+    wl = WORKLOADS[name]
+    W, n_cold = 64, 300
+    cache, cfg, k, v = _cache(wl, 1, n_cold, W, W, seed=9, spare=8)
+    G = cfg.num_q_heads // cfg.num_kv_heads
+    q = queries(wl, 0, 9)[:1]
+    old = _hot_max(q, k, n_cold, cfg.num_kv_heads)[0]
+    # new token: in kv head 0, K = 4 q of query head 0 (q.k = 4 |q|^2, far above the window)
+    k_new = np.zeros((1, cfg.num_kv_heads, 1, cfg.head_dim), dtype=np.float16)
+    v_new = (np.arange(cfg.num_kv_heads * cfg.head_dim, dtype=np.float64)
+             .reshape(1, cfg.num_kv_heads, 1, cfg.head_dim) % 7 - 3).astype(np.float16)
+    k_new[0, 0, 0] = (4.0 * q[0, 0].astype(np.float64)).astype(np.float16)
+    for h in range(1, cfg.num_kv_heads):
+        k_new[0, h, 0] = k[0, h, n_cold]        # elsewhere a copy of an existing hot key
+    cache.evict_window(torch.from_numpy(k_new).cuda(), torch.from_numpy(v_new).cuda())
+    hk, hv = cache.hot_ring()
+    hk = hk.cpu().numpy().astype(np.float64)[0]
+    hv = hv.cpu().numpy().astype(np.float64)[0]
+    new = np.array([(hk[h // G] @ q[0, h].astype(np.float64)).max() for h in range(cfg.num_q_heads)])
+    assert new[0] > old.max() * 1.5
+    thr = 0.5 * (old.max() + new[0])           # only head 0's new maximum reaches it
+    hs = torch.zeros((1, cfg.num_q_heads), dtype=torch.int32, device="cuda")
+    out = cache.decode_attention_gated(torch.from_numpy(q).cuda(), thr, head_skip=hs)
+    assert cache.get_status() == 0
+    skip_gpu = hs.cpu().numpy()[0]
+    assert skip_gpu[0] == 1 and skip_gpu[1:].sum() == (new[1:] >= thr).sum()
+    nc = cache.counts()[0]
+    signs, S = oracle_signs_S(cfg)
+    ck, cv = [], []
+    for h in range(cfg.num_kv_heads):
+        exp = cache.export_cold(0, h, 0, nc)
+        ck.append(codes_from_export(exp, cfg, True))
+        cv.append(codes_from_export(exp, cfg, False))
+    ref, skip = O.decode_attention_gated(q[0].astype(np.float64), hk, hv, ck, cv, signs, S,
+                                         cfg.num_kv_heads, thr)
+    np.testing.assert_array_equal(skip_gpu, skip.astype(np.int32))
+    e = rel_err(out.cpu().numpy()[0].astype(np.float64), ref)
+    assert np.all(e <= ATTN_RTOL), e.max()
     cache.close()
