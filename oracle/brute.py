@@ -151,3 +151,15 @@ def decode_one_head_gated(q, hot_k, hot_v, cold_k, cold_v, signs, S, b_r, b_thet
     if skipped:
         return decode_one_head(q, hot_k, hot_v, [], [], signs, S, b_r, b_theta, sigma), True
     return decode_one_head(q, hot_k, hot_v, cold_k, cold_v, signs, S, b_r, b_theta, sigma), False
+
+
+def tc_write_loops(A, k, v, lam, eta):
+    """A <- lambda A + eta k v^T, element by element (lists of lists)."""
+    d = len(A)
+    return [[lam * A[i][j] + eta * k[i] * v[j] for j in range(d)] for i in range(d)]
+
+
+def tc_read_loops(q, A):
+    """r_j = sum_i q_i A_ij."""
+    d = len(A)
+    return [sum(q[i] * A[i][j] for i in range(d)) for j in range(d)]

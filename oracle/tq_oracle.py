@@ -509,6 +509,52 @@ def decode_attention_gated(q: np.ndarray, hot_k: np.ndarray, hot_v: np.ndarray,
     return np.where(skip[:, None], hot_only, full), skip
 
 
+# ---------------------------------------------------------------------------
+# Tensor Cache second tier ("Tensor Cache: Eviction-conditioned Associative
+# Memory for Transformers", section "Metodología", items "Mecanismo de
+# Escritura", "Mecanismo de Lectura" and "Fusión").  The ring of W tokens is
+# the first level; every token the ring displaces is written into a d x d
+# outer-product matrix A per kv head, and queries read A back.
+# READINGS: lambda and eta are one scalar pair per kv head (the page learns
+# them per head; here they are given); the gate g is one scalar per query
+# head; A starts at zero; the local output y_local is the exact softmax
+# attention over the ring (the same as ``decode_attention`` with no cold
+# tokens).
+# ---------------------------------------------------------------------------
+
+def tc_write(A: np.ndarray, k: np.ndarray, v: np.ndarray, lam: float, eta: float) -> np.ndarray:
+    """One eviction: A <- lambda A + eta (k outer v)."""
+    return lam * np.asarray(A, dtype=np.float64) + eta * np.outer(
+        np.asarray(k, dtype=np.float64), np.asarray(v, dtype=np.float64))
+
+
+def tc_write_sequence(A: np.ndarray, ks: np.ndarray, vs: np.ndarray, lam: float,
+                      eta: float) -> np.ndarray:
+    """Evictions in order (oldest first), one ``tc_write`` each."""
+    for k, v in zip(ks, vs):
+        A = tc_write(A, k, v, lam, eta)
+    return A
+
+
+def tc_decode(q: np.ndarray, hot_k: np.ndarray, hot_v: np.ndarray, A: np.ndarray,
+              gate: np.ndarray, num_kv_heads: int,
+              softmax_scale: Optional[float] = None) -> np.ndarray:
+    """y = y_local + sigmoid(g) (q A) per query head h, with y_local the
+    softmax attention over h's ring and A = A[kv head of h] ([Hkv, d, d])."""
+    q = np.asarray(q, dtype=np.float64)
+    hq = q.shape[0]
+    g = hq // num_kv_heads
+    y_local = decode_attention(q, hot_k, hot_v, None, None, None, None, num_kv_heads,
+                               softmax_scale)
+    out = np.empty_like(y_local)
+    for h in range(hq):
+        m = q[h] @ np.asarray(A[h // g], dtype=np.float64)
+        gh = float(gate[h])          # logistic sigmoid, evaluated without overflow
+        sig = 1.0 / (1.0 + math.exp(-gh)) if gh >= 0 else math.exp(gh) / (1.0 + math.exp(gh))
+        out[h] = y_local[h] + sig * m
+    return out
+
+
 def attention_reference(q: np.ndarray, k: np.ndarray, v: np.ndarray,
                         num_kv_heads: int, softmax_scale: Optional[float] = None) -> np.ndarray:
     """Textbook softmax(q K^T * sigma) V per query head, fp64 (GQA mapping)."""

@@ -116,3 +116,16 @@ def test_gated_decode_matches_brute(d, m, b):
             assert ref_skip == skip[h]
             np.testing.assert_allclose(out[h], ref, rtol=1e-12, atol=1e-12)
         assert skip.sum() == (gmax >= thr).sum()
+
+
+def test_tc_write_and_read_match_loops():
+    rng = np.random.default_rng(31)
+    d = 6
+    A = rng.standard_normal((d, d))
+    Al = A.tolist()
+    for _ in range(5):
+        k, v, q = rng.standard_normal((3, d))
+        A = O.tc_write(A, k, v, 0.8, 0.3)
+        Al = B.tc_write_loops(Al, list(k), list(v), 0.8, 0.3)
+        np.testing.assert_allclose(A, Al, rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(q @ A, B.tc_read_loops(list(q), Al), rtol=1e-12, atol=1e-12)

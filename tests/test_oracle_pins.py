@@ -472,3 +472,55 @@ def test_gate_boundary_and_empty_hot_window():
     out, skip = O.decode_attention_gated(q, empty, hv[:, :0], ck, cv, signs, S, hkv, -math.inf)
     assert not skip.any()
     np.testing.assert_array_equal(out, O.decode_attention(q, empty, hv[:, :0], ck, cv, signs, S, hkv))
+
+
+# ---- Tensor Cache second tier (outer-product memory of evicted tokens) ----
+
+def test_tc_sequence_equals_weighted_closed_form():
+    """Sequential writes equal the weighted sum the page's parallel scan
+    computes: A_E = lambda^E A_0 + eta sum_e lambda^(E-1-e) k_e v_e^T,
+    written here as one matrix product K^T diag(w) V."""
+    rng = np.random.default_rng(21)
+    d, E, lam, eta = 8, 37, 0.93, 0.4
+    A0 = rng.standard_normal((d, d))
+    K = rng.standard_normal((E, d))
+    V = rng.standard_normal((E, d))
+    seq = O.tc_write_sequence(A0, K, V, lam, eta)
+    w = eta * lam ** (E - 1 - np.arange(E))
+    closed = lam ** E * A0 + K.T @ (w[:, None] * V)
+    np.testing.assert_allclose(seq, closed, rtol=1e-12, atol=1e-12)
+    # lambda = eta = 1: the plain sum of outer products K^T V
+    np.testing.assert_allclose(O.tc_write_sequence(np.zeros((d, d)), K, V, 1.0, 1.0), K.T @ V,
+                               rtol=1e-12, atol=1e-12)
+
+
+def test_tc_read_is_linear_attention_identity():
+    """q (k outer v) = <q, k> v: one write into an empty memory returns the
+    value scaled by eta times the key's inner product with the query."""
+    rng = np.random.default_rng(22)
+    d = 16
+    q, k, v = rng.standard_normal((3, d))
+    A = O.tc_write(np.zeros((d, d)), k, v, 0.5, 0.25)
+    np.testing.assert_allclose(q @ A, 0.25 * (q @ k) * v, rtol=1e-12, atol=1e-14)
+
+
+def test_tc_decode_gate_limits():
+    """A closed gate (g -> -inf) leaves textbook softmax attention over the
+    ring (scipy's softmax); g = 0 adds half the memory read; with an empty
+    memory the gate has no effect."""
+    from scipy.special import softmax
+    rng = np.random.default_rng(23)
+    hq, hkv, W, d = 4, 2, 6, 8
+    q = rng.standard_normal((hq, d))
+    hk = rng.standard_normal((hkv, W, d))
+    hv = rng.standard_normal((hkv, W, d))
+    A = rng.standard_normal((hkv, d, d))
+    closed = O.tc_decode(q, hk, hv, A, np.full(hq, -800.0), hkv)
+    half = O.tc_decode(q, hk, hv, A, np.zeros(hq), hkv)
+    empty = O.tc_decode(q, hk, hv, np.zeros((hkv, d, d)), rng.standard_normal(hq), hkv)
+    for h in range(hq):
+        g = h // (hq // hkv)
+        local = softmax(hk[g] @ q[h] / math.sqrt(d)) @ hv[g]
+        np.testing.assert_allclose(closed[h], local, rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(empty[h], local, rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(half[h], local + 0.5 * (q[h] @ A[g]), rtol=1e-12, atol=1e-12)
