@@ -44,6 +44,9 @@ def parse():
     ap.add_argument("--gate-quantile", type=float, default=None,
                     help="decode with the threshold-gated cold tier; each layer's threshold is this "
                          "quantile of its heads' hot-window maxima q.k at the start")
+    ap.add_argument("--tensor-cache", action="store_true",
+                    help="decode with the Tensor Cache tier: evicted tokens go to an outer-product "
+                         "memory instead of the compressed cold store")
     ap.add_argument("--encode", action="store_true",
                     help="time the prefill encode (tq_encode_append of 4096-token chunks) instead")
     return ap.parse_args()
@@ -274,12 +277,18 @@ def run_gpu(args, wl):
     for layer in range(L):
         gen.manual_seed(1_000_003 * (args.seed + 1) + 7919 * layer + rank)
         c = tq.TQCache(cfg, device=dev)
+        if args.tensor_cache:      # fixed synthetic decay, write rate and gate
+            c.enable_tensor_cache([0.995] * wl.num_kv_heads, [0.05] * wl.num_kv_heads,
+                                  [0.0] * wl.num_q_heads)
         pos = 0
         while pos < wl.cold:
             n = min(chunk, wl.cold - pos)
             k = gen_kv(wl, layer, args.seed, 0, wl.batch, pos, n, dev, gen)
             v = gen_kv(wl, layer, args.seed, 1, wl.batch, pos, n, dev, gen)
-            c.encode_append(k, v)
+            if args.tensor_cache:  # the whole context streams through the ring into A
+                c.evict_window(k, v)
+            else:
+                c.encode_append(k, v)
             pos += n
         k = gen_kv(wl, layer, args.seed, 0, wl.batch, 0, wl.hot, dev, gen)
         v = gen_kv(wl, layer, args.seed, 1, wl.batch, 0, wl.hot, dev, gen)
@@ -325,6 +334,8 @@ def run_gpu(args, wl):
             caches[l].decode_attention_gated(q, gate_tau[l], out=out, head_skip=skip_bufs[l])
 
     step_idx = [0]
+    seen = [wl.cold + wl.hot] * L        # tokens inserted per (row, kv head), per layer
+    tc_bytes = 12 * wl.head_dim * wl.head_dim   # A read + written (update), read (decode), float32
 
     def one_step(ev_pairs=None):
         s = step_idx[0]
@@ -334,8 +345,13 @@ def run_gpu(args, wl):
         for l in range(L):
             caches[l].evict_window(knew[l][s], vnew[l][s])
             nc, nh, _ = caches[l].counts()
-            keys += units * (nc + nh)
-            abytes += units * (nc * cold_tok_bytes + nh * hot_tok_bytes)
+            seen[l] += 1
+            if args.tensor_cache:
+                keys += units * seen[l]
+                abytes += units * (nh * hot_tok_bytes + tc_bytes)
+            else:
+                keys += units * (nc + nh)
+                abytes += units * (nc * cold_tok_bytes + nh * hot_tok_bytes)
             if ev_pairs is not None:
                 caches[l].set_attend_events(*ev_pairs[l])
             attend(l, qs[l], outs[l])
@@ -422,7 +438,8 @@ def run_gpu(args, wl):
             dk, dv, dq, do = views[l]
             caches[l].evict_window(dk, dv)
             nc, nh, _ = caches[l].counts()
-            e2e_keys += units * (nc + nh)
+            seen[l] += 1
+            e2e_keys += units * (seen[l] if args.tensor_cache else nc + nh)
             attend(l, dq, do)
         hout.copy_(dout, non_blocking=True)
         d2h = dout.numel() * 4
@@ -489,7 +506,21 @@ def run_gpu(args, wl):
                                    "bytes_per_launch": read / L,
                                    "bytes_note": "cold bytes of the units the last step read"})
         result["hbm"] = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and gate_tau is None:
+    if args.tensor_cache:
+        step_gbs = bytes_total / (ms / 1e3) / 1e9
+        result["metric"] = ("Tensor Cache decode: context tokens/s (softmax over the ring + "
+                            "outer-product memory of the evicted tokens)")
+        result["config"]["tensor_cache"] = {"lambda": 0.995, "eta": 0.05, "gate": 0.0,
+                                            "memory_per_unit_bytes": 4 * wl.head_dim ** 2}
+        result["roofline"] = {"bound": "hbm", "achieved": step_gbs, "peak": hbm_peak, "unit": "GB/s",
+                              "frac": step_gbs / hbm_peak, "traffic": None,
+                              "kernel": "whole decode step (ring attention, A update, A read)",
+                              "peak_kind": peak_kind,
+                              "bytes_note": "512 B per ring token + 12 d^2 B of A per unit and layer"}
+        result["hbm"] = None
+        result["gpu_launches"] = L * (2 + 3 + 1) * args.steps
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and gate_tau is None and \
+            not args.tensor_cache:
         sample = oracle_sample(wl, args.seed, kv_heads=1)
         time_oracle(sample)
         tt, kk = 0.0, 0

@@ -16,7 +16,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libtq.so")
-SOURCES = ["tq_host.cu", "tq_encode.cu", "tq_decode.cu", "tq_gate.cu", "tq_search.cu"]
+SOURCES = ["tq_host.cu", "tq_encode.cu", "tq_decode.cu", "tq_gate.cu", "tq_tcache.cu", "tq_search.cu"]
 HEADERS = ["tq_internal.cuh", "tq_encode_core.cuh", os.path.join("..", "..", "include", "tq.h")]
 
 NVCC_FLAGS = [

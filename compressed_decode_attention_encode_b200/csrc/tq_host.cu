@@ -112,6 +112,10 @@ struct tq_cache {
   int32_t n_hot;
   int32_t ring_pos;
   int32_t dirty_lo, dirty_n;   // ring slots the last tq_evict_window wrote
+  float* tc;                   // Tensor Cache tier: A [units, d, d], or null
+  float* tc_lam;               // [Hkv]
+  float* tc_eta;               // [Hkv]
+  float* tc_sig;               // [Hq] sigmoid(g)
   int num_sms;
   int ctas_per_sm;
   int device;
@@ -178,6 +182,7 @@ tq_status tq_cache_create(const tq_config* cfg, void* hot_mem, void* cold_mem,
   c->ring_pos = 0;
   c->dirty_lo = 0;
   c->dirty_n = 0;
+  c->tc = c->tc_lam = c->tc_eta = c->tc_sig = nullptr;
   if (cudaGetDevice(&c->device) != cudaSuccess ||
       cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, c->device) != cudaSuccess) {
     delete c;
@@ -258,6 +263,39 @@ tq_status tq_evict_window(tq_cache* c, const void* k_new, const void* v_new, int
   if (!c || !k_new || !v_new || n < 1) return TQ_ERR_INVALID_ARG;
   const int W = c->cfg.hot_window;
   const int64_t E = std::max<int64_t>(0, (int64_t)c->n_hot + n - W);
+  if (c->tc) {
+    // Tensor Cache tier: the displaced tokens are written into A (before
+    // the ring write overwrites their slots); the cold store is untouched
+    if (E > 0) {
+      TcUpdateArgs t{};
+      t.A = c->tc;
+      t.lam = c->tc_lam;
+      t.eta = c->tc_eta;
+      t.ring_k = c->hot_k();
+      t.ring_v = c->hot_v();
+      t.src_k = (const __half*)k_new;
+      t.src_v = (const __half*)v_new;
+      t.units = c->cfg.batch * c->cfg.num_kv_heads;
+      t.Hkv = c->cfg.num_kv_heads;
+      t.W = W;
+      t.d = c->cfg.head_dim;
+      t.nA = (int)std::min<int64_t>(E, c->n_hot);
+      t.ring_start = ((c->ring_pos - c->n_hot) % W + W) % W;
+      t.nB = (int)(E - t.nA);
+      t.src_tokens = n;
+      if (launch_tc_update(t, stream) != cudaSuccess) return TQ_ERR_CUDA;
+    }
+    const int first = std::max(0, n - W);
+    if (launch_ring_write(c->hot_k(), c->hot_v(), (const __half*)k_new, (const __half*)v_new,
+                          c->cfg.batch * c->cfg.num_kv_heads, W, c->cfg.head_dim, n, first,
+                          c->ring_pos, stream) != cudaSuccess)
+      return TQ_ERR_CUDA;
+    c->n_hot = (int32_t)std::min<int64_t>(W, (int64_t)c->n_hot + n);
+    c->dirty_lo = (int32_t)(((int64_t)c->ring_pos + first) % W);
+    c->dirty_n = std::min(n, W);
+    c->ring_pos = (int32_t)(((int64_t)c->ring_pos + n) % W);
+    return TQ_OK;
+  }
   if (c->n_cold + E > c->cfg.cold_capacity) return TQ_ERR_CAPACITY;
   // Steady state (a full window, a few new tokens): each new token evicts
   // the token in the slot it takes, and one launch does both.
@@ -431,6 +469,18 @@ static tq_status launch_decode(tq_cache* c, const void* q, float* out, float sof
     ca.n_active = gate->n_active;
   }
   if (launch_combine(ca, stream) != cudaSuccess) return TQ_ERR_CUDA;
+  if (c->tc) {
+    TcReadArgs tr{};
+    tr.A = c->tc;
+    tr.sig = c->tc_sig;
+    tr.q = (const __half*)q;
+    tr.out = out;
+    tr.units = units;
+    tr.G = a.G;
+    tr.Hq = cf.num_q_heads;
+    tr.d = d;
+    if (launch_tc_read(tr, stream) != cudaSuccess) return TQ_ERR_CUDA;
+  }
   return TQ_OK;
 }
 
@@ -470,6 +520,50 @@ tq_status tq_decode_attention_gated(tq_cache* c, const void* q, float* out, floa
   return launch_decode(c, q, out, softmax_scale, pl, (__half*)(c->ws + c->W.qrot),
                        (__half*)(c->ws + c->W.qsk), (float*)(c->ws + c->W.qscale),
                        (float*)(c->ws + c->W.part), stream, &gb);
+}
+
+static size_t tc_matrix_bytes(const tq_config& c) {
+  return round_up(sizeof(float) * c.batch * c.num_kv_heads * c.head_dim * c.head_dim, kAlign);
+}
+
+tq_status tq_tc_bytes(const tq_config* cfg, size_t* bytes) {
+  if (!cfg || !bytes) return TQ_ERR_INVALID_ARG;
+  const tq_status st = check_config(cfg);
+  if (st != TQ_OK) return st;
+  *bytes = tc_matrix_bytes(*cfg) +
+           round_up(sizeof(float) * (2 * cfg->num_kv_heads + cfg->num_q_heads), kAlign);
+  return TQ_OK;
+}
+
+tq_status tq_tc_enable(tq_cache* c, void* tc_mem, const float* lambda, const float* eta,
+                       const float* gate, cudaStream_t stream) {
+  if (!c || !tc_mem || !lambda || !eta || !gate || (uintptr_t)tc_mem % kAlign) return TQ_ERR_INVALID_ARG;
+  if (c->tc) return TQ_ERR_INVALID_ARG;                     // already enabled
+  const tq_config& cf = c->cfg;
+  const int hkv = cf.num_kv_heads, hq = cf.num_q_heads;
+  std::vector<float> par(2 * hkv + hq);
+  for (int h = 0; h < hkv; ++h) {
+    if (!std::isfinite(lambda[h]) || !std::isfinite(eta[h])) return TQ_ERR_INVALID_ARG;
+    par[h] = lambda[h];
+    par[hkv + h] = eta[h];
+  }
+  for (int h = 0; h < hq; ++h) {
+    if (std::isnan(gate[h])) return TQ_ERR_INVALID_ARG;
+    const double g = gate[h];                              // logistic sigmoid without overflow
+    par[2 * hkv + h] = (float)(g >= 0 ? 1.0 / (1.0 + std::exp(-g)) : std::exp(g) / (1.0 + std::exp(g)));
+  }
+  float* A = (float*)tc_mem;
+  float* p = (float*)((uint8_t*)tc_mem + tc_matrix_bytes(cf));
+  cudaError_t e = cudaMemsetAsync(A, 0, tc_matrix_bytes(cf), stream);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(p, par.data(), sizeof(float) * par.size(), cudaMemcpyHostToDevice, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);   // `par` is released on return
+  if (e != cudaSuccess) return TQ_ERR_CUDA;
+  c->tc = A;
+  c->tc_lam = p;
+  c->tc_eta = p + hkv;
+  c->tc_sig = p + 2 * hkv;
+  return TQ_OK;
 }
 
 tq_status tq_set_attend_events(tq_cache* c, cudaEvent_t start, cudaEvent_t stop) {

@@ -254,6 +254,37 @@ struct GateArgs {
 
 cudaError_t launch_gate(const GateArgs& a, cudaStream_t s);
 
+// ---- Tensor Cache second tier -----------------------------------------
+// Per unit a d x d float32 matrix A; per kv head lambda, eta; per query
+// head sigmoid(g).  Evicted tokens e = 0 .. E-1 (oldest first: nA ring
+// slots from ring_start, then the first nB new tokens) are written as
+// A <- lambda^E A + eta sum_e lambda^(E-1-e) k_e v_e^T, which equals E
+// sequential writes A <- lambda A + eta k_e v_e^T.
+struct TcUpdateArgs {
+  float* A;                 // [units, d, d]
+  const float* lam;         // [Hkv]
+  const float* eta;         // [Hkv]
+  const __half* ring_k;     // [units, W, d]
+  const __half* ring_v;
+  const __half* src_k;      // [units, src_tokens, d]
+  const __half* src_v;
+  int units, Hkv, W, d;
+  int nA, ring_start;
+  int nB, src_tokens;
+};
+
+// out[h] += sigmoid(g_h) (q_h A_unit) for every query head h.
+struct TcReadArgs {
+  const float* A;           // [units, d, d]
+  const float* sig;         // [Hq]  sigmoid(g)
+  const __half* q;          // [B*Hq, d]
+  float* out;               // [B*Hq, d]
+  int units, G, Hq, d;
+};
+
+cudaError_t launch_tc_update(const TcUpdateArgs& a, cudaStream_t s);
+cudaError_t launch_tc_read(const TcReadArgs& a, cudaStream_t s);
+
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s);
 
 // ---- vector search ----------------------------------------------------

@@ -60,6 +60,8 @@ SIGNATURES = [
     ("tq_decode_attention_static", c_int32, [c_void_p, c_void_p, c_void_p, c_float, c_void_p]),
     ("tq_decode_attention_gated", c_int32, [c_void_p, c_void_p, c_void_p, c_float, c_float, c_void_p,
                                             c_void_p]),
+    ("tq_tc_bytes", c_int32, [POINTER(tq_config), POINTER(c_size_t)]),
+    ("tq_tc_enable", c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
     ("tq_get_status", c_int32, [c_void_p, c_void_p]),
     ("tq_set_attend_events", c_int32, [c_void_p, c_void_p, c_void_p]),
     ("tq_export_cold", c_int32, [c_void_p, c_int32, c_int32, c_int64, c_int64, c_void_p,
@@ -163,6 +165,22 @@ def tq_decode_attention_gated(handle: int, q_ptr: int, out_ptr: int, scale: floa
                               head_skip_ptr, stream: int) -> None:
     _check(lib().tq_decode_attention_gated(handle, q_ptr, out_ptr, scale, threshold, head_skip_ptr,
                                            stream), "tq_decode_attention_gated")
+
+
+def tq_tc_bytes(cfg: tq_config) -> int:
+    n = c_size_t()
+    _check(lib().tq_tc_bytes(ctypes.byref(cfg), ctypes.byref(n)), "tq_tc_bytes")
+    return n.value
+
+
+def tq_tc_enable(handle: int, tc_ptr: int, lam, eta, gate, stream: int) -> None:
+    def arr(x):
+        a = np.ascontiguousarray(np.asarray(x, dtype=np.float32))
+        return a, a.ctypes.data_as(c_void_p)
+    la, lp = arr(lam)
+    ea, ep = arr(eta)
+    ga, gp = arr(gate)
+    _check(lib().tq_tc_enable(handle, tc_ptr, lp, ep, gp, stream), "tq_tc_enable")
 
 
 def tq_get_status(handle: int, stream: int) -> int:
@@ -269,6 +287,20 @@ class TQCache:
         tq_decode_attention_gated(self.handle, self._dev16(q), _ptr(out), softmax_scale,
                                   float(threshold), hs, _stream_handle(stream))
         return out
+
+    def enable_tensor_cache(self, lam, eta, gate, stream=None):
+        """Switch evictions to the Tensor Cache tier: lam, eta per kv head,
+        gate (g, before the sigmoid) per query head.  Returns the view of A
+        [B, Hkv, d, d] (float32, on the device)."""
+        import torch
+        c = self.cfg
+        if len(lam) != c.num_kv_heads or len(eta) != c.num_kv_heads or len(gate) != c.num_q_heads:
+            raise ValueError("lam, eta: one per kv head; gate: one per query head")
+        self.tc_mem = torch.empty(tq_tc_bytes(c), dtype=torch.uint8, device=self.device)
+        tq_tc_enable(self.handle, _ptr(self.tc_mem), lam, eta, gate, _stream_handle(stream))
+        n = c.batch * c.num_kv_heads * c.head_dim * c.head_dim
+        return self.tc_mem[: 4 * n].view(torch.float32).view(c.batch, c.num_kv_heads, c.head_dim,
+                                                             c.head_dim)
 
     def get_status(self, stream=None) -> int:
         return tq_get_status(self.handle, _stream_handle(stream))

@@ -224,6 +224,34 @@ tq_status tq_decode_attention_gated(tq_cache* cache, const void* q, float* out,
                                     cudaStream_t stream);
 
 /*
+ * Tensor Cache second tier ("Tensor Cache: Eviction-conditioned Associative
+ * Memory for Transformers", section "Metodología"): an alternative to the
+ * compressed cold store.  Once enabled on a handle:
+ *   - every token the hot ring displaces in tq_evict_window is written into
+ *     a d x d float32 matrix A of its (row, kv head) instead of the cold
+ *     store: A <- lambda A + eta (k outer v), in eviction order (a run of E
+ *     evictions is applied at once as lambda^E A + eta sum_e
+ *     lambda^(E-1-e) k_e v_e^T, the same value);
+ *   - every decode call adds sigmoid(g_h) (q_h A) to query head h's output
+ *     (q_h the fp16 query, A that of its kv head), after the softmax over
+ *     the ring and over any cold tokens appended before enabling.
+ * lambda, eta and g are learned on the page; here they are given.
+ *
+ * tq_tc_bytes: device bytes of the tier's buffer for a configuration: A as
+ *   [B, Hkv, d, d] float32 (256-byte aligned), then lambda [Hkv], eta [Hkv]
+ *   and sigmoid(g) [Hq] as float32.
+ * tq_tc_enable: binds the caller's buffer (256-byte aligned, at least
+ *   tq_tc_bytes; owned by the caller, kept until tq_cache_destroy), sets A
+ *   to zero and copies the parameters (host arrays lambda [Hkv], eta [Hkv],
+ *   gate [Hq]); synchronizes `stream`.  TQ_ERR_INVALID_ARG for a NULL or
+ *   misaligned pointer, a non-finite lambda or eta, a NaN gate, or a handle
+ *   that already has the tier.
+ */
+tq_status tq_tc_bytes(const tq_config* cfg, size_t* bytes);
+tq_status tq_tc_enable(tq_cache* cache, void* tc_mem, const float* lambda, const float* eta,
+                       const float* gate, cudaStream_t stream);
+
+/*
  * Synchronize `stream`, then return and clear the latched device status
  * (TQ_OK, TQ_ERR_RANGE or TQ_ERR_TIMEOUT; TQ_ERR_UNSUPPORTED when the
  * attention kernel found its dynamic shared memory at a window address its

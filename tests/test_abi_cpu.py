@@ -153,3 +153,14 @@ def test_vector_codes_bytes():
     r = lambda x: -(-x // 256) * 256
     assert cb == r(n * 128) + r(n * 32) + 2 * r(n * 2)
     assert wb > 0
+
+
+def test_tensor_cache_bytes():
+    """The Tensor Cache tier's buffer: A as [B, Hkv, d, d] float32, then
+    lambda, eta [Hkv] and sigmoid(g) [Hq], each part 256-byte aligned."""
+    cfg = tq.make_config(8, 32, 8, 128, 512, 1000, 3, 3, 128)
+    assert tq.tq_tc_bytes(cfg) == 8 * 8 * 128 * 128 * 4 + 256
+    cfg = tq.make_config(1, 6, 2, 64, 64, 0, 2, 2, 64)
+    assert tq.tq_tc_bytes(cfg) == 2 * 64 * 64 * 4 + 256
+    with pytest.raises(tq.TQError):
+        tq.tq_tc_bytes(tq.make_config(1, 6, 4, 64, 64, 0, 2, 2, 64))   # Hq not a multiple of Hkv
