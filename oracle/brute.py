@@ -163,3 +163,23 @@ def tc_read_loops(q, A):
     """r_j = sum_i q_i A_ij."""
     d = len(A)
     return [sum(q[i] * A[i][j] for i in range(d)) for j in range(d)]
+
+
+def value_estimate_loops(rec, S, b_r, b_theta):
+    """One value record with QJL bits, rotated domain: s16/L * c_r (cos, sin)
+    per pair plus sqrt(pi/2)/m * rn16 * sum_i S_i (+1 or -1)."""
+    L = 2 ** b_r - 1
+    nt = 2 ** b_theta
+    d = 2 * len(rec["cr"])
+    y = [0.0] * d
+    for j in range(len(rec["cr"])):
+        a = (rec["ct"][j] * (2.0 * math.pi)) / nt
+        y[2 * j] = rec["s16"] / L * rec["cr"][j] * math.cos(a)
+        y[2 * j + 1] = rec["s16"] / L * rec["cr"][j] * math.sin(a)
+    m = len(S)
+    c = rec["rn16"] * math.sqrt(math.pi / 2.0) / m
+    for i in range(m):
+        sgn = 1.0 if rec["bits"][i] else -1.0
+        for k in range(d):
+            y[k] += c * sgn * float(S[i][k])
+    return y

@@ -510,6 +510,67 @@ def decode_attention_gated(q: np.ndarray, hot_k: np.ndarray, hot_v: np.ndarray,
 
 
 # ---------------------------------------------------------------------------
+# Value-side QJL ("TurboQuant: kompresja KV-cache ...", section "Kompensacja
+# błędów przez QJL": the residual is coded with one bit per projection; here
+# applied to values as well as keys).  A value's record then also carries its
+# m sign bits and rn16, and the cold part of the output uses the residual's
+# QJL reconstruction sqrt(pi/2)/m * rn16 * S^T (2 bits - 1), whose expectation
+# over S is the residual itself.  READING: the same S as the keys; the
+# correction is added in the rotated domain before R^T, as c S^T (sum_t p_t
+# rn_t (2 bits_t - 1)) per query head with c = sqrt(pi/2)/m.
+# ---------------------------------------------------------------------------
+
+def qjl_vector_estimate(S: np.ndarray, bits: np.ndarray, rn: np.ndarray) -> np.ndarray:
+    """Per record the estimate of its residual vector r (rotated domain):
+    sqrt(pi/2)/m * rn * S^T (2 bits - 1).  bits [N, m], rn [N] -> [N, d]."""
+    S64 = np.asarray(S, dtype=np.float32).astype(np.float64)
+    m = S64.shape[0]
+    sg = 2.0 * np.asarray(bits, dtype=np.float64) - 1.0
+    return (sg @ S64) * (np.asarray(rn, dtype=np.float64) * (QJL_CONST / m))[:, None]
+
+
+def decode_attention_vqjl(q: np.ndarray, hot_k: np.ndarray, hot_v: np.ndarray,
+                          cold_k: Optional[Codes], cold_v: Optional[Codes],
+                          signs: np.ndarray, S: np.ndarray, num_kv_heads: int,
+                          softmax_scale: Optional[float] = None) -> np.ndarray:
+    """``decode_attention`` whose cold values also carry QJL bits: the cold
+    sum becomes sum_t p_t (s16_t/(2^b_r-1) v_hat_unit_t + r_hat_t) with
+    r_hat from ``qjl_vector_estimate``, then R^T.  cold_v entries need
+    ``bits`` and ``rn16``."""
+    q = np.asarray(q, dtype=np.float64)
+    hq, d = q.shape
+    g = hq // num_kv_heads
+    sigma = (1.0 / math.sqrt(d)) if softmax_scale is None else float(softmax_scale)
+    out = np.zeros((hq, d), dtype=np.float64)
+    for h in range(hq):
+        kvh = h // g
+        logits = []
+        if hot_k is not None and hot_k.shape[1] > 0:
+            logits.append(sigma * (np.asarray(hot_k[kvh], dtype=np.float64) @ q[h]))
+        n_cold = 0
+        if cold_k is not None and cold_k[kvh] is not None and cold_k[kvh].s16.shape[0] > 0:
+            n_cold = cold_k[kvh].s16.shape[0]
+            logits.append(sigma * key_inner_products(q[h], signs, S, cold_k[kvh]))
+        lg = np.concatenate(logits) if logits else np.zeros(0)
+        if lg.size == 0:
+            continue
+        p = np.exp(lg - lg.max())
+        p = p / p.sum()
+        n_hot = lg.size - n_cold
+        o = np.zeros(d, dtype=np.float64)
+        if n_hot:
+            o += p[:n_hot] @ np.asarray(hot_v[kvh], dtype=np.float64)
+        if n_cold:
+            cv = cold_v[kvh]
+            L = (1 << cv.b_r) - 1
+            y_hat = (cv.s16 / L)[:, None] * dequant_unit(cv.cr, cv.ct, cv.b_theta)
+            r_hat = qjl_vector_estimate(S, cv.bits, cv.rn16)
+            o += rotate_inverse(p[n_hot:] @ (y_hat + r_hat), signs)
+        out[h] = o
+    return out
+
+
+# ---------------------------------------------------------------------------
 # Tensor Cache second tier ("Tensor Cache: Eviction-conditioned Associative
 # Memory for Transformers", section "Metodología", items "Mecanismo de
 # Escritura", "Mecanismo de Lectura" and "Fusión").  The ring of W tokens is

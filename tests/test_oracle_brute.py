@@ -129,3 +129,18 @@ def test_tc_write_and_read_match_loops():
         Al = B.tc_write_loops(Al, list(k), list(v), 0.8, 0.3)
         np.testing.assert_allclose(A, Al, rtol=1e-12, atol=1e-12)
         np.testing.assert_allclose(q @ A, B.tc_read_loops(list(q), Al), rtol=1e-12, atol=1e-12)
+
+
+def test_value_qjl_estimate_matches_loops():
+    rng = np.random.default_rng(43)
+    d, m, b_r, b_t = 8, 8, 3, 3
+    signs = O.rotation_signs(4, d)
+    S = O.qjl_matrix(4, m, d)
+    x = rng.standard_normal((6, d))
+    c = O.encode(x, signs, S, b_r, b_t)
+    L = (1 << b_r) - 1
+    est = (c.s16 / L)[:, None] * O.dequant_unit(c.cr, c.ct, b_t) + O.qjl_vector_estimate(S, c.bits, c.rn16)
+    Sl = S.astype(np.float64).tolist()
+    for t in range(6):
+        rec = dict(s16=c.s16[t], cr=list(c.cr[t]), ct=list(c.ct[t]), rn16=c.rn16[t], bits=list(c.bits[t]))
+        np.testing.assert_allclose(est[t], B.value_estimate_loops(rec, Sl, b_r, b_t), rtol=1e-12, atol=1e-12)

@@ -524,3 +524,60 @@ def test_tc_decode_gate_limits():
         np.testing.assert_allclose(closed[h], local, rtol=1e-12, atol=1e-14)
         np.testing.assert_allclose(empty[h], local, rtol=1e-12, atol=1e-14)
         np.testing.assert_allclose(half[h], local + 0.5 * (q[h] @ A[g]), rtol=1e-12, atol=1e-12)
+
+
+# ---- value-side QJL (the residual's sign sketch reconstructs the vector) ---
+
+def test_qjl_vector_estimate_unbiased_and_variance():
+    """For s ~ N(0, I), E[sign(<s, r>) s] = sqrt(2/pi) r/|r|, so the
+    estimate sqrt(pi/2)/m |r| S^T sign(S r) has mean r; its variance falls
+    as 1/m."""
+    rng = np.random.default_rng(41)
+    d, N = 16, 6000
+    r = rng.standard_normal(d)
+    nr = np.linalg.norm(r)
+
+    def draws(m):
+        est = np.empty((N, d))
+        for t in range(N):
+            S = rng.standard_normal((m, d)).astype(np.float32)
+            bits = (S.astype(np.float64) @ r >= 0)[None]
+            est[t] = O.qjl_vector_estimate(S, bits, np.array([nr]))[0]
+        return est
+
+    e4 = draws(4)
+    e16 = draws(16)
+    for e in (e4, e16):
+        se = e.std(axis=0) / math.sqrt(N)
+        assert np.all(np.abs(e.mean(axis=0) - r) < 4.5 * se)
+    ratio = e4.var(axis=0).sum() / e16.var(axis=0).sum()
+    assert 3.0 < ratio < 5.0
+
+
+def test_value_qjl_attention_converges_to_exact_values():
+    """With the values' residual sketched by m bits, the cold part of the
+    output tends to the one with exact (rotated) values as m grows: the
+    error at m = 4096 is far below the error of the codes alone."""
+    rng = np.random.default_rng(42)
+    hq, hkv, d, nc, b = 2, 1, 16, 12, 2
+    q = rng.standard_normal((hq, d))
+    kx = rng.standard_normal((nc, d))
+    vx = rng.standard_normal((nc, d))
+    signs = O.rotation_signs(9, d)
+    errs = []
+    for m in (0, 64, 4096):
+        S = O.qjl_matrix(9, max(m, 8), d)
+        ck = [O.encode(kx, signs, S, b, b)]
+        cv = [O.encode(vx, signs, S, b, b)]
+        if m == 0:
+            out = O.decode_attention(q, None, None, ck, cv, signs, S, hkv)
+        else:
+            out = O.decode_attention_vqjl(q, None, None, ck, cv, signs, S, hkv)
+        # the same logits with exact values: p from the cold logits
+        exact = np.zeros((hq, d))
+        for h in range(hq):
+            lg = O.key_inner_products(q[h], signs, S, ck[0]) / math.sqrt(d)
+            p = np.exp(lg - lg.max())
+            exact[h] = (p / p.sum()) @ vx
+        errs.append(np.abs(out - exact).max())
+    assert errs[2] < 0.25 * errs[0] and errs[2] < errs[1]
