@@ -518,7 +518,7 @@ def run_gpu(args, wl):
                               "peak_kind": peak_kind,
                               "bytes_note": "512 B per ring token + 12 d^2 B of A per unit and layer"}
         result["hbm"] = None
-        result["gpu_launches"] = L * (2 + 3 + 1) * args.steps
+        result["gpu_launches"] = L * (2 + 2 + 1) * args.steps   # no q-prep without cold tokens
     if rank == 0 and world == 1 and not args.no_cpu_baseline and gate_tau is None and \
             not args.tensor_cache:
         sample = oracle_sample(wl, args.seed, kv_heads=1)

@@ -402,7 +402,9 @@ static tq_status launch_decode(tq_cache* c, const void* q, float* out, float sof
   qa.heads = cf.batch * cf.num_q_heads;
   qa.d = d;
   qa.m = cf.qjl_bits;
-  if (launch_qprep(qa, stream) != cudaSuccess) return TQ_ERR_CUDA;
+  // q-prep's outputs feed only the cold logits; a gated call always runs it
+  // (its gate is q-prep's programmatic dependent)
+  if ((pl.cold_ctas > 0 || gate) && launch_qprep(qa, stream) != cudaSuccess) return TQ_ERR_CUDA;
   if (gate) {
     GateArgs ga{};
     ga.q = (const __half*)q;

@@ -11,9 +11,11 @@
 //              eta lambda^(E-1-e) k_e v_e^T), equal to E sequential writes.
 //              Algorithmic bytes per unit: 8 d^2 (A read and written) plus
 //              4 d per evicted token.
-//   tc_read    one block per unit, one thread per column: every element of
-//              A is read once and multiplied by all G query heads of the
-//              unit.  4 d^2 bytes per unit.
+//   tc_read    one block per unit: 4 row groups x one thread per column,
+//              each thread loading its 1/4 column of A at once; every
+//              element of A is read once and multiplied by all G query heads
+//              of the unit, and the row groups' sums meet in shared memory.
+//              4 d^2 bytes per unit.
 #include <cmath>
 
 #include "tq_internal.cuh"
@@ -24,6 +26,7 @@ namespace {
 constexpr int kTcRows = 16;          // rows of A per update block
 constexpr int kTcBatch = 32;         // evicted tokens staged per pass
 constexpr int kTcMaxGroup = 8;
+constexpr int kTcReadSplit = 4;      // row groups of A per read block (threads = d x 4)
 
 template <int D>
 __global__ void __launch_bounds__(D) tc_update_kernel(const TcUpdateArgs a) {
@@ -68,28 +71,45 @@ __global__ void __launch_bounds__(D) tc_update_kernel(const TcUpdateArgs a) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(D) tc_read_kernel(const TcReadArgs a) {
+__global__ void __launch_bounds__(D * kTcReadSplit) tc_read_kernel(const TcReadArgs a) {
+  constexpr int R = D / kTcReadSplit;               // rows of A per thread
   __shared__ float qs[kTcMaxGroup][D];
+  __shared__ float part[kTcReadSplit - 1][kTcMaxGroup][D];
   const int unit = blockIdx.x, t = threadIdx.x;
+  const int col = t % D, grp = t / D;               // column, and row group of R rows
   const int head0 = unit * a.G;                     // b * Hq + kvh * G
-  for (int x = t; x < a.G * D; x += D) qs[x / D][x % D] = __half2float(a.q[(size_t)head0 * D + x]);
+  for (int x = t; x < a.G * D; x += D * kTcReadSplit)
+    qs[x / D][x % D] = __half2float(a.q[(size_t)head0 * D + x]);
+  const float* Au = a.A + (size_t)unit * D * D + (size_t)grp * R * D + col;
+  float av[R];
+#pragma unroll
+  for (int i = 0; i < R; ++i) av[i] = Au[(size_t)i * D];   // every load before any use
   __syncthreads();
-  const float* Au = a.A + (size_t)unit * D * D;
   float m[kTcMaxGroup];
 #pragma unroll
-  for (int g = 0; g < kTcMaxGroup; ++g) m[g] = 0.f;
-#pragma unroll 8
-  for (int i = 0; i < D; ++i) {
-    const float aij = Au[(size_t)i * D + t];
+  for (int g = 0; g < kTcMaxGroup; ++g) {
+    m[g] = 0.f;
+    if (g < a.G) {
+#pragma unroll
+      for (int i = 0; i < R; ++i) m[g] = fmaf(qs[g][grp * R + i], av[i], m[g]);
+    }
+  }
+  if (grp > 0) {
 #pragma unroll
     for (int g = 0; g < kTcMaxGroup; ++g)
-      if (g < a.G) m[g] = fmaf(qs[g][i], aij, m[g]);
+      if (g < a.G) part[grp - 1][g][col] = m[g];
   }
+  __syncthreads();
+  if (grp == 0) {
 #pragma unroll
-  for (int g = 0; g < kTcMaxGroup; ++g) {
-    if (g < a.G) {
-      const int h = head0 + g;
-      a.out[(size_t)h * D + t] += a.sig[h % a.Hq] * m[g];
+    for (int g = 0; g < kTcMaxGroup; ++g) {
+      if (g < a.G) {
+        float sum = m[g];
+#pragma unroll
+        for (int r = 0; r < kTcReadSplit - 1; ++r) sum += part[r][g][col];
+        const int h = head0 + g;
+        a.out[(size_t)h * D + col] += a.sig[h % a.Hq] * sum;
+      }
     }
   }
 }
@@ -110,9 +130,9 @@ cudaError_t launch_tc_update(const TcUpdateArgs& a, cudaStream_t s) {
 cudaError_t launch_tc_read(const TcReadArgs& a, cudaStream_t s) {
   if (a.G > kTcMaxGroup) return cudaErrorInvalidValue;
   if (a.d == 64)
-    tc_read_kernel<64><<<a.units, 64, 0, s>>>(a);
+    tc_read_kernel<64><<<a.units, 64 * kTcReadSplit, 0, s>>>(a);
   else if (a.d == 128)
-    tc_read_kernel<128><<<a.units, 128, 0, s>>>(a);
+    tc_read_kernel<128><<<a.units, 128 * kTcReadSplit, 0, s>>>(a);
   else
     return cudaErrorInvalidValue;
   return cudaGetLastError();
