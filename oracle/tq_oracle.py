@@ -571,6 +571,71 @@ def decode_attention_vqjl(q: np.ndarray, hot_k: np.ndarray, hot_v: np.ndarray,
 
 
 # ---------------------------------------------------------------------------
+# Attention-weighted promotion ("Monarch v3 ...", section "Cómo funciona",
+# item "Promoción Ponderada por Atención": cold tokens that receive high
+# attention return to the hot region, with a persistence mechanism against
+# thrashing; the benchmark command's --promotion-threshold 0.15 and
+# --sticky-threshold 3).  Oracle only (no kernel yet).
+# READINGS: a cold token's attention mass at a step is the mean, over the
+# query heads of its kv head, of its softmax weight in that step's decode;
+# its counter rises by one at every step where the mass is at least the
+# threshold and returns to 0 at any step where it is not; the token is
+# promoted at the step its counter reaches the sticky threshold, and its
+# counter is cleared.  A promoted token leaves the cold store and enters the
+# ring with its dequantized K and V, R^T (s16/(2^b_r-1) * unit pairs)
+# rounded to fp16; the ring's oldest token is then evicted to cold as usual.
+# ---------------------------------------------------------------------------
+
+def cold_attention_mass(p_cold: np.ndarray, num_kv_heads: int) -> np.ndarray:
+    """p_cold [Hq, n_cold] softmax weights of the cold tokens -> [Hkv, n_cold],
+    the mean over each kv head's query heads."""
+    p = np.asarray(p_cold, dtype=np.float64)
+    g = p.shape[0] // num_kv_heads
+    return p.reshape(num_kv_heads, g, -1).mean(axis=1)
+
+
+def promotion_step(counters: np.ndarray, mass: np.ndarray, threshold: float, sticky: int):
+    """One decode step of the sticky counters: returns (new counters, the
+    tokens promoted now).  counters and mass have the same shape."""
+    hit = np.asarray(mass, dtype=np.float64) >= threshold
+    c = np.where(hit, np.asarray(counters) + 1, 0)
+    promote = c >= sticky
+    return np.where(promote, 0, c), promote
+
+
+def cold_softmax_weights(q: np.ndarray, hot_k: np.ndarray, cold_k, signs: np.ndarray,
+                         S: Optional[np.ndarray], num_kv_heads: int,
+                         softmax_scale: Optional[float] = None) -> np.ndarray:
+    """The softmax weights ``decode_attention`` gives the cold tokens of each
+    query head (one softmax over hot and cold): [Hq, n_cold]."""
+    q = np.asarray(q, dtype=np.float64)
+    hq, d = q.shape
+    g = hq // num_kv_heads
+    sigma = (1.0 / math.sqrt(d)) if softmax_scale is None else float(softmax_scale)
+    n_cold = cold_k[0].s16.shape[0]
+    out = np.zeros((hq, n_cold))
+    for h in range(hq):
+        kvh = h // g
+        lc = sigma * key_inner_products(q[h], signs, S, cold_k[kvh])
+        lh = (sigma * (np.asarray(hot_k[kvh], dtype=np.float64) @ q[h])
+              if hot_k is not None and hot_k.shape[1] > 0 else np.zeros(0))
+        mx = max(lc.max(), lh.max() if lh.size else -np.inf)
+        den = np.exp(lc - mx).sum() + np.exp(lh - mx).sum()
+        out[h] = np.exp(lc - mx) / den
+    return out
+
+
+def dequant_vectors(codes: Codes, signs: np.ndarray) -> np.ndarray:
+    """fp16 reconstruction of coded vectors in the original basis:
+    R^T (s16/(2^b_r-1) * c_r (cos, sin)), rounded to fp16 (the hot ring's
+    format)."""
+    L = (1 << codes.b_r) - 1
+    y_hat = (np.asarray(codes.s16, dtype=np.float64) / L)[:, None] * dequant_unit(
+        codes.cr, codes.ct, codes.b_theta)
+    return fp16_round(rotate_inverse(y_hat, signs))
+
+
+# ---------------------------------------------------------------------------
 # Tensor Cache second tier ("Tensor Cache: Eviction-conditioned Associative
 # Memory for Transformers", section "Metodología", items "Mecanismo de
 # Escritura", "Mecanismo de Lectura" and "Fusión").  The ring of W tokens is

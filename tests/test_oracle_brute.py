@@ -144,3 +144,21 @@ def test_value_qjl_estimate_matches_loops():
     for t in range(6):
         rec = dict(s16=c.s16[t], cr=list(c.cr[t]), ct=list(c.ct[t]), rn16=c.rn16[t], bits=list(c.bits[t]))
         np.testing.assert_allclose(est[t], B.value_estimate_loops(rec, Sl, b_r, b_t), rtol=1e-12, atol=1e-12)
+
+
+def test_promoted_vectors_match_loops():
+    """A promoted token's fp16 K / V: the polar reconstruction rotated back,
+    against the loop restatement (dense Sylvester matrix, struct halves)."""
+    rng = np.random.default_rng(52)
+    d, b_r, b_t = 8, 4, 3
+    signs = O.rotation_signs(6, d)
+    c = O.encode(rng.standard_normal((5, d)), signs, None, b_r, b_t)
+    got = O.dequant_vectors(c, signs)
+    L = 2 ** b_r - 1
+    for t in range(5):
+        y = []
+        for j in range(d // 2):
+            a = c.ct[t][j] * 2.0 * math.pi / 2 ** b_t
+            y += [c.s16[t] / L * c.cr[t][j] * math.cos(a), c.s16[t] / L * c.cr[t][j] * math.sin(a)]
+        ref = [B.to_half(x) for x in B.rotate_inverse(y, list(signs))]
+        np.testing.assert_allclose(got[t], ref, rtol=0, atol=1e-6 * max(1.0, max(abs(x) for x in ref)))

@@ -581,3 +581,42 @@ def test_value_qjl_attention_converges_to_exact_values():
             exact[h] = (p / p.sum()) @ vx
         errs.append(np.abs(out - exact).max())
     assert errs[2] < 0.25 * errs[0] and errs[2] < errs[1]
+
+
+# ---- attention-weighted promotion with sticky counters (Monarch) ----------
+
+def test_promotion_counters_worked_sequence():
+    """Threshold 0.15, sticky 3, worked by hand: a miss resets the count,
+    equality counts as a hit, the third hit in a row promotes and clears."""
+    masses = [0.2, 0.15, 0.1, 0.3, 0.16, 0.9, 0.9, 0.0]
+    want_c = [1, 2, 0, 1, 2, 0, 1, 0]
+    want_p = [False, False, False, False, False, True, False, False]
+    c = np.zeros(1, dtype=np.int64)
+    for m, wc, wp in zip(masses, want_c, want_p):
+        c, p = O.promotion_step(c, np.array([m]), 0.15, 3)
+        assert c[0] == wc and p[0] == wp
+
+
+def test_cold_mass_and_weights():
+    """With no hot window each kv head's cold masses sum to 1; with one, the
+    cold weights and the hot weights of every head sum to 1 (recomputed
+    here from the hot logits with scipy's logsumexp)."""
+    from scipy.special import logsumexp
+    rng = np.random.default_rng(51)
+    hq, hkv, d, nc, nh = 4, 2, 8, 10, 3
+    q = rng.standard_normal((hq, d))
+    signs = O.rotation_signs(2, d)
+    S = O.qjl_matrix(2, 8, d)
+    ck = [O.encode(rng.standard_normal((nc, d)), signs, S, 3, 3) for _ in range(hkv)]
+    hk = rng.standard_normal((hkv, nh, d))
+    w0 = O.cold_softmax_weights(q, None, ck, signs, S, hkv)
+    np.testing.assert_allclose(O.cold_attention_mass(w0, hkv).sum(axis=1), 1.0, rtol=1e-12)
+    w = O.cold_softmax_weights(q, hk, ck, signs, S, hkv)
+    for h in range(hq):
+        g = h // (hq // hkv)
+        lc = O.key_inner_products(q[h], signs, S, ck[g]) / math.sqrt(d)
+        lh = hk[g] @ q[h] / math.sqrt(d)
+        lse = logsumexp(np.concatenate([lc, lh]))
+        np.testing.assert_allclose(w[h], np.exp(lc - lse), rtol=1e-12)
+    m = O.cold_attention_mass(w, hkv)
+    np.testing.assert_allclose(m[0], w[:2].mean(axis=0), rtol=1e-15)
