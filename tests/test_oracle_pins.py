@@ -620,3 +620,23 @@ def test_cold_mass_and_weights():
         np.testing.assert_allclose(w[h], np.exp(lc - lse), rtol=1e-12)
     m = O.cold_attention_mass(w, hkv)
     np.testing.assert_allclose(m[0], w[:2].mean(axis=0), rtol=1e-15)
+
+
+def test_qjl_vector_estimate_error_closed_form():
+    """E|r_hat - r|^2 = |r|^2 (pi d / (2 m) - 1 / m) for the sign-sketch
+    estimate of a vector (from E|s|^2 = d and E[sign(<s, r>) s] =
+    sqrt(2/pi) r/|r| for s ~ N(0, I)); so the sketch lowers a value's error
+    only when m > pi d / 2."""
+    rng = np.random.default_rng(44)
+    d, N = 16, 4000
+    r = rng.standard_normal(d)
+    nr2 = float(r @ r)
+    for m in (8, 32):
+        errs = np.empty(N)
+        for t in range(N):
+            S = rng.standard_normal((m, d)).astype(np.float32)
+            bits = (S.astype(np.float64) @ r >= 0)[None]
+            e = O.qjl_vector_estimate(S, bits, np.array([math.sqrt(nr2)]))[0] - r
+            errs[t] = e @ e
+        want = nr2 * (math.pi * d / (2 * m) - 1.0 / m)
+        assert abs(errs.mean() - want) < 4 * errs.std() / math.sqrt(N), (m, errs.mean(), want)
