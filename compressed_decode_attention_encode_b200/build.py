@@ -16,8 +16,9 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libtq.so")
-SOURCES = ["tq_host.cu", "tq_encode.cu", "tq_decode.cu", "tq_gate.cu", "tq_tcache.cu", "tq_search.cu"]
-HEADERS = ["tq_internal.cuh", "tq_encode_core.cuh", os.path.join("..", "..", "include", "tq.h")]
+SOURCES = ["tq_host.cu", "tq_encode.cu", "tq_decode.cu", "tq_gate.cu", "tq_tcache.cu", "tq_search.cu",
+           "tq_attend_64_64.cu", "tq_attend_64_128.cu", "tq_attend_128_64.cu", "tq_attend_128_128.cu"]
+HEADERS = ["tq_internal.cuh", "tq_encode_core.cuh", "tq_attend.cuh", os.path.join("..", "..", "include", "tq.h")]
 
 NVCC_FLAGS = [
     "-O3", "-lineinfo", "-std=c++17",
@@ -42,14 +43,34 @@ def _stale() -> bool:
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
+    """Compile each source to an object (in parallel, under _build/ at the
+    repository root), then link them into libtq.so."""
     if not force and not _stale():
         return LIB
+    from concurrent.futures import ThreadPoolExecutor
+
+    obj_dir = os.path.join(ROOT, "_build")
+    os.makedirs(obj_dir, exist_ok=True)
+    compile_flags = [f for f in NVCC_FLAGS if f != "-shared"]
+    jobs = []
+    for src in SOURCES:
+        obj = os.path.join(obj_dir, os.path.splitext(src)[0] + ".o")
+        jobs.append((obj, [nvcc_path(), *compile_flags, "-I", os.path.join(ROOT, "include"),
+                           "-c", "-o", obj, os.path.join(CSRC, src)]))
+
+    def run(job):
+        if verbose:
+            print(" ".join(job[1]), file=sys.stderr)
+        subprocess.run(job[1], check=True)
+
+    with ThreadPoolExecutor(max_workers=len(jobs)) as pool:
+        list(pool.map(run, jobs))
     tmp = LIB + ".tmp"
-    cmd = [nvcc_path(), *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"),
-           "-o", tmp, *[os.path.join(CSRC, s) for s in SOURCES]]
+    link = [nvcc_path(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared",
+            "-Xcompiler", "-fPIC", "-o", tmp, *[o for o, _ in jobs]]
     if verbose:
-        print(" ".join(cmd), file=sys.stderr)
-    subprocess.run(cmd, check=True)
+        print(" ".join(link), file=sys.stderr)
+    subprocess.run(link, check=True)
     os.replace(tmp, LIB)
     return LIB
 

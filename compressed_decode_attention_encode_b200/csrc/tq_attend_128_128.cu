@@ -1,0 +1,11 @@
+// Attention kernels for head_dim 128 and 128 QJL bits (every code width and
+// head map; see tq_attend.cuh).
+#include "tq_attend.cuh"
+
+namespace tq {
+
+att::AttendFn attend_pick_128_128(int bw, int b_theta, int G, bool gate, int* smem) {
+  return att::attend_fn_dm<128, 128>(bw, b_theta, G, gate, smem);
+}
+
+}  // namespace tq

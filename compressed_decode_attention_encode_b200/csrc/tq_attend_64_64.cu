@@ -1,0 +1,11 @@
+// Attention kernels for head_dim 64 and 64 QJL bits (every code width and
+// head map; see tq_attend.cuh).
+#include "tq_attend.cuh"
+
+namespace tq {
+
+att::AttendFn attend_pick_64_64(int bw, int b_theta, int G, bool gate, int* smem) {
+  return att::attend_fn_dm<64, 64>(bw, b_theta, G, gate, smem);
+}
+
+}  // namespace tq

@@ -184,7 +184,8 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
       }, val, mask);
       merge_word(reinterpret_cast<uint32_t*>(tb + L.off_vc + lane_word_offset(w, l, L.vwt)), val, mask);
     }
-    // sign words: lanes (gid = 2c + e, tig); m/4 bits per (token, tig)
+    // sign words: lanes (gid = 2c + e, tig); m/4 signs per (token, tig), local
+    // sign j at chunk bit sign_chunk_bit(j, h, m)
     const int qb = L.m / 4;
     for (int q = lane; q < 8 * L.sw; q += 32) {
       const int ch = q / L.sw, w = q % L.sw;
@@ -193,14 +194,14 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
       uint32_t val = 0u, mask = 0u;
       for (int h = 0; h < 2; ++h) {
         const int s = e + 2 * h;
-        const int bit0 = h * qb - 32 * w;        // chunk bit of this token's first sign
-        if (!inr[s] || bit0 >= 32 || bit0 + qb <= 0) continue;
-        // qb is 16 or 32: the token's bits lie in one word
-        const int i0 = tig * qb;                 // first canonical sign index
-        const uint32_t src = kb[s * 8 + (i0 >> 5)] >> (i0 & 31);
-        const uint32_t m32 = qb == 32 ? 0xffffffffu : ((1u << qb) - 1u);
-        val |= (src & m32) << bit0;
-        mask |= m32 << bit0;
+        if (!inr[s]) continue;
+        for (int j = 0; j < qb; ++j) {
+          const int bit = sign_chunk_bit(j, h, L.m) - 32 * w;
+          if (bit < 0 || bit >= 32) continue;
+          const int i = tig * qb + j;            // canonical sign index
+          val |= ((kb[s * 8 + (i >> 5)] >> (i & 31)) & 1u) << bit;
+          mask |= 1u << bit;
+        }
       }
       merge_word(reinterpret_cast<uint32_t*>(tb + L.off_ks + lane_word_offset(w, l, L.sw)), val, mask);
     }
@@ -395,17 +396,20 @@ __global__ void __launch_bounds__(2 * D) encode_small_kernel(EncodeArgs a) {
     }, val, mask);
     merge_atomic(tb + L.off_vc + lane_word_offset(w, 4 * gv + cgrp, L.vwt), val, mask);
   }
-  // sign words: lanes (gid, tig); m/4 bits per (token, tig), in one word
+  // sign words: lanes (gid, tig); m/4 signs per (token, tig), local sign j
+  // at chunk bit sign_chunk_bit(j, h, m)
   const int qb = L.m / 4;
   for (int q = tid; q < 4 * L.sw; q += blockDim.x) {
     const int tg = q / L.sw, w = q % L.sw;
-    const int bit0 = h * qb - 32 * w;
-    if (bit0 >= 32 || bit0 + qb <= 0) continue;
-    const int i0 = tg * qb;
-    const uint32_t srcw = bits[i0 >> 5] >> (i0 & 31);
-    const uint32_t m32 = qb == 32 ? 0xffffffffu : ((1u << qb) - 1u);
-    merge_atomic(tb + L.off_ks + lane_word_offset(w, 4 * gid + tg, L.sw), (srcw & m32) << bit0,
-                 m32 << bit0);
+    uint32_t val = 0u, mask = 0u;
+    for (int j = 0; j < qb; ++j) {
+      const int bit = sign_chunk_bit(j, h, L.m) - 32 * w;
+      if (bit < 0 || bit >= 32) continue;
+      const int i = tg * qb + j;
+      val |= ((bits[i >> 5] >> (i & 31)) & 1u) << bit;
+      mask |= 1u << bit;
+    }
+    merge_atomic(tb + L.off_ks + lane_word_offset(w, 4 * gid + tg, L.sw), val, mask);
   }
   if (tid == 0) {
     uint16_t* ks = reinterpret_cast<uint16_t*>(tb + L.off_ksc);

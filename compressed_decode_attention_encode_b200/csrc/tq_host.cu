@@ -57,7 +57,8 @@ bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 }  // namespace
 
 struct WsLayout {
-  size_t status, signs, S, St, qrot, qsk, qscale, part, gate, gate_max, total;
+  size_t status, signs, S, St, q, part, gate, gate_max, total;
+  QBufsLayout ql;               // query transforms, at offset q
 };
 
 static WsLayout ws_layout(const tq_config& c) {
@@ -70,9 +71,8 @@ static WsLayout ws_layout(const tq_config& c) {
   w.signs = off;  off += round_up(sizeof(double) * c.head_dim, kAlign);
   w.S = off;      off += round_up(sizeof(float) * c.head_dim * c.qjl_bits, kAlign);
   w.St = off;     off += round_up(sizeof(float) * c.head_dim * c.qjl_bits, kAlign);
-  w.qrot = off;   off += round_up(2 * 2 * heads * c.head_dim, kAlign);
-  w.qsk = off;    off += round_up(2 * heads * c.qjl_bits, kAlign);
-  w.qscale = off; off += round_up(sizeof(float) * 2 * heads, kAlign);
+  w.ql = qbufs_layout(heads, c.head_dim, c.qjl_bits);
+  w.q = off;      off += w.ql.total;
   w.part = off;   off += round_up(sizeof(float) * units * (kSlotsCold + kSlotsHot) * G * (c.head_dim + 2), kAlign);
   // gated decode: head_skip [heads], unit_pos [units], alist [units + 1], n_active, then the
   // gate blocks' maxima [heads, ceil(W / kGateRowsMin)]
@@ -121,6 +121,7 @@ struct tq_cache {
   int device;
   cudaEvent_t ev_start;
   cudaEvent_t ev_stop;
+  unsigned long long wait_limit_ns;   // attention kernel's bounded waits (tq_set_wait_limit)
   __half* hot_k() const { return (__half*)hot; }
   __half* hot_v() const {
     return (__half*)(hot + (size_t)cfg.batch * cfg.num_kv_heads * cfg.hot_window * cfg.head_dim * 2);
@@ -183,6 +184,7 @@ tq_status tq_cache_create(const tq_config* cfg, void* hot_mem, void* cold_mem,
   c->dirty_lo = 0;
   c->dirty_n = 0;
   c->tc = c->tc_lam = c->tc_eta = c->tc_sig = nullptr;
+  c->wait_limit_ns = kDefaultWaitLimitNs;
   if (cudaGetDevice(&c->device) != cudaSuccess ||
       cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, c->device) != cudaSuccess) {
     delete c;
@@ -345,8 +347,10 @@ static SplitPlan make_plan(int64_t n_cold, int n_hot, int units, int ctas, bool 
   SplitPlan pl{};
   pl.cold_blocks = cold_blocks;
   pl.hot_tiles = hot_tiles;
-  pl.slots_cold = kSlotsCold;
-  pl.slots_hot = kSlotsHot;
+  // tight: a side with no work reserves no slots (the kernels only use
+  // slots below the counts they compute from the same plan)
+  pl.slots_cold = tight ? 0 : kSlotsCold;
+  pl.slots_hot = tight ? 0 : kSlotsHot;
   if (Nh > 0) {
     int64_t tpc = (Nh + ctas - 1) / ctas;
     // a unit's tiles may span at most kSlotsHot - 2 CTAs
@@ -381,8 +385,8 @@ struct GateBuffers {
 // partials into the output rows.  Scratch buffers are the caller's
 // (workspace or static scratch).
 static tq_status launch_decode(tq_cache* c, const void* q, float* out, float softmax_scale,
-                               const SplitPlan& pl, __half* qrot, __half* qsk, float* qscale,
-                               float* part, cudaStream_t stream, const GateBuffers* gate = nullptr) {
+                               const SplitPlan& pl, const QBufs& qb, float* part, cudaStream_t stream,
+                               const GateBuffers* gate = nullptr) {
   const tq_config& cf = c->cfg;
   const int d = cf.head_dim;
   const int units = cf.batch * cf.num_kv_heads;
@@ -396,12 +400,11 @@ static tq_status launch_decode(tq_cache* c, const void* q, float* out, float sof
   qa.q = (const __half*)q;
   qa.signs = c->signs();
   qa.St = c->St();
-  qa.qrot = qrot;
-  qa.qsk = qsk;
-  qa.qscale = qscale;
+  qa.out = qb;
   qa.heads = cf.batch * cf.num_q_heads;
   qa.d = d;
   qa.m = cf.qjl_bits;
+  qa.b_theta = cf.b_theta;
   // q-prep's outputs feed only the cold logits; a gated call always runs it
   // (its gate is q-prep's programmatic dependent)
   if ((pl.cold_ctas > 0 || gate) && launch_qprep(qa, stream) != cudaSuccess) return TQ_ERR_CUDA;
@@ -429,9 +432,10 @@ static tq_status launch_decode(tq_cache* c, const void* q, float* out, float sof
   }
   AttendArgs a{};
   a.q = (const __half*)q;
-  a.qrot = qrot;
-  a.qsk = qsk;
-  a.qscale = qscale;
+  a.qrot = qb.qrot;
+  a.qk8 = qb.qk8;
+  a.qs8 = qb.qs8;
+  a.qscale = qb.qscale;
   a.hot_k = c->hot_k();
   a.hot_v = c->hot_v();
   a.cold = c->cold;
@@ -447,6 +451,7 @@ static tq_status launch_decode(tq_cache* c, const void* q, float* out, float sof
   a.n_cold = c->n_cold;
   a.plan = pl;
   a.log2e_sigma = (float)(1.4426950408889634 * (double)sigma);
+  a.wait_limit_ns = c->wait_limit_ns;
   if (gate) {
     a.alist = gate->alist;
     a.n_active = gate->n_active;
@@ -456,6 +461,7 @@ static tq_status launch_decode(tq_cache* c, const void* q, float* out, float sof
   if (c->ev_stop && cudaEventRecord(c->ev_stop, stream) != cudaSuccess) return TQ_ERR_CUDA;
   CombineArgs ca{};
   ca.part = part;
+  ca.status = c->status();
   ca.signs = c->signs();
   ca.out = out;
   ca.units = units;
@@ -493,8 +499,7 @@ tq_status tq_decode_attention(tq_cache* c, const void* q, float* out, float soft
     return TQ_ERR_INVALID_ARG;
   const int units = c->cfg.batch * c->cfg.num_kv_heads;
   const SplitPlan pl = make_plan(c->n_cold, c->n_hot, units, c->num_sms * c->ctas_per_sm, false);
-  return launch_decode(c, q, out, softmax_scale, pl, (__half*)(c->ws + c->W.qrot),
-                       (__half*)(c->ws + c->W.qsk), (float*)(c->ws + c->W.qscale),
+  return launch_decode(c, q, out, softmax_scale, pl, qbufs_at(c->ws + c->W.q, c->W.ql),
                        (float*)(c->ws + c->W.part), stream);
 }
 
@@ -519,8 +524,7 @@ tq_status tq_decode_attention_gated(tq_cache* c, const void* q, float* out, floa
   if (pl.cold_ctas == 0 && pl.hot_ctas == 0 &&        // nothing cached: no head skips
       cudaMemsetAsync(gb.head_skip, 0, sizeof(int) * heads, stream) != cudaSuccess)
     return TQ_ERR_CUDA;
-  return launch_decode(c, q, out, softmax_scale, pl, (__half*)(c->ws + c->W.qrot),
-                       (__half*)(c->ws + c->W.qsk), (float*)(c->ws + c->W.qscale),
+  return launch_decode(c, q, out, softmax_scale, pl, qbufs_at(c->ws + c->W.q, c->W.ql),
                        (float*)(c->ws + c->W.part), stream, &gb);
 }
 
@@ -565,6 +569,12 @@ tq_status tq_tc_enable(tq_cache* c, void* tc_mem, const float* lambda, const flo
   c->tc_lam = p;
   c->tc_eta = p + hkv;
   c->tc_sig = p + 2 * hkv;
+  return TQ_OK;
+}
+
+tq_status tq_set_wait_limit(tq_cache* c, int64_t limit_ns) {
+  if (!c) return TQ_ERR_INVALID_ARG;
+  c->wait_limit_ns = limit_ns < 0 ? kDefaultWaitLimitNs : (unsigned long long)limit_ns;
   return TQ_OK;
 }
 
@@ -627,19 +637,16 @@ tq_status tq_decode_attention_static(tq_cache* c, const void* q, float* out, flo
   // unit cut to the most any unit can receive under this plan.
   const SplitPlan pl = make_plan(c->n_cold, c->n_hot, units, c->num_sms * c->ctas_per_sm, true);
 
-  // scratch layout: rotated queries | q'' | per-head scales | partials
-  size_t off = 0;
-  const size_t o_qrot = off;   off += round_up((size_t)2 * 2 * heads * d, kAlign);
-  const size_t o_qsk = off;    off += round_up((size_t)2 * heads * m, kAlign);
-  const size_t o_qscale = off; off += round_up(sizeof(float) * 2 * heads, kAlign);
+  // scratch layout: query transforms | partials
+  const QBufsLayout ql = qbufs_layout((size_t)heads, d, m);
+  size_t off = ql.total;
   const size_t o_part = off;
   off += round_up(sizeof(float) * units * (size_t)(pl.slots_cold + pl.slots_hot) * G * (d + 2), kAlign);
   if (off > kStaticScratchBytes) return TQ_ERR_CAPACITY;   // too large for the static scratch
 
   uint8_t* base = (uint8_t*)static_scratch_address(current);
   if (!base) return TQ_ERR_CUDA;
-  return launch_decode(c, q, out, softmax_scale, pl, (__half*)(base + o_qrot), (__half*)(base + o_qsk),
-                       (float*)(base + o_qscale), (float*)(base + o_part), stream);
+  return launch_decode(c, q, out, softmax_scale, pl, qbufs_at(base, ql), (float*)(base + o_part), stream);
 }
 
 tq_status tq_get_status(tq_cache* c, cudaStream_t stream) {
@@ -716,10 +723,10 @@ tq_status tq_export_cold(tq_cache* c, int32_t row, int32_t kv_head, int64_t star
       uint8_t* out = k_bits + i * L.sg_bytes;
       std::memset(out, 0, L.sg_bytes);
       const int qb = L.m / 4;
-      for (int tig = 0; tig < 4; ++tig) {
-        const uint32_t v = chunk_bits(tile + L.off_ks, 4 * gid + tig, L.sw, h * qb, qb == 32 ? 32 : qb);
-        put_bits(out, tig * qb, qb == 32 ? v : (v & ((1u << qb) - 1)), qb);
-      }
+      for (int tig = 0; tig < 4; ++tig)
+        for (int j = 0; j < qb; ++j)
+          put_bits(out, tig * qb + j, chunk_bits(tile + L.off_ks, 4 * gid + tig, L.sw,
+                                                 sign_chunk_bit(j, h, L.m), 1), 1);
     }
     const uint16_t* ks = reinterpret_cast<const uint16_t*>(tile + L.off_ksc);
     const uint16_t* vs = reinterpret_cast<const uint16_t*>(tile + L.off_vsc);

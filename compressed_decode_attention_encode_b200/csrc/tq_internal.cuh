@@ -20,14 +20,23 @@ constexpr int kTilesPerBlock = kTokensPerBlock / kTokensPerTile;
 constexpr int kStatusRange = 1;
 constexpr int kStatusTimeout = 2;
 constexpr int kStatusLayout = 4;    // a kernel found shared memory where its layout does not fit
+// Latched errors after which an attention launch wrote no partials: while
+// one is latched, the merge writes NaN rather than stale partials.
+constexpr int kStatusNoPartials = kStatusTimeout | kStatusLayout;
+
+// Default limit of the attention kernel's bounded mbarrier waits.
+constexpr unsigned long long kDefaultWaitLimitNs = 2000000000ull;
 
 // Cold-store layout.  Per (row, kv head): 64-token blocks of 4 tiles.  A
 // tile (16 tokens) is laid out fragment-major for the decode warp that
 // reads it: lane l = 4*gid + tig owns
 //   K codes : tokens gid and gid+8, pairs [tig*PT, tig*PT + PT), PT = d/8
 //             (code k of token half h at bit (h*PT + k)*bw of the lane chunk)
-//   K signs : tokens gid and gid+8, sign bits [tig*m/4, (tig+1)*m/4)
-//             (m = 128: word h = token half h; m = 64: bits 16h.. of word 0)
+//   K signs : tokens gid and gid+8, sign bits [tig*m/4, (tig+1)*m/4); local
+//             sign j = 8 s + 4 hf + e (e < 4) of token half h sits at bit
+//             8 e + 2 s + hf of word h (m = 128) or at bit 8 e + 4 h + 2 s +
+//             hf of word 0 (m = 64): a shift by 2 s + hf (+ 4 h) and a mask
+//             0x01010101 give the 0/1 bytes of one int8 MMA operand
 //   V codes : tokens 2tig, 2tig+1, 2tig+8, 2tig+9 (slot 0..3), pairs
 //             [gid*PV, gid*PV + PV), PV = d/16 (code k of slot s at bit
 //             (s*PV + k)*bw)
@@ -59,6 +68,13 @@ __host__ __device__ inline int words_for_bits(int bits) { return (bits + 31) / 3
 __host__ __device__ inline int lane_word_offset(int w, int l, int nw) {
   const int width = ((w | 1) < nw) ? 8 : 4;
   return (w >> 1) * 256 + l * width + (w & 1) * 4;
+}
+
+// Bit of the lane's sign chunk (words concatenated) holding local sign j
+// (0 <= j < m/4) of token half h.
+__host__ __device__ inline int sign_chunk_bit(int j, int h, int m) {
+  const int e = j & 3, hf = (j >> 2) & 1, s = j >> 3;
+  return m == 128 ? 32 * h + 8 * e + 2 * s + hf : 8 * e + 4 * h + 2 * s + hf;
 }
 
 __host__ __device__ inline Layout layout_of(int d, int b_r, int b_theta, int m, int64_t capacity) {
@@ -146,15 +162,53 @@ cudaError_t launch_ring_write(__half* ring_k, __half* ring_v, const __half* k_ne
                               int first, int ring_pos, cudaStream_t s);
 
 // ---- decode -------------------------------------------------------------
+// Query transforms of one decode call (written by q-prep, per query head h):
+//   qrot   [h][2][d]       q' * a1 as fp16 hi and lo parts (a1 a power of 2)
+//   qk8    [h][2][d/16][32] int8 planes (hi, lo) of the projections of q'
+//                          on the slot directions, in int8 B-fragment order
+//   qs8    [h][2][m/32][32] int8 planes of q'' = S q', B-fragment order
+//   qscale [h][4]          1/a1, alpha_k, alpha_s (the planes' value of one
+//                          unit: x = alpha (256 hi + lo)), and the integer
+//                          sum of q'' / alpha_s (int32 bits)
+// Byte (plane, s, t, 4 hf + e) of qk8 is slot e of pair t * d/8 + 2 s + hf;
+// of qs8 it is sign t * m/4 + 8 s + 4 hf + e.
+struct QBufs {
+  __half* qrot;
+  int8_t* qk8;
+  int8_t* qs8;
+  float* qscale;
+};
+
+// Offsets of the query transforms in a scratch area (256-byte aligned).
+struct QBufsLayout {
+  size_t qrot, qk8, qs8, qscale, total;
+};
+
+inline QBufsLayout qbufs_layout(size_t heads, int d, int m) {
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+  QBufsLayout l{};
+  size_t off = 0;
+  l.qrot = off;   off += up(heads * 2 * d * 2);
+  l.qk8 = off;    off += up(heads * 2 * (d / 16) * 32);
+  l.qs8 = off;    off += up(heads * 2 * (m / 32) * 32);
+  l.qscale = off; off += up(heads * 4 * sizeof(float));
+  l.total = off;
+  return l;
+}
+
+inline QBufs qbufs_at(uint8_t* base, const QBufsLayout& l) {
+  return QBufs{(__half*)(base + l.qrot), (int8_t*)(base + l.qk8), (int8_t*)(base + l.qs8),
+               (float*)(base + l.qscale)};
+}
+
 struct QPrepArgs {
   const __half* q;          // [B*Hq, d]
   const double* signs;      // [d]
   const float* St;          // [d, m]
-  __half* qrot;             // [B*Hq, 2, d]  q' * alpha' as fp16 hi and lo parts
-  __half* qsk;              // [B*Hq, m]     q'' * alpha'' in sign-fragment order
-  float* qscale;            // [B*Hq, 2]     1/alpha', 1/alpha''
+  QBufs out;
   int heads;                // B*Hq
   int d, m;
+  int b_theta;              // slot directions: 2^(b_theta-1) (b_theta <= 3), else unused
 };
 
 cudaError_t launch_qprep(const QPrepArgs& a, cudaStream_t s);
@@ -195,9 +249,10 @@ __host__ __device__ inline void gated_cold_split(int64_t n_active, int64_t nb, i
 // Partial record per (unit, slot, head): {m (log2 units), l, o[d]}.
 struct AttendArgs {
   const __half* q;          // [B*Hq, d]  (hot logits use q itself)
-  const __half* qrot;       // [B*Hq, 2, d]
-  const __half* qsk;        // [B*Hq, m]
-  const float* qscale;      // [B*Hq, 2]
+  const __half* qrot;       // query transforms (QBufs)
+  const int8_t* qk8;
+  const int8_t* qs8;
+  const float* qscale;
   const __half* hot_k;      // [units, W, d]
   const __half* hot_v;
   const uint8_t* cold;
@@ -209,6 +264,10 @@ struct AttendArgs {
   int W, n_hot;
   int64_t n_cold;
   float log2e_sigma;        // log2(e) * softmax scale
+  // Limit of each bounded wait for a cold tile's bulk copy; 0 makes every
+  // such wait give up at once (a forced timeout).  The copies already issued
+  // are then drained under kDefaultWaitLimitNs before the CTA exits.
+  unsigned long long wait_limit_ns;
   // gated calls only (null otherwise): the units whose cold tier is read,
   // in unit order, and their count (written by gate_kernel)
   const int* alist;         // [units + 1]
@@ -220,6 +279,7 @@ int attend_ctas_per_sm(const Layout& L, int G);
 
 struct CombineArgs {
   const float* part;
+  const int* status;        // device status word: NaN output while kStatusNoPartials is latched
   const double* signs;
   float* out;               // [B*Hq, d]
   SplitPlan plan;

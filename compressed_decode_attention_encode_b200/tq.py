@@ -64,6 +64,7 @@ SIGNATURES = [
     ("tq_tc_enable", c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
     ("tq_get_status", c_int32, [c_void_p, c_void_p]),
     ("tq_set_attend_events", c_int32, [c_void_p, c_void_p, c_void_p]),
+    ("tq_set_wait_limit", c_int32, [c_void_p, c_int64]),
     ("tq_export_cold", c_int32, [c_void_p, c_int32, c_int32, c_int64, c_int64, c_void_p,
                                  c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
     ("tq_vec_bytes", c_int32, [POINTER(tq_vec_config), c_int64, c_int32, POINTER(c_size_t),
@@ -191,6 +192,10 @@ def tq_set_attend_events(handle: int, start: int, stop: int) -> None:
     _check(lib().tq_set_attend_events(handle, start, stop), "tq_set_attend_events")
 
 
+def tq_set_wait_limit(handle: int, limit_ns: int) -> None:
+    _check(lib().tq_set_wait_limit(handle, limit_ns), "tq_set_wait_limit")
+
+
 def tq_rotation_signs(seed: int, d: int) -> np.ndarray:
     out = np.empty(d, dtype=np.int8)
     _check(lib().tq_rotation_signs(seed, d, out.ctypes.data_as(POINTER(c_int8))),
@@ -310,6 +315,11 @@ class TQCache:
         decode calls (None, None stops recording)."""
         tq_set_attend_events(self.handle, start.cuda_event if start is not None else None,
                              stop.cuda_event if stop is not None else None)
+
+    def set_wait_limit(self, limit_ns: int):
+        """Bounded-wait limit of the attention kernel (ns; 0 forces a
+        timeout at the first wait, < 0 restores the default)."""
+        tq_set_wait_limit(self.handle, limit_ns)
 
     def counts(self):
         return tq_cache_counts(self.handle)

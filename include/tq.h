@@ -255,8 +255,10 @@ tq_status tq_tc_enable(tq_cache* cache, void* tc_mem, const float* lambda, const
  * Synchronize `stream`, then return and clear the latched device status
  * (TQ_OK, TQ_ERR_RANGE or TQ_ERR_TIMEOUT; TQ_ERR_UNSUPPORTED when the
  * attention kernel found its dynamic shared memory at a window address its
- * table layout does not fit, in which case it wrote no output), or
- * TQ_ERR_CUDA if the stream itself reports an error.
+ * table layout does not fit), or TQ_ERR_CUDA if the stream itself reports
+ * an error.  After a timeout or that layout error an attention launch has
+ * written no partial results, so every decode call on the handle writes NaN
+ * to all of `out` until this call has cleared the status.
  */
 tq_status tq_get_status(tq_cache* cache, cudaStream_t stream);
 
@@ -346,6 +348,17 @@ tq_status tq_export_vectors(tq_vec_index* index, const void* codes, int64_t star
  * to stop recording.  The events are borrowed, not owned.
  */
 tq_status tq_set_attend_events(tq_cache* cache, cudaEvent_t start, cudaEvent_t stop);
+
+/*
+ * Limit of each bounded wait in the attention kernel (the wait for a cold
+ * tile's bulk copy; the pages have no counterpart: this serves failure
+ * testing).  limit_ns < 0 restores the default of 2 s.  limit_ns = 0 makes
+ * every such wait give up at once, without polling, which forces the
+ * timeout path: the kernel latches TQ_ERR_TIMEOUT, waits (under the default
+ * limit) for the copies it already issued, and returns without partials.
+ * Applies to the following decode calls on this handle.
+ */
+tq_status tq_set_wait_limit(tq_cache* cache, int64_t limit_ns);
 
 /*
  * The library's own seeded method randomness (host only, no GPU needed),

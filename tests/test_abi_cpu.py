@@ -106,6 +106,7 @@ def test_null_arguments_rejected_before_device(lib):
     assert lib.tq_evict_window(None, None, None, 1, None) == 1
     assert lib.tq_decode_attention(None, None, None, 0.0, None) == 1
     assert lib.tq_get_status(None, None) == 1
+    assert lib.tq_set_wait_limit(None, 0) == 1
     assert lib.tq_cache_destroy(None) == 0
     assert lib.tq_rotation_signs(0, 0, None) == 1
 

@@ -35,7 +35,10 @@ def _oracle_codes(exp, dim, b_r, b_t, m):
 
 
 def _check_topk(scores, idx, ref_scores, k):
-    """GPU (scores, idx) [nq, k] against oracle scores [nq, n]."""
+    """GPU (scores, idx) [nq, k] against oracle scores [nq, n]: the returned
+    entries are valid (each within tol of the oracle's k-th best, scores
+    matching, no duplicates, descending) and complete (nothing scoring more
+    than tol above the lowest returned entry was left out)."""
     swaps = 0
     for i in range(ref_scores.shape[0]):
         row = ref_scores[i]
@@ -45,6 +48,11 @@ def _check_topk(scores, idx, ref_scores, k):
         got = idx[i]
         assert len(set(got.tolist())) == k, "duplicate indices"
         assert np.all(row[got] >= kth - tol), (i, row[got].min(), kth)
+        # complete: every entry that beats the lowest returned one by more
+        # than the tolerance was returned
+        must = np.nonzero(row > row[got].min() + tol)[0]
+        missing = set(must.tolist()) - set(got.tolist())
+        assert not missing, (i, sorted(missing)[:5])
         np.testing.assert_allclose(scores[i], row[got], rtol=0, atol=tol)
         assert np.all(np.diff(scores[i]) <= tol)            # descending
         swaps += len(set(order[:k].tolist()) - set(got.tolist()))

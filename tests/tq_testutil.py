@@ -111,3 +111,30 @@ def rel_err(got: np.ndarray, ref: np.ndarray) -> np.ndarray:
     num = np.linalg.norm(got - ref, axis=-1)
     den = np.linalg.norm(ref, axis=-1)
     return num / np.maximum(den, 1e-30)
+
+
+def oracle_decode_unit(cache: tq.TQCache, row: int, kv_head: int, q_row: np.ndarray,
+                       hot_k_unit: np.ndarray, hot_v_unit: np.ndarray, signs, S, scale=None):
+    """fp64 oracle attention for the query heads of one (row, kv head) unit,
+    fed the GPU's cold records of that unit only; [G, d]."""
+    cfg = cache.cfg
+    G = cfg.num_q_heads // cfg.num_kv_heads
+    nc = cache.counts()[0]
+    ck = cv = None
+    if nc:
+        exp = cache.export_cold(row, kv_head, 0, nc)
+        ck = [codes_from_export(exp, cfg, True)]
+        cv = [codes_from_export(exp, cfg, False)]
+    q = q_row[kv_head * G:(kv_head + 1) * G].astype(np.float64)
+    return O.decode_attention(q, hot_k_unit[None].astype(np.float64),
+                              hot_v_unit[None].astype(np.float64), ck, cv, signs, S, 1, scale)
+
+
+def cold_blocks_per_cta_lower_bound(units: int, n_cold: int) -> int:
+    """A lower bound on the cold blocks each attention CTA streams for this
+    cache, whatever the occupancy (at most 8 CTAs per SM): the plan gives a
+    CTA ceil(units * blocks / CTAs) blocks."""
+    import torch
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    blocks = units * ((n_cold + tq.TOKENS_PER_BLOCK - 1) // tq.TOKENS_PER_BLOCK)
+    return blocks // (sms * 8)
