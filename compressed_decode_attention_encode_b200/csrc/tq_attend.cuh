@@ -28,6 +28,7 @@
 #pragma once
 
 #include <cfloat>
+#include <type_traits>
 
 #include "tq_internal.cuh"
 
@@ -66,6 +67,16 @@ __device__ __forceinline__ void mma_s8(int (&c)[4], uint32_t a0, uint32_t a1, ui
       "{%8,%9}, {%0,%1,%2,%3};\n"
       : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// The same with a zero accumulator in (the first k-step of a product).
+__device__ __forceinline__ void mma_s8_z(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%10,%10,%10,%10};\n"
+      : "=r"(c[0]), "=r"(c[1]), "=r"(c[2]), "=r"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(0));
 }
 
 __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
@@ -126,11 +137,6 @@ __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count) : "memory");
 }
 
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes)
-               : "memory");
-}
-
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -142,11 +148,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Waits for phase `parity` of an mbarrier, giving up after `limit_ns`; a
-// limit of 0 gives up at once, without polling (a forced timeout).
+// Waits for phase `parity` of an mbarrier, giving up after `limit_ns`.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
                                                   unsigned long long limit_ns) {
-  if (limit_ns == 0) return false;
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   while (!mbar_try_wait(bar, parity)) {
@@ -155,21 +159,8 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
   return true;
 }
 
-// Global -> shared bulk copy completing on an mbarrier (no multicast).
-__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes,
-                                         uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(dst),
-      "l"(src), "r"(bytes), "r"(bar)
-      : "memory");
-}
-
 __device__ __forceinline__ void fence_barrier_init() {
   asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
-}
-
-__device__ __forceinline__ void fence_proxy_async() {
-  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
 }
 
 __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
@@ -186,16 +177,16 @@ __device__ __forceinline__ uint32_t sign_bytes(uint32_t x, int sh) {
 // named by the BW-bit field at bit `pos` of the lane's word stream (`pos`
 // is a compile-time constant after unrolling), plus `lane_off` (the lane's
 // copy inside the entry): one shift (a funnel shift for a field straddling
-// two words) and one three-input logic op, written in PTX so that the
-// compiler keeps it at two instructions.
+// two words) and one three-input logic op.
 template <int BW, int SH, int NW>
 __device__ __forceinline__ uint32_t lut_offset(const uint32_t (&w)[NW], int pos, uint32_t lane_off) {
   constexpr uint32_t kMask = ((1u << BW) - 1u) << SH;
   const int wi = pos >> 5, bi = pos & 31;
   uint32_t t, r;
   if (bi + BW <= 32 || wi + 1 >= NW) {
-    if (bi >= SH) asm("shr.b32 %0, %1, %2;" : "=r"(t) : "r"(w[wi]), "r"(bi - SH));
-    else asm("shl.b32 %0, %1, %2;" : "=r"(t) : "r"(w[wi]), "r"(SH - bi));
+    if (bi > SH) asm("shr.b32 %0, %1, %2;" : "=r"(t) : "r"(w[wi]), "r"(bi - SH));
+    else if (bi == SH) t = w[wi];
+    else t = w[wi] << (SH - bi);
   } else {
     asm("shf.r.wrap.b32 %0, %1, %2, %3;" : "=r"(t) : "r"(w[wi]), "r"(w[wi + 1]), "r"(bi - SH));
   }
@@ -220,10 +211,9 @@ struct AttendShape {
   static constexpr int NT = D / 16;                 // K k-steps (8 pairs each) == PV m-tiles
   static constexpr int QS = M / 32;                 // k-steps of the int8 QJL product
   static constexpr int PT = P / 4;                  // K pairs per lane (per token)
-  static constexpr int PV = P / 8;                  // V pairs per lane (per token)
   static constexpr int KWT = (2 * PT * BW + 31) / 32;
   static constexpr int SW = (2 * (M / 4) + 31) / 32;
-  static constexpr int VWT = (4 * PV * BW + 31) / 32;
+  static constexpr int VWT = KWT;                   // V codes: the K layout
   static constexpr int OFF_KC = 0;
   static constexpr int OFF_KS = OFF_KC + 128 * KWT;
   static constexpr int OFF_KSC = OFF_KS + 128 * SW;
@@ -426,7 +416,7 @@ __device__ __forceinline__ void flush_partial(WarpState<NT, HPL>& st, bool hot, 
     for (int w = 0; w < 4; ++w) mx = fmaxf(mx, mw[w * 8 + g]);
     f[hh] = st.ref[hh] == kNegInf ? 0.f : fast_exp2(st.ref[hh] - mx) * (hot ? 1.f : inv_levels);
   }
-  constexpr int P8 = D / 16;   // (D/2) / 8 pairs per gid for the cold mapping
+  constexpr int PT = D / 8;    // cold rows: pair (gid / 2) * PT + 2 i + r2, component gid % 2
   // the 4 warps add their rows in turn: no two threads touch one word at once
   for (int w = 0; w < 4; ++w) {
     if (warp == w) {
@@ -434,7 +424,7 @@ __device__ __forceinline__ void flush_partial(WarpState<NT, HPL>& st, bool hot, 
       for (int i = 0; i < NT; ++i) {
 #pragma unroll
         for (int r2 = 0; r2 < 2; ++r2) {
-          const int dim = hot ? (16 * i + gid + 8 * r2) : (2 * (P8 * gid + i) + r2);
+          const int dim = hot ? (16 * i + gid + 8 * r2) : (2 * ((gid >> 1) * PT + 2 * i + r2) + (gid & 1));
 #pragma unroll
           for (int hh = 0; hh < HPL; ++hh) {
             const int g = lane_head<HMAP>(tig, hh);
@@ -547,9 +537,20 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
       const int64_t uid = GATE ? (int64_t)a.alist[u] : u;
       nsrc = a.cold + ((size_t)uid * a.L.blocks_per_unit + (size_t)nblk_b) * S::BLOCK + warp * S::TT;
     }
-    auto fetch_next = [&](int s) {       // lane 0: the next tile into stage s
-      mbar_expect_tx(bar_w + 8 * s, S::TT);
-      bulk_g2s(ring_w + s * S::TT, nsrc, S::TT, bar_w + 8 * s);
+    // The next tile into stage s: every lane advances the (warp-uniform)
+    // stream; lane 0 alone arms the barrier and issues the copy, predicated
+    // rather than branched around.  `after_reads` orders the warp's reads of
+    // the stage's previous tile before the asynchronous write.
+    auto fetch_next = [&](int s, bool after_reads) {
+      const uint32_t bar = bar_w + 8 * s;
+      asm volatile(
+          "{\n .reg .pred p, f;\n setp.eq.u32 p, %0, 0;\n setp.ne.u32 f, %5, 0;\n"
+          " and.pred f, f, p;\n"
+          " @f fence.proxy.async.shared::cta;\n"
+          " @p mbarrier.arrive.expect_tx.shared::cta.b64 _, [%1], %2;\n"
+          " @p cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%3], [%4], %2, [%1];\n}\n"
+          ::"r"(lane), "r"(bar), "r"(S::TT), "r"(ring_w + s * S::TT), "l"(nsrc), "r"((int)after_reads)
+          : "memory");
       ++issued;
       nsrc += S::BLOCK;
       if (++nblk_b == nbi) {
@@ -564,8 +565,9 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
     if (lane == 0) {
       for (int s = 0; s < S::NS; ++s) mbar_init(bar_w + 8 * s, 1);
       fence_barrier_init();
-      for (int s = 0; s < S::NS && s < nblk; ++s) fetch_next(s);
     }
+    __syncwarp();
+    for (int s = 0; s < S::NS && s < nblk; ++s) fetch_next(s, false);
     // Tables of the code words e = (c_r << b_theta) | c_theta, one copy per
     // lane (the merge area is free at this point for the 2^bw distinct
     // entries, built once each).
@@ -600,11 +602,11 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
     __syncthreads();
 
     // B operands, loaded per unit:
-    //   SLOT  bk[nq][s]: the two int8 planes' projections of q' (column gid:
-    //         head 4 nq + gid / 2, plane gid % 2); bs[nq][s]: those of q''
+    //   SLOT  bk[nq][s]: the two int8 planes' projections of q' (column
+    //         2 t + pl: plane pl of head lane_head(t, nq)); bs[nq][s]:
+    //         those of q''
     //   HILO  bq[s]: q'_hi / q'_lo (packed: even / odd column of each head),
-    //         bq2[s]: q'_lo when not packed; bs as SLOT (one column group
-    //         of heads 0..3 when packed, else two)
+    //         bq2[s]: q'_lo when not packed; bs as SLOT
     constexpr int NQS = HPL;             // int8 column groups of the QJL product
     constexpr int kAccSplit = 2;         // independent accumulator chains
     uint32_t bk[SLOT ? NQ : 1][SLOT ? S::NT : 1][2];
@@ -612,103 +614,89 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
     uint32_t bs[NQS][S::QS][2];
     float kpol[HPL], kqjl[HPL];
     int qsum[HPL];
-    int unit_cur = -1;                    // active-list position when gated
-    int uid_cur = 0;                      // gated: the unit itself (alist[unit_cur])
-    int slot_cur = 0;
+    const bool forced_timeout = a.wait_limit_ns == 0;
     bool aborted = false;
-    int unit = (int)(f_lo / nb);          // advanced incrementally: no division per block
-    int blk = (int)(f_lo - (int64_t)unit * nb);   // block inside the unit (< 2^31)
-    const int tail = (int)(a.n_cold - (int64_t)(nbi - 1) * S::TB);   // valid tokens of a unit's last block
-    for (int i = 0; i < nblk; ++i, ++blk) {
-      if (blk == nbi) {
-        blk = 0;
-        ++unit;
+
+    // Loads the B operands and logit constants of unit position `u`.
+    auto setup_unit = [&](int u) {
+      const int uid = GATE ? a.alist[u] : u;
+      const int b = uid / a.Hkv, kvh = uid % a.Hkv;
+      const int head0 = b * a.Hq + kvh * G;
+#pragma unroll
+      for (int nq = 0; nq < NQS; ++nq) {
+        const int hc = lane_head<HMAP>(gid >> 1, nq), pln = gid & 1;
+        const bool live = hc < G;
+        const uint2* qs = reinterpret_cast<const uint2*>(a.qs8 + ((size_t)(head0 + hc) * 2 + pln) * S::QS * 32) + tig;
+#pragma unroll
+        for (int s = 0; s < S::QS; ++s) {
+          const uint2 v = live ? qs[4 * s] : make_uint2(0u, 0u);
+          bs[nq][s][0] = v.x;
+          bs[nq][s][1] = v.y;
+        }
+        if constexpr (SLOT) {
+          const uint2* qk = reinterpret_cast<const uint2*>(a.qk8 + ((size_t)(head0 + hc) * 2 + pln) * S::NT * 32) + tig;
+#pragma unroll
+          for (int s = 0; s < S::NT; ++s) {
+            const uint2 v = live ? qk[4 * s] : make_uint2(0u, 0u);
+            bk[nq][s][0] = v.x;
+            bk[nq][s][1] = v.y;
+          }
+        }
       }
-      if (unit != unit_cur) {
-        if (unit_cur >= 0) {
-          flush_partial<D, S::NT, HPL, HMAP>(st, false, inv_levels, G, merge,
-                                  a.part + (((size_t)(GATE ? uid_cur : unit_cur) * slots + slot_cur) * G) * (D + 2));
-          st.reset();
-        }
-        unit_cur = unit;
-        if constexpr (GATE) uid_cur = a.alist[unit];
-        slot_cur = c - (int)(((int64_t)unit * nb) / cold_bpc());
-        const int uid = GATE ? uid_cur : unit;
-        const int b = uid / a.Hkv, kvh = uid % a.Hkv;
-        const int head0 = b * a.Hq + kvh * G;
-        // int8 B columns: column 2 t + pl of group nq is plane pl of head
-        // lane_head(t, nq), so that lane tig's accumulator columns 2 tig,
-        // 2 tig + 1 are the two planes of its head number nq
+      if constexpr (!SLOT) {
+        // B column gid: head gid (8 heads) or, packed, head gid / 2 with
+        // column parity 0 = q'_hi, 1 = q'_lo (the A_lo product uses the
+        // even columns only)
+        const int hcol = PACKQ ? (gid >> 1) : gid;
+        const bool odd = PACKQ && (gid & 1);
+        if (hcol < G) {
+          const uint32_t* qp = reinterpret_cast<const uint32_t*>(a.qrot + (size_t)(head0 + hcol) * 2 * D) + S::PT * tig;
+          const int o1 = odd ? S::P : 0;
 #pragma unroll
-        for (int nq = 0; nq < NQS; ++nq) {
-          const int hc = lane_head<HMAP>(gid >> 1, nq), pln = gid & 1;
-          const bool live = hc < G;
-          const uint2* qs = reinterpret_cast<const uint2*>(a.qs8 + ((size_t)(head0 + hc) * 2 + pln) * S::QS * 32) + tig;
-#pragma unroll
-          for (int s = 0; s < S::QS; ++s) {
-            const uint2 v = live ? qs[4 * s] : make_uint2(0u, 0u);
-            bs[nq][s][0] = v.x;
-            bs[nq][s][1] = v.y;
-          }
-          if constexpr (SLOT) {
-            const uint2* qk = reinterpret_cast<const uint2*>(a.qk8 + ((size_t)(head0 + hc) * 2 + pln) * S::NT * 32) + tig;
-#pragma unroll
-            for (int s = 0; s < S::NT; ++s) {
-              const uint2 v = live ? qk[4 * s] : make_uint2(0u, 0u);
-              bk[nq][s][0] = v.x;
-              bk[nq][s][1] = v.y;
-            }
-          }
-        }
-        if constexpr (!SLOT) {
-          // B column gid: head gid (8 heads) or, packed, head gid / 2 with
-          // column parity 0 = q'_hi, 1 = q'_lo (the A_lo product uses the
-          // even columns only)
-          const int hcol = PACKQ ? (gid >> 1) : gid;
-          const bool odd = PACKQ && (gid & 1);
-          if (hcol < G) {
-            const uint32_t* qp = reinterpret_cast<const uint32_t*>(a.qrot + (size_t)(head0 + hcol) * 2 * D) + S::PT * tig;
-            const int o1 = odd ? S::P : 0;
-#pragma unroll
-            for (int s = 0; s < S::NT; ++s) {
-              bq[s][0] = qp[o1 + 2 * s];
-              bq[s][1] = qp[o1 + 2 * s + 1];
-              if constexpr (!PACKQ) {
-                bq2[s][0] = qp[S::P + 2 * s];
-                bq2[s][1] = qp[S::P + 2 * s + 1];
-              }
-            }
-          } else {
-#pragma unroll
-            for (int s = 0; s < S::NT; ++s) bq[s][0] = bq[s][1] = 0u;
+          for (int s = 0; s < S::NT; ++s) {
+            bq[s][0] = qp[o1 + 2 * s];
+            bq[s][1] = qp[o1 + 2 * s + 1];
             if constexpr (!PACKQ) {
-#pragma unroll
-              for (int s = 0; s < S::NT; ++s) bq2[s][0] = bq2[s][1] = 0u;
+              bq2[s][0] = qp[S::P + 2 * s];
+              bq2[s][1] = qp[S::P + 2 * s + 1];
             }
           }
-        }
+        } else {
 #pragma unroll
-        for (int hh = 0; hh < HPL; ++hh) {
-          const int g = lane_head<HMAP>(tig, hh);
-          const float* qsc = a.qscale + 4 * (size_t)(head0 + g);
-          const bool live = g < G;
-          kpol[hh] = live ? a.log2e_sigma * (SLOT ? qsc[1] : qsc[0]) * inv_levels : 0.f;
-          kqjl[hh] = live ? a.log2e_sigma * kSqrtHalfPi / (float)M * qsc[2] : 0.f;
-          qsum[hh] = live ? __float_as_int(qsc[3]) : 0;
+          for (int s = 0; s < S::NT; ++s) bq[s][0] = bq[s][1] = 0u;
+          if constexpr (!PACKQ) {
+#pragma unroll
+            for (int s = 0; s < S::NT; ++s) bq2[s][0] = bq2[s][1] = 0u;
+          }
         }
       }
-      // ---- wait for this tile's stage of the warp's ring --------------------
-      const int stage = i % S::NS;
+#pragma unroll
+      for (int hh = 0; hh < HPL; ++hh) {
+        const int g = lane_head<HMAP>(tig, hh);
+        const float* qsc = a.qscale + 4 * (size_t)(head0 + g);
+        const bool live = g < G;
+        kpol[hh] = live ? a.log2e_sigma * (SLOT ? qsc[1] : qsc[0]) * inv_levels : 0.f;
+        kqjl[hh] = live ? a.log2e_sigma * kSqrtHalfPi / (float)M * qsc[2] : 0.f;
+        qsum[hh] = live ? __float_as_int(qsc[3]) : 0;
+      }
+      return uid;
+    };
+
+    // One 16-token tile of block i (stage i % NS of the warp's ring): wait
+    // for its copy, compute, refill the stage with block i + NS.  MASKED
+    // tiles (a unit's last block) hold `nvalid` < 16 valid tokens.
+    auto tile_step = [&](int i, auto masked, int nvalid) {
+      constexpr bool MASKED = decltype(masked)::value;
+      const int stage = i % S::NS;         // NS need not be a power of two
       if (!aborted) {
-        const bool got = mbar_wait_bounded(bar_w + 8 * stage, (uint32_t)((i / S::NS) & 1), a.wait_limit_ns);
+        const bool got = !forced_timeout &&
+                         mbar_wait_bounded(bar_w + 8 * stage, (uint32_t)((i / S::NS) & 1), a.wait_limit_ns);
         if (!__all_sync(kFull, got)) {
           aborted = true;
           if (lane == 0) *abort_flag = 1;
         }
       }
-      const int left = (blk == nbi - 1 ? tail : S::TB) - tb;
-      if (!aborted && left > 0) {
-      const int nvalid = left < 16 ? (int)left : 16;     // valid tokens of this warp's tile
+      if (!aborted && (!MASKED || nvalid > 0)) {
       const uint32_t tile = ring_w + stage * S::TT;
 
       uint32_t kw[S::KWT], sw[S::SW], vw[S::VWT];
@@ -720,7 +708,7 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
 
       // ---- QJL part: 0/1 sign bytes (bit 8e + 2s + hf of the token's word;
       // for m = 64 the two tokens share one word, token gid + 8 at +4) ------
-      int cq[kAccSplit][NQS][4] = {};
+      int cq[NQS][4];
 #pragma unroll
       for (int s = 0; s < S::QS; ++s) {
         uint32_t r0, r1, r2, r3;
@@ -736,10 +724,13 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
           r3 = sign_bytes(sw[0], 4 + 2 * s + 1);
         }
 #pragma unroll
-        for (int nq = 0; nq < NQS; ++nq) mma_s8(cq[s % kAccSplit][nq], r0, r1, r2, r3, bs[nq][s][0], bs[nq][s][1]);
+        for (int nq = 0; nq < NQS; ++nq) {
+          if (s == 0) mma_s8_z(cq[nq], r0, r1, r2, r3, bs[nq][s][0], bs[nq][s][1]);
+          else mma_s8(cq[nq], r0, r1, r2, r3, bs[nq][s][0], bs[nq][s][1]);
+        }
       }
 
-      const bool v0 = gid < nvalid, v1 = gid + 8 < nvalid;
+      const bool v0 = !MASKED || gid < nvalid, v1 = !MASKED || gid + 8 < nvalid;
       const float sk0 = __half2float(__ushort_as_half((unsigned short)(ksc.x & 0xffffu)));
       const float sk1 = __half2float(__ushort_as_half((unsigned short)(ksc.x >> 16)));
       const float rn0 = __half2float(__ushort_as_half((unsigned short)(ksc.y & 0xffffu)));
@@ -750,16 +741,14 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
       for (int hh = 0; hh < HPL; ++hh) {       // group hh, columns 2 tig (hi), 2 tig + 1 (lo)
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
-          const int hi = cq[0][hh][2 * j] + cq[1][hh][2 * j];
-          const int lo = cq[0][hh][2 * j + 1] + cq[1][hh][2 * j + 1];
-          qj[j][hh] = (float)(2 * (256 * hi + lo) - qsum[hh]);
+          qj[j][hh] = (float)(2 * (256 * cq[hh][2 * j] + cq[hh][2 * j + 1]) - qsum[hh]);
         }
       }
       // entry j: token gid + 8 (j / HPL), head j % HPL
       float l2[2 * HPL];
       if constexpr (SLOT) {
         // ---- polar part: int8 slots . projection planes ------------------
-        int ck[kAccSplit][NQ][4] = {};
+        int ck[NQ][4];
 #pragma unroll
         for (int s = 0; s < S::NT; ++s) {
           const uint32_t o0 = lut_offset<BW, 7>(kw, (2 * s) * BW, lane_lut);
@@ -768,12 +757,15 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
           const uint32_t o3 = lut_offset<BW, 7>(kw, (S::PT + 2 * s + 1) * BW, lane_lut);
           const uint32_t a0 = lut_at<0>(o0), a1 = lut_at<0>(o1), a2 = lut_at<0>(o2), a3 = lut_at<0>(o3);
 #pragma unroll
-          for (int nq = 0; nq < NQ; ++nq) mma_s8(ck[s % kAccSplit][nq], a0, a1, a2, a3, bk[nq][s][0], bk[nq][s][1]);
+          for (int nq = 0; nq < NQ; ++nq) {
+            if (s == 0) mma_s8_z(ck[nq], a0, a1, a2, a3, bk[nq][s][0], bk[nq][s][1]);
+            else mma_s8(ck[nq], a0, a1, a2, a3, bk[nq][s][0], bk[nq][s][1]);
+          }
         }
 #pragma unroll
         for (int hh = 0; hh < HPL; ++hh) {
-          const int p0 = 256 * (ck[0][hh][0] + ck[1][hh][0]) + ck[0][hh][1] + ck[1][hh][1];
-          const int p1 = 256 * (ck[0][hh][2] + ck[1][hh][2]) + ck[0][hh][3] + ck[1][hh][3];
+          const int p0 = 256 * ck[hh][0] + ck[hh][1];
+          const int p1 = 256 * ck[hh][2] + ck[hh][3];
           l2[hh] = v0 ? fmaf(rn0 * kqjl[hh], qj[0][hh], sk0 * kpol[hh] * (float)p0) : kNegInf;
           l2[HPL + hh] = v1 ? fmaf(rn1 * kqjl[hh], qj[1][hh], sk1 * kpol[hh] * (float)p1) : kNegInf;
         }
@@ -819,24 +811,52 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
       uint32_t pb0, pb1;
       pv_fragments<HPL>(pv, pb0, pb1);
 
-      // ---- P V: V codes of pairs PV*gid + j for tokens 2tig, 2tig+1, +8, +9
+      // ---- P V: m-tile j's rows are the 4 lanes' pairs tig*PT + 2j (rows
+      // 0-7) and tig*PT + 2j + 1 (rows 8-15).  A lane's lookup of its pair
+      // of token gid (gid + 8) is row gid of an 8x8 [token x dim] fragment;
+      // movmatrix transposes it into the [dim x token] A fragment.
       constexpr int VOFF = SLOT ? S::LUT_BYTES : 0;    // the values' fp16 table
 #pragma unroll
       for (int j = 0; j < S::NT; ++j) {
-        const uint32_t L0 = lut_at<VOFF>(lut_offset<BW, 7>(vw, (0 * S::PV + j) * BW, lane_lut));
-        const uint32_t L1 = lut_at<VOFF>(lut_offset<BW, 7>(vw, (1 * S::PV + j) * BW, lane_lut));
-        const uint32_t L2 = lut_at<VOFF>(lut_offset<BW, 7>(vw, (2 * S::PV + j) * BW, lane_lut));
-        const uint32_t L3 = lut_at<VOFF>(lut_offset<BW, 7>(vw, (3 * S::PV + j) * BW, lane_lut));
-        mma16816(st.O[j], __byte_perm(L0, L1, 0x5410), __byte_perm(L0, L1, 0x7632),
-                 __byte_perm(L2, L3, 0x5410), __byte_perm(L2, L3, 0x7632), pb0, pb1);
+        const uint32_t L0 = lut_at<VOFF>(lut_offset<BW, 7>(vw, (2 * j) * BW, lane_lut));
+        const uint32_t L1 = lut_at<VOFF>(lut_offset<BW, 7>(vw, (2 * j + 1) * BW, lane_lut));
+        const uint32_t L2 = lut_at<VOFF>(lut_offset<BW, 7>(vw, (S::PT + 2 * j) * BW, lane_lut));
+        const uint32_t L3 = lut_at<VOFF>(lut_offset<BW, 7>(vw, (S::PT + 2 * j + 1) * BW, lane_lut));
+        mma16816(st.O[j], movmatrix_trans(L0), movmatrix_trans(L1), movmatrix_trans(L2),
+                 movmatrix_trans(L3), pb0, pb1);
       }
       }   // tile compute
       // ---- refill the stage with this warp's tile of block i + NS --------
       __syncwarp();
-      if (lane == 0 && !aborted && i + S::NS < nblk) {
-        fence_proxy_async();
-        fetch_next(stage);
+      if (!aborted && i + S::NS < nblk) fetch_next(stage, true);
+    };
+
+    // The run as segments of one unit each: the blocks before a unit's last
+    // one are full; its last block holds `tail` tokens.
+    const int tail = (int)(a.n_cold - (int64_t)(nbi - 1) * S::TB);   // valid tokens of a unit's last block
+    const std::integral_constant<bool, false> full_tile{};
+    const std::integral_constant<bool, true> masked_tile{};
+    int unit = (int)(f_lo / nb);
+    int blk = (int)(f_lo - (int64_t)unit * nb);   // block inside the unit (< 2^31)
+    int i = 0;
+    while (i < nblk) {
+      const int uid = setup_unit(unit);
+      const int slot = c - (int)(((int64_t)unit * nb) / cold_bpc());
+      const int seg = (nbi - blk) < (nblk - i) ? (nbi - blk) : (nblk - i);   // this unit's blocks in the run
+      const bool ends_unit = blk + seg == nbi;
+      const int n_full = (ends_unit && tail < S::TB) ? seg - 1 : seg;
+      const int i_end = i + seg, i_full = i + n_full;
+      for (; i < i_full; ++i) tile_step(i, full_tile, 16);
+      if (i < i_end) {
+        const int left = tail - tb;
+        tile_step(i, masked_tile, left < 16 ? left : 16);
+        ++i;
       }
+      flush_partial<D, S::NT, HPL, HMAP>(st, false, inv_levels, G, merge,
+                                         a.part + (((size_t)uid * slots + slot) * G) * (D + 2));
+      st.reset();
+      ++unit;
+      blk = 0;
     }
     __syncthreads();
     if (*abort_flag) {
@@ -849,11 +869,6 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
           mbar_wait_bounded(bar_w + 8 * s, (uint32_t)((n_s - 1) & 1), kDefaultWaitLimitNs);
         }
       return;
-    }
-    if (unit_cur >= 0) {
-      flush_partial<D, S::NT, HPL, HMAP>(st, false, inv_levels, G, merge,
-                              a.part + (((size_t)(GATE ? uid_cur : unit_cur) * slots + slot_cur) * G) * (D + 2));
-      st.reset();
     }
   }
   if (c < pl.hot_ctas) {

@@ -171,15 +171,16 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
       }, val, mask);
       merge_word(reinterpret_cast<uint32_t*>(tb + L.off_kc + lane_word_offset(w, l, L.kwt)), val, mask);
     }
-    // V code words: lanes (gid_v, tig = c), codes q: slot q / pv, pair gid_v*pv + q % pv
+    // V code words: the K layout
     for (int q = lane; q < 8 * L.vwt; q += 32) {
-      const int gv = q / L.vwt, w = q % L.vwt;
-      const int l = 4 * gv + c;
+      const int ch = q / L.vwt, w = q % L.vwt;
+      const int e = ch / 4, tig = ch % 4;
+      const int l = 4 * (2 * c + e) + tig;
       uint32_t val, mask;
-      chunk_word(w, 4 * L.pv, bw, [&](int qi, uint32_t* out) {
-        const int s = qi / L.pv, k = qi % L.pv;
+      chunk_word(w, 2 * L.pt, bw, [&](int qi, uint32_t* out) {
+        const int h = qi / L.pt, k = qi % L.pt, s = e + 2 * h;
         if (!inr[s]) return false;
-        *out = vc[s * P + gv * L.pv + k];
+        *out = vc[s * P + tig * L.pt + k];
         return true;
       }, val, mask);
       merge_word(reinterpret_cast<uint32_t*>(tb + L.off_vc + lane_word_offset(w, l, L.vwt)), val, mask);
@@ -384,17 +385,16 @@ __global__ void __launch_bounds__(2 * D) encode_small_kernel(EncodeArgs a) {
     }, val, mask);
     merge_atomic(tb + L.off_kc + lane_word_offset(w, 4 * gid + tg, L.kwt), val, mask);
   }
-  // V code words: lanes (gv, c = gid / 2), codes q of slot s: pair gv * pv + q % pv
-  const int cgrp = gid >> 1, slot_v = (gid & 1) + 2 * h;
-  for (int q = tid; q < 8 * L.vwt; q += blockDim.x) {
-    const int gv = q / L.vwt, w = q % L.vwt;
+  // V code words: the K layout
+  for (int q = tid; q < 4 * L.vwt; q += blockDim.x) {
+    const int tg = q / L.vwt, w = q % L.vwt;
     uint32_t val, mask;
-    chunk_word(w, 4 * L.pv, bw, [&](int qi, uint32_t* out) {
-      if (qi / L.pv != slot_v) return false;
-      *out = codes[P + gv * L.pv + qi % L.pv];
+    chunk_word(w, 2 * L.pt, bw, [&](int qi, uint32_t* out) {
+      if (qi / L.pt != h) return false;
+      *out = codes[P + tg * L.pt + qi % L.pt];
       return true;
     }, val, mask);
-    merge_atomic(tb + L.off_vc + lane_word_offset(w, 4 * gv + cgrp, L.vwt), val, mask);
+    merge_atomic(tb + L.off_vc + lane_word_offset(w, 4 * gid + tg, L.vwt), val, mask);
   }
   // sign words: lanes (gid, tig); m/4 signs per (token, tig), local sign j
   // at chunk bit sign_chunk_bit(j, h, m)

@@ -713,10 +713,9 @@ tq_status tq_export_cold(tq_cache* c, int32_t row, int32_t kv_head, int64_t star
     if (v_codes) {
       uint8_t* out = v_codes + i * L.kc_bytes;
       std::memset(out, 0, L.kc_bytes);
-      const int tig = (r % 8) / 2, slot = (r % 2) + 2 * h;
       for (int p = 0; p < L.pairs; ++p) {
-        const int gv = p / L.pv, k = p % L.pv;
-        put_bits(out, p * bw, chunk_bits(tile + L.off_vc, 4 * gv + tig, L.vwt, (slot * L.pv + k) * bw, bw), bw);
+        const int tig = p / L.pt, k = p % L.pt;
+        put_bits(out, p * bw, chunk_bits(tile + L.off_vc, 4 * gid + tig, L.vwt, (h * L.pt + k) * bw, bw), bw);
       }
     }
     if (k_bits) {

@@ -37,9 +37,10 @@ constexpr unsigned long long kDefaultWaitLimitNs = 2000000000ull;
 //             8 e + 2 s + hf of word h (m = 128) or at bit 8 e + 4 h + 2 s +
 //             hf of word 0 (m = 64): a shift by 2 s + hf (+ 4 h) and a mask
 //             0x01010101 give the 0/1 bytes of one int8 MMA operand
-//   V codes : tokens 2tig, 2tig+1, 2tig+8, 2tig+9 (slot 0..3), pairs
-//             [gid*PV, gid*PV + PV), PV = d/16 (code k of slot s at bit
-//             (s*PV + k)*bw)
+//   V codes : as the K codes (tokens gid and gid+8, pairs [tig*PT,
+//             tig*PT + PT)): a lane's looked-up pair is one row of an 8x8
+//             [token x dim] fragment, which movmatrix turns into the
+//             [dim x token] operand of the P V product
 // Per-lane word streams are stored "2-word-major": words 2g, 2g+1 of every
 // lane sit together (8 bytes per lane) so a warp reads them with one
 // conflict-free 64-bit load.  Per-token scalars are grouped by gid:
@@ -54,7 +55,7 @@ struct Layout {
   int m;            // QJL bits
   int kc_bytes;     // canonical packed code bytes per vector: pairs * bw / 8
   int sg_bytes;     // m / 8
-  int pt, pv;       // pairs per lane in the K / V fragments
+  int pt;           // pairs per lane (per token) in the K and V fragments
   int kwt, sw, vwt; // 32-bit words per lane: K codes, K signs, V codes
   int off_kc, off_ks, off_ksc, off_vc, off_vsc;   // plane offsets inside a tile
   int tile_bytes;
@@ -88,10 +89,9 @@ __host__ __device__ inline Layout layout_of(int d, int b_r, int b_theta, int m, 
   L.kc_bytes = L.pairs * L.bw / 8;
   L.sg_bytes = m / 8;
   L.pt = L.pairs / 4;
-  L.pv = L.pairs / 8;
   L.kwt = words_for_bits(2 * L.pt * L.bw);
   L.sw = words_for_bits(2 * (m / 4));
-  L.vwt = words_for_bits(4 * L.pv * L.bw);
+  L.vwt = L.kwt;
   L.off_kc = 0;
   L.off_ks = L.off_kc + 128 * L.kwt;
   L.off_ksc = L.off_ks + 128 * L.sw;

@@ -575,7 +575,7 @@ def decode_attention_vqjl(q: np.ndarray, hot_k: np.ndarray, hot_v: np.ndarray,
 # item "Promoción Ponderada por Atención": cold tokens that receive high
 # attention return to the hot region, with a persistence mechanism against
 # thrashing; the benchmark command's --promotion-threshold 0.15 and
-# --sticky-threshold 3).  Oracle only (no kernel yet).
+# --sticky-threshold 3).
 # READINGS: a cold token's attention mass at a step is the mean, over the
 # query heads of its kv head, of its softmax weight in that step's decode;
 # its counter rises by one at every step where the mass is at least the
@@ -584,6 +584,7 @@ def decode_attention_vqjl(q: np.ndarray, hot_k: np.ndarray, hot_v: np.ndarray,
 # counter is cleared.  A promoted token leaves the cold store and enters the
 # ring with its dequantized K and V, R^T (s16/(2^b_r-1) * unit pairs)
 # rounded to fp16; the ring's oldest token is then evicted to cold as usual.
+# ``PromotingUnit`` replays a unit step by step.
 # ---------------------------------------------------------------------------
 
 def cold_attention_mass(p_cold: np.ndarray, num_kv_heads: int) -> np.ndarray:
@@ -633,6 +634,89 @@ def dequant_vectors(codes: Codes, signs: np.ndarray) -> np.ndarray:
     y_hat = (np.asarray(codes.s16, dtype=np.float64) / L)[:, None] * dequant_unit(
         codes.cr, codes.ct, codes.b_theta)
     return fp16_round(rotate_inverse(y_hat, signs))
+
+
+class PromotingUnit:
+    """One (batch row, kv head) of a cache with attention-weighted promotion:
+    a hot ring of W tokens, a cold list indexed by cold position, the sticky
+    counters and the tokens promoted by the last decode.
+
+    READINGS (beyond those of ``promotion_step`` above): a decode decides the
+    promotions from its own masses; they are applied at the next insert,
+    where the promoted tokens (their dequantized fp16 K and V, oldest cold
+    index first) enter the ring before the new tokens, so that a new token
+    is the newest; every insert into a full ring evicts the oldest ring
+    token, and an evicted token takes the cold index of the earliest still
+    open promoted position (ascending), or is appended when none is left.
+    So each unit's cold list grows by exactly the number of new tokens.  A
+    promotion decided while the ring is not full is dropped (the token stays
+    cold; its counter was cleared).  The vectors held here are whatever the
+    caller inserts: fp16 values for the ring, raw vectors for the cold list
+    (the caller encodes them)."""
+
+    def __init__(self, W: int, d: int, threshold: float, sticky: int):
+        self.W, self.d = W, d
+        self.threshold, self.sticky = float(threshold), int(sticky)
+        self.ring_k = np.zeros((W, d))
+        self.ring_v = np.zeros((W, d))
+        self.ring_pos = 0
+        self.n_hot = 0
+        self.cold_k: list = []           # cold position -> raw key vector
+        self.cold_v: list = []
+        self.counters = np.zeros(0, dtype=np.int64)
+        self.pending: list = []          # cold positions promoted by the last decode
+
+    def append_cold(self, k: np.ndarray, v: np.ndarray) -> None:
+        """Prefill: tokens encoded straight into the cold list."""
+        for kk, vv in zip(np.asarray(k, dtype=np.float64), np.asarray(v, dtype=np.float64)):
+            self.cold_k.append(kk.copy())
+            self.cold_v.append(vv.copy())
+        self.counters = np.concatenate([self.counters, np.zeros(len(k), dtype=np.int64)])
+
+    def insert(self, k_new: np.ndarray, v_new: np.ndarray, promoted_k: np.ndarray,
+               promoted_v: np.ndarray) -> list:
+        """Insert the pending promoted tokens (given as their fp16
+        dequantization, in ``pending`` order) and then the new tokens;
+        returns the cold positions written, in eviction order."""
+        holes = list(self.pending)
+        self.pending = []
+        assert len(promoted_k) == len(holes)
+        seq_k = list(np.asarray(promoted_k, dtype=np.float64)) + list(np.asarray(k_new, dtype=np.float64))
+        seq_v = list(np.asarray(promoted_v, dtype=np.float64)) + list(np.asarray(v_new, dtype=np.float64))
+        written = []
+        for kk, vv in zip(seq_k, seq_v):
+            if self.n_hot == self.W:
+                old_k = self.ring_k[self.ring_pos].copy()
+                old_v = self.ring_v[self.ring_pos].copy()
+                if holes:
+                    i = holes.pop(0)
+                    self.cold_k[i], self.cold_v[i] = old_k, old_v
+                    self.counters[i] = 0
+                else:
+                    i = len(self.cold_k)
+                    self.cold_k.append(old_k)
+                    self.cold_v.append(old_v)
+                    self.counters = np.append(self.counters, 0)
+                written.append(i)
+            else:
+                self.n_hot += 1
+            self.ring_k[self.ring_pos] = kk
+            self.ring_v[self.ring_pos] = vv
+            self.ring_pos = (self.ring_pos + 1) % self.W
+        assert not holes, "promotions are only kept while the ring is full"
+        return written
+
+    def after_decode(self, mass: np.ndarray) -> np.ndarray:
+        """Counters after a decode whose cold tokens got ``mass``; returns the
+        promoted positions (ascending), which become ``pending``."""
+        self.counters, promote = promotion_step(self.counters, mass, self.threshold, self.sticky)
+        if self.n_hot < self.W:
+            promote = np.zeros_like(promote)
+        self.pending = [int(i) for i in np.nonzero(promote)[0]]
+        return np.array(self.pending, dtype=np.int64)
+
+    def hot_slots(self):
+        return self.ring_k, self.ring_v
 
 
 # ---------------------------------------------------------------------------

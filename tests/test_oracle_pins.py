@@ -640,3 +640,71 @@ def test_qjl_vector_estimate_error_closed_form():
             errs[t] = e @ e
         want = nr2 * (math.pi * d / (2 * m) - 1.0 / m)
         assert abs(errs.mean() - want) < 4 * errs.std() / math.sqrt(N), (m, errs.mean(), want)
+
+
+def _tags(xs):
+    return [int(round(float(x[0]))) for x in xs]
+
+
+def test_promoting_unit_hand_worked_trace():
+    """W = 2, threshold 0.15, sticky 2, tokens tagged by value; worked by
+    hand: a promoted token re-enters the ring before the new token, the
+    eviction it causes takes the promoted cold position, the next one is
+    appended."""
+    u = O.PromotingUnit(W=2, d=1, threshold=0.15, sticky=2)
+    a, b, c, d, e, f, g = ([[float(t)]] for t in (1, 2, 3, 4, 5, 6, 7))
+    u.append_cold(np.array(a + b + c), np.array(a + b + c))
+    assert u.insert(np.array(d + e), np.array(d + e), np.zeros((0, 1)), np.zeros((0, 1))) == []
+    assert list(u.after_decode(np.array([0.1, 0.5, 0.0]))) == []
+    assert list(u.counters) == [0, 1, 0]
+    assert u.insert(np.array(f), np.array(f), np.zeros((0, 1)), np.zeros((0, 1))) == [3]   # d appended
+    assert list(u.after_decode(np.array([0.2, 0.6, 0.0, 0.3]))) == [1]                    # b promoted
+    assert list(u.counters) == [1, 0, 0, 1]
+    b_deq = np.array([[1002.0]])           # stands in for b's fp16 dequantization
+    assert u.insert(np.array(g), np.array(g), b_deq, b_deq) == [1, 4]   # e takes b's place, f appended
+    assert _tags(u.cold_k) == [1, 5, 3, 4, 6]
+    assert list(u.counters) == [1, 0, 0, 1, 0]
+    assert _tags(u.ring_k) == [7, 1002] and u.ring_pos == 1
+    assert list(u.after_decode(np.array([0.0, 0.0, 0.0, 0.0, 0.9]))) == []
+    assert list(u.counters) == [0, 0, 0, 0, 1]
+
+
+def test_promoting_unit_drops_promotions_before_the_ring_is_full():
+    u = O.PromotingUnit(W=3, d=1, threshold=0.15, sticky=1)
+    u.append_cold(np.array([[1.0]]), np.array([[1.0]]))
+    u.insert(np.array([[2.0]]), np.array([[2.0]]), np.zeros((0, 1)), np.zeros((0, 1)))
+    assert list(u.after_decode(np.array([0.9]))) == [] and u.pending == []
+    assert list(u.counters) == [0]
+
+
+def test_promoting_unit_conserves_tokens():
+    """Random masses over many steps: every inserted token is in the ring or
+    the cold list exactly once (a promoted one as its stand-in), the cold
+    list grows by one per inserted token once the ring is full, and no step
+    promotes more than floor(1 / threshold) tokens."""
+    rng = np.random.default_rng(61)
+    W, thr = 4, 0.15
+    u = O.PromotingUnit(W=W, d=1, threshold=thr, sticky=2)
+    u.append_cold(np.arange(100, 110, dtype=np.float64)[:, None], np.zeros((10, 1)))
+    u.insert(np.arange(200, 204, dtype=np.float64)[:, None], np.zeros((4, 1)), np.zeros((0, 1)),
+             np.zeros((0, 1)))
+    alive = set(range(100, 110)) | set(range(200, 204))
+    nxt = 300
+    for step in range(200):
+        n_before = len(u.cold_k)
+        # a promoted token t re-enters as a stand-in tagged 10 t + 5
+        old = [int(round(u.cold_k[i][0])) for i in u.pending]
+        for t in old:
+            alive.remove(t)
+            alive.add(10 * t + 5)
+        prom_tags = np.array([[10.0 * t + 5] for t in old]).reshape(-1, 1)
+        u.insert(np.array([[float(nxt)]]), np.zeros((1, 1)), prom_tags, np.zeros_like(prom_tags))
+        alive.add(nxt)
+        nxt += 1
+        assert len(u.cold_k) == n_before + 1
+        have = sorted(_tags(u.cold_k) + _tags(u.ring_k))
+        assert have == sorted(alive)
+        n = len(u.cold_k)
+        raw = rng.dirichlet(np.full(n, 0.05))          # a peaked mass vector summing to 1
+        p = u.after_decode(raw * rng.uniform(0.5, 1.0))
+        assert len(p) <= int(1 / thr)
