@@ -17,7 +17,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libtq.so")
 SOURCES = ["tq_host.cu", "tq_encode.cu", "tq_decode.cu", "tq_gate.cu", "tq_tcache.cu", "tq_search.cu",
-           "tq_attend_64_64.cu", "tq_attend_64_128.cu", "tq_attend_128_64.cu", "tq_attend_128_128.cu"]
+           "tq_promote.cu", "tq_attend_64_64.cu", "tq_attend_64_128.cu", "tq_attend_128_64.cu", "tq_attend_128_128.cu"]
 HEADERS = ["tq_internal.cuh", "tq_encode_core.cuh", "tq_attend.cuh", os.path.join("..", "..", "include", "tq.h")]
 
 NVCC_FLAGS = [

@@ -459,10 +459,15 @@ __device__ __forceinline__ void flush_partial(WarpState<NT, HPL>& st, bool hot, 
 // ---------------------------------------------------------------------------
 // The kernel.  SLOT selects the int8 polar path (b_theta <= 3); HMAP the
 // heads a lane holds on the cold path (HMAP_PACK for groups of up to 4;
-// HMAP_SPLIT for larger SLOT groups, HMAP_PAIR for larger HILO groups).
+// HMAP_SPLIT for larger SLOT groups, HMAP_PAIR for larger HILO groups);
+// MODE: plain, gated (the cold tier of listed units only) or with every
+// cold token's logits written out (promotion).
 // ---------------------------------------------------------------------------
-template <int D, int M, int BW, bool SLOT, int HMAP, bool GATE>
+enum { MODE_PLAIN = 0, MODE_GATED = 1, MODE_LOGITS = 2 };
+
+template <int D, int M, int BW, bool SLOT, int HMAP, int MODE>
 __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(const AttendArgs a) {
+  constexpr bool GATE = MODE == MODE_GATED;
   using S = AttendShape<D, M, BW>;
   constexpr int HPL = HMAP == HMAP_PACK ? 1 : 2;     // query heads per lane on the cold path
   constexpr int NQ = SLOT ? HPL : 1;                 // int8 MMAs per k-step (column groups)
@@ -685,7 +690,7 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
     // One 16-token tile of block i (stage i % NS of the warp's ring): wait
     // for its copy, compute, refill the stage with block i + NS.  MASKED
     // tiles (a unit's last block) hold `nvalid` < 16 valid tokens.
-    auto tile_step = [&](int i, auto masked, int nvalid) {
+    auto tile_step = [&](int i, auto masked, int nvalid, int uid, int64_t tok0) {
       constexpr bool MASKED = decltype(masked)::value;
       const int stage = i % S::NS;         // NS need not be a power of two
       if (!aborted) {
@@ -803,6 +808,15 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
           l2[3] = v1 ? fmaf(rn1 * kqjl[1], qj[1][1], sk1 * kpol[1] * cp[3]) : kNegInf;
         }
       }
+      if constexpr (MODE == MODE_LOGITS) {     // promotion: every valid token's logits
+#pragma unroll
+        for (int hh = 0; hh < HPL; ++hh) {
+          const int g = lane_head<HMAP>(tig, hh);
+          float* lp = a.logits + ((size_t)uid * a.logit_capacity + tok0 + gid) * G + g;
+          if (g < G && v0) lp[0] = l2[hh];
+          if (g < G && v1) lp[8 * G] = l2[HPL + hh];
+        }
+      }
       // V weights of tokens past the end are 0 (their records are not written)
       const float sv0 = v0 ? __half2float(__ushort_as_half((unsigned short)(vsc & 0xffffu))) : 0.f;
       const float sv1 = v1 ? __half2float(__ushort_as_half((unsigned short)(vsc >> 16))) : 0.f;
@@ -846,10 +860,11 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
       const bool ends_unit = blk + seg == nbi;
       const int n_full = (ends_unit && tail < S::TB) ? seg - 1 : seg;
       const int i_end = i + seg, i_full = i + n_full;
-      for (; i < i_full; ++i) tile_step(i, full_tile, 16);
+      const int64_t tok_first = (int64_t)(blk - i) * S::TB + tb;   // + 64 i: this warp's first token
+      for (; i < i_full; ++i) tile_step(i, full_tile, 16, uid, tok_first + (int64_t)i * S::TB);
       if (i < i_end) {
         const int left = tail - tb;
-        tile_step(i, masked_tile, left < 16 ? left : 16);
+        tile_step(i, masked_tile, left < 16 ? left : 16, uid, tok_first + (int64_t)i * S::TB);
         ++i;
       }
       flush_partial<D, S::NT, HPL, HMAP>(st, false, inv_levels, G, merge,
@@ -971,29 +986,34 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
 // ---------------------------------------------------------------------------
 typedef void (*AttendFn)(const AttendArgs);
 
+template <int D, int M, int BW, bool SLOT, int HMAP>
+AttendFn attend_fn_mode(int mode) {
+  if (mode == MODE_GATED) return attend_kernel<D, M, BW, SLOT, HMAP, MODE_GATED>;
+  if (mode == MODE_LOGITS) return attend_kernel<D, M, BW, SLOT, HMAP, MODE_LOGITS>;
+  return attend_kernel<D, M, BW, SLOT, HMAP, MODE_PLAIN>;
+}
+
 template <int D, int M, int BW, bool SLOT>
-AttendFn attend_fn_bw(int hmap, bool gate) {
+AttendFn attend_fn_bw(int hmap, int mode) {
   if constexpr (SLOT) {
-    if (hmap == HMAP_PACK)
-      return gate ? attend_kernel<D, M, BW, true, HMAP_PACK, true> : attend_kernel<D, M, BW, true, HMAP_PACK, false>;
-    return gate ? attend_kernel<D, M, BW, true, HMAP_SPLIT, true> : attend_kernel<D, M, BW, true, HMAP_SPLIT, false>;
+    if (hmap == HMAP_PACK) return attend_fn_mode<D, M, BW, true, HMAP_PACK>(mode);
+    return attend_fn_mode<D, M, BW, true, HMAP_SPLIT>(mode);
   } else {
-    if (hmap == HMAP_PACK)
-      return gate ? attend_kernel<D, M, BW, false, HMAP_PACK, true> : attend_kernel<D, M, BW, false, HMAP_PACK, false>;
-    return gate ? attend_kernel<D, M, BW, false, HMAP_PAIR, true> : attend_kernel<D, M, BW, false, HMAP_PAIR, false>;
+    if (hmap == HMAP_PACK) return attend_fn_mode<D, M, BW, false, HMAP_PACK>(mode);
+    return attend_fn_mode<D, M, BW, false, HMAP_PAIR>(mode);
   }
 }
 
 // SLOT for b_theta <= 3 (code widths 2..8), HILO for b_theta >= 4 (5..8).
 template <int D, int M>
-AttendFn attend_fn_dm(int bw, int b_theta, int G, bool gate, int* smem) {
+AttendFn attend_fn_dm(int bw, int b_theta, int G, int mode, int* smem) {
   const bool slot = b_theta <= 3;
   const int hmap = G <= 4 ? HMAP_PACK : (slot ? HMAP_SPLIT : HMAP_PAIR);
 #define TQ_BW_CASE(B)                                                             \
   case B:                                                                         \
     *smem = AttendShape<D, M, B>::SMEM;                                           \
-    if (slot) return attend_fn_bw<D, M, B, true>(hmap, gate);                     \
-    if constexpr (B >= 5) return attend_fn_bw<D, M, B, false>(hmap, gate);        \
+    if (slot) return attend_fn_bw<D, M, B, true>(hmap, mode);                     \
+    if constexpr (B >= 5) return attend_fn_bw<D, M, B, false>(hmap, mode);        \
     return nullptr;
   switch (bw) {
     TQ_BW_CASE(2)
@@ -1011,9 +1031,9 @@ AttendFn attend_fn_dm(int bw, int b_theta, int G, bool gate, int* smem) {
 }  // namespace att
 
 // Per-(D, M) pickers, one per instantiation file.
-att::AttendFn attend_pick_64_64(int bw, int b_theta, int G, bool gate, int* smem);
-att::AttendFn attend_pick_64_128(int bw, int b_theta, int G, bool gate, int* smem);
-att::AttendFn attend_pick_128_64(int bw, int b_theta, int G, bool gate, int* smem);
-att::AttendFn attend_pick_128_128(int bw, int b_theta, int G, bool gate, int* smem);
+att::AttendFn attend_pick_64_64(int bw, int b_theta, int G, int mode, int* smem);
+att::AttendFn attend_pick_64_128(int bw, int b_theta, int G, int mode, int* smem);
+att::AttendFn attend_pick_128_64(int bw, int b_theta, int G, int mode, int* smem);
+att::AttendFn attend_pick_128_128(int bw, int b_theta, int G, int mode, int* smem);
 
 }  // namespace tq

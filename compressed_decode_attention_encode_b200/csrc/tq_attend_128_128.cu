@@ -4,8 +4,8 @@
 
 namespace tq {
 
-att::AttendFn attend_pick_128_128(int bw, int b_theta, int G, bool gate, int* smem) {
-  return att::attend_fn_dm<128, 128>(bw, b_theta, G, gate, smem);
+att::AttendFn attend_pick_128_128(int bw, int b_theta, int G, int mode, int* smem) {
+  return att::attend_fn_dm<128, 128>(bw, b_theta, G, mode, smem);
 }
 
 }  // namespace tq

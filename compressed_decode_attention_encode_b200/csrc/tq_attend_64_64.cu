@@ -4,8 +4,8 @@
 
 namespace tq {
 
-att::AttendFn attend_pick_64_64(int bw, int b_theta, int G, bool gate, int* smem) {
-  return att::attend_fn_dm<64, 64>(bw, b_theta, G, gate, smem);
+att::AttendFn attend_pick_64_64(int bw, int b_theta, int G, int mode, int* smem) {
+  return att::attend_fn_dm<64, 64>(bw, b_theta, G, mode, smem);
 }
 
 }  // namespace tq

@@ -303,31 +303,35 @@ __global__ void combine_kernel(const CombineArgs a) {
   const float res = mx == kNegInf ? 0.f
                                   : (oh + (float)a.signs[t] * x * rsqrtf((float)D)) / lsum;
   a.out[(size_t)hg * D + t] = res;
+  if (a.ml != nullptr && t == 0) {      // the softmax's normaliser, for promotion
+    a.ml[2 * (size_t)hg] = mx;
+    a.ml[2 * (size_t)hg + 1] = lsum;
+  }
 }
 
 // ---------------------------------------------------------------------------
 // dispatch
 // ---------------------------------------------------------------------------
-att::AttendFn pick_attend(const Layout& L, int G, bool gate, int* smem) {
-  if (L.d == 64 && L.m == 64) return attend_pick_64_64(L.bw, L.b_theta, G, gate, smem);
-  if (L.d == 64 && L.m == 128) return attend_pick_64_128(L.bw, L.b_theta, G, gate, smem);
-  if (L.d == 128 && L.m == 64) return attend_pick_128_64(L.bw, L.b_theta, G, gate, smem);
-  if (L.d == 128 && L.m == 128) return attend_pick_128_128(L.bw, L.b_theta, G, gate, smem);
+att::AttendFn pick_attend(const Layout& L, int G, int mode, int* smem) {
+  if (L.d == 64 && L.m == 64) return attend_pick_64_64(L.bw, L.b_theta, G, mode, smem);
+  if (L.d == 64 && L.m == 128) return attend_pick_64_128(L.bw, L.b_theta, G, mode, smem);
+  if (L.d == 128 && L.m == 64) return attend_pick_128_64(L.bw, L.b_theta, G, mode, smem);
+  if (L.d == 128 && L.m == 128) return attend_pick_128_128(L.bw, L.b_theta, G, mode, smem);
   return nullptr;
 }
 
 }  // namespace
 
 int attend_ctas_per_sm(const Layout& L, int G) {
-  int smem = 0;
-  att::AttendFn fn = pick_attend(L, G, false, &smem);
-  att::AttendFn fg = pick_attend(L, G, true, &smem);
-  if (!fn || !fg) return 0;
-  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
-      cudaFuncSetAttribute(fg, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-    return 0;
-  int n = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, att::kThreads, smem) != cudaSuccess) return 0;
+  int smem = 0, n = 0;
+  for (int mode = att::MODE_PLAIN; mode <= att::MODE_LOGITS; ++mode) {
+    att::AttendFn fn = pick_attend(L, G, mode, &smem);
+    if (!fn || cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return 0;
+    if (mode == att::MODE_PLAIN &&
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, att::kThreads, smem) != cudaSuccess)
+      return 0;
+  }
   return n;
 }
 
@@ -367,7 +371,8 @@ cudaError_t launch_qprep(const QPrepArgs& a, cudaStream_t s) {
 
 cudaError_t launch_attend(const AttendArgs& a, cudaStream_t s) {
   int smem = 0;
-  att::AttendFn fn = pick_attend(a.L, a.G, a.alist != nullptr, &smem);
+  const int mode = a.alist ? att::MODE_GATED : (a.logits ? att::MODE_LOGITS : att::MODE_PLAIN);
+  att::AttendFn fn = pick_attend(a.L, a.G, mode, &smem);
   if (!fn) return cudaErrorInvalidValue;
   const int grid = a.plan.cold_ctas > a.plan.hot_ctas ? a.plan.cold_ctas : a.plan.hot_ctas;
   if (grid == 0) return cudaSuccess;

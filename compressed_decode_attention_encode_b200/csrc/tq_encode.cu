@@ -233,7 +233,7 @@ __global__ void __launch_bounds__(2 * D) encode_small_kernel(EncodeArgs a) {
   constexpr int P = D / 2;
   constexpr int NW = D / 32;                 // warps per team
   const Layout& L = a.L;
-  const int64_t n = (int64_t)a.nA + a.nB;
+  const int64_t n = a.promo ? (int64_t)(kPromoMax + a.n_new) : (int64_t)a.nA + a.nB;
   const int unit = (int)(blockIdx.x / n);
   const int64_t e = blockIdx.x % n;
   const int tid = threadIdx.x, team = tid / D, el = tid % D;
@@ -255,18 +255,35 @@ __global__ void __launch_bounds__(2 * D) encode_small_kernel(EncodeArgs a) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
   const __half* src;
-  if (e < a.nA) {
+  int64_t dest = a.cold_start + e;           // cold position written
+  const __half* nsrc = nullptr;              // the slot's new occupant (write_new)
+  if (a.promo) {
+    // insert e of this unit: its promoted tokens first, then the new ones
+    const PromoUnitState* st = a.promo + unit;
+    const int k = st->n_pend;
+    if (e >= k + a.n_new) {                  // (the whole CTA) nothing to insert
+      async_copy_wait();
+      return;
+    }
+    const int slot = (int)((st->ring_pos + e) % a.W);
+    src = (team ? a.ring_v : a.ring_k) + ((int64_t)unit * a.W + slot) * D;
+    if (e < k) {
+      dest = st->pend_idx[e];
+      nsrc = (team ? a.promo_v : a.promo_k) + ((int64_t)unit * kPromoMax + e) * D;
+    } else {
+      dest = a.cold_start + (e - k);
+      nsrc = (team ? a.src_v : a.src_k) + ((int64_t)unit * a.src_tokens + (e - k)) * D;
+    }
+  } else if (e < a.nA) {
     const int slot = (int)((a.ring_start + e) % a.W);
     src = (team ? a.ring_v : a.ring_k) + ((int64_t)unit * a.W + slot) * D;
+    if (a.write_new) nsrc = (team ? a.src_v : a.src_k) + ((int64_t)unit * a.src_tokens + e) * D;
   } else {
     src = (team ? a.src_v : a.src_k) + ((int64_t)unit * a.src_tokens + (e - a.nA)) * D;
   }
   // ---- rotation: y = H (D x) / sqrt(d) ----------------------------------
   const __half xin = src[el];
-  if (a.write_new) {         // the slot just read now takes the new token (same thread, same element)
-    const __half* nsrc = (team ? a.src_v : a.src_k) + ((int64_t)unit * a.src_tokens + e) * D;
-    const_cast<__half*>(src)[el] = nsrc[el];
-  }
+  if (nsrc) const_cast<__half*>(src)[el] = nsrc[el];   // the slot just read takes its new occupant
   double x = __dmul_rn((double)__half2float(xin), a.signs[el]);
 #pragma unroll
   for (int h = 1; h < D; h <<= 1) {
@@ -362,7 +379,7 @@ __global__ void __launch_bounds__(2 * D) encode_small_kernel(EncodeArgs a) {
   __syncthreads();
 
   // ---- merge the token's fields into its tile ------------------------------
-  const int64_t tok = a.cold_start + e;
+  const int64_t tok = dest;
   const int64_t tile = tok / kTokensPerTile;
   const int r = (int)(tok % kTokensPerTile), gid = r % 8, h = r / 8;
   uint8_t* tb = a.cold + ((int64_t)unit * L.blocks_per_unit + tile / kTilesPerBlock) * L.block_bytes +
@@ -444,9 +461,9 @@ __global__ void ring_write_kernel(__half* ring_k, __half* ring_v, const __half* 
 template <int D>
 cudaError_t launch_encode_d(const EncodeArgs& a, cudaStream_t s) {
   const int warps = 8;
-  const int64_t n = (int64_t)a.nA + a.nB;
+  const int64_t n = a.promo ? (int64_t)(kPromoMax + a.n_new) : (int64_t)a.nA + a.nB;
   if (n == 0) return cudaSuccess;
-  if (D <= 128 && n <= kSmallEncodeTokens) {
+  if (D <= 128 && (n <= kSmallEncodeTokens || a.promo)) {
     const size_t smem = small_st_offset(D) + (size_t)D * a.L.m * sizeof(float);
     if (smem > 48 * 1024) {
       const cudaError_t e = cudaFuncSetAttribute(encode_small_kernel<D>,

@@ -122,6 +122,10 @@ struct tq_cache {
   cudaEvent_t ev_start;
   cudaEvent_t ev_stop;
   unsigned long long wait_limit_ns;   // attention kernel's bounded waits (tq_set_wait_limit)
+  // attention-weighted promotion (tq_promotion_enable), or null
+  uint8_t* promo;
+  float promo_threshold;
+  int promo_sticky;
   __half* hot_k() const { return (__half*)hot; }
   __half* hot_v() const {
     return (__half*)(hot + (size_t)cfg.batch * cfg.num_kv_heads * cfg.hot_window * cfg.head_dim * 2);
@@ -131,6 +135,51 @@ struct tq_cache {
   float* S() const { return (float*)(ws + W.S); }
   float* St() const { return (float*)(ws + W.St); }
 };
+
+// Promotion buffer: per-unit state | logits [units][capacity][G] fp32 |
+// per-head (max, sum) | dequantized promoted tokens [units][8][2][d] fp16.
+struct PromoLayout {
+  size_t state, logits, ml, staging, total;
+};
+
+static PromoLayout promo_layout(const tq_config& c) {
+  const size_t units = (size_t)c.batch * c.num_kv_heads;
+  const size_t G = (size_t)(c.num_q_heads / c.num_kv_heads);
+  PromoLayout p{};
+  size_t off = 0;
+  p.state = off;   off += round_up(sizeof(PromoUnitState) * units, kAlign);
+  p.logits = off;  off += round_up(sizeof(float) * units * (size_t)c.cold_capacity * G, kAlign);
+  p.ml = off;      off += round_up(sizeof(float) * 2 * (size_t)c.batch * c.num_q_heads, kAlign);
+  p.staging = off; off += round_up(2 * units * kPromoMax * 2 * (size_t)c.head_dim, kAlign);
+  p.total = off;
+  return p;
+}
+
+static PromoArgs promo_args(const tq_cache* c) {
+  const tq_config& cf = c->cfg;
+  const PromoLayout pl = promo_layout(cf);
+  const size_t units = (size_t)cf.batch * cf.num_kv_heads;
+  PromoArgs a{};
+  a.logits = (const float*)(c->promo + pl.logits);
+  a.ml = (const float*)(c->promo + pl.ml);
+  a.state = (PromoUnitState*)(c->promo + pl.state);
+  a.cold = c->cold;
+  a.promo_k = (__half*)(c->promo + pl.staging);
+  a.promo_v = a.promo_k + units * kPromoMax * cf.head_dim;
+  a.signs = c->signs();
+  a.inv_sqrt_d = 1.0 / std::sqrt((double)cf.head_dim);
+  a.L = c->L;
+  a.units = (int)units;
+  a.G = cf.num_q_heads / cf.num_kv_heads;
+  a.Hq = cf.num_q_heads;
+  a.Hkv = cf.num_kv_heads;
+  a.n_cold = c->n_cold;
+  a.capacity = cf.cold_capacity;
+  a.threshold = c->promo_threshold;
+  a.sticky = c->promo_sticky;
+  a.ring_full = c->n_hot == cf.hot_window;
+  return a;
+}
 
 extern "C" {
 
@@ -185,6 +234,7 @@ tq_status tq_cache_create(const tq_config* cfg, void* hot_mem, void* cold_mem,
   c->dirty_n = 0;
   c->tc = c->tc_lam = c->tc_eta = c->tc_sig = nullptr;
   c->wait_limit_ns = kDefaultWaitLimitNs;
+  c->promo = nullptr;
   if (cudaGetDevice(&c->device) != cudaSuccess ||
       cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, c->device) != cudaSuccess) {
     delete c;
@@ -299,6 +349,32 @@ tq_status tq_evict_window(tq_cache* c, const void* k_new, const void* v_new, int
     return TQ_OK;
   }
   if (c->n_cold + E > c->cfg.cold_capacity) return TQ_ERR_CAPACITY;
+  if (c->promo && c->n_hot == W) {
+    // Promotion enabled and the window full: unit u inserts its pending
+    // promoted tokens, then the n new ones, at its own ring position; the
+    // first evictions take the promoted tokens' cold positions, the last n
+    // are appended (so every unit's cold count grows by n).
+    if (n > W - kPromoMax) return TQ_ERR_INVALID_ARG;
+    PromoArgs pa = promo_args(c);
+    if (launch_promo_dequant(pa, stream) != cudaSuccess) return TQ_ERR_CUDA;
+    EncodeArgs a = base_encode_args(c);
+    a.ring_k = c->hot_k();
+    a.ring_v = c->hot_v();
+    a.src_k = (const __half*)k_new;
+    a.src_v = (const __half*)v_new;
+    a.src_tokens = n;
+    a.promo = pa.state;
+    a.promo_k = pa.promo_k;
+    a.promo_v = pa.promo_v;
+    a.n_new = n;
+    if (launch_encode(a, stream) != cudaSuccess) return TQ_ERR_CUDA;
+    if (launch_promo_ring(pa.state, pa.units, W, n, -1, stream) != cudaSuccess) return TQ_ERR_CUDA;
+    c->n_cold += n;
+    c->dirty_lo = 0;
+    c->dirty_n = W;
+    c->ring_pos = (int32_t)(((int64_t)c->ring_pos + n) % W);
+    return TQ_OK;
+  }
   // Steady state (a full window, a few new tokens): each new token evicts
   // the token in the slot it takes, and one launch does both.
   const bool fused = E == n && c->n_hot == W && n <= W && n <= kSmallEncodeTokens;
@@ -327,6 +403,10 @@ tq_status tq_evict_window(tq_cache* c, const void* k_new, const void* v_new, int
   c->dirty_lo = (int32_t)(((int64_t)c->ring_pos + std::max(0, n - W)) % W);
   c->dirty_n = std::min(n, W);
   c->ring_pos = (int32_t)(((int64_t)c->ring_pos + n) % W);
+  if (c->promo &&   // until the window is full every unit shares the host's ring position
+      launch_promo_ring((PromoUnitState*)(c->promo + promo_layout(c->cfg).state),
+                        c->cfg.batch * c->cfg.num_kv_heads, W, 0, c->ring_pos, stream) != cudaSuccess)
+    return TQ_ERR_CUDA;
   return TQ_OK;
 }
 
@@ -456,6 +536,13 @@ static tq_status launch_decode(tq_cache* c, const void* q, float* out, float sof
     a.alist = gate->alist;
     a.n_active = gate->n_active;
   }
+  const bool promo = c->promo != nullptr && gate == nullptr;
+  PromoArgs pa{};
+  if (promo) {
+    pa = promo_args(c);
+    a.logits = const_cast<float*>(pa.logits);
+    a.logit_capacity = cf.cold_capacity;
+  }
   if (c->ev_start && cudaEventRecord(c->ev_start, stream) != cudaSuccess) return TQ_ERR_CUDA;
   if (launch_attend(a, stream) != cudaSuccess) return TQ_ERR_CUDA;
   if (c->ev_stop && cudaEventRecord(c->ev_stop, stream) != cudaSuccess) return TQ_ERR_CUDA;
@@ -476,7 +563,9 @@ static tq_status launch_decode(tq_cache* c, const void* q, float* out, float sof
     ca.unit_pos = gate->unit_pos;
     ca.n_active = gate->n_active;
   }
+  if (promo) ca.ml = const_cast<float*>(pa.ml);
   if (launch_combine(ca, stream) != cudaSuccess) return TQ_ERR_CUDA;
+  if (promo && pl.cold_ctas > 0 && launch_promo_mass(pa, stream) != cudaSuccess) return TQ_ERR_CUDA;
   if (c->tc) {
     TcReadArgs tr{};
     tr.A = c->tc;
@@ -508,6 +597,7 @@ tq_status tq_decode_attention_gated(tq_cache* c, const void* q, float* out, floa
   if (!c || !q || !out || !(softmax_scale >= 0.0f) || std::isinf(softmax_scale) ||
       std::isnan(threshold) || (uintptr_t)q % 16)
     return TQ_ERR_INVALID_ARG;
+  if (c->promo) return TQ_ERR_UNSUPPORTED;      // promotion counts the ungated decode's masses
   const tq_config& cf = c->cfg;
   const int units = cf.batch * cf.num_kv_heads;
   const int heads = cf.batch * cf.num_q_heads;
@@ -544,7 +634,7 @@ tq_status tq_tc_bytes(const tq_config* cfg, size_t* bytes) {
 tq_status tq_tc_enable(tq_cache* c, void* tc_mem, const float* lambda, const float* eta,
                        const float* gate, cudaStream_t stream) {
   if (!c || !tc_mem || !lambda || !eta || !gate || (uintptr_t)tc_mem % kAlign) return TQ_ERR_INVALID_ARG;
-  if (c->tc) return TQ_ERR_INVALID_ARG;                     // already enabled
+  if (c->tc || c->promo) return TQ_ERR_INVALID_ARG;         // already enabled, or promotion on
   const tq_config& cf = c->cfg;
   const int hkv = cf.num_kv_heads, hq = cf.num_q_heads;
   std::vector<float> par(2 * hkv + hq);
@@ -569,6 +659,66 @@ tq_status tq_tc_enable(tq_cache* c, void* tc_mem, const float* lambda, const flo
   c->tc_lam = p;
   c->tc_eta = p + hkv;
   c->tc_sig = p + 2 * hkv;
+  return TQ_OK;
+}
+
+tq_status tq_promotion_bytes(const tq_config* cfg, size_t* bytes) {
+  if (!cfg || !bytes) return TQ_ERR_INVALID_ARG;
+  const tq_status st = check_config(cfg);
+  if (st != TQ_OK) return st;
+  *bytes = promo_layout(*cfg).total;
+  return TQ_OK;
+}
+
+tq_status tq_promotion_enable(tq_cache* c, void* mem, float threshold, int32_t sticky,
+                              cudaStream_t stream) {
+  if (!c || !mem || (uintptr_t)mem % kAlign || !(threshold >= 0.125f && threshold <= 1.0f) ||
+      sticky < 1 || c->cfg.hot_window <= kPromoMax)
+    return TQ_ERR_INVALID_ARG;
+  if (c->tc || c->promo) return TQ_ERR_INVALID_ARG;        // Tensor Cache tier, or already on
+  const size_t units = (size_t)c->cfg.batch * c->cfg.num_kv_heads;
+  std::vector<PromoUnitState> st(units);
+  for (auto& u : st) {
+    for (int i = 0; i < kPromoMax; ++i) {
+      u.cnt_idx[i] = -1;
+      u.cnt_val[i] = 0;
+      u.pend_idx[i] = -1;
+    }
+    u.n_cnt = u.n_pend = 0;
+    u.ring_pos = c->ring_pos;
+    for (int& x : u.pad) x = 0;
+  }
+  cudaError_t e = cudaMemcpyAsync(mem, st.data(), sizeof(PromoUnitState) * units, cudaMemcpyHostToDevice,
+                                  stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);   // `st` is released on return
+  if (e != cudaSuccess) return TQ_ERR_CUDA;
+  c->promo = (uint8_t*)mem;
+  c->promo_threshold = threshold;
+  c->promo_sticky = sticky;
+  return TQ_OK;
+}
+
+tq_status tq_promotion_state(tq_cache* c, int32_t* out, cudaStream_t stream) {
+  if (!c || !out) return TQ_ERR_INVALID_ARG;
+  if (!c->promo) return TQ_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return TQ_ERR_CUDA;
+  const size_t units = (size_t)c->cfg.batch * c->cfg.num_kv_heads;
+  std::vector<PromoUnitState> st(units);
+  if (cudaMemcpy(st.data(), c->promo + promo_layout(c->cfg).state, sizeof(PromoUnitState) * units,
+                 cudaMemcpyDeviceToHost) != cudaSuccess)
+    return TQ_ERR_CUDA;
+  for (size_t u = 0; u < units; ++u) {
+    int32_t* o = out + u * 28;
+    o[0] = st[u].n_cnt;
+    o[1] = st[u].n_pend;
+    o[2] = st[u].ring_pos;
+    o[3] = 0;
+    for (int i = 0; i < kPromoMax; ++i) {
+      o[4 + i] = st[u].cnt_idx[i];
+      o[12 + i] = st[u].cnt_val[i];
+      o[20 + i] = st[u].pend_idx[i];
+    }
+  }
   return TQ_OK;
 }
 

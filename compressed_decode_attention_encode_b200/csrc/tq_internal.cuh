@@ -104,6 +104,23 @@ __host__ __device__ inline Layout layout_of(int d, int b_r, int b_theta, int m, 
 }
 
 
+// ---- attention-weighted promotion ---------------------------------------
+// At most this many tokens per (row, kv head) are counted or promoted per
+// decode step: with a threshold >= 1/8 no more can reach it, because a
+// unit's cold masses sum to at most 1.
+constexpr int kPromoMax = 8;
+
+// Per-(row, kv head) state in the caller's promotion buffer (128 bytes).
+struct PromoUnitState {
+  int cnt_idx[kPromoMax];   // cold positions with a running count (ascending), -1 unused
+  int cnt_val[kPromoMax];
+  int n_cnt;
+  int pend_idx[kPromoMax];  // promoted by the last decode, not yet in the ring (ascending)
+  int n_pend;
+  int ring_pos;             // next ring slot of this unit
+  int pad[5];
+};
+
 // ---- encode -------------------------------------------------------------
 // Encodes a sequence of E vectors per unit (unit = row * Hkv + kv head), K
 // and V in one launch: the first nA come from ring slots (ring_start + e)
@@ -131,6 +148,15 @@ struct EncodeArgs {
   // (ring_start + e) mod W, token e's CTA writes src_k/src_v token e into
   // that same slot, so the ring write needs no launch of its own.
   int write_new;
+  // Eviction with promotion (per-token path; null otherwise): unit u
+  // inserts its n_pend promoted tokens (promo_k/v) and then n_new new ones
+  // (src) at its own ring position; insert e evicts ring slot (ring_pos +
+  // e) mod W into cold position pend_idx[e] (e < n_pend) or cold_start +
+  // e - n_pend, and takes that slot.
+  const PromoUnitState* promo;
+  const __half* promo_k;
+  const __half* promo_v;
+  int n_new;
 };
 
 // Global -> shared copy of `bytes` (a multiple of 16, both addresses 16-byte
@@ -264,6 +290,10 @@ struct AttendArgs {
   int W, n_hot;
   int64_t n_cold;
   float log2e_sigma;        // log2(e) * softmax scale
+  // When non-null (promotion enabled): every valid cold token's log2-domain
+  // logit of every query head, [units][logit_capacity][G].
+  float* logits;
+  int64_t logit_capacity;
   // Limit of each bounded wait for a cold tile's bulk copy; 0 makes every
   // such wait give up at once (a forced timeout).  The copies already issued
   // are then drained under kDefaultWaitLimitNs before the CTA exits.
@@ -279,6 +309,7 @@ int attend_ctas_per_sm(const Layout& L, int G);
 
 struct CombineArgs {
   const float* part;
+  float* ml;                // null, or [B*Hq][2]: each head's final max (log2) and sum
   const int* status;        // device status word: NaN output while kStatusNoPartials is latched
   const double* signs;
   float* out;               // [B*Hq, d]
@@ -313,6 +344,29 @@ struct GateArgs {
 };
 
 cudaError_t launch_gate(const GateArgs& a, cudaStream_t s);
+
+// ---- promotion kernels --------------------------------------------------
+struct PromoArgs {
+  const float* logits;      // [units][capacity][G] log2-domain logits of the last decode
+  const float* ml;          // [B*Hq][2] each head's final max (log2) and sum
+  PromoUnitState* state;    // [units]
+  const uint8_t* cold;
+  __half* promo_k;          // [units][kPromoMax][d] dequantized promoted tokens
+  __half* promo_v;
+  const double* signs;
+  double inv_sqrt_d;
+  Layout L;
+  int units, G, Hq, Hkv;
+  int64_t n_cold, capacity;
+  float threshold;
+  int sticky;
+  int ring_full;            // promotions are kept only while the hot window is full
+};
+
+cudaError_t launch_promo_mass(const PromoArgs& a, cudaStream_t s);
+cudaError_t launch_promo_dequant(const PromoArgs& a, cudaStream_t s);
+cudaError_t launch_promo_ring(PromoUnitState* state, int units, int W, int n_new, int set_to,
+                              cudaStream_t s);
 
 // ---- Tensor Cache second tier -----------------------------------------
 // Per unit a d x d float32 matrix A; per kv head lambda, eta; per query

@@ -65,6 +65,9 @@ SIGNATURES = [
     ("tq_get_status", c_int32, [c_void_p, c_void_p]),
     ("tq_set_attend_events", c_int32, [c_void_p, c_void_p, c_void_p]),
     ("tq_set_wait_limit", c_int32, [c_void_p, c_int64]),
+    ("tq_promotion_bytes", c_int32, [POINTER(tq_config), POINTER(c_size_t)]),
+    ("tq_promotion_enable", c_int32, [c_void_p, c_void_p, c_float, c_int32, c_void_p]),
+    ("tq_promotion_state", c_int32, [c_void_p, c_void_p, c_void_p]),
     ("tq_export_cold", c_int32, [c_void_p, c_int32, c_int32, c_int64, c_int64, c_void_p,
                                  c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
     ("tq_vec_bytes", c_int32, [POINTER(tq_vec_config), c_int64, c_int32, POINTER(c_size_t),
@@ -192,6 +195,16 @@ def tq_set_attend_events(handle: int, start: int, stop: int) -> None:
     _check(lib().tq_set_attend_events(handle, start, stop), "tq_set_attend_events")
 
 
+def tq_promotion_bytes(cfg: tq_config) -> int:
+    n = c_size_t()
+    _check(lib().tq_promotion_bytes(ctypes.byref(cfg), ctypes.byref(n)), "tq_promotion_bytes")
+    return n.value
+
+
+def tq_promotion_enable(handle: int, mem_ptr: int, threshold: float, sticky: int, stream: int) -> None:
+    _check(lib().tq_promotion_enable(handle, mem_ptr, threshold, sticky, stream), "tq_promotion_enable")
+
+
 def tq_set_wait_limit(handle: int, limit_ns: int) -> None:
     _check(lib().tq_set_wait_limit(handle, limit_ns), "tq_set_wait_limit")
 
@@ -315,6 +328,28 @@ class TQCache:
         decode calls (None, None stops recording)."""
         tq_set_attend_events(self.handle, start.cuda_event if start is not None else None,
                              stop.cuda_event if stop is not None else None)
+
+    def enable_promotion(self, threshold=0.15, sticky=3, stream=None):
+        """Attention-weighted promotion (sticky counters) on this handle;
+        the library's buffer comes from PyTorch."""
+        import torch
+        self.promo_mem = torch.empty(tq_promotion_bytes(self.cfg), dtype=torch.uint8, device=self.device)
+        tq_promotion_enable(self.handle, _ptr(self.promo_mem), float(threshold), int(sticky),
+                            _stream_handle(stream))
+
+    def promotion_state(self, stream=None):
+        """Per (row, kv head): dict of counted positions -> counts, the
+        promoted positions not yet moved, and the ring position."""
+        units = self.cfg.batch * self.cfg.num_kv_heads
+        out = np.zeros((units, 28), dtype=np.int32)
+        _check(lib().tq_promotion_state(self.handle, out.ctypes.data, _stream_handle(stream)),
+               "tq_promotion_state")
+        res = []
+        for u in range(units):
+            o = out[u]
+            res.append(dict(counts={int(o[4 + i]): int(o[12 + i]) for i in range(o[0])},
+                            pending=[int(x) for x in o[20:20 + o[1]]], ring_pos=int(o[2])))
+        return res
 
     def set_wait_limit(self, limit_ns: int):
         """Bounded-wait limit of the attention kernel (ns; 0 forces a

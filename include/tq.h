@@ -252,6 +252,48 @@ tq_status tq_tc_enable(tq_cache* cache, void* tc_mem, const float* lambda, const
                        const float* gate, cudaStream_t stream);
 
 /*
+ * Attention-weighted promotion with sticky counters ("Monarch v3 ...",
+ * section "Cómo funciona", item "Promoción Ponderada por Atención": cold
+ * tokens that draw much attention return to the full-precision hot region,
+ * with a persistence count against thrashing; the page's benchmark uses a
+ * threshold of 0.15 and a sticky count of 3).  Once enabled on a handle:
+ *   - every tq_decode_attention (and _static) call also finds, per (row, kv
+ *     head), the cold tokens whose mass -- the mean over the kv head's query
+ *     heads of the token's softmax weight in that call -- is >= threshold.
+ *     A token's count rises by one at each call where it is such a hit and
+ *     returns to 0 at any call where it is not; at `sticky` it is promoted
+ *     and its count cleared.  Promotions are dropped while the hot window
+ *     is not yet full.
+ *   - the next tq_evict_window inserts, per (row, kv head), its promoted
+ *     tokens first -- their K and V dequantized to fp16, R^T (s16/(2^b_r-1)
+ *     c_r (cos, sin)), in ascending cold position -- and then the n new
+ *     tokens.  Every insert evicts the ring's oldest token: the first ones
+ *     take the promoted tokens' cold positions, the last n are appended, so
+ *     every (row, kv head) keeps the same cold count.  Ring positions then
+ *     differ per (row, kv head); decode attention is order-free in the ring.
+ * tq_promotion_bytes: size of the caller's buffer (per-unit state, every
+ *   cold token's logits [B*Hkv, cold_capacity, G] as float32, the heads'
+ *   softmax normalisers, the promoted tokens' fp16 staging).
+ * tq_promotion_enable: binds that buffer (256-byte aligned, kept until
+ *   tq_cache_destroy), synchronizes `stream`.  TQ_ERR_INVALID_ARG for a NULL
+ *   or misaligned buffer, a threshold outside [1/8, 1] (at most 8 tokens per
+ *   (row, kv head) can then be hits, since their masses sum to at most 1),
+ *   sticky < 1, a hot window of 8 tokens or fewer, a handle with the Tensor
+ *   Cache tier, or promotion already on.  Afterwards tq_evict_window returns
+ *   TQ_ERR_INVALID_ARG for n > hot_window - 8 once the window is full, and
+ *   tq_decode_attention_gated returns TQ_ERR_UNSUPPORTED.
+ * tq_promotion_state: copies the per-(row, kv head) state to a HOST array
+ *   out[B*Hkv][28] (synchronizes `stream`): [0] tokens with a running count,
+ *   [1] tokens promoted by the last decode and not yet moved, [2] the ring
+ *   position, [3] 0, [4..11] the counted cold positions (ascending, -1 when
+ *   unused), [12..19] their counts, [20..27] the promoted cold positions.
+ */
+tq_status tq_promotion_bytes(const tq_config* cfg, size_t* bytes);
+tq_status tq_promotion_enable(tq_cache* cache, void* mem, float threshold, int32_t sticky,
+                              cudaStream_t stream);
+tq_status tq_promotion_state(tq_cache* cache, int32_t* out, cudaStream_t stream);
+
+/*
  * Synchronize `stream`, then return and clear the latched device status
  * (TQ_OK, TQ_ERR_RANGE or TQ_ERR_TIMEOUT; TQ_ERR_UNSUPPORTED when the
  * attention kernel found its dynamic shared memory at a window address its
