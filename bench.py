@@ -47,6 +47,8 @@ def parse():
     ap.add_argument("--tensor-cache", action="store_true",
                     help="decode with the Tensor Cache tier: evicted tokens go to an outer-product "
                          "memory instead of the compressed cold store")
+    ap.add_argument("--promotion", action="store_true",
+                    help="decode with attention-weighted promotion (threshold 0.15, sticky 3)")
     ap.add_argument("--encode", action="store_true",
                     help="time the prefill encode (tq_encode_append of 4096-token chunks) instead")
     return ap.parse_args()
@@ -293,6 +295,8 @@ def run_gpu(args, wl):
         k = gen_kv(wl, layer, args.seed, 0, wl.batch, 0, wl.hot, dev, gen)
         v = gen_kv(wl, layer, args.seed, 1, wl.batch, 0, wl.hot, dev, gen)
         c.evict_window(k, v)
+        if args.promotion:         # the page's benchmark setting
+            c.enable_promotion(0.15, 3)
         if c.get_status() != 0:
             raise RuntimeError("device status after prefill")
         caches.append(c)
@@ -352,6 +356,8 @@ def run_gpu(args, wl):
             else:
                 keys += units * (nc + nh)
                 abytes += units * (nc * cold_tok_bytes + nh * hot_tok_bytes)
+                if args.promotion:      # the attention kernel also writes every cold logit
+                    abytes += units * nc * wl.group * 4
             if ev_pairs is not None:
                 caches[l].set_attend_events(*ev_pairs[l])
             attend(l, qs[l], outs[l])
@@ -398,6 +404,8 @@ def run_gpu(args, wl):
     ms = max_over_ranks(ms, dev)
     # evict: per-token encode (ring write fused); decode: qprep, [gate,] attend, combine
     launches_per_step = L * (1 + 3 + (gate_tau is not None))
+    if args.promotion:   # evict: dequant, encode, ring positions; decode: + the mass kernel
+        launches_per_step = L * (3 + 4)
 
     # ---- e2e: host buffers through the public API ------------------------
     # Each step's inputs (every layer's new K, V token and queries) travel in
@@ -506,6 +514,18 @@ def run_gpu(args, wl):
                                    "bytes_per_launch": read / L,
                                    "bytes_note": "cold bytes of the units the last step read"})
         result["hbm"] = None
+    if args.promotion:
+        st = [caches[l].promotion_state() for l in range(L)]
+        result["metric"] = ("decode with attention-weighted promotion: context keys/s "
+                            "(threshold 0.15, sticky count 3)")
+        result["config"]["promotion"] = {"threshold": 0.15, "sticky": 3}
+        result["promotion"] = {
+            "counted_tokens_last_step": sum(len(u["counts"]) for x in st for u in x),
+            "pending_promotions_last_step": sum(len(u["pending"]) for x in st for u in x),
+        }
+        result["roofline"]["traffic"] = None
+        result["roofline"]["bytes_note"] = ("cold and hot bytes plus the cold tokens' logits "
+                                            "the attention kernel writes (4 B per token and head)")
     if args.tensor_cache:
         step_gbs = bytes_total / (ms / 1e3) / 1e9
         result["metric"] = ("Tensor Cache decode: context tokens/s (softmax over the ring + "
@@ -520,7 +540,7 @@ def run_gpu(args, wl):
         result["hbm"] = None
         result["gpu_launches"] = L * (2 + 2 + 1) * args.steps   # no q-prep without cold tokens
     if rank == 0 and world == 1 and not args.no_cpu_baseline and gate_tau is None and \
-            not args.tensor_cache:
+            not args.tensor_cache and not args.promotion:
         sample = oracle_sample(wl, args.seed, kv_heads=1)
         time_oracle(sample)
         tt, kk = 0.0, 0

@@ -460,14 +460,17 @@ __device__ __forceinline__ void flush_partial(WarpState<NT, HPL>& st, bool hot, 
 // The kernel.  SLOT selects the int8 polar path (b_theta <= 3); HMAP the
 // heads a lane holds on the cold path (HMAP_PACK for groups of up to 4;
 // HMAP_SPLIT for larger SLOT groups, HMAP_PAIR for larger HILO groups);
-// MODE: plain, gated (the cold tier of listed units only) or with every
-// cold token's logits written out (promotion).
+// MODE: plain, gated (the cold tier of listed units only), with every
+// cold token's logits written out (promotion), or ragged (per-row counts
+// from a RowTable: the units' blocks and tiles are flattened by prefix
+// sums, so rows of any length share the CTAs evenly).
 // ---------------------------------------------------------------------------
-enum { MODE_PLAIN = 0, MODE_GATED = 1, MODE_LOGITS = 2 };
+enum { MODE_PLAIN = 0, MODE_GATED = 1, MODE_LOGITS = 2, MODE_RAGGED = 3 };
 
 template <int D, int M, int BW, bool SLOT, int HMAP, int MODE>
 __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(const AttendArgs a) {
   constexpr bool GATE = MODE == MODE_GATED;
+  constexpr bool RAGGED = MODE == MODE_RAGGED;
   using S = AttendShape<D, M, BW>;
   constexpr int HPL = HMAP == HMAP_PACK ? 1 : 2;     // query heads per lane on the cold path
   constexpr int NQ = SLOT ? HPL : 1;                 // int8 MMAs per k-step (column groups)
@@ -520,28 +523,65 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
   };
   if (c < (GATE ? g_ctas : pl.cold_ctas)) {
     // ============ cold run: blocks [c * bpc, (c + 1) * bpc) ============
-    const int64_t nb = pl.cold_blocks;
-    const int64_t total = cold_units() * nb;
+    // Positions of the run: units (gated: active-list positions), each with
+    // pos_blocks(p) blocks starting at flattened block pos_off(p); ragged
+    // runs skip the units of rows without cold tokens.
+    const int n_rows = a.units / a.Hkv;
+    auto row_blocks = [&](int b) -> int { return (a.rows->n_cold[b] + S::TB - 1) / S::TB; };
+    auto pos_blocks = [&](int p) -> int {
+      if constexpr (RAGGED) return row_blocks(p / a.Hkv); else return (int)pl.cold_blocks;
+    };
+    auto pos_off = [&](int p) -> int64_t {
+      if constexpr (RAGGED) {
+        const int b = p / a.Hkv;
+        return a.rows->cold_pre[b] + (int64_t)(p % a.Hkv) * row_blocks(b);
+      } else {
+        return (int64_t)p * pl.cold_blocks;
+      }
+    };
+    auto pos_tail = [&](int p) -> int {     // valid tokens of the position's last block
+      if constexpr (RAGGED) return a.rows->n_cold[p / a.Hkv] - (pos_blocks(p) - 1) * S::TB;
+      else return (int)(a.n_cold - (pl.cold_blocks - 1) * S::TB);
+    };
+    auto pos_next = [&](int p) -> int {
+      if constexpr (RAGGED) {
+        if ((p + 1) % a.Hkv != 0) return p + 1;
+        int b = (p + 1) / a.Hkv;
+        while (b < n_rows && a.rows->n_cold[b] == 0) ++b;
+        return b * a.Hkv;
+      } else {
+        return p + 1;
+      }
+    };
+    // (gated: alist[n_active] exists, so the run's last step may look one past)
+    auto pos_uid = [&](int p) -> int { if constexpr (GATE) return a.alist[p]; else return p; };
+    const int64_t total = RAGGED ? (int64_t)a.rows->cold_pre[n_rows] : cold_units() * pl.cold_blocks;
     const int64_t f_lo = (int64_t)c * cold_bpc();
     const int64_t f_hi = f_lo + cold_bpc() < total ? f_lo + cold_bpc() : total;
     const int nblk = (int)(f_hi - f_lo);
-    const int nbi = (int)nb;
+    int p_first, blk_first;
+    if constexpr (RAGGED) {      // the row holding block f_lo: the last b with cold_pre[b] <= f_lo
+      int lo = 0, hi = n_rows - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (a.rows->cold_pre[mid] <= f_lo) lo = mid; else hi = mid - 1;
+      }
+      const int nbr = row_blocks(lo);
+      const int64_t off = f_lo - a.rows->cold_pre[lo];
+      p_first = lo * a.Hkv + (int)(off / nbr);
+      blk_first = (int)(off % nbr);
+    } else {
+      p_first = (int)(f_lo / pl.cold_blocks);
+      blk_first = (int)(f_lo - (int64_t)p_first * pl.cold_blocks);
+    }
     const uint32_t bar_w = smem_addr(bars) + 8 * S::NS * warp;           // this warp's barriers
     const uint32_t ring_w = smem_addr(ring) + S::NS * S::TT * warp;      // this warp's stages
     // The warp's tile stream: `nsrc` is the next tile to fetch (block
-    // `nblk_b` of its unit); it advances a block at a time and skips a
-    // unit's unused blocks at the unit's end.  `issued` counts the copies.
-    const uint8_t* nsrc;
-    int nblk_b = 0, issued = 0;
-    int fpos = 0;                        // gated: active-list position of nsrc's unit
-    const size_t unit_gap = (size_t)(a.L.blocks_per_unit - nb) * S::BLOCK;
-    {
-      const int64_t u = f_lo / nb;
-      nblk_b = (int)(f_lo - u * nb);
-      fpos = (int)u;
-      const int64_t uid = GATE ? (int64_t)a.alist[u] : u;
-      nsrc = a.cold + ((size_t)uid * a.L.blocks_per_unit + (size_t)nblk_b) * S::BLOCK + warp * S::TT;
-    }
+    // `nblk_b` of position `fpos`, which has `fnb` blocks); at a position's
+    // end it moves to block 0 of the next one.  `issued` counts the copies.
+    int fpos = p_first, nblk_b = blk_first, fnb = pos_blocks(p_first), issued = 0;
+    const uint8_t* nsrc =
+        a.cold + ((size_t)pos_uid(fpos) * a.L.blocks_per_unit + (size_t)nblk_b) * S::BLOCK + warp * S::TT;
     // The next tile into stage s: every lane advances the (warp-uniform)
     // stream; lane 0 alone arms the barrier and issues the copy, predicated
     // rather than branched around.  `after_reads` orders the warp's reads of
@@ -558,12 +598,12 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
           : "memory");
       ++issued;
       nsrc += S::BLOCK;
-      if (++nblk_b == nbi) {
+      if (++nblk_b == fnb) {
         nblk_b = 0;
-        if constexpr (GATE)   // alist[n_active] exists (and is 0) for the run's last step
-          nsrc = a.cold + (size_t)a.alist[++fpos] * a.L.blocks_per_unit * S::BLOCK + warp * S::TT;
-        else
-          nsrc += unit_gap;
+        fpos = pos_next(fpos);
+        if (RAGGED && fpos >= a.units) return;    // the run's last block has been issued
+        fnb = pos_blocks(fpos);
+        nsrc = a.cold + (size_t)pos_uid(fpos) * a.L.blocks_per_unit * S::BLOCK + warp * S::TT;
       }
     };
     if (tid == 0) *abort_flag = 0;
@@ -624,7 +664,7 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
 
     // Loads the B operands and logit constants of unit position `u`.
     auto setup_unit = [&](int u) {
-      const int uid = GATE ? a.alist[u] : u;
+      const int uid = pos_uid(u);
       const int b = uid / a.Hkv, kvh = uid % a.Hkv;
       const int head0 = b * a.Hq + kvh * G;
 #pragma unroll
@@ -845,19 +885,18 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
       if (!aborted && i + S::NS < nblk) fetch_next(stage, true);
     };
 
-    // The run as segments of one unit each: the blocks before a unit's last
-    // one are full; its last block holds `tail` tokens.
-    const int tail = (int)(a.n_cold - (int64_t)(nbi - 1) * S::TB);   // valid tokens of a unit's last block
+    // The run as segments of one position each: the blocks before a unit's
+    // last one are full; its last block holds pos_tail(p) tokens.
     const std::integral_constant<bool, false> full_tile{};
     const std::integral_constant<bool, true> masked_tile{};
-    int unit = (int)(f_lo / nb);
-    int blk = (int)(f_lo - (int64_t)unit * nb);   // block inside the unit (< 2^31)
+    int pos = p_first, blk = blk_first;
     int i = 0;
     while (i < nblk) {
-      const int uid = setup_unit(unit);
-      const int slot = c - (int)(((int64_t)unit * nb) / cold_bpc());
-      const int seg = (nbi - blk) < (nblk - i) ? (nbi - blk) : (nblk - i);   // this unit's blocks in the run
-      const bool ends_unit = blk + seg == nbi;
+      const int uid = setup_unit(pos);
+      const int nbp = pos_blocks(pos), tail = pos_tail(pos);
+      const int slot = c - (int)(pos_off(pos) / cold_bpc());
+      const int seg = (nbp - blk) < (nblk - i) ? (nbp - blk) : (nblk - i);   // this unit's blocks in the run
+      const bool ends_unit = blk + seg == nbp;
       const int n_full = (ends_unit && tail < S::TB) ? seg - 1 : seg;
       const int i_end = i + seg, i_full = i + n_full;
       const int64_t tok_first = (int64_t)(blk - i) * S::TB + tb;   // + 64 i: this warp's first token
@@ -870,7 +909,7 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
       flush_partial<D, S::NT, HPL, HMAP>(st, false, inv_levels, G, merge,
                                          a.part + (((size_t)uid * slots + slot) * G) * (D + 2));
       st.reset();
-      ++unit;
+      pos = pos_next(pos);
       blk = 0;
     }
     __syncthreads();
@@ -888,8 +927,35 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
   }
   if (c < pl.hot_ctas) {
     // ====== then hot tiles [c * tpc, (c + 1) * tpc): the ring is idle ======
-    const int ht = pl.hot_tiles;
-    const int64_t total = (int64_t)a.units * ht;
+    // units with uniform hot counts, or (ragged) per-row counts with the
+    // units' tiles flattened by prefix sums, skipping rows without hot tokens
+    const int n_rows = a.units / a.Hkv;
+    auto row_tiles = [&](int b) -> int { return (a.rows->n_hot[b] + S::TB - 1) / S::TB; };
+    auto unit_tiles = [&](int u) -> int {
+      if constexpr (RAGGED) return row_tiles(u / a.Hkv); else return pl.hot_tiles;
+    };
+    auto unit_hoff = [&](int u) -> int64_t {
+      if constexpr (RAGGED) {
+        const int b = u / a.Hkv;
+        return a.rows->hot_pre[b] + (int64_t)(u % a.Hkv) * row_tiles(b);
+      } else {
+        return (int64_t)u * pl.hot_tiles;
+      }
+    };
+    auto unit_nhot = [&](int u) -> int {
+      if constexpr (RAGGED) return a.rows->n_hot[u / a.Hkv]; else return a.n_hot;
+    };
+    auto unit_next = [&](int u) -> int {
+      if constexpr (RAGGED) {
+        if ((u + 1) % a.Hkv != 0) return u + 1;
+        int b = (u + 1) / a.Hkv;
+        while (b < n_rows && a.rows->n_hot[b] == 0) ++b;
+        return b * a.Hkv;
+      } else {
+        return u + 1;
+      }
+    };
+    const int64_t total = RAGGED ? (int64_t)a.rows->hot_pre[n_rows] : (int64_t)a.units * pl.hot_tiles;
     const int64_t f_lo = (int64_t)c * pl.hot_tpc;
     const int64_t f_hi = f_lo + pl.hot_tpc < total ? f_lo + pl.hot_tpc : total;
     constexpr int CH = D / 8;        // 16-byte chunks per token row
@@ -897,12 +963,27 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
     sh.reset();
     uint32_t qh[S::NT][2];
     int unit_cur = -1, slot_cur = 0;
-    int unit = (int)(f_lo / ht);
-    int tile = (int)(f_lo - (int64_t)unit * ht);
+    int unit, tile;
+    if constexpr (RAGGED) {
+      int lo = 0, hi = n_rows - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (a.rows->hot_pre[mid] <= f_lo) lo = mid; else hi = mid - 1;
+      }
+      const int htr = row_tiles(lo);
+      const int64_t off = f_lo - a.rows->hot_pre[lo];
+      unit = lo * a.Hkv + (int)(off / htr);
+      tile = (int)(off % htr);
+    } else {
+      unit = (int)(f_lo / pl.hot_tiles);
+      tile = (int)(f_lo - (int64_t)unit * pl.hot_tiles);
+    }
+    int ht = unit_tiles(unit);
     for (int64_t f = f_lo; f < f_hi; ++f, ++tile) {
       if (tile == ht) {
         tile = 0;
-        ++unit;
+        unit = unit_next(unit);
+        ht = unit_tiles(unit);
       }
       if (unit != unit_cur) {
         if (unit_cur >= 0) {
@@ -911,7 +992,7 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
           sh.reset();
         }
         unit_cur = unit;
-        slot_cur = pl.slots_cold + (c - (int)(((int64_t)unit * ht) / pl.hot_tpc));
+        slot_cur = pl.slots_cold + (c - (int)(unit_hoff(unit) / pl.hot_tpc));
         const int b = unit / a.Hkv, kvh = unit % a.Hkv;
         const int head0 = b * a.Hq + kvh * G;
         if (gid < G) {
@@ -926,6 +1007,7 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
           for (int s = 0; s < S::NT; ++s) qh[s][0] = qh[s][1] = 0u;
         }
       }
+      const int n_hot_u = unit_nhot(unit);
       // the tile's K rows, then (in the same buffer) its V rows
       auto stage_rows = [&](const __half* src) {
         __syncthreads();
@@ -933,13 +1015,13 @@ __global__ void __launch_bounds__(kThreads, kAttendMinBlocks) attend_kernel(cons
           const int r = i / CH, cc = i % CH;
           const int slot = tile * S::TB + r;
           uint4 v = make_uint4(0u, 0u, 0u, 0u);
-          if (slot < a.n_hot)
+          if (slot < n_hot_u)
             v = __ldg(reinterpret_cast<const uint4*>(src + ((size_t)unit * a.W + slot) * D) + cc);
           *reinterpret_cast<uint4*>(ring + r * S::RS + cc * 16) = v;
         }
         __syncthreads();
       };
-      const int nvalid = a.n_hot - tile * S::TB < S::TB ? a.n_hot - tile * S::TB : S::TB;
+      const int nvalid = n_hot_u - tile * S::TB < S::TB ? n_hot_u - tile * S::TB : S::TB;
       const bool live = tb < nvalid;
       const uint32_t base = smem_addr(ring);
       const int mi = lane >> 3, rr = lane & 7;
@@ -990,6 +1072,7 @@ template <int D, int M, int BW, bool SLOT, int HMAP>
 AttendFn attend_fn_mode(int mode) {
   if (mode == MODE_GATED) return attend_kernel<D, M, BW, SLOT, HMAP, MODE_GATED>;
   if (mode == MODE_LOGITS) return attend_kernel<D, M, BW, SLOT, HMAP, MODE_LOGITS>;
+  if (mode == MODE_RAGGED) return attend_kernel<D, M, BW, SLOT, HMAP, MODE_RAGGED>;
   return attend_kernel<D, M, BW, SLOT, HMAP, MODE_PLAIN>;
 }
 

@@ -213,7 +213,19 @@ __global__ void combine_kernel(const CombineArgs a) {
   const int slots = pl.slots_cold + pl.slots_hot;
   const float* base = a.part + (size_t)unit * slots * a.G * (D + 2);
   int nc = 0, nh = 0;
-  if (pl.cold_ctas > 0 && pl.cold_blocks > 0) {
+  if (a.rows != nullptr) {             // ragged: the unit's own blocks and tiles
+    const int b = unit / a.Hkv, h = unit % a.Hkv;
+    const int64_t nb = (a.rows->n_cold[b] + kTokensPerBlock - 1) / kTokensPerBlock;
+    const int64_t ht = (a.rows->n_hot[b] + kTokensPerBlock - 1) / kTokensPerBlock;
+    if (nb > 0) {
+      const int64_t off = a.rows->cold_pre[b] + h * nb;
+      nc = (int)((off + nb - 1) / pl.cold_bpc - off / pl.cold_bpc + 1);
+    }
+    if (ht > 0) {
+      const int64_t off = a.rows->hot_pre[b] + h * ht;
+      nh = (int)((off + ht - 1) / pl.hot_tpc - off / pl.hot_tpc + 1);
+    }
+  } else if (pl.cold_ctas > 0 && pl.cold_blocks > 0) {
     const int64_t nb = pl.cold_blocks;
     if (a.unit_pos == nullptr) {
       nc = (int)(((unit + 1) * nb - 1) / pl.cold_bpc - (unit * nb) / pl.cold_bpc + 1);
@@ -227,7 +239,7 @@ __global__ void combine_kernel(const CombineArgs a) {
       }
     }
   }
-  if (pl.hot_ctas > 0 && pl.hot_tiles > 0) {
+  if (a.rows == nullptr && pl.hot_ctas > 0 && pl.hot_tiles > 0) {
     const int64_t ht = pl.hot_tiles;
     nh = (int)(((unit + 1) * ht - 1) / pl.hot_tpc - (unit * ht) / pl.hot_tpc + 1);
   }
@@ -324,7 +336,7 @@ att::AttendFn pick_attend(const Layout& L, int G, int mode, int* smem) {
 
 int attend_ctas_per_sm(const Layout& L, int G) {
   int smem = 0, n = 0;
-  for (int mode = att::MODE_PLAIN; mode <= att::MODE_LOGITS; ++mode) {
+  for (int mode = att::MODE_PLAIN; mode <= att::MODE_RAGGED; ++mode) {
     att::AttendFn fn = pick_attend(L, G, mode, &smem);
     if (!fn || cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return 0;
@@ -371,12 +383,27 @@ cudaError_t launch_qprep(const QPrepArgs& a, cudaStream_t s) {
 
 cudaError_t launch_attend(const AttendArgs& a, cudaStream_t s) {
   int smem = 0;
-  const int mode = a.alist ? att::MODE_GATED : (a.logits ? att::MODE_LOGITS : att::MODE_PLAIN);
+  const int mode = a.alist ? att::MODE_GATED
+                 : a.logits ? att::MODE_LOGITS
+                 : a.rows ? att::MODE_RAGGED : att::MODE_PLAIN;
   att::AttendFn fn = pick_attend(a.L, a.G, mode, &smem);
   if (!fn) return cudaErrorInvalidValue;
   const int grid = a.plan.cold_ctas > a.plan.hot_ctas ? a.plan.cold_ctas : a.plan.hot_ctas;
   if (grid == 0) return cudaSuccess;
   fn<<<grid, att::kThreads, smem, s>>>(a);
+  return cudaGetLastError();
+}
+
+namespace {
+__global__ void rows_upload_kernel(RowTable* dst, const RowTable src) {
+  const int32_t* s = reinterpret_cast<const int32_t*>(&src);
+  int32_t* d = reinterpret_cast<int32_t*>(dst);
+  for (int i = threadIdx.x; i < (int)(sizeof(RowTable) / 4); i += blockDim.x) d[i] = s[i];
+}
+}  // namespace
+
+cudaError_t launch_rows_upload(RowTable* dst, const RowTable& src, cudaStream_t s) {
+  rows_upload_kernel<<<1, 256, 0, s>>>(dst, src);
   return cudaGetLastError();
 }
 

@@ -82,6 +82,42 @@ __device__ __forceinline__ void chunk_word(int w, int ncodes, int bw, F code_of,
   }
 }
 
+// What one launch writes for a unit: n tokens at cold positions cold_start
+// .. cold_start + n - 1, the first nA read from ring slots (ring_start + e)
+// mod W, the rest from source tokens e - nA.  Uniform over the units, or
+// (ragged batch) from the unit's row: an append of n_new tokens, or an
+// insert of n_new tokens that evicts max(0, n_hot + n_new - W), the ring's
+// oldest first.
+struct UnitSpan {
+  int64_t cold_start, n;
+  int nA, ring_start;
+};
+
+__device__ __forceinline__ UnitSpan unit_span(const EncodeArgs& a, int unit) {
+  UnitSpan u;
+  if (a.rows != nullptr) {
+    const RowTable* r = a.rows;
+    const int b = unit / a.Hkv;
+    u.cold_start = r->n_cold[b];
+    if (a.ring_k == nullptr) {
+      u.n = r->n_new[b];
+      u.nA = 0;
+      u.ring_start = 0;
+    } else {
+      const int e = r->n_hot[b] + r->n_new[b] - a.W;
+      u.n = e > 0 ? e : 0;
+      u.nA = (int)(u.n < r->n_hot[b] ? u.n : r->n_hot[b]);
+      u.ring_start = ((r->ring_pos[b] - r->n_hot[b]) % a.W + a.W) % a.W;
+    }
+  } else {
+    u.cold_start = a.cold_start;
+    u.n = (int64_t)a.nA + a.nB;
+    u.nA = a.nA;
+    u.ring_start = a.ring_start;
+  }
+  return u;
+}
+
 // One warp per group of 4 tokens {2c, 2c+1, 2c+8, 2c+9} of a 16-token tile:
 // exactly the tokens whose fragment-major words can share a 32-bit word, so
 // no two warps ever write the same word.  D = padded length (power of two).
@@ -101,8 +137,8 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
 
   const Layout& L = a.L;
   const int bw = L.bw;
-  const int64_t n = (int64_t)a.nA + a.nB;
-  if (n == 0) return;
+  const int64_t n = (int64_t)a.nA + a.nB;    // (uniform; a ragged launch takes its counts per unit)
+  if (a.rows == nullptr && n == 0) return;
   // S^T in shared memory when it fits: the sign loop then waits on shared
   // memory instead of a chain of L2 round trips (the decode-step eviction
   // encodes one token per unit, so latency is all there is).
@@ -114,15 +150,20 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
     __syncthreads();
     St = sst;
   }
-  const int64_t t_first = a.cold_start / kTokensPerTile;
-  const int64_t t_last = (a.cold_start + n - 1) / kTokensPerTile;
-  const int64_t groups = (t_last - t_first + 1) * 4;
+  // uniform: every unit writes the same tile range; ragged: each its own,
+  // within groups_max groups
+  const int64_t groups = a.rows ? a.groups_max
+                                : ((a.cold_start + n - 1) / kTokensPerTile - a.cold_start / kTokensPerTile + 1) * 4;
   const int64_t jobs = (int64_t)a.units * groups;
 
   for (int64_t job = (int64_t)blockIdx.x * warps + warp; job < jobs;
        job += (int64_t)gridDim.x * warps) {
     const int unit = (int)(job / groups);
     const int64_t g = job % groups;
+    const UnitSpan us = unit_span(a, unit);
+    if (us.n == 0) continue;
+    const int64_t t_first = us.cold_start / kTokensPerTile;
+    if (g >= ((us.cold_start + us.n - 1) / kTokensPerTile - t_first + 1) * 4) continue;
     const int64_t tile = t_first + g / 4;
     const int c = (int)(g % 4);
     bool inr[4];
@@ -132,8 +173,8 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
     for (int s = 0; s < 4; ++s) {
       const int r = 2 * c + (s & 1) + 8 * (s >> 1);
       const int64_t t = tile * kTokensPerTile + r;
-      seq[s] = t - a.cold_start;
-      inr[s] = seq[s] >= 0 && seq[s] < n;
+      seq[s] = t - us.cold_start;
+      inr[s] = seq[s] >= 0 && seq[s] < us.n;
       any |= inr[s];
     }
     if (!any) continue;
@@ -142,13 +183,13 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
       const int64_t e = seq[s];
       const __half* ksrc;
       const __half* vsrc;
-      if (e < a.nA) {
-        const int slot = (int)((a.ring_start + e) % a.W);
+      if (e < us.nA) {
+        const int slot = (int)((us.ring_start + e) % a.W);
         ksrc = a.ring_k + ((int64_t)unit * a.W + slot) * D;
         vsrc = a.ring_v + ((int64_t)unit * a.W + slot) * D;
       } else {
-        ksrc = a.src_k + ((int64_t)unit * a.src_tokens + (e - a.nA)) * D;
-        vsrc = a.src_v + ((int64_t)unit * a.src_tokens + (e - a.nA)) * D;
+        ksrc = a.src_k + ((int64_t)unit * a.src_tokens + (e - us.nA)) * D;
+        vsrc = a.src_v + ((int64_t)unit * a.src_tokens + (e - us.nA)) * D;
       }
       encode_vector<D>(a, St, ksrc, true, rbuf, kc + s * P, kb + s * 8, sc + s * 4, sc + s * 4 + 1);
       encode_vector<D>(a, St, vsrc, false, rbuf, vc + s * P, nullptr, sc + s * 4 + 2, nullptr);
@@ -233,7 +274,8 @@ __global__ void __launch_bounds__(2 * D) encode_small_kernel(EncodeArgs a) {
   constexpr int P = D / 2;
   constexpr int NW = D / 32;                 // warps per team
   const Layout& L = a.L;
-  const int64_t n = a.promo ? (int64_t)(kPromoMax + a.n_new) : (int64_t)a.nA + a.nB;
+  const int64_t n = a.promo ? (int64_t)(kPromoMax + a.n_new)
+                  : a.rows ? (int64_t)a.n_max : (int64_t)a.nA + a.nB;
   const int unit = (int)(blockIdx.x / n);
   const int64_t e = blockIdx.x % n;
   const int tid = threadIdx.x, team = tid / D, el = tid % D;
@@ -274,12 +316,20 @@ __global__ void __launch_bounds__(2 * D) encode_small_kernel(EncodeArgs a) {
       dest = a.cold_start + (e - k);
       nsrc = (team ? a.src_v : a.src_k) + ((int64_t)unit * a.src_tokens + (e - k)) * D;
     }
-  } else if (e < a.nA) {
-    const int slot = (int)((a.ring_start + e) % a.W);
-    src = (team ? a.ring_v : a.ring_k) + ((int64_t)unit * a.W + slot) * D;
-    if (a.write_new) nsrc = (team ? a.src_v : a.src_k) + ((int64_t)unit * a.src_tokens + e) * D;
   } else {
-    src = (team ? a.src_v : a.src_k) + ((int64_t)unit * a.src_tokens + (e - a.nA)) * D;
+    const UnitSpan us = unit_span(a, unit);
+    if (e >= us.n) {                         // (the whole CTA) nothing for this unit
+      async_copy_wait();
+      return;
+    }
+    dest = us.cold_start + e;
+    if (e < us.nA) {
+      const int slot = (int)((us.ring_start + e) % a.W);
+      src = (team ? a.ring_v : a.ring_k) + ((int64_t)unit * a.W + slot) * D;
+      if (a.write_new) nsrc = (team ? a.src_v : a.src_k) + ((int64_t)unit * a.src_tokens + e) * D;
+    } else {
+      src = (team ? a.src_v : a.src_k) + ((int64_t)unit * a.src_tokens + (e - us.nA)) * D;
+    }
   }
   // ---- rotation: y = H (D x) / sqrt(d) ----------------------------------
   const __half xin = src[el];
@@ -439,7 +489,7 @@ __global__ void __launch_bounds__(2 * D) encode_small_kernel(EncodeArgs a) {
 
 __global__ void ring_write_kernel(__half* ring_k, __half* ring_v, const __half* k_new,
                                   const __half* v_new, int units, int W, int d, int n,
-                                  int first, int ring_pos) {
+                                  int first, int ring_pos, const RowTable* rows, int Hkv) {
   const int chunks = d / 8;   // 16-byte chunks per token
   const int64_t per_unit = (int64_t)(n - first) * chunks;
   const int64_t total = 2 * (int64_t)units * per_unit;
@@ -451,7 +501,13 @@ __global__ void ring_write_kernel(__half* ring_k, __half* ring_v, const __half* 
     const int64_t r = j % per_unit;
     const int i = first + (int)(r / chunks);
     const int c = (int)(r % chunks);
-    const int slot = (int)(((int64_t)ring_pos + i) % W);
+    int rp = ring_pos;
+    if (rows != nullptr) {          // ragged: row b writes its tokens [max(0, n_b - W), n_b)
+      const int b = unit / Hkv, nb = rows->n_new[b];
+      if (i >= nb || i < nb - W) continue;
+      rp = rows->ring_pos[b];
+    }
+    const int slot = (int)(((int64_t)rp + i) % W);
     const uint4* s = reinterpret_cast<const uint4*>((is_k ? k_new : v_new) + ((int64_t)unit * n + i) * d) + c;
     uint4* dst = reinterpret_cast<uint4*>((is_k ? ring_k : ring_v) + ((int64_t)unit * W + slot) * d) + c;
     *dst = *s;
@@ -461,7 +517,8 @@ __global__ void ring_write_kernel(__half* ring_k, __half* ring_v, const __half* 
 template <int D>
 cudaError_t launch_encode_d(const EncodeArgs& a, cudaStream_t s) {
   const int warps = 8;
-  const int64_t n = a.promo ? (int64_t)(kPromoMax + a.n_new) : (int64_t)a.nA + a.nB;
+  const int64_t n = a.promo ? (int64_t)(kPromoMax + a.n_new)
+                  : a.rows ? (int64_t)a.n_max : (int64_t)a.nA + a.nB;
   if (n == 0) return cudaSuccess;
   if (D <= 128 && (n <= kSmallEncodeTokens || a.promo)) {
     const size_t smem = small_st_offset(D) + (size_t)D * a.L.m * sizeof(float);
@@ -482,8 +539,9 @@ cudaError_t launch_encode_d(const EncodeArgs& a, cudaStream_t s) {
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, encode_small_kernel<D>, a);
   }
-  const int64_t tiles = (a.cold_start + n - 1) / kTokensPerTile - a.cold_start / kTokensPerTile + 1;
-  const int64_t jobs = (int64_t)a.units * tiles * 4;
+  const int64_t jobs = a.rows ? (int64_t)a.units * a.groups_max
+                               : (int64_t)a.units * 4 *
+                                     ((a.cold_start + n - 1) / kTokensPerTile - a.cold_start / kTokensPerTile + 1);
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -513,14 +571,14 @@ cudaError_t launch_encode(const EncodeArgs& a, cudaStream_t s) {
 
 cudaError_t launch_ring_write(__half* ring_k, __half* ring_v, const __half* k_new,
                               const __half* v_new, int units, int W, int d, int n, int first,
-                              int ring_pos, cudaStream_t s) {
+                              int ring_pos, cudaStream_t s, const RowTable* rows, int Hkv) {
   const int64_t total = 2 * (int64_t)units * (n - first) * (d / 8);
   if (total <= 0) return cudaSuccess;
   const int threads = 256;
   const int64_t want = (total + threads - 1) / threads;
   const int grid = (int)(want < 4096 ? want : 4096);
   ring_write_kernel<<<grid, threads, 0, s>>>(ring_k, ring_v, k_new, v_new, units, W, d, n, first,
-                                             ring_pos);
+                                             ring_pos, rows, Hkv);
   return cudaGetLastError();
 }
 

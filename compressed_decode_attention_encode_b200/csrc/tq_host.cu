@@ -57,7 +57,7 @@ bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 }  // namespace
 
 struct WsLayout {
-  size_t status, signs, S, St, q, part, gate, gate_max, total;
+  size_t status, signs, S, St, q, part, gate, gate_max, rows, total;
   QBufsLayout ql;               // query transforms, at offset q
 };
 
@@ -79,6 +79,7 @@ static WsLayout ws_layout(const tq_config& c) {
   const size_t gate_chunks = (c.hot_window + kGateRowsMin - 1) / kGateRowsMin;
   w.gate = off;   off += round_up(sizeof(int) * (heads + 2 * units + 2), kAlign);
   w.gate_max = off; off += round_up(sizeof(float) * heads * std::max<size_t>(gate_chunks, 1), kAlign);
+  w.rows = off;   off += round_up(sizeof(RowTable), kAlign);   // per-row counts of a ragged batch
   w.total = off;
   return w;
 }
@@ -122,6 +123,12 @@ struct tq_cache {
   cudaEvent_t ev_start;
   cudaEvent_t ev_stop;
   unsigned long long wait_limit_ns;   // attention kernel's bounded waits (tq_set_wait_limit)
+  // per batch row: cold tokens, valid hot tokens, next ring slot.  While
+  // they are equal across rows (`ragged` false) the scalars above hold them
+  // and the uniform paths run; otherwise the kernels read a RowTable.
+  std::vector<int64_t> row_cold;
+  std::vector<int32_t> row_hot, row_pos;
+  bool ragged;
   // attention-weighted promotion (tq_promotion_enable), or null
   uint8_t* promo;
   float promo_threshold;
@@ -181,6 +188,53 @@ static PromoArgs promo_args(const tq_cache* c) {
   return a;
 }
 
+// ---- per-row state -----------------------------------------------------
+// After a uniform operation every row takes the scalars' values; after a
+// ragged one the scalars are set from the rows when those agree again.
+static void rows_from_scalars(tq_cache* c) {
+  std::fill(c->row_cold.begin(), c->row_cold.end(), c->n_cold);
+  std::fill(c->row_hot.begin(), c->row_hot.end(), c->n_hot);
+  std::fill(c->row_pos.begin(), c->row_pos.end(), c->ring_pos);
+}
+
+static void scalars_from_rows(tq_cache* c) {
+  const int B = c->cfg.batch;
+  bool same = true;
+  for (int b = 1; b < B; ++b)
+    same &= c->row_cold[b] == c->row_cold[0] && c->row_hot[b] == c->row_hot[0] &&
+            c->row_pos[b] == c->row_pos[0];
+  c->ragged = !same;
+  c->n_cold = *std::max_element(c->row_cold.begin(), c->row_cold.end());
+  c->n_hot = *std::max_element(c->row_hot.begin(), c->row_hot.end());
+  c->ring_pos = c->row_pos[0];
+  c->dirty_lo = 0;
+  c->dirty_n = c->cfg.hot_window;      // the gate reads the whole window after a ragged step
+}
+
+// The row table of the current counts (n_new per row, and the decode's
+// prefix sums of blocks / tiles), written into the workspace.
+static RowTable build_rows(const tq_cache* c, const int32_t* n_new) {
+  const int B = c->cfg.batch, H = c->cfg.num_kv_heads;
+  RowTable t{};
+  t.cold_pre[0] = t.hot_pre[0] = 0;
+  for (int b = 0; b < B; ++b) {
+    t.n_cold[b] = (int32_t)c->row_cold[b];
+    t.n_hot[b] = c->row_hot[b];
+    t.ring_pos[b] = c->row_pos[b];
+    t.n_new[b] = n_new ? n_new[b] : 0;
+    t.cold_pre[b + 1] = t.cold_pre[b] + H * (int32_t)((c->row_cold[b] + kTokensPerBlock - 1) / kTokensPerBlock);
+    t.hot_pre[b + 1] = t.hot_pre[b] + H * ((c->row_hot[b] + kTokensPerBlock - 1) / kTokensPerBlock);
+  }
+  return t;
+}
+
+static tq_status upload_rows(tq_cache* c, const int32_t* n_new, cudaStream_t stream, RowTable* out = nullptr) {
+  const RowTable t = build_rows(c, n_new);
+  if (out) *out = t;
+  if (launch_rows_upload((RowTable*)(c->ws + c->W.rows), t, stream) != cudaSuccess) return TQ_ERR_CUDA;
+  return TQ_OK;
+}
+
 extern "C" {
 
 const char* tq_status_string(tq_status s) {
@@ -235,6 +289,10 @@ tq_status tq_cache_create(const tq_config* cfg, void* hot_mem, void* cold_mem,
   c->tc = c->tc_lam = c->tc_eta = c->tc_sig = nullptr;
   c->wait_limit_ns = kDefaultWaitLimitNs;
   c->promo = nullptr;
+  c->row_cold.assign(cfg->batch, 0);
+  c->row_hot.assign(cfg->batch, 0);
+  c->row_pos.assign(cfg->batch, 0);
+  c->ragged = false;
   if (cudaGetDevice(&c->device) != cudaSuccess ||
       cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, c->device) != cudaSuccess) {
     delete c;
@@ -294,15 +352,17 @@ static EncodeArgs base_encode_args(tq_cache* c) {
   return a;
 }
 
-tq_status tq_encode_append(tq_cache* c, const void* k, const void* v, int64_t n, cudaStream_t stream) {
-  if (!c || n < 0) return TQ_ERR_INVALID_ARG;
+// Append n tokens to every row (rows share their counts); source tokens
+// are [units, src_tokens, d].
+static tq_status encode_append_uniform(tq_cache* c, const void* k, const void* v, int64_t n,
+                                       int64_t src_tokens, cudaStream_t stream) {
   if (n == 0) return TQ_OK;
   if (!k || !v) return TQ_ERR_INVALID_ARG;
   if (c->n_cold + n > c->cfg.cold_capacity) return TQ_ERR_CAPACITY;
   EncodeArgs a = base_encode_args(c);
   a.src_k = (const __half*)k;
   a.src_v = (const __half*)v;
-  a.src_tokens = n;
+  a.src_tokens = src_tokens;
   a.nB = n;
   a.nA = 0;
   if (launch_encode(a, stream) != cudaSuccess) return TQ_ERR_CUDA;
@@ -310,9 +370,9 @@ tq_status tq_encode_append(tq_cache* c, const void* k, const void* v, int64_t n,
   return TQ_OK;
 }
 
-tq_status tq_evict_window(tq_cache* c, const void* k_new, const void* v_new, int32_t n,
-                          cudaStream_t stream) {
-  if (!c || !k_new || !v_new || n < 1) return TQ_ERR_INVALID_ARG;
+// Insert n tokens into every row's ring (rows share their counts).
+static tq_status evict_window_uniform(tq_cache* c, const void* k_new, const void* v_new, int32_t n,
+                                      cudaStream_t stream) {
   const int W = c->cfg.hot_window;
   const int64_t E = std::max<int64_t>(0, (int64_t)c->n_hot + n - W);
   if (c->tc) {
@@ -410,6 +470,138 @@ tq_status tq_evict_window(tq_cache* c, const void* k_new, const void* v_new, int
   return TQ_OK;
 }
 
+tq_status tq_encode_append(tq_cache* c, const void* k, const void* v, int64_t n, cudaStream_t stream) {
+  if (!c || n < 0) return TQ_ERR_INVALID_ARG;
+  if (c->ragged) {
+    if (n > INT32_MAX) return TQ_ERR_INVALID_ARG;
+    std::vector<int32_t> rows(c->cfg.batch, (int32_t)n);
+    return tq_encode_append_rows(c, k, v, n, rows.data(), stream);
+  }
+  const tq_status st = encode_append_uniform(c, k, v, n, n, stream);
+  if (st == TQ_OK) rows_from_scalars(c);
+  return st;
+}
+
+tq_status tq_evict_window(tq_cache* c, const void* k_new, const void* v_new, int32_t n,
+                          cudaStream_t stream) {
+  if (!c || !k_new || !v_new || n < 1) return TQ_ERR_INVALID_ARG;
+  if (c->ragged) {
+    std::vector<int32_t> rows(c->cfg.batch, n);
+    return tq_evict_window_rows(c, k_new, v_new, n, rows.data(), stream);
+  }
+  const tq_status st = evict_window_uniform(c, k_new, v_new, n, stream);
+  if (st == TQ_OK) rows_from_scalars(c);
+  return st;
+}
+
+// Most 4-token groups of 16-token tiles any row's units write when row b
+// writes cold positions [n_cold_b, n_cold_b + cnt[b]).
+static int64_t max_groups(const tq_cache* c, const std::vector<int64_t>& cnt) {
+  int64_t g = 0;
+  for (int b = 0; b < c->cfg.batch; ++b)
+    if (cnt[b] > 0) {
+      const int64_t s = c->row_cold[b], e = s + cnt[b] - 1;
+      g = std::max<int64_t>(g, (e / kTokensPerTile - s / kTokensPerTile + 1) * 4);
+    }
+  return g;
+}
+
+tq_status tq_encode_append_rows(tq_cache* c, const void* k, const void* v, int64_t n_max,
+                                const int32_t* n_rows, cudaStream_t stream) {
+  if (!c || !n_rows || n_max < 0) return TQ_ERR_INVALID_ARG;
+  const int B = c->cfg.batch;
+  bool any = false, same = true;
+  int64_t mx = 0;
+  for (int b = 0; b < B; ++b) {
+    if (n_rows[b] < 0 || n_rows[b] > n_max) return TQ_ERR_INVALID_ARG;
+    any |= n_rows[b] > 0;
+    same &= n_rows[b] == n_rows[0];
+    mx = std::max<int64_t>(mx, n_rows[b]);
+  }
+  if (!any) return TQ_OK;
+  if (!k || !v) return TQ_ERR_INVALID_ARG;
+  for (int b = 0; b < B; ++b)
+    if (c->row_cold[b] + n_rows[b] > c->cfg.cold_capacity) return TQ_ERR_CAPACITY;
+  if (same && !c->ragged) {
+    const tq_status st = encode_append_uniform(c, k, v, n_rows[0], n_max, stream);
+    if (st == TQ_OK) rows_from_scalars(c);
+    return st;
+  }
+  if (B > kMaxRaggedRows || c->tc || c->promo) return TQ_ERR_UNSUPPORTED;
+  if (upload_rows(c, n_rows, stream) != TQ_OK) return TQ_ERR_CUDA;
+  EncodeArgs a = base_encode_args(c);
+  a.src_k = (const __half*)k;
+  a.src_v = (const __half*)v;
+  a.src_tokens = n_max;
+  a.rows = (const RowTable*)(c->ws + c->W.rows);
+  a.Hkv = c->cfg.num_kv_heads;
+  a.n_max = (int)mx;
+  a.groups_max = max_groups(c, std::vector<int64_t>(n_rows, n_rows + B));
+  if (launch_encode(a, stream) != cudaSuccess) return TQ_ERR_CUDA;
+  for (int b = 0; b < B; ++b) c->row_cold[b] += n_rows[b];
+  scalars_from_rows(c);
+  return TQ_OK;
+}
+
+tq_status tq_evict_window_rows(tq_cache* c, const void* k_new, const void* v_new, int32_t n_max,
+                               const int32_t* n_rows, cudaStream_t stream) {
+  if (!c || !n_rows || !k_new || !v_new || n_max < 1) return TQ_ERR_INVALID_ARG;
+  const int B = c->cfg.batch, W = c->cfg.hot_window;
+  bool any = false, same = true;
+  std::vector<int64_t> ev(B);
+  int64_t emax = 0;
+  for (int b = 0; b < B; ++b) {
+    if (n_rows[b] < 0 || n_rows[b] > n_max) return TQ_ERR_INVALID_ARG;
+    any |= n_rows[b] > 0;
+    same &= n_rows[b] == n_rows[0];
+    ev[b] = std::max<int64_t>(0, (int64_t)c->row_hot[b] + n_rows[b] - W);
+    emax = std::max(emax, ev[b]);
+    if (c->row_cold[b] + ev[b] > c->cfg.cold_capacity) return TQ_ERR_CAPACITY;
+  }
+  if (!any) return TQ_OK;
+  if (same && !c->ragged && n_rows[0] == n_max) {
+    const tq_status st = evict_window_uniform(c, k_new, v_new, n_max, stream);
+    if (st == TQ_OK) rows_from_scalars(c);
+    return st;
+  }
+  if (B > kMaxRaggedRows || c->tc || c->promo) return TQ_ERR_UNSUPPORTED;
+  if (upload_rows(c, n_rows, stream) != TQ_OK) return TQ_ERR_CUDA;
+  const RowTable* rows = (const RowTable*)(c->ws + c->W.rows);
+  if (emax > 0) {
+    EncodeArgs a = base_encode_args(c);
+    a.ring_k = c->hot_k();
+    a.ring_v = c->hot_v();
+    a.src_k = (const __half*)k_new;
+    a.src_v = (const __half*)v_new;
+    a.src_tokens = n_max;
+    a.rows = rows;
+    a.Hkv = c->cfg.num_kv_heads;
+    a.n_max = (int)emax;
+    a.groups_max = max_groups(c, ev);
+    if (launch_encode(a, stream) != cudaSuccess) return TQ_ERR_CUDA;
+  }
+  if (launch_ring_write(c->hot_k(), c->hot_v(), (const __half*)k_new, (const __half*)v_new,
+                        B * c->cfg.num_kv_heads, W, c->cfg.head_dim, n_max, 0, 0, stream, rows,
+                        c->cfg.num_kv_heads) != cudaSuccess)
+    return TQ_ERR_CUDA;
+  for (int b = 0; b < B; ++b) {
+    c->row_cold[b] += ev[b];
+    c->row_hot[b] = std::min(W, c->row_hot[b] + n_rows[b]);
+    c->row_pos[b] = (int32_t)(((int64_t)c->row_pos[b] + n_rows[b]) % W);
+  }
+  scalars_from_rows(c);
+  return TQ_OK;
+}
+
+tq_status tq_cache_row_counts(const tq_cache* c, int32_t row, int64_t* n_cold, int32_t* n_hot,
+                              int32_t* ring_pos) {
+  if (!c || row < 0 || row >= c->cfg.batch) return TQ_ERR_INVALID_ARG;
+  if (n_cold) *n_cold = c->row_cold[row];
+  if (n_hot) *n_hot = c->row_hot[row];
+  if (ring_pos) *ring_pos = c->row_pos[row];
+  return TQ_OK;
+}
+
 // Split plan: one wave of `ctas` CTAs.  Every CTA streams an equal run of
 // the flattened (unit, cold block) list; CTAs [0, hot_ctas) then also take
 // hot_tpc hot tiles each (one for the usual window sizes), so the latency
@@ -449,6 +641,55 @@ static SplitPlan make_plan(int64_t n_cold, int n_hot, int units, int ctas, bool 
   return pl;
 }
 
+// The split of a ragged batch: the units' blocks (tiles) are flattened by
+// the table's prefix sums; blocks per CTA follow the uniform rule with the
+// longest row's block count; `tight` sizes the slots to the most CTAs any
+// unit spans.
+static SplitPlan make_plan_ragged(const RowTable& t, int B, int H, int ctas, bool tight) {
+  const int TB = kTokensPerBlock;
+  int64_t maxnb = 0, maxht = 0;
+  for (int b = 0; b < B; ++b) {
+    maxnb = std::max<int64_t>(maxnb, (t.n_cold[b] + TB - 1) / TB);
+    maxht = std::max<int64_t>(maxht, (t.n_hot[b] + TB - 1) / TB);
+  }
+  const int64_t N = t.cold_pre[B], Nh = t.hot_pre[B];
+  SplitPlan pl{};
+  pl.cold_blocks = maxnb;
+  pl.hot_tiles = (int)maxht;
+  pl.slots_cold = tight ? 0 : kSlotsCold;
+  pl.slots_hot = tight ? 0 : kSlotsHot;
+  auto span = [](int64_t off, int64_t n, int64_t per) { return n > 0 ? (int)((off + n - 1) / per - off / per + 1) : 0; };
+  if (Nh > 0) {
+    int64_t tpc = (Nh + ctas - 1) / ctas;
+    tpc = std::max<int64_t>(tpc, maxht > 1 ? (maxht - 1 + kSlotsHot - 3) / (kSlotsHot - 2) : 1);
+    pl.hot_tpc = (int)tpc;
+    pl.hot_ctas = (int)((Nh + tpc - 1) / tpc);
+    if (tight) {
+      int mx = 0;
+      for (int b = 0; b < B; ++b) {
+        const int64_t ht = (t.n_hot[b] + TB - 1) / TB;
+        for (int h = 0; h < H; ++h) mx = std::max(mx, span(t.hot_pre[b] + h * ht, ht, tpc));
+      }
+      pl.slots_hot = mx;
+    }
+  }
+  if (N > 0) {
+    int64_t bpc = (N + ctas - 1) / ctas;
+    bpc = std::max<int64_t>(bpc, maxnb > 1 ? (maxnb - 1 + kSlotsCold - 3) / (kSlotsCold - 2) : 1);
+    pl.cold_bpc = bpc;
+    pl.cold_ctas = (int)((N + bpc - 1) / bpc);
+    if (tight) {
+      int mx = 0;
+      for (int b = 0; b < B; ++b) {
+        const int64_t nb = (t.n_cold[b] + TB - 1) / TB;
+        for (int h = 0; h < H; ++h) mx = std::max(mx, span(t.cold_pre[b] + h * nb, nb, bpc));
+      }
+      pl.slots_cold = mx;
+    }
+  }
+  return pl;
+}
+
 // Gated decode: the workspace's gate area and the caller's threshold.
 struct GateBuffers {
   int* head_skip;
@@ -466,7 +707,7 @@ struct GateBuffers {
 // (workspace or static scratch).
 static tq_status launch_decode(tq_cache* c, const void* q, float* out, float softmax_scale,
                                const SplitPlan& pl, const QBufs& qb, float* part, cudaStream_t stream,
-                               const GateBuffers* gate = nullptr) {
+                               const GateBuffers* gate = nullptr, const RowTable* rows = nullptr) {
   const tq_config& cf = c->cfg;
   const int d = cf.head_dim;
   const int units = cf.batch * cf.num_kv_heads;
@@ -530,6 +771,7 @@ static tq_status launch_decode(tq_cache* c, const void* q, float* out, float sof
   a.n_hot = c->n_hot;
   a.n_cold = c->n_cold;
   a.plan = pl;
+  a.rows = rows;
   a.log2e_sigma = (float)(1.4426950408889634 * (double)sigma);
   a.wait_limit_ns = c->wait_limit_ns;
   if (gate) {
@@ -557,6 +799,7 @@ static tq_status launch_decode(tq_cache* c, const void* q, float* out, float sof
   ca.Hq = cf.num_q_heads;
   ca.d = d;
   ca.plan = pl;
+  ca.rows = rows;
   ca.batch = cf.batch;
   if (gate) {
     ca.head_skip = gate->head_skip;
@@ -587,6 +830,14 @@ tq_status tq_decode_attention(tq_cache* c, const void* q, float* out, float soft
       (uintptr_t)q % 16)
     return TQ_ERR_INVALID_ARG;
   const int units = c->cfg.batch * c->cfg.num_kv_heads;
+  if (c->ragged) {
+    RowTable t;
+    if (upload_rows(c, nullptr, stream, &t) != TQ_OK) return TQ_ERR_CUDA;
+    const SplitPlan pl = make_plan_ragged(t, c->cfg.batch, c->cfg.num_kv_heads,
+                                          c->num_sms * c->ctas_per_sm, false);
+    return launch_decode(c, q, out, softmax_scale, pl, qbufs_at(c->ws + c->W.q, c->W.ql),
+                         (float*)(c->ws + c->W.part), stream, nullptr, (const RowTable*)(c->ws + c->W.rows));
+  }
   const SplitPlan pl = make_plan(c->n_cold, c->n_hot, units, c->num_sms * c->ctas_per_sm, false);
   return launch_decode(c, q, out, softmax_scale, pl, qbufs_at(c->ws + c->W.q, c->W.ql),
                        (float*)(c->ws + c->W.part), stream);
@@ -597,7 +848,7 @@ tq_status tq_decode_attention_gated(tq_cache* c, const void* q, float* out, floa
   if (!c || !q || !out || !(softmax_scale >= 0.0f) || std::isinf(softmax_scale) ||
       std::isnan(threshold) || (uintptr_t)q % 16)
     return TQ_ERR_INVALID_ARG;
-  if (c->promo) return TQ_ERR_UNSUPPORTED;      // promotion counts the ungated decode's masses
+  if (c->promo || c->ragged) return TQ_ERR_UNSUPPORTED;   // uniform batches, no promotion
   const tq_config& cf = c->cfg;
   const int units = cf.batch * cf.num_kv_heads;
   const int heads = cf.batch * cf.num_q_heads;
@@ -635,6 +886,7 @@ tq_status tq_tc_enable(tq_cache* c, void* tc_mem, const float* lambda, const flo
                        const float* gate, cudaStream_t stream) {
   if (!c || !tc_mem || !lambda || !eta || !gate || (uintptr_t)tc_mem % kAlign) return TQ_ERR_INVALID_ARG;
   if (c->tc || c->promo) return TQ_ERR_INVALID_ARG;         // already enabled, or promotion on
+  if (c->ragged) return TQ_ERR_UNSUPPORTED;
   const tq_config& cf = c->cfg;
   const int hkv = cf.num_kv_heads, hq = cf.num_q_heads;
   std::vector<float> par(2 * hkv + hq);
@@ -676,6 +928,7 @@ tq_status tq_promotion_enable(tq_cache* c, void* mem, float threshold, int32_t s
       sticky < 1 || c->cfg.hot_window <= kPromoMax)
     return TQ_ERR_INVALID_ARG;
   if (c->tc || c->promo) return TQ_ERR_INVALID_ARG;        // Tensor Cache tier, or already on
+  if (c->ragged) return TQ_ERR_UNSUPPORTED;
   const size_t units = (size_t)c->cfg.batch * c->cfg.num_kv_heads;
   std::vector<PromoUnitState> st(units);
   for (auto& u : st) {
@@ -785,7 +1038,10 @@ tq_status tq_decode_attention_static(tq_cache* c, const void* q, float* out, flo
 
   // The same split plan as tq_decode_attention, with the partial slots per
   // unit cut to the most any unit can receive under this plan.
-  const SplitPlan pl = make_plan(c->n_cold, c->n_hot, units, c->num_sms * c->ctas_per_sm, true);
+  RowTable t{};
+  if (c->ragged) t = build_rows(c, nullptr);    // (a ragged batch has at most kMaxRaggedRows rows)
+  const SplitPlan pl = c->ragged ? make_plan_ragged(t, cf.batch, cf.num_kv_heads, c->num_sms * c->ctas_per_sm, true)
+                                 : make_plan(c->n_cold, c->n_hot, units, c->num_sms * c->ctas_per_sm, true);
 
   // scratch layout: query transforms | partials
   const QBufsLayout ql = qbufs_layout((size_t)heads, d, m);
@@ -796,7 +1052,10 @@ tq_status tq_decode_attention_static(tq_cache* c, const void* q, float* out, flo
 
   uint8_t* base = (uint8_t*)static_scratch_address(current);
   if (!base) return TQ_ERR_CUDA;
-  return launch_decode(c, q, out, softmax_scale, pl, qbufs_at(base, ql), (float*)(base + o_part), stream);
+  if (c->ragged && launch_rows_upload((RowTable*)(c->ws + c->W.rows), t, stream) != cudaSuccess)
+    return TQ_ERR_CUDA;
+  return launch_decode(c, q, out, softmax_scale, pl, qbufs_at(base, ql), (float*)(base + o_part), stream,
+                       nullptr, c->ragged ? (const RowTable*)(c->ws + c->W.rows) : nullptr);
 }
 
 tq_status tq_get_status(tq_cache* c, cudaStream_t stream) {
@@ -816,7 +1075,7 @@ tq_status tq_export_cold(tq_cache* c, int32_t row, int32_t kv_head, int64_t star
                          uint8_t* k_codes, uint8_t* k_bits, uint16_t* k_s16, uint16_t* k_rn16,
                          uint8_t* v_codes, uint16_t* v_s16, cudaStream_t stream) {
   if (!c || row < 0 || row >= c->cfg.batch || kv_head < 0 || kv_head >= c->cfg.num_kv_heads ||
-      start < 0 || count < 0 || start + count > c->n_cold)
+      start < 0 || count < 0 || start + count > c->row_cold[row])
     return TQ_ERR_INVALID_ARG;
   if (count == 0) return TQ_OK;
   if (cudaStreamSynchronize(stream) != cudaSuccess) return TQ_ERR_CUDA;

@@ -104,6 +104,23 @@ __host__ __device__ inline Layout layout_of(int d, int b_r, int b_theta, int m, 
 }
 
 
+// ---- ragged batches: per-row lengths -------------------------------------
+// When the rows of a batch hold different numbers of cold or hot tokens,
+// the kernels read each row's counts from this table (in the workspace,
+// written by one small launch whenever the counts change).
+constexpr int kMaxRaggedRows = 128;
+
+struct RowTable {
+  int32_t n_cold[kMaxRaggedRows];         // cold tokens of row b (before an append / insert)
+  int32_t n_hot[kMaxRaggedRows];          // valid hot tokens
+  int32_t ring_pos[kMaxRaggedRows];       // next ring slot
+  int32_t n_new[kMaxRaggedRows];          // tokens the current append / insert brings to row b
+  int32_t cold_pre[kMaxRaggedRows + 1];   // (decode) cold blocks of the units of rows before b
+  int32_t hot_pre[kMaxRaggedRows + 1];    // (decode) hot tiles of the units of rows before b
+};
+
+cudaError_t launch_rows_upload(RowTable* dst, const RowTable& src, cudaStream_t s);
+
 // ---- attention-weighted promotion ---------------------------------------
 // At most this many tokens per (row, kv head) are counted or promoted per
 // decode step: with a threshold >= 1/8 no more can reach it, because a
@@ -157,6 +174,15 @@ struct EncodeArgs {
   const __half* promo_k;
   const __half* promo_v;
   int n_new;
+  // Ragged batch (null otherwise): row b = unit / Hkv appends rows->n_new[b]
+  // tokens at rows->n_cold[b] (ring_k null), or inserts them into its ring
+  // (evicting max(0, n_hot + n_new - W) tokens, the ring's oldest first);
+  // source tokens are [units, src_tokens = n_max, d].  groups_max: the most
+  // 4-token groups of 16-token tiles any unit writes (warp path).
+  const RowTable* rows;
+  int Hkv;
+  int n_max;
+  int64_t groups_max;
 };
 
 // Global -> shared copy of `bytes` (a multiple of 16, both addresses 16-byte
@@ -182,10 +208,13 @@ constexpr int64_t kSmallEncodeTokens = 8;
 
 cudaError_t launch_encode(const EncodeArgs& a, cudaStream_t s);
 
-// Copies new tokens i in [first, n) into ring slots (ring_pos + i) mod W.
+// Copies new tokens i in [first, n) into ring slots (ring_pos + i) mod W
+// (ragged: row b's tokens i in [max(0, n_new - W), n_new) at its own ring
+// position, from [units, n, d]).
 cudaError_t launch_ring_write(__half* ring_k, __half* ring_v, const __half* k_new,
                               const __half* v_new, int units, int W, int d, int n,
-                              int first, int ring_pos, cudaStream_t s);
+                              int first, int ring_pos, cudaStream_t s,
+                              const RowTable* rows = nullptr, int Hkv = 1);
 
 // ---- decode -------------------------------------------------------------
 // Query transforms of one decode call (written by q-prep, per query head h):
@@ -290,6 +319,9 @@ struct AttendArgs {
   int W, n_hot;
   int64_t n_cold;
   float log2e_sigma;        // log2(e) * softmax scale
+  // Ragged batch (the attention kernel's RAGGED mode): per-row counts and
+  // the units' block / tile prefix sums.
+  const RowTable* rows;
   // When non-null (promotion enabled): every valid cold token's log2-domain
   // logit of every query head, [units][logit_capacity][G].
   float* logits;
@@ -309,6 +341,7 @@ int attend_ctas_per_sm(const Layout& L, int G);
 
 struct CombineArgs {
   const float* part;
+  const RowTable* rows;     // ragged batch, or null
   float* ml;                // null, or [B*Hq][2]: each head's final max (log2) and sum
   const int* status;        // device status word: NaN output while kStatusNoPartials is latched
   const double* signs;

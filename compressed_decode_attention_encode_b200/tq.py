@@ -55,6 +55,10 @@ SIGNATURES = [
     ("tq_cache_destroy", c_int32, [c_void_p]),
     ("tq_cache_counts", c_int32, [c_void_p, POINTER(c_int64), POINTER(c_int32), POINTER(c_int32)]),
     ("tq_encode_append", c_int32, [c_void_p, c_void_p, c_void_p, c_int64, c_void_p]),
+    ("tq_encode_append_rows", c_int32, [c_void_p, c_void_p, c_void_p, c_int64, c_void_p, c_void_p]),
+    ("tq_evict_window_rows", c_int32, [c_void_p, c_void_p, c_void_p, c_int32, c_void_p, c_void_p]),
+    ("tq_cache_row_counts", c_int32, [c_void_p, c_int32, POINTER(c_int64), POINTER(c_int32),
+                                      POINTER(c_int32)]),
     ("tq_evict_window", c_int32, [c_void_p, c_void_p, c_void_p, c_int32, c_void_p]),
     ("tq_decode_attention", c_int32, [c_void_p, c_void_p, c_void_p, c_float, c_void_p]),
     ("tq_decode_attention_static", c_int32, [c_void_p, c_void_p, c_void_p, c_float, c_void_p]),
@@ -358,6 +362,26 @@ class TQCache:
 
     def counts(self):
         return tq_cache_counts(self.handle)
+
+    def row_counts(self, row: int):
+        nc, nh, rp = c_int64(), c_int32(), c_int32()
+        _check(lib().tq_cache_row_counts(self.handle, row, ctypes.byref(nc), ctypes.byref(nh),
+                                         ctypes.byref(rp)), "tq_cache_row_counts")
+        return nc.value, nh.value, rp.value
+
+    def encode_append_rows(self, k, v, n_rows, stream=None):
+        """Row b appends its first n_rows[b] tokens of k, v [B, Hkv, n_max, d]."""
+        rows = np.ascontiguousarray(np.asarray(n_rows, dtype=np.int32))
+        _check(lib().tq_encode_append_rows(self.handle, self._dev16(k), self._dev16(v), k.shape[2],
+                                           rows.ctypes.data, _stream_handle(stream)),
+               "tq_encode_append_rows")
+
+    def evict_window_rows(self, k_new, v_new, n_rows, stream=None):
+        """Row b inserts its first n_rows[b] tokens of k_new, v_new [B, Hkv, n_max, d]."""
+        rows = np.ascontiguousarray(np.asarray(n_rows, dtype=np.int32))
+        _check(lib().tq_evict_window_rows(self.handle, self._dev16(k_new), self._dev16(v_new),
+                                          k_new.shape[2], rows.ctypes.data, _stream_handle(stream)),
+               "tq_evict_window_rows")
 
     def hot_ring(self):
         """Views of the fp16 hot rings K, V: [B, Hkv, W, d] (slot order)."""

@@ -119,9 +119,14 @@ tq_status tq_cache_create(const tq_config* cfg, void* hot_mem, void* cold_mem,
 /* Free the host handle (device buffers stay the caller's). NULL is a no-op. */
 tq_status tq_cache_destroy(tq_cache* cache);
 
-/* Host-side counters: compressed tokens, valid hot tokens, next ring slot. */
+/* Host-side counters: compressed tokens, valid hot tokens, next ring slot.
+ * For a ragged batch (rows with different counts): the largest n_cold and
+ * n_hot over the rows and row 0's ring slot; tq_cache_row_counts gives
+ * each row's own. */
 tq_status tq_cache_counts(const tq_cache* cache, int64_t* n_cold,
                           int32_t* n_hot, int32_t* ring_pos);
+tq_status tq_cache_row_counts(const tq_cache* cache, int32_t row, int64_t* n_cold,
+                              int32_t* n_hot, int32_t* ring_pos);
 
 /*
  * Compress n new tokens straight into the cold store (prefill path).
@@ -154,6 +159,30 @@ tq_status tq_encode_append(tq_cache* cache, const void* k, const void* v,
  */
 tq_status tq_evict_window(tq_cache* cache, const void* k_new,
                           const void* v_new, int32_t n, cudaStream_t stream);
+
+/*
+ * Per-row lengths (ragged batches): the rows of a batch -- sequences of
+ * different lengths -- append and insert different numbers of tokens, and
+ * every later call attends each row's own tokens (the per-row lengths of
+ * the "TurboQuant: kompresja KV-cache ..." page's format; no row is padded
+ * in the cold store).
+ *   k, v / k_new, v_new  device fp16 [B, Hkv, n_max, d]; row b's first
+ *               n_rows[b] tokens are used (0 <= n_rows[b] <= n_max)
+ *   n_rows      HOST int32 [B]
+ * tq_encode_append_rows appends row b's tokens at its own cold count;
+ * tq_evict_window_rows inserts them into its own ring (a full ring evicts
+ * its oldest tokens into the row's cold store, as tq_evict_window).
+ * TQ_ERR_CAPACITY (nothing launched) if a row would exceed cold_capacity.
+ * While the rows' counts differ, the batch may have at most 128 rows
+ * (TQ_ERR_UNSUPPORTED otherwise), and the threshold-gated decode, the
+ * Tensor Cache tier and promotion are unavailable (TQ_ERR_UNSUPPORTED);
+ * tq_encode_append / tq_evict_window then act as the _rows calls with the
+ * same n for every row.  Uniform inputs take the uniform paths.
+ */
+tq_status tq_encode_append_rows(tq_cache* cache, const void* k, const void* v, int64_t n_max,
+                                const int32_t* n_rows, cudaStream_t stream);
+tq_status tq_evict_window_rows(tq_cache* cache, const void* k_new, const void* v_new,
+                               int32_t n_max, const int32_t* n_rows, cudaStream_t stream);
 
 /*
  * Single-token decode attention over hot U cold tokens.
