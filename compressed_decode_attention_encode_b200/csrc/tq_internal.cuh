@@ -444,8 +444,8 @@ struct VecEncodeArgs {
   const float* St;          // [d, m]
   double inv_sqrt_d;
   int* status;
-  uint8_t* codes;           // [n][d/2]
-  uint8_t* signs_out;       // [n][32]
+  uint8_t* codes;           // [n/32][d/32][32][16 B]: 32-vector groups, 16-byte chunks
+  uint8_t* signs_out;       // [n/32][2][32][16 B]
   uint16_t* s16_out;        // [n]
   uint16_t* rn16_out;       // [n]
 };
@@ -455,7 +455,9 @@ struct VecQPrepArgs {
   int nq, dim, d, m;
   const double* signs;
   const float* St;
-  __half* A;                // [nq, d + 256] fp16 MMA operand
+  int kq;                   // QJL k-steps of 16 (search_qjl_steps)
+  int half_last;            // the last QJL k-step takes the high half of its word only
+  __half* A;                // query tiles of 128 rows, UMMA core-matrix order
   float* qscale;            // [nq]
 };
 
@@ -467,10 +469,13 @@ struct SearchArgs {
   const uint16_t* rn16;
   int64_t n;
   int nq, d, b_theta, nsplit;
+  int kq, half_last;        // as in VecQPrepArgs
   float inv_levels;         // 1 / (2^b_r - 1)
   float qjl_const;          // sqrt(pi/2) / m
-  float* part_s;            // [nq][nsplit][2][16]
+  float* part_s;            // [nq][nsplit][16]
   int* part_i;
+  int* status;              // latched kStatusTimeout
+  unsigned long long wait_limit_ns;
 };
 
 struct MergeArgs {

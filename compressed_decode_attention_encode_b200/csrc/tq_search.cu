@@ -4,19 +4,23 @@
 // database for vector search / RAG).
 //
 //   vec_encode_kernel   float32 vectors -> codes, one warp per vector; the
-//                       float64 decision path of the KV encoder.
+//                       float64 decision path of the KV encoder.  Records
+//                       are stored in groups of 32 vectors, 16-byte chunks
+//                       chunk-major, so that a warp reading one chunk of 32
+//                       vectors reads 512 contiguous bytes.
 //   vec_qprep_kernel    q' = R q, q'' = S q' written as the fp16 A operand of
-//                       the search MMAs, in the fragments' column order.
-//   search_kernel       per CTA (8 warps): 64 queries x a contiguous run of
-//                       database vectors.  The database side is dequantized
-//                       straight into mma.sync B fragments (one shared LUT
-//                       load per polar pair, scaled by the vector's
-//                       s16/(2^b_r-1); sign bits become +-rn16*sqrt(pi/2)/m
-//                       with one LOP3), so each looked-up register feeds 4
-//                       MMAs.  Each thread compares its accumulators with
-//                       its queries' current k-th best and appends only
-//                       better candidates to a per-query buffer, which a
-//                       warp re-selects when it could overflow.
+//                       the search MMAs: tiles of 128 queries in the tensor
+//                       cores' K-major core-matrix order.
+//   search_umma_kernel  per CTA: 128 queries (A, resident in shared memory)
+//                       against a contiguous run of the database, 256
+//                       vectors per round.  Eight producer warps dequantize
+//                       the round's vectors straight into the B operand
+//                       (fp16 c_r (cos, sin) from a shared LUT times
+//                       s16/(2^b_r-1); QJL signs as +-rn16 sqrt(pi/2)/m);
+//                       one thread issues tcgen05.mma (M 128, N 256, K 16)
+//                       into one of two fp32 accumulators in tensor memory;
+//                       four epilogue warps read the scores back (thread =
+//                       query) and keep each query's 16 best.
 //   topk_merge_kernel   merges the per-split candidate lists.
 #include <cmath>
 #include <cstring>
@@ -30,24 +34,50 @@ namespace {
 
 using enc::encode_vector_any;
 using enc::kFull;
-constexpr int kQT = 64;                  // queries per CTA
 constexpr int kListK = 16;               // best candidates kept per (query, split); k <= kListK
 constexpr int kMaxSplits = 32;           // database splits per search (grid y)
 constexpr float kNegInf = -INFINITY;
 
-__device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                         uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%0,%1,%2,%3};\n"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
+// Search tile shape (tcgen05, one CTA per SM).
+constexpr int kM = 128;                  // queries per CTA = MMA M = tensor-memory lanes
+constexpr int kN = 256;                  // database vectors per round = MMA N
+constexpr int kKStg = 2;                 // k-steps (16 k each) per B stage
+constexpr int kNB = 3;                   // B stages in the ring
+constexpr int kQ = 16;                   // candidate queue entries per query
+constexpr int kEpiWarps = 4;             // warps 0-3: tensor-memory lane quarters 0-3
+constexpr int kProdWarps = 8;            // warps 4-11: one database vector per thread per round
+constexpr int kMmaWarp = kEpiWarps + kProdWarps;
+constexpr int kSearchThreads = (kMmaWarp + 1) * 32;
+constexpr int kKStepB = kN * 32;         // bytes of one B k-step (256 rows x 16 fp16)
+constexpr int kStageBytes = kKStg * kKStepB;
+constexpr int kKStepA = kM * 32;         // bytes of one A k-step
+constexpr uint32_t kTmemCols = 2 * kN;   // two fp32 accumulators
+// Instruction descriptor of tcgen05.mma kind::f16: fp32 accumulator (bits
+// 4-5 = 1), fp16 A and B (bits 7-12 = 0), both K-major (bits 15-16 = 0),
+// N >> 3 at bit 17, M >> 4 at bit 24.
+constexpr uint32_t kIdesc = (1u << 4) | ((uint32_t)(kN >> 3) << 17) | ((uint32_t)(kM >> 4) << 24);
 
-__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
+// Dynamic shared memory of the search kernel.
+struct SearchSmem {
+  static constexpr int LUT = 0;                              // 256 entries x 32 lane copies x 4 B
+  static constexpr int B = LUT + 256 * 32 * 4;               // kNB stages
+  static constexpr int QUEUE = B + kNB * kStageBytes;        // [kQ][kM] (score, index)
+  static constexpr int BAR = QUEUE + kQ * kM * 8;            // full[kNB], empty[kNB], acc_full[2], acc_empty[2], done
+  static constexpr int TMEM_SLOT = BAR + 8 * (2 * kNB + 5);
+  static constexpr int ABORT = TMEM_SLOT + 4;
+  static constexpr int A = (ABORT + 4 + 127) / 128 * 128;    // ks A k-steps
+  static size_t bytes(int ks) { return (size_t)A + (size_t)ks * kKStepA; }
+};
+
+// QJL k-steps of the search operands for m sign bits.  Sign word w (bits
+// 32w..32w+31) fills two k-steps: k-step half h, chunk kc, half2 u holds
+// bits 15-u' (low half) and 31-u' (high half) of the word, u' = 8h + 4kc + u,
+// so one shift and one logic op turn a sign word into a B register.  When
+// the last word holds only 8 needed bits (m % 32 == 8), they are bits 0-7,
+// all in the low halves of h = 1, and h = 0 is skipped.
+__host__ __device__ inline int search_qjl_steps(int m) {
+  const int r = m % 32;
+  return 2 * (m / 32) + (r == 0 ? 0 : (r == 8 ? 1 : 2));
 }
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
@@ -62,6 +92,190 @@ __device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
 // (score, index) order of the result: higher score first, then lower index.
 __device__ __forceinline__ bool better(float s, int i, float t, int j) {
   return s > t || (s == t && i < j);
+}
+
+// ---- shared memory, barriers, tensor memory ---------------------------------
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ float2 lds64f(uint32_t addr) {
+  float2 v;
+  asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void sts64f(uint32_t addr, float x, float y) {
+  asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(x), "f"(y) : "memory");
+}
+
+__device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+               : "memory");
+}
+
+__device__ __forceinline__ uint4 ldg_stream(const uint4* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Waits for phase `parity` of an mbarrier.  Gives up when another role has
+// raised the CTA's abort flag, or after `limit_ns` (then raises it and
+// latches kStatusTimeout).
+__device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, unsigned long long limit_ns,
+                                              volatile int* abort_flag, int* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*abort_flag) return false;
+    if (global_ns() - t0 > limit_ns) {
+      *abort_flag = 1;
+      atomicOr(status, kStatusTimeout);
+      return false;
+    }
+  }
+  return true;
+}
+
+// One lane waits, the warp learns the outcome.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, unsigned long long limit_ns,
+                                          volatile int* abort_flag, int* status) {
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0) ok = wait_or_abort(bar, parity, limit_ns, abort_flag, status) ? 1 : 0;
+  return __shfl_sync(kFull, ok, 0) != 0;
+}
+
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// K-major, no-swizzle shared-memory matrix descriptor: core matrices of 8
+// rows x 16 bytes; the two 8-element K halves of a k-step 128 bytes apart
+// (leading byte offset), 8-row groups 256 bytes apart (stride byte offset);
+// descriptor version 1 at bit 46.
+__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3fffu) | ((uint64_t)(128 >> 4) << 16) | ((uint64_t)(256 >> 4) << 32) |
+         (1ull << 46);
+}
+
+__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// The mbarrier's arrival once every tcgen05.mma this thread issued so far
+// has completed.
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc(uint32_t slot_saddr, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot_saddr),
+               "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// 32 consecutive fp32 columns of this thread's tensor-memory lane.  The
+// wait names the registers so that no use of them moves above it.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+      "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+        "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+        "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+                 "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+                 "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]),
+                 "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]),
+                 "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+               :
+               : "memory");
+}
+
+// ---- the per-query best list -------------------------------------------------
+// Inserts (s, v) into a list sorted by (score desc, index asc) whose
+// indices are all below v: v goes after every entry scoring >= s.
+template <int K>
+__device__ __forceinline__ void list_insert(float (&ts)[K], int (&ti)[K], float s, int v) {
+  bool pc = false;
+  float ps = 0.f;
+  int pi = 0;
+#pragma unroll
+  for (int j = 0; j < K; ++j) {
+    const bool c = s > ts[j];
+    const float os = ts[j];
+    const int oi = ti[j];
+    ts[j] = pc ? ps : (c ? s : os);
+    ti[j] = pc ? pi : (c ? v : oi);
+    pc = c;
+    ps = os;
+    pi = oi;
+  }
+}
+
+// r[j] for a run-time j in [0, 8).
+__device__ __forceinline__ uint32_t select8(const uint32_t* r, int j) {
+  const uint32_t a0 = (j & 1) ? r[1] : r[0], a1 = (j & 1) ? r[3] : r[2];
+  const uint32_t a2 = (j & 1) ? r[5] : r[4], a3 = (j & 1) ? r[7] : r[6];
+  const uint32_t b0 = (j & 2) ? a1 : a0, b1 = (j & 2) ? a3 : a2;
+  return (j & 4) ? b1 : b0;
 }
 
 // ---------------------------------------------------------------------------
@@ -90,10 +304,16 @@ __global__ void __launch_bounds__(256) vec_encode_kernel(const VecEncodeArgs a) 
     encode_vector_any<D>(a.L, a.signs, a.St, a.inv_sqrt_d, a.status, load, true, rbuf, codes, bits,
                          sc, sc + 1);
     const int64_t g = a.start + v;
-    uint8_t* dst = a.codes + g * P;
+    // group g / 32, chunk-major: byte b of vector g at chunk b / 16
+    uint8_t* grp = a.codes + (g >> 5) * (32 * P) + (g & 31) * 16;
 #pragma unroll
-    for (int k = 0; k < PL; ++k) dst[lane * PL + k] = codes[lane * PL + k];
-    if (lane < 8) reinterpret_cast<uint32_t*>(a.signs_out + g * 32)[lane] = bits[lane];
+    for (int k = 0; k < PL; ++k) {
+      const int b = lane * PL + k;
+      grp[(b >> 4) * 512 + (b & 15)] = codes[b];
+    }
+    if (lane < 8)
+      *reinterpret_cast<uint32_t*>(a.signs_out + (g >> 5) * 1024 + (lane >> 2) * 512 + (g & 31) * 16 +
+                                   (lane & 3) * 4) = bits[lane];
     if (lane == 0) {
       a.s16_out[g] = sc[0];
       a.rn16_out[g] = sc[1];
@@ -103,22 +323,22 @@ __global__ void __launch_bounds__(256) vec_encode_kernel(const VecEncodeArgs a) 
 }
 
 // ---------------------------------------------------------------------------
-// query prep: one warp per query
+// query prep: one warp per query row of the 128-row tiles (rows past nq are
+// written as zeros)
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(256) vec_qprep_kernel(const VecQPrepArgs a) {
-  constexpr int E = D / 32, P = D / 2, PT = P / 4;
-  constexpr int KA = D + 256;
+  constexpr int E = D / 32;
   __shared__ float sq[8][D];
   __shared__ float sqq[8][256];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int q = blockIdx.x * 8 + warp;
-  if (q >= a.nq) return;
+  const bool live = q < a.nq;
   float x[E];
 #pragma unroll
   for (int i = 0; i < E; ++i) {
     const int j = lane * E + i;
-    x[i] = j < a.dim ? a.q[(size_t)q * a.dim + j] * (float)a.signs[j] : 0.f;
+    x[i] = (live && j < a.dim) ? a.q[(size_t)q * a.dim + j] * (float)a.signs[j] : 0.f;
   }
 #pragma unroll
   for (int hh = 1; hh < D; hh <<= 1) {
@@ -150,7 +370,7 @@ __global__ void __launch_bounds__(256) vec_qprep_kernel(const VecQPrepArgs a) {
   __syncwarp();
   for (int i = lane; i < 256; i += 32) {
     float acc = 0.f;
-    if (i < a.m)
+    if (live && i < a.m)
       for (int j = 0; j < D; ++j) acc = fmaf(__ldg(a.St + (size_t)j * a.m + i), sq[warp][j], acc);
     sqq[warp][i] = acc;
     amax = fmaxf(amax, fabsf(acc));
@@ -159,118 +379,59 @@ __global__ void __launch_bounds__(256) vec_qprep_kernel(const VecQPrepArgs a) {
   for (int o = 16; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, o));
   const float al = amax > 0.f ? exp2f(-floorf(log2f(amax))) : 1.f;
   __syncwarp();
-  __half* row = a.A + (size_t)q * KA;
-  // polar columns: k-step s, column w of 16: pair PT*tig + 2s + (w >= 8)
-  for (int c = lane; c < D; c += 32) {
-    const int s = c / 16, w = c % 16;
-    const int tig = (w % 8) / 2, e = w % 2;
-    const int pair = PT * tig + 2 * s + (w >= 8 ? 1 : 0);
-    row[c] = __float2half_rn(sq[warp][2 * pair + e] * al);
+  // element (row r, k) of the tile: k-step k/16 (kKStepA bytes), 8-row group
+  // r/8 (256 B), K half (k/8)%2 (128 B), row r%8 (16 B), k%8
+  const int ks = D / 16 + a.kq;
+  __half* tile = a.A + (size_t)(q / kM) * ks * (kKStepA / 2);
+  const int r = q % kM;
+  auto put = [&](int k, float v) {
+    tile[(k >> 4) * (kKStepA / 2) + (r >> 3) * 128 + ((k >> 3) & 1) * 64 + (r & 7) * 8 + (k & 7)] =
+        __float2half_rn(v);
+  };
+  for (int k = lane; k < D; k += 32) put(k, sq[warp][k] * al);
+  for (int c = lane; c < a.kq * 16; c += 32) {
+    const int t = c >> 4, kc = (c >> 3) & 1, u = (c >> 1) & 3, e = c & 1;
+    const int h = (t == a.kq - 1 && a.half_last) ? 1 : (t & 1);
+    const int up = 8 * h + 4 * kc + u;
+    const int bit = 32 * (t >> 1) + (e ? 31 - up : 15 - up);
+    put(D + c, bit < a.m ? sqq[warp][bit] * al : 0.f);
   }
-  // QJL columns: sign word 2 tig + s/8, half2 slot u = 2 (s % 8) + (w >= 8)
-  for (int c = lane; c < 256; c += 32) {
-    const int s = c / 16, w = c % 16;
-    const int tig = (w % 8) / 2, e = w % 2, r = w >= 8 ? 1 : 0;
-    const int word = 2 * tig + s / 8, u = 2 * (s % 8) + r;
-    const int idx = 32 * word + (e ? 31 - u : 15 - u);
-    row[D + c] = __float2half_rn(idx < a.m ? sqq[warp][idx] * al : 0.f);
-  }
-  if (lane == 0) a.qscale[q] = 1.f / al;
+  if (live && lane == 0) a.qscale[q] = 1.f / al;
 }
 
 // ---------------------------------------------------------------------------
 // search
 // ---------------------------------------------------------------------------
-// Per CTA: kQT = 64 queries (4 MMA m-tiles, A operand in shared memory)
-// against a contiguous run of the database, kStepVec = 128 vectors per step
-// (8 warps x 2 n-tiles of 8).  Scores never go to shared memory: each
-// thread compares its accumulators with the query's current k-th best
-// (`thr`) and appends only better candidates to the query's buffer; a warp
-// re-selects a query's k best whenever its buffer could overflow in the
-// next step.
+// Rounds of kN database vectors; each round's k-steps (D/16 polar, then kq
+// QJL) pass through a ring of kNB B stages of kKStg k-steps:
+//   producers  --full[slot]-->  MMA thread  --empty[slot] (commit)-->  producers
+//   MMA thread --acc_full[b] (commit)--> epilogue --acc_empty[b]--> MMA thread
+// Every wait is bounded; a timeout raises the CTA's abort flag, which ends
+// every role's loop, and the kernel still waits for its issued MMAs and
+// frees its tensor memory before it returns.
 template <int D>
-struct SearchShape {
-  static constexpr int P = D / 2;
-  static constexpr int PT = P / 4;            // code bytes per lane per vector
-  static constexpr int KS_POL = D / 16;       // polar k-steps
-  static constexpr int KS_QJL = 16;           // QJL k-steps (256 sign slots)
-  static constexpr int KA = D + 256;
-  static constexpr int AS = KA + 8;           // padded A row (halves)
-  static constexpr int WARPS = 8;
-  static constexpr int NJ = 2;                // n-tiles per warp per step
-  static constexpr int STEP = WARPS * NJ * 8; // vectors per step
-  static constexpr int CAP = kListK + STEP + 32;   // candidate slots per query
-  static constexpr int OFF_CAND = kQT * AS * 2;
-  static constexpr int OFF_CNT = OFF_CAND + kQT * CAP * 8;
-  static constexpr int OFF_THR = OFF_CNT + kQT * 4;
-  static constexpr int SMEM = OFF_THR + kQT * 4;
-};
-
-// Warp: replaces query q's candidates (n of them, (score, index) pairs) by
-// its best min(n, K), in order, and returns the new count; *thr becomes the
-// K-th best score (-inf while fewer than K are known).
-template <int CAP, int K>
-__device__ int select_top(float2* cand, int n, float* thr) {
-  constexpr int PER = (CAP + 31) / 32;
-  const int lane = threadIdx.x & 31;
-  float sv[PER];
-  int iv[PER];
-#pragma unroll
-  for (int r = 0; r < PER; ++r) {
-    const int e = r * 32 + lane;
-    const float2 c = e < n ? cand[e] : make_float2(kNegInf, 0.f);
-    sv[r] = c.x;
-    iv[r] = e < n ? __float_as_int(c.y) : 0x7fffffff;
-  }
-  __syncwarp();
-  const int keep = n < K ? n : K;
-  for (int k = 0; k < keep; ++k) {
-    // this lane's best, then the warp's (score desc, index asc)
-    float bs = sv[0];
-    int bi = iv[0], br = 0;
-#pragma unroll
-    for (int r = 1; r < PER; ++r)
-      if (better(sv[r], iv[r], bs, bi)) { bs = sv[r]; bi = iv[r]; br = r; }
-    float ws = bs;
-    int wi = bi;
-#pragma unroll
-    for (int o = 16; o; o >>= 1) {
-      const float os = __shfl_xor_sync(kFull, ws, o);
-      const int oi = __shfl_xor_sync(kFull, wi, o);
-      if (better(os, oi, ws, wi)) { ws = os; wi = oi; }
-    }
-    if (bs == ws && bi == wi) {          // the owner drops it from its registers
-#pragma unroll
-      for (int r = 0; r < PER; ++r)
-        if (r == br) { sv[r] = kNegInf; iv[r] = 0x7fffffff; }
-    }
-    if (lane == 0) cand[k] = make_float2(ws, __int_as_float(wi));
-  }
-  __syncwarp();
-  if (lane == 0) *thr = keep == K ? cand[K - 1].x : kNegInf;
-  __syncwarp();
-  return keep;
-}
-
-template <int D, int K>
-__global__ void __launch_bounds__(256, 1) search_kernel(const SearchArgs a) {
-  using S = SearchShape<D>;
-  extern __shared__ __align__(16) uint8_t smem[];
-  __shared__ __align__(16) uint32_t lut[256 * 32];
-  __half* As = reinterpret_cast<__half*>(smem);
-  float2* cand = reinterpret_cast<float2*>(smem + S::OFF_CAND);
-  int* cnt = reinterpret_cast<int*>(smem + S::OFF_CNT);
-  float* thr = reinterpret_cast<float*>(smem + S::OFF_THR);
-
+__global__ void __launch_bounds__(kSearchThreads, 1) search_umma_kernel(const SearchArgs a) {
+  using U = SearchSmem;
+  constexpr int KP = D / 16;      // polar k-steps
+  constexpr int CW = D / 8;       // code words per vector (one byte per pair)
+  extern __shared__ __align__(1024) uint8_t smem[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int gid = lane >> 2, tig = lane & 3;
-  const int q0 = blockIdx.x * kQT;
-  const int nq_tile = a.nq - q0 < kQT ? a.nq - q0 : kQT;
-  const int64_t per = (a.n + gridDim.y - 1) / gridDim.y;
-  const int64_t v_lo = (int64_t)blockIdx.y * per;
-  const int64_t v_hi = v_lo + per < a.n ? v_lo + per : a.n;
+  const int ks = KP + a.kq;
+  const uint32_t sbase = smem_addr(smem);
+  const uint32_t lut_s = sbase + U::LUT, b_s = sbase + U::B, a_s = sbase + U::A;
+  const uint32_t bar_full = sbase + U::BAR, bar_empty = bar_full + 8 * kNB;
+  const uint32_t bar_accf = bar_empty + 8 * kNB, bar_acce = bar_accf + 16, bar_done = bar_acce + 16;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + U::ABORT);
+
+  // this CTA's run: rounds [r0, r1) of the database
+  const int64_t rounds = (a.n + kN - 1) / kN;
+  const int64_t r0 = rounds * blockIdx.y / gridDim.y, r1 = rounds * (blockIdx.y + 1) / gridDim.y;
+  const int nr = (int)(r1 - r0);
+  const int64_t v_lo = r0 * kN;
+  const int64_t v_hi = r1 * kN < a.n ? r1 * kN : a.n;
 
   // LUT of c_r * (cos, sin)(2 pi c_th / 2^b_th), one copy per lane
+  uint32_t* lut = reinterpret_cast<uint32_t*>(smem + U::LUT);
   for (int e = tid; e < 256 * 32; e += blockDim.x) {
     const int w = e >> 5;
     const int cr = w >> a.b_theta, ct = w & ((1 << a.b_theta) - 1);
@@ -279,134 +440,245 @@ __global__ void __launch_bounds__(256, 1) search_kernel(const SearchArgs a) {
     const __half2 h = __floats2half2_rn((float)cr * cs, (float)cr * sn);
     lut[e] = *reinterpret_cast<const uint32_t*>(&h);
   }
-  // A tile: the CTA's queries (rows past nq are zero)
-  for (int i = tid; i < kQT * (S::KA / 8); i += blockDim.x) {
-    const int r = i / (S::KA / 8), cc = i % (S::KA / 8);
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (r < nq_tile) v = *reinterpret_cast<const uint4*>(a.A + (size_t)(q0 + r) * S::KA + cc * 8);
-    *reinterpret_cast<uint4*>(As + r * S::AS + cc * 8) = v;
+  // A: this CTA's query tile, already in core-matrix order
+  {
+    const uint4* src = reinterpret_cast<const uint4*>(a.A) + (size_t)blockIdx.x * ks * (kKStepA / 16);
+    uint4* dst = reinterpret_cast<uint4*>(smem + U::A);
+    for (int i = tid; i < ks * (kKStepA / 16); i += blockDim.x) dst[i] = src[i];
   }
-  for (int q = tid; q < kQT; q += blockDim.x) {
-    cnt[q] = 0;
-    thr[q] = kNegInf;
+  fence_proxy_async();            // the tensor cores read A through the async proxy
+  if (tid == 0) {
+    for (int i = 0; i < kNB; ++i) {
+      mbar_init(bar_full + 8 * i, kProdWarps);
+      mbar_init(bar_empty + 8 * i, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar_accf + 8 * i, 1);
+      mbar_init(bar_acce + 8 * i, kEpiWarps);
+    }
+    mbar_init(bar_done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
   }
+  if (warp == kMmaWarp) tmem_alloc(sbase + U::TMEM_SLOT, kTmemCols);
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + U::TMEM_SLOT);
 
-  const uint32_t a_base = smem_addr(As);
-  const int mi = lane >> 3, rr = lane & 7;
-  const uint32_t lane4 = (uint32_t)lane * 4u;
-  const char* lutb = reinterpret_cast<const char*>(lut);
-
-  for (int64_t c0 = v_lo; c0 < v_hi; c0 += S::STEP) {
-    // ---- B operand data for this warp's n-tiles (8 vectors each) --------
-    uint32_t cw[S::NJ][S::PT / 4];
-    uint32_t sg[S::NJ][2];
-    uint32_t sa[S::NJ], sb[S::NJ];
+  if (warp < kEpiWarps) {
+    // ---------------- epilogue: thread = query row 32 warp + lane ----------
+    const int qr = 32 * warp + lane;
+    float ts[kListK];
+    int ti[kListK];
 #pragma unroll
-    for (int j = 0; j < S::NJ; ++j) {
-      const int64_t v = c0 + warp * (8 * S::NJ) + j * 8 + gid;
-      if (v < v_hi) {
-        const uint32_t* cp = reinterpret_cast<const uint32_t*>(a.codes + v * S::P + S::PT * tig);
-#pragma unroll
-        for (int k = 0; k < S::PT / 4; ++k) cw[j][k] = __ldg(cp + k);
-        const uint2 s2 = __ldg(reinterpret_cast<const uint2*>(a.signs + v * 32 + 8 * tig));
-        sg[j][0] = s2.x;
-        sg[j][1] = s2.y;
-        const float s16 = __half2float(__ushort_as_half(__ldg(a.s16 + v)));
-        const float rn = __half2float(__ushort_as_half(__ldg(a.rn16 + v)));
-        const __half ah = __float2half_rn(s16 * a.inv_levels);
-        const __half bh = __float2half_rn(rn * a.qjl_const);
-        const uint32_t au = __half_as_ushort(ah), bu = __half_as_ushort(bh);
-        sa[j] = au | (au << 16);
-        sb[j] = (bu | (bu << 16)) | 0x80008000u;
-      } else {
-#pragma unroll
-        for (int k = 0; k < S::PT / 4; ++k) cw[j][k] = 0u;
-        sg[j][0] = sg[j][1] = 0u;
-        sa[j] = 0u;
-        sb[j] = 0u;        // +-0: vectors past the run score 0 (not appended below)
-      }
+    for (int j = 0; j < kListK; ++j) {
+      ts[j] = kNegInf;
+      ti[j] = 0x7fffffff;
     }
-    float acc[4][S::NJ][4];
-#pragma unroll
-    for (int m = 0; m < 4; ++m)
-#pragma unroll
-      for (int j = 0; j < S::NJ; ++j) acc[m][j][0] = acc[m][j][1] = acc[m][j][2] = acc[m][j][3] = 0.f;
-
-    // ---- polar part ----------------------------------------------------
-#pragma unroll
-    for (int s = 0; s < S::KS_POL; ++s) {
-      uint32_t af[4][4];
-#pragma unroll
-      for (int m = 0; m < 4; ++m)
-        ldsm_x4(af[m], a_base + ((16 * m + rr + (mi & 1) * 8) * S::AS + 16 * s + (mi >> 1) * 8) * 2);
-#pragma unroll
-      for (int j = 0; j < S::NJ; ++j) {
-        const uint32_t w = cw[j][(2 * s) / 4];
-        const uint32_t c0b = (w >> (8 * ((2 * s) % 4))) & 0xffu;
-        const uint32_t c1b = (w >> (8 * ((2 * s + 1) % 4))) & 0xffu;
-        const uint32_t b0 = hmul2_u32(*reinterpret_cast<const uint32_t*>(lutb + (c0b * 128u + lane4)), sa[j]);
-        const uint32_t b1 = hmul2_u32(*reinterpret_cast<const uint32_t*>(lutb + (c1b * 128u + lane4)), sa[j]);
-#pragma unroll
-        for (int m = 0; m < 4; ++m) mma16816(acc[m][j], af[m][0], af[m][1], af[m][2], af[m][3], b0, b1);
+    float thr = kNegInf;
+    int cnt = 0;
+    const uint32_t qbase = sbase + U::QUEUE + qr * 8;     // entry i at + i * kM * 8
+    auto flush = [&]() {
+      const int mx = __reduce_max_sync(kFull, cnt);
+      for (int i = 0; i < mx; ++i) {
+        if (i < cnt) {
+          const float2 c = lds64f(qbase + i * (kM * 8));
+          list_insert<kListK>(ts, ti, c.x, __float_as_int(c.y));
+        }
       }
-    }
-    // ---- QJL part: +-b from the sign bits -------------------------------
+      cnt = 0;
+      thr = ts[kListK - 1];
+    };
+    for (int r = 0; r < nr; ++r) {
+      const int ab = r & 1;
+      if (!warp_wait(bar_accf + 8 * ab, (uint32_t)((r >> 1) & 1), a.wait_limit_ns, abort_flag, a.status))
+        break;
+      tc_fence_after();
+      const int64_t vr = v_lo + (int64_t)r * kN;
+      const int valid = (int)(v_hi - vr < kN ? v_hi - vr : kN);
+      const uint32_t taddr = tmem + ((uint32_t)(32 * warp) << 16) + (uint32_t)(ab * kN);
+#pragma unroll 1
+      for (int c = 0; c < kN / 32; ++c) {
+        uint32_t sv[32];
+        tmem_ld32(taddr + 32 * c, sv);
 #pragma unroll
-    for (int s = 0; s < S::KS_QJL; ++s) {
-      uint32_t af[4][4];
+        for (int t = 0; t < 4; ++t) {
+          const int col = 32 * c + 8 * t;
+          uint32_t m = 0;
 #pragma unroll
-      for (int m = 0; m < 4; ++m)
-        ldsm_x4(af[m], a_base + ((16 * m + rr + (mi & 1) * 8) * S::AS + D + 16 * s + (mi >> 1) * 8) * 2);
-      const int u = 2 * (s % 8);
-#pragma unroll
-      for (int j = 0; j < S::NJ; ++j) {
-        const uint32_t x = sg[j][s / 8];
-        const uint32_t b0 = ((x << u) & 0x80008000u) ^ sb[j];
-        const uint32_t b1 = ((x << (u + 1)) & 0x80008000u) ^ sb[j];
-#pragma unroll
-        for (int m = 0; m < 4; ++m) mma16816(acc[m][j], af[m][0], af[m][1], af[m][2], af[m][3], b0, b1);
-      }
-    }
-    // ---- candidates: scores at least the query's current k-th best -------
-#pragma unroll
-    for (int m = 0; m < 4; ++m) {
-#pragma unroll
-      for (int r2 = 0; r2 < 2; ++r2) {
-        const int q = 16 * m + gid + 8 * r2;
-        if (q >= nq_tile) continue;
-        const float t = thr[q];
-#pragma unroll
-        for (int j = 0; j < S::NJ; ++j) {
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            const int64_t v = c0 + warp * (8 * S::NJ) + j * 8 + 2 * tig + c;
-            const float sc = acc[m][j][2 * r2 + c];
-            if (v < v_hi && sc >= t) {
-              const int pos = atomicAdd(&cnt[q], 1);
-              cand[q * S::CAP + pos] = make_float2(sc, __int_as_float((int)v));
+          for (int u = 0; u < 8; ++u) m |= (__uint_as_float(sv[8 * t + u]) > thr ? 1u : 0u) << u;
+          const int nv = valid - col;
+          if (nv < 8) m &= nv <= 0 ? 0u : ((1u << nv) - 1u);
+          if (__any_sync(kFull, m != 0)) {
+            while (m) {
+              const int j = __ffs(m) - 1;
+              m &= m - 1;
+              sts64f(qbase + cnt * (kM * 8), __uint_as_float(select8(sv + 8 * t, j)),
+                     __int_as_float((int)(vr + col + j)));
+              ++cnt;
             }
+            if (__any_sync(kFull, cnt > kQ - 8)) flush();
           }
         }
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_acce + 8 * ab);
     }
-    __syncthreads();
-    // ---- re-select where the next step could overflow a buffer ----------
-    for (int q = warp; q < nq_tile; q += S::WARPS) {
-      const int n = cnt[q];
-      if (n > S::CAP - S::STEP) cnt[q] = select_top<S::CAP, K>(cand + q * S::CAP, n, thr + q);
+    flush();
+    const int q = blockIdx.x * kM + qr;
+    if (q < a.nq) {
+      const size_t base = ((size_t)q * gridDim.y + blockIdx.y) * kListK;
+#pragma unroll
+      for (int j = 0; j < kListK; ++j) {
+        a.part_s[base + j] = ts[j];
+        a.part_i[base + j] = ti[j];
+      }
     }
-    __syncthreads();
+  } else if (warp < kMmaWarp) {
+    // ---------------- producers: thread = vector n of each round -----------
+    const int pw = warp - kEpiWarps;
+    const int n = 32 * pw + lane;
+    const uint32_t row_off = (uint32_t)((n >> 3) * 256 + (n & 7) * 16);   // core-matrix row of vector n
+    const uint32_t lut_lane = lut_s + 4 * lane;
+    uint32_t cw[CW], sg[8], sa = 0, sb = 0;
+    uint32_t ncw[CW], nsg[8], nsa = 0, nsb = 0;
+    auto load = [&](int r, uint32_t (&w)[CW], uint32_t (&g)[8], uint32_t& xa, uint32_t& xb) {
+      const int64_t v = v_lo + (int64_t)r * kN + n;
+      if (r < nr && v < v_hi) {
+        const int64_t grp = v >> 5;                // lane == v % 32
+        const uint4* cp = reinterpret_cast<const uint4*>(a.codes + grp * (32 * (D / 2))) + lane;
+#pragma unroll
+        for (int c = 0; c < CW / 4; ++c) {
+          const uint4 t = ldg_stream(cp + 32 * c);
+          w[4 * c] = t.x;
+          w[4 * c + 1] = t.y;
+          w[4 * c + 2] = t.z;
+          w[4 * c + 3] = t.w;
+        }
+        const uint4* sp = reinterpret_cast<const uint4*>(a.signs + grp * 1024) + lane;
+        const uint4 s0 = ldg_stream(sp), s1 = ldg_stream(sp + 32);
+        g[0] = s0.x; g[1] = s0.y; g[2] = s0.z; g[3] = s0.w;
+        g[4] = s1.x; g[5] = s1.y; g[6] = s1.z; g[7] = s1.w;
+        const float s16 = __half2float(__ushort_as_half(__ldg(a.s16 + v)));
+        const float rn = __half2float(__ushort_as_half(__ldg(a.rn16 + v)));
+        const uint32_t au = __half_as_ushort(__float2half_rn(s16 * a.inv_levels));
+        const uint32_t bu = __half_as_ushort(__float2half_rn(rn * a.qjl_const));
+        xa = au | (au << 16);
+        xb = (bu | (bu << 16)) | 0x80008000u;     // -b; a set sign bit flips it to +b
+      } else {
+#pragma unroll
+        for (int c = 0; c < CW; ++c) w[c] = 0u;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) g[c] = 0u;
+        xa = 0u;
+        xb = 0u;                                   // columns past the run score 0 (masked later)
+      }
+    };
+    load(0, cw, sg, sa, sb);
+    uint32_t slot = 0, phase = 0;
+    auto acquire = [&]() {
+      return warp_wait(bar_empty + 8 * slot, phase ^ 1u, a.wait_limit_ns, abort_flag, a.status);
+    };
+    auto release = [&]() {
+      fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_full + 8 * slot);
+      if (++slot == kNB) {
+        slot = 0;
+        phase ^= 1u;
+      }
+    };
+    for (int r = 0; r < nr; ++r) {
+      load(r + 1, ncw, nsg, nsa, nsb);
+#pragma unroll
+      for (int s = 0; s < KP; ++s) {
+        const int j = s % kKStg;
+        if (j == 0 && !acquire()) goto producers_done;
+        const uint32_t dst = b_s + slot * kStageBytes + j * kKStepB + row_off;
+#pragma unroll
+        for (int kc = 0; kc < 2; ++kc) {
+          const uint32_t w = cw[2 * s + kc];
+          uint32_t h[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint32_t b = __byte_perm(w, 0u, 0x4440u + i);
+            h[i] = hmul2_u32(lds32(lut_lane + (b << 7)), sa);
+          }
+          sts128(dst + kc * 128, h[0], h[1], h[2], h[3]);
+        }
+        if (j == kKStg - 1) release();
+      }
+#pragma unroll
+      for (int t = 0; t < 16; ++t) {
+        if (t < a.kq) {
+          const int j = (KP + t) % kKStg;
+          if (j == 0 && !acquire()) goto producers_done;
+          const uint32_t dst = b_s + slot * kStageBytes + j * kKStepB + row_off;
+          const uint32_t x = sg[t >> 1];
+          const int h = (t == a.kq - 1 && a.half_last) ? 1 : (t & 1);
+#pragma unroll
+          for (int kc = 0; kc < 2; ++kc) {
+            const int u0 = 8 * h + 4 * kc;
+            sts128(dst + kc * 128, ((x << u0) & 0x80008000u) ^ sb, ((x << (u0 + 1)) & 0x80008000u) ^ sb,
+                   ((x << (u0 + 2)) & 0x80008000u) ^ sb, ((x << (u0 + 3)) & 0x80008000u) ^ sb);
+          }
+          if (j == kKStg - 1 || t == a.kq - 1) release();
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < CW; ++c) cw[c] = ncw[c];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) sg[c] = nsg[c];
+      sa = nsa;
+      sb = nsb;
+    }
+  producers_done:;
+  } else if (lane == 0) {
+    // ---------------- MMA issue (one thread) --------------------------------
+    uint32_t slot = 0, phase = 0;
+    for (int r = 0; r < nr; ++r) {
+      const int ab = r & 1;
+      if (!wait_or_abort(bar_acce + 8 * ab, (uint32_t)(((r >> 1) & 1) ^ 1), a.wait_limit_ns, abort_flag,
+                         a.status))
+        break;
+      tc_fence_after();
+      const uint32_t d_t = tmem + (uint32_t)(ab * kN);
+      bool ok = true;
+      for (int s = 0; s < ks; s += kKStg) {
+        if (!wait_or_abort(bar_full + 8 * slot, phase, a.wait_limit_ns, abort_flag, a.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const int nst = ks - s < kKStg ? ks - s : kKStg;
+        for (int j = 0; j < nst; ++j)
+          umma_f16(d_t, umma_desc(a_s + (s + j) * kKStepA), umma_desc(b_s + slot * kStageBytes + j * kKStepB),
+                   kIdesc, (s + j) > 0 ? 1u : 0u);
+        umma_commit(bar_empty + 8 * slot);
+        if (++slot == kNB) {
+          slot = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok) break;
+      umma_commit(bar_accf + 8 * ab);
+    }
+    // every issued MMA has finished before tensor memory is freed
+    umma_commit(bar_done);
+    const uint64_t t0 = global_ns();
+    while (!mbar_try_wait(bar_done, 0u))
+      if (global_ns() - t0 > a.wait_limit_ns) {
+        atomicOr(a.status, kStatusTimeout);
+        break;
+      }
   }
-  // ---- this CTA's list per query --------------------------------------------
-  for (int q = warp; q < nq_tile; q += S::WARPS) {
-    const int n = select_top<S::CAP, K>(cand + q * S::CAP, cnt[q], thr + q);
-    const size_t base = ((size_t)(q0 + q) * gridDim.y + blockIdx.y) * K;
-    for (int j = lane; j < K; j += 32) {
-      const float2 c = j < n ? cand[q * S::CAP + j] : make_float2(kNegInf, __int_as_float(0x7fffffff));
-      a.part_s[base + j] = c.x;
-      a.part_i[base + j] = __float_as_int(c.y);
-    }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
   }
 }
 
@@ -463,12 +735,12 @@ cudaError_t launch_vec_encode_d(const VecEncodeArgs& a, cudaStream_t s) {
 
 template <int D>
 cudaError_t launch_search_d(const SearchArgs& a, cudaStream_t s) {
-  using S = SearchShape<D>;
-  if (cudaFuncSetAttribute(search_kernel<D, kListK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           S::SMEM) != cudaSuccess)
+  const size_t smem = SearchSmem::bytes(D / 16 + a.kq);
+  if (cudaFuncSetAttribute(search_umma_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
     return cudaErrorInvalidValue;
-  dim3 grid((a.nq + kQT - 1) / kQT, a.nsplit);
-  search_kernel<D, kListK><<<grid, 32 * S::WARPS, S::SMEM, s>>>(a);
+  dim3 grid((a.nq + kM - 1) / kM, a.nsplit);
+  search_umma_kernel<D><<<grid, kSearchThreads, smem, s>>>(a);
   return cudaGetLastError();
 }
 
@@ -484,7 +756,7 @@ cudaError_t launch_vec_encode(const VecEncodeArgs& a, cudaStream_t s) {
 }
 
 cudaError_t launch_vec_qprep(const VecQPrepArgs& a, cudaStream_t s) {
-  const int grid = (a.nq + 7) / 8;
+  const int grid = (a.nq + kM - 1) / kM * (kM / 8);     // whole 128-row tiles
   switch (a.d) {
     case 64: vec_qprep_kernel<64><<<grid, 256, 0, s>>>(a); break;
     case 128: vec_qprep_kernel<128><<<grid, 256, 0, s>>>(a); break;
@@ -532,8 +804,9 @@ struct VecCodesLayout {
 VecCodesLayout vec_codes_layout(int d, int64_t n) {
   VecCodesLayout l{};
   size_t off = 0;
-  l.codes = off; off += vround((size_t)n * (d / 2));
-  l.signs = off; off += vround((size_t)n * 32);
+  const size_t groups = (size_t)((n + 31) / 32);            // whole groups of 32 vectors
+  l.codes = off; off += vround(groups * 32 * (d / 2));
+  l.signs = off; off += vround(groups * 32 * 32);
   l.s16 = off;   off += vround((size_t)n * 2);
   l.rn16 = off;  off += vround((size_t)n * 2);
   l.total = off;
@@ -550,7 +823,7 @@ VecWsLayout vec_ws_layout(int d, int m, int max_q) {
   w.status = off; off += kVAlign;
   w.signs = off;  off += vround(sizeof(double) * d);
   w.St = off;     off += vround(sizeof(float) * (size_t)d * m);
-  w.A = off;      off += vround((size_t)2 * max_q * (d + 256));
+  w.A = off;      off += vround((size_t)((max_q + kM - 1) / kM) * (d / 16 + search_qjl_steps(m)) * kKStepA);
   w.qscale = off; off += vround(sizeof(float) * max_q);
   w.part_s = off; off += vround(sizeof(float) * (size_t)max_q * kMaxSplits * kListK);
   w.part_i = off; off += vround(sizeof(int) * (size_t)max_q * kMaxSplits * kListK);
@@ -649,7 +922,8 @@ tq_status tq_vec_destroy(tq_vec_index* index) {
 
 tq_status tq_encode_vectors(tq_vec_index* v, const float* x, int64_t start, int64_t count,
                             void* codes, cudaStream_t stream) {
-  if (!v || !codes || start < 0 || count < 0 || start + count > v->n) return TQ_ERR_INVALID_ARG;
+  if (!v || !codes || start < 0 || count < 0 || start + count > v->n || ((uintptr_t)codes % kVAlign))
+    return TQ_ERR_INVALID_ARG;
   if (count == 0) return TQ_OK;
   if (!x) return TQ_ERR_INVALID_ARG;
   VecEncodeArgs a{};
@@ -672,7 +946,8 @@ tq_status tq_encode_vectors(tq_vec_index* v, const float* x, int64_t start, int6
 
 tq_status tq_ip_search(tq_vec_index* v, const void* codes, const float* q, int32_t nq, int32_t k,
                        float* scores, int32_t* idx, cudaStream_t stream) {
-  if (!v || !codes || !q || !scores || !idx || nq < 1 || nq > v->max_q || k < 1 || k > kListK)
+  if (!v || !codes || !q || !scores || !idx || nq < 1 || nq > v->max_q || k < 1 || k > kListK ||
+      ((uintptr_t)codes % kVAlign))
     return TQ_ERR_INVALID_ARG;
   VecQPrepArgs qa{};
   qa.q = q;
@@ -682,14 +957,16 @@ tq_status tq_ip_search(tq_vec_index* v, const void* codes, const float* q, int32
   qa.m = v->cfg.qjl_bits;
   qa.signs = (const double*)(v->ws + v->W.signs);
   qa.St = (const float*)(v->ws + v->W.St);
+  qa.kq = search_qjl_steps(v->cfg.qjl_bits);
+  qa.half_last = v->cfg.qjl_bits % 32 == 8 ? 1 : 0;
   qa.A = (__half*)(v->ws + v->W.A);
   qa.qscale = (float*)(v->ws + v->W.qscale);
   if (launch_vec_qprep(qa, stream) != cudaSuccess) return TQ_ERR_CUDA;
-  // one wave: query tiles x database splits ~ the SM count
-  const int qtiles = (nq + 63) / 64;
+  // one wave of one CTA per SM: query tiles x database splits
+  const int qtiles = (nq + kM - 1) / kM;
   int nsplit = std::max(1, v->num_sms / qtiles);
   nsplit = std::min(nsplit, kMaxSplits);
-  nsplit = (int)std::min<int64_t>(nsplit, (v->n + 127) / 128);
+  nsplit = (int)std::min<int64_t>(nsplit, (v->n + kN - 1) / kN);
   SearchArgs sa{};
   const uint8_t* base = (const uint8_t*)codes;
   sa.A = qa.A;
@@ -702,6 +979,10 @@ tq_status tq_ip_search(tq_vec_index* v, const void* codes, const float* q, int32
   sa.d = v->d;
   sa.b_theta = v->cfg.b_theta;
   sa.nsplit = nsplit;
+  sa.kq = qa.kq;
+  sa.half_last = qa.half_last;
+  sa.status = (int*)(v->ws + v->W.status);
+  sa.wait_limit_ns = kDefaultWaitLimitNs;
   sa.inv_levels = 1.0f / (float)((1 << v->cfg.b_r) - 1);
   sa.qjl_const = (float)(std::sqrt(M_PI / 2.0) / v->cfg.qjl_bits);
   sa.part_s = (float*)(v->ws + v->W.part_s);
@@ -719,6 +1000,18 @@ tq_status tq_ip_search(tq_vec_index* v, const void* codes, const float* q, int32
   return launch_topk_merge(ma, stream) == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
 }
 
+tq_status tq_vec_get_status(tq_vec_index* v, cudaStream_t stream) {
+  if (!v) return TQ_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return TQ_ERR_CUDA;
+  int word = 0;
+  int* st = (int*)(v->ws + v->W.status);
+  if (cudaMemcpy(&word, st, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return TQ_ERR_CUDA;
+  if (word != 0 && cudaMemset(st, 0, sizeof(int)) != cudaSuccess) return TQ_ERR_CUDA;
+  if (word & kStatusTimeout) return TQ_ERR_TIMEOUT;
+  if (word & kStatusRange) return TQ_ERR_RANGE;
+  return TQ_OK;
+}
+
 tq_status tq_export_vectors(tq_vec_index* v, const void* codes, int64_t start, int64_t count,
                             uint8_t* codes_out, uint8_t* bits_out, uint16_t* s16_out,
                             uint16_t* rn16_out, cudaStream_t stream) {
@@ -727,13 +1020,25 @@ tq_status tq_export_vectors(tq_vec_index* v, const void* codes, int64_t start, i
   if (cudaStreamSynchronize(stream) != cudaSuccess) return TQ_ERR_CUDA;
   const uint8_t* base = (const uint8_t*)codes;
   const int P = v->d / 2, mb = v->cfg.qjl_bits / 8;
+  // the groups of 32 vectors that hold [start, start + count)
+  const int64_t g0 = start / 32, g1 = (start + count + 31) / 32;
   cudaError_t e = cudaSuccess;
-  // bw = 8: the canonical LSB-first stream is one byte per pair
-  if (codes_out) e = cudaMemcpy(codes_out, base + v->C.codes + start * P, (size_t)count * P, cudaMemcpyDeviceToHost);
+  if (codes_out) {
+    // bw = 8: the canonical LSB-first stream is one byte per pair
+    std::vector<uint8_t> tmp((size_t)(g1 - g0) * 32 * P);
+    e = cudaMemcpy(tmp.data(), base + v->C.codes + g0 * 32 * P, tmp.size(), cudaMemcpyDeviceToHost);
+    for (int64_t i = 0; e == cudaSuccess && i < count; ++i) {
+      const int64_t g = start + i, off = (g / 32 - g0) * 32 * P + (g % 32) * 16;
+      for (int b = 0; b < P; ++b) codes_out[i * P + b] = tmp[off + (b / 16) * 512 + b % 16];
+    }
+  }
   if (e == cudaSuccess && bits_out) {
-    std::vector<uint8_t> tmp((size_t)count * 32);
-    e = cudaMemcpy(tmp.data(), base + v->C.signs + start * 32, tmp.size(), cudaMemcpyDeviceToHost);
-    for (int64_t i = 0; e == cudaSuccess && i < count; ++i) std::memcpy(bits_out + i * mb, tmp.data() + i * 32, mb);
+    std::vector<uint8_t> tmp((size_t)(g1 - g0) * 1024);
+    e = cudaMemcpy(tmp.data(), base + v->C.signs + g0 * 1024, tmp.size(), cudaMemcpyDeviceToHost);
+    for (int64_t i = 0; e == cudaSuccess && i < count; ++i) {
+      const int64_t g = start + i, off = (g / 32 - g0) * 1024 + (g % 32) * 16;
+      for (int b = 0; b < mb; ++b) bits_out[i * mb + b] = tmp[off + (b / 16) * 512 + b % 16];
+    }
   }
   if (e == cudaSuccess && s16_out) e = cudaMemcpy(s16_out, base + v->C.s16 + start * 2, (size_t)count * 2, cudaMemcpyDeviceToHost);
   if (e == cudaSuccess && rn16_out) e = cudaMemcpy(rn16_out, base + v->C.rn16 + start * 2, (size_t)count * 2, cudaMemcpyDeviceToHost);

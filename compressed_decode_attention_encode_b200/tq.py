@@ -82,6 +82,7 @@ SIGNATURES = [
     ("tq_encode_vectors", c_int32, [c_void_p, c_void_p, c_int64, c_int64, c_void_p, c_void_p]),
     ("tq_ip_search", c_int32, [c_void_p, c_void_p, c_void_p, c_int32, c_int32, c_void_p, c_void_p,
                                c_void_p]),
+    ("tq_vec_get_status", c_int32, [c_void_p, c_void_p]),
     ("tq_export_vectors", c_int32, [c_void_p, c_void_p, c_int64, c_int64, c_void_p, c_void_p,
                                     c_void_p, c_void_p, c_void_p]),
     ("tq_rotation_signs", c_int32, [c_uint64, c_int32, POINTER(c_int8)]),
@@ -465,6 +466,10 @@ class TQVecIndex:
                                   scores.data_ptr(), idx.data_ptr(), _stream_handle(stream)),
                "tq_ip_search")
         return scores, idx
+
+    def get_status(self, stream=None):
+        """Latched device status of the searches (0 = TQ_OK); clears it."""
+        return lib().tq_vec_get_status(self.handle, _stream_handle(stream))
 
     def export(self, start, count, stream=None):
         d = 64

@@ -371,9 +371,13 @@ typedef struct tq_vec_index tq_vec_index;
 
 /*
  * Sizes for an index over n vectors:
- *   codes_bytes      the packed database: codes [n][d/2] (one byte per pair),
- *                    sign bits [n][32] (m bits, zero-padded to 256), s16 [n],
- *                    rn16 [n]; each section 256-byte aligned.
+ *   codes_bytes      the packed database (256-byte aligned): codes (one
+ *                    byte per pair, d/2 per vector) and sign bits (m bits
+ *                    zero-padded to 32 bytes per vector) in groups of 32
+ *                    vectors, each vector's bytes in 16-byte chunks stored
+ *                    chunk-major inside the group ([n/32][chunk][32][16]);
+ *                    then s16 [n] and rn16 [n]; each section 256-byte
+ *                    aligned.  tq_export_vectors returns the canonical form.
  *   workspace_bytes  D, S, query transforms for up to `max_queries` queries
  *                    and the per-split top-k partials of a search.
  */
@@ -397,10 +401,17 @@ tq_status tq_encode_vectors(tq_vec_index* index, const float* x, int64_t start,
  * Top-k estimated inner products of nq queries (device float32 [nq, d_in])
  * against all n encoded vectors.  scores: device float32 [nq, k]; idx:
  * device int32 [nq, k].  1 <= k <= 16, nq <= max_queries.  The products
- * run on tensor cores (fp16 operands, fp32 accumulation).
+ * run on tensor cores (tcgen05, fp16 operands, fp32 accumulation), 128
+ * queries per CTA.  The kernel's waits are bounded: one that gives up
+ * latches TQ_ERR_TIMEOUT in the index's status word (tq_vec_get_status)
+ * and that search's results are undefined.
  */
 tq_status tq_ip_search(tq_vec_index* index, const void* codes, const float* q, int32_t nq,
                        int32_t k, float* scores, int32_t* idx, cudaStream_t stream);
+
+/* The latched device status of an index's searches (synchronizes the
+ * stream, then clears it): TQ_OK or TQ_ERR_TIMEOUT. */
+tq_status tq_vec_get_status(tq_vec_index* index, cudaStream_t stream);
 
 /*
  * Canonical records of database vectors [start, start + count) to HOST

@@ -90,12 +90,30 @@ def test_search_topk_parity(n, nq, k):
     dim, m = 200, 200
     index, x, q = _build(n, dim, m=m, nq=nq)
     scores, idx = index.search(torch.from_numpy(q).cuda(), k=k)
+    assert index.get_status() == 0
     scores, idx = scores.cpu().numpy(), idx.cpu().numpy()
     d = _padded(dim)
     codes = _oracle_codes(index.export(0, n), dim, 4, 4, m)
     ref = O.ip_scores(q.astype(np.float64), O.rotation_signs(0, d), O.qjl_matrix(0, m, d), codes)
     swaps = _check_topk(scores, idx, ref, k)
     print(f"n={n} nq={nq} k={k} tolerated swaps={swaps}")
+    index.close()
+
+
+@pytest.mark.parametrize("dim,m", [(64, 8), (100, 24), (128, 40), (128, 128), (256, 256)])
+def test_search_qjl_step_shapes(dim, m):
+    """Every QJL k-step arrangement: whole sign words, a last word with 8
+    needed bits (one k-step), with 24 (two); two query tiles, the second
+    ragged; a database that ends inside a round of 256."""
+    n, nq, k = 1700, 130, 5
+    index, x, q = _build(n, dim, m=m, nq=nq, vec_seed=2)
+    scores, idx = index.search(torch.from_numpy(q).cuda(), k=k)
+    assert index.get_status() == 0
+    scores, idx = scores.cpu().numpy(), idx.cpu().numpy()
+    d = _padded(dim)
+    codes = _oracle_codes(index.export(0, n), dim, 4, 4, m)
+    ref = O.ip_scores(q.astype(np.float64), O.rotation_signs(0, d), O.qjl_matrix(0, m, d), codes)
+    _check_topk(scores, idx, ref, k)
     index.close()
 
 
@@ -111,6 +129,7 @@ def test_search_full_size_sampled_queries():
         index.encode(torch.from_numpy(mixture_vectors(sw, 0, s, min(chunk, sw.n - s))).cuda(), start=s)
     q = mixture_queries(sw, 0)
     scores, idx = index.search(torch.from_numpy(q).cuda(), k=sw.k)
+    assert index.get_status() == 0
     scores, idx = scores.cpu().numpy(), idx.cpu().numpy()
     d = _padded(sw.dim)
     signs, S = O.rotation_signs(0, d), O.qjl_matrix(0, sw.qjl_bits, d)
