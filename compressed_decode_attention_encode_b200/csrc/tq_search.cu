@@ -9,18 +9,19 @@
 //                       chunk-major, so that a warp reading one chunk of 32
 //                       vectors reads 512 contiguous bytes.
 //   vec_qprep_kernel    q' = R q, q'' = S q' written as the fp16 A operand of
-//                       the search MMAs: tiles of 128 queries in the tensor
-//                       cores' K-major core-matrix order.
-//   search_umma_kernel  per CTA: 128 queries (A, resident in shared memory)
-//                       against a contiguous run of the database, 256
+//                       the search MMAs, one row per query (rows padded to
+//                       whole tiles of 128 with zeros).
+//   search_umma_kernel  per CTA: 128 queries (A, resident in tensor memory)
+//                       against a contiguous run of the database, 128
 //                       vectors per round.  Eight producer warps dequantize
-//                       the round's vectors straight into the B operand
-//                       (fp16 c_r (cos, sin) from a shared LUT times
+//                       the round's vectors straight into the B operand in
+//                       shared memory (fp16 c_r (cos, sin) from a LUT times
 //                       s16/(2^b_r-1); QJL signs as +-rn16 sqrt(pi/2)/m);
-//                       one thread issues tcgen05.mma (M 128, N 256, K 16)
-//                       into one of two fp32 accumulators in tensor memory;
-//                       four epilogue warps read the scores back (thread =
-//                       query) and keep each query's 16 best.
+//                       one thread issues tcgen05.mma (M 128, N 128, K 16,
+//                       A from tensor memory) into one of two fp32
+//                       accumulators; eight epilogue warps read the scores
+//                       back (thread = query, one warp group per round
+//                       parity) and keep each query's 16 best.
 //   topk_merge_kernel   merges the per-split candidate lists.
 #include <cmath>
 #include <cstring>
@@ -40,18 +41,18 @@ constexpr float kNegInf = -INFINITY;
 
 // Search tile shape (tcgen05, one CTA per SM).
 constexpr int kM = 128;                  // queries per CTA = MMA M = tensor-memory lanes
-constexpr int kN = 256;                  // database vectors per round = MMA N
-constexpr int kKStg = 2;                 // k-steps (16 k each) per B stage
-constexpr int kNB = 3;                   // B stages in the ring
-constexpr int kQ = 16;                   // candidate queue entries per query
-constexpr int kEpiWarps = 4;             // warps 0-3: tensor-memory lane quarters 0-3
-constexpr int kProdWarps = 8;            // warps 4-11: one database vector per thread per round
+constexpr int kN = 128;                  // database vectors per round = MMA N
+constexpr int kKStg = 4;                 // k-steps (16 k each) per B stage
+constexpr int kNB = 8;                   // B stages in the ring
+constexpr int kQ = 16;                   // candidate queue entries per (query, round parity)
+constexpr int kEpiWarps = 8;             // warps 0-7: lane quarter w % 4, rounds of parity w / 4
+constexpr int kProdWarps = 8;            // warps 8-15: vector 32 (w % 4) + lane, k-step half w / 4
 constexpr int kMmaWarp = kEpiWarps + kProdWarps;
 constexpr int kSearchThreads = (kMmaWarp + 1) * 32;
-constexpr int kKStepB = kN * 32;         // bytes of one B k-step (256 rows x 16 fp16)
+constexpr int kKStepB = kN * 32;         // bytes of one B k-step (128 rows x 16 fp16)
 constexpr int kStageBytes = kKStg * kKStepB;
-constexpr int kKStepA = kM * 32;         // bytes of one A k-step
-constexpr uint32_t kTmemCols = 2 * kN;   // two fp32 accumulators
+constexpr uint32_t kTmemCols = 512;      // accumulators at columns 0 and kN, A from column 2 kN
+constexpr uint32_t kTmemA = 2 * kN;
 // Instruction descriptor of tcgen05.mma kind::f16: fp32 accumulator (bits
 // 4-5 = 1), fp16 A and B (bits 7-12 = 0), both K-major (bits 15-16 = 0),
 // N >> 3 at bit 17, M >> 4 at bit 24.
@@ -61,20 +62,20 @@ constexpr uint32_t kIdesc = (1u << 4) | ((uint32_t)(kN >> 3) << 17) | ((uint32_t
 struct SearchSmem {
   static constexpr int LUT = 0;                              // 256 entries x 32 lane copies x 4 B
   static constexpr int B = LUT + 256 * 32 * 4;               // kNB stages
-  static constexpr int QUEUE = B + kNB * kStageBytes;        // [kQ][kM] (score, index)
-  static constexpr int BAR = QUEUE + kQ * kM * 8;            // full[kNB], empty[kNB], acc_full[2], acc_empty[2], done
+  static constexpr int QUEUE = B + kNB * kStageBytes;        // [kQ][8 warps x 32] (score, index)
+  static constexpr int BAR = QUEUE + kQ * kEpiWarps * 32 * 8;  // full[kNB], empty[kNB], acc_full[2], acc_empty[2], done
   static constexpr int TMEM_SLOT = BAR + 8 * (2 * kNB + 5);
   static constexpr int ABORT = TMEM_SLOT + 4;
-  static constexpr int A = (ABORT + 4 + 127) / 128 * 128;    // ks A k-steps
-  static size_t bytes(int ks) { return (size_t)A + (size_t)ks * kKStepA; }
+  static constexpr int BYTES = (ABORT + 4 + 127) / 128 * 128;
 };
 
 // QJL k-steps of the search operands for m sign bits.  Sign word w (bits
-// 32w..32w+31) fills two k-steps: k-step half h, chunk kc, half2 u holds
-// bits 15-u' (low half) and 31-u' (high half) of the word, u' = 8h + 4kc + u,
-// so one shift and one logic op turn a sign word into a B register.  When
-// the last word holds only 8 needed bits (m % 32 == 8), they are bits 0-7,
-// all in the low halves of h = 1, and h = 0 is skipped.
+// 32w..32w+31) fills k-steps 2w and 2w + 1 (half h = 0, 1): in half h,
+// chunk kc, half2 u holds bits 15-u' (low half) and 31-u' (high half) of the
+// word, u' = 8h + 4kc + u, so one shift and one logic op turn a sign word
+// into a B register.  When the last word holds only 8 needed bits
+// (m % 32 == 8), they are bits 0-7, all in the low halves of h = 1, and
+// h = 0 is skipped.
 __host__ __device__ inline int search_qjl_steps(int m) {
   const int r = m % 32;
   return 2 * (m / 32) + (r == 0 ? 0 : (r == 8 ? 1 : 2));
@@ -95,12 +96,6 @@ __device__ __forceinline__ bool better(float s, int i, float t, int j) {
 }
 
 // ---- shared memory, barriers, tensor memory ---------------------------------
-__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
-  uint32_t v;
-  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
-  return v;
-}
-
 __device__ __forceinline__ float2 lds64f(uint32_t addr) {
   float2 v;
   asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr) : "memory");
@@ -109,11 +104,6 @@ __device__ __forceinline__ float2 lds64f(uint32_t addr) {
 
 __device__ __forceinline__ void sts64f(uint32_t addr, float x, float y) {
   asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(x), "f"(y) : "memory");
-}
-
-__device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
-               : "memory");
 }
 
 __device__ __forceinline__ uint4 ldg_stream(const uint4* p) {
@@ -200,13 +190,31 @@ __device__ __forceinline__ uint64_t umma_desc(uint32_t saddr) {
          (1ull << 46);
 }
 
-__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                         uint32_t accumulate) {
+// D (+)= A B^T, kind::f16, A in tensor memory (lane = row, fp16 element k
+// of a row in 32-bit column k / 2, even k in the low half), B by descriptor.
+__device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
   asm volatile(
       "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
+}
+
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
 }
 
 // The mbarrier's arrival once every tcgen05.mma this thread issued so far
@@ -379,15 +387,10 @@ __global__ void __launch_bounds__(256) vec_qprep_kernel(const VecQPrepArgs a) {
   for (int o = 16; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, o));
   const float al = amax > 0.f ? exp2f(-floorf(log2f(amax))) : 1.f;
   __syncwarp();
-  // element (row r, k) of the tile: k-step k/16 (kKStepA bytes), 8-row group
-  // r/8 (256 B), K half (k/8)%2 (128 B), row r%8 (16 B), k%8
-  const int ks = D / 16 + a.kq;
-  __half* tile = a.A + (size_t)(q / kM) * ks * (kKStepA / 2);
-  const int r = q % kM;
-  auto put = [&](int k, float v) {
-    tile[(k >> 4) * (kKStepA / 2) + (r >> 3) * 128 + ((k >> 3) & 1) * 64 + (r & 7) * 8 + (k & 7)] =
-        __float2half_rn(v);
-  };
+  // row q of the operand: D polar columns, then kq k-steps of QJL columns
+  const int ka = D + 16 * a.kq;
+  __half* row = a.A + (size_t)q * ka;
+  auto put = [&](int k, float v) { row[k] = __float2half_rn(v); };
   for (int k = lane; k < D; k += 32) put(k, sq[warp][k] * al);
   for (int c = lane; c < a.kq * 16; c += 32) {
     const int t = c >> 4, kc = (c >> 3) & 1, u = (c >> 1) & 3, e = c & 1;
@@ -405,20 +408,25 @@ __global__ void __launch_bounds__(256) vec_qprep_kernel(const VecQPrepArgs a) {
 // Rounds of kN database vectors; each round's k-steps (D/16 polar, then kq
 // QJL) pass through a ring of kNB B stages of kKStg k-steps:
 //   producers  --full[slot]-->  MMA thread  --empty[slot] (commit)-->  producers
-//   MMA thread --acc_full[b] (commit)--> epilogue --acc_empty[b]--> MMA thread
-// Every wait is bounded; a timeout raises the CTA's abort flag, which ends
-// every role's loop, and the kernel still waits for its issued MMAs and
-// frees its tensor memory before it returns.
+//   MMA thread --acc_full[b] (commit)--> epilogue group b --acc_empty[b]--> MMA thread
+// Round r accumulates in tensor-memory columns [kN (r % 2), kN (r % 2 + 1))
+// and is read back by epilogue group r % 2 (warps 4 (r % 2) .. + 3), so each
+// query keeps two best lists, one per round parity.  Every wait is bounded;
+// a timeout raises the CTA's abort flag, which ends every role's loop, and
+// the kernel still waits for its issued MMAs and frees its tensor memory
+// before it returns.
 template <int D>
 __global__ void __launch_bounds__(kSearchThreads, 1) search_umma_kernel(const SearchArgs a) {
   using U = SearchSmem;
-  constexpr int KP = D / 16;      // polar k-steps
-  constexpr int CW = D / 8;       // code words per vector (one byte per pair)
+  constexpr int KP = D / 16;      // polar k-steps (a multiple of kKStg)
+  constexpr int PC = D / 64;      // polar chunks (16 code bytes) per producer thread
+  static_assert(KP % kKStg == 0, "polar k-steps fill whole stages");
   extern __shared__ __align__(1024) uint8_t smem[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int ks = KP + a.kq;
+  const int nst = (ks + kKStg - 1) / kKStg;   // stages per round
   const uint32_t sbase = smem_addr(smem);
-  const uint32_t lut_s = sbase + U::LUT, b_s = sbase + U::B, a_s = sbase + U::A;
+  const uint32_t b_s = sbase + U::B;
   const uint32_t bar_full = sbase + U::BAR, bar_empty = bar_full + 8 * kNB;
   const uint32_t bar_accf = bar_empty + 8 * kNB, bar_acce = bar_accf + 16, bar_done = bar_acce + 16;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + U::ABORT);
@@ -440,13 +448,6 @@ __global__ void __launch_bounds__(kSearchThreads, 1) search_umma_kernel(const Se
     const __half2 h = __floats2half2_rn((float)cr * cs, (float)cr * sn);
     lut[e] = *reinterpret_cast<const uint32_t*>(&h);
   }
-  // A: this CTA's query tile, already in core-matrix order
-  {
-    const uint4* src = reinterpret_cast<const uint4*>(a.A) + (size_t)blockIdx.x * ks * (kKStepA / 16);
-    uint4* dst = reinterpret_cast<uint4*>(smem + U::A);
-    for (int i = tid; i < ks * (kKStepA / 16); i += blockDim.x) dst[i] = src[i];
-  }
-  fence_proxy_async();            // the tensor cores read A through the async proxy
   if (tid == 0) {
     for (int i = 0; i < kNB; ++i) {
       mbar_init(bar_full + 8 * i, kProdWarps);
@@ -454,7 +455,7 @@ __global__ void __launch_bounds__(kSearchThreads, 1) search_umma_kernel(const Se
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar_accf + 8 * i, 1);
-      mbar_init(bar_acce + 8 * i, kEpiWarps);
+      mbar_init(bar_acce + 8 * i, kEpiWarps / 2);
     }
     mbar_init(bar_done, 1);
     *abort_flag = 0;
@@ -465,10 +466,26 @@ __global__ void __launch_bounds__(kSearchThreads, 1) search_umma_kernel(const Se
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + U::TMEM_SLOT);
+  // A: warps 0-3 copy their 32 query rows into tensor memory, one k-step
+  // (8 columns) per store
+  if (warp < 4) {
+    const uint4* src = reinterpret_cast<const uint4*>(a.A + ((size_t)blockIdx.x * kM + 32 * warp + lane) * (16 * ks));
+    const uint32_t ta = tmem + ((uint32_t)(32 * warp) << 16) + kTmemA;
+    for (int s = 0; s < ks; ++s) {
+      const uint4 x0 = src[2 * s], x1 = src[2 * s + 1];
+      const uint32_t r[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+      tmem_st8(ta + 8 * s, r);
+    }
+    tmem_wait_st();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
 
   if (warp < kEpiWarps) {
-    // ---------------- epilogue: thread = query row 32 warp + lane ----------
-    const int qr = 32 * warp + lane;
+    // ---------------- epilogue: thread = query row 32 (warp % 4) + lane ----
+    const int quarter = warp & 3, par = warp >> 2;
+    const int qr = 32 * quarter + lane;
     float ts[kListK];
     int ti[kListK];
 #pragma unroll
@@ -478,58 +495,59 @@ __global__ void __launch_bounds__(kSearchThreads, 1) search_umma_kernel(const Se
     }
     float thr = kNegInf;
     int cnt = 0;
-    const uint32_t qbase = sbase + U::QUEUE + qr * 8;     // entry i at + i * kM * 8
+    const uint32_t qbase = sbase + U::QUEUE + (uint32_t)(32 * warp + lane) * 8;   // entry i at + i * 2048
+    constexpr uint32_t kQStride = kEpiWarps * 32 * 8;
     auto flush = [&]() {
       const int mx = __reduce_max_sync(kFull, cnt);
       for (int i = 0; i < mx; ++i) {
         if (i < cnt) {
-          const float2 c = lds64f(qbase + i * (kM * 8));
+          const float2 c = lds64f(qbase + i * kQStride);
           list_insert<kListK>(ts, ti, c.x, __float_as_int(c.y));
         }
       }
       cnt = 0;
       thr = ts[kListK - 1];
     };
-    for (int r = 0; r < nr; ++r) {
-      const int ab = r & 1;
-      if (!warp_wait(bar_accf + 8 * ab, (uint32_t)((r >> 1) & 1), a.wait_limit_ns, abort_flag, a.status))
+    const uint32_t taddr = tmem + ((uint32_t)(32 * quarter) << 16) + (uint32_t)(par * kN);
+    for (int r = par; r < nr; r += 2) {
+      if (!warp_wait(bar_accf + 8 * par, (uint32_t)((r >> 1) & 1), a.wait_limit_ns, abort_flag, a.status))
         break;
       tc_fence_after();
       const int64_t vr = v_lo + (int64_t)r * kN;
       const int valid = (int)(v_hi - vr < kN ? v_hi - vr : kN);
-      const uint32_t taddr = tmem + ((uint32_t)(32 * warp) << 16) + (uint32_t)(ab * kN);
 #pragma unroll 1
       for (int c = 0; c < kN / 32; ++c) {
         uint32_t sv[32];
         tmem_ld32(taddr + 32 * c, sv);
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
+          const float* f = reinterpret_cast<const float*>(sv + 8 * t);
+          const float mx = fmaxf(max3f(f[0], f[1], f[2]), max3f(max3f(f[3], f[4], f[5]), f[6], f[7]));
           const int col = 32 * c + 8 * t;
+          if (!__any_sync(kFull, mx > thr && col < valid)) continue;
           uint32_t m = 0;
 #pragma unroll
-          for (int u = 0; u < 8; ++u) m |= (__uint_as_float(sv[8 * t + u]) > thr ? 1u : 0u) << u;
+          for (int u = 0; u < 8; ++u) m |= (f[u] > thr ? 1u : 0u) << u;
           const int nv = valid - col;
-          if (nv < 8) m &= nv <= 0 ? 0u : ((1u << nv) - 1u);
-          if (__any_sync(kFull, m != 0)) {
-            while (m) {
-              const int j = __ffs(m) - 1;
-              m &= m - 1;
-              sts64f(qbase + cnt * (kM * 8), __uint_as_float(select8(sv + 8 * t, j)),
-                     __int_as_float((int)(vr + col + j)));
-              ++cnt;
-            }
-            if (__any_sync(kFull, cnt > kQ - 8)) flush();
+          if (nv < 8) m &= (1u << nv) - 1u;
+          while (m) {
+            const int j = __ffs(m) - 1;
+            m &= m - 1;
+            sts64f(qbase + cnt * kQStride, __uint_as_float(select8(sv + 8 * t, j)),
+                   __int_as_float((int)(vr + col + j)));
+            ++cnt;
           }
+          if (__any_sync(kFull, cnt > kQ - 8)) flush();
         }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar_acce + 8 * ab);
+      if (lane == 0) mbar_arrive(bar_acce + 8 * par);
     }
     flush();
     const int q = blockIdx.x * kM + qr;
     if (q < a.nq) {
-      const size_t base = ((size_t)q * gridDim.y + blockIdx.y) * kListK;
+      const size_t base = (((size_t)q * gridDim.y + blockIdx.y) * 2 + par) * kListK;
 #pragma unroll
       for (int j = 0; j < kListK; ++j) {
         a.part_s[base + j] = ts[j];
@@ -537,30 +555,36 @@ __global__ void __launch_bounds__(kSearchThreads, 1) search_umma_kernel(const Se
       }
     }
   } else if (warp < kMmaWarp) {
-    // ---------------- producers: thread = vector n of each round -----------
+    // ---------------- producers --------------------------------------------
+    // thread: vector n of each round; half h takes the polar chunks c with
+    // c % 2 == h (k-steps 2c, 2c + 1) and the sign words w with w % 2 == h
+    // (QJL k-steps 2w, 2w + 1): k-steps 4j + 2h, 4j + 2h + 1 of every stage j.
     const int pw = warp - kEpiWarps;
-    const int n = 32 * pw + lane;
+    const int h = pw >> 2;
+    const int n = 32 * (pw & 3) + lane;
     const uint32_t row_off = (uint32_t)((n >> 3) * 256 + (n & 7) * 16);   // core-matrix row of vector n
-    const uint32_t lut_lane = lut_s + 4 * lane;
-    uint32_t cw[CW], sg[8], sa = 0, sb = 0;
-    uint32_t ncw[CW], nsg[8], nsa = 0, nsb = 0;
-    auto load = [&](int r, uint32_t (&w)[CW], uint32_t (&g)[8], uint32_t& xa, uint32_t& xb) {
+    const uint32_t* lutp = lut + lane;
+    uint32_t cw[4 * PC], sg[4], sa = 0, sb = 0;
+    uint32_t ncw[4 * PC], nsg[4], nsa = 0, nsb = 0;
+    auto load = [&](int r, uint32_t (&w)[4 * PC], uint32_t (&g)[4], uint32_t& xa, uint32_t& xb) {
       const int64_t v = v_lo + (int64_t)r * kN + n;
       if (r < nr && v < v_hi) {
         const int64_t grp = v >> 5;                // lane == v % 32
         const uint4* cp = reinterpret_cast<const uint4*>(a.codes + grp * (32 * (D / 2))) + lane;
 #pragma unroll
-        for (int c = 0; c < CW / 4; ++c) {
-          const uint4 t = ldg_stream(cp + 32 * c);
-          w[4 * c] = t.x;
-          w[4 * c + 1] = t.y;
-          w[4 * c + 2] = t.z;
-          w[4 * c + 3] = t.w;
+        for (int i = 0; i < PC; ++i) {
+          const uint4 t = ldg_stream(cp + 32 * (2 * i + h));
+          w[4 * i] = t.x;
+          w[4 * i + 1] = t.y;
+          w[4 * i + 2] = t.z;
+          w[4 * i + 3] = t.w;
         }
         const uint4* sp = reinterpret_cast<const uint4*>(a.signs + grp * 1024) + lane;
         const uint4 s0 = ldg_stream(sp), s1 = ldg_stream(sp + 32);
-        g[0] = s0.x; g[1] = s0.y; g[2] = s0.z; g[3] = s0.w;
-        g[4] = s1.x; g[5] = s1.y; g[6] = s1.z; g[7] = s1.w;
+        g[0] = h ? s0.y : s0.x;      // words h, 2 + h, 4 + h, 6 + h
+        g[1] = h ? s0.w : s0.z;
+        g[2] = h ? s1.y : s1.x;
+        g[3] = h ? s1.w : s1.z;
         const float s16 = __half2float(__ushort_as_half(__ldg(a.s16 + v)));
         const float rn = __half2float(__ushort_as_half(__ldg(a.rn16 + v)));
         const uint32_t au = __half_as_ushort(__float2half_rn(s16 * a.inv_levels));
@@ -569,9 +593,9 @@ __global__ void __launch_bounds__(kSearchThreads, 1) search_umma_kernel(const Se
         xb = (bu | (bu << 16)) | 0x80008000u;     // -b; a set sign bit flips it to +b
       } else {
 #pragma unroll
-        for (int c = 0; c < CW; ++c) w[c] = 0u;
+        for (int c = 0; c < 4 * PC; ++c) w[c] = 0u;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) g[c] = 0u;
+        for (int c = 0; c < 4; ++c) g[c] = 0u;
         xa = 0u;
         xb = 0u;                                   // columns past the run score 0 (masked later)
       }
@@ -590,47 +614,56 @@ __global__ void __launch_bounds__(kSearchThreads, 1) search_umma_kernel(const Se
         phase ^= 1u;
       }
     };
+    auto stage_ptr = [&](int j) {          // this thread's row of k-step j of the current stage
+      return reinterpret_cast<uint4*>(smem + U::B + slot * kStageBytes + j * kKStepB + row_off);
+    };
     for (int r = 0; r < nr; ++r) {
       load(r + 1, ncw, nsg, nsa, nsb);
+      // polar stages: chunk 2 st + h -> k-steps 4 st + 2 h, 4 st + 2 h + 1
 #pragma unroll
-      for (int s = 0; s < KP; ++s) {
-        const int j = s % kKStg;
-        if (j == 0 && !acquire()) goto producers_done;
-        const uint32_t dst = b_s + slot * kStageBytes + j * kKStepB + row_off;
+      for (int st = 0; st < KP / kKStg; ++st) {
+        if (!acquire()) goto producers_done;
 #pragma unroll
-        for (int kc = 0; kc < 2; ++kc) {
-          const uint32_t w = cw[2 * s + kc];
-          uint32_t h[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const uint32_t b = __byte_perm(w, 0u, 0x4440u + i);
-            h[i] = hmul2_u32(lds32(lut_lane + (b << 7)), sa);
-          }
-          sts128(dst + kc * 128, h[0], h[1], h[2], h[3]);
-        }
-        if (j == kKStg - 1) release();
-      }
-#pragma unroll
-      for (int t = 0; t < 16; ++t) {
-        if (t < a.kq) {
-          const int j = (KP + t) % kKStg;
-          if (j == 0 && !acquire()) goto producers_done;
-          const uint32_t dst = b_s + slot * kStageBytes + j * kKStepB + row_off;
-          const uint32_t x = sg[t >> 1];
-          const int h = (t == a.kq - 1 && a.half_last) ? 1 : (t & 1);
+        for (int e = 0; e < 2; ++e) {
+          uint4* dst = stage_ptr(2 * h + e);
 #pragma unroll
           for (int kc = 0; kc < 2; ++kc) {
-            const int u0 = 8 * h + 4 * kc;
-            sts128(dst + kc * 128, ((x << u0) & 0x80008000u) ^ sb, ((x << (u0 + 1)) & 0x80008000u) ^ sb,
-                   ((x << (u0 + 2)) & 0x80008000u) ^ sb, ((x << (u0 + 3)) & 0x80008000u) ^ sb);
+            const uint32_t w = cw[4 * st + 2 * e + kc];
+            uint32_t q4[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) q4[i] = hmul2_u32(lutp[__byte_perm(w, 0u, 0x4440u + i) << 5], sa);
+            dst[kc * 8] = make_uint4(q4[0], q4[1], q4[2], q4[3]);
           }
-          if (j == kKStg - 1 || t == a.kq - 1) release();
+        }
+        release();
+      }
+      // QJL stages: word 2 qs + h -> k-steps t = 4 qs + 2 h + e
+#pragma unroll
+      for (int qs = 0; qs < 4; ++qs) {
+        if (4 * qs < a.kq) {
+          if (!acquire()) goto producers_done;
+          const uint32_t x = sg[qs];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int t = 4 * qs + 2 * h + e;
+            if (t < a.kq) {
+              const int hw = (t == a.kq - 1 && a.half_last) ? 1 : e;
+              uint4* dst = stage_ptr(2 * h + e);
+#pragma unroll
+              for (int kc = 0; kc < 2; ++kc) {
+                const int u0 = 8 * hw + 4 * kc;
+                dst[kc * 8] = make_uint4(((x << u0) & 0x80008000u) ^ sb, ((x << (u0 + 1)) & 0x80008000u) ^ sb,
+                                         ((x << (u0 + 2)) & 0x80008000u) ^ sb, ((x << (u0 + 3)) & 0x80008000u) ^ sb);
+              }
+            }
+          }
+          release();
         }
       }
 #pragma unroll
-      for (int c = 0; c < CW; ++c) cw[c] = ncw[c];
+      for (int c = 0; c < 4 * PC; ++c) cw[c] = ncw[c];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) sg[c] = nsg[c];
+      for (int c = 0; c < 4; ++c) sg[c] = nsg[c];
       sa = nsa;
       sb = nsb;
     }
@@ -646,16 +679,17 @@ __global__ void __launch_bounds__(kSearchThreads, 1) search_umma_kernel(const Se
       tc_fence_after();
       const uint32_t d_t = tmem + (uint32_t)(ab * kN);
       bool ok = true;
-      for (int s = 0; s < ks; s += kKStg) {
+      for (int st = 0; st < nst; ++st) {
         if (!wait_or_abort(bar_full + 8 * slot, phase, a.wait_limit_ns, abort_flag, a.status)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const int nst = ks - s < kKStg ? ks - s : kKStg;
-        for (int j = 0; j < nst; ++j)
-          umma_f16(d_t, umma_desc(a_s + (s + j) * kKStepA), umma_desc(b_s + slot * kStageBytes + j * kKStepB),
-                   kIdesc, (s + j) > 0 ? 1u : 0u);
+        const int s0 = st * kKStg;
+        const int n_in = ks - s0 < kKStg ? ks - s0 : kKStg;
+        for (int j = 0; j < n_in; ++j)
+          umma_f16_ts(d_t, tmem + kTmemA + 8 * (s0 + j), umma_desc(b_s + slot * kStageBytes + j * kKStepB),
+                      kIdesc, (s0 + j) > 0 ? 1u : 0u);
         umma_commit(bar_empty + 8 * slot);
         if (++slot == kNB) {
           slot = 0;
@@ -735,7 +769,7 @@ cudaError_t launch_vec_encode_d(const VecEncodeArgs& a, cudaStream_t s) {
 
 template <int D>
 cudaError_t launch_search_d(const SearchArgs& a, cudaStream_t s) {
-  const size_t smem = SearchSmem::bytes(D / 16 + a.kq);
+  const size_t smem = SearchSmem::BYTES;
   if (cudaFuncSetAttribute(search_umma_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return cudaErrorInvalidValue;
@@ -823,10 +857,10 @@ VecWsLayout vec_ws_layout(int d, int m, int max_q) {
   w.status = off; off += kVAlign;
   w.signs = off;  off += vround(sizeof(double) * d);
   w.St = off;     off += vround(sizeof(float) * (size_t)d * m);
-  w.A = off;      off += vround((size_t)((max_q + kM - 1) / kM) * (d / 16 + search_qjl_steps(m)) * kKStepA);
+  w.A = off;      off += vround((size_t)((max_q + kM - 1) / kM) * kM * (d + 16 * search_qjl_steps(m)) * 2);
   w.qscale = off; off += vround(sizeof(float) * max_q);
-  w.part_s = off; off += vround(sizeof(float) * (size_t)max_q * kMaxSplits * kListK);
-  w.part_i = off; off += vround(sizeof(int) * (size_t)max_q * kMaxSplits * kListK);
+  w.part_s = off; off += vround(sizeof(float) * (size_t)max_q * kMaxSplits * 2 * kListK);
+  w.part_i = off; off += vround(sizeof(int) * (size_t)max_q * kMaxSplits * 2 * kListK);
   w.total = off;
   return w;
 }
@@ -993,7 +1027,7 @@ tq_status tq_ip_search(tq_vec_index* v, const void* codes, const float* q, int32
   ma.part_i = sa.part_i;
   ma.qscale = qa.qscale;
   ma.nq = nq;
-  ma.nsplit = nsplit;
+  ma.nsplit = 2 * nsplit;            // two lists (round parities) per split
   ma.k = k;
   ma.scores = scores;
   ma.idx = idx;
