@@ -42,15 +42,14 @@ constexpr float kNegInf = -INFINITY;
 // Search tile shape (tcgen05, one CTA per SM).
 constexpr int kM = 128;                  // queries per CTA = MMA M = tensor-memory lanes
 constexpr int kN = 128;                  // database vectors per round = MMA N
-constexpr int kKStg = 4;                 // k-steps (16 k each) per B stage
-constexpr int kNB = 8;                   // B stages in the ring
+constexpr int kRingKSteps = 32;          // B ring: 32 k-steps (16 k each) of kN rows
+constexpr int kMaxStages = 8;            // stages of the ring: 4 k-steps (d = 64) or 8
 constexpr int kQ = 16;                   // candidate queue entries per (query, round parity)
 constexpr int kEpiWarps = 8;             // warps 0-7: lane quarter w % 4, rounds of parity w / 4
 constexpr int kProdWarps = 8;            // warps 8-15: vector 32 (w % 4) + lane, k-step half w / 4
 constexpr int kMmaWarp = kEpiWarps + kProdWarps;
 constexpr int kSearchThreads = (kMmaWarp + 1) * 32;
 constexpr int kKStepB = kN * 32;         // bytes of one B k-step (128 rows x 16 fp16)
-constexpr int kStageBytes = kKStg * kKStepB;
 constexpr uint32_t kTmemCols = 512;      // accumulators at columns 0 and kN, A from column 2 kN
 constexpr uint32_t kTmemA = 2 * kN;
 // Instruction descriptor of tcgen05.mma kind::f16: fp32 accumulator (bits
@@ -61,10 +60,10 @@ constexpr uint32_t kIdesc = (1u << 4) | ((uint32_t)(kN >> 3) << 17) | ((uint32_t
 // Dynamic shared memory of the search kernel.
 struct SearchSmem {
   static constexpr int LUT = 0;                              // 256 entries x 32 lane copies x 4 B
-  static constexpr int B = LUT + 256 * 32 * 4;               // kNB stages
-  static constexpr int QUEUE = B + kNB * kStageBytes;        // [kQ][8 warps x 32] (score, index)
-  static constexpr int BAR = QUEUE + kQ * kEpiWarps * 32 * 8;  // full[kNB], empty[kNB], acc_full[2], acc_empty[2], done
-  static constexpr int TMEM_SLOT = BAR + 8 * (2 * kNB + 5);
+  static constexpr int B = LUT + 256 * 32 * 4;               // the B ring
+  static constexpr int QUEUE = B + kRingKSteps * kKStepB;    // [kQ][8 warps x 32] (score, index)
+  static constexpr int BAR = QUEUE + kQ * kEpiWarps * 32 * 8;  // full[8], empty[8], acc_full[2], acc_empty[2], done
+  static constexpr int TMEM_SLOT = BAR + 8 * (2 * kMaxStages + 5);
   static constexpr int ABORT = TMEM_SLOT + 4;
   static constexpr int BYTES = (ABORT + 4 + 127) / 128 * 128;
 };
@@ -139,6 +138,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait that may suspend the thread (it issues nothing meanwhile) until
+// the phase completes or about kSuspendNs have passed.
+constexpr uint32_t kSuspendNs = 1000000;
+__device__ __forceinline__ bool mbar_wait_suspend(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(kSuspendNs)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits for phase `parity` of an mbarrier.  Gives up when another role has
 // raised the CTA's abort flag, or after `limit_ns` (then raises it and
 // latches kStatusTimeout).
@@ -146,7 +159,7 @@ __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, uns
                                               volatile int* abort_flag, int* status) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
-  while (!mbar_try_wait(bar, parity)) {
+  while (!mbar_wait_suspend(bar, parity)) {
     if (*abort_flag) return false;
     if (global_ns() - t0 > limit_ns) {
       *abort_flag = 1;
@@ -406,7 +419,7 @@ __global__ void __launch_bounds__(256) vec_qprep_kernel(const VecQPrepArgs a) {
 // search
 // ---------------------------------------------------------------------------
 // Rounds of kN database vectors; each round's k-steps (D/16 polar, then kq
-// QJL) pass through a ring of kNB B stages of kKStg k-steps:
+// QJL) pass through a ring of NB B stages of KSTG k-steps:
 //   producers  --full[slot]-->  MMA thread  --empty[slot] (commit)-->  producers
 //   MMA thread --acc_full[b] (commit)--> epilogue group b --acc_empty[b]--> MMA thread
 // Round r accumulates in tensor-memory columns [kN (r % 2), kN (r % 2 + 1))
@@ -418,17 +431,21 @@ __global__ void __launch_bounds__(256) vec_qprep_kernel(const VecQPrepArgs a) {
 template <int D>
 __global__ void __launch_bounds__(kSearchThreads, 1) search_umma_kernel(const SearchArgs a) {
   using U = SearchSmem;
-  constexpr int KP = D / 16;      // polar k-steps (a multiple of kKStg)
+  constexpr int KP = D / 16;      // polar k-steps
   constexpr int PC = D / 64;      // polar chunks (16 code bytes) per producer thread
-  static_assert(KP % kKStg == 0, "polar k-steps fill whole stages");
+  constexpr int KSTG = D >= 128 ? 8 : 4;   // k-steps per stage
+  constexpr int NB = kRingKSteps / KSTG;   // stages in the ring
+  constexpr int CPS = KSTG / 4;            // chunks (or sign words) per producer thread per stage
+  constexpr int STAGE_BYTES = KSTG * kKStepB;
+  static_assert(KP % KSTG == 0 && NB <= kMaxStages, "polar k-steps fill whole stages");
   extern __shared__ __align__(1024) uint8_t smem[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int ks = KP + a.kq;
-  const int nst = (ks + kKStg - 1) / kKStg;   // stages per round
+  const int nst = (ks + KSTG - 1) / KSTG;   // stages per round
   const uint32_t sbase = smem_addr(smem);
   const uint32_t b_s = sbase + U::B;
-  const uint32_t bar_full = sbase + U::BAR, bar_empty = bar_full + 8 * kNB;
-  const uint32_t bar_accf = bar_empty + 8 * kNB, bar_acce = bar_accf + 16, bar_done = bar_acce + 16;
+  const uint32_t bar_full = sbase + U::BAR, bar_empty = bar_full + 8 * kMaxStages;
+  const uint32_t bar_accf = bar_empty + 8 * kMaxStages, bar_acce = bar_accf + 16, bar_done = bar_acce + 16;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + U::ABORT);
 
   // this CTA's run: rounds [r0, r1) of the database
@@ -449,7 +466,7 @@ __global__ void __launch_bounds__(kSearchThreads, 1) search_umma_kernel(const Se
     lut[e] = *reinterpret_cast<const uint32_t*>(&h);
   }
   if (tid == 0) {
-    for (int i = 0; i < kNB; ++i) {
+    for (int i = 0; i < NB; ++i) {
       mbar_init(bar_full + 8 * i, kProdWarps);
       mbar_init(bar_empty + 8 * i, 1);
     }
@@ -558,15 +575,16 @@ __global__ void __launch_bounds__(kSearchThreads, 1) search_umma_kernel(const Se
     // ---------------- producers --------------------------------------------
     // thread: vector n of each round; half h takes the polar chunks c with
     // c % 2 == h (k-steps 2c, 2c + 1) and the sign words w with w % 2 == h
-    // (QJL k-steps 2w, 2w + 1): k-steps 4j + 2h, 4j + 2h + 1 of every stage j.
+    // (QJL k-steps 2w, 2w + 1): k-steps 4i + 2h, 4i + 2h + 1 (i < KSTG / 4)
+    // of every stage.
     const int pw = warp - kEpiWarps;
     const int h = pw >> 2;
     const int n = 32 * (pw & 3) + lane;
     const uint32_t row_off = (uint32_t)((n >> 3) * 256 + (n & 7) * 16);   // core-matrix row of vector n
     const uint32_t* lutp = lut + lane;
-    uint32_t cw[4 * PC], sg[4], sa = 0, sb = 0;
-    uint32_t ncw[4 * PC], nsg[4], nsa = 0, nsb = 0;
-    auto load = [&](int r, uint32_t (&w)[4 * PC], uint32_t (&g)[4], uint32_t& xa, uint32_t& xb) {
+    uint32_t cw[4 * PC], sg[4], raw = 0;          // raw: s16 | rn16 << 16
+    uint32_t ncw[4 * PC], nsg[4], nraw = 0;
+    auto load = [&](int r, uint32_t (&w)[4 * PC], uint32_t (&g)[4], uint32_t& x) {
       const int64_t v = v_lo + (int64_t)r * kN + n;
       if (r < nr && v < v_hi) {
         const int64_t grp = v >> 5;                // lane == v % 32
@@ -585,22 +603,16 @@ __global__ void __launch_bounds__(kSearchThreads, 1) search_umma_kernel(const Se
         g[1] = h ? s0.w : s0.z;
         g[2] = h ? s1.y : s1.x;
         g[3] = h ? s1.w : s1.z;
-        const float s16 = __half2float(__ushort_as_half(__ldg(a.s16 + v)));
-        const float rn = __half2float(__ushort_as_half(__ldg(a.rn16 + v)));
-        const uint32_t au = __half_as_ushort(__float2half_rn(s16 * a.inv_levels));
-        const uint32_t bu = __half_as_ushort(__float2half_rn(rn * a.qjl_const));
-        xa = au | (au << 16);
-        xb = (bu | (bu << 16)) | 0x80008000u;     // -b; a set sign bit flips it to +b
+        x = (uint32_t)__ldg(a.s16 + v) | ((uint32_t)__ldg(a.rn16 + v) << 16);
       } else {
 #pragma unroll
         for (int c = 0; c < 4 * PC; ++c) w[c] = 0u;
 #pragma unroll
         for (int c = 0; c < 4; ++c) g[c] = 0u;
-        xa = 0u;
-        xb = 0u;                                   // columns past the run score 0 (masked later)
+        x = 0u;                                    // columns past the run score 0 (masked later)
       }
     };
-    load(0, cw, sg, sa, sb);
+    load(0, cw, sg, raw);
     uint32_t slot = 0, phase = 0;
     auto acquire = [&]() {
       return warp_wait(bar_empty + 8 * slot, phase ^ 1u, a.wait_limit_ns, abort_flag, a.status);
@@ -609,51 +621,69 @@ __global__ void __launch_bounds__(kSearchThreads, 1) search_umma_kernel(const Se
       fence_proxy_async();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_full + 8 * slot);
-      if (++slot == kNB) {
+      if (++slot == NB) {
         slot = 0;
         phase ^= 1u;
       }
     };
-    auto stage_ptr = [&](int j) {          // this thread's row of k-step j of the current stage
-      return reinterpret_cast<uint4*>(smem + U::B + slot * kStageBytes + j * kKStepB + row_off);
+    auto kstep_ptr = [&](int j) {          // this thread's row of k-step j of the current stage
+      return reinterpret_cast<uint4*>(smem + U::B + slot * STAGE_BYTES + j * kKStepB + row_off);
     };
     for (int r = 0; r < nr; ++r) {
-      load(r + 1, ncw, nsg, nsa, nsb);
-      // polar stages: chunk 2 st + h -> k-steps 4 st + 2 h, 4 st + 2 h + 1
+      load(r + 1, ncw, nsg, nraw);
+      // the scales loaded a round ago: s16/(2^b_r-1) for the polar values,
+      // -rn16 sqrt(pi/2)/m for the QJL ones (a set sign bit makes it +)
+      uint32_t sa, sb;
+      {
+        const float s16 = __half2float(__ushort_as_half((unsigned short)(raw & 0xffffu)));
+        const float rn = __half2float(__ushort_as_half((unsigned short)(raw >> 16)));
+        const uint32_t au = __half_as_ushort(__float2half_rn(s16 * a.inv_levels));
+        const uint32_t bu = __half_as_ushort(__float2half_rn(rn * a.qjl_const));
+        sa = au | (au << 16);
+        sb = raw ? ((bu | (bu << 16)) | 0x80008000u) : 0u;
+      }
+      // polar stages: chunk 2i + h (i = CPS st + i2) -> k-steps 4 i2 + 2h + e
 #pragma unroll
-      for (int st = 0; st < KP / kKStg; ++st) {
+      for (int st = 0; st < KP / KSTG; ++st) {
         if (!acquire()) goto producers_done;
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          uint4* dst = stage_ptr(2 * h + e);
+        for (int i2 = 0; i2 < CPS; ++i2) {
+          const int i = CPS * st + i2;
 #pragma unroll
-          for (int kc = 0; kc < 2; ++kc) {
-            const uint32_t w = cw[4 * st + 2 * e + kc];
-            uint32_t q4[4];
+          for (int e = 0; e < 2; ++e) {
+            uint4* dst = kstep_ptr(4 * i2 + 2 * h + e);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) q4[i] = hmul2_u32(lutp[__byte_perm(w, 0u, 0x4440u + i) << 5], sa);
-            dst[kc * 8] = make_uint4(q4[0], q4[1], q4[2], q4[3]);
+            for (int kc = 0; kc < 2; ++kc) {
+              const uint32_t w = cw[4 * i + 2 * e + kc];
+              uint32_t q4[4];
+#pragma unroll
+              for (int u = 0; u < 4; ++u) q4[u] = hmul2_u32(lutp[__byte_perm(w, 0u, 0x4440u + u) << 5], sa);
+              dst[kc * 8] = make_uint4(q4[0], q4[1], q4[2], q4[3]);
+            }
           }
         }
         release();
       }
-      // QJL stages: word 2 qs + h -> k-steps t = 4 qs + 2 h + e
+      // QJL stages: word 2 (CPS qs + i2) + h -> k-steps t = KSTG qs + 4 i2 + 2h + e
 #pragma unroll
-      for (int qs = 0; qs < 4; ++qs) {
-        if (4 * qs < a.kq) {
+      for (int qs = 0; qs < 16 / KSTG; ++qs) {
+        if (KSTG * qs < a.kq) {
           if (!acquire()) goto producers_done;
-          const uint32_t x = sg[qs];
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int t = 4 * qs + 2 * h + e;
-            if (t < a.kq) {
-              const int hw = (t == a.kq - 1 && a.half_last) ? 1 : e;
-              uint4* dst = stage_ptr(2 * h + e);
+          for (int i2 = 0; i2 < CPS; ++i2) {
+            const uint32_t x = sg[CPS * qs + i2];
 #pragma unroll
-              for (int kc = 0; kc < 2; ++kc) {
-                const int u0 = 8 * hw + 4 * kc;
-                dst[kc * 8] = make_uint4(((x << u0) & 0x80008000u) ^ sb, ((x << (u0 + 1)) & 0x80008000u) ^ sb,
-                                         ((x << (u0 + 2)) & 0x80008000u) ^ sb, ((x << (u0 + 3)) & 0x80008000u) ^ sb);
+            for (int e = 0; e < 2; ++e) {
+              const int t = KSTG * qs + 4 * i2 + 2 * h + e;
+              if (t < a.kq) {
+                const int hw = (t == a.kq - 1 && a.half_last) ? 1 : e;
+                uint4* dst = kstep_ptr(4 * i2 + 2 * h + e);
+#pragma unroll
+                for (int kc = 0; kc < 2; ++kc) {
+                  const int u0 = 8 * hw + 4 * kc;
+                  dst[kc * 8] = make_uint4(((x << u0) & 0x80008000u) ^ sb, ((x << (u0 + 1)) & 0x80008000u) ^ sb,
+                                           ((x << (u0 + 2)) & 0x80008000u) ^ sb, ((x << (u0 + 3)) & 0x80008000u) ^ sb);
+                }
               }
             }
           }
@@ -664,49 +694,56 @@ __global__ void __launch_bounds__(kSearchThreads, 1) search_umma_kernel(const Se
       for (int c = 0; c < 4 * PC; ++c) cw[c] = ncw[c];
 #pragma unroll
       for (int c = 0; c < 4; ++c) sg[c] = nsg[c];
-      sa = nsa;
-      sb = nsb;
+      raw = nraw;
     }
   producers_done:;
-  } else if (lane == 0) {
-    // ---------------- MMA issue (one thread) --------------------------------
+  } else {
+    // ---------------- MMA issue (warp kMmaWarp; one elected lane issues) ----
+    uint32_t elected;
+    asm volatile("{\n .reg .pred p;\n elect.sync _|p, 0xffffffff;\n selp.u32 %0, 1, 0, p;\n}\n" : "=r"(elected));
     uint32_t slot = 0, phase = 0;
     for (int r = 0; r < nr; ++r) {
       const int ab = r & 1;
-      if (!wait_or_abort(bar_acce + 8 * ab, (uint32_t)(((r >> 1) & 1) ^ 1), a.wait_limit_ns, abort_flag,
-                         a.status))
+      if (!warp_wait(bar_acce + 8 * ab, (uint32_t)(((r >> 1) & 1) ^ 1), a.wait_limit_ns, abort_flag, a.status))
         break;
       tc_fence_after();
       const uint32_t d_t = tmem + (uint32_t)(ab * kN);
       bool ok = true;
       for (int st = 0; st < nst; ++st) {
-        if (!wait_or_abort(bar_full + 8 * slot, phase, a.wait_limit_ns, abort_flag, a.status)) {
+        if (!warp_wait(bar_full + 8 * slot, phase, a.wait_limit_ns, abort_flag, a.status)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const int s0 = st * kKStg;
-        const int n_in = ks - s0 < kKStg ? ks - s0 : kKStg;
-        for (int j = 0; j < n_in; ++j)
-          umma_f16_ts(d_t, tmem + kTmemA + 8 * (s0 + j), umma_desc(b_s + slot * kStageBytes + j * kKStepB),
-                      kIdesc, (s0 + j) > 0 ? 1u : 0u);
-        umma_commit(bar_empty + 8 * slot);
-        if (++slot == kNB) {
+        const int s0 = st * KSTG;
+        const int n_in = ks - s0 < KSTG ? ks - s0 : KSTG;
+        if (elected) {
+          for (int j = 0; j < n_in; ++j)
+            umma_f16_ts(d_t, tmem + kTmemA + 8 * (s0 + j), umma_desc(b_s + slot * STAGE_BYTES + j * kKStepB),
+                        kIdesc, (s0 + j) > 0 ? 1u : 0u);
+          umma_commit(bar_empty + 8 * slot);
+        }
+        __syncwarp();
+        if (++slot == NB) {
           slot = 0;
           phase ^= 1u;
         }
       }
       if (!ok) break;
-      umma_commit(bar_accf + 8 * ab);
+      if (elected) umma_commit(bar_accf + 8 * ab);
+      __syncwarp();
     }
     // every issued MMA has finished before tensor memory is freed
-    umma_commit(bar_done);
-    const uint64_t t0 = global_ns();
-    while (!mbar_try_wait(bar_done, 0u))
-      if (global_ns() - t0 > a.wait_limit_ns) {
-        atomicOr(a.status, kStatusTimeout);
-        break;
-      }
+    if (elected) {
+      umma_commit(bar_done);
+      const uint64_t t0 = global_ns();
+      while (!mbar_try_wait(bar_done, 0u))
+        if (global_ns() - t0 > a.wait_limit_ns) {
+          atomicOr(a.status, kStatusTimeout);
+          break;
+        }
+    }
+    __syncwarp();
   }
   tc_fence_before();
   __syncthreads();
