@@ -20,8 +20,8 @@
 //                       one thread issues tcgen05.mma (M 128, N 128, K 16,
 //                       A from tensor memory) into one of two fp32
 //                       accumulators; eight epilogue warps read the scores
-//                       back (thread = query, one warp group per round
-//                       parity) and keep each query's 16 best.
+//                       back (thread = query, one warp group per column
+//                       half) and keep each query's 16 best per half.
 //   topk_merge_kernel   merges the per-split candidate lists.
 #include <cmath>
 #include <cstring>
@@ -45,7 +45,7 @@ constexpr int kN = 128;                  // database vectors per round = MMA N
 constexpr int kRingKSteps = 32;          // B ring: 32 k-steps (16 k each) of kN rows
 constexpr int kMaxStages = 8;            // stages of the ring: 4 k-steps (d = 64) or 8
 constexpr int kQ = 16;                   // candidate queue entries per (query, round parity)
-constexpr int kEpiWarps = 8;             // warps 0-7: lane quarter w % 4, rounds of parity w / 4
+constexpr int kEpiWarps = 8;             // warps 0-7: lane quarter w % 4, column half w / 4
 constexpr int kProdWarps = 8;            // warps 8-15: vector 32 (w % 4) + lane, k-step half w / 4
 constexpr int kMmaWarp = kEpiWarps + kProdWarps;
 constexpr int kSearchThreads = (kMmaWarp + 1) * 32;
@@ -105,12 +105,20 @@ __device__ __forceinline__ void sts64f(uint32_t addr, float x, float y) {
   asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(x), "f"(y) : "memory");
 }
 
-__device__ __forceinline__ uint4 ldg_stream(const uint4* p) {
-  uint4 v;
+// Streaming loads straight into the destination registers (nothing reads
+// them until a round later, so the loads stay in flight meanwhile).
+__device__ __forceinline__ void ldg_stream4(const void* p, uint32_t& x, uint32_t& y, uint32_t& z, uint32_t& w) {
   asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "=r"(x), "=r"(y), "=r"(z), "=r"(w)
                : "l"(p));
-  return v;
+}
+
+__device__ __forceinline__ void ldg_stream1(const void* p, uint32_t& x) {
+  asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(x) : "l"(p));
+}
+
+__device__ __forceinline__ void ldg_stream_u16(const void* p, uint32_t& x) {
+  asm volatile("ld.global.nc.L1::no_allocate.u16 %0, [%1];" : "=r"(x) : "l"(p));
 }
 
 __device__ __forceinline__ uint64_t global_ns() {
@@ -422,9 +430,10 @@ __global__ void __launch_bounds__(256) vec_qprep_kernel(const VecQPrepArgs a) {
 // QJL) pass through a ring of NB B stages of KSTG k-steps:
 //   producers  --full[slot]-->  MMA thread  --empty[slot] (commit)-->  producers
 //   MMA thread --acc_full[b] (commit)--> epilogue group b --acc_empty[b]--> MMA thread
-// Round r accumulates in tensor-memory columns [kN (r % 2), kN (r % 2 + 1))
-// and is read back by epilogue group r % 2 (warps 4 (r % 2) .. + 3), so each
-// query keeps two best lists, one per round parity.  Every wait is bounded;
+// Round r accumulates in tensor-memory columns [kN (r % 2), kN (r % 2 + 1));
+// epilogue group g (warps 4g .. 4g + 3) reads the round's columns
+// [kN/2 g, kN/2 (g + 1)), so each query keeps two best lists, one per
+// column half.  Every wait is bounded;
 // a timeout raises the CTA's abort flag, which ends every role's loop, and
 // the kernel still waits for its issued MMAs and frees its tensor memory
 // before it returns.
@@ -472,7 +481,7 @@ __global__ void __launch_bounds__(kSearchThreads, 1) search_umma_kernel(const Se
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar_accf + 8 * i, 1);
-      mbar_init(bar_acce + 8 * i, kEpiWarps / 2);
+      mbar_init(bar_acce + 8 * i, kEpiWarps);
     }
     mbar_init(bar_done, 1);
     *abort_flag = 0;
@@ -501,7 +510,8 @@ __global__ void __launch_bounds__(kSearchThreads, 1) search_umma_kernel(const Se
 
   if (warp < kEpiWarps) {
     // ---------------- epilogue: thread = query row 32 (warp % 4) + lane ----
-    const int quarter = warp & 3, par = warp >> 2;
+    // warp group g = warp / 4 reads columns [64 g, 64 g + 64) of every round
+    const int quarter = warp & 3, grp = warp >> 2;
     const int qr = 32 * quarter + lane;
     float ts[kListK];
     int ti[kListK];
@@ -525,26 +535,36 @@ __global__ void __launch_bounds__(kSearchThreads, 1) search_umma_kernel(const Se
       cnt = 0;
       thr = ts[kListK - 1];
     };
-    const uint32_t taddr = tmem + ((uint32_t)(32 * quarter) << 16) + (uint32_t)(par * kN);
-    for (int r = par; r < nr; r += 2) {
-      if (!warp_wait(bar_accf + 8 * par, (uint32_t)((r >> 1) & 1), a.wait_limit_ns, abort_flag, a.status))
+    const uint32_t taddr = tmem + ((uint32_t)(32 * quarter) << 16) + (uint32_t)(grp * (kN / 2));
+    for (int r = 0; r < nr; ++r) {
+      const int ab = r & 1;
+      if (!warp_wait(bar_accf + 8 * ab, (uint32_t)((r >> 1) & 1), a.wait_limit_ns, abort_flag, a.status))
         break;
       tc_fence_after();
       const int64_t vr = v_lo + (int64_t)r * kN;
       const int valid = (int)(v_hi - vr < kN ? v_hi - vr : kN);
 #pragma unroll 1
-      for (int c = 0; c < kN / 32; ++c) {
+      for (int c = 0; c < kN / 64; ++c) {
         uint32_t sv[32];
-        tmem_ld32(taddr + 32 * c, sv);
+        tmem_ld32(taddr + (uint32_t)(ab * kN + 32 * c), sv);
+        const float* f = reinterpret_cast<const float*>(sv);
+        const int col0 = grp * (kN / 2) + 32 * c;
+        // sub-chunks of 8 columns holding a score above the lane's threshold
+        uint32_t hit = 0;
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
-          const float* f = reinterpret_cast<const float*>(sv + 8 * t);
-          const float mx = fmaxf(max3f(f[0], f[1], f[2]), max3f(max3f(f[3], f[4], f[5]), f[6], f[7]));
-          const int col = 32 * c + 8 * t;
-          if (!__any_sync(kFull, mx > thr && col < valid)) continue;
+          const float mx = fmaxf(max3f(f[8 * t], f[8 * t + 1], f[8 * t + 2]),
+                                 max3f(max3f(f[8 * t + 3], f[8 * t + 4], f[8 * t + 5]), f[8 * t + 6], f[8 * t + 7]));
+          hit |= (mx > thr && col0 + 8 * t < valid) ? (1u << t) : 0u;
+        }
+        const uint32_t any = __reduce_or_sync(kFull, hit);
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          if (!(any & (1u << t))) continue;
+          const int col = col0 + 8 * t;
           uint32_t m = 0;
 #pragma unroll
-          for (int u = 0; u < 8; ++u) m |= (f[u] > thr ? 1u : 0u) << u;
+          for (int u = 0; u < 8; ++u) m |= (f[8 * t + u] > thr ? 1u : 0u) << u;
           const int nv = valid - col;
           if (nv < 8) m &= (1u << nv) - 1u;
           while (m) {
@@ -559,12 +579,12 @@ __global__ void __launch_bounds__(kSearchThreads, 1) search_umma_kernel(const Se
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar_acce + 8 * par);
+      if (lane == 0) mbar_arrive(bar_acce + 8 * ab);
     }
     flush();
     const int q = blockIdx.x * kM + qr;
     if (q < a.nq) {
-      const size_t base = (((size_t)q * gridDim.y + blockIdx.y) * 2 + par) * kListK;
+      const size_t base = (((size_t)q * gridDim.y + blockIdx.y) * 2 + grp) * kListK;
 #pragma unroll
       for (int j = 0; j < kListK; ++j) {
         a.part_s[base + j] = ts[j];
@@ -582,37 +602,35 @@ __global__ void __launch_bounds__(kSearchThreads, 1) search_umma_kernel(const Se
     const int n = 32 * (pw & 3) + lane;
     const uint32_t row_off = (uint32_t)((n >> 3) * 256 + (n & 7) * 16);   // core-matrix row of vector n
     const uint32_t* lutp = lut + lane;
-    uint32_t cw[4 * PC], sg[4], raw = 0;          // raw: s16 | rn16 << 16
-    uint32_t ncw[4 * PC], nsg[4], nraw = 0;
-    auto load = [&](int r, uint32_t (&w)[4 * PC], uint32_t (&g)[4], uint32_t& x) {
+    uint32_t cw[4 * PC], sg[4];
+    uint32_t ncw[4 * PC], nsg[4];
+    uint32_t raw_s = 0, raw_r = 0, nraw_s = 0, nraw_r = 0;   // s16, rn16 bits
+    auto load = [&](int r, uint32_t (&w)[4 * PC], uint32_t (&g)[4], uint32_t& xs, uint32_t& xr) {
       const int64_t v = v_lo + (int64_t)r * kN + n;
       if (r < nr && v < v_hi) {
         const int64_t grp = v >> 5;                // lane == v % 32
-        const uint4* cp = reinterpret_cast<const uint4*>(a.codes + grp * (32 * (D / 2))) + lane;
+        const uint8_t* cp = a.codes + grp * (32 * (D / 2)) + 16 * lane;
 #pragma unroll
-        for (int i = 0; i < PC; ++i) {
-          const uint4 t = ldg_stream(cp + 32 * (2 * i + h));
-          w[4 * i] = t.x;
-          w[4 * i + 1] = t.y;
-          w[4 * i + 2] = t.z;
-          w[4 * i + 3] = t.w;
-        }
-        const uint4* sp = reinterpret_cast<const uint4*>(a.signs + grp * 1024) + lane;
-        const uint4 s0 = ldg_stream(sp), s1 = ldg_stream(sp + 32);
-        g[0] = h ? s0.y : s0.x;      // words h, 2 + h, 4 + h, 6 + h
-        g[1] = h ? s0.w : s0.z;
-        g[2] = h ? s1.y : s1.x;
-        g[3] = h ? s1.w : s1.z;
-        x = (uint32_t)__ldg(a.s16 + v) | ((uint32_t)__ldg(a.rn16 + v) << 16);
+        for (int i = 0; i < PC; ++i)
+          ldg_stream4(cp + 512 * (2 * i + h), w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+        // sign words h, 2 + h (chunk 0) and 4 + h, 6 + h (chunk 1)
+        const uint8_t* sp = a.signs + grp * 1024 + 16 * lane + 4 * h;
+        ldg_stream1(sp, g[0]);
+        ldg_stream1(sp + 8, g[1]);
+        ldg_stream1(sp + 512, g[2]);
+        ldg_stream1(sp + 520, g[3]);
+        ldg_stream_u16(a.s16 + v, xs);
+        ldg_stream_u16(a.rn16 + v, xr);
       } else {
 #pragma unroll
         for (int c = 0; c < 4 * PC; ++c) w[c] = 0u;
 #pragma unroll
         for (int c = 0; c < 4; ++c) g[c] = 0u;
-        x = 0u;                                    // columns past the run score 0 (masked later)
+        xs = 0u;                                   // columns past the run score 0 (masked later)
+        xr = 0u;
       }
     };
-    load(0, cw, sg, raw);
+    load(0, cw, sg, raw_s, raw_r);
     uint32_t slot = 0, phase = 0;
     auto acquire = [&]() {
       return warp_wait(bar_empty + 8 * slot, phase ^ 1u, a.wait_limit_ns, abort_flag, a.status);
@@ -630,17 +648,17 @@ __global__ void __launch_bounds__(kSearchThreads, 1) search_umma_kernel(const Se
       return reinterpret_cast<uint4*>(smem + U::B + slot * STAGE_BYTES + j * kKStepB + row_off);
     };
     for (int r = 0; r < nr; ++r) {
-      load(r + 1, ncw, nsg, nraw);
+      load(r + 1, ncw, nsg, nraw_s, nraw_r);
       // the scales loaded a round ago: s16/(2^b_r-1) for the polar values,
       // -rn16 sqrt(pi/2)/m for the QJL ones (a set sign bit makes it +)
       uint32_t sa, sb;
       {
-        const float s16 = __half2float(__ushort_as_half((unsigned short)(raw & 0xffffu)));
-        const float rn = __half2float(__ushort_as_half((unsigned short)(raw >> 16)));
+        const float s16 = __half2float(__ushort_as_half((unsigned short)raw_s));
+        const float rn = __half2float(__ushort_as_half((unsigned short)raw_r));
         const uint32_t au = __half_as_ushort(__float2half_rn(s16 * a.inv_levels));
         const uint32_t bu = __half_as_ushort(__float2half_rn(rn * a.qjl_const));
         sa = au | (au << 16);
-        sb = raw ? ((bu | (bu << 16)) | 0x80008000u) : 0u;
+        sb = (bu | (bu << 16)) | 0x80008000u;
       }
       // polar stages: chunk 2i + h (i = CPS st + i2) -> k-steps 4 i2 + 2h + e
 #pragma unroll
@@ -694,7 +712,8 @@ __global__ void __launch_bounds__(kSearchThreads, 1) search_umma_kernel(const Se
       for (int c = 0; c < 4 * PC; ++c) cw[c] = ncw[c];
 #pragma unroll
       for (int c = 0; c < 4; ++c) sg[c] = nsg[c];
-      raw = nraw;
+      raw_s = nraw_s;
+      raw_r = nraw_r;
     }
   producers_done:;
   } else {
@@ -1064,7 +1083,7 @@ tq_status tq_ip_search(tq_vec_index* v, const void* codes, const float* q, int32
   ma.part_i = sa.part_i;
   ma.qscale = qa.qscale;
   ma.nq = nq;
-  ma.nsplit = 2 * nsplit;            // two lists (round parities) per split
+  ma.nsplit = 2 * nsplit;            // two lists (column halves) per split
   ma.k = k;
   ma.scores = scores;
   ma.idx = idx;
