@@ -352,75 +352,102 @@ __global__ void __launch_bounds__(256) vec_encode_kernel(const VecEncodeArgs a) 
 }
 
 // ---------------------------------------------------------------------------
-// query prep: one warp per query row of the 128-row tiles (rows past nq are
-// written as zeros)
+// query prep: 8 query rows per CTA of 256 threads (rows past nq are written
+// as zeros).  Each warp rotates one query (q' = R q); then thread i forms
+// q''_i = sum_j S_ij q'_j for the 8 queries (each element of S^T read once
+// per CTA, four q' values per shared load); then each warp scales and writes
+// its row.
 // ---------------------------------------------------------------------------
+constexpr int kQpRows = 8;
+
 template <int D>
 __global__ void __launch_bounds__(256) vec_qprep_kernel(const VecQPrepArgs a) {
   constexpr int E = D / 32;
-  __shared__ float sq[8][D];
-  __shared__ float sqq[8][256];
+  extern __shared__ float qsm[];
+  float* sq = qsm;                       // [8][D]   q'
+  float* sqq = qsm + kQpRows * D;        // [8][256] q''
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int q = blockIdx.x * 8 + warp;
-  const bool live = q < a.nq;
-  float x[E];
+  const int q0 = blockIdx.x * kQpRows;
+  for (int rq = warp; rq < kQpRows; rq += 8) {
+    const int q = q0 + rq;
+    const bool live = q < a.nq;
+    float x[E];
 #pragma unroll
-  for (int i = 0; i < E; ++i) {
-    const int j = lane * E + i;
-    x[i] = (live && j < a.dim) ? a.q[(size_t)q * a.dim + j] * (float)a.signs[j] : 0.f;
-  }
+    for (int i = 0; i < E; ++i) {
+      const int j = lane * E + i;
+      x[i] = (live && j < a.dim) ? a.q[(size_t)q * a.dim + j] * (float)a.signs[j] : 0.f;
+    }
 #pragma unroll
-  for (int hh = 1; hh < D; hh <<= 1) {
-    if (hh < E) {
+    for (int hh = 1; hh < D; hh <<= 1) {
+      if (hh < E) {
 #pragma unroll
-      for (int i = 0; i < E; ++i)
-        if (!(i & hh)) {
-          const float p = x[i], r = x[i + hh];
-          x[i] = p + r;
-          x[i + hh] = p - r;
+        for (int i = 0; i < E; ++i)
+          if (!(i & hh)) {
+            const float p = x[i], r = x[i + hh];
+            x[i] = p + r;
+            x[i + hh] = p - r;
+          }
+      } else {
+        const int lm = hh / E;
+#pragma unroll
+        for (int i = 0; i < E; ++i) {
+          const float o = __shfl_xor_sync(kFull, x[i], lm);
+          x[i] = (lane & lm) ? (o - x[i]) : (x[i] + o);
         }
-    } else {
-      const int lm = hh / E;
-#pragma unroll
-      for (int i = 0; i < E; ++i) {
-        const float o = __shfl_xor_sync(kFull, x[i], lm);
-        x[i] = (lane & lm) ? (o - x[i]) : (x[i] + o);
       }
     }
-  }
-  const float inv = rsqrtf((float)D);
-  float amax = 0.f;
+    const float inv = rsqrtf((float)D);
 #pragma unroll
-  for (int i = 0; i < E; ++i) {
-    x[i] *= inv;
-    sq[warp][lane * E + i] = x[i];
-    amax = fmaxf(amax, fabsf(x[i]));
+    for (int i = 0; i < E; ++i) sq[rq * D + lane * E + i] = x[i] * inv;
   }
-  __syncwarp();
-  for (int i = lane; i < 256; i += 32) {
-    float acc = 0.f;
-    if (live && i < a.m)
-      for (int j = 0; j < D; ++j) acc = fmaf(__ldg(a.St + (size_t)j * a.m + i), sq[warp][j], acc);
-    sqq[warp][i] = acc;
-    amax = fmaxf(amax, fabsf(acc));
-  }
+  __syncthreads();
+  {
+    const int i = threadIdx.x;           // output index of q''
+    float acc[kQpRows];
 #pragma unroll
-  for (int o = 16; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, o));
-  const float al = amax > 0.f ? exp2f(-floorf(log2f(amax))) : 1.f;
-  __syncwarp();
-  // row q of the operand: D polar columns, then kq k-steps of QJL columns
+    for (int r = 0; r < kQpRows; ++r) acc[r] = 0.f;
+    if (i < a.m) {
+      for (int j = 0; j < D; j += 4) {
+        float sv[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sv[e] = __ldg(a.St + (size_t)(j + e) * a.m + i);
+#pragma unroll
+        for (int r = 0; r < kQpRows; ++r) {
+          const float4 x = *reinterpret_cast<const float4*>(sq + r * D + j);
+          acc[r] = fmaf(sv[0], x.x, acc[r]);
+          acc[r] = fmaf(sv[1], x.y, acc[r]);
+          acc[r] = fmaf(sv[2], x.z, acc[r]);
+          acc[r] = fmaf(sv[3], x.w, acc[r]);
+        }
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < kQpRows; ++r) sqq[r * 256 + i] = acc[r];
+  }
+  __syncthreads();
   const int ka = D + 16 * a.kq;
-  __half* row = a.A + (size_t)q * ka;
-  auto put = [&](int k, float v) { row[k] = __float2half_rn(v); };
-  for (int k = lane; k < D; k += 32) put(k, sq[warp][k] * al);
-  for (int c = lane; c < a.kq * 16; c += 32) {
-    const int t = c >> 4, kc = (c >> 3) & 1, u = (c >> 1) & 3, e = c & 1;
-    const int h = (t == a.kq - 1 && a.half_last) ? 1 : (t & 1);
-    const int up = 8 * h + 4 * kc + u;
-    const int bit = 32 * (t >> 1) + (e ? 31 - up : 15 - up);
-    put(D + c, bit < a.m ? sqq[warp][bit] * al : 0.f);
+  for (int rq = warp; rq < kQpRows; rq += 8) {
+    const int q = q0 + rq;
+    const float* xq = sq + rq * D;
+    const float* xqq = sqq + rq * 256;
+    float amax = 0.f;
+    for (int k = lane; k < D; k += 32) amax = fmaxf(amax, fabsf(xq[k]));
+    for (int k = lane; k < a.m; k += 32) amax = fmaxf(amax, fabsf(xqq[k]));
+#pragma unroll
+    for (int o = 16; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, o));
+    const float al = amax > 0.f ? exp2f(-floorf(log2f(amax))) : 1.f;
+    // row q of the operand: D polar columns, then kq k-steps of QJL columns
+    __half* row = a.A + (size_t)q * ka;
+    for (int k = lane; k < D; k += 32) row[k] = __float2half_rn(xq[k] * al);
+    for (int c = lane; c < a.kq * 16; c += 32) {
+      const int t = c >> 4, kc = (c >> 3) & 1, u = (c >> 1) & 3, e = c & 1;
+      const int h = (t == a.kq - 1 && a.half_last) ? 1 : (t & 1);
+      const int up = 8 * h + 4 * kc + u;
+      const int bit = 32 * (t >> 1) + (e ? 31 - up : 15 - up);
+      row[D + c] = __float2half_rn(bit < a.m ? xqq[bit] * al : 0.f);
+    }
+    if (q < a.nq && lane == 0) a.qscale[q] = 1.f / al;
   }
-  if (live && lane == 0) a.qscale[q] = 1.f / al;
 }
 
 // ---------------------------------------------------------------------------
@@ -772,40 +799,55 @@ __global__ void __launch_bounds__(kSearchThreads, 1) search_umma_kernel(const Se
   }
 }
 
-// One thread per query: the k best of its nsplit candidate lists.
+// One warp per query: the k best of its candidate lists (each sorted by
+// (score desc, index asc), padded with (-inf, INT_MAX)).  Lane l holds the
+// heads of lists l and l + 32; each of the k rounds takes the warp's best
+// head and advances that list.
 template <int K>
-__global__ void topk_merge_kernel(const MergeArgs a) {
-  const int q = blockIdx.x * blockDim.x + threadIdx.x;
+__global__ void __launch_bounds__(256) topk_merge_kernel(const MergeArgs a) {
+  const int lane = threadIdx.x & 31;
+  const int q = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (q >= a.nq) return;
-  float ts[K];
-  int ti[K];
-#pragma unroll
-  for (int j = 0; j < K; ++j) {
-    ts[j] = kNegInf;
-    ti[j] = 0x7fffffff;
-  }
   const int lists = a.nsplit;
   const size_t base = (size_t)q * lists * K;
-  for (int e = 0; e < lists * K; ++e) {
-    float sv = a.part_s[base + e];
-    int iv = a.part_i[base + e];
-    if (!better(sv, iv, ts[K - 1], ti[K - 1])) continue;
-#pragma unroll
-    for (int j = 0; j < K; ++j) {
-      if (better(sv, iv, ts[j], ti[j])) {
-        const float t = ts[j];
-        const int ii = ti[j];
-        ts[j] = sv;
-        ti[j] = iv;
-        sv = t;
-        iv = ii;
-      }
+  int pos[2] = {0, 0};
+  float hs[2];
+  int hi[2];
+  auto head = [&](int h) {
+    const int l = lane + 32 * h;
+    if (l < lists && pos[h] < K) {
+      hs[h] = a.part_s[base + (size_t)l * K + pos[h]];
+      hi[h] = a.part_i[base + (size_t)l * K + pos[h]];
+    } else {
+      hs[h] = kNegInf;
+      hi[h] = 0x7fffffff;
     }
-  }
+  };
+  head(0);
+  head(1);
   const float sc = a.qscale[q];
   for (int j = 0; j < a.k; ++j) {
-    a.scores[(size_t)q * a.k + j] = ts[j] * sc;
-    a.idx[(size_t)q * a.k + j] = ti[j];
+    const int mine = better(hs[1], hi[1], hs[0], hi[0]) ? 1 : 0;
+    float bs = hs[mine];
+    int bi = hi[mine];
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      const float os = __shfl_xor_sync(kFull, bs, o);
+      const int oi = __shfl_xor_sync(kFull, bi, o);
+      if (better(os, oi, bs, bi)) {
+        bs = os;
+        bi = oi;
+      }
+    }
+    // database indices are unique across the lists: one lane owns the winner
+    if (bs == hs[mine] && bi == hi[mine] && bi != 0x7fffffff) {
+      ++pos[mine];
+      head(mine);
+    }
+    if (lane == 0) {
+      a.scores[(size_t)q * a.k + j] = bs * sc;
+      a.idx[(size_t)q * a.k + j] = bi;
+    }
   }
 }
 
@@ -845,15 +887,24 @@ cudaError_t launch_vec_encode(const VecEncodeArgs& a, cudaStream_t s) {
   return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_vec_qprep(const VecQPrepArgs& a, cudaStream_t s) {
-  const int grid = (a.nq + kM - 1) / kM * (kM / 8);     // whole 128-row tiles
-  switch (a.d) {
-    case 64: vec_qprep_kernel<64><<<grid, 256, 0, s>>>(a); break;
-    case 128: vec_qprep_kernel<128><<<grid, 256, 0, s>>>(a); break;
-    case 256: vec_qprep_kernel<256><<<grid, 256, 0, s>>>(a); break;
-    default: return cudaErrorInvalidValue;
-  }
+template <int D>
+cudaError_t launch_vec_qprep_d(const VecQPrepArgs& a, cudaStream_t s) {
+  const int grid = (a.nq + kM - 1) / kM * (kM / kQpRows);     // whole 128-row tiles
+  const size_t smem = sizeof(float) * kQpRows * (D + 256);
+  if (cudaFuncSetAttribute(vec_qprep_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return cudaErrorInvalidValue;
+  vec_qprep_kernel<D><<<grid, 256, smem, s>>>(a);
   return cudaGetLastError();
+}
+
+cudaError_t launch_vec_qprep(const VecQPrepArgs& a, cudaStream_t s) {
+  switch (a.d) {
+    case 64: return launch_vec_qprep_d<64>(a, s);
+    case 128: return launch_vec_qprep_d<128>(a, s);
+    case 256: return launch_vec_qprep_d<256>(a, s);
+  }
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_search(const SearchArgs& a, cudaStream_t s) {
@@ -866,7 +917,7 @@ cudaError_t launch_search(const SearchArgs& a, cudaStream_t s) {
 }
 
 cudaError_t launch_topk_merge(const MergeArgs& a, cudaStream_t s) {
-  topk_merge_kernel<16><<<(a.nq + 127) / 128, 128, 0, s>>>(a);
+  topk_merge_kernel<kListK><<<(a.nq + 7) / 8, 256, 0, s>>>(a);
   return cudaGetLastError();
 }
 
