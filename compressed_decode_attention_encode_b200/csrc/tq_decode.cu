@@ -204,6 +204,8 @@ __global__ void combine_kernel(const CombineArgs a) {
   // The next step's eviction encode may start its prologue now (it waits
   // for this kernel before reading its inputs).
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // launched as a programmatic dependent of the attention kernel
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int hg = blockIdx.x;
   const int b = hg / a.Hq, hq = hg % a.Hq;
   const int kvh = hq / a.G, g = hq % a.G;
@@ -408,8 +410,18 @@ cudaError_t launch_rows_upload(RowTable* dst, const RowTable& src, cudaStream_t 
 }
 
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s) {
-  combine_kernel<<<a.batch * a.Hq, a.d, 0, s>>>(a);
-  return cudaGetLastError();
+  // programmatic dependent launch: the kernel waits for the attention
+  // kernel before it reads the partials
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.batch * a.Hq);
+  cfg.blockDim = dim3(a.d);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, combine_kernel, a);
 }
 
 }  // namespace tq
