@@ -57,14 +57,18 @@ def parse():
 # DRAM bytes (read + write) of one attention launch on the default workload,
 # from an ncu capture, keyed by the SHA-1 of the kernel source it was taken
 # on; any other source reports null (the counters no longer describe it).
+# DRAM bytes (read + write) of one attention launch on the llama8b workload,
+# from an ncu capture of such a launch, keyed by the
+# SHA-1 of the kernel's source; a changed kernel reports null until captured
+# again.
 ATTEND_TRAFFIC = {
-    "2d5160ea3994dae680db2d0ef2465534ce58ab42": 261371392 + 3991552,
+    "d16f271aa746a9be5796851f85296458defa66c1": 261319680 + 3596544,
 }
 
 
 def attend_traffic(same_workload: bool):
     import hashlib
-    src = os.path.join(ROOT, "compressed_decode_attention_encode_b200", "csrc", "tq_decode.cu")
+    src = os.path.join(ROOT, "compressed_decode_attention_encode_b200", "csrc", "tq_attend.cuh")
     h = hashlib.sha1(open(src, "rb").read()).hexdigest()
     return ATTEND_TRAFFIC.get(h) if same_workload else None
 
@@ -553,15 +557,28 @@ def run_gpu(args, wl):
             not args.tensor_cache and not args.promotion:
         sample = oracle_sample(wl, args.seed, kv_heads=1)
         time_oracle(sample)
-        tt, kk = 0.0, 0
-        while tt < 10.0:
-            dt, k_ = time_oracle(sample)
-            tt += dt
-            kk += k_
+
+        def rate(seconds):
+            tt, kk = 0.0, 0
+            while tt < seconds:
+                dt, k_ = time_oracle(sample)
+                tt += dt
+                kk += k_
+            return kk / tt
+        v_all = rate(10.0)
+        v_one = None
+        try:
+            import threadpoolctl
+            with threadpoolctl.threadpool_limits(limits=1):
+                v_one = rate(5.0)
+        except Exception:
+            pass
         result["cpu_baseline"] = {
-            "value": kk / tt, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
+            "value": v_all, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
+            "value_1_thread": v_one, "cores_1_thread": 1,
             "sample": f"fp64 oracle decode attention, 1 batch row x 1 kv head (4 q heads) of "
-                      f"layer 0 ({wl.cold} cold + {wl.hot} hot tokens), repeated for ~10 s"}
+                      f"layer 0 ({wl.cold} cold + {wl.hot} hot tokens), repeated for ~10 s on "
+                      f"all threads, then ~5 s with the thread pools limited to one thread"}
     for c in caches:
         c.close()
     if rank == 0:

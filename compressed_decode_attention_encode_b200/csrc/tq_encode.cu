@@ -25,10 +25,11 @@ constexpr int kStStageBytes = 64 * 1024;   // largest S^T staged in shared memor
 
 __host__ __device__ constexpr bool st_staged(int d, int m) { return d * m * 4 <= kStStageBytes; }
 
-// Per-block shared memory: [warps][D] doubles (residuals), per-warp code /
-// sign / scalar staging, then S^T when staged (16-byte aligned).
+// Per-block shared memory: [warps][4][D] doubles (the residuals of a warp's
+// four keys), per-warp code / sign / scalar staging, then S^T when staged
+// (16-byte aligned).
 __host__ __device__ constexpr size_t st_offset(int d, int warps) {
-  return ((size_t)warps * d * sizeof(double) + (size_t)warps * (8 * (d / 2) + 4 * 32 + 32) + 15) /
+  return ((size_t)warps * 4 * d * sizeof(double) + (size_t)warps * (8 * (d / 2) + 4 * 32 + 32) + 15) /
          16 * 16;
 }
 
@@ -38,12 +39,12 @@ __host__ __device__ constexpr size_t small_st_offset(int d) {
   return ((size_t)2 * d * 8 + (size_t)2 * (d / 32) * 8 + (size_t)d + 16 + 8 + 15) / 16 * 16;
 }
 
-template <int D>
+template <int D, bool SKETCH = true>
 __device__ __forceinline__ void encode_vector(const EncodeArgs& a, const float* St,
                                               const __half* src, bool is_key,
                                               double* rbuf, uint8_t* codes, uint32_t* bits,
                                               uint16_t* s16_out, uint16_t* rn16_out) {
-  encode_vector_any<D>(a.L, a.signs, St, a.inv_sqrt_d, a.status,
+  encode_vector_any<D, SKETCH>(a.L, a.signs, St, a.inv_sqrt_d, a.status,
                        [&](int lane, double (&x)[D / 32]) { load_vec<D / 32>(src, lane, x); },
                        is_key, rbuf, codes, bits, s16_out, rn16_out);
 }
@@ -128,8 +129,8 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
   const int warp = threadIdx.x >> 5;
   const int warps = blockDim.x >> 5;
   extern __shared__ double smem[];
-  double* rbuf = smem + warp * D;
-  uint8_t* wbase = reinterpret_cast<uint8_t*>(smem + warps * D) + warp * (8 * P + 4 * 32 + 32);
+  double* rbuf = smem + warp * 4 * D;        // [4][D] the job's key residuals
+  uint8_t* wbase = reinterpret_cast<uint8_t*>(smem + warps * 4 * D) + warp * (8 * P + 4 * 32 + 32);
   uint8_t* kc = wbase;                       // [4][P] key code words
   uint8_t* vc = wbase + 4 * P;               // [4][P] value code words
   uint32_t* kb = reinterpret_cast<uint32_t*>(wbase + 8 * P);   // [4][8] sign words
@@ -191,9 +192,13 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
         ksrc = a.src_k + ((int64_t)unit * a.src_tokens + (e - us.nA)) * D;
         vsrc = a.src_v + ((int64_t)unit * a.src_tokens + (e - us.nA)) * D;
       }
-      encode_vector<D>(a, St, ksrc, true, rbuf, kc + s * P, kb + s * 8, sc + s * 4, sc + s * 4 + 1);
-      encode_vector<D>(a, St, vsrc, false, rbuf, vc + s * P, nullptr, sc + s * 4 + 2, nullptr);
+      encode_vector<D, false>(a, St, ksrc, true, rbuf + s * D, kc + s * P, kb + s * 8, sc + s * 4,
+                              sc + s * 4 + 1);
+      encode_vector<D>(a, St, vsrc, false, nullptr, vc + s * P, nullptr, sc + s * 4 + 2, nullptr);
     }
+    // the four keys' sign words in one pass over S^T
+    if (L.m <= 128) qjl_sketch_block<D, 4, 4>(L.m, St, rbuf, inr, kb, 8);
+    else qjl_sketch_block<D, 4, 8>(L.m, St, rbuf, inr, kb, 8);
     __syncwarp();
 
     uint8_t* tb = a.cold + ((int64_t)unit * L.blocks_per_unit + tile / kTilesPerBlock) * L.block_bytes +

@@ -47,8 +47,10 @@ __device__ __forceinline__ void load_vec(const __half* p, int lane, double (&x)[
 // and the raw fp16 scalars.  Whole warp; returns nothing else.
 // `load(lane, x)` fills the lane's D/32 consecutive input elements (padded
 // coordinates read as 0).  `L` supplies b_r, b_theta and m; `St` is S^T
-// [D, m] (global or shared memory); `signs` the rotation diagonal.
-template <int D, typename Loader>
+// [D, m] (global or shared memory); `signs` the rotation diagonal.  With
+// SKETCH false a key stops after its residual (left in rbuf[0..D)) and its
+// norm; qjl_sketch_block then forms the sign words of several keys at once.
+template <int D, bool SKETCH = true, typename Loader>
 __device__ __forceinline__ void encode_vector_any(const Layout& L, const double* signs,
                                                   const float* St, double inv_sqrt_d, int* status,
                                                   Loader load, bool is_key, double* rbuf,
@@ -144,6 +146,7 @@ __device__ __forceinline__ void encode_vector_any(const Layout& L, const double*
 #pragma unroll
     for (int i = 0; i < E; ++i) rbuf[lane * E + i] = r[i];
     __syncwarp();
+    if constexpr (!SKETCH) return;
     // (S r)_i for the lane's outputs i = lane + 32 k, all k at once so that
     // the loads of a batch of rows of S^T are in flight together; each
     // output still sums over j in ascending order.
@@ -177,6 +180,51 @@ __device__ __forceinline__ void encode_vector_any(const Layout& L, const double*
         const unsigned word = __ballot_sync(kFull, lane + 32 * k < m && acc[k] >= 0.0);
         if (lane == 0) bits[k] = word;
       }
+    }
+  }
+  __syncwarp();
+}
+
+// QJL sign words of NV residuals at once (whole warp): r_v = rbuf[v D ..
+// v D + D), words written to bits[v * bits_stride + k] for the vectors with
+// live[v].  Lane outputs i = lane + 32 k as in encode_vector_any; each S^T
+// value is loaded and widened once and feeds NV fp64 FMAs, and each output
+// still sums over j in ascending order (the same FMAs as one vector alone).
+template <int D, int NV, int NK>
+__device__ __forceinline__ void qjl_sketch_block(int m, const float* St, const double* rbuf,
+                                                 const bool (&live)[NV], uint32_t* bits, int bits_stride) {
+  const int lane = threadIdx.x & 31;
+  double acc[NV][NK];
+#pragma unroll
+  for (int v = 0; v < NV; ++v)
+#pragma unroll
+    for (int k = 0; k < NK; ++k) acc[v][k] = 0.0;
+  constexpr int JB = 2;
+  for (int j0 = 0; j0 < D; j0 += JB) {
+    double sv[JB][NK];
+#pragma unroll
+    for (int jj = 0; jj < JB; ++jj)
+#pragma unroll
+      for (int k = 0; k < NK; ++k) {
+        const int i = lane + 32 * k;
+        sv[jj][k] = i < m ? (double)St[(size_t)(j0 + jj) * m + i] : 0.0;
+      }
+#pragma unroll
+    for (int jj = 0; jj < JB; ++jj) {
+#pragma unroll
+      for (int v = 0; v < NV; ++v) {
+        const double rj = rbuf[v * D + j0 + jj];
+#pragma unroll
+        for (int k = 0; k < NK; ++k) acc[v][k] = fma(sv[jj][k], rj, acc[v][k]);
+      }
+    }
+  }
+#pragma unroll
+  for (int v = 0; v < NV; ++v) {
+#pragma unroll
+    for (int k = 0; k < NK; ++k) {
+      const unsigned word = __ballot_sync(kFull, lane + 32 * k < m && acc[v][k] >= 0.0);
+      if (lane == 0 && live[v] && 32 * k < m) bits[v * bits_stride + k] = word;
     }
   }
   __syncwarp();
