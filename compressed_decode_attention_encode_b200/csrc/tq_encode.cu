@@ -40,11 +40,11 @@ __host__ __device__ constexpr size_t small_st_offset(int d) {
 }
 
 template <int D, bool SKETCH = true>
-__device__ __forceinline__ void encode_vector(const EncodeArgs& a, const float* St,
+__device__ __forceinline__ void encode_vector(const EncodeArgs& a, const float* St, const double2* atab,
                                               const __half* src, bool is_key,
                                               double* rbuf, uint8_t* codes, uint32_t* bits,
                                               uint16_t* s16_out, uint16_t* rn16_out) {
-  encode_vector_any<D, SKETCH>(a.L, a.signs, St, a.inv_sqrt_d, a.status,
+  encode_vector_any<D, SKETCH>(a.L, a.signs, St, atab, a.inv_sqrt_d, a.status,
                        [&](int lane, double (&x)[D / 32]) { load_vec<D / 32>(src, lane, x); },
                        is_key, rbuf, codes, bits, s16_out, rn16_out);
 }
@@ -140,12 +140,15 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
   const int bw = L.bw;
   const int64_t n = (int64_t)a.nA + a.nB;    // (uniform; a ragged launch takes its counts per unit)
   if (a.rows == nullptr && n == 0) return;
+  __shared__ double2 atab[kAngleTableEntries];
+  angle_tables(1 << L.b_theta, atab, threadIdx.x, blockDim.x);
+  __syncthreads();
   // S^T in shared memory when it fits: the sign loop then waits on shared
   // memory instead of a chain of L2 round trips (the decode-step eviction
   // encodes one token per unit, so latency is all there is).
   const float* St = a.St;
+  float* sst = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(smem) + st_offset(D, warps));
   if (st_staged(D, L.m)) {
-    float* sst = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(smem) + st_offset(D, warps));
     async_copy_g2s(sst, a.St, D * L.m * 4);
     async_copy_wait();
     __syncthreads();
@@ -192,12 +195,15 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
         ksrc = a.src_k + ((int64_t)unit * a.src_tokens + (e - us.nA)) * D;
         vsrc = a.src_v + ((int64_t)unit * a.src_tokens + (e - us.nA)) * D;
       }
-      encode_vector<D, false>(a, St, ksrc, true, rbuf + s * D, kc + s * P, kb + s * 8, sc + s * 4,
+      encode_vector<D, false>(a, St, atab, ksrc, true, rbuf + s * D, kc + s * P, kb + s * 8, sc + s * 4,
                               sc + s * 4 + 1);
-      encode_vector<D>(a, St, vsrc, false, nullptr, vc + s * P, nullptr, sc + s * 4 + 2, nullptr);
+      encode_vector<D>(a, St, atab, vsrc, false, nullptr, vc + s * P, nullptr, sc + s * 4 + 2, nullptr);
     }
-    // the four keys' sign words in one pass over S^T
-    if (L.m <= 128) qjl_sketch_block<D, 4, 4>(L.m, St, rbuf, inr, kb, 8);
+    // the four keys' sign words in one pass over S^T (shared-memory loads
+    // at fixed offsets for the staged m = 64 and m = 128)
+    if (st_staged(D, L.m) && L.m == 128) qjl_sketch_block<D, 4, 4, 128>(128, sst, rbuf, inr, kb, 8);
+    else if (st_staged(D, L.m) && L.m == 64) qjl_sketch_block<D, 4, 2, 64>(64, sst, rbuf, inr, kb, 8);
+    else if (L.m <= 128) qjl_sketch_block<D, 4, 4>(L.m, St, rbuf, inr, kb, 8);
     else qjl_sketch_block<D, 4, 8>(L.m, St, rbuf, inr, kb, 8);
     __syncwarp();
 
@@ -209,10 +215,10 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
       const int e = ch / 4, tig = ch % 4;
       const int l = 4 * (2 * c + e) + tig;
       uint32_t val, mask;
-      chunk_word(w, 2 * L.pt, bw, [&](int qi, uint32_t* out) {
-        const int h = qi / L.pt, k = qi % L.pt, s = e + 2 * h;
+      chunk_word(w, 2 * (P / 4), bw, [&](int qi, uint32_t* out) {
+        const int h = qi / (P / 4), k = qi % (P / 4), s = e + 2 * h;
         if (!inr[s]) return false;
-        *out = kc[s * P + tig * L.pt + k];
+        *out = kc[s * P + tig * (P / 4) + k];
         return true;
       }, val, mask);
       merge_word(reinterpret_cast<uint32_t*>(tb + L.off_kc + lane_word_offset(w, l, L.kwt)), val, mask);
@@ -223,10 +229,10 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
       const int e = ch / 4, tig = ch % 4;
       const int l = 4 * (2 * c + e) + tig;
       uint32_t val, mask;
-      chunk_word(w, 2 * L.pt, bw, [&](int qi, uint32_t* out) {
-        const int h = qi / L.pt, k = qi % L.pt, s = e + 2 * h;
+      chunk_word(w, 2 * (P / 4), bw, [&](int qi, uint32_t* out) {
+        const int h = qi / (P / 4), k = qi % (P / 4), s = e + 2 * h;
         if (!inr[s]) return false;
-        *out = vc[s * P + tig * L.pt + k];
+        *out = vc[s * P + tig * (P / 4) + k];
         return true;
       }, val, mask);
       merge_word(reinterpret_cast<uint32_t*>(tb + L.off_vc + lane_word_offset(w, l, L.vwt)), val, mask);
@@ -296,6 +302,9 @@ __global__ void __launch_bounds__(2 * D) encode_small_kernel(EncodeArgs a) {
   uint16_t* sc = reinterpret_cast<uint16_t*>(bits + 4);        // s16_k, rn16, s16_v
   float* sst = reinterpret_cast<float*>(sm) + small_st_offset(D) / 4;   // S^T [D][m]
   async_copy_g2s(sst, a.St, D * L.m * 4);      // lands while the rotation and polar steps run
+  __shared__ double2 atab[kAngleTableEntries];
+  angle_tables(1 << L.b_theta, atab, tid, blockDim.x);
+  __syncthreads();
   // Launched as a programmatic dependent of the kernel before it: S^T (set
   // at cache creation) may be fetched early, the inputs only once that
   // kernel has finished.
@@ -358,10 +367,12 @@ __global__ void __launch_bounds__(2 * D) encode_small_kernel(EncodeArgs a) {
   // ---- polar (even threads own pair el / 2) -------------------------------
   const double y1 = __shfl_xor_sync(kFull, x, 1);
   const bool ev = !(el & 1);
-  double rho = 0.0, th = 0.0;
+  const int nt = 1 << L.b_theta;
+  double rho = 0.0;
+  int ct = 0;
   if (ev) {
     rho = __dsqrt_rn(__dadd_rn(__dmul_rn(x, x), __dmul_rn(y1, y1)));
-    th = atan2(y1, x);
+    ct = angle_code(x, y1, nt, atab);
   }
   double mr = rho;
 #pragma unroll
@@ -378,14 +389,12 @@ __global__ void __launch_bounds__(2 * D) encode_small_kernel(EncodeArgs a) {
   }
   const double s16 = f16_bits_to_f64(s16b);
   const bool zero = (s16 == 0.0);
-  const int Lr = (1 << L.b_r) - 1, nt = 1 << L.b_theta;
-  int cr = 0, ct = 0;
+  const int Lr = (1 << L.b_r) - 1;
+  int cr = 0;
   if (ev) {
     const double tr = __dmul_rn(__ddiv_rn(rho, zero ? 1.0 : s16), (double)Lr);
     const int c = (int)rint(tr);
     cr = c < 0 ? 0 : (c > Lr ? Lr : c);
-    const double tt = __ddiv_rn(__dmul_rn(th, (double)nt), kTwoPi);
-    ct = ((int)rint(tt)) & (nt - 1);
     if (zero) { cr = 0; ct = 0; }
     codes[team * P + el / 2] = (uint8_t)((cr << L.b_theta) | ct);
   }
@@ -395,11 +404,9 @@ __global__ void __launch_bounds__(2 * D) encode_small_kernel(EncodeArgs a) {
   double ss = 0.0;
   if (team == 0 && ev) {
     const double rh = __ddiv_rn(__dmul_rn((double)cr, s16), (double)Lr);
-    const double ang = __ddiv_rn(__dmul_rn((double)ct, kTwoPi), (double)nt);
-    double sn, cs;
-    sincos(ang, &sn, &cs);
-    const double r0 = __dsub_rn(x, __dmul_rn(rh, cs));
-    const double r1 = __dsub_rn(y1, __dmul_rn(rh, sn));
+    const double2 csn = atab[angle_cs_offset(nt) + ct];     // cos, sin of c_theta 2 pi / nt
+    const double r0 = __dsub_rn(x, __dmul_rn(rh, csn.x));
+    const double r1 = __dsub_rn(y1, __dmul_rn(rh, csn.y));
     xb[el] = r0;
     xb[el + 1] = r1;
     ss = __dadd_rn(__dmul_rn(r0, r0), __dmul_rn(r1, r1));
@@ -450,9 +457,9 @@ __global__ void __launch_bounds__(2 * D) encode_small_kernel(EncodeArgs a) {
   for (int q = tid; q < 4 * L.kwt; q += blockDim.x) {
     const int tg = q / L.kwt, w = q % L.kwt;
     uint32_t val, mask;
-    chunk_word(w, 2 * L.pt, bw, [&](int qi, uint32_t* out) {
-      if (qi / L.pt != h) return false;
-      *out = codes[tg * L.pt + qi % L.pt];
+    chunk_word(w, 2 * (P / 4), bw, [&](int qi, uint32_t* out) {
+      if (qi / (P / 4) != h) return false;
+      *out = codes[tg * (P / 4) + qi % (P / 4)];
       return true;
     }, val, mask);
     merge_atomic(tb + L.off_kc + lane_word_offset(w, 4 * gid + tg, L.kwt), val, mask);
@@ -461,9 +468,9 @@ __global__ void __launch_bounds__(2 * D) encode_small_kernel(EncodeArgs a) {
   for (int q = tid; q < 4 * L.vwt; q += blockDim.x) {
     const int tg = q / L.vwt, w = q % L.vwt;
     uint32_t val, mask;
-    chunk_word(w, 2 * L.pt, bw, [&](int qi, uint32_t* out) {
-      if (qi / L.pt != h) return false;
-      *out = codes[P + tg * L.pt + qi % L.pt];
+    chunk_word(w, 2 * (P / 4), bw, [&](int qi, uint32_t* out) {
+      if (qi / (P / 4) != h) return false;
+      *out = codes[P + tg * (P / 4) + qi % (P / 4)];
       return true;
     }, val, mask);
     merge_atomic(tb + L.off_vc + lane_word_offset(w, 4 * gid + tg, L.vwt), val, mask);

@@ -22,6 +22,57 @@ __device__ __forceinline__ double f16_bits_to_f64(uint16_t h) {
   return (double)__half2float(__ushort_as_half(h));
 }
 
+// Angle tables of a block (nt = 2^b_theta codes), built once by
+// angle_tables before the block's first encode:
+//   bnd[0]      (cos, sin)(pi / nt): the half-sector rotation
+//   bnd[1 + j]  (cos, sin)(2 pi (j + 1) / nt), j < nt/4 - 1: the sector
+//               boundaries inside the first quadrant
+//   cs[c]       (cos, sin)(c 2 pi / nt) as the residual step computes them,
+//               at angle_cs_offset(nt) + c
+constexpr int kMaxAngleCodes = 128;
+constexpr int kAngleTableEntries = kMaxAngleCodes / 4 + kMaxAngleCodes;
+
+__host__ __device__ constexpr int angle_cs_offset(int nt) { return nt >= 4 ? nt / 4 : 1; }
+
+__device__ __forceinline__ void angle_tables(int nt, double2* tab, int tid, int nthreads) {
+  const int nb = angle_cs_offset(nt);
+  for (int e = tid; e < nb + nt; e += nthreads) {
+    double sn, cs;
+    if (e < nb) {
+      if (e == 0) sincospi(1.0 / (double)nt, &sn, &cs);
+      else sincospi(2.0 * (double)e / (double)nt, &sn, &cs);
+    } else {
+      const int c = e - nb;
+      sincos(__ddiv_rn(__dmul_rn((double)c, kTwoPi), (double)nt), &sn, &cs);
+    }
+    tab[e] = make_double2(cs, sn);
+  }
+}
+
+// The angle code of (x, y): the nearest of the nt directions c 2 pi / nt,
+// i.e. floor(theta nt / (2 pi) + 1/2) mod nt for theta = atan2(y, x).  The
+// pair is rotated by half a sector, its quadrant read off the signs, and its
+// sector inside the quadrant found by cross products with the boundary
+// directions; rounding moves a decision only for pairs within about 1e-15
+// of a sector boundary (the origin gets code 0, as atan2(0, 0) = 0 does).
+__device__ __forceinline__ int angle_code(double x, double y, int nt, const double2* bnd) {
+  const double2 r = bnd[0];
+  const double xr = fma(x, r.x, -__dmul_rn(y, r.y));
+  const double yr = fma(x, r.y, __dmul_rn(y, r.x));
+  int q;
+  double u, v;                               // the pair turned into the first quadrant
+  if (yr >= 0.0 && xr > 0.0) { q = 0; u = xr; v = yr; }
+  else if (yr > 0.0) { q = 1; u = yr; v = -xr; }
+  else if (xr < 0.0) { q = 2; u = -xr; v = -yr; }
+  else if (yr < 0.0) { q = 3; u = -yr; v = xr; }
+  else return 0;                             // the origin
+  if (nt == 2) return q >> 1;
+  const int per = nt >> 2;                   // sectors per quadrant
+  int j = 0;
+  while (j < per - 1 && fma(bnd[1 + j].x, v, -__dmul_rn(bnd[1 + j].y, u)) >= 0.0) ++j;
+  return (q * per + j) & (nt - 1);
+}
+
 template <int E>
 __device__ __forceinline__ void load_vec(const __half* p, int lane, double (&x)[E]) {
   const __half* q = p + lane * E;
@@ -47,12 +98,14 @@ __device__ __forceinline__ void load_vec(const __half* p, int lane, double (&x)[
 // and the raw fp16 scalars.  Whole warp; returns nothing else.
 // `load(lane, x)` fills the lane's D/32 consecutive input elements (padded
 // coordinates read as 0).  `L` supplies b_r, b_theta and m; `St` is S^T
-// [D, m] (global or shared memory); `signs` the rotation diagonal.  With
+// [D, m] (global or shared memory); `signs` the rotation diagonal; `atab`
+// the block's angle tables (angle_tables).  With
 // SKETCH false a key stops after its residual (left in rbuf[0..D)) and its
 // norm; qjl_sketch_block then forms the sign words of several keys at once.
 template <int D, bool SKETCH = true, typename Loader>
 __device__ __forceinline__ void encode_vector_any(const Layout& L, const double* signs,
-                                                  const float* St, double inv_sqrt_d, int* status,
+                                                  const float* St, const double2* atab,
+                                                  double inv_sqrt_d, int* status,
                                                   Loader load, bool is_key, double* rbuf,
                                                   uint8_t* codes, uint32_t* bits,
                                                   uint16_t* s16_out, uint16_t* rn16_out) {
@@ -90,14 +143,15 @@ __device__ __forceinline__ void encode_vector_any(const Layout& L, const double*
 #pragma unroll
   for (int i = 0; i < E; ++i) x[i] = __dmul_rn(x[i], inv_sqrt_d);
 
-  // ---- polar: rho, theta per pair; scale s16 = fp16(max rho) ------------
-  double rho[PL], th[PL];
+  // ---- polar: rho and the angle code per pair; scale s16 = fp16(max rho) --
+  double rho[PL];
+  int ct[PL];
   double smax = 0.0;
 #pragma unroll
   for (int k = 0; k < PL; ++k) {
     const double y0 = x[2 * k], y1 = x[2 * k + 1];
     rho[k] = __dsqrt_rn(__dadd_rn(__dmul_rn(y0, y0), __dmul_rn(y1, y1)));
-    th[k] = atan2(y1, y0);
+    ct[k] = angle_code(y0, y1, nt, atab);
     smax = fmax(smax, rho[k]);
   }
 #pragma unroll
@@ -111,14 +165,12 @@ __device__ __forceinline__ void encode_vector_any(const Layout& L, const double*
   const bool zero = (s16 == 0.0);
 
   // ---- codes ---------------------------------------------------------------
-  int cr[PL], ct[PL];
+  int cr[PL];
 #pragma unroll
   for (int k = 0; k < PL; ++k) {
     const double tr = __dmul_rn(__ddiv_rn(rho[k], zero ? 1.0 : s16), (double)Lr);
     const int c = (int)rint(tr);
     cr[k] = c < 0 ? 0 : (c > Lr ? Lr : c);
-    const double tt = __ddiv_rn(__dmul_rn(th[k], (double)nt), kTwoPi);
-    ct[k] = ((int)rint(tt)) & (nt - 1);
     if (zero) { cr[k] = 0; ct[k] = 0; }
     codes[lane * PL + k] = (uint8_t)((cr[k] << L.b_theta) | ct[k]);
   }
@@ -131,11 +183,9 @@ __device__ __forceinline__ void encode_vector_any(const Layout& L, const double*
 #pragma unroll
     for (int k = 0; k < PL; ++k) {
       const double rh = __ddiv_rn(__dmul_rn((double)cr[k], s16), (double)Lr);
-      const double ang = __ddiv_rn(__dmul_rn((double)ct[k], kTwoPi), (double)nt);
-      double sn, cs;
-      sincos(ang, &sn, &cs);
-      r[2 * k] = __dsub_rn(x[2 * k], __dmul_rn(rh, cs));
-      r[2 * k + 1] = __dsub_rn(x[2 * k + 1], __dmul_rn(rh, sn));
+      const double2 csn = atab[angle_cs_offset(nt) + ct[k]];   // cos, sin of c_theta 2 pi / nt
+      r[2 * k] = __dsub_rn(x[2 * k], __dmul_rn(rh, csn.x));
+      r[2 * k + 1] = __dsub_rn(x[2 * k + 1], __dmul_rn(rh, csn.y));
       ss = __dadd_rn(ss, __dadd_rn(__dmul_rn(r[2 * k], r[2 * k]), __dmul_rn(r[2 * k + 1], r[2 * k + 1])));
     }
 #pragma unroll
@@ -190,9 +240,11 @@ __device__ __forceinline__ void encode_vector_any(const Layout& L, const double*
 // live[v].  Lane outputs i = lane + 32 k as in encode_vector_any; each S^T
 // value is loaded and widened once and feeds NV fp64 FMAs, and each output
 // still sums over j in ascending order (the same FMAs as one vector alone).
-template <int D, int NV, int NK>
-__device__ __forceinline__ void qjl_sketch_block(int m, const float* St, const double* rbuf,
+// MC: m when known at compile time (0: the run-time m).
+template <int D, int NV, int NK, int MC = 0>
+__device__ __forceinline__ void qjl_sketch_block(int m_rt, const float* St, const double* rbuf,
                                                  const bool (&live)[NV], uint32_t* bits, int bits_stride) {
+  const int m = MC ? MC : m_rt;
   const int lane = threadIdx.x & 31;
   double acc[NV][NK];
 #pragma unroll

@@ -319,6 +319,9 @@ __global__ void __launch_bounds__(256) vec_encode_kernel(const VecEncodeArgs a) 
   uint8_t* codes = reinterpret_cast<uint8_t*>(vsmem + warps * D) + warp * (P + 64);
   uint32_t* bits = reinterpret_cast<uint32_t*>(codes + P);      // 8 words
   uint16_t* sc = reinterpret_cast<uint16_t*>(codes + P + 32);   // s16, rn16
+  __shared__ double2 atab[enc::kAngleTableEntries];
+  enc::angle_tables(1 << a.L.b_theta, atab, threadIdx.x, blockDim.x);
+  __syncthreads();
   for (int64_t v = (int64_t)blockIdx.x * warps + warp; v < a.count; v += (int64_t)gridDim.x * warps) {
     const float* src = a.x + v * a.dim;
     auto load = [&](int ln, double (&x)[E]) {
@@ -330,7 +333,7 @@ __global__ void __launch_bounds__(256) vec_encode_kernel(const VecEncodeArgs a) 
     };
     if (lane < 8) bits[lane] = 0u;
     __syncwarp();
-    encode_vector_any<D>(a.L, a.signs, a.St, a.inv_sqrt_d, a.status, load, true, rbuf, codes, bits,
+    encode_vector_any<D>(a.L, a.signs, a.St, atab, a.inv_sqrt_d, a.status, load, true, rbuf, codes, bits,
                          sc, sc + 1);
     const int64_t g = a.start + v;
     // group g / 32, chunk-major: byte b of vector g at chunk b / 16
