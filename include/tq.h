@@ -201,6 +201,13 @@ tq_status tq_evict_window_rows(tq_cache* cache, const void* k_new, const void* v
  *   out    device fp32 [B, Hq, d]
  *   softmax_scale  sigma; 0 selects 1/sqrt(d)
  * With no valid token at all, out is zero.
+ * Ordering: the call's first kernel (q-prep) is a programmatic dependent
+ * launch of whatever the stream ran before it, and it reads q before it
+ * waits for that kernel.  So the kernel that writes q must not signal its
+ * dependents early (griddepcontrol.launch_dependents /
+ * cudaTriggerProgrammaticLaunchCompletion before its writes of q): ordinary
+ * kernels, PyTorch's included, never do, and the library's own kernels do
+ * not write q.  Everything else the call reads is read after the wait.
  */
 tq_status tq_decode_attention(tq_cache* cache, const void* q, float* out,
                               float softmax_scale, cudaStream_t stream);
