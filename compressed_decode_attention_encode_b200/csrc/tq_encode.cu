@@ -146,10 +146,12 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
   // S^T in shared memory when it fits: the sign loop then waits on shared
   // memory instead of a chain of L2 round trips (the decode-step eviction
   // encodes one token per unit, so latency is all there is).
+  // (m = 64 or 128: S^T in lane order, read by qjl_sketch_lanes)
+  const bool lanes = st_staged(D, L.m) && (L.m == 64 || L.m == 128);
   const float* St = a.St;
   float* sst = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(smem) + st_offset(D, warps));
   if (st_staged(D, L.m)) {
-    async_copy_g2s(sst, a.St, D * L.m * 4);
+    async_copy_g2s(sst, lanes ? a.Stl : a.St, D * L.m * 4);
     async_copy_wait();
     __syncthreads();
     St = sst;
@@ -199,10 +201,10 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
                               sc + s * 4 + 1);
       encode_vector<D>(a, St, atab, vsrc, false, nullptr, vc + s * P, nullptr, sc + s * 4 + 2, nullptr);
     }
-    // the four keys' sign words in one pass over S^T (shared-memory loads
-    // at fixed offsets for the staged m = 64 and m = 128)
-    if (st_staged(D, L.m) && L.m == 128) qjl_sketch_block<D, 4, 4, 128>(128, sst, rbuf, inr, kb, 8);
-    else if (st_staged(D, L.m) && L.m == 64) qjl_sketch_block<D, 4, 2, 64>(64, sst, rbuf, inr, kb, 8);
+    // the four keys' sign words in one pass over S^T (lane order when staged
+    // for m = 64 or 128)
+    if (lanes && L.m == 128) qjl_sketch_lanes<D, 4, 4>(sst, rbuf, inr, kb, 8);
+    else if (lanes) qjl_sketch_lanes<D, 4, 2>(sst, rbuf, inr, kb, 8);
     else if (L.m <= 128) qjl_sketch_block<D, 4, 4>(L.m, St, rbuf, inr, kb, 8);
     else qjl_sketch_block<D, 4, 8>(L.m, St, rbuf, inr, kb, 8);
     __syncwarp();

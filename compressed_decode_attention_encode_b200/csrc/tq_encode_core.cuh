@@ -283,5 +283,58 @@ __device__ __forceinline__ void qjl_sketch_block(int m_rt, const float* St, cons
 }
 
 
+// The same sign words from S^T in lane order (stl: [D][32][NK] floats in
+// shared memory, element (j, l, k) = S^T[j][l + 32 k], m = 32 NK): each
+// lane reads its NK values of a row with one vector load and two residual
+// values of a key with one; the FMAs and their order are those of
+// qjl_sketch_block.
+template <int D, int NV, int NK>
+__device__ __forceinline__ void qjl_sketch_lanes(const float* stl, const double* rbuf, const bool (&live)[NV],
+                                                 uint32_t* bits, int bits_stride) {
+  static_assert(NK == 2 || NK == 4, "m = 64 or 128");
+  const int lane = threadIdx.x & 31;
+  double acc[NV][NK];
+#pragma unroll
+  for (int v = 0; v < NV; ++v)
+#pragma unroll
+    for (int k = 0; k < NK; ++k) acc[v][k] = 0.0;
+  for (int j0 = 0; j0 < D; j0 += 2) {
+    double sv[2][NK];
+#pragma unroll
+    for (int jj = 0; jj < 2; ++jj) {
+      const float* row = stl + ((j0 + jj) * 32 + lane) * NK;
+      if constexpr (NK == 4) {
+        const float4 f = *reinterpret_cast<const float4*>(row);
+        sv[jj][0] = (double)f.x;
+        sv[jj][1] = (double)f.y;
+        sv[jj][2] = (double)f.z;
+        sv[jj][3] = (double)f.w;
+      } else {
+        const float2 f = *reinterpret_cast<const float2*>(row);
+        sv[jj][0] = (double)f.x;
+        sv[jj][1] = (double)f.y;
+      }
+    }
+#pragma unroll
+    for (int v = 0; v < NV; ++v) {
+      const double2 r2 = *reinterpret_cast<const double2*>(rbuf + v * D + j0);
+#pragma unroll
+      for (int k = 0; k < NK; ++k) {
+        acc[v][k] = fma(sv[0][k], r2.x, acc[v][k]);
+        acc[v][k] = fma(sv[1][k], r2.y, acc[v][k]);
+      }
+    }
+  }
+#pragma unroll
+  for (int v = 0; v < NV; ++v) {
+#pragma unroll
+    for (int k = 0; k < NK; ++k) {
+      const unsigned word = __ballot_sync(kFull, acc[v][k] >= 0.0);
+      if (lane == 0 && live[v]) bits[v * bits_stride + k] = word;
+    }
+  }
+  __syncwarp();
+}
+
 }  // namespace enc
 }  // namespace tq

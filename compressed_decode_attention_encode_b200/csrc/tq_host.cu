@@ -57,7 +57,7 @@ bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 }  // namespace
 
 struct WsLayout {
-  size_t status, signs, S, St, q, part, gate, gate_max, rows, total;
+  size_t status, signs, Stl, St, q, part, gate, gate_max, rows, total;
   QBufsLayout ql;               // query transforms, at offset q
 };
 
@@ -69,7 +69,7 @@ static WsLayout ws_layout(const tq_config& c) {
   size_t off = 0;
   w.status = off; off += kAlign;
   w.signs = off;  off += round_up(sizeof(double) * c.head_dim, kAlign);
-  w.S = off;      off += round_up(sizeof(float) * c.head_dim * c.qjl_bits, kAlign);
+  w.Stl = off;    off += round_up(sizeof(float) * c.head_dim * 32 * ((c.qjl_bits + 31) / 32), kAlign);
   w.St = off;     off += round_up(sizeof(float) * c.head_dim * c.qjl_bits, kAlign);
   w.ql = qbufs_layout(heads, c.head_dim, c.qjl_bits);
   w.q = off;      off += w.ql.total;
@@ -139,7 +139,7 @@ struct tq_cache {
   }
   int* status() const { return (int*)(ws + W.status); }
   double* signs() const { return (double*)(ws + W.signs); }
-  float* S() const { return (float*)(ws + W.S); }
+  float* Stl() const { return (float*)(ws + W.Stl); }
   float* St() const { return (float*)(ws + W.St); }
 };
 
@@ -305,16 +305,20 @@ tq_status tq_cache_create(const tq_config* cfg, void* hot_mem, void* cold_mem,
   }
   const int d = cfg->head_dim, m = cfg->qjl_bits;
   std::vector<double> signs(d);
-  std::vector<float> S((size_t)m * d), St((size_t)m * d);
+  const int nk = (m + 31) / 32;
+  std::vector<float> S((size_t)m * d), St((size_t)m * d), Stl((size_t)d * 32 * nk, 0.f);
   gen_signs(cfg->seed, d, signs.data());
   gen_qjl(cfg->seed, m, d, S.data());
   for (int i = 0; i < m; ++i)
-    for (int j = 0; j < d; ++j) St[(size_t)j * m + i] = S[(size_t)i * d + j];
+    for (int j = 0; j < d; ++j) {
+      St[(size_t)j * m + i] = S[(size_t)i * d + j];
+      Stl[((size_t)j * 32 + i % 32) * nk + i / 32] = S[(size_t)i * d + j];
+    }
   // Pageable sources: cudaMemcpyAsync returns once the data is staged, so
   // the vectors may be released when the calls return.
   cudaError_t e = cudaMemsetAsync(c->status(), 0, kAlign, stream);
   if (e == cudaSuccess) e = cudaMemcpyAsync(c->signs(), signs.data(), sizeof(double) * d, cudaMemcpyHostToDevice, stream);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(c->S(), S.data(), sizeof(float) * S.size(), cudaMemcpyHostToDevice, stream);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(c->Stl(), Stl.data(), sizeof(float) * Stl.size(), cudaMemcpyHostToDevice, stream);
   if (e == cudaSuccess) e = cudaMemcpyAsync(c->St(), St.data(), sizeof(float) * St.size(), cudaMemcpyHostToDevice, stream);
   if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
   if (e != cudaSuccess) {
@@ -347,6 +351,7 @@ static EncodeArgs base_encode_args(tq_cache* c) {
   a.L = c->L;
   a.signs = c->signs();
   a.St = c->St();
+  a.Stl = c->Stl();
   a.status = c->status();
   a.inv_sqrt_d = 1.0 / std::sqrt((double)c->cfg.head_dim);
   return a;

@@ -159,6 +159,7 @@ struct EncodeArgs {
   Layout L;
   const double* signs;      // [d]
   const float* St;          // S transposed, [d, m]
+  const float* Stl;         // S^T by lane: [d][32][ceil(m/32)], element (j, l, k) = S^T[j][l + 32 k]
   int* status;
   double inv_sqrt_d;        // 1 / sqrt(d), correctly rounded on the host
   // Steady-state eviction (per-token path only): after reading ring slot
