@@ -141,7 +141,7 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
   const int64_t n = (int64_t)a.nA + a.nB;    // (uniform; a ragged launch takes its counts per unit)
   if (a.rows == nullptr && n == 0) return;
   __shared__ double2 atab[kAngleTableEntries];
-  angle_tables(1 << L.b_theta, atab, threadIdx.x, blockDim.x);
+  angle_tables(1 << L.b_theta, a.atab, atab, threadIdx.x, blockDim.x);
   __syncthreads();
   // S^T in shared memory when it fits: the sign loop then waits on shared
   // memory instead of a chain of L2 round trips (the decode-step eviction
@@ -287,10 +287,10 @@ __global__ void __launch_bounds__(2 * D) encode_small_kernel(EncodeArgs a) {
   constexpr int P = D / 2;
   constexpr int NW = D / 32;                 // warps per team
   const Layout& L = a.L;
-  const int64_t n = a.promo ? (int64_t)(kPromoMax + a.n_new)
-                  : a.rows ? (int64_t)a.n_max : (int64_t)a.nA + a.nB;
-  const int unit = (int)(blockIdx.x / n);
-  const int64_t e = blockIdx.x % n;
+  // (a few tokens per unit: 32-bit index arithmetic)
+  const int n = a.promo ? kPromoMax + a.n_new : a.rows ? a.n_max : (int)(a.nA + a.nB);
+  const int unit = (int)blockIdx.x / n;
+  const int e = (int)blockIdx.x % n;
   const int tid = threadIdx.x, team = tid / D, el = tid % D;
   const int lane = tid & 31, wt = el >> 5;
   // A following launch that opted in (the decode step's q-prep, which does
@@ -305,7 +305,7 @@ __global__ void __launch_bounds__(2 * D) encode_small_kernel(EncodeArgs a) {
   float* sst = reinterpret_cast<float*>(sm) + small_st_offset(D) / 4;   // S^T [D][m]
   async_copy_g2s(sst, a.St, D * L.m * 4);      // lands while the rotation and polar steps run
   __shared__ double2 atab[kAngleTableEntries];
-  angle_tables(1 << L.b_theta, atab, tid, blockDim.x);
+  angle_tables(1 << L.b_theta, a.atab, atab, tid, blockDim.x);
   __syncthreads();
   // Launched as a programmatic dependent of the kernel before it: S^T (set
   // at cache creation) may be fetched early, the inputs only once that
@@ -429,12 +429,20 @@ __global__ void __launch_bounds__(2 * D) encode_small_kernel(EncodeArgs a) {
       if ((rnb & 0x7c00u) == 0x7c00u) atomicOr(a.status, kStatusRange);
       sc[1] = rnb;
     }
+    // (S r)_i as four interleaved partial sums (j mod 4), so the FMA
+    // chain is a quarter as long; a sign can differ from another summation
+    // order only within float64 rounding of zero
     for (int i0 = 0; i0 < L.m; i0 += D) {
       const int i = i0 + el;
       double acc = 0.0;
       if (i < L.m) {
+        double p4[4] = {0.0, 0.0, 0.0, 0.0};
 #pragma unroll 8
-        for (int j = 0; j < D; ++j) acc = fma((double)sst[j * L.m + i], xb[j], acc);
+        for (int j = 0; j < D; j += 4) {
+#pragma unroll
+          for (int t = 0; t < 4; ++t) p4[t] = fma((double)sst[(j + t) * L.m + i], xb[j + t], p4[t]);
+        }
+        acc = __dadd_rn(__dadd_rn(p4[0], p4[1]), __dadd_rn(p4[2], p4[3]));
       }
       const unsigned word = __ballot_sync(kFull, i < L.m && acc >= 0.0);
       if (lane == 0 && i < L.m) bits[i >> 5] = word;
@@ -455,42 +463,51 @@ __global__ void __launch_bounds__(2 * D) encode_small_kernel(EncodeArgs a) {
     atomicOr(w, val & mask);
   };
   const int bw = L.bw;
-  // K code words: lanes (gid, tig), codes q of half h: pair tig * pt + q % pt
-  for (int q = tid; q < 4 * L.kwt; q += blockDim.x) {
-    const int tg = q / L.kwt, w = q % L.kwt;
-    uint32_t val, mask;
-    chunk_word(w, 2 * (P / 4), bw, [&](int qi, uint32_t* out) {
-      if (qi / (P / 4) != h) return false;
-      *out = codes[tg * (P / 4) + qi % (P / 4)];
-      return true;
-    }, val, mask);
-    merge_atomic(tb + L.off_kc + lane_word_offset(w, 4 * gid + tg, L.kwt), val, mask);
-  }
-  // V code words: the K layout
-  for (int q = tid; q < 4 * L.vwt; q += blockDim.x) {
-    const int tg = q / L.vwt, w = q % L.vwt;
-    uint32_t val, mask;
-    chunk_word(w, 2 * (P / 4), bw, [&](int qi, uint32_t* out) {
-      if (qi / (P / 4) != h) return false;
-      *out = codes[P + tg * (P / 4) + qi % (P / 4)];
-      return true;
-    }, val, mask);
-    merge_atomic(tb + L.off_vc + lane_word_offset(w, 4 * gid + tg, L.vwt), val, mask);
-  }
-  // sign words: lanes (gid, tig); m/4 signs per (token, tig), local sign j
-  // at chunk bit sign_chunk_bit(j, h, m)
-  const int qb = L.m / 4;
-  for (int q = tid; q < 4 * L.sw; q += blockDim.x) {
-    const int tg = q / L.sw, w = q % L.sw;
-    uint32_t val = 0u, mask = 0u;
-    for (int j = 0; j < qb; ++j) {
-      const int bit = sign_chunk_bit(j, h, L.m) - 32 * w;
-      if (bit < 0 || bit >= 32) continue;
-      const int i = tg * qb + j;
-      val |= ((bits[i >> 5] >> (i & 31)) & 1u) << bit;
-      mask |= 1u << bit;
+  constexpr int PT = P / 4;                  // pairs per lane group and token
+  const uint32_t cm = (1u << bw) - 1u;
+  const int nwarps = blockDim.x >> 5, warp = tid >> 5;
+  // One warp per (plane, lane group tg) and word: lane k holds this token's
+  // code k (pair tg * PT + k, at bit (h PT + k) bw of the group's stream) or
+  // sign bit k, and the word's bits and mask come from two OR-reductions.
+  // Jobs 0-3: key codes, 4-7: value codes, 8-11: sign words.
+  for (int job = warp; job < 12; job += nwarps) {
+    const int tg = job & 3;
+    if (job < 8) {
+      const bool vplane = job >= 4;
+      const int nw = vplane ? L.vwt : L.kwt;
+      uint8_t* plane = tb + (vplane ? L.off_vc : L.off_kc);
+      const uint32_t c = lane < PT ? codes[(vplane ? P : 0) + tg * PT + lane] : 0u;
+      const int bit0 = (h * PT + lane) * bw;
+      const int w_lo = (h * PT * bw) >> 5, w_hi = ((h + 1) * PT * bw - 1) >> 5;
+      for (int w = w_lo; w <= w_hi; ++w) {
+        uint32_t v = 0u, mk = 0u;
+        const int b = bit0 - 32 * w;
+        if (lane < PT && b > -bw && b < 32) {
+          v = b >= 0 ? c << b : c >> -b;
+          mk = b >= 0 ? cm << b : cm >> -b;
+        }
+        v = __reduce_or_sync(kFull, v);
+        mk = __reduce_or_sync(kFull, mk);
+        if (lane == 0) merge_atomic(plane + lane_word_offset(w, 4 * gid + tg, nw), v, mk);
+      }
+    } else {
+      // sign j of this token and lane group: canonical index tg * m/4 + j,
+      // chunk bit sign_chunk_bit(j, h, m)
+      const int qb = L.m / 4;
+      uint32_t bitv = 0u;
+      int pos = -1;
+      if (lane < qb) {
+        const int i = tg * qb + lane;
+        bitv = (bits[i >> 5] >> (i & 31)) & 1u;
+        pos = sign_chunk_bit(lane, h, L.m);
+      }
+      for (int w = 0; w < L.sw; ++w) {
+        const bool mine = pos >= 32 * w && pos < 32 * w + 32;
+        const uint32_t v = __reduce_or_sync(kFull, mine ? bitv << (pos - 32 * w) : 0u);
+        const uint32_t mk = __reduce_or_sync(kFull, mine ? 1u << (pos - 32 * w) : 0u);
+        if (lane == 0) merge_atomic(tb + L.off_ks + lane_word_offset(w, 4 * gid + tg, L.sw), v, mk);
+      }
     }
-    merge_atomic(tb + L.off_ks + lane_word_offset(w, 4 * gid + tg, L.sw), val, mask);
   }
   if (tid == 0) {
     uint16_t* ks = reinterpret_cast<uint16_t*>(tb + L.off_ksc);

@@ -22,31 +22,16 @@ __device__ __forceinline__ double f16_bits_to_f64(uint16_t h) {
   return (double)__half2float(__ushort_as_half(h));
 }
 
-// Angle tables of a block (nt = 2^b_theta codes), built once by
-// angle_tables before the block's first encode:
+// Angle tables (nt = 2^b_theta codes), built on the host when a handle is
+// created (angle_table_host) and copied into a block's shared memory by
+// angle_tables before its first encode:
 //   bnd[0]      (cos, sin)(pi / nt): the half-sector rotation
 //   bnd[1 + j]  (cos, sin)(2 pi (j + 1) / nt), j < nt/4 - 1: the sector
 //               boundaries inside the first quadrant
-//   cs[c]       (cos, sin)(c 2 pi / nt) as the residual step computes them,
-//               at angle_cs_offset(nt) + c
-constexpr int kMaxAngleCodes = 128;
-constexpr int kAngleTableEntries = kMaxAngleCodes / 4 + kMaxAngleCodes;
-
-__host__ __device__ constexpr int angle_cs_offset(int nt) { return nt >= 4 ? nt / 4 : 1; }
-
-__device__ __forceinline__ void angle_tables(int nt, double2* tab, int tid, int nthreads) {
-  const int nb = angle_cs_offset(nt);
-  for (int e = tid; e < nb + nt; e += nthreads) {
-    double sn, cs;
-    if (e < nb) {
-      if (e == 0) sincospi(1.0 / (double)nt, &sn, &cs);
-      else sincospi(2.0 * (double)e / (double)nt, &sn, &cs);
-    } else {
-      const int c = e - nb;
-      sincos(__ddiv_rn(__dmul_rn((double)c, kTwoPi), (double)nt), &sn, &cs);
-    }
-    tab[e] = make_double2(cs, sn);
-  }
+//   cs[c]       (cos, sin)(c 2 pi / nt), at angle_cs_offset(nt) + c: the
+//               dequantized directions of the residual step
+__device__ __forceinline__ void angle_tables(int nt, const double2* src, double2* tab, int tid, int nthreads) {
+  for (int e = tid; e < angle_cs_offset(nt) + nt; e += nthreads) tab[e] = src[e];
 }
 
 // The angle code of (x, y): the nearest of the nt directions c 2 pi / nt,

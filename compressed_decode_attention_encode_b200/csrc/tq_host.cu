@@ -57,7 +57,7 @@ bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 }  // namespace
 
 struct WsLayout {
-  size_t status, signs, Stl, St, q, part, gate, gate_max, rows, total;
+  size_t status, signs, Stl, St, atab, q, part, gate, gate_max, rows, total;
   QBufsLayout ql;               // query transforms, at offset q
 };
 
@@ -71,6 +71,7 @@ static WsLayout ws_layout(const tq_config& c) {
   w.signs = off;  off += round_up(sizeof(double) * c.head_dim, kAlign);
   w.Stl = off;    off += round_up(sizeof(float) * c.head_dim * 32 * ((c.qjl_bits + 31) / 32), kAlign);
   w.St = off;     off += round_up(sizeof(float) * c.head_dim * c.qjl_bits, kAlign);
+  w.atab = off;   off += round_up(sizeof(double) * 2 * kAngleTableEntries, kAlign);
   w.ql = qbufs_layout(heads, c.head_dim, c.qjl_bits);
   w.q = off;      off += w.ql.total;
   w.part = off;   off += round_up(sizeof(float) * units * (kSlotsCold + kSlotsHot) * G * (c.head_dim + 2), kAlign);
@@ -140,6 +141,7 @@ struct tq_cache {
   int* status() const { return (int*)(ws + W.status); }
   double* signs() const { return (double*)(ws + W.signs); }
   float* Stl() const { return (float*)(ws + W.Stl); }
+  double2* atab() const { return (double2*)(ws + W.atab); }
   float* St() const { return (float*)(ws + W.St); }
 };
 
@@ -319,6 +321,9 @@ tq_status tq_cache_create(const tq_config* cfg, void* hot_mem, void* cold_mem,
   cudaError_t e = cudaMemsetAsync(c->status(), 0, kAlign, stream);
   if (e == cudaSuccess) e = cudaMemcpyAsync(c->signs(), signs.data(), sizeof(double) * d, cudaMemcpyHostToDevice, stream);
   if (e == cudaSuccess) e = cudaMemcpyAsync(c->Stl(), Stl.data(), sizeof(float) * Stl.size(), cudaMemcpyHostToDevice, stream);
+  std::vector<double> atab(2 * kAngleTableEntries, 0.0);
+  angle_table_host(1 << cfg->b_theta, atab.data());
+  if (e == cudaSuccess) e = cudaMemcpyAsync(c->atab(), atab.data(), sizeof(double) * atab.size(), cudaMemcpyHostToDevice, stream);
   if (e == cudaSuccess) e = cudaMemcpyAsync(c->St(), St.data(), sizeof(float) * St.size(), cudaMemcpyHostToDevice, stream);
   if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
   if (e != cudaSuccess) {
@@ -352,6 +357,7 @@ static EncodeArgs base_encode_args(tq_cache* c) {
   a.signs = c->signs();
   a.St = c->St();
   a.Stl = c->Stl();
+  a.atab = c->atab();
   a.status = c->status();
   a.inv_sqrt_d = 1.0 / std::sqrt((double)c->cfg.head_dim);
   return a;

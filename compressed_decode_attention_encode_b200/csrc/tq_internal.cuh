@@ -2,6 +2,7 @@
 // Layout of the packed cold store, kernel argument blocks and launchers.
 #pragma once
 
+#include <cmath>
 #include <cstddef>
 #include <cstdint>
 #include <cuda_fp16.h>
@@ -76,6 +77,27 @@ __host__ __device__ inline int lane_word_offset(int w, int l, int nw) {
 __host__ __device__ inline int sign_chunk_bit(int j, int h, int m) {
   const int e = j & 3, hf = (j >> 2) & 1, s = j >> 3;
   return m == 128 ? 32 * h + 8 * e + 2 * s + hf : 8 * e + 4 * h + 2 * s + hf;
+}
+
+// Angle tables of the encoders (see angle_tables): at most 2^7 angle codes.
+constexpr int kMaxAngleCodes = 128;
+constexpr int kAngleTableEntries = kMaxAngleCodes / 4 + kMaxAngleCodes;
+
+__host__ __device__ constexpr int angle_cs_offset(int nt) { return nt >= 4 ? nt / 4 : 1; }
+
+// Host: the (cos, sin) entries for nt angle codes into out[2 e], out[2 e + 1]
+// (entries: the half-sector rotation, the first quadrant's inner sector
+// boundaries, then the nt code directions c 2 pi / nt).
+inline void angle_table_host(int nt, double* out) {
+  const double two_pi = 6.283185307179586476925286766559;
+  const int nb = angle_cs_offset(nt);
+  for (int e = 0; e < nb + nt; ++e) {
+    const double a = e == 0 ? two_pi / 2.0 / (double)nt
+                   : e < nb ? two_pi * (double)e / (double)nt
+                            : (double)(e - nb) * two_pi / (double)nt;
+    out[2 * e] = std::cos(a);
+    out[2 * e + 1] = std::sin(a);
+  }
 }
 
 __host__ __device__ inline Layout layout_of(int d, int b_r, int b_theta, int m, int64_t capacity) {
@@ -160,6 +182,7 @@ struct EncodeArgs {
   const double* signs;      // [d]
   const float* St;          // S transposed, [d, m]
   const float* Stl;         // S^T by lane: [d][32][ceil(m/32)], element (j, l, k) = S^T[j][l + 32 k]
+  const double2* atab;      // angle tables (angle_table_host)
   int* status;
   double inv_sqrt_d;        // 1 / sqrt(d), correctly rounded on the host
   // Steady-state eviction (per-token path only): after reading ring slot
@@ -443,6 +466,7 @@ struct VecEncodeArgs {
   Layout L;                 // d (padded), b_r, b_theta, m
   const double* signs;
   const float* St;          // [d, m]
+  const double2* atab;      // angle tables (angle_table_host)
   double inv_sqrt_d;
   int* status;
   uint8_t* codes;           // [n/32][d/32][32][16 B]: 32-vector groups, 16-byte chunks

@@ -319,8 +319,8 @@ __global__ void __launch_bounds__(256) vec_encode_kernel(const VecEncodeArgs a) 
   uint8_t* codes = reinterpret_cast<uint8_t*>(vsmem + warps * D) + warp * (P + 64);
   uint32_t* bits = reinterpret_cast<uint32_t*>(codes + P);      // 8 words
   uint16_t* sc = reinterpret_cast<uint16_t*>(codes + P + 32);   // s16, rn16
-  __shared__ double2 atab[enc::kAngleTableEntries];
-  enc::angle_tables(1 << a.L.b_theta, atab, threadIdx.x, blockDim.x);
+  __shared__ double2 atab[kAngleTableEntries];
+  enc::angle_tables(1 << a.L.b_theta, a.atab, atab, threadIdx.x, blockDim.x);
   __syncthreads();
   for (int64_t v = (int64_t)blockIdx.x * warps + warp; v < a.count; v += (int64_t)gridDim.x * warps) {
     const float* src = a.x + v * a.dim;
@@ -958,7 +958,7 @@ VecCodesLayout vec_codes_layout(int d, int64_t n) {
 }
 
 struct VecWsLayout {
-  size_t status, signs, St, A, qscale, part_s, part_i, total;
+  size_t status, signs, St, atab, A, qscale, part_s, part_i, total;
 };
 
 VecWsLayout vec_ws_layout(int d, int m, int max_q) {
@@ -967,6 +967,7 @@ VecWsLayout vec_ws_layout(int d, int m, int max_q) {
   w.status = off; off += kVAlign;
   w.signs = off;  off += vround(sizeof(double) * d);
   w.St = off;     off += vround(sizeof(float) * (size_t)d * m);
+  w.atab = off;   off += vround(sizeof(double) * 2 * kAngleTableEntries);
   w.A = off;      off += vround((size_t)((max_q + kM - 1) / kM) * kM * (d + 16 * search_qjl_steps(m)) * 2);
   w.qscale = off; off += vround(sizeof(float) * max_q);
   w.part_s = off; off += vround(sizeof(float) * (size_t)max_q * kMaxSplits * 2 * kListK);
@@ -1050,6 +1051,9 @@ tq_status tq_vec_create(const tq_vec_config* cfg, int64_t n, int32_t max_queries
   cudaError_t e = cudaMemsetAsync(v->ws + v->W.status, 0, kVAlign, stream);
   if (e == cudaSuccess) e = cudaMemcpyAsync(v->ws + v->W.signs, signs.data(), sizeof(double) * d, cudaMemcpyHostToDevice, stream);
   if (e == cudaSuccess) e = cudaMemcpyAsync(v->ws + v->W.St, St.data(), sizeof(float) * St.size(), cudaMemcpyHostToDevice, stream);
+  std::vector<double> atab(2 * kAngleTableEntries, 0.0);
+  angle_table_host(1 << cfg->b_theta, atab.data());
+  if (e == cudaSuccess) e = cudaMemcpyAsync(v->ws + v->W.atab, atab.data(), sizeof(double) * atab.size(), cudaMemcpyHostToDevice, stream);
   if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
   if (e != cudaSuccess) {
     delete v;
@@ -1078,6 +1082,7 @@ tq_status tq_encode_vectors(tq_vec_index* v, const float* x, int64_t start, int6
   a.L = v->L;
   a.signs = (const double*)(v->ws + v->W.signs);
   a.St = (const float*)(v->ws + v->W.St);
+  a.atab = (const double2*)(v->ws + v->W.atab);
   a.inv_sqrt_d = 1.0 / std::sqrt((double)v->d);
   a.status = (int*)(v->ws + v->W.status);
   uint8_t* base = (uint8_t*)codes;
