@@ -49,6 +49,41 @@ __device__ __forceinline__ void encode_vector(const EncodeArgs& a, const float* 
                        is_key, rbuf, codes, bits, s16_out, rn16_out);
 }
 
+// One bulk copy of S^T into shared memory, completed on an mbarrier, and a
+// bounded wait for it (a copy that never lands latches kStatusTimeout; the
+// decode's merge then writes NaN).
+__device__ __forceinline__ void st_bulk_copy(uint32_t bar, void* dst, const void* src, uint32_t bytes) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar) : "memory");
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          (uint32_t)__cvta_generic_to_shared(dst)),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void st_bulk_wait(uint32_t bar, int* status) {
+  uint32_t ok = 0;
+  uint64_t t0 = 0;
+  for (int it = 0;; ++it) {
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], 0, %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(1000000u)
+        : "memory");
+    if (ok) return;
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    if (it == 0) t0 = t;
+    else if (t - t0 > kDefaultWaitLimitNs) {
+      atomicOr(status, kStatusTimeout);
+      return;
+    }
+  }
+}
+
 // Merges `val` into the 32-bit word at `addr` under `mask` (bits of tokens
 // written by this launch); bits of other tokens are kept.
 __device__ __forceinline__ void merge_word(uint32_t* addr, uint32_t val, uint32_t mask) {
@@ -303,10 +338,13 @@ __global__ void __launch_bounds__(2 * D) encode_small_kernel(EncodeArgs a) {
   uint32_t* bits = reinterpret_cast<uint32_t*>(codes + 2 * P); // [4] key sign words
   uint16_t* sc = reinterpret_cast<uint16_t*>(bits + 4);        // s16_k, rn16, s16_v
   float* sst = reinterpret_cast<float*>(sm) + small_st_offset(D) / 4;   // S^T [D][m]
-  async_copy_g2s(sst, a.St, D * L.m * 4);      // lands while the rotation and polar steps run
+  __shared__ uint64_t st_bar;
   __shared__ double2 atab[kAngleTableEntries];
+  const uint32_t bar = (uint32_t)__cvta_generic_to_shared(&st_bar);
+  // S^T lands while the rotation and polar steps run (one bulk copy); the
+  // angle tables are published by the rotation's first block barrier
+  if (tid == 0) st_bulk_copy(bar, sst, a.St, (uint32_t)(D * L.m * 4));
   angle_tables(1 << L.b_theta, a.atab, atab, tid, blockDim.x);
-  __syncthreads();
   // Launched as a programmatic dependent of the kernel before it: S^T (set
   // at cache creation) may be fetched early, the inputs only once that
   // kernel has finished.
@@ -320,7 +358,7 @@ __global__ void __launch_bounds__(2 * D) encode_small_kernel(EncodeArgs a) {
     const PromoUnitState* st = a.promo + unit;
     const int k = st->n_pend;
     if (e >= k + a.n_new) {                  // (the whole CTA) nothing to insert
-      async_copy_wait();
+      if (tid == 0) st_bulk_wait(bar, a.status);
       return;
     }
     const int slot = (int)((st->ring_pos + e) % a.W);
@@ -335,7 +373,7 @@ __global__ void __launch_bounds__(2 * D) encode_small_kernel(EncodeArgs a) {
   } else {
     const UnitSpan us = unit_span(a, unit);
     if (e >= us.n) {                         // (the whole CTA) nothing for this unit
-      async_copy_wait();
+      if (tid == 0) st_bulk_wait(bar, a.status);
       return;
     }
     dest = us.cold_start + e;
@@ -415,40 +453,47 @@ __global__ void __launch_bounds__(2 * D) encode_small_kernel(EncodeArgs a) {
   }
 #pragma unroll
   for (int o = 16; o; o >>= 1) ss = __dadd_rn(ss, __shfl_xor_sync(kFull, ss, o));
-  async_copy_wait();
+  st_bulk_wait(bar, a.status);
   __syncthreads();            // residual complete, S^T staged, reduction slots free
   if (team == 0) {
     if (lane == 0) red[wt] = ss;
   }
   __syncthreads();
-  if (team == 0) {
-    if (el == 0) {
-      double tot = red[0];
-      for (int w = 1; w < NW; ++w) tot = __dadd_rn(tot, red[w]);
-      const uint16_t rnb = f64_to_f16_bits(__dsqrt_rn(tot));
-      if ((rnb & 0x7c00u) == 0x7c00u) atomicOr(a.status, kStatusRange);
-      sc[1] = rnb;
-    }
-    // (S r)_i as four interleaved partial sums (j mod 4), so the FMA
-    // chain is a quarter as long; a sign can differ from another summation
-    // order only within float64 rounding of zero
-    for (int i0 = 0; i0 < L.m; i0 += D) {
-      const int i = i0 + el;
-      double acc = 0.0;
-      if (i < L.m) {
-        double p4[4] = {0.0, 0.0, 0.0, 0.0};
-#pragma unroll 8
-        for (int j = 0; j < D; j += 4) {
+  if (team == 0 && el == 0) {
+    double tot = red[0];
+    for (int w = 1; w < NW; ++w) tot = __dadd_rn(tot, red[w]);
+    const uint16_t rnb = f64_to_f16_bits(__dsqrt_rn(tot));
+    if ((rnb & 0x7c00u) == 0x7c00u) atomicOr(a.status, kStatusRange);
+    sc[1] = rnb;
+  }
+  // (S r)_i: team t sums j in [t D/2, (t + 1) D/2) as four interleaved
+  // partial sums; team 1 hands its half to team 0 through its (now free)
+  // exchange buffer.  A sign can differ from another summation order only
+  // within float64 rounding of zero.
+  const double* rres = sm;                   // the key residual (team 0's buffer)
+  double* pbuf = sm + D;
+  for (int i0 = 0; i0 < L.m; i0 += D) {
+    const int i = i0 + el;
+    double part = 0.0;
+    if (i < L.m) {
+      double p4[4] = {0.0, 0.0, 0.0, 0.0};
+      const int j0 = team * (D / 2);
+#pragma unroll 4
+      for (int j = j0; j < j0 + D / 2; j += 4) {
 #pragma unroll
-          for (int t = 0; t < 4; ++t) p4[t] = fma((double)sst[(j + t) * L.m + i], xb[j + t], p4[t]);
-        }
-        acc = __dadd_rn(__dadd_rn(p4[0], p4[1]), __dadd_rn(p4[2], p4[3]));
+        for (int t = 0; t < 4; ++t) p4[t] = fma((double)sst[(j + t) * L.m + i], rres[j + t], p4[t]);
       }
+      part = __dadd_rn(__dadd_rn(p4[0], p4[1]), __dadd_rn(p4[2], p4[3]));
+    }
+    if (team == 1) pbuf[el] = part;
+    __syncthreads();
+    if (team == 0) {
+      const double acc = __dadd_rn(part, pbuf[el]);
       const unsigned word = __ballot_sync(kFull, i < L.m && acc >= 0.0);
       if (lane == 0 && i < L.m) bits[i >> 5] = word;
     }
+    __syncthreads();
   }
-  __syncthreads();
 
   // ---- merge the token's fields into its tile ------------------------------
   const int64_t tok = dest;
