@@ -190,33 +190,39 @@ __device__ __forceinline__ void qprep_body(const QPrepArgs& a) {
 // ---------------------------------------------------------------------------
 // combine
 // ---------------------------------------------------------------------------
-// One block per query head, one thread per output dimension.  The split
-// records' (m, l) pairs are read once by as many threads, so every global
-// load of the block is independent of the others; R^T is applied to the
-// cold sum with butterflies in registers (shuffles) and, for strides of a
-// warp or more, through shared memory.
-constexpr int kCombineMaxSlots = 128;
+// One warp per query head (kCombineHeads heads per block), lane i holding
+// output dims [PD i, PD i + PD).  The kernel moves a few KB per head and
+// is bound by load latency, so its loads go out together: the o vectors of
+// the first kCombineChunk slots before anything waits on a load, the (m, l)
+// pairs of every slot spread over the lanes.  R^T is applied to the cold
+// sum with butterflies inside the lane and across lanes (shuffles): no
+// shared memory, no barrier.
+constexpr int kCombineMaxSlots = kSlotsCold + kSlotsHot;
+constexpr int kCombineChunk = 16;    // slots whose o vectors are in flight together
+constexpr int kCombineHeads = 4;     // warps (query heads) per block
 
-__global__ void combine_kernel(const CombineArgs a) {
-  __shared__ float sw[kCombineMaxSlots];     // per-slot weight 2^(m_s - m)
-  __shared__ float red[2][8];
-  __shared__ float xbuf[256];
+template <int D>
+__global__ void __launch_bounds__(32 * kCombineHeads) combine_kernel(const CombineArgs a) {
+  constexpr int PD = D / 32;
+  constexpr int CH = kCombineChunk;
+  constexpr int MS = kCombineMaxSlots / 32;   // (m, l) pairs per lane
   // The next step's eviction encode may start its prologue now (it waits
   // for this kernel before reading its inputs).
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   // launched as a programmatic dependent of the attention kernel
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  const int hg = blockIdx.x;
+  const int lane = threadIdx.x & 31;
+  const int hg = blockIdx.x * kCombineHeads + (threadIdx.x >> 5);
+  if (hg >= a.batch * a.Hq) return;          // (warp-uniform)
   const int b = hg / a.Hq, hq = hg % a.Hq;
   const int kvh = hq / a.G, g = hq % a.G;
   const int unit = b * a.Hkv + kvh;
-  const int D = a.d, t = threadIdx.x, lane = t & 31, warp = t >> 5, nw = blockDim.x >> 5;
   const SplitPlan& pl = a.plan;
   const int slots = pl.slots_cold + pl.slots_hot;
   const float* base = a.part + (size_t)unit * slots * a.G * (D + 2);
   int nc = 0, nh = 0;
   if (a.rows != nullptr) {             // ragged: the unit's own blocks and tiles
-    const int b = unit / a.Hkv, h = unit % a.Hkv;
+    const int h = unit % a.Hkv;
     const int64_t nb = (a.rows->n_cold[b] + kTokensPerBlock - 1) / kTokensPerBlock;
     const int64_t ht = (a.rows->n_hot[b] + kTokensPerBlock - 1) / kTokensPerBlock;
     if (nb > 0) {
@@ -246,78 +252,123 @@ __global__ void combine_kernel(const CombineArgs a) {
     nh = (int)(((unit + 1) * ht - 1) / pl.hot_tpc - (unit * ht) / pl.hot_tpc + 1);
   }
   const int ns = nc + nh;
-  if (*(volatile const int*)a.status & kStatusNoPartials) {
-    // an attention launch gave up without writing its partials (a latched
-    // timeout or layout error): the output is NaN until the status is read
-    a.out[(size_t)hg * D + t] = __int_as_float(0x7fc00000);
-    return;
-  }
   auto rec = [&](int s) {
     return base + ((size_t)(s < nc ? s : pl.slots_cold + (s - nc)) * a.G + g) * (D + 2);
   };
-  // ---- m = max over slots, then w_s and l = sum w_s l_s ----------------------
-  float ms[kCombineMaxSlots / 64], ls[kCombineMaxSlots / 64];
-  float mx = kNegInf;
+  // this lane's dims of slot s's o vector (records are 8-byte aligned)
+  auto load_o = [&](int s, float (&o)[PD]) {
+    const float* pp = rec(s) + 2 + lane * PD;
 #pragma unroll
-  for (int k = 0; k < kCombineMaxSlots / 64; ++k) {
-    const int s = t + k * blockDim.x;
+    for (int k = 0; k < PD; k += 2) {
+      const float2 v = *reinterpret_cast<const float2*>(pp + k);
+      o[k] = v.x;
+      o[k + 1] = v.y;
+    }
+  };
+  float ov[CH][PD];
+#pragma unroll
+  for (int u = 0; u < CH; ++u) {
+    if (u < ns) {
+      load_o(u, ov[u]);
+    } else {
+#pragma unroll
+      for (int k = 0; k < PD; ++k) ov[u][k] = 0.f;
+    }
+  }
+  float ms[MS], ls[MS];
+#pragma unroll
+  for (int k = 0; k < MS; ++k) {
+    const int s = lane + 32 * k;
     ms[k] = kNegInf;
     ls[k] = 0.f;
     if (s < ns) {
-      const float* pp = rec(s);
-      ms[k] = pp[0];
-      ls[k] = pp[1];
+      const float2 v = *reinterpret_cast<const float2*>(rec(s));
+      ms[k] = v.x;
+      ls[k] = v.y;
     }
-    mx = fmaxf(mx, ms[k]);
   }
+  float* orow = a.out + (size_t)hg * D + lane * PD;
+  if (*(volatile const int*)a.status & kStatusNoPartials) {
+    // an attention launch gave up without writing its partials (a latched
+    // timeout or layout error): the output is NaN until the status is read
+#pragma unroll
+    for (int k = 0; k < PD; ++k) orow[k] = __int_as_float(0x7fc00000);
+    return;
+  }
+  // ---- m = max over slots, then w_s and l = sum w_s l_s ----------------------
+  float mx = kNegInf;
+#pragma unroll
+  for (int k = 0; k < MS; ++k) mx = fmaxf(mx, ms[k]);
 #pragma unroll
   for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, o));
-  if (lane == 0) red[0][warp] = mx;
-  __syncthreads();
-  mx = red[0][0];
-  for (int w = 1; w < nw; ++w) mx = fmaxf(mx, red[0][w]);
-  float lsum = 0.f;
+  float w[MS], lsum = 0.f;
 #pragma unroll
-  for (int k = 0; k < kCombineMaxSlots / 64; ++k) {
-    const int s = t + k * blockDim.x;
-    if (s < ns) {
-      const float w = ms[k] == kNegInf ? 0.f : exp2f(ms[k] - mx);
-      sw[s] = w;
-      lsum += w * ls[k];
-    }
+  for (int k = 0; k < MS; ++k) {
+    w[k] = ms[k] == kNegInf ? 0.f : exp2f(ms[k] - mx);
+    lsum += w[k] * ls[k];
   }
 #pragma unroll
   for (int o = 16; o; o >>= 1) lsum += __shfl_xor_sync(kFull, lsum, o);
-  if (lane == 0) red[1][warp] = lsum;
-  __syncthreads();
-  lsum = 0.f;
-  for (int w = 0; w < nw; ++w) lsum += red[1][w];
-  // ---- weighted sums of the o vectors (independent loads) --------------------
-  float oc = 0.f, oh = 0.f;
-  if (mx != kNegInf) {
-#pragma unroll 8
-    for (int s = 0; s < nc; ++s) oc += sw[s] * rec(s)[2 + t];
-#pragma unroll 4
-    for (int s = nc; s < ns; ++s) oh += sw[s] * rec(s)[2 + t];
-  }
-  // ---- R^T on the cold sum: unnormalised Hadamard, then signs / sqrt(d) ------
-  float x = oc;
+  // ---- weighted sums of the o vectors ------------------------------------------
+  // (slot s's weight sits in lane s % 32, register s / 32; s is warp-uniform)
+  auto weight = [&](int s) {
+    const int k = s >> 5;
+    float x = w[0];
 #pragma unroll
-  for (int h = 1; h < 32; h <<= 1) {
-    const float o = __shfl_xor_sync(kFull, x, h);
-    x = (t & h) ? (o - x) : (x + o);
+    for (int kk = 1; kk < MS; ++kk)
+      if (k == kk) x = w[kk];
+    return __shfl_sync(kFull, x, s & 31);
+  };
+  float oc[PD], oh[PD];
+#pragma unroll
+  for (int k = 0; k < PD; ++k) oc[k] = oh[k] = 0.f;
+  auto accum = [&](int s, const float (&o)[PD]) {
+    const float ws = weight(s);
+    if (s < nc) {
+#pragma unroll
+      for (int k = 0; k < PD; ++k) oc[k] += ws * o[k];
+    } else {
+#pragma unroll
+      for (int k = 0; k < PD; ++k) oh[k] += ws * o[k];
+    }
+  };
+  if (mx != kNegInf) {
+#pragma unroll
+    for (int u = 0; u < CH; ++u)
+      if (u < ns) accum(u, ov[u]);
+    for (int s0 = CH; s0 < ns; s0 += CH) {
+#pragma unroll
+      for (int u = 0; u < CH; ++u)
+        if (s0 + u < ns) load_o(s0 + u, ov[u]);
+#pragma unroll
+      for (int u = 0; u < CH; ++u)
+        if (s0 + u < ns) accum(s0 + u, ov[u]);
+    }
   }
-  for (int h = 32; h < D; h <<= 1) {
-    xbuf[t] = x;
-    __syncthreads();
-    const float o = xbuf[t ^ h];
-    __syncthreads();
-    x = (t & h) ? (o - x) : (x + o);
-  }
-  const float res = mx == kNegInf ? 0.f
-                                  : (oh + (float)a.signs[t] * x * rsqrtf((float)D)) / lsum;
-  a.out[(size_t)hg * D + t] = res;
-  if (a.ml != nullptr && t == 0) {      // the softmax's normaliser, for promotion
+  // ---- R^T on the cold sum: unnormalised Hadamard (dim i = PD lane + k),
+  // strides below PD inside the lane, the others across lanes; then the
+  // signs and 1/sqrt(d) ----------------------------------------------------------
+#pragma unroll
+  for (int h = 1; h < PD; h <<= 1)
+#pragma unroll
+    for (int k = 0; k < PD; ++k)
+      if (!(k & h)) {
+        const float x = oc[k], y = oc[k + h];
+        oc[k] = x + y;
+        oc[k + h] = x - y;
+      }
+#pragma unroll
+  for (int h = 1; h < 32; h <<= 1)
+#pragma unroll
+    for (int k = 0; k < PD; ++k) {
+      const float o = __shfl_xor_sync(kFull, oc[k], h);
+      oc[k] = (lane & h) ? (o - oc[k]) : (oc[k] + o);
+    }
+  const float rs = rsqrtf((float)D);
+#pragma unroll
+  for (int k = 0; k < PD; ++k)
+    orow[k] = mx == kNegInf ? 0.f : (oh[k] + (float)a.signs[lane * PD + k] * oc[k] * rs) / lsum;
+  if (a.ml != nullptr && lane == 0) {   // the softmax's normaliser, for promotion
     a.ml[2 * (size_t)hg] = mx;
     a.ml[2 * (size_t)hg + 1] = lsum;
   }
@@ -410,18 +461,20 @@ cudaError_t launch_rows_upload(RowTable* dst, const RowTable& src, cudaStream_t 
 }
 
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s) {
+  if (a.d != 64 && a.d != 128) return cudaErrorInvalidValue;
   // programmatic dependent launch: the kernel waits for the attention
   // kernel before it reads the partials
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(a.batch * a.Hq);
-  cfg.blockDim = dim3(a.d);
+  cfg.gridDim = dim3((a.batch * a.Hq + kCombineHeads - 1) / kCombineHeads);
+  cfg.blockDim = dim3(32 * kCombineHeads);
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, combine_kernel, a);
+  if (a.d == 64) return cudaLaunchKernelEx(&cfg, combine_kernel<64>, a);
+  return cudaLaunchKernelEx(&cfg, combine_kernel<128>, a);
 }
 
 }  // namespace tq
