@@ -39,16 +39,6 @@ __host__ __device__ constexpr size_t small_st_offset(int d) {
   return ((size_t)2 * d * 8 + (size_t)2 * (d / 32) * 8 + (size_t)d + 16 + 8 + 15) / 16 * 16;
 }
 
-template <int D, bool SKETCH = true>
-__device__ __forceinline__ void encode_vector(const EncodeArgs& a, const float* St, const double2* atab,
-                                              const __half* src, bool is_key,
-                                              double* rbuf, uint8_t* codes, uint32_t* bits,
-                                              uint16_t* s16_out, uint16_t* rn16_out) {
-  encode_vector_any<D, SKETCH>(a.L, a.signs, St, atab, a.inv_sqrt_d, a.status,
-                       [&](int lane, double (&x)[D / 32]) { load_vec<D / 32>(src, lane, x); },
-                       is_key, rbuf, codes, bits, s16_out, rn16_out);
-}
-
 // One bulk copy of S^T into shared memory, completed on an mbarrier, and a
 // bounded wait for it (a copy that never lands latches kStatusTimeout; the
 // decode's merge then writes NaN).
@@ -232,9 +222,8 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
         ksrc = a.src_k + ((int64_t)unit * a.src_tokens + (e - us.nA)) * D;
         vsrc = a.src_v + ((int64_t)unit * a.src_tokens + (e - us.nA)) * D;
       }
-      encode_vector<D, false>(a, St, atab, ksrc, true, rbuf + s * D, kc + s * P, kb + s * 8, sc + s * 4,
-                              sc + s * 4 + 1);
-      encode_vector<D>(a, St, atab, vsrc, false, nullptr, vc + s * P, nullptr, sc + s * 4 + 2, nullptr);
+      encode_kv_pair<D>(a.L, a.signs, atab, a.inv_sqrt_d, a.status, ksrc, vsrc, rbuf + s * D, kc + s * P,
+                        vc + s * P, sc + s * 4, sc + s * 4 + 1, sc + s * 4 + 2);
     }
     // the four keys' sign words in one pass over S^T (lane order when staged
     // for m = 64 or 128)

@@ -220,6 +220,142 @@ __device__ __forceinline__ void encode_vector_any(const Layout& L, const double*
   __syncwarp();
 }
 
+// A key and a value of one token at once (whole warp; the bulk encode):
+// the steps of encode_vector_any for the two vectors, interleaved stage by
+// stage so that every stage has two independent float64 chains.  Each
+// vector sees exactly the operations encode_vector_any applies to it, so
+// the codes are the same.  The key stops after its residual (kept in rbuf
+// for a sketch blocked over keys).
+template <int D>
+__device__ __forceinline__ void encode_kv_pair(const Layout& L, const double* signs, const double2* atab,
+                                               double inv_sqrt_d, int* status, const __half* ksrc,
+                                               const __half* vsrc, double* rbuf, uint8_t* kcodes,
+                                               uint8_t* vcodes, uint16_t* ks16_out, uint16_t* rn16_out,
+                                               uint16_t* vs16_out) {
+  constexpr int E = D / 32;      // elements per lane
+  constexpr int PL = E / 2;      // pairs per lane
+  const int lane = threadIdx.x & 31;
+  const int Lr = (1 << L.b_r) - 1;
+  const int nt = 1 << L.b_theta;
+
+  // ---- rotation: y = H (D x) / sqrt(d), key (v = 0) and value (v = 1) ------
+  double x[2][E];
+  load_vec<E>(ksrc, lane, x[0]);
+  load_vec<E>(vsrc, lane, x[1]);
+#pragma unroll
+  for (int i = 0; i < E; ++i) {
+    const double sg = signs[lane * E + i];
+    x[0][i] = __dmul_rn(x[0][i], sg);
+    x[1][i] = __dmul_rn(x[1][i], sg);
+  }
+#pragma unroll
+  for (int h = 1; h < D; h <<= 1) {
+    if (h < E) {
+#pragma unroll
+      for (int i = 0; i < E; ++i) {
+        if (!(i & h)) {
+#pragma unroll
+          for (int v = 0; v < 2; ++v) {
+            const double p = x[v][i], q = x[v][i + h];
+            x[v][i] = __dadd_rn(p, q);
+            x[v][i + h] = __dsub_rn(p, q);
+          }
+        }
+      }
+    } else {
+      const int lm = h / E;
+#pragma unroll
+      for (int i = 0; i < E; ++i) {
+#pragma unroll
+        for (int v = 0; v < 2; ++v) {
+          const double o = __shfl_xor_sync(kFull, x[v][i], lm);
+          x[v][i] = (lane & lm) ? __dsub_rn(o, x[v][i]) : __dadd_rn(x[v][i], o);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < E; ++i) {
+    x[0][i] = __dmul_rn(x[0][i], inv_sqrt_d);
+    x[1][i] = __dmul_rn(x[1][i], inv_sqrt_d);
+  }
+
+  // ---- polar: rho and the angle code per pair; scale s16 = fp16(max rho) --
+  double rho[2][PL];
+  int ct[2][PL];
+  double smax[2] = {0.0, 0.0};
+#pragma unroll
+  for (int k = 0; k < PL; ++k) {
+#pragma unroll
+    for (int v = 0; v < 2; ++v) {
+      const double y0 = x[v][2 * k], y1 = x[v][2 * k + 1];
+      rho[v][k] = __dsqrt_rn(__dadd_rn(__dmul_rn(y0, y0), __dmul_rn(y1, y1)));
+      ct[v][k] = angle_code(y0, y1, nt, atab);
+      smax[v] = fmax(smax[v], rho[v][k]);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    smax[0] = fmax(smax[0], __shfl_xor_sync(kFull, smax[0], o));
+    smax[1] = fmax(smax[1], __shfl_xor_sync(kFull, smax[1], o));
+  }
+  uint16_t s16b[2];
+  double s16[2];
+  bool zero[2];
+#pragma unroll
+  for (int v = 0; v < 2; ++v) {
+    s16b[v] = f64_to_f16_bits(smax[v]);
+    if ((s16b[v] & 0x7c00u) == 0x7c00u) {   // overflow: latch, store a zero record
+      if (lane == 0) atomicOr(status, kStatusRange);
+      s16b[v] = 0;
+    }
+    s16[v] = f16_bits_to_f64(s16b[v]);
+    zero[v] = (s16[v] == 0.0);
+  }
+
+  // ---- codes ---------------------------------------------------------------
+  int cr[2][PL];
+#pragma unroll
+  for (int k = 0; k < PL; ++k) {
+#pragma unroll
+    for (int v = 0; v < 2; ++v) {
+      const double tr = __dmul_rn(__ddiv_rn(rho[v][k], zero[v] ? 1.0 : s16[v]), (double)Lr);
+      const int c = (int)rint(tr);
+      cr[v][k] = c < 0 ? 0 : (c > Lr ? Lr : c);
+      if (zero[v]) {
+        cr[v][k] = 0;
+        ct[v][k] = 0;
+      }
+    }
+    kcodes[lane * PL + k] = (uint8_t)((cr[0][k] << L.b_theta) | ct[0][k]);
+    vcodes[lane * PL + k] = (uint8_t)((cr[1][k] << L.b_theta) | ct[1][k]);
+  }
+  if (lane == 0) {
+    *ks16_out = s16b[0];
+    *vs16_out = s16b[1];
+  }
+
+  // ---- the key's residual r = y - y_hat and its norm rn16 -----------------
+  double r[E];
+  double ss = 0.0;
+#pragma unroll
+  for (int k = 0; k < PL; ++k) {
+    const double rh = __ddiv_rn(__dmul_rn((double)cr[0][k], s16[0]), (double)Lr);
+    const double2 csn = atab[angle_cs_offset(nt) + ct[0][k]];   // cos, sin of c_theta 2 pi / nt
+    r[2 * k] = __dsub_rn(x[0][2 * k], __dmul_rn(rh, csn.x));
+    r[2 * k + 1] = __dsub_rn(x[0][2 * k + 1], __dmul_rn(rh, csn.y));
+    ss = __dadd_rn(ss, __dadd_rn(__dmul_rn(r[2 * k], r[2 * k]), __dmul_rn(r[2 * k + 1], r[2 * k + 1])));
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) ss = __dadd_rn(ss, __shfl_xor_sync(kFull, ss, o));
+  const uint16_t rnb = f64_to_f16_bits(__dsqrt_rn(ss));
+  if ((rnb & 0x7c00u) == 0x7c00u && lane == 0) atomicOr(status, kStatusRange);
+  if (lane == 0) *rn16_out = rnb;
+#pragma unroll
+  for (int i = 0; i < E; ++i) rbuf[lane * E + i] = r[i];
+  __syncwarp();
+}
+
 // QJL sign words of NV residuals at once (whole warp): r_v = rbuf[v D ..
 // v D + D), words written to bits[v * bits_stride + k] for the vectors with
 // live[v].  Lane outputs i = lane + 32 k as in encode_vector_any; each S^T
