@@ -82,32 +82,6 @@ __device__ __forceinline__ void merge_word(uint32_t* addr, uint32_t val, uint32_
   *addr = val;
 }
 
-// Bits of word w of a lane chunk whose codes are laid out at code index q
-// (bit q*bw); `code_of(q, &c)` returns false for codes of tokens that this
-// launch does not write.
-template <typename F>
-__device__ __forceinline__ void chunk_word(int w, int ncodes, int bw, F code_of, uint32_t& val,
-                                           uint32_t& mask) {
-  val = 0u;
-  mask = 0u;
-  const uint32_t cm = (1u << bw) - 1u;
-  int q0 = (32 * w) / bw - 1;
-  if (q0 < 0) q0 = 0;
-  for (int q = q0; q < ncodes && q * bw < 32 * (w + 1); ++q) {
-    const int bit = q * bw - 32 * w;
-    if (bit + bw <= 0) continue;
-    uint32_t c;
-    if (!code_of(q, &c)) continue;
-    if (bit >= 0) {
-      val |= c << bit;
-      mask |= cm << bit;
-    } else {
-      val |= c >> (-bit);
-      mask |= cm >> (-bit);
-    }
-  }
-}
-
 // What one launch writes for a unit: n tokens at cold positions cold_start
 // .. cold_start + n - 1, the first nA read from ring slots (ring_start + e)
 // mod W, the rest from source tokens e - nA.  Uniform over the units, or
@@ -209,6 +183,8 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
       any |= inr[s];
     }
     if (!any) continue;
+    const unsigned inm = (unsigned)inr[0] | ((unsigned)inr[1] << 1) | ((unsigned)inr[2] << 2) |
+                         ((unsigned)inr[3] << 3);   // (bit s: token s is written)
     for (int s = 0; s < 4; ++s) {
       if (!inr[s]) continue;
       const int64_t e = seq[s];
@@ -235,57 +211,88 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
 
     uint8_t* tb = a.cold + ((int64_t)unit * L.blocks_per_unit + tile / kTilesPerBlock) * L.block_bytes +
                   (tile % kTilesPerBlock) * L.tile_bytes;
-    // K code words: lanes (gid = 2c + e, tig), codes q: half h = q / pt, pair tig*pt + q % pt
-    for (int q = lane; q < 8 * L.kwt; q += 32) {
-      const int ch = q / L.kwt, w = q % L.kwt;
-      const int e = ch / 4, tig = ch % 4;
+    // ---- the job's fields into the fragment-major words ------------------
+    // Lane chunk ch = 4 e + tig (tile lane 4 (2c + e) + tig) holds codes
+    // q = h PT + k (pair tig PT + k of token e + 2h) at chunk bit q bw.
+    // Codes: lane (kv, ch, h) packs its PT codes into whole words with a
+    // 64-bit shift register; when PT bw is not a multiple of 32 the two
+    // halves share a word, which the h = 0 lane completes with its
+    // neighbour's part.  Only bits of tokens this launch writes are merged.
+    {
+      constexpr int PT = P / 4;
+      const int kv = lane >> 4, ch = (lane >> 1) & 7, h = lane & 1;
+      const int e = ch >> 2, tig = ch & 3, sl = e + 2 * h;
       const int l = 4 * (2 * c + e) + tig;
-      uint32_t val, mask;
-      chunk_word(w, 2 * (P / 4), bw, [&](int qi, uint32_t* out) {
-        const int h = qi / (P / 4), k = qi % (P / 4), s = e + 2 * h;
-        if (!inr[s]) return false;
-        *out = kc[s * P + tig * (P / 4) + k];
-        return true;
-      }, val, mask);
-      merge_word(reinterpret_cast<uint32_t*>(tb + L.off_kc + lane_word_offset(w, l, L.kwt)), val, mask);
-    }
-    // V code words: the K layout
-    for (int q = lane; q < 8 * L.vwt; q += 32) {
-      const int ch = q / L.vwt, w = q % L.vwt;
-      const int e = ch / 4, tig = ch % 4;
-      const int l = 4 * (2 * c + e) + tig;
-      uint32_t val, mask;
-      chunk_word(w, 2 * (P / 4), bw, [&](int qi, uint32_t* out) {
-        const int h = qi / (P / 4), k = qi % (P / 4), s = e + 2 * h;
-        if (!inr[s]) return false;
-        *out = vc[s * P + tig * (P / 4) + k];
-        return true;
-      }, val, mask);
-      merge_word(reinterpret_cast<uint32_t*>(tb + L.off_vc + lane_word_offset(w, l, L.vwt)), val, mask);
-    }
-    // sign words: lanes (gid = 2c + e, tig); m/4 signs per (token, tig), local
-    // sign j at chunk bit sign_chunk_bit(j, h, m)
-    const int qb = L.m / 4;
-    for (int q = lane; q < 8 * L.sw; q += 32) {
-      const int ch = q / L.sw, w = q % L.sw;
-      const int e = ch / 4, tig = ch % 4;
-      const int l = 4 * (2 * c + e) + tig;
-      uint32_t val = 0u, mask = 0u;
-      for (int h = 0; h < 2; ++h) {
-        const int s = e + 2 * h;
-        if (!inr[s]) continue;
-        for (int j = 0; j < qb; ++j) {
-          const int bit = sign_chunk_bit(j, h, L.m) - 32 * w;
-          if (bit < 0 || bit >= 32) continue;
-          const int i = tig * qb + j;            // canonical sign index
-          val |= ((kb[s * 8 + (i >> 5)] >> (i & 31)) & 1u) << bit;
-          mask |= 1u << bit;
+      const uint32_t* src = reinterpret_cast<const uint32_t*>((kv ? vc : kc) + sl * P + tig * PT);
+      uint8_t* plane = tb + (kv ? L.off_vc : L.off_kc);
+      const int nw = kv ? L.vwt : L.kwt;
+      const bool live = (inm >> sl) & 1u;
+      const uint32_t cm = live ? (1u << bw) - 1u : 0u;
+      const bool shared = ((PT * bw) & 31) != 0;
+      const int bit0 = h * PT * bw;
+      int w = bit0 >> 5, nb = bit0 & 31;
+      uint64_t acc = 0u, am = 0u;
+      uint32_t hv = 0u, hm = 0u;         // h = 1: its part of the shared word
+      bool first = true;
+#pragma unroll
+      for (int k4 = 0; k4 < PT / 4; ++k4) {
+        const uint32_t cw = live ? src[k4] : 0u;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          acc |= (uint64_t)((cw >> (8 * k)) & 0xffu) << nb;
+          am |= (uint64_t)cm << nb;
+          nb += bw;
+          if (nb >= 32) {
+            if (h == 1 && first && shared) {
+              hv = (uint32_t)acc;
+              hm = (uint32_t)am;
+            } else {
+              merge_word(reinterpret_cast<uint32_t*>(plane + lane_word_offset(w, l, nw)), (uint32_t)acc,
+                         (uint32_t)am);
+            }
+            first = false;
+            acc >>= 32;
+            am >>= 32;
+            nb -= 32;
+            ++w;
+          }
         }
       }
-      merge_word(reinterpret_cast<uint32_t*>(tb + L.off_ks + lane_word_offset(w, l, L.sw)), val, mask);
+      const uint32_t ov = __shfl_down_sync(kFull, hv, 1), om = __shfl_down_sync(kFull, hm, 1);
+      if (nb > 0)   // h = 0: the shared word; h = 1: the chunk's last, partial word
+        merge_word(reinterpret_cast<uint32_t*>(plane + lane_word_offset(w, l, nw)),
+                   (uint32_t)acc | (h == 0 ? ov : 0u), (uint32_t)am | (h == 0 ? om : 0u));
+    }
+    // Signs (m = 64 or 128): local sign j of token half h sits at chunk bit
+    // sign_chunk_bit(j, h, m); lane (ch, h) < 16 permutes its token's m/4
+    // signs of this chunk with compile-time positions (m = 64: both halves
+    // share the word, combined by shuffle).
+    {
+      const int ch = (lane >> 1) & 7, h = lane & 1;
+      const int e = ch >> 2, tig = ch & 3, sl = e + 2 * h;
+      const int l = 4 * (2 * c + e) + tig;
+      const bool live = lane < 16 && ((inm >> sl) & 1u);
+      const int qb = L.m / 4;
+      const uint32_t kw = live ? kb[sl * 8 + ((tig * qb) >> 5)] >> ((tig * qb) & 31) : 0u;
+      uint32_t pv = 0u, pm = 0u;
+      if (L.m == 128) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) pv |= ((kw >> j) & 1u) << sign_chunk_bit(j, 0, 128);
+        pm = live ? 0xffffffffu : 0u;
+      } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) pv |= ((kw >> j) & 1u) << sign_chunk_bit(j, 0, 64);
+        pv <<= 4 * h;
+        pm = live ? 0x0f0f0f0fu << (4 * h) : 0u;
+        pv |= __shfl_xor_sync(kFull, pv, 1);
+        pm |= __shfl_xor_sync(kFull, pm, 1);
+      }
+      if (lane < 16 && (L.m == 128 || h == 0))
+        merge_word(reinterpret_cast<uint32_t*>(tb + L.off_ks + lane_word_offset(L.m == 128 ? h : 0, l, L.sw)),
+                   pv, pm);
     }
     // scalars
-    if (lane < 4 && inr[lane]) {
+    if (lane < 4 && ((inm >> lane) & 1u)) {
       const int s = lane;
       const int e = s & 1, h = s >> 1, gid = 2 * c + e;
       uint16_t* ks = reinterpret_cast<uint16_t*>(tb + L.off_ksc);
