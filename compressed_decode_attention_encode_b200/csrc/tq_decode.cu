@@ -190,30 +190,34 @@ __device__ __forceinline__ void qprep_body(const QPrepArgs& a) {
 // ---------------------------------------------------------------------------
 // combine
 // ---------------------------------------------------------------------------
-// One warp per query head (kCombineHeads heads per block), lane i holding
-// output dims [PD i, PD i + PD).  The kernel moves a few KB per head and
-// is bound by load latency, so its loads go out together: the o vectors of
-// the first kCombineChunk slots before anything waits on a load, the (m, l)
-// pairs of every slot spread over the lanes.  R^T is applied to the cold
-// sum with butterflies inside the lane and across lanes (shuffles): no
-// shared memory, no barrier.
+// One block per query head; its kCombineWarps warps split the head's slots
+// (contiguous quarters), lane i holding output dims [PD i, PD i + PD).  The
+// kernel moves a few KB per head and is bound by load latency, so its loads
+// go out together: a warp's (m, l) pairs one per lane, the o vectors of up
+// to kCombineChunk of its slots before anything waits on a load.  Each warp
+// merges its slots against its own max; the warps' (m, l, o) are then
+// rescaled to the head's max and added in warp order through shared memory,
+// and warp 0 applies R^T to the cold sum with butterflies inside the lane
+// and across lanes (shuffles).
 constexpr int kCombineMaxSlots = kSlotsCold + kSlotsHot;
 constexpr int kCombineChunk = 16;    // slots whose o vectors are in flight together
-constexpr int kCombineHeads = 4;     // warps (query heads) per block
+constexpr int kCombineWarps = 4;     // warps per head (slots per warp <= 32)
+static_assert(kCombineMaxSlots <= 32 * kCombineWarps, "one (m, l) pair per lane");
 
 template <int D>
-__global__ void __launch_bounds__(32 * kCombineHeads) combine_kernel(const CombineArgs a) {
+__global__ void __launch_bounds__(32 * kCombineWarps) combine_kernel(const CombineArgs a) {
   constexpr int PD = D / 32;
   constexpr int CH = kCombineChunk;
-  constexpr int MS = kCombineMaxSlots / 32;   // (m, l) pairs per lane
+  constexpr int NW = kCombineWarps;
+  __shared__ float s_ml[NW][2];
+  __shared__ float s_o[NW][2][D];
   // The next step's eviction encode may start its prologue now (it waits
   // for this kernel before reading its inputs).
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   // launched as a programmatic dependent of the attention kernel
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  const int lane = threadIdx.x & 31;
-  const int hg = blockIdx.x * kCombineHeads + (threadIdx.x >> 5);
-  if (hg >= a.batch * a.Hq) return;          // (warp-uniform)
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int hg = blockIdx.x;
   const int b = hg / a.Hq, hq = hg % a.Hq;
   const int kvh = hq / a.G, g = hq % a.G;
   const int unit = b * a.Hkv + kvh;
@@ -265,84 +269,95 @@ __global__ void __launch_bounds__(32 * kCombineHeads) combine_kernel(const Combi
       o[k + 1] = v.y;
     }
   };
+  const int lo = warp * ns / NW, hi = (warp + 1) * ns / NW;   // this warp's slots
   float ov[CH][PD];
 #pragma unroll
   for (int u = 0; u < CH; ++u) {
-    if (u < ns) {
-      load_o(u, ov[u]);
+    if (lo + u < hi) {
+      load_o(lo + u, ov[u]);
     } else {
 #pragma unroll
       for (int k = 0; k < PD; ++k) ov[u][k] = 0.f;
     }
   }
-  float ms[MS], ls[MS];
-#pragma unroll
-  for (int k = 0; k < MS; ++k) {
-    const int s = lane + 32 * k;
-    ms[k] = kNegInf;
-    ls[k] = 0.f;
-    if (s < ns) {
-      const float2 v = *reinterpret_cast<const float2*>(rec(s));
-      ms[k] = v.x;
-      ls[k] = v.y;
-    }
+  float ms = kNegInf, ls = 0.f;              // slot lo + lane
+  if (lo + lane < hi) {
+    const float2 v = *reinterpret_cast<const float2*>(rec(lo + lane));
+    ms = v.x;
+    ls = v.y;
   }
   float* orow = a.out + (size_t)hg * D + lane * PD;
   if (*(volatile const int*)a.status & kStatusNoPartials) {
     // an attention launch gave up without writing its partials (a latched
     // timeout or layout error): the output is NaN until the status is read
+    if (warp == 0)
 #pragma unroll
-    for (int k = 0; k < PD; ++k) orow[k] = __int_as_float(0x7fc00000);
+      for (int k = 0; k < PD; ++k) orow[k] = __int_as_float(0x7fc00000);
     return;
   }
-  // ---- m = max over slots, then w_s and l = sum w_s l_s ----------------------
-  float mx = kNegInf;
+  // ---- this warp: m_w = max over its slots, w_s = 2^(m_s - m_w), l_w -------
+  float mw = ms;
 #pragma unroll
-  for (int k = 0; k < MS; ++k) mx = fmaxf(mx, ms[k]);
+  for (int o = 16; o; o >>= 1) mw = fmaxf(mw, __shfl_xor_sync(kFull, mw, o));
+  const float ws = ms == kNegInf ? 0.f : exp2f(ms - mw);
+  float lw = ws * ls;
 #pragma unroll
-  for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, o));
-  float w[MS], lsum = 0.f;
-#pragma unroll
-  for (int k = 0; k < MS; ++k) {
-    w[k] = ms[k] == kNegInf ? 0.f : exp2f(ms[k] - mx);
-    lsum += w[k] * ls[k];
-  }
-#pragma unroll
-  for (int o = 16; o; o >>= 1) lsum += __shfl_xor_sync(kFull, lsum, o);
-  // ---- weighted sums of the o vectors ------------------------------------------
-  // (slot s's weight sits in lane s % 32, register s / 32; s is warp-uniform)
-  auto weight = [&](int s) {
-    const int k = s >> 5;
-    float x = w[0];
-#pragma unroll
-    for (int kk = 1; kk < MS; ++kk)
-      if (k == kk) x = w[kk];
-    return __shfl_sync(kFull, x, s & 31);
-  };
+  for (int o = 16; o; o >>= 1) lw += __shfl_xor_sync(kFull, lw, o);
   float oc[PD], oh[PD];
 #pragma unroll
   for (int k = 0; k < PD; ++k) oc[k] = oh[k] = 0.f;
-  auto accum = [&](int s, const float (&o)[PD]) {
-    const float ws = weight(s);
+  auto accum = [&](int s, const float (&o)[PD]) {   // (s warp-uniform)
+    const float wt = __shfl_sync(kFull, ws, s - lo);
     if (s < nc) {
 #pragma unroll
-      for (int k = 0; k < PD; ++k) oc[k] += ws * o[k];
+      for (int k = 0; k < PD; ++k) oc[k] += wt * o[k];
     } else {
 #pragma unroll
-      for (int k = 0; k < PD; ++k) oh[k] += ws * o[k];
+      for (int k = 0; k < PD; ++k) oh[k] += wt * o[k];
     }
   };
-  if (mx != kNegInf) {
+  if (mw != kNegInf) {
 #pragma unroll
     for (int u = 0; u < CH; ++u)
-      if (u < ns) accum(u, ov[u]);
-    for (int s0 = CH; s0 < ns; s0 += CH) {
+      if (lo + u < hi) accum(lo + u, ov[u]);
+    for (int s0 = lo + CH; s0 < hi; s0 += CH) {
 #pragma unroll
       for (int u = 0; u < CH; ++u)
-        if (s0 + u < ns) load_o(s0 + u, ov[u]);
+        if (s0 + u < hi) load_o(s0 + u, ov[u]);
 #pragma unroll
       for (int u = 0; u < CH; ++u)
-        if (s0 + u < ns) accum(s0 + u, ov[u]);
+        if (s0 + u < hi) accum(s0 + u, ov[u]);
+    }
+  }
+  if (lane == 0) {
+    s_ml[warp][0] = mw;
+    s_ml[warp][1] = lw;
+  }
+#pragma unroll
+  for (int k = 0; k < PD; ++k) {
+    s_o[warp][0][lane * PD + k] = oc[k];
+    s_o[warp][1][lane * PD + k] = oh[k];
+  }
+  __syncthreads();
+  if (warp != 0) return;
+  // ---- the head: m = max of the warps' maxima; each warp's sums scaled by
+  // 2^(m_w - m) and added in warp order ------------------------------------
+  float mx = s_ml[0][0];
+#pragma unroll
+  for (int w = 1; w < NW; ++w) mx = fmaxf(mx, s_ml[w][0]);
+  float lsum = 0.f;
+#pragma unroll
+  for (int k = 0; k < PD; ++k) oc[k] = oh[k] = 0.f;
+  if (mx != kNegInf) {
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+      const float f = s_ml[w][0] == kNegInf ? 0.f : exp2f(s_ml[w][0] - mx);
+      lsum += f * s_ml[w][1];
+#pragma unroll
+      for (int k = 0; k < PD; ++k) {
+        oc[k] += f * s_o[w][0][lane * PD + k];
+        oh[k] += f * s_o[w][1][lane * PD + k];
+      }
     }
   }
   // ---- R^T on the cold sum: unnormalised Hadamard (dim i = PD lane + k),
@@ -465,8 +480,8 @@ cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s) {
   // programmatic dependent launch: the kernel waits for the attention
   // kernel before it reads the partials
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((a.batch * a.Hq + kCombineHeads - 1) / kCombineHeads);
-  cfg.blockDim = dim3(32 * kCombineHeads);
+  cfg.gridDim = dim3(a.batch * a.Hq);
+  cfg.blockDim = dim3(32 * kCombineWarps);
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
